@@ -1,0 +1,218 @@
+"""Seeded synthetic inputs for KV compaction problems.
+
+This module only draws random numbers and lays them out; it holds none of
+the compaction arithmetic, so both the CPU oracle's tests and the CUDA path
+consume exactly the same arrays from it.
+
+The pages ("Fast KV Compaction via Attention Matching", the zhichai.net deep
+dive §2.2-§2.4 and the xinfinite.net article §5) evaluate on QuALITY,
+LongHealth and AIME 2025 with Qwen3-4B / Llama-3.1-8B; neither the datasets
+nor the weights are available, so heads shaped like those models stand in:
+
+* ``iid``      - small i.i.d. head: K, Q ~ N(0,1)·d^-1/4, V ~ N(0,1).
+* ``structured`` - per head a rank-32 key subspace: K = 2·U·Bᵀ + 0.3·E,
+  four large-norm "sink" keys at positions 0-3, reference queries that are
+  Dirichlet mixtures of four random keys plus 0.3·noise, V ~ N(0,1).
+
+All draws use ``numpy.random.default_rng(seed)`` (PCG64) in float64 and are
+then rounded once to the storage dtype (fp32, or bf16 round-to-nearest-even
+through torch's CPU cast).  Every array is returned both as the storage
+tensor (what the GPU reads) and as its exact float64 upcast (what the oracle
+reads).
+"""
+from __future__ import annotations
+
+import dataclasses
+import math
+from typing import List, Optional
+
+import numpy as np
+import torch
+
+_DT = {"bf16": torch.bfloat16, "fp32": torch.float32}
+
+
+def round_to(x: np.ndarray, dtype: str) -> torch.Tensor:
+    """Round a float64 array once to the storage dtype (RNE), as a CPU tensor."""
+    return torch.from_numpy(np.ascontiguousarray(x, dtype=np.float64)).to(_DT[dtype])
+
+
+def upcast(t: torch.Tensor) -> np.ndarray:
+    """Exact float64 view of a stored tensor (bf16 and fp32 embed in fp64)."""
+    return t.detach().to("cpu").to(torch.float64).numpy()
+
+
+@dataclasses.dataclass
+class Head:
+    """One compaction problem in storage dtype plus its float64 upcast."""
+    Q: torch.Tensor          # [n, d]
+    K: torch.Tensor          # [T, d]
+    V: torch.Tensor          # [T, d]
+    key_bias: Optional[np.ndarray] = None   # [T] float32-valued prior bias, or None
+
+    @property
+    def n(self) -> int:
+        return self.Q.shape[0]
+
+    @property
+    def T(self) -> int:
+        return self.K.shape[0]
+
+    @property
+    def d(self) -> int:
+        return self.K.shape[1]
+
+    def f64(self):
+        return upcast(self.Q), upcast(self.K), upcast(self.V)
+
+
+def iid_head(seed: int, n: int, T: int, d: int, dtype: str = "fp32") -> Head:
+    """Small i.i.d. head: Q, K ~ N(0,1)·d^-1/4, V ~ N(0,1) (draw order Q, K, V)."""
+    rng = np.random.default_rng(seed)
+    s = d ** -0.25
+    Q = rng.standard_normal((n, d)) * s
+    K = rng.standard_normal((T, d)) * s
+    V = rng.standard_normal((T, d))
+    return Head(round_to(Q, dtype), round_to(K, dtype), round_to(V, dtype))
+
+
+def _structured_keys(rng: np.random.Generator, T: int, d: int, rank: int,
+                     sinks: int, B: np.ndarray) -> np.ndarray:
+    U = rng.standard_normal((T, rank))
+    E = rng.standard_normal((T, d))
+    K = 2.0 * U @ B.T + 0.3 * E
+    if sinks:
+        med = float(np.median(np.linalg.norm(K, axis=1)))
+        for s in range(min(sinks, T)):
+            z = rng.standard_normal(rank)
+            u = B @ (z / np.linalg.norm(z))
+            K[s] = 4.0 * med * u
+    return K
+
+
+def _mixture_queries(rng: np.random.Generator, K: np.ndarray, n: int,
+                     first: int = 0) -> np.ndarray:
+    """q = Σ_{l<4} a_l k_{j_l} + 0.3·ε with a ~ Dirichlet(1,1,1,1) and the j_l
+    uniform over keys [first, T) (sink keys are never mixture components, so
+    a query's logit range stays that of an ordinary key match)."""
+    T, d = K.shape
+    j = rng.integers(first, T, size=(n, 4))
+    a = rng.dirichlet(np.ones(4), size=n)
+    return np.einsum("nl,nld->nd", a, K[j]) + 0.3 * rng.standard_normal((n, d))
+
+
+def structured_head(seed: int, n: int, T: int, d: int = 128, rank: int = 32,
+                    sinks: int = 4, dtype: str = "bf16") -> Head:
+    """Structured head (rank-32 keys + noise, sink keys, mixture queries).
+
+    Draw order: basis B (QR of an N(0,1) d×rank matrix), U, E, one unit vector
+    per sink, then the query mixture indices, Dirichlet weights and noise,
+    then V.
+    """
+    rng = np.random.default_rng(seed)
+    B, _ = np.linalg.qr(rng.standard_normal((d, rank)))
+    K = _structured_keys(rng, T, d, rank, sinks, B)
+    Kr = upcast(round_to(K, dtype))
+    Q = _mixture_queries(rng, Kr, n, first=min(sinks, T - 1))
+    V = rng.standard_normal((T, d))
+    return Head(round_to(Q, dtype), round_to(K, dtype), round_to(V, dtype))
+
+
+def long_sequence_chunks(seed: int, T_total: int, chunk: int, n: int, d: int = 128,
+                         rank: int = 32, dtype: str = "bf16") -> List[Head]:
+    """One long structured key/value sequence split KV-based into contiguous
+    chunks (sinks only at global positions 0-3, hence only in chunk 0); each
+    chunk gets its own reference queries drawn against its own keys."""
+    rng = np.random.default_rng(seed)
+    B, _ = np.linalg.qr(rng.standard_normal((d, rank)))
+    K = _structured_keys(rng, T_total, d, rank, 4, B)
+    V = rng.standard_normal((T_total, d))
+    Kt, Vt = round_to(K, dtype), round_to(V, dtype)
+    heads = []
+    for c0 in range(0, T_total, chunk):
+        c1 = min(T_total, c0 + chunk)
+        qrng = np.random.default_rng(seed + 100000 * (c0 // chunk + 1))
+        Q = _mixture_queries(qrng, upcast(Kt[c0:c1]), n, first=4 if c0 == 0 else 0)
+        heads.append(Head(round_to(Q, dtype), Kt[c0:c1].clone(), Vt[c0:c1].clone()))
+    return heads
+
+
+def budget_for_ratio(T: int, ratio: float) -> int:
+    """t = round-half-up(T / ratio), at least 1."""
+    return max(1, int(math.floor(T / ratio + 0.5)))
+
+
+def lognormal_budgets(seed: int, num_heads: int, total: int, sigma: float = 0.8,
+                      lo: int = 4, hi: int = 1024) -> List[int]:
+    """Non-uniform per-head budgets: raw_h = exp(sigma·z_h), a common scale s
+    found by bisection so that Σ clip(s·raw_h, lo, hi) = total, then floored
+    with the remainder handed out by largest fractional part (ties → lower h)."""
+    rng = np.random.default_rng(seed)
+    raw = np.exp(sigma * rng.standard_normal(num_heads))
+
+    def tot(s):
+        return float(np.clip(s * raw, lo, hi).sum())
+
+    a, b = 0.0, 1.0
+    while tot(b) < total:
+        b *= 2.0
+    for _ in range(200):
+        mid = 0.5 * (a + b)
+        if tot(mid) < total:
+            a = mid
+        else:
+            b = mid
+    x = np.clip(b * raw, lo, hi)
+    base = np.floor(x).astype(np.int64)
+    rem = int(total - base.sum())
+    frac = x - base
+    order = sorted(range(num_heads), key=lambda h: (-frac[h], h))
+    for h in order:
+        if rem <= 0:
+            break
+        if base[h] < hi:
+            base[h] += 1
+            rem -= 1
+    return [int(v) for v in base]
+
+
+# ----------------------------------------------------------------------------
+# Named workloads (sizes of the pages' settings; see module docstring)
+# ----------------------------------------------------------------------------
+
+@dataclasses.dataclass
+class Workload:
+    name: str
+    heads: List[Head]
+    budgets: List[int]
+    topk: int
+    refit_every: int
+    dtype: str
+    note: str = ""
+
+
+def single_head_fp32(seed: int = 1000) -> Workload:
+    """One i.i.d. fp32 head, T=256, d=64, n=512, t=16, plain OMP (k=1, R=1)."""
+    h = iid_head(seed, n=512, T=256, d=64, dtype="fp32")
+    return Workload("single_head_fp32_T256_n512_d64_t16", [h], [16], 1, 1, "fp32")
+
+
+def qwen3_4b_layer(num_heads: int = 8, T: int = 8192, n: int = 8192, ratio: float = 50.0,
+                   seed_base: int = 2000) -> Workload:
+    """One Qwen3-4B-shaped layer: 8 KV heads, d=128, T=n=8192, bf16, 50× (t=164),
+    top-k=4 with a refit every 2 rounds."""
+    heads = [structured_head(seed_base + h, n=n, T=T) for h in range(num_heads)]
+    t = budget_for_ratio(T, ratio)
+    return Workload(f"qwen3_4b_layer_H{num_heads}_T{T}_n{n}_d128_t{t}", heads,
+                    [t] * num_heads, 4, 2, "bf16")
+
+
+def qwen3_4b_model(num_heads: int = 288, T: int = 8192, n: int = 8192, ratio: float = 50.0,
+                   seed_base: int = 4000) -> Workload:
+    """Full Qwen3-4B-shaped model (36 layers × 8 KV heads) with log-normal
+    non-uniform budgets summing to T·H/ratio, clipped to [4, 1024]."""
+    heads = [structured_head(seed_base + h, n=n, T=T) for h in range(num_heads)]
+    total = int(math.floor(T * num_heads / ratio + 0.5))
+    budgets = lognormal_budgets(seed_base + 999, num_heads, total)
+    return Workload(f"qwen3_4b_model_H{num_heads}_T{T}_n{n}_d128_lognormal", heads,
+                    budgets, 4, 2, "bf16")
