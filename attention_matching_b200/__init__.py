@@ -1,0 +1,246 @@
+"""B200 (sm_100a) Attention-Matching KV compaction (AM-OMP).
+
+Thin ctypes binding over the C ABI in include/am_b200.h: it only marshals
+torch tensors to pointers and sizes; every step of the compaction runs in the
+library's CUDA kernels.  The library is built in-tree by
+``attention_matching_b200._build.build()`` (or ``__graft_entry__.build()``).
+There is no CPU fallback: without the shared library or a CUDA device the
+calls raise.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Dict, Optional, Sequence
+
+__all__ = ["AmError", "AmOpts", "lib", "library_path", "workspace_size", "compact_heads",
+           "get_status", "profile_enable", "profile_collect", "kernel_launches", "STAGES",
+           "STATUS", "BF16", "FP32"]
+
+BF16, FP32 = 0, 1
+STATUS = {
+    0: "AM_OK", 1: "AM_ERR_INVALID_ARG", 2: "AM_ERR_BUDGET", 3: "AM_ERR_WORKSPACE",
+    4: "AM_ERR_NONFINITE", 5: "AM_ERR_CUDA", 6: "AM_ERR_TIMEOUT", 7: "AM_ERR_UNSUPPORTED",
+    8: "AM_WARN_NOT_CONVERGED", 9: "AM_ERR_NOT_SPD",
+}
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+
+
+def library_path() -> str:
+    return os.path.join(_HERE, "_lib", "libam_b200.so")
+
+
+class AmError(RuntimeError):
+    def __init__(self, code: int, where: str):
+        self.code = code
+        super().__init__(f"{where}: {STATUS.get(code, code)}")
+
+
+class AmOpts(ctypes.Structure):
+    """Mirror of am_opts_t (include/am_b200.h); field order and types match."""
+    _fields_ = [
+        ("in_dtype", ctypes.c_int32),
+        ("topk", ctypes.c_int32),
+        ("refit_every", ctypes.c_int32),
+        ("nnls_max_iter", ctypes.c_int32),
+        ("scale", ctypes.c_float),
+        ("ridge", ctypes.c_float),
+        ("w_floor_rel", ctypes.c_float),
+        ("reserved0", ctypes.c_float),
+        ("shift", ctypes.c_void_p),
+        ("key_bias", ctypes.c_void_p),
+        ("pick_order", ctypes.c_void_p),
+        ("pick_corr", ctypes.c_void_p),
+        ("shift_out", ctypes.c_void_p),
+        ("residual_out", ctypes.c_void_p),
+        ("w_out", ctypes.c_void_p),
+    ]
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """Load the shared library once; raise loudly if it has not been built."""
+    global _lib
+    if _lib is None:
+        path = library_path()
+        if not os.path.exists(path):
+            raise RuntimeError(f"{path} is missing: build it with attention_matching_b200._build.build()")
+        L = ctypes.CDLL(path)
+        c_int, c_void_p, c_size_t = ctypes.c_int32, ctypes.c_void_p, ctypes.c_size_t
+        P_i32 = ctypes.POINTER(ctypes.c_int32)
+        P_i64 = ctypes.POINTER(ctypes.c_int64)
+        L.am_default_opts.argtypes = [ctypes.POINTER(AmOpts)]
+        L.am_default_opts.restype = c_int
+        L.am_workspace_size.argtypes = [c_int, c_int, c_int, c_int, P_i32, ctypes.POINTER(AmOpts),
+                                        ctypes.POINTER(c_size_t)]
+        L.am_workspace_size.restype = c_int
+        L.am_compact_heads.argtypes = [c_void_p, c_void_p, c_void_p, c_int, c_int, c_int, c_int, P_i32,
+                                       ctypes.POINTER(AmOpts), c_void_p, c_size_t, P_i64,
+                                       c_void_p, c_void_p, c_void_p, c_void_p, c_void_p]
+        L.am_compact_heads.restype = c_int
+        L.am_get_status.argtypes = [c_void_p, c_int, P_i32, c_void_p]
+        L.am_get_status.restype = c_int
+        L.am_status_string.argtypes = [c_int]
+        L.am_status_string.restype = ctypes.c_char_p
+        L.am_version.argtypes = []
+        L.am_version.restype = c_int
+        L.am_profile_enable.argtypes = [c_int]
+        L.am_profile_enable.restype = c_int
+        L.am_profile_collect.argtypes = [ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_int64)]
+        L.am_profile_collect.restype = c_int
+        L.am_kernel_launches.argtypes = []
+        L.am_kernel_launches.restype = ctypes.c_int64
+        _lib = L
+    return _lib
+
+
+def _i32_array(vals: Sequence[int]):
+    return (ctypes.c_int32 * len(vals))(*[int(v) for v in vals])
+
+
+def make_opts(dtype: int = BF16, topk: int = 1, refit_every: int = 1, scale: float = 0.0,
+              ridge: float = 1e-6, w_floor_rel: float = 1e-12, nnls_max_iter: int = 0) -> AmOpts:
+    o = AmOpts()
+    rc = lib().am_default_opts(ctypes.byref(o))
+    if rc:
+        raise AmError(rc, "am_default_opts")
+    o.in_dtype, o.topk, o.refit_every, o.nnls_max_iter = dtype, topk, refit_every, nnls_max_iter
+    o.scale, o.ridge, o.w_floor_rel = scale, ridge, w_floor_rel
+    return o
+
+
+def workspace_size(n: int, T: int, d: int, budgets: Sequence[int], opts: AmOpts) -> int:
+    out = ctypes.c_size_t(0)
+    rc = lib().am_workspace_size(n, T, d, len(budgets), _i32_array(budgets), ctypes.byref(opts),
+                                 ctypes.byref(out))
+    if rc:
+        raise AmError(rc, "am_workspace_size")
+    return int(out.value)
+
+
+def _ptr(t) -> Optional[int]:
+    return None if t is None else t.data_ptr()
+
+
+def compact_heads(Q, K, V, budgets: Sequence[int], topk: int = 1, refit_every: int = 1,
+                  shift=None, key_bias=None, ridge: float = 1e-6, w_floor_rel: float = 1e-12,
+                  scale: float = 0.0, nnls_max_iter: int = 0, workspace=None, trace: bool = False,
+                  stream=None, check: bool = True) -> Dict:
+    """Compact H heads on the GPU.
+
+    Q [H, n, d], K [H, T, d], V [H, T, d]: contiguous tensors, bf16 or fp32,
+    all on the current CUDA device or all on the host (then copied in, and the
+    outputs copied back to the host).
+    budgets: H ints in [1, T].  shift [H] fp32 and key_bias [H, T] fp32 are
+    optional CUDA tensors.  Returns a dict of CUDA tensors in the packed
+    varlen layout (C_k, beta, C_v, indices, cu_t) plus, with ``trace``, the
+    pick order, pick correlations, shift used, mass residual and weights.
+    """
+    import torch
+    host = not (Q.is_cuda or K.is_cuda or V.is_cuda)
+    if host:
+        # host inputs: copy in (asynchronously from pinned memory), run, copy out
+        dev = torch.device("cuda", torch.cuda.current_device())
+        Q, K, V = (x.to(dev, non_blocking=True) for x in (Q, K, V))
+    if not (Q.is_cuda and K.is_cuda and V.is_cuda):
+        raise ValueError("Q, K, V must all be CUDA tensors or all host tensors")
+    H, n, d = Q.shape
+    T = K.shape[1]
+    if K.shape != (H, T, d) or V.shape != (H, T, d) or len(budgets) != H:
+        raise ValueError("shape mismatch")
+    if Q.dtype != K.dtype or Q.dtype != V.dtype or Q.dtype not in (torch.bfloat16, torch.float32):
+        raise ValueError("Q, K, V must share dtype bf16 or fp32")
+    for t in (Q, K, V):
+        if not t.is_contiguous():
+            raise ValueError("inputs must be contiguous")
+    dt = BF16 if Q.dtype == torch.bfloat16 else FP32
+    dev = Q.device
+    opts = make_opts(dt, topk, refit_every, scale, ridge, w_floor_rel, nnls_max_iter)
+    if shift is not None:
+        shift = shift.to(device=dev, dtype=torch.float32).contiguous()
+        opts.shift = shift.data_ptr()
+    if key_bias is not None:
+        key_bias = key_bias.to(device=dev, dtype=torch.float32).contiguous()
+        opts.key_bias = key_bias.data_ptr()
+    cu = [0]
+    for t in budgets:
+        cu.append(cu[-1] + int(t))
+    tot = cu[-1]
+    out = {
+        "C_k": torch.empty((tot, d), dtype=Q.dtype, device=dev),
+        "beta": torch.empty((tot,), dtype=torch.float32, device=dev),
+        "C_v": torch.empty((tot, d), dtype=torch.float32, device=dev),
+        "indices": torch.empty((tot,), dtype=torch.int32, device=dev),
+        "cu_t": torch.tensor(cu, dtype=torch.int64),
+    }
+    if trace:
+        out["pick_order"] = torch.empty((tot,), dtype=torch.int32, device=dev)
+        out["pick_corr"] = torch.empty((tot,), dtype=torch.float32, device=dev)
+        out["shift"] = torch.empty((H,), dtype=torch.float32, device=dev)
+        out["residual"] = torch.empty((H,), dtype=torch.float64, device=dev)
+        out["w"] = torch.empty((tot,), dtype=torch.float32, device=dev)
+        opts.pick_order = out["pick_order"].data_ptr()
+        opts.pick_corr = out["pick_corr"].data_ptr()
+        opts.shift_out = out["shift"].data_ptr()
+        opts.residual_out = out["residual"].data_ptr()
+        opts.w_out = out["w"].data_ptr()
+    need = workspace_size(n, T, d, budgets, opts)
+    if workspace is None or workspace.numel() * workspace.element_size() < need:
+        workspace = torch.empty((need,), dtype=torch.uint8, device=dev)
+    offs = (ctypes.c_int64 * (H + 1))(*cu)
+    if stream is None:
+        stream = torch.cuda.current_stream(dev).cuda_stream
+    rc = lib().am_compact_heads(Q.data_ptr(), K.data_ptr(), V.data_ptr(), n, T, d, H,
+                                _i32_array(budgets), ctypes.byref(opts), workspace.data_ptr(),
+                                workspace.numel() * workspace.element_size(), offs,
+                                out["C_k"].data_ptr(), out["beta"].data_ptr(), out["C_v"].data_ptr(),
+                                out["indices"].data_ptr(), ctypes.c_void_p(stream))
+    if rc:
+        raise AmError(rc, "am_compact_heads")
+    out["workspace"] = workspace
+    if host:
+        for k in ("C_k", "beta", "C_v", "indices", "pick_order", "pick_corr", "shift", "residual", "w"):
+            if k in out:
+                out[k] = out[k].to("cpu")
+    if check:
+        per_head, worst = get_status(workspace, H, stream)
+        out["status"] = per_head
+        if worst not in (0, 8):
+            raise AmError(worst, "am_compact_heads (device)")
+    return out
+
+
+STAGES = ["shift", "phi", "target", "init", "corr", "select", "gram", "nnls", "resid",
+          "finalize", "design", "normal", "solve"]
+
+
+def profile_enable(on: bool = True) -> None:
+    """Bracket every library kernel launch with CUDA events (stage timing)."""
+    lib().am_profile_enable(1 if on else 0)
+
+
+def profile_collect() -> Dict[str, Dict[str, float]]:
+    """Wait for the recorded events; per stage: device ms and launch count."""
+    ms = (ctypes.c_double * len(STAGES))()
+    n = (ctypes.c_int64 * len(STAGES))()
+    rc = lib().am_profile_collect(ms, n)
+    if rc:
+        raise AmError(rc, "am_profile_collect")
+    return {name: {"ms": ms[k], "launches": int(n[k])} for k, name in enumerate(STAGES)}
+
+
+def kernel_launches() -> int:
+    return int(lib().am_kernel_launches())
+
+
+def get_status(workspace, H: int, stream=None):
+    """Synchronise and read the per-head device status words."""
+    import torch
+    if stream is None:
+        stream = torch.cuda.current_stream(workspace.device).cuda_stream
+    arr = (ctypes.c_int32 * H)()
+    worst = lib().am_get_status(workspace.data_ptr(), H, arr, ctypes.c_void_p(stream))
+    return list(arr), int(worst)

@@ -1,0 +1,309 @@
+// C ABI entry points: argument checks, workspace plan, launch sequence.
+//
+// One call compacts H independent heads (the per-(layer, KV-head) problems of
+// "Fast KV Compaction via Attention Matching", zhichai.net deep dive §1.6;
+// varlen packing of non-uniform budgets per the zhichai.net/en summary,
+// "Engineering Practicality").  All work is enqueued on the caller's stream;
+// no device memory is allocated here.
+#include "am_internal.cuh"
+
+#include <math.h>
+#include <string.h>
+
+#include <algorithm>
+#include <vector>
+
+namespace am {
+namespace {
+
+constexpr size_t kAlign = 256;
+
+size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
+
+struct Layout {
+  // byte offsets from the workspace base
+  size_t tables, status, shift, np, mm, rr_part;
+  size_t phiT, m, Y, r, corr, sel;
+  size_t picks, pick_corr, plist, sorted_slot;
+  size_t bvec, w, w_eff;
+  size_t G, L, AtA, A, AtY;
+  size_t total;
+  size_t tables_bytes;
+};
+
+struct Tables {
+  std::vector<int32_t> t;
+  std::vector<int64_t> cu_t, cu_t2;
+  std::vector<int32_t> order;
+  std::vector<int> active;   // active heads per pass
+  int max_t = 0;
+  int64_t sum_t = 0, sum_t2 = 0;
+};
+
+Layout plan(int n, int T, int d, int H, int64_t sum_t, int64_t sum_t2) {
+  Layout L{};
+  const size_t ldn = (size_t)round_up(n, 32);
+  size_t o = 0;
+  auto take = [&](size_t bytes) { size_t at = o; o = align_up(o + bytes); return at; };
+  L.status = take(kWsHeaderBytes + (size_t)H * 4) + kWsHeaderBytes;   // header precedes status
+  L.tables_bytes = (size_t)H * 4 + (size_t)(H + 1) * 8 * 2 + (size_t)H * 4;
+  L.tables = take(L.tables_bytes);
+  L.shift = take((size_t)H * 4);
+  L.np = take((size_t)H * 4);
+  L.mm = take((size_t)H * 8);
+  L.rr_part = take((size_t)H * kRedBlocks * 8);
+  L.phiT = take((size_t)H * T * ldn * 4);
+  L.m = take((size_t)H * ldn * 8);
+  L.r = take((size_t)H * ldn * 4);
+  L.Y = take((size_t)H * n * d * 4);
+  L.corr = take((size_t)H * T * 4);
+  L.sel = take((size_t)H * T);
+  L.picks = take((size_t)sum_t * 4);
+  L.pick_corr = take((size_t)sum_t * 4);
+  L.plist = take((size_t)sum_t * 4);
+  L.sorted_slot = take((size_t)sum_t * 4);
+  L.bvec = take((size_t)sum_t * 8);
+  L.w = take((size_t)sum_t * 8);
+  L.w_eff = take((size_t)sum_t * 8);
+  L.G = take((size_t)sum_t2 * 8);
+  L.L = take((size_t)sum_t2 * 8);
+  L.AtA = take((size_t)sum_t2 * 8);
+  L.A = take((size_t)sum_t * ldn * 4);
+  L.AtY = take((size_t)sum_t * d * 8);
+  L.total = o;
+  return L;
+}
+
+am_status_t check_shape(int n, int T, int d, int H, const int32_t* budgets, const am_opts_t* opts,
+                        Tables* tb) {
+  if (!budgets || !opts) return AM_ERR_INVALID_ARG;
+  if (n < 1 || T < 1 || d < 1 || H < 1) return AM_ERR_INVALID_ARG;
+  if (opts->in_dtype != AM_BF16 && opts->in_dtype != AM_FP32) return AM_ERR_INVALID_ARG;
+  if (d > 256) return AM_ERR_UNSUPPORTED;
+  if (opts->topk < 1 || opts->refit_every < 1) return AM_ERR_INVALID_ARG;
+  if ((int64_t)opts->topk * opts->refit_every > kMaxPicksPerPass) return AM_ERR_UNSUPPORTED;
+  if (opts->nnls_max_iter < 0) return AM_ERR_INVALID_ARG;
+  if (!(opts->ridge >= 0.f) || !isfinite(opts->ridge)) return AM_ERR_INVALID_ARG;
+  if (!(opts->w_floor_rel > 0.f) || !(opts->w_floor_rel < 1.f)) return AM_ERR_INVALID_ARG;
+  if (!isfinite(opts->scale)) return AM_ERR_INVALID_ARG;
+  if ((int64_t)n * d > (1ll << 31) || (int64_t)T * round_up(n, 32) > (1ll << 40))
+    return AM_ERR_UNSUPPORTED;
+  const int kR = opts->topk * opts->refit_every;
+  tb->t.assign(budgets, budgets + H);
+  tb->cu_t.assign(H + 1, 0);
+  tb->cu_t2.assign(H + 1, 0);
+  std::vector<int> passes(H);
+  for (int h = 0; h < H; ++h) {
+    const int t = budgets[h];
+    if (t < 1 || t > T) return AM_ERR_BUDGET;
+    tb->cu_t[h + 1] = tb->cu_t[h] + t;
+    tb->cu_t2[h + 1] = tb->cu_t2[h] + (int64_t)t * t;
+    tb->max_t = std::max(tb->max_t, t);
+    passes[h] = num_passes(t, kR);
+  }
+  tb->sum_t = tb->cu_t[H];
+  tb->sum_t2 = tb->cu_t2[H];
+  tb->order.resize(H);
+  for (int h = 0; h < H; ++h) tb->order[h] = h;
+  std::stable_sort(tb->order.begin(), tb->order.end(),
+                   [&](int a, int b) { return passes[a] > passes[b]; });
+  const int maxp = passes[tb->order[0]];
+  tb->active.assign(maxp, 0);
+  for (int q = 0; q < maxp; ++q)
+    for (int h = 0; h < H; ++h) tb->active[q] += passes[h] > q;
+  return AM_OK;
+}
+
+Work bind(const Layout& L, char* base) {
+  Work w{};
+  w.status = reinterpret_cast<int32_t*>(base + L.status);
+  w.shift = reinterpret_cast<float*>(base + L.shift);
+  w.np = reinterpret_cast<int32_t*>(base + L.np);
+  w.mm = reinterpret_cast<double*>(base + L.mm);
+  w.rr_part = reinterpret_cast<double*>(base + L.rr_part);
+  w.phiT = reinterpret_cast<float*>(base + L.phiT);
+  w.m = reinterpret_cast<double*>(base + L.m);
+  w.r = reinterpret_cast<float*>(base + L.r);
+  w.Y = reinterpret_cast<float*>(base + L.Y);
+  w.corr = reinterpret_cast<float*>(base + L.corr);
+  w.sel = reinterpret_cast<uint8_t*>(base + L.sel);
+  w.picks = reinterpret_cast<int32_t*>(base + L.picks);
+  w.pick_corr = reinterpret_cast<float*>(base + L.pick_corr);
+  w.plist = reinterpret_cast<int32_t*>(base + L.plist);
+  w.sorted_slot = reinterpret_cast<int32_t*>(base + L.sorted_slot);
+  w.bvec = reinterpret_cast<double*>(base + L.bvec);
+  w.w = reinterpret_cast<double*>(base + L.w);
+  w.w_eff = reinterpret_cast<double*>(base + L.w_eff);
+  w.G = reinterpret_cast<double*>(base + L.G);
+  w.L = reinterpret_cast<double*>(base + L.L);
+  w.AtA = reinterpret_cast<double*>(base + L.AtA);
+  w.A = reinterpret_cast<float*>(base + L.A);
+  w.AtY = reinterpret_cast<double*>(base + L.AtY);
+  return w;
+}
+
+// Packs the host tables in the device order cu_t | cu_t2 | t | order.
+void pack_tables(const Tables& tb, int H, std::vector<unsigned char>* out, Work* w, char* dev) {
+  const size_t b_cu = (size_t)(H + 1) * 8;
+  out->resize(2 * b_cu + 2 * (size_t)H * 4);
+  unsigned char* o = out->data();
+  memcpy(o, tb.cu_t.data(), b_cu);
+  memcpy(o + b_cu, tb.cu_t2.data(), b_cu);
+  memcpy(o + 2 * b_cu, tb.t.data(), (size_t)H * 4);
+  memcpy(o + 2 * b_cu + (size_t)H * 4, tb.order.data(), (size_t)H * 4);
+  w->cu_t = reinterpret_cast<int64_t*>(dev);
+  w->cu_t2 = reinterpret_cast<int64_t*>(dev + b_cu);
+  w->t = reinterpret_cast<int32_t*>(dev + 2 * b_cu);
+  w->order = reinterpret_cast<int32_t*>(dev + 2 * b_cu + (size_t)H * 4);
+}
+
+Problem make_problem(int n, int T, int d, int H, const am_opts_t* o, const Tables& tb) {
+  Problem p{};
+  p.H = H; p.n = n; p.T = T; p.d = d;
+  p.ldn = round_up(n, 32);
+  p.in_dtype = o->in_dtype;
+  p.scale = o->scale > 0.f ? o->scale : (float)(1.0 / sqrt((double)d));
+  p.topk = o->topk;
+  p.refit_every = o->refit_every;
+  p.kR = o->topk * o->refit_every;
+  p.nnls_max_iter = o->nnls_max_iter;
+  p.ridge = o->ridge;
+  p.w_floor_rel = o->w_floor_rel;
+  p.max_t = tb.max_t;
+  p.has_bias = o->key_bias != nullptr;
+  return p;
+}
+
+struct WsHeader {
+  uint32_t magic;
+  int32_t H;
+};
+
+}  // namespace
+}  // namespace am
+
+using namespace am;
+
+extern "C" {
+
+am_status_t am_default_opts(am_opts_t* opts) {
+  if (!opts) return AM_ERR_INVALID_ARG;
+  memset(opts, 0, sizeof(*opts));
+  opts->in_dtype = AM_BF16;
+  opts->topk = 1;
+  opts->refit_every = 1;
+  opts->scale = 0.f;
+  opts->ridge = 1e-6f;
+  opts->w_floor_rel = 1e-12f;
+  return AM_OK;
+}
+
+am_status_t am_workspace_size(int32_t n, int32_t T, int32_t d, int32_t num_heads,
+                              const int32_t* budgets, const am_opts_t* opts, size_t* bytes) {
+  if (!bytes) return AM_ERR_INVALID_ARG;
+  Tables tb;
+  am_status_t st = check_shape(n, T, d, num_heads, budgets, opts, &tb);
+  if (st != AM_OK) return st;
+  *bytes = plan(n, T, d, num_heads, tb.sum_t, tb.sum_t2).total;
+  return AM_OK;
+}
+
+am_status_t am_compact_heads(const void* Q, const void* K, const void* V, int32_t n, int32_t T,
+                             int32_t d, int32_t H, const int32_t* budgets, const am_opts_t* opts,
+                             void* workspace, size_t workspace_bytes, const int64_t* out_offsets,
+                             void* C_k, float* beta, float* C_v, int32_t* indices, void* stream) {
+  if (!Q || !K || !V || !C_k || !beta || !C_v || !indices || !out_offsets) return AM_ERR_INVALID_ARG;
+  Tables tb;
+  am_status_t st = check_shape(n, T, d, H, budgets, opts, &tb);
+  if (st != AM_OK) return st;
+  for (int h = 0; h <= H; ++h)
+    if (out_offsets[h] != tb.cu_t[h]) return AM_ERR_INVALID_ARG;
+  if (!workspace || ((uintptr_t)workspace % kAlign) != 0) return AM_ERR_WORKSPACE;
+  const Layout L = plan(n, T, d, H, tb.sum_t, tb.sum_t2);
+  if (workspace_bytes < L.total) return AM_ERR_WORKSPACE;
+
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  char* base = reinterpret_cast<char*>(workspace);
+  Work w = bind(L, base);
+  std::vector<unsigned char> host_tables;
+  pack_tables(tb, H, &host_tables, &w, base + L.tables);
+  const Problem p = make_problem(n, T, d, H, opts, tb);
+
+  WsHeader hdr{kWsMagic, H};
+#define AM_TRY(x)                      \
+  do {                                 \
+    if ((x) != cudaSuccess) return AM_ERR_CUDA; \
+  } while (0)
+  // Pageable sources: both copies are staged before cudaMemcpyAsync returns.
+  AM_TRY(cudaMemcpyAsync(base, &hdr, sizeof(hdr), cudaMemcpyHostToDevice, s));
+  AM_TRY(cudaMemcpyAsync(base + L.tables, host_tables.data(), host_tables.size(),
+                         cudaMemcpyHostToDevice, s));
+  AM_TRY(cudaMemsetAsync(w.status, 0, (size_t)H * 4, s));
+
+  const bool tc = phi_tc_supported(p);
+  if (opts->shift) {
+    AM_TRY(launch_shift_copy(opts->shift, w.shift, H, s));
+  } else if (tc) {
+    AM_TRY(launch_shift_init(w.shift, H, s));
+    AM_TRY(launch_shift_max_tc(p, Q, K, opts->key_bias, w, reinterpret_cast<uint32_t*>(w.shift), s));
+    AM_TRY(launch_shift_decode(w.shift, H, s));
+  } else {
+    AM_TRY(launch_shift_max(p, Q, K, opts->key_bias, w.shift, s));
+  }
+  if (tc) {
+    AM_TRY(launch_phi_tc(p, Q, K, V, opts->key_bias, w, s));
+  } else {
+    AM_TRY(launch_phi(p, Q, K, opts->key_bias, w, s));
+    AM_TRY(launch_y_m(p, V, w, s));
+  }
+  AM_TRY(launch_omp_init(p, w, s));
+  for (int pass = 0; pass < (int)tb.active.size(); ++pass)
+    AM_TRY(launch_omp_pass(p, w, pass, tb.active[pass], s));
+  if (opts->residual_out) AM_TRY(launch_residual_norm(p, w, opts->residual_out, s));
+  AM_TRY(launch_finalize(p, w, K, opts->key_bias, C_k, beta, indices, opts->w_out, opts->pick_order,
+                         opts->pick_corr, s));
+  AM_TRY(launch_value_fit(p, w, C_v, s));
+  if (opts->shift_out) AM_TRY(launch_shift_copy(w.shift, opts->shift_out, H, s));
+#undef AM_TRY
+  return AM_OK;
+}
+
+am_status_t am_get_status(const void* workspace, int32_t H, int32_t* per_head, void* stream) {
+  if (!workspace || H < 1) return AM_ERR_INVALID_ARG;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(s) != cudaSuccess) return AM_ERR_CUDA;
+  WsHeader hdr{};
+  if (cudaMemcpy(&hdr, workspace, sizeof(hdr), cudaMemcpyDeviceToHost) != cudaSuccess) return AM_ERR_CUDA;
+  if (hdr.magic != kWsMagic || hdr.H != H) return AM_ERR_WORKSPACE;
+  std::vector<int32_t> raw(H);
+  if (cudaMemcpy(raw.data(), reinterpret_cast<const char*>(workspace) + kWsHeaderBytes, (size_t)H * 4,
+                 cudaMemcpyDeviceToHost) != cudaSuccess)
+    return AM_ERR_CUDA;
+  int worst = 0;
+  for (int h = 0; h < H; ++h) {
+    const int code = raw[h] % 1000;
+    if (per_head) per_head[h] = code;
+    if (raw[h] > worst) worst = raw[h];
+  }
+  return (am_status_t)(worst % 1000);
+}
+
+const char* am_status_string(am_status_t s) {
+  switch (s) {
+    case AM_OK: return "ok";
+    case AM_ERR_INVALID_ARG: return "invalid argument";
+    case AM_ERR_BUDGET: return "budget outside [1, T]";
+    case AM_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
+    case AM_ERR_NONFINITE: return "non-finite feature or solution";
+    case AM_ERR_CUDA: return "CUDA runtime error";
+    case AM_ERR_TIMEOUT: return "bounded device wait ran out";
+    case AM_ERR_UNSUPPORTED: return "unsupported shape or dtype";
+    case AM_WARN_NOT_CONVERGED: return "NNLS stopped at its iteration cap";
+    case AM_ERR_NOT_SPD: return "value-fit matrix not positive definite";
+  }
+  return "unknown status";
+}
+
+int32_t am_version(void) { return 100; }
+
+}  // extern "C"

@@ -1,0 +1,109 @@
+// Internal declarations shared by the library's translation units.
+// Nothing here is part of the C ABI (include/am_b200.h is).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+#include "am_b200.h"
+
+namespace am {
+
+constexpr int kWsHeaderBytes = 256;      // magic + head count, then status words
+constexpr uint32_t kWsMagic = 0x414d4232u;  // "AMB2"
+constexpr int kMaxPicksPerPass = 64;     // k·R upper bound handled per pass
+constexpr int kNnlsThreads = 256;
+constexpr int kCholThreads = 256;
+
+// Problem-wide constants, passed by value to every kernel.
+struct Problem {
+  int H, n, T, d;
+  int ldn;            // leading dimension of per-query rows, n rounded up to 32
+  int in_dtype;       // AM_BF16 / AM_FP32
+  float scale;        // logit scale
+  int topk, refit_every, kR;
+  int nnls_max_iter;  // 0 → 3·t + 50
+  float ridge, w_floor_rel;
+  int max_t;          // max_h t_h
+  int has_bias;
+};
+
+// Device pointers into the caller's workspace (see plan_workspace()).
+struct Work {
+  int32_t* status;      // [H]
+  int32_t* t;           // [H] budgets
+  int64_t* cu_t;        // [H+1] packed output offsets
+  int64_t* cu_t2;       // [H+1] offsets of per-head t×t blocks
+  int32_t* order;       // [H] heads sorted by pass count, descending
+  float* shift;         // [H]
+  float* phiT;          // [H][T][ldn] key-major features Φᵀ
+  double* m;            // [H][ldn] mass: fp64 sum of the stored fp32 features
+  float* Y;             // [H][n][d]
+  float* r;             // [H][ldn] residual (fp32 copy read by the correlation pass)
+  float* corr;          // [H][T]
+  uint8_t* sel;         // [H][T] selected flags
+  int32_t* picks;       // [Σt] pick order
+  float* pick_corr;     // [Σt]
+  double* G;            // [Σt²] Gram of the picks (pick-order indexing)
+  double* bvec;         // [Σt] Φ_Sᵀ m
+  double* w;            // [Σt] NNLS weights (pick order)
+  double* L;            // [Σt²] Cholesky factor scratch (global fallback)
+  int32_t* plist;       // [Σt] NNLS passive list (factor order)
+  int32_t* np;          // [H] passive count
+  double* mm;           // [H] ‖m‖²
+  double* rr_part;      // [H][kRedBlocks] partial ‖r‖²
+  int32_t* sorted_slot; // [Σt] pick slot of each ascending-position output row
+  double* w_eff;        // [Σt] floored weights, ascending-position order
+  float* A;             // [Σt][ldn] design matrix, key-major
+  double* AtA;          // [Σt²]
+  double* AtY;          // [Σt][d]
+};
+
+constexpr int kRedBlocks = 64;   // partial-sum slots per head for ‖r‖²
+
+// ---- launchers (each file defines its own) ----
+// feature pass (am_phi_simt.cu)
+cudaError_t launch_shift_max(const Problem& p, const void* Q, const void* K, const float* key_bias,
+                             float* shift, cudaStream_t s);
+cudaError_t launch_phi(const Problem& p, const void* Q, const void* K, const float* key_bias,
+                       const Work& w, cudaStream_t s);
+cudaError_t launch_y_m(const Problem& p, const void* V, const Work& w, cudaStream_t s);
+cudaError_t launch_shift_copy(const float* src, float* dst, int H, cudaStream_t s);
+cudaError_t launch_shift_init(float* shift, int H, cudaStream_t s);
+cudaError_t launch_shift_decode(float* shift, int H, cudaStream_t s);
+// tensor-core feature pass (am_phi_tc.cu): bf16 inputs, d in {64, 128}
+bool phi_tc_supported(const Problem& p);
+cudaError_t launch_shift_max_tc(const Problem& p, const void* Q, const void* K, const float* key_bias,
+                                const Work& w, uint32_t* shift_ord, cudaStream_t s);
+cudaError_t launch_phi_tc(const Problem& p, const void* Q, const void* K, const void* V, const float* key_bias,
+                          const Work& w, cudaStream_t s);
+// OMP engine (am_omp.cu)
+cudaError_t launch_omp_init(const Problem& p, const Work& w, cudaStream_t s);
+cudaError_t launch_omp_pass(const Problem& p, const Work& w, int pass, int active_heads,
+                            cudaStream_t s);
+cudaError_t launch_residual_norm(const Problem& p, const Work& w, double* residual_out,
+                                 cudaStream_t s);
+// value fit and packing (am_valfit.cu)
+cudaError_t launch_finalize(const Problem& p, const Work& w, const void* K, const float* key_bias,
+                            void* C_k, float* beta, int32_t* indices, float* w_out,
+                            int32_t* pick_order, float* pick_corr, cudaStream_t s);
+cudaError_t launch_value_fit(const Problem& p, const Work& w, float* C_v, cudaStream_t s);
+
+// ---- small device helpers ----
+__host__ __device__ inline int round_up(int x, int a) { return (x + a - 1) / a * a; }
+
+__device__ __forceinline__ float load_in(const void* base, int64_t idx, int dtype) {
+  if (dtype == AM_BF16) return __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(base)[idx]);
+  return reinterpret_cast<const float*>(base)[idx];
+}
+
+__device__ __forceinline__ void record_status(int32_t* status, int code) {
+  // keep the most severe (largest) code; errors outrank the warning
+  atomicMax(status, code == AM_WARN_NOT_CONVERGED ? 1000 + code : 2000 + code);
+}
+
+// Number of OMP passes for budget t: one correlation pass per refit interval.
+__host__ __device__ inline int num_passes(int t, int kR) { return (t + kR - 1) / kR; }
+
+}  // namespace am

@@ -1,0 +1,633 @@
+// OMP key selection with NNLS refits, batched over heads.
+//
+// "Fast KV Compaction via Attention Matching": zhichai.net deep dive §1.6
+// (r = m; repeat: j* = argmax_{j∉S} rᵀΦ_{:,j}, S ∪= {j*}, refit w ≥ 0 by
+// NNLS, r = m − Φ_S w); xinfinite.net article §2 step 2 (Fig. 1, Fig. 2:
+// NNLS solved on the GPU) and §3 (top-k batched selection with lazy refit,
+// Table 1).
+//
+// One "pass" covers R rounds of k picks: the residual does not change
+// between refits, so those R rounds take the next k·R keys of one
+// correlation vector.  A pass is five launches over the active heads:
+//   k_corr    c = Φᵀ r                 (HBM-bound GEMV over key-major Φᵀ)
+//   k_select  top-(k·R) unselected keys, ties to the lowest index
+//   k_gram    new rows/columns of G = Φ_SᵀΦ_S and b = Φ_Sᵀm (fp64 sums)
+//   k_nnls    active-set NNLS on (G, b), warm-started from the last refit
+//   k_resid   r = m − Φ_S w (fp64 sums, stored fp32)
+#include "am_internal.cuh"
+#include "am_profile.cuh"
+#include "am_linalg.cuh"
+
+#include <float.h>
+
+namespace am {
+namespace {
+
+__device__ __forceinline__ void pass_range(const Problem& p, int t, int pass, int& s0, int& s1) {
+  s0 = min(pass * p.kR, t);
+  s1 = min(s0 + p.kR, t);
+}
+
+// ---------------------------------------------------------------- init ----
+__global__ void k_init(Problem p, Work w) {
+  const int h = blockIdx.x;
+  __shared__ double scratch[33];
+  const double* m = w.m + (int64_t)h * p.ldn;
+  double acc = 0.0;
+  for (int i = threadIdx.x; i < p.n; i += blockDim.x) acc += m[i] * m[i];
+  acc = block_sum(acc, scratch);
+  if (threadIdx.x == 0) {
+    w.mm[h] = acc;
+    w.np[h] = 0;
+    if (!(acc > 0.0) || !isfinite(acc)) record_status(w.status + h, AM_ERR_NONFINITE);
+  }
+  uint8_t* sel = w.sel + (int64_t)h * p.T;
+  for (int j = threadIdx.x; j < p.T; j += blockDim.x) sel[j] = 0;
+}
+
+// ----------------------------------------------------------- correlation --
+// One warp per 4 key rows; 128-bit streaming loads of Φᵀ, r from L1.
+constexpr int kCorrRowsPerWarp = 4;
+constexpr int kCorrWarps = 8;
+constexpr int kCorrRowsPerBlock = kCorrRowsPerWarp * kCorrWarps;
+
+__global__ void __launch_bounds__(256) k_corr(Problem p, Work w, int pass) {
+  const int h = w.order[blockIdx.y];
+  const int t = w.t[h];
+  if (pass * p.kR >= t) return;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int j0 = blockIdx.x * kCorrRowsPerBlock + warp * kCorrRowsPerWarp;
+  if (j0 >= p.T) return;
+  const float4* r4 = reinterpret_cast<const float4*>(w.r + (int64_t)h * p.ldn);
+  const float4* rows[kCorrRowsPerWarp];
+#pragma unroll
+  for (int q = 0; q < kCorrRowsPerWarp; ++q) {
+    int j = min(j0 + q, p.T - 1);
+    rows[q] = reinterpret_cast<const float4*>(w.phiT + ((int64_t)h * p.T + j) * p.ldn);
+  }
+  float acc[kCorrRowsPerWarp] = {0.f, 0.f, 0.f, 0.f};
+  const int n4 = p.ldn >> 2;
+  int i = lane;
+  for (; i + 32 < n4; i += 64) {
+    float4 ra = __ldg(r4 + i), rb = __ldg(r4 + i + 32);
+    float4 xa[kCorrRowsPerWarp], xb[kCorrRowsPerWarp];
+#pragma unroll
+    for (int q = 0; q < kCorrRowsPerWarp; ++q) {
+      xa[q] = __ldcs(rows[q] + i);
+      xb[q] = __ldcs(rows[q] + i + 32);
+    }
+#pragma unroll
+    for (int q = 0; q < kCorrRowsPerWarp; ++q) {
+      acc[q] = fmaf(xa[q].x, ra.x, acc[q]); acc[q] = fmaf(xa[q].y, ra.y, acc[q]);
+      acc[q] = fmaf(xa[q].z, ra.z, acc[q]); acc[q] = fmaf(xa[q].w, ra.w, acc[q]);
+      acc[q] = fmaf(xb[q].x, rb.x, acc[q]); acc[q] = fmaf(xb[q].y, rb.y, acc[q]);
+      acc[q] = fmaf(xb[q].z, rb.z, acc[q]); acc[q] = fmaf(xb[q].w, rb.w, acc[q]);
+    }
+  }
+  for (; i < n4; i += 32) {
+    float4 ra = __ldg(r4 + i);
+#pragma unroll
+    for (int q = 0; q < kCorrRowsPerWarp; ++q) {
+      float4 x = __ldcs(rows[q] + i);
+      acc[q] = fmaf(x.x, ra.x, acc[q]); acc[q] = fmaf(x.y, ra.y, acc[q]);
+      acc[q] = fmaf(x.z, ra.z, acc[q]); acc[q] = fmaf(x.w, ra.w, acc[q]);
+    }
+  }
+#pragma unroll
+  for (int q = 0; q < kCorrRowsPerWarp; ++q) {
+    float v = acc[q];
+    for (int o = 16; o; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    if (lane == 0 && j0 + q < p.T) w.corr[(int64_t)h * p.T + j0 + q] = v;
+  }
+}
+
+// -------------------------------------------------------------- select ----
+__global__ void __launch_bounds__(1024) k_select(Problem p, Work w, int pass) {
+  const int h = w.order[blockIdx.x];
+  const int t = w.t[h];
+  int s0, s1;
+  pass_range(p, t, pass, s0, s1);
+  if (s0 >= s1) return;
+  __shared__ float sv[32];
+  __shared__ int si[32];
+  __shared__ int bad;
+  const float* c = w.corr + (int64_t)h * p.T;
+  uint8_t* sel = w.sel + (int64_t)h * p.T;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  if (threadIdx.x == 0) bad = 0;
+  __syncthreads();
+  for (int q = s0; q < s1; ++q) {
+    float bv = -INFINITY;
+    int bi = INT_MAX;
+    for (int j = threadIdx.x; j < p.T; j += blockDim.x) {
+      if (sel[j]) continue;
+      float v = c[j];
+      if (v != v) { v = -INFINITY; bad = 1; }
+      if (v > bv || (v == bv && j < bi)) { bv = v; bi = j; }
+    }
+    for (int o = 16; o; o >>= 1) {
+      float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+      int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+      if (ov > bv || (ov == bv && oi < bi)) { bv = ov; bi = oi; }
+    }
+    if (lane == 0) { sv[warp] = bv; si[warp] = bi; }
+    __syncthreads();
+    if (warp == 0) {
+      bv = lane < (int)(blockDim.x >> 5) ? sv[lane] : -INFINITY;
+      bi = lane < (int)(blockDim.x >> 5) ? si[lane] : INT_MAX;
+      for (int o = 16; o; o >>= 1) {
+        float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+        int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+        if (ov > bv || (ov == bv && oi < bi)) { bv = ov; bi = oi; }
+      }
+      if (lane == 0) {
+        if (bi == INT_MAX) {  // everything left is -inf: take the lowest free key
+          for (int j = 0; j < p.T; ++j)
+            if (!sel[j]) { bi = j; break; }
+          bad = 1;
+        }
+        const int64_t o = w.cu_t[h] + q;
+        w.picks[o] = bi;
+        w.pick_corr[o] = bv;
+        sel[bi] = 1;
+      }
+    }
+    __syncthreads();
+  }
+  if (threadIdx.x == 0 && bad) record_status(w.status + h, AM_ERR_NONFINITE);
+}
+
+// ---------------------------------------------------------------- gram ----
+// Block (a, head): G[a][b] for the new picks b ∈ [s0, s1) (and the mirror
+// G[b][a] when a is an old pick); b_vec[a] = φ_aᵀm when a is new.
+constexpr int kGramGroup = 8;
+
+// Dot products (fp64 sums of fp32 products) of one row with nb <= 8 rows.
+__device__ __forceinline__ void block_dots(const float4* ra, const float4* const* rb, int nb, int n4,
+                                           double (*red)[kGramGroup + 1], double* out) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  double acc[kGramGroup];
+#pragma unroll
+  for (int bb = 0; bb < kGramGroup; ++bb) acc[bb] = 0.0;
+  for (int i = threadIdx.x; i < n4; i += blockDim.x) {
+    const float4 x = ra[i];
+#pragma unroll
+    for (int bb = 0; bb < kGramGroup; ++bb) {
+      if (bb < nb) {
+        const float4 y = rb[bb][i];
+        acc[bb] += (double)x.x * y.x + (double)x.y * y.y + (double)x.z * y.z + (double)x.w * y.w;
+      }
+    }
+  }
+#pragma unroll
+  for (int bb = 0; bb < kGramGroup; ++bb) {
+    const double v = warp_sum(acc[bb]);
+    if (lane == 0) red[warp][bb] = v;
+  }
+  __syncthreads();
+  if (threadIdx.x < nb) {
+    double v = 0.0;
+    for (int k = 0; k < (int)(blockDim.x >> 5); ++k) v += red[k][threadIdx.x];
+    out[threadIdx.x] = v;
+  }
+  __syncthreads();
+}
+
+__global__ void __launch_bounds__(256) k_gram(Problem p, Work w, int pass) {
+  const int h = w.order[blockIdx.y];
+  const int t = w.t[h];
+  int s0, s1;
+  pass_range(p, t, pass, s0, s1);
+  const int a = blockIdx.x;
+  if (s0 >= s1 || a >= s1) return;
+  __shared__ double red[8][kGramGroup + 1];
+  __shared__ double res[kGramGroup];
+  const int64_t base = w.cu_t[h];
+  const int64_t gbase = w.cu_t2[h];
+  const int n4 = p.ldn >> 2;
+  const float* P0 = w.phiT + (int64_t)h * p.T * p.ldn;
+  const float4* ra = reinterpret_cast<const float4*>(P0 + (int64_t)w.picks[base + a] * p.ldn);
+  const float4* rb[kGramGroup];
+  for (int g0 = s0; g0 < s1; g0 += kGramGroup) {
+    const int nb = min(kGramGroup, s1 - g0);
+#pragma unroll
+    for (int bb = 0; bb < kGramGroup; ++bb)
+      rb[bb] = reinterpret_cast<const float4*>(P0 + (int64_t)w.picks[base + min(g0 + bb, s1 - 1)] * p.ldn);
+    block_dots(ra, rb, nb, n4, red, res);
+    if (threadIdx.x < nb) {
+      const int b = g0 + threadIdx.x;
+      w.G[gbase + (int64_t)a * t + b] = res[threadIdx.x];
+      if (a < s0) w.G[gbase + (int64_t)b * t + a] = res[threadIdx.x];
+    }
+    __syncthreads();
+  }
+  if (a >= s0) {   // b_a = φ_aᵀ m with the fp64 mass
+    const double2* m2 = reinterpret_cast<const double2*>(w.m + (int64_t)h * p.ldn);
+    double acc = 0.0;
+    for (int i = threadIdx.x; i < n4; i += blockDim.x) {
+      const float4 x = ra[i];
+      const double2 u = m2[2 * i], v = m2[2 * i + 1];
+      acc += (double)x.x * u.x + (double)x.y * u.y + (double)x.z * v.x + (double)x.w * v.y;
+    }
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    acc = warp_sum(acc);
+    if (lane == 0) red[warp][0] = acc;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      double v = 0.0;
+      for (int k = 0; k < (int)(blockDim.x >> 5); ++k) v += red[k][0];
+      w.bvec[base + a] = v;
+    }
+  }
+}
+
+// ---------------------------------------------------------------- NNLS ----
+// Lawson-Hanson active set on the normal equations G w = b in fp64, with
+// the Cholesky factor of G restricted to the passive set kept across refits
+// (appended to as variables enter; rebuilt when one leaves).  Entering
+// variables are added in blocks; if an entering block contains a variable
+// that will not grow, the refit continues one variable at a time.
+struct NnlsSmem {
+  double* x;      // [t] current weights (pick-slot indexed)
+  double* z;      // [t] solve buffer (factor-position indexed)
+  double* g;      // [t] gradient b − G x
+  int* P;         // [t] passive list, factor order
+  int* inP;       // [t] 1 if in P
+  int* blocked;   // [t]
+  int* add;       // [t] variables entering this outer iteration
+  double* L;      // packed factor (shared or global)
+};
+
+__host__ __device__ inline size_t nnls_vec_bytes(int t) {
+  return (size_t)t * (3 * sizeof(double) + 4 * sizeof(int)) + 64 * sizeof(double) + 16 * sizeof(int);
+}
+__host__ __device__ inline size_t nnls_tri_bytes(int t) { return (size_t)t * (t + 1) / 2 * sizeof(double); }
+constexpr size_t kSmemCap = 227 * 1024;
+
+__global__ void __launch_bounds__(kNnlsThreads) k_nnls(Problem p, Work w, int pass, int l_in_smem_max) {
+  extern __shared__ __align__(16) unsigned char smem[];
+  const int h = w.order[blockIdx.x];
+  const int t = w.t[h];
+  int s0, s1;
+  pass_range(p, t, pass, s0, s1);
+  if (s0 >= s1) return;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int np_old = w.np[h];
+  const int64_t base = w.cu_t[h];
+  const int64_t gbase = w.cu_t2[h];
+  const double* G = w.G + gbase;
+  const double* b = w.bvec + base;
+
+  NnlsSmem S;
+  S.x = reinterpret_cast<double*>(smem);
+  S.z = S.x + t;
+  S.g = S.z + t;
+  double* red = S.g + t;                       // 64 doubles
+  int* ints = reinterpret_cast<int*>(red + 64);
+  int* ctl = ints;                             // 16 ints of control
+  S.P = ints + 16;
+  S.inP = S.P + t;
+  S.blocked = S.inP + t;
+  S.add = S.blocked + t;
+  const bool l_smem = t <= l_in_smem_max;
+  double* Lg = w.L + gbase;
+  S.L = l_smem ? reinterpret_cast<double*>(S.add + t) : Lg;   // 64 + 16t bytes past red: 8-aligned
+  // ctl[0] = np, ctl[1] = nadd, ctl[2] = single_mode, ctl[3] = done/flags,
+  // ctl[4] = argmin, ctl[5] = nneg, ctl[6] = failed factor index, ctl[7] = scratch
+  const int maxit = p.nnls_max_iter > 0 ? p.nnls_max_iter : 3 * t + 50;
+  const double mnorm = sqrt(w.mm[h]);
+
+  for (int l = tid; l < s1; l += blockDim.x) {
+    S.x[l] = l < s0 ? w.w[base + l] : 0.0;
+    S.inP[l] = 0;
+    S.blocked[l] = 0;
+  }
+  for (int q = tid; q < np_old; q += blockDim.x) S.P[q] = w.plist[base + q];
+  if (l_smem)
+    for (int64_t e = tid; e < tri(np_old, 0); e += blockDim.x) S.L[e] = Lg[e];
+  if (tid == 0) { ctl[0] = np_old; ctl[2] = 0; ctl[3] = 0; }
+  __syncthreads();
+  for (int q = tid; q < np_old; q += blockDim.x) S.inP[S.P[q]] = 1;
+  __syncthreads();
+
+  auto diag = [&](int l) { return G[(int64_t)l * t + l]; };
+  int iter = 0;
+  bool converged = false;
+
+  // Rebuild the factor of G[P, P] from scratch; drops dependent variables.
+  auto refactor = [&]() {
+    for (;;) {
+      const int np = ctl[0];
+      for (int a = warp; a < np; a += blockDim.x >> 5)
+        for (int c = lane; c <= a; c += 32) S.L[tri(a, c)] = G[(int64_t)S.P[a] * t + S.P[c]];
+      __syncthreads();
+      int badk = block_cholesky_packed(S.L, np, [&](int k) { return 1e-13 * diag(S.P[k]); }, &ctl[6]);
+      if (badk < 0) return;
+      if (tid == 0) {
+        int l = S.P[badk];
+        S.inP[l] = 0;
+        S.blocked[l] = 1;
+        S.x[l] = 0.0;
+        for (int q = badk; q + 1 < np; ++q) S.P[q] = S.P[q + 1];
+        ctl[0] = np - 1;
+      }
+      __syncthreads();
+    }
+  };
+
+  for (;;) {
+    // ---- gradient over non-passive variables, choose entering set ----
+    const int np = ctl[0];
+    for (int q = tid; q < np; q += blockDim.x) S.z[q] = S.x[S.P[q]];   // x gathered to factor order
+    __syncthreads();
+    for (int l = tid; l < s1; l += blockDim.x) {
+      double gl = -INFINITY;
+      if (!S.inP[l] && !S.blocked[l]) {
+        const double* Gl = G + (int64_t)l * t;
+        double acc = b[l];
+        for (int q = 0; q < np; ++q) acc -= Gl[S.P[q]] * S.z[q];
+        const double dl = diag(l);
+        gl = dl > 0.0 ? acc / (sqrt(dl) * mnorm) : -INFINITY;   // scale-free gradient
+      }
+      S.g[l] = gl;
+    }
+    __syncthreads();
+    if (warp == 0) {
+      const double tol = 1e-11;
+      int nadd = 0;
+      if (ctl[2]) {                         // single mode: argmax only
+        double bv = tol;
+        int bi = -1;
+        for (int l = lane; l < s1; l += 32)
+          if (S.g[l] > bv) { bv = S.g[l]; bi = l; }
+        for (int o = 16; o; o >>= 1) {
+          double ov = __shfl_xor_sync(0xffffffffu, bv, o);
+          int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+          if (ov > bv || (ov == bv && oi >= 0 && (bi < 0 || oi < bi))) { bv = ov; bi = oi; }
+        }
+        if (lane == 0 && bi >= 0) { S.add[0] = bi; nadd = 1; }
+      } else {
+        for (int l0 = 0; l0 < s1; l0 += 32) {
+          int l = l0 + lane;
+          bool c = l < s1 && S.g[l] > tol;
+          unsigned msk = __ballot_sync(0xffffffffu, c);
+          if (c) S.add[nadd + __popc(msk & ((1u << lane) - 1))] = l;
+          nadd += __popc(msk);
+        }
+      }
+      nadd = __shfl_sync(0xffffffffu, nadd, 0);
+      if (lane == 0) ctl[1] = nadd;
+    }
+    __syncthreads();
+    const int nadd = ctl[1];
+    if (nadd == 0) { converged = true; break; }
+
+    // ---- append entering variables to the factor (warp 0) ----
+    if (warp == 0) {
+      for (int e = 0; e < nadd; ++e) {
+        const int l = S.add[e];
+        const int npc = ctl[0];
+        double* row = S.L + tri(npc, 0);
+        const double* Gl = G + (int64_t)l * t;
+        for (int q = lane; q < npc; q += 32) row[q] = Gl[S.P[q]];
+        __syncwarp();
+        warp_forward_solve(S.L, row, npc);
+        double ss = 0.0;
+        for (int q = lane; q < npc; q += 32) ss += row[q] * row[q];
+        ss = warp_sum(ss);
+        const double delta = diag(l) - ss;
+        if (delta > 1e-13 * diag(l)) {
+          if (lane == 0) {
+            row[npc] = sqrt(delta);
+            S.P[npc] = l;
+            S.inP[l] = 1;
+            ctl[0] = npc + 1;
+          }
+        } else if (lane == 0) {
+          S.blocked[l] = 1;
+        }
+        __syncwarp();
+      }
+    }
+    __syncthreads();
+
+    // ---- inner loop: solve on P, step back toward feasibility ----
+    bool abort = false;
+    for (;;) {
+      if (++iter > maxit) { abort = true; break; }
+      const int npc = ctl[0];
+      for (int q = tid; q < npc; q += blockDim.x) S.z[q] = b[S.P[q]];
+      __syncthreads();
+      if (warp == 0) {
+        warp_forward_solve(S.L, S.z, npc);
+        warp_backward_solve(S.L, S.z, npc);
+      }
+      __syncthreads();
+      // min step ratio over non-positive entries
+      double best = INFINITY;
+      int bq = -1, nneg = 0;
+      for (int q = tid; q < npc; q += blockDim.x) {
+        const double zq = S.z[q];
+        if (!(zq > 0.0)) {
+          ++nneg;
+          const double xq = S.x[S.P[q]];
+          const double den = xq - zq;
+          const double ratio = den > 0.0 ? xq / den : 0.0;
+          if (ratio < best || (ratio == best && q < bq)) { best = ratio; bq = q; }
+        }
+      }
+      // block argmin
+      for (int o = 16; o; o >>= 1) {
+        double ov = __shfl_xor_sync(0xffffffffu, best, o);
+        int oq = __shfl_xor_sync(0xffffffffu, bq, o);
+        int on = __shfl_xor_sync(0xffffffffu, nneg, o);
+        nneg += on;
+        if (ov < best || (ov == best && oq >= 0 && (bq < 0 || oq < bq))) { best = ov; bq = oq; }
+      }
+      if (tid == 0) { ctl[5] = 0; }
+      __syncthreads();
+      if (lane == 0) { red[warp] = best; reinterpret_cast<int*>(red + 16)[warp] = bq; atomicAdd(&ctl[5], nneg); }
+      __syncthreads();
+      if (tid == 0) {
+        double bv = INFINITY;
+        int bi = -1;
+        for (int k = 0; k < (int)(blockDim.x >> 5); ++k) {
+          double v = red[k];
+          int qi = reinterpret_cast<int*>(red + 16)[k];
+          if (qi >= 0 && (v < bv || (v == bv && qi < bi))) { bv = v; bi = qi; }
+        }
+        red[32] = bv;
+        ctl[4] = bi;
+      }
+      __syncthreads();
+      if (ctl[5] == 0) {   // all positive: accept
+        for (int q = tid; q < npc; q += blockDim.x) S.x[S.P[q]] = S.z[q];
+        __syncthreads();
+        break;
+      }
+      const double alpha = red[32];
+      if (alpha == 0.0) {
+        // entering variables that will not grow: drop them
+        if (tid == 0) {
+          int k = 0;
+          const bool single = ctl[2];
+          for (int q = 0; q < npc; ++q) {
+            const int l = S.P[q];
+            if (!(S.z[q] > 0.0) && S.x[l] == 0.0) {
+              S.inP[l] = 0;
+              if (single) S.blocked[l] = 1;
+            } else {
+              S.P[k++] = l;
+            }
+          }
+          ctl[0] = k;
+          ctl[2] = 1;
+        }
+      } else {
+        const int qmin = ctl[4];
+        for (int q = tid; q < npc; q += blockDim.x) {
+          const int l = S.P[q];
+          double v = S.x[l] + alpha * (S.z[q] - S.x[l]);
+          if (q == qmin) v = 0.0;
+          S.x[l] = v;
+        }
+        __syncthreads();
+        if (tid == 0) {
+          int k = 0;
+          for (int q = 0; q < npc; ++q) {
+            const int l = S.P[q];
+            if (S.x[l] <= 0.0) { S.inP[l] = 0; S.x[l] = 0.0; }
+            else S.P[k++] = l;
+          }
+          ctl[0] = k;
+        }
+      }
+      __syncthreads();
+      refactor();
+      __syncthreads();
+    }
+    if (abort) break;
+  }
+  __syncthreads();
+
+  // ---- write back ----
+  const int npf = ctl[0];
+  for (int l = tid; l < s1; l += blockDim.x) w.w[base + l] = S.inP[l] ? S.x[l] : 0.0;
+  for (int q = tid; q < npf; q += blockDim.x) w.plist[base + q] = S.P[q];
+  if (l_smem)
+    for (int64_t e = tid; e < tri(npf, 0); e += blockDim.x) Lg[e] = S.L[e];
+  if (tid == 0) {
+    w.np[h] = npf;
+    if (!converged) record_status(w.status + h, AM_WARN_NOT_CONVERGED);
+  }
+}
+
+// ------------------------------------------------------------ residual ----
+// r = m − Φ_S w over all current picks; fp64 sums, fp32 store; partial ‖r‖².
+constexpr int kResidThreads = 128;
+constexpr int kResidChunk = 512;   // picks staged in shared memory at a time
+
+__global__ void __launch_bounds__(kResidThreads) k_resid(Problem p, Work w, int pass) {
+  const int h = w.order[blockIdx.y];
+  const int t = w.t[h];
+  int s0, s1;
+  pass_range(p, t, pass, s0, s1);
+  if (s0 >= s1) return;
+  __shared__ int sj[kResidChunk];
+  __shared__ double sw[kResidChunk];
+  __shared__ double scratch[33];
+  const int64_t base = w.cu_t[h];
+  const float* P0 = w.phiT + (int64_t)h * p.T * p.ldn;
+  const int n4 = p.ldn >> 2;
+  double rr = 0.0;
+  for (int i4 = blockIdx.x * kResidThreads + threadIdx.x; i4 - (int)threadIdx.x < n4;
+       i4 += gridDim.x * kResidThreads) {
+    const bool live = i4 < n4;
+    double acc[4] = {0.0, 0.0, 0.0, 0.0};
+    if (live) {
+      const double2* m2 = reinterpret_cast<const double2*>(w.m + (int64_t)h * p.ldn);
+      const double2 u = m2[2 * i4], v = m2[2 * i4 + 1];
+      acc[0] = u.x; acc[1] = u.y; acc[2] = v.x; acc[3] = v.y;
+    }
+    for (int c0 = 0; c0 < s1; c0 += kResidChunk) {
+      const int cn = min(kResidChunk, s1 - c0);
+      __syncthreads();
+      for (int q = threadIdx.x; q < cn; q += blockDim.x) {
+        sj[q] = w.picks[base + c0 + q];
+        sw[q] = w.w[base + c0 + q];
+      }
+      __syncthreads();
+      if (live) {
+        for (int q = 0; q < cn; ++q) {
+          const double wl = sw[q];
+          if (wl == 0.0) continue;
+          float4 x = reinterpret_cast<const float4*>(P0 + (int64_t)sj[q] * p.ldn)[i4];
+          acc[0] -= x.x * wl; acc[1] -= x.y * wl; acc[2] -= x.z * wl; acc[3] -= x.w * wl;
+        }
+      }
+    }
+    if (live) {
+      float4 o = make_float4((float)acc[0], (float)acc[1], (float)acc[2], (float)acc[3]);
+      reinterpret_cast<float4*>(w.r + (int64_t)h * p.ldn)[i4] = o;
+      rr += acc[0] * acc[0] + acc[1] * acc[1] + acc[2] * acc[2] + acc[3] * acc[3];
+    }
+  }
+  rr = block_sum(rr, scratch);
+  if (threadIdx.x == 0) w.rr_part[(int64_t)h * kRedBlocks + blockIdx.x] = rr;
+}
+
+__global__ void k_residual_norm(Problem p, Work w, int nblk, double* out) {
+  const int h = blockIdx.x * blockDim.x + threadIdx.x;
+  if (h >= p.H) return;
+  double s = 0.0;
+  for (int k = 0; k < nblk; ++k) s += w.rr_part[(int64_t)h * kRedBlocks + k];
+  out[h] = sqrt(s / w.mm[h]);
+}
+
+int resid_blocks(const Problem& p) {
+  int n4 = p.ldn / 4;
+  int b = (n4 + kResidThreads - 1) / kResidThreads;
+  return b < kRedBlocks ? b : kRedBlocks;
+}
+
+}  // namespace
+
+// Dynamic shared memory of k_nnls: the vectors for max_t, plus the packed
+// factor for the largest tl <= max_t that still fits; heads with t <= tl keep
+// their factor in shared memory, larger ones in the workspace.
+size_t nnls_smem_bytes(int max_t, int* l_in_smem_max) {
+  const size_t vec = nnls_vec_bytes(max_t);
+  int tl = 0;
+  while (tl < max_t && vec + nnls_tri_bytes(tl + 1) <= kSmemCap) ++tl;
+  *l_in_smem_max = tl;
+  return vec + nnls_tri_bytes(tl);
+}
+
+cudaError_t launch_omp_init(const Problem& p, const Work& w, cudaStream_t s) {
+  AM_LAUNCH(AM_STAGE_INIT, s, k_init<<<p.H, 256, 0, s>>>(p, w));
+  return cudaGetLastError();
+}
+
+cudaError_t launch_omp_pass(const Problem& p, const Work& w, int pass, int active, cudaStream_t s) {
+  if (active <= 0) return cudaSuccess;
+  dim3 gc((p.T + kCorrRowsPerBlock - 1) / kCorrRowsPerBlock, active);
+  AM_LAUNCH(AM_STAGE_CORR, s, k_corr<<<gc, 256, 0, s>>>(p, w, pass));
+  AM_LAUNCH(AM_STAGE_SELECT, s, k_select<<<active, 1024, 0, s>>>(p, w, pass));
+  const int s1max = (pass + 1) * p.kR < p.max_t ? (pass + 1) * p.kR : p.max_t;
+  dim3 gg(s1max, active);
+  AM_LAUNCH(AM_STAGE_GRAM, s, k_gram<<<gg, 256, 0, s>>>(p, w, pass));
+  int lcap;
+  size_t sm = nnls_smem_bytes(p.max_t, &lcap);
+  cudaFuncSetAttribute(k_nnls, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemCap);
+  AM_LAUNCH(AM_STAGE_NNLS, s, k_nnls<<<active, kNnlsThreads, sm, s>>>(p, w, pass, lcap));
+  dim3 gr(resid_blocks(p), active);
+  AM_LAUNCH(AM_STAGE_RESID, s, k_resid<<<gr, kResidThreads, 0, s>>>(p, w, pass));
+  return cudaGetLastError();
+}
+
+cudaError_t launch_residual_norm(const Problem& p, const Work& w, double* out, cudaStream_t s) {
+  AM_LAUNCH(AM_STAGE_RESID, s, k_residual_norm<<<(p.H + 127) / 128, 128, 0, s>>>(p, w, resid_blocks(p), out));
+  return cudaGetLastError();
+}
+
+}  // namespace am

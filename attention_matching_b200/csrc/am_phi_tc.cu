@@ -1,0 +1,516 @@
+// Feature pass on the 5th-generation tensor cores (tcgen05, TMEM, TMA) for
+// bf16 inputs with d in {64, 128}.
+//
+// "Fast KV Compaction via Attention Matching", zhichai.net deep dive §1.6:
+// Φ_ij = exp(q_i·k_j) and m_i = Σ_j Φ_ij (with the 1/√d scale, an optional
+// prior key bias and one per-head shift); xinfinite.net article §2 step 3:
+// the value fit targets the original local attention output Y = ΦV/m.
+//
+// One CTA per (head, 128-query block), 8 warps:
+//   warp 0   TMA producer: the query block once, then (key, value) tiles of
+//            64 keys through a 3-stage ring
+//   warp 1   MMA issuer (one thread): S = Q·Kᵀ into one of two TMEM
+//            accumulators (kind::f16, bf16 in, fp32 out), then Y += P·V
+//            from the epilogue's P tiles (PHI mode)
+//   warp 2   TMEM allocation and release
+//   warps 4-7 epilogue: thread r owns query row r (TMEM lane r); per tile it
+//            reads 64 logits, forms p = exp(s·scale + b − c), adds p to the
+//            fp64 mass, writes Φᵀ (a warp writes 32 consecutive queries of one
+//            key: 128-byte coalesced), and stores p split as bf16 hi + lo
+//            (p = hi + lo to 16 bits) into a swizzled K-major operand for Y.
+// MAX mode computes only max_ij (s·scale + b) per head (the shift).
+//
+// Every mbarrier wait is bounded by a clock budget; on expiry the CTA records
+// AM_ERR_TIMEOUT, stops issuing work, drains what it issued and releases TMEM.
+#include "am_internal.cuh"
+#include "am_profile.cuh"
+
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <float.h>
+
+namespace am {
+namespace {
+
+constexpr int BM = 128;        // queries per CTA (TMEM lanes)
+constexpr int BN = 64;         // keys per tile
+constexpr int STAGES = 3;      // key/value ring depth
+constexpr int kThreads = 256;
+constexpr int kEpiWarp0 = 4;   // first epilogue warp
+constexpr uint32_t kTmemCols = 256;
+constexpr long long kWaitBudgetCycles = 4000000000ll;   // ~2 s at 2 GHz
+
+enum Mode { MODE_MAX = 0, MODE_PHI = 1 };
+
+// ---- shared-memory plan (bytes); operand tiles 1024-aligned for SW128 ----
+struct Plan {
+  int d;
+  uint32_t q_bytes, k_bytes, v_bytes, p_bytes;
+  uint32_t off_q, off_k, off_v, off_p, off_bias, off_bar, total;
+};
+
+__host__ __device__ inline Plan make_plan(int d, int mode) {
+  Plan P{};
+  P.d = d;
+  P.q_bytes = BM * d * 2;
+  P.k_bytes = BN * d * 2;
+  P.v_bytes = mode == MODE_PHI ? BN * d * 2 : 0;
+  P.p_bytes = mode == MODE_PHI ? BM * BN * 2 : 0;   // one of hi / lo
+  uint32_t o = 0;
+  P.off_q = o; o += P.q_bytes;
+  P.off_k = o; o += STAGES * P.k_bytes;
+  P.off_v = o; o += STAGES * P.v_bytes;
+  P.off_p = o; o += 2 * 2 * P.p_bytes;               // 2 buffers × (hi, lo)
+  P.off_bias = o; o += 2 * BN * 4;
+  P.off_bar = o; o += 32 * 8;
+  P.total = o + 1024;                                 // slack to align the base
+  return P;
+}
+
+// ---- PTX wrappers ----
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count));
+}
+
+__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
+               : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Bounded wait: false if the CTA aborted (here or elsewhere) before completion.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
+                                          int32_t* status) {
+  const long long t0 = clock64();
+  while (!mbar_try_wait(bar, parity)) {
+    if (*abort_flag) return false;
+    if (clock64() - t0 > kWaitBudgetCycles) {
+      *abort_flag = 1;
+      record_status(status, AM_ERR_TIMEOUT);
+      return false;
+    }
+  }
+  return true;
+}
+
+__device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, uint64_t* bar, int x, int y,
+                                            int z) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cta.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4, %5}], [%2];"
+      ::"r"(smem_u32(dst)), "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x), "r"(y), "r"(z)
+      : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+__device__ __forceinline__ void tc_commit(uint64_t* bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
+               : "memory");
+}
+
+__device__ __forceinline__ void tc_mma(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                       uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}"
+      ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// 32 lanes × 32 consecutive 32-bit columns: thread t gets row (lane base + t).
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
+  uint32_t r[32];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+        "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+        "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+#pragma unroll
+  for (int k = 0; k < 32; ++k) v[k] = __uint_as_float(r[k]);
+}
+
+__device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+
+// Shared-memory matrix descriptor, SWIZZLE_128B (sm_100 encoding 2), version 1.
+__device__ __forceinline__ uint64_t smem_desc(uint32_t addr, uint32_t lbo_bytes, uint32_t sbo_bytes) {
+  uint64_t desc = 0;
+  desc |= (uint64_t)((addr >> 4) & 0x3FFF);
+  desc |= (uint64_t)((lbo_bytes >> 4) & 0x3FFF) << 16;
+  desc |= (uint64_t)((sbo_bytes >> 4) & 0x3FFF) << 32;
+  desc |= (uint64_t)1 << 46;                       // version
+  desc |= (uint64_t)2 << 61;                       // SWIZZLE_128B
+  return desc;
+}
+
+// Instruction descriptor, kind::f16: bf16 A/B, fp32 D, M = 128.
+__host__ __device__ constexpr uint32_t instr_desc(int n, bool b_mn_major) {
+  return (1u << 4)                       // D format F32
+         | (1u << 7)                     // A format BF16
+         | (1u << 10)                    // B format BF16
+         | ((b_mn_major ? 1u : 0u) << 16)
+         | ((uint32_t)(n >> 3) << 17)    // N >> 3
+         | ((uint32_t)(BM >> 4) << 24);  // M >> 4
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+
+__device__ __forceinline__ uint32_t f2ord(float f) {
+  uint32_t u = __float_as_uint(f);
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+template <int D, int MODE>
+__global__ void __launch_bounds__(kThreads, 1)
+k_phi_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+         const __grid_constant__ CUtensorMap tmV, Problem p, Work w, const float* __restrict__ key_bias,
+         uint32_t* __restrict__ shift_ord) {
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  constexpr int KB = D / 64;                       // 128-byte K-blocks per row
+  const Plan P = make_plan(D, MODE);
+  unsigned char* sm = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  unsigned char* sQ = sm + P.off_q;
+  unsigned char* sK = sm + P.off_k;
+  unsigned char* sV = sm + P.off_v;
+  unsigned char* sP = sm + P.off_p;
+  float* sBias = reinterpret_cast<float*>(sm + P.off_bias);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sm + P.off_bar);
+  uint64_t* q_full = bars + 0;
+  uint64_t* kv_full = bars + 1;             // [STAGES]
+  uint64_t* kv_empty = bars + 1 + STAGES;   // [STAGES]
+  uint64_t* s_full = bars + 1 + 2 * STAGES; // [2]
+  uint64_t* s_empty = s_full + 2;           // [2]
+  uint64_t* p_full = s_full + 4;            // [2]
+  uint64_t* p_empty = s_full + 6;           // [2]
+  uint64_t* y_full = s_full + 8;
+  uint64_t* drain = s_full + 9;
+  __shared__ uint32_t s_tmem;
+  __shared__ int s_abort;
+  __shared__ float s_red[4];
+  __shared__ int s_stop[2];
+  __shared__ int s_stop_y;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int nqb = (p.n + BM - 1) / BM;
+  const int h = blockIdx.x / nqb;
+  const int q0 = (blockIdx.x % nqb) * BM;
+  const int NT = (p.T + BN - 1) / BN;
+  int32_t* status = w.status + h;
+  volatile int* abort_flag = &s_abort;
+
+  if (threadIdx.x == 0) {
+    s_abort = 0;
+    mbar_init(q_full, 1);
+    for (int s = 0; s < STAGES; ++s) { mbar_init(kv_full + s, 1); mbar_init(kv_empty + s, 1); }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(s_full + b, 1);
+      mbar_init(s_empty + b, 128);
+      mbar_init(p_full + b, 128);
+      mbar_init(p_empty + b, 1);
+    }
+    mbar_init(y_full, 1);
+    mbar_init(drain, 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 2) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(&s_tmem)),
+                 "r"(kTmemCols));
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = s_tmem;
+  const uint32_t tS[2] = {tmem, tmem + BN};
+  const uint32_t tY = tmem + 2 * BN;
+
+  if (warp == 0) {
+    // ------------------------------------------------ TMA producer ----
+    if (lane == 0) {
+      mbar_expect_tx(q_full, P.q_bytes);
+      for (int kb = 0; kb < KB; ++kb) tma_load_3d(sQ + kb * BM * 128, &tmQ, q_full, kb * 64, q0, h);
+      int issued[STAGES] = {};
+      for (int j = 0; j < NT; ++j) {
+        const int s = j % STAGES, use = j / STAGES;
+        if (use > 0 && !mbar_wait(kv_empty + s, (use - 1) & 1, abort_flag, status)) break;
+        mbar_expect_tx(kv_full + s, P.k_bytes + P.v_bytes);
+        for (int kb = 0; kb < KB; ++kb)
+          tma_load_3d(sK + s * P.k_bytes + kb * BN * 128, &tmK, kv_full + s, kb * 64, j * BN, h);
+        if (MODE == MODE_PHI)
+          for (int kb = 0; kb < KB; ++kb)
+            tma_load_3d(sV + s * P.v_bytes + kb * BN * 128, &tmV, kv_full + s, kb * 64, j * BN, h);
+        issued[s] = use + 1;
+      }
+      // copies still in flight must land before the CTA releases its memory
+      mbar_wait(q_full, 0, abort_flag, status);
+      for (int s = 0; s < STAGES; ++s)
+        if (issued[s] > 0) {
+          const long long t0 = clock64();
+          while (!mbar_try_wait(kv_full + s, (issued[s] - 1) & 1) && clock64() - t0 < kWaitBudgetCycles) {}
+        }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------- MMA issuer ----
+    if (lane == 0) {
+      const uint32_t idesc1 = instr_desc(BN, false);
+      const uint32_t idesc2 = instr_desc(D, true);
+      bool ok = mbar_wait(q_full, 0, abort_flag, status);
+      tc_fence_after();
+      auto gemm2 = [&](int jj) -> bool {
+        const int b = jj & 1, bu = jj >> 1, s = jj % STAGES;
+        if (!mbar_wait(p_full + b, bu & 1, abort_flag, status)) return false;
+        tc_fence_after();
+        const uint32_t vbase = smem_u32(sV + s * P.v_bytes);
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+          const uint32_t pbase = smem_u32(sP + (b * 2 + half) * P.p_bytes);
+#pragma unroll
+          for (int kk = 0; kk < BN / 16; ++kk) {
+            const uint64_t ad = smem_desc(pbase + kk * 32, 16, 1024);
+            const uint64_t bd = smem_desc(vbase + kk * 16 * 128, BN * 128, 1024);
+            tc_mma(tY, ad, bd, idesc2, (jj > 0 || half > 0 || kk > 0) ? 1u : 0u);
+          }
+        }
+        tc_commit(p_empty + b);
+        tc_commit(kv_empty + s);
+        return true;
+      };
+      int j = 0;
+      for (; ok && j < NT; ++j) {
+        const int s = j % STAGES, use = j / STAGES, b = j & 1, bu = j >> 1;
+        if (!mbar_wait(kv_full + s, use & 1, abort_flag, status)) { ok = false; break; }
+        if (bu > 0 && !mbar_wait(s_empty + b, (bu - 1) & 1, abort_flag, status)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t qbase = smem_u32(sQ), kbase = smem_u32(sK + s * P.k_bytes);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t koff = kk >> 2;   // 128-byte K-block
+          const uint64_t ad = smem_desc(qbase + koff * BM * 128 + (kk & 3) * 32, 16, 1024);
+          const uint64_t bd = smem_desc(kbase + koff * BN * 128 + (kk & 3) * 32, 16, 1024);
+          tc_mma(tS[b], ad, bd, idesc1, kk > 0 ? 1u : 0u);
+        }
+        tc_commit(s_full + b);
+        if (MODE == MODE_MAX) tc_commit(kv_empty + s);
+        if (MODE == MODE_PHI && j > 0 && !gemm2(j - 1)) { ok = false; break; }
+      }
+      if (MODE == MODE_PHI && ok && NT > 0) ok = gemm2(NT - 1);
+      if (MODE == MODE_PHI) tc_commit(y_full);
+      // drain: every MMA this thread issued has completed before TMEM is freed
+      tc_commit(drain);
+      const long long t0 = clock64();
+      while (!mbar_try_wait(drain, 0) && clock64() - t0 < kWaitBudgetCycles) {}
+    }
+  } else if (warp >= kEpiWarp0) {
+    // --------------------------------------------------- epilogue ----
+    const int et = threadIdx.x - kEpiWarp0 * 32;     // 0..127 = TMEM lane = query row
+    const int qd = warp - kEpiWarp0;                 // lane quadrant
+    const int i = q0 + et;
+    const bool row_live = i < p.n;
+    const float scale = p.scale;
+    const float c = MODE == MODE_PHI ? w.shift[h] : 0.f;
+    double mrow = 0.0;
+    float mx = -FLT_MAX;
+    const uint32_t lane_addr = (uint32_t)(qd * 32) << 16;
+    float* phi_base = w.phiT + (int64_t)h * p.T * p.ldn;
+    bool ok = true;
+    for (int j = 0; j < NT; ++j) {
+      const int b = j & 1, bu = j >> 1;
+      // One thread waits (S tile ready; P buffer free again) and publishes a
+      // stop flag, so all 128 epilogue threads leave the loop together.
+      if (et == 0) {
+        bool good = mbar_wait(s_full + b, bu & 1, abort_flag, status);
+        if (good && MODE == MODE_PHI && bu > 0) good = mbar_wait(p_empty + b, (bu - 1) & 1, abort_flag, status);
+        s_stop[b] = good ? 0 : 1;
+      }
+      // this tile's (bias − shift) per key, shared by the 128 rows
+      if (et < BN) {
+        const int jg = j * BN + et;
+        const float bj = (p.has_bias && jg < p.T) ? key_bias[(int64_t)h * p.T + jg] : 0.f;
+        sBias[b * BN + et] = MODE == MODE_PHI ? bj - c : bj;
+      }
+      asm volatile("bar.sync 1, 128;" ::: "memory");
+      if (s_stop[b]) { ok = false; break; }
+      tc_fence_after();
+      float v[BN];
+      tmem_ld32(tS[b] + lane_addr, *reinterpret_cast<float(*)[32]>(&v[0]));
+      tmem_ld32(tS[b] + lane_addr + 32, *reinterpret_cast<float(*)[32]>(&v[32]));
+      tmem_wait_ld();
+      tc_fence_before();
+      mbar_arrive(s_empty + b);
+      const int kvalid = min(BN, p.T - j * BN);
+      const float* bias_t = sBias + b * BN;
+      if constexpr (MODE == MODE_MAX) {
+        if (row_live) {
+#pragma unroll
+          for (int cc = 0; cc < BN; ++cc)
+            if (cc < kvalid) mx = fmaxf(mx, fmaf(v[cc], scale, bias_t[cc]));
+        }
+        continue;
+      } else {
+      // p = exp(s·scale + b − c): one rounding of the argument
+#pragma unroll
+      for (int cc = 0; cc < BN; ++cc) {
+        const float x = fmaf(v[cc], scale, bias_t[cc]);
+        v[cc] = (row_live && cc < kvalid) ? expf(x) : 0.f;
+      }
+      double part = 0.0;
+#pragma unroll
+      for (int cc = 0; cc < BN; ++cc) part += (double)v[cc];
+      mrow += part;
+      if (i < p.ldn) {
+        float* col = phi_base + (int64_t)(j * BN) * p.ldn + i;
+#pragma unroll
+        for (int cc = 0; cc < BN; ++cc)
+          if (cc < kvalid) col[(int64_t)cc * p.ldn] = v[cc];
+      }
+      // P tile for Y += P·V: K-major, 128-byte rows, 16-byte chunks XOR-swizzled by row
+      unsigned char* hi_row = sP + (b * 2 + 0) * P.p_bytes + et * 128;
+      unsigned char* lo_row = sP + (b * 2 + 1) * P.p_bytes + et * 128;
+#pragma unroll
+      for (int ch = 0; ch < 8; ++ch) {
+        uint32_t hv[4], lv[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float a0 = v[ch * 8 + 2 * e], a1 = v[ch * 8 + 2 * e + 1];
+          const float h0 = __bfloat162float(__float2bfloat16_rn(a0));
+          const float h1 = __bfloat162float(__float2bfloat16_rn(a1));
+          hv[e] = pack_bf16x2(h0, h1);
+          lv[e] = pack_bf16x2(a0 - h0, a1 - h1);
+        }
+        const int pc = ch ^ (et & 7);
+        *reinterpret_cast<uint4*>(hi_row + pc * 16) = make_uint4(hv[0], hv[1], hv[2], hv[3]);
+        *reinterpret_cast<uint4*>(lo_row + pc * 16) = make_uint4(lv[0], lv[1], lv[2], lv[3]);
+      }
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      mbar_arrive(p_full + b);
+      }
+    }
+    if (MODE == MODE_MAX) {
+      for (int o = 16; o; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+      if (lane == 0) s_red[qd] = mx;
+      asm volatile("bar.sync 1, 128;" ::: "memory");
+      if (et == 0) {
+        const float v = fmaxf(fmaxf(s_red[0], s_red[1]), fmaxf(s_red[2], s_red[3]));
+        atomicMax(shift_ord + h, f2ord(v));
+      }
+    } else {
+      if (et == 0) s_stop_y = (ok && mbar_wait(y_full, 0, abort_flag, status)) ? 0 : 1;
+      asm volatile("bar.sync 1, 128;" ::: "memory");
+      if (!s_stop_y) {
+        tc_fence_after();
+        float* yrow = w.Y + ((int64_t)h * p.n + i) * p.d;
+#pragma unroll
+        for (int c0 = 0; c0 < D; c0 += 32) {
+          float y[32];
+          tmem_ld32(tY + lane_addr + c0, y);
+          tmem_wait_ld();
+          if (row_live) {
+#pragma unroll
+            for (int cc = 0; cc < 32; cc += 4)
+              *reinterpret_cast<float4*>(yrow + c0 + cc) =
+                  make_float4((float)(y[cc] / mrow), (float)(y[cc + 1] / mrow), (float)(y[cc + 2] / mrow),
+                              (float)(y[cc + 3] / mrow));
+          }
+        }
+        if (i < p.ldn) {
+          const double mv = row_live ? mrow : 0.0;
+          w.m[(int64_t)h * p.ldn + i] = mv;
+          w.r[(int64_t)h * p.ldn + i] = (float)mv;
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 2) asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols));
+}
+
+// ---- host: tensor maps ----
+PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    cudaDriverEntryPointQueryResult q;
+    void* ptr = nullptr;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+  }
+  return fn;
+}
+
+// [H][rows][d] bf16, box = 64 elements (128 B) × box_rows × 1, 128-byte swizzle.
+bool make_map(CUtensorMap* map, const void* base, int H, int rows, int d, int box_rows) {
+  auto enc = get_encode();
+  if (!enc) return false;
+  cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)rows, (cuuint64_t)H};
+  cuuint64_t strides[2] = {(cuuint64_t)d * 2, (cuuint64_t)rows * d * 2};
+  cuuint32_t box[3] = {64, (cuuint32_t)box_rows, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+template <int D, int MODE>
+cudaError_t launch_tc(const Problem& p, const void* Q, const void* K, const void* V, const float* key_bias,
+                      const Work& w, uint32_t* shift_ord, cudaStream_t s) {
+  CUtensorMap mq, mk, mv;
+  if (!make_map(&mq, Q, p.H, p.n, D, BM) || !make_map(&mk, K, p.H, p.T, D, BN) ||
+      !make_map(&mv, MODE == MODE_PHI ? V : K, p.H, p.T, D, BN))
+    return cudaErrorInvalidValue;
+  const Plan P = make_plan(D, MODE);
+  auto kern = k_phi_tc<D, MODE>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)P.total);
+  if (e != cudaSuccess) return e;
+  const int grid = p.H * ((p.n + BM - 1) / BM);
+  AM_LAUNCH(MODE == MODE_PHI ? AM_STAGE_PHI : AM_STAGE_SHIFT, s,
+            kern<<<grid, kThreads, P.total, s>>>(mq, mk, mv, p, w, key_bias, shift_ord));
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+bool phi_tc_supported(const Problem& p) { return p.in_dtype == AM_BF16 && (p.d == 64 || p.d == 128); }
+
+cudaError_t launch_shift_max_tc(const Problem& p, const void* Q, const void* K, const float* key_bias,
+                                const Work& w, uint32_t* shift_ord, cudaStream_t s) {
+  return p.d == 64 ? launch_tc<64, MODE_MAX>(p, Q, K, nullptr, key_bias, w, shift_ord, s)
+                   : launch_tc<128, MODE_MAX>(p, Q, K, nullptr, key_bias, w, shift_ord, s);
+}
+
+cudaError_t launch_phi_tc(const Problem& p, const void* Q, const void* K, const void* V, const float* key_bias,
+                          const Work& w, cudaStream_t s) {
+  return p.d == 64 ? launch_tc<64, MODE_PHI>(p, Q, K, V, key_bias, w, nullptr, s)
+                   : launch_tc<128, MODE_PHI>(p, Q, K, V, key_bias, w, nullptr, s);
+}
+
+}  // namespace am

@@ -1,0 +1,272 @@
+// Bias, packing and value fit, batched over heads.
+//
+// "Fast KV Compaction via Attention Matching": zhichai.net deep dive §1.6
+// (β = log w); xinfinite.net article §2 step 3 and the youleyou.com rewrite
+// (with C_k and β fixed, C_v is an ordinary least-squares fit of the local
+// attention output); zhichai.net/en summary, "Engineering Practicality"
+// (varlen per-head packing of the compacted cache).
+//
+//   k_finalize  rank picks by key position; β = b_S + log max(w, floor);
+//               packed indices, β and C_k = K[S]
+//   k_design    A_il = Φ_{i,S_l} w_l / Σ_l' Φ_{i,S_l'} w_l'  (key-major [t][ldn])
+//   k_normal    AᵀA and AᵀY with fp64 sums of fp32 products
+//   k_solve     λ = ridge·tr(AᵀA)/t, Cholesky of AᵀA + λI, C_v = (AᵀA + λI)⁻¹AᵀY
+#include "am_internal.cuh"
+#include "am_profile.cuh"
+#include "am_linalg.cuh"
+
+namespace am {
+namespace {
+
+__global__ void __launch_bounds__(256) k_finalize(Problem p, Work w, const void* K,
+                                                  const float* key_bias, void* C_k, float* beta,
+                                                  int32_t* indices, float* w_out,
+                                                  int32_t* pick_order, float* pick_corr) {
+  const int h = blockIdx.x;
+  const int t = w.t[h];
+  const int64_t base = w.cu_t[h];
+  __shared__ double scratch[33];
+  // rank of each pick by key position (keys are distinct)
+  for (int l = threadIdx.x; l < t; l += blockDim.x) {
+    const int j = w.picks[base + l];
+    int rank = 0;
+    for (int q = 0; q < t; ++q) rank += w.picks[base + q] < j;
+    w.sorted_slot[base + rank] = l;
+    indices[base + rank] = j;
+  }
+  double wmax = 0.0;
+  for (int l = threadIdx.x; l < t; l += blockDim.x) wmax = fmax(wmax, w.w[base + l]);
+  for (int o = 16; o; o >>= 1) wmax = fmax(wmax, __shfl_xor_sync(0xffffffffu, wmax, o));
+  if ((threadIdx.x & 31) == 0) scratch[threadIdx.x >> 5] = wmax;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    double v = 0.0;
+    for (int k = 0; k < (int)(blockDim.x >> 5); ++k) v = fmax(v, scratch[k]);
+    scratch[32] = v;
+  }
+  __syncthreads();
+  wmax = scratch[32];
+  const double floor_w = wmax > 0.0 ? (double)p.w_floor_rel * wmax : (double)p.w_floor_rel;
+  for (int q = threadIdx.x; q < t; q += blockDim.x) {
+    const int l = w.sorted_slot[base + q];
+    const int j = w.picks[base + l];
+    const double wl = w.w[base + l];
+    const double we = fmax(wl, floor_w);
+    w.w_eff[base + q] = we;
+    const double bj = p.has_bias ? (double)key_bias[(int64_t)h * p.T + j] : 0.0;
+    beta[base + q] = (float)(bj + log(we));
+    if (w_out) w_out[base + q] = (float)wl;
+    if (pick_order) pick_order[base + l] = j;
+    if (pick_corr) pick_corr[base + l] = w.pick_corr[base + l];
+  }
+  __syncthreads();
+  // C_k rows: exact copies of the chosen keys in the input dtype
+  const int64_t total = (int64_t)t * p.d;
+  for (int64_t e = threadIdx.x; e < total; e += blockDim.x) {
+    const int q = (int)(e / p.d), c = (int)(e % p.d);
+    const int j = indices[base + q];
+    const int64_t src = ((int64_t)h * p.T + j) * p.d + c;
+    const int64_t dst = (base + q) * p.d + c;
+    if (p.in_dtype == AM_BF16)
+      reinterpret_cast<__nv_bfloat16*>(C_k)[dst] = reinterpret_cast<const __nv_bfloat16*>(K)[src];
+    else
+      reinterpret_cast<float*>(C_k)[dst] = reinterpret_cast<const float*>(K)[src];
+  }
+}
+
+constexpr int kDesignThreads = 256;
+constexpr int kDesignChunk = 256;
+
+__global__ void __launch_bounds__(kDesignThreads) k_design(Problem p, Work w) {
+  const int h = blockIdx.y;
+  const int t = w.t[h];
+  const int64_t base = w.cu_t[h];
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  __shared__ int sj[kDesignChunk];
+  __shared__ double sw[kDesignChunk];
+  const float* P0 = w.phiT + (int64_t)h * p.T * p.ldn;
+  const bool live = i < p.n;
+  double D = 0.0;
+  for (int c0 = 0; c0 < t; c0 += kDesignChunk) {
+    const int cn = min(kDesignChunk, t - c0);
+    __syncthreads();
+    for (int q = threadIdx.x; q < cn; q += blockDim.x) {
+      sj[q] = w.picks[base + w.sorted_slot[base + c0 + q]];
+      sw[q] = w.w_eff[base + c0 + q];
+    }
+    __syncthreads();
+    if (live)
+      for (int q = 0; q < cn; ++q) D += (double)P0[(int64_t)sj[q] * p.ldn + i] * sw[q];
+  }
+  const double invD = (live && D > 0.0) ? 1.0 / D : 0.0;
+  for (int c0 = 0; c0 < t; c0 += kDesignChunk) {
+    const int cn = min(kDesignChunk, t - c0);
+    __syncthreads();
+    for (int q = threadIdx.x; q < cn; q += blockDim.x) {
+      sj[q] = w.picks[base + w.sorted_slot[base + c0 + q]];
+      sw[q] = w.w_eff[base + c0 + q];
+    }
+    __syncthreads();
+    if (i < p.ldn)
+      for (int q = 0; q < cn; ++q) {
+        const double a = live ? (double)P0[(int64_t)sj[q] * p.ldn + i] * sw[q] * invD : 0.0;
+        w.A[(base + c0 + q) * p.ldn + i] = (float)a;
+      }
+  }
+}
+
+// AᵀA (upper tile triangle, mirrored) and AᵀY; one 32×32 output tile per block.
+__global__ void __launch_bounds__(256) k_normal(Problem p, Work w) {
+  const int h = blockIdx.y;
+  const int t = w.t[h];
+  const int ta = (t + 31) / 32, td = (p.d + 31) / 32;
+  const int ntri = ta * (ta + 1) / 2;
+  int tile = blockIdx.x;
+  if (tile >= ntri + ta * td) return;
+  bool gram = tile < ntri;
+  int ta0, tb0;   // tile row/col
+  if (gram) {
+    int r = 0;
+    while (tile >= ta - r) { tile -= ta - r; ++r; }
+    ta0 = r;
+    tb0 = r + tile;
+  } else {
+    tile -= ntri;
+    ta0 = tile / td;
+    tb0 = tile % td;
+  }
+  const int a0 = ta0 * 32, b0 = tb0 * 32;
+  const int64_t base = w.cu_t[h];
+  __shared__ float As[32][33];
+  __shared__ float Bs[32][33];
+  const int tx = threadIdx.x % 16, ty = threadIdx.x / 16;
+  double acc[2][2] = {{0.0, 0.0}, {0.0, 0.0}};
+  const float* Yh = w.Y + (int64_t)h * p.n * p.d;
+  for (int i0 = 0; i0 < p.n; i0 += 32) {
+    __syncthreads();
+    for (int e = threadIdx.x; e < 32 * 32; e += blockDim.x) {
+      const int rr = e / 32, ii = e % 32;
+      const int a = a0 + rr, i = i0 + ii;
+      As[ii][rr] = (a < t && i < p.n) ? w.A[(base + a) * p.ldn + i] : 0.f;
+      if (gram) {
+        const int b = b0 + rr;
+        Bs[ii][rr] = (b < t && i < p.n) ? w.A[(base + b) * p.ldn + i] : 0.f;
+      }
+    }
+    if (!gram) {
+      for (int e = threadIdx.x; e < 32 * 32; e += blockDim.x) {
+        const int ii = e / 32, cc = e % 32;
+        const int i = i0 + ii, c = b0 + cc;
+        Bs[ii][cc] = (i < p.n && c < p.d) ? Yh[(int64_t)i * p.d + c] : 0.f;
+      }
+    }
+    __syncthreads();
+#pragma unroll 8
+    for (int ii = 0; ii < 32; ++ii) {
+      const double x0 = As[ii][ty * 2], x1 = As[ii][ty * 2 + 1];
+      const double y0 = Bs[ii][tx * 2], y1 = Bs[ii][tx * 2 + 1];
+      acc[0][0] += x0 * y0; acc[0][1] += x0 * y1;
+      acc[1][0] += x1 * y0; acc[1][1] += x1 * y1;
+    }
+  }
+  const int64_t gbase = w.cu_t2[h];
+#pragma unroll
+  for (int u = 0; u < 2; ++u)
+#pragma unroll
+    for (int v = 0; v < 2; ++v) {
+      const int a = a0 + ty * 2 + u, b = b0 + tx * 2 + v;
+      if (gram) {
+        if (a < t && b < t) {
+          w.AtA[gbase + (int64_t)a * t + b] = acc[u][v];
+          w.AtA[gbase + (int64_t)b * t + a] = acc[u][v];
+        }
+      } else if (a < t && b < p.d) {
+        w.AtY[(base + a) * p.d + b] = acc[u][v];
+      }
+    }
+}
+
+__global__ void __launch_bounds__(kCholThreads) k_solve(Problem p, Work w, float* C_v, int l_smem_max) {
+  extern __shared__ __align__(16) unsigned char smem[];
+  const int h = blockIdx.x;
+  const int t = w.t[h];
+  const int64_t base = w.cu_t[h];
+  const int64_t gbase = w.cu_t2[h];
+  __shared__ double scratch[33];
+  __shared__ int flag;
+  const double* M = w.AtA + gbase;
+  double tr = 0.0;
+  for (int a = threadIdx.x; a < t; a += blockDim.x) tr += M[(int64_t)a * t + a];
+  tr = block_sum(tr, scratch);
+  const double lam = (double)p.ridge * tr / t;
+  double* L = t <= l_smem_max ? reinterpret_cast<double*>(smem) : w.L + gbase;
+  for (int a = threadIdx.x >> 5; a < t; a += blockDim.x >> 5)
+    for (int c = threadIdx.x & 31; c <= a; c += 32)
+      L[tri(a, c)] = M[(int64_t)a * t + c] + (a == c ? lam : 0.0);
+  __syncthreads();
+  const int bad = block_cholesky_packed(L, t, [](int) { return 0.0; }, &flag);
+  double* X = w.AtY + base * p.d;
+  if (bad >= 0) {
+    if (threadIdx.x == 0) record_status(w.status + h, AM_ERR_NOT_SPD);
+    for (int64_t e = threadIdx.x; e < (int64_t)t * p.d; e += blockDim.x) C_v[base * p.d + e] = 0.f;
+    return;
+  }
+  // one right-hand-side column per thread; four partial sums for ILP
+  for (int c = threadIdx.x; c < p.d; c += blockDim.x) {
+    for (int k = 0; k < t; ++k) {
+      const double* Lk = L + tri(k, 0);
+      double s0 = X[(int64_t)k * p.d + c], s1 = 0.0, s2 = 0.0, s3 = 0.0;
+      int j = 0;
+      for (; j + 3 < k; j += 4) {
+        s0 -= Lk[j] * X[(int64_t)j * p.d + c];
+        s1 -= Lk[j + 1] * X[(int64_t)(j + 1) * p.d + c];
+        s2 -= Lk[j + 2] * X[(int64_t)(j + 2) * p.d + c];
+        s3 -= Lk[j + 3] * X[(int64_t)(j + 3) * p.d + c];
+      }
+      for (; j < k; ++j) s0 -= Lk[j] * X[(int64_t)j * p.d + c];
+      X[(int64_t)k * p.d + c] = ((s0 + s1) + (s2 + s3)) / Lk[k];
+    }
+    for (int k = t - 1; k >= 0; --k) {
+      double s0 = X[(int64_t)k * p.d + c], s1 = 0.0, s2 = 0.0, s3 = 0.0;
+      int j = k + 1;
+      for (; j + 3 < t; j += 4) {
+        s0 -= L[tri(j, k)] * X[(int64_t)j * p.d + c];
+        s1 -= L[tri(j + 1, k)] * X[(int64_t)(j + 1) * p.d + c];
+        s2 -= L[tri(j + 2, k)] * X[(int64_t)(j + 2) * p.d + c];
+        s3 -= L[tri(j + 3, k)] * X[(int64_t)(j + 3) * p.d + c];
+      }
+      for (; j < t; ++j) s0 -= L[tri(j, k)] * X[(int64_t)j * p.d + c];
+      const double xk = ((s0 + s1) + (s2 + s3)) / L[tri(k, k)];
+      X[(int64_t)k * p.d + c] = xk;
+      C_v[(base + k) * p.d + c] = (float)xk;
+    }
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_finalize(const Problem& p, const Work& w, const void* K, const float* key_bias,
+                            void* C_k, float* beta, int32_t* indices, float* w_out,
+                            int32_t* pick_order, float* pick_corr, cudaStream_t s) {
+  AM_LAUNCH(AM_STAGE_FINALIZE, s, k_finalize<<<p.H, 256, 0, s>>>(p, w, K, key_bias, C_k, beta, indices, w_out, pick_order, pick_corr));
+  return cudaGetLastError();
+}
+
+cudaError_t launch_value_fit(const Problem& p, const Work& w, float* C_v, cudaStream_t s) {
+  dim3 gd((p.ldn + kDesignThreads - 1) / kDesignThreads, p.H);
+  AM_LAUNCH(AM_STAGE_DESIGN, s, k_design<<<gd, kDesignThreads, 0, s>>>(p, w));
+  const int ta = (p.max_t + 31) / 32, td = (p.d + 31) / 32;
+  dim3 gn(ta * (ta + 1) / 2 + ta * td, p.H);
+  AM_LAUNCH(AM_STAGE_NORMAL, s, k_normal<<<gn, 256, 0, s>>>(p, w));
+  // heads with t <= tl keep the factor in shared memory, larger ones in the
+  // workspace; 1 KB is left for the kernel's static shared memory
+  const size_t cap = 226 * 1024;
+  int tl = 0;
+  while (tl < p.max_t && (size_t)(tl + 1) * (tl + 2) / 2 * sizeof(double) <= cap) ++tl;
+  const size_t sm = (size_t)tl * (tl + 1) / 2 * sizeof(double);
+  cudaFuncSetAttribute(k_solve, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)cap);
+  AM_LAUNCH(AM_STAGE_SOLVE, s, k_solve<<<p.H, kCholThreads, sm, s>>>(p, w, C_v, tl));
+  return cudaGetLastError();
+}
+
+}  // namespace am

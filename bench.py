@@ -1,0 +1,387 @@
+#!/usr/bin/env python
+"""Throughput of AM-OMP KV compaction on B200: KV-head compactions per second.
+
+One step = one am_compact_heads call over a batch of synthetic heads already
+resident in HBM: shift → Φ pass → OMP passes (correlation, selection, Gram,
+NNLS, residual) → β, packing → value fit.  Default workload: one
+Qwen3-4B-shaped layer (8 KV heads, T = n = 8192, d = 128, bf16, 50×
+budget t = 164, top-k 4 with a refit every 2 rounds).
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+N > 1 runs under torch.distributed.run, one rank per GPU; every rank
+compacts its own heads (the problems are independent: weak scaling, no
+collective on the data path); the timed region is bracketed by a barrier and
+a device synchronize and the time is the max over ranks.
+
+Timing: per-step CUDA events on the compute stream; a 256 MiB buffer is
+written between timed steps to flush L2.  Stage times come from the
+library's own event brackets (am_profile_*), giving the live roofline of the
+dominant kernel.  `--impl reference` times the float64 CPU oracle on a
+bounded sample of the same workload instead.
+"""
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "KV-head compactions/sec and seconds per full-model compaction, 1 B200"
+LAYERS_QWEN3_4B = 36
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="qwen3_4b_layer",
+                    choices=["qwen3_4b_layer", "single_head_fp32", "qwen3_4b_model"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    return ap.parse_args()
+
+
+def build_workload(name, rank):
+    from attention_matching_b200 import workloads as W
+    if name == "qwen3_4b_layer":
+        return W.qwen3_4b_layer(seed_base=2000 + 1000 * rank)
+    if name == "qwen3_4b_model":
+        return W.qwen3_4b_model(seed_base=4000 + 1000 * rank)
+    return W.single_head_fp32(seed=1000 + rank)
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            pk = json.load(f)
+        return {"hbm_gbs": float(pk["hbm_gbs"]), "bf16_tflops": float(pk["bf16_tflops"]),
+                "bf16_tflops_sustained": float(pk.get("bf16_tflops_sustained", pk["bf16_tflops"])),
+                "sm_max_mhz": float(pk.get("sm_max_mhz", 1965.0)), "source": "measured"}
+    except Exception:
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+                "sm_max_mhz": 1965.0, "source": "fallback"}
+
+
+# ---------------------------------------------------------------- clocks ----
+class ClockSampler:
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id):
+        self.gpu_id = gpu_id
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        cmd = ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "200"]
+        if self.gpu_id is not None:
+            cmd += ["-i", str(self.gpu_id)]
+        try:
+            self.proc = subprocess.Popen(cmd, stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except Exception:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        rows = []
+        for ln in self.lines:
+            parts = [x.strip() for x in ln.split(",")]
+            if len(parts) != 8:
+                continue
+            try:
+                rows.append((float(parts[0]), float(parts[1]), parts[4:]))
+            except ValueError:
+                continue
+        if not rows:
+            return None
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[k] for _, _, r in rows for k in range(4) if r[k].lower() == "active"})
+        return {"sm_mhz": statistics.median(r[0] for r in rows), "sm_max_mhz": max(r[1] for r in rows),
+                "reasons": reasons, "samples": len(rows)}
+
+
+def gpu_smi_id(torch, dev):
+    try:
+        u = str(torch.cuda.get_device_properties(dev).uuid)
+        return u if u.startswith("GPU-") else "GPU-" + u
+    except Exception:
+        vis = os.environ.get("CUDA_VISIBLE_DEVICES", "")
+        first = vis.split(",")[0] if vis else str(dev)
+        return first if first.isdigit() else None
+
+
+# ------------------------------------------------------------ cpu oracle ----
+def oracle_sample(wl, max_heads):
+    """Time the float64 oracle on the first heads of the workload (bounded)."""
+    import numpy as np
+    from oracle import am_oracle as O
+    try:
+        from threadpoolctl import threadpool_info
+        cores = max([x.get("num_threads", 1) for x in threadpool_info()] or [1])
+    except Exception:
+        cores = os.cpu_count() or 1
+    t0 = time.perf_counter()
+    done = 0
+    for h in range(min(max_heads, len(wl.heads))):
+        Q, K, V = wl.heads[h].f64()
+        O.compact_head(Q, K, V, wl.budgets[h], wl.topk, wl.refit_every)
+        done += 1
+    dt = time.perf_counter() - t0
+    return done, dt, cores
+
+
+def cpu_baseline(wl, heads=1):
+    done, dt, cores = oracle_sample(wl, heads)
+    return {"value": done / dt, "unit": "heads/s", "cores": cores, "kind": "oracle",
+            "sample": f"{done} of {len(wl.heads)} heads of {wl.name}, float64 NumPy/SciPy oracle, "
+                      f"{dt:.1f} s wall on the host"}
+
+
+# -------------------------------------------------------------- roofline ----
+def stage_models(wl, n, T, d, H, ldn, passes):
+    """Algorithmic bytes / flops of one launch of the main kernels."""
+    return {
+        "corr": {"bound": "hbm", "bytes": H * (T * ldn * 4 + ldn * 4 + T * 4)},
+        "phi": {"bound": "alu", "flops": 2.0 * H * n * T * d, "bytes": H * T * ldn * 4},
+        "target": {"bound": "alu", "flops": 2.0 * H * n * T * d, "bytes": H * T * ldn * 4},
+        "shift": {"bound": "alu", "flops": 2.0 * H * n * T * d},
+    }
+
+
+def roofline(stages, steps, models, peaks, clocks, traffic_info):
+    per = {k: v for k, v in stages.items() if v["launches"] > 0}
+    dom = max(per, key=lambda k: per[k]["ms"])
+    launches = per[dom]["launches"]
+    avg_ms = per[dom]["ms"] / launches
+    m = models.get(dom)
+    out = {"kernel": dom, "avg_launch_ms": avg_ms, "launches_per_step": launches / steps}
+    if m is None:
+        out.update({"bound": None, "achieved": None, "peak": None, "unit": None, "frac": None, "traffic": None})
+        return out
+    if m["bound"] == "hbm":
+        ach = m["bytes"] / (avg_ms * 1e-3) / 1e9
+        out.update({"bound": "hbm", "achieved": ach, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                    "frac": ach / peaks["hbm_gbs"], "peak_source": peaks["source"] + " hbm_gbs",
+                    "algorithmic_bytes_per_launch": m["bytes"]})
+    else:
+        # fp32 FMA pipes: 148 SMs x 128 lanes x 2 flops x SM clock
+        mhz = (clocks or {}).get("sm_mhz") or peaks["sm_max_mhz"]
+        peak = 148 * 128 * 2 * mhz * 1e6 / 1e12
+        ach = m["flops"] / (avg_ms * 1e-3) / 1e12
+        out.update({"bound": "alu", "achieved": ach, "peak": peak, "unit": "TFLOP/s", "frac": ach / peak,
+                    "peak_source": "fp32 FMA: 148 SMs x 128 lanes x 2 x median SM clock",
+                    "algorithmic_flops_per_launch": m["flops"]})
+    out["traffic"] = traffic_info.get(dom)
+    return out
+
+
+def committed_traffic():
+    """DRAM bytes per launch from the committed ncu summary, valid only while
+    the kernel sources still hash to what was profiled."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            rec = json.load(f)
+    except Exception:
+        return {}
+    out = {}
+    for k, v in rec.items():
+        src = os.path.join(ROOT, v["source"])
+        try:
+            h = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+        except Exception:
+            continue
+        if h == v["source_sha256_16"]:
+            out[k] = v["dram_bytes_per_launch"]
+    return out
+
+
+# ------------------------------------------------------------------ arms ----
+def run_reference(args, rank, world):
+    if rank != 0:
+        return 0
+    wl = build_workload(args.workload, 0)
+    per_step_heads = 1
+    times = []
+    for i in range(args.warmup + args.steps):
+        done, dt, cores = oracle_sample(wl, per_step_heads)
+        if i >= args.warmup:
+            times.append(dt / done)
+    ms = 1e3 * statistics.mean(times)
+    value = 1e3 / ms
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "heads/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": wl.name, "sample": "1 head per step"},
+        "cpu_baseline": {"value": value, "unit": "heads/s", "cores": cores, "kind": "oracle",
+                         "sample": f"1 head of {wl.name} per step, float64 oracle on the host"},
+        "e2e": {"value": value, "unit": "heads/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line))
+    return 0
+
+
+def run_ours(args, rank, world, local_rank):
+    import torch
+    import attention_matching_b200 as am
+    dist = None
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=dev)
+
+    wl = build_workload(args.workload, rank)
+    H = len(wl.heads)
+    n, T, d = wl.heads[0].n, wl.heads[0].T, wl.heads[0].d
+    Qh = torch.stack([h.Q for h in wl.heads]).contiguous()
+    Kh = torch.stack([h.K for h in wl.heads]).contiguous()
+    Vh = torch.stack([h.V for h in wl.heads]).contiguous()
+    Q, K, V = Qh.to(dev), Kh.to(dev), Vh.to(dev)
+    kw = dict(topk=wl.topk, refit_every=wl.refit_every)
+    opts = am.make_opts(am.BF16 if Q.dtype == torch.bfloat16 else am.FP32, wl.topk, wl.refit_every)
+    ws = torch.empty((am.workspace_size(n, T, d, wl.budgets, opts),), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    flush = torch.empty((256 << 20,), dtype=torch.uint8, device=dev)
+
+    first = am.compact_heads(Q, K, V, wl.budgets, workspace=ws, **kw)   # checks device status
+    for _ in range(args.warmup):
+        am.compact_heads(Q, K, V, wl.budgets, workspace=ws, check=False, **kw)
+    torch.cuda.synchronize()
+
+    clocks = ClockSampler(gpu_smi_id(torch, local_rank))
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    am.profile_enable(True)
+    l0 = am.kernel_launches()
+    evs = []
+    for _ in range(args.steps):
+        flush.fill_(1)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        am.compact_heads(Q, K, V, wl.budgets, workspace=ws, check=False, **kw)
+        b.record(stream)
+        evs.append((a, b))
+    torch.cuda.synchronize()
+    launches = am.kernel_launches() - l0
+    am.profile_enable(False)
+    stages = am.profile_collect()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    step_ms = [a.elapsed_time(b) for a, b in evs]
+    ms = statistics.mean(step_ms)
+    ms_t = torch.tensor([ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(ms_t, op=dist.ReduceOp.MAX)
+    ms = float(ms_t.item())
+    _, worst = am.get_status(ws, H)
+
+    # end to end through the public API with pinned host buffers
+    e2e = None
+    if not args.no_e2e:
+        Qp, Kp, Vp = Qh.pin_memory(), Kh.pin_memory(), Vh.pin_memory()
+        am.compact_heads(Qp, Kp, Vp, wl.budgets, workspace=ws, check=False, **kw)
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        ev2 = []
+        d2h = 0
+        for _ in range(args.steps):
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            o = am.compact_heads(Qp, Kp, Vp, wl.budgets, workspace=ws, check=False, **kw)
+            b.record(stream)
+            ev2.append((a, b))
+            d2h = sum(o[k].numel() * o[k].element_size() for k in ("C_k", "beta", "C_v", "indices"))
+        torch.cuda.synchronize()
+        e_ms = statistics.mean(a.elapsed_time(b) for a, b in ev2)
+        e_t = torch.tensor([e_ms], dtype=torch.float64, device=dev)
+        if world > 1:
+            dist.all_reduce(e_t, op=dist.ReduceOp.MAX)
+        e_ms = float(e_t.item())
+        e2e = {"value": H * world / (e_ms * 1e-3), "unit": "heads/s",
+               "h2d_bytes_per_step": sum(x.numel() * x.element_size() for x in (Qh, Kh, Vh)),
+               "d2h_bytes_per_step": d2h, "ms_per_step": e_ms}
+
+    if world > 1:
+        dist.barrier()
+    if rank != 0:
+        if world > 1:
+            dist.destroy_process_group()
+        return 0
+
+    ldn = (n + 31) // 32 * 32
+    passes = max((t + wl.topk * wl.refit_every - 1) // (wl.topk * wl.refit_every) for t in wl.budgets)
+    peaks = load_peaks()
+    rf = roofline(stages, args.steps, stage_models(wl, n, T, d, H, ldn, passes), peaks, clk,
+                  committed_traffic())
+    value = H * world / (ms * 1e-3)
+    per_step_stage = {k: round(v["ms"] / args.steps, 4) for k, v in stages.items() if v["launches"]}
+    cfg = {"workload": wl.name, "heads_per_gpu": H, "n": n, "T": T, "d": d,
+           "budgets": wl.budgets if H <= 8 else f"{sum(wl.budgets)} total, min {min(wl.budgets)} max {max(wl.budgets)}",
+           "topk": wl.topk, "refit_every": wl.refit_every, "phi_storage": "fp32",
+           "l2": "256 MiB buffer written between timed steps",
+           "stage_ms_per_step": per_step_stage, "device_status": worst}
+    if args.workload == "qwen3_4b_layer":
+        cfg["s_per_model_extrapolated_x36_layers"] = LAYERS_QWEN3_4B * ms * 1e-3
+    if args.workload == "qwen3_4b_model":
+        cfg["s_per_model"] = ms * 1e-3
+    line = {
+        "metric": METRIC, "value": value, "unit": "heads/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16" if Q.dtype == torch.bfloat16 else "fp32",
+        "data": "synthetic: seeded structured heads shaped like the pages' workloads (no datasets or weights)",
+        "config": cfg, "roofline": rf, "gpu_launches": launches, "clocks": clk,
+    }
+    if e2e is not None:
+        line["e2e"] = e2e
+    if world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(wl, heads=1)
+    print(json.dumps(line))
+    if world > 1:
+        dist.destroy_process_group()
+    del first
+    return 0
+
+
+def main():
+    args = parse_args()
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        return run_reference(args, rank, world)
+    return run_ours(args, rank, world, local_rank)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

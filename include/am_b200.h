@@ -1,0 +1,170 @@
+/*
+ * am_b200.h — C ABI of the B200 (sm_100a) Attention-Matching KV compaction
+ * library (AM-OMP).
+ *
+ * The operation ("Fast KV Compaction via Attention Matching"):
+ *   zhichai.net deep dive §1.3-§1.6 — attention mass, the per-token scalar
+ *     bias β, the mass-feature matrix Φ_ij = exp(q_i·k_j), target mass
+ *     m = Φ·1, greedy OMP key selection with an NNLS refit after each pick,
+ *     and β = log w;
+ *   xinfinite.net article §2 (steps 2 and 3, Fig. 1 and Fig. 2) — NNLS bias
+ *     fit (projected gradient on the GPU in the authors' version), value fit
+ *     by ordinary least squares; §3 and Table 1 — top-k batched selection
+ *     with lazy refit ("OMP-fast");
+ *   zhichai.net/en summary, "The Three-Step Closed-Form Pipeline" and
+ *     "Engineering Practicality" (varlen per-head packing).
+ *
+ * For every head h independently, with s_ij = (q_i·k_j)·scale + b_j:
+ *   Φ_ij = exp(s_ij − c_h),  m_i = Σ_j Φ_ij,
+ *   S  = t_h keys chosen greedily: each round appends the kk = min(k, t−|S|)
+ *        unselected keys with the largest c_j = Σ_i r_i Φ_ij (ties → lowest
+ *        index); on every R-th round and the last, w = NNLS(Φ_S, m) and
+ *        r = m − Φ_S w,
+ *   β_l = b_{S_l} + log max(w_l, w_floor_rel·max w),
+ *   Y_i = Σ_j Φ_ij V_j / m_i,  A_il = softmax_l(Q C_kᵀ·scale + β)_i,
+ *   C_v = (AᵀA + λI)⁻¹ AᵀY with λ = ridge·tr(AᵀA)/t_h.
+ *
+ * Conventions shared by every entry point
+ *   - All tensor pointers are DEVICE pointers unless marked "host".
+ *   - The caller owns every buffer; nothing is allocated inside a call.
+ *   - Work is enqueued on `stream` (a cudaStream_t passed as void*; NULL is
+ *     the legacy default stream); the call returns before it finishes.
+ *   - Argument errors are returned synchronously and nothing is enqueued.
+ *     Device-side per-head conditions (NNLS iteration limit, a Cholesky
+ *     pivot that is not positive, non-finite features) are written to status
+ *     words inside the workspace; read them with am_get_status().
+ *   - No entry point calls exit(), throws, or falls back to the CPU.
+ */
+#ifndef AM_B200_H
+#define AM_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum am_status {
+  AM_OK = 0,
+  AM_ERR_INVALID_ARG = 1,     /* null pointer, bad size or option          */
+  AM_ERR_BUDGET = 2,          /* a budget outside [1, T]                   */
+  AM_ERR_WORKSPACE = 3,       /* workspace missing, misaligned or too small */
+  AM_ERR_NONFINITE = 4,       /* (device) a non-finite feature or solution  */
+  AM_ERR_CUDA = 5,            /* a CUDA runtime call failed                 */
+  AM_ERR_TIMEOUT = 6,         /* (device) a bounded wait ran out            */
+  AM_ERR_UNSUPPORTED = 7,     /* shape or dtype this build does not handle  */
+  AM_WARN_NOT_CONVERGED = 8,  /* (device) NNLS stopped at its iteration cap */
+  AM_ERR_NOT_SPD = 9          /* (device) value-fit matrix not positive definite */
+} am_status_t;
+
+typedef enum am_dtype { AM_BF16 = 0, AM_FP32 = 1 } am_dtype_t;
+
+/* Options.  Fill with am_default_opts() and override fields. */
+typedef struct am_opts {
+  int32_t in_dtype;        /* am_dtype_t of Q_ref, K, V and of the C_k output   */
+  int32_t topk;            /* k: keys appended per OMP round (1 = plain OMP)     */
+  int32_t refit_every;     /* R: rounds between NNLS refits (1 = every round)    */
+  int32_t nnls_max_iter;   /* active-set iteration cap per refit (0 = 3·t + 50)  */
+  float scale;             /* logit scale; <= 0 selects 1/sqrt(d)                */
+  float ridge;             /* λ = ridge·tr(AᵀA)/t (default 1e-6); must be >= 0   */
+  float w_floor_rel;       /* β floor: w >= w_floor_rel·max(w) (default 1e-12)   */
+  float reserved0;
+  /* Optional device inputs */
+  const float* shift;      /* [H] per-head shift c_h, or NULL: c_h = max_ij s_ij
+                              computed on the device                              */
+  const float* key_bias;   /* [H][T] prior per-key bias b (an already compacted
+                              block's β), or NULL for b = 0                       */
+  /* Optional device outputs (NULL = not written) */
+  int32_t* pick_order;     /* [Σt] keys in greedy pick order, packed like indices */
+  float* pick_corr;        /* [Σt] correlation c_j of each pick when it was made  */
+  float* shift_out;        /* [H] shift used                                     */
+  double* residual_out;    /* [H] ‖m − Φ_S w‖ / ‖m‖ after the last refit          */
+  float* w_out;            /* [Σt] NNLS weights, aligned with indices            */
+} am_opts_t;
+
+/* Fill *opts with defaults: bf16 inputs, k = 1, R = 1, scale = 1/sqrt(d),
+ * ridge = 1e-6, w_floor_rel = 1e-12, every optional pointer NULL. */
+am_status_t am_default_opts(am_opts_t* opts);
+
+/* Device workspace needed by am_compact_heads for this problem.
+ *   n, T, d          reference queries, keys per head, head dim (d in {64, 128}
+ *                    for bf16 inputs; any d in [1, 256] for fp32 inputs)
+ *   num_heads        H
+ *   budgets          host int32 [H], 1 <= t_h <= T
+ *   opts             as passed to am_compact_heads
+ *   bytes            host out
+ * The dominant term is H·T·round_up(n, 32)·4 bytes of stored features. */
+am_status_t am_workspace_size(int32_t n, int32_t T, int32_t d, int32_t num_heads,
+                              const int32_t* budgets, const am_opts_t* opts,
+                              size_t* bytes);
+
+/* Compact H independent heads.
+ *   Q_ref   [H][n][d], K [H][T][d], V [H][T][d], row-major, dtype opts->in_dtype
+ *   budgets host int32 [H]
+ *   out_offsets host int64 [H+1]: out_offsets[0] = 0,
+ *           out_offsets[h+1] = out_offsets[h] + budgets[h] (checked)
+ *   workspace   device, 256-byte aligned, >= am_workspace_size() bytes
+ *   Outputs, packed per head at out_offsets[h] (the varlen layout), rows in
+ *   ascending original key position:
+ *     C_k      [Σt][d]  dtype opts->in_dtype (exact copies of the chosen keys)
+ *     beta     [Σt]     fp32
+ *     C_v      [Σt][d]  fp32
+ *     indices  [Σt]     int32, position of each kept key within its head
+ *   stream  cudaStream_t as void*
+ * Inputs must not alias outputs or the workspace.  The workspace must not be
+ * shared by two calls in flight at once. */
+am_status_t am_compact_heads(const void* Q_ref, const void* K, const void* V,
+                             int32_t n, int32_t T, int32_t d, int32_t num_heads,
+                             const int32_t* budgets, const am_opts_t* opts,
+                             void* workspace, size_t workspace_bytes,
+                             const int64_t* out_offsets,
+                             void* C_k, float* beta, float* C_v, int32_t* indices,
+                             void* stream);
+
+/* Synchronise `stream`, then copy the per-head device status words of the last
+ * call that used `workspace` into host per_head[H] (may be NULL) and return the
+ * most severe one (AM_OK if all heads succeeded). */
+am_status_t am_get_status(const void* workspace, int32_t num_heads,
+                          int32_t* per_head, void* stream);
+
+/* Stage timing.  While enabled, every kernel launch made by
+ * am_compact_heads is bracketed by CUDA events recorded on the call's stream
+ * (event creation is the only host-side cost; no device memory is used).
+ * am_profile_collect() waits for the recorded events, adds up the device time
+ * and the launch count per stage into ms[AM_STAGE_COUNT] and
+ * launches[AM_STAGE_COUNT] (host arrays, either may be NULL), and clears the
+ * record.  Process-wide; not meant for concurrent calls from several threads. */
+typedef enum am_stage {
+  AM_STAGE_SHIFT = 0,    /* c_h = max logit                         */
+  AM_STAGE_PHI = 1,      /* Φᵀ = exp(s − c_h)                        */
+  AM_STAGE_TARGET = 2,   /* Y = ΦV/m and m                           */
+  AM_STAGE_INIT = 3,     /* ‖m‖², selection flags                    */
+  AM_STAGE_CORR = 4,     /* c = Φᵀ r                                 */
+  AM_STAGE_SELECT = 5,   /* top-k·R unselected keys                  */
+  AM_STAGE_GRAM = 6,     /* Φ_SᵀΦ_S, Φ_Sᵀm updates                   */
+  AM_STAGE_NNLS = 7,     /* active-set NNLS refit                    */
+  AM_STAGE_RESID = 8,    /* r = m − Φ_S w                            */
+  AM_STAGE_FINALIZE = 9, /* sort, β, C_k, indices                    */
+  AM_STAGE_DESIGN = 10,  /* A = rownorm(Φ_S diag w)                  */
+  AM_STAGE_NORMAL = 11,  /* AᵀA, AᵀY                                 */
+  AM_STAGE_SOLVE = 12,   /* ridge Cholesky, C_v                      */
+  AM_STAGE_COUNT = 13
+} am_stage_t;
+
+am_status_t am_profile_enable(int32_t on);
+am_status_t am_profile_collect(double* ms, int64_t* launches);
+
+/* Total number of kernels this library has launched in the process. */
+int64_t am_kernel_launches(void);
+
+/* Static description of a status code. */
+const char* am_status_string(am_status_t status);
+
+/* Library version, major·10000 + minor·100 + patch. */
+int32_t am_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* AM_B200_H */

@@ -1,0 +1,115 @@
+"""GPU-vs-oracle acceptance checks shared by the GPU tests.
+
+Tolerances (float work; the index decisions are compared by a teacher-forced
+replay because near-ties may legitimately go either way):
+
+* picks: the oracle replays the GPU's pick order; each GPU pick must be one
+  of the oracle's own top-kk for that round, or have a correlation within
+  1e-4·|c_max| of the oracle's kk-th best;
+* index sets: identical whenever every round of the oracle's own run
+  separates its kk-th and (kk+1)-th correlations by more than 1e-4·|c_max|;
+* mass residual ‖m − Φ_S w‖/‖m‖ (both evaluated in float64 by the harness):
+  within 1e-3 of the oracle's;
+* β: within 1e-3 absolute where the oracle's w >= 1e-6·max(w); elsewhere both
+  sides' β − b_S at most log(1e-6·max w) + 1e-3; compared against the
+  oracle re-run on the GPU's own picks when the index sets differ;
+* reconstructed output softmax(Q C_kᵀ/√d + β) C_v, in float64: relative
+  Frobenius distance to the oracle's at most 2e-3.
+"""
+import math
+
+import numpy as np
+
+from oracle import am_oracle as O
+
+GAP_TOL = 1e-4
+RES_TOL = 1e-3
+BETA_TOL = 1e-3
+OUT_TOL = 2e-3
+W_CMP_REL = 1e-6
+
+
+def split_head(out, h):
+    """Slice head h of the packed GPU outputs to float64 numpy arrays."""
+    a, b = int(out["cu_t"][h]), int(out["cu_t"][h + 1])
+    g = {k: out[k][a:b].detach().cpu() for k in ("C_k", "beta", "C_v", "indices")}
+    res = {
+        "indices": g["indices"].numpy().astype(np.int64),
+        "C_k": g["C_k"].double().numpy(),
+        "beta": g["beta"].double().numpy(),
+        "C_v": g["C_v"].double().numpy(),
+    }
+    if "pick_order" in out:
+        res["pick_order"] = out["pick_order"][a:b].cpu().numpy().astype(np.int64).tolist()
+        res["w"] = out["w"][a:b].cpu().double().numpy()
+        res["residual_dev"] = float(out["residual"][h].cpu())
+    return res
+
+
+def check_head(g, Q, K, V, t, topk, refit, shift, key_bias=None, oracle_res=None, label=""):
+    """Run every acceptance rule for one head; returns a dict of measurements."""
+    if oracle_res is None:
+        oracle_res = O.compact_head(Q, K, V, t, topk, refit, shift=shift, key_bias=key_bias)
+    o = oracle_res
+    rep = {"label": label}
+    # the GPU keeps ascending, distinct key positions
+    idx = g["indices"]
+    assert len(idx) == t and np.all(np.diff(idx) > 0) and idx[0] >= 0 and idx[-1] < K.shape[0], label
+    np.testing.assert_array_equal(g["C_k"], K[idx], err_msg=label)
+
+    # teacher-forced replay of the GPU's pick order
+    forced = O.compact_head(Q, K, V, t, topk, refit, shift=shift, key_bias=key_bias,
+                            forced_picks=g["pick_order"])
+    worst_slack = 0.0
+    for rec in forced["rounds"]:
+        scale = max(abs(rec["c_max"]), 1e-300)
+        for j in rec["picks"]:
+            if j in rec["own"]:
+                continue
+            slack = (rec["c_kth"] - rec["c"][j]) / scale
+            worst_slack = max(worst_slack, slack)
+            assert slack <= GAP_TOL, f"{label}: pick {j} in round {rec['round']} trails by {slack:.3g}"
+    rep["pick_slack"] = worst_slack
+
+    gaps = [(r["c_kth"] - r["c_next"]) / max(abs(r["c_max"]), 1e-300)
+            for r in o["rounds"] if r["c_next"] is not None]
+    rep["min_gap"] = min(gaps) if gaps else math.inf
+    same = np.array_equal(idx, o["indices"])
+    rep["same_set"] = bool(same)
+    if rep["min_gap"] > GAP_TOL:
+        assert same, f"{label}: index sets differ although every gap > {GAP_TOL}"
+
+    Phi, m, _ = O.mass_features(Q, K, shift, key_bias=key_bias)
+    # the GPU's weights, aligned with its ascending indices
+    w_gpu = np.exp(g["beta"] - (0.0 if key_bias is None else np.asarray(key_bias)[idx]))
+    res_gpu = O.mass_residual(Phi, m, idx, w_gpu)
+    rep["res_gpu"], rep["res_oracle"] = res_gpu, o["residual"]
+    assert abs(res_gpu - o["residual"]) <= RES_TOL, f"{label}: residual {res_gpu} vs {o['residual']}"
+
+    ref = o if same else forced
+    ref_beta = ref["beta"] if same else ref["beta"]
+    ref_idx = ref["indices"]
+    assert np.array_equal(ref_idx, idx)
+    wmax = ref["w"].max()
+    big = ref["w"] >= W_CMP_REL * wmax
+    prior = np.zeros(t) if key_bias is None else np.asarray(key_bias, np.float64)[idx]
+    dbeta = np.abs(g["beta"] - ref_beta)
+    rep["beta_maxdiff"] = float(dbeta[big].max()) if big.any() else 0.0
+    assert rep["beta_maxdiff"] <= BETA_TOL, f"{label}: beta differs by {rep['beta_maxdiff']}"
+    if (~big).any():
+        lim = math.log(W_CMP_REL * wmax) + BETA_TOL
+        assert np.all(g["beta"][~big] - prior[~big] <= lim), f"{label}: small-weight beta above floor rule"
+
+    O_gpu = O.reconstructed_output(Q, g["C_k"], g["beta"], g["C_v"])
+    O_ref = O.reconstructed_output(Q, o["C_k"], o["beta"], o["C_v"])
+    rel = np.linalg.norm(O_gpu - O_ref) / np.linalg.norm(O_ref)
+    rep["out_rel"] = float(rel)
+    assert rel <= OUT_TOL, f"{label}: output relative error {rel}"
+    rep["fit_err_gpu"] = float(np.linalg.norm(O_gpu - o["Y"]) / np.linalg.norm(o["Y"]))
+    rep["fit_err_oracle"] = float(np.linalg.norm(O_ref - o["Y"]) / np.linalg.norm(o["Y"]))
+    return rep
+
+
+def shift_for(Q, K, key_bias=None):
+    """The shared per-head shift: max logit in float64, rounded to fp32."""
+    return float(np.float32(O.max_logit(Q, K, key_bias=key_bias)))

@@ -1,0 +1,87 @@
+"""The C-ABI library loads and exports every symbol include/am_b200.h
+declares; host-side argument errors come back synchronously (no GPU needed:
+each of these returns before the first CUDA call)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import attention_matching_b200 as am
+
+HDR = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include", "am_b200.h")
+
+
+def declared_functions():
+    src = open(HDR).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(am_[a-z_]+)\s*\(", src)))
+
+
+def test_library_exports_every_declared_symbol():
+    names = declared_functions()
+    assert "am_compact_heads" in names and len(names) >= 6
+    L = am.lib()
+    for n in names:
+        assert hasattr(L, n), n
+
+
+def test_opts_struct_layout_matches_header():
+    # 8 four-byte fields then 7 pointers
+    assert ctypes.sizeof(am.AmOpts) == 8 * 4 + 7 * 8
+
+
+def test_defaults_and_status_strings():
+    o = am.make_opts()
+    assert (o.in_dtype, o.topk, o.refit_every) == (am.BF16, 1, 1)
+    assert abs(o.ridge - 1e-6) < 1e-12 and abs(o.w_floor_rel - 1e-12) < 1e-18
+    L = am.lib()
+    for code in range(10):
+        assert L.am_status_string(code)
+    assert L.am_version() >= 100
+
+
+def test_workspace_size_scales_with_features():
+    o = am.make_opts(am.BF16, 4, 2)
+    a = am.workspace_size(8192, 8192, 128, [164] * 8, o)
+    assert a >= 8 * 8192 * 8192 * 4
+    assert am.workspace_size(1000, 1100, 128, [13, 22, 8], o) < a
+
+
+@pytest.mark.parametrize("bad", [
+    dict(budgets=[0]), dict(budgets=[301]), dict(topk=0), dict(refit_every=0),
+    dict(topk=16, refit_every=8), dict(d=300), dict(ridge=-1.0), dict(w_floor_rel=0.0),
+])
+def test_workspace_size_rejects(bad):
+    args = dict(n=512, T=300, d=64, budgets=[16], topk=1, refit_every=1, ridge=1e-6, w_floor_rel=1e-12)
+    args.update(bad)
+    o = am.make_opts(am.FP32, args["topk"], args["refit_every"], ridge=args["ridge"],
+                     w_floor_rel=args["w_floor_rel"])
+    with pytest.raises(am.AmError):
+        am.workspace_size(args["n"], args["T"], args["d"], args["budgets"], o)
+
+
+def _call(**over):
+    L = am.lib()
+    o = am.make_opts(am.FP32)
+    H, n, T, d = 1, 64, 32, 16
+    budgets = (ctypes.c_int32 * H)(4)
+    offs = (ctypes.c_int64 * (H + 1))(0, 4)
+    args = dict(Q=1 << 20, K=1 << 21, V=1 << 22, n=n, T=T, d=d, H=H, budgets=budgets, opts=ctypes.byref(o),
+                ws=None, ws_bytes=0, offs=offs, Ck=1 << 23, beta=1 << 24, Cv=1 << 25, idx=1 << 26)
+    args.update(over)
+    return L.am_compact_heads(args["Q"], args["K"], args["V"], args["n"], args["T"], args["d"], args["H"],
+                              args["budgets"], args["opts"], args["ws"], args["ws_bytes"], args["offs"],
+                              args["Ck"], args["beta"], args["Cv"], args["idx"], None)
+
+
+def test_compact_heads_argument_errors_are_synchronous():
+    assert _call(Q=None) == 1                       # null input
+    assert _call(n=0) == 1                          # bad size
+    bad_budget = (ctypes.c_int32 * 1)(33)
+    assert _call(budgets=bad_budget) == 2           # budget > T
+    bad_offs = (ctypes.c_int64 * 2)(0, 5)
+    assert _call(offs=bad_offs) == 1                # offsets disagree with budgets
+    assert _call(ws=None) == 3                      # no workspace
+    assert _call(ws=4096 + 8, ws_bytes=1 << 30) == 3  # misaligned workspace
+    assert _call(ws=4096, ws_bytes=16) == 3          # too small

@@ -1,0 +1,119 @@
+"""GPU parity: the CUDA path, called through the C ABI, against the float64
+oracle on the same seeded inputs (rules in tests/parity.py)."""
+import numpy as np
+import pytest
+import torch
+
+from attention_matching_b200 import workloads as W
+from oracle import am_oracle as O
+from tests.parity import check_head, shift_for, split_head
+
+pytestmark = pytest.mark.gpu
+
+needs_cuda = pytest.mark.skipif(not torch.cuda.is_available(), reason="needs a CUDA device")
+
+
+def _stack(heads, attr):
+    return torch.stack([getattr(h, attr) for h in heads]).contiguous().cuda()
+
+
+def run_gpu(heads, budgets, topk, refit, shifts=None, key_bias=None, **kw):
+    import attention_matching_b200 as am
+    Q, K, V = _stack(heads, "Q"), _stack(heads, "K"), _stack(heads, "V")
+    sh = None if shifts is None else torch.tensor(shifts, dtype=torch.float32).cuda()
+    kb = None if key_bias is None else torch.tensor(np.stack(key_bias), dtype=torch.float32).cuda()
+    return am.compact_heads(Q, K, V, budgets, topk=topk, refit_every=refit, shift=sh, key_bias=kb,
+                            trace=True, **kw)
+
+
+def check_all(heads, budgets, topk, refit, key_bias=None, sample=None, label=""):
+    shifts = [shift_for(*h.f64()[:2], key_bias=None if key_bias is None else key_bias[i])
+              for i, h in enumerate(heads)]
+    out = run_gpu(heads, budgets, topk, refit, shifts, key_bias)
+    assert all(s in (0, 8) for s in out["status"]), out["status"]
+    reps = []
+    for h in (range(len(heads)) if sample is None else sample):
+        Q, K, V = heads[h].f64()
+        kb = None if key_bias is None else np.asarray(key_bias[h], np.float64)
+        g = split_head(out, h)
+        reps.append(check_head(g, Q, K, V, budgets[h], topk, refit, shifts[h], kb,
+                               label=f"{label} head {h}"))
+    return out, reps
+
+
+@needs_cuda
+def test_single_head_fp32_plain_omp():
+    wl = W.single_head_fp32()
+    _, reps = check_all(wl.heads, wl.budgets, 1, 1, label="fp32 T256 n512 d64 t16")
+    assert reps[0]["same_set"]
+
+
+@needs_cuda
+def test_structured_bf16_ragged_nonuniform():
+    # n, T not multiples of the 64-wide tiles; budgets differ per head
+    heads = [W.structured_head(300 + h, n=1000, T=1100) for h in range(3)]
+    check_all(heads, [13, 22, 8], 4, 2, label="bf16 ragged")
+
+
+@needs_cuda
+def test_structured_bf16_d64():
+    heads = [W.structured_head(310 + h, n=640, T=700, d=64, rank=16) for h in range(2)]
+    check_all(heads, [20, 33], 4, 2, label="bf16 d64")
+
+
+@needs_cuda
+def test_prior_key_bias():
+    heads = [W.structured_head(320 + h, n=512, T=600) for h in range(2)]
+    rng = np.random.default_rng(321)
+    kb = [np.float32(np.log(rng.uniform(1.0, 3.0, size=600))) for _ in heads]
+    check_all(heads, [16, 24], 4, 2, key_bias=kb, label="prior bias")
+
+
+@needs_cuda
+def test_budget_edges():
+    # t = 1, t = T (exact: w = 1, zero residual), tiny T below one tile
+    heads = [W.iid_head(330, n=96, T=40, d=32), W.iid_head(331, n=96, T=40, d=32)]
+    out, reps = check_all(heads, [1, 40], 1, 1, label="edges")
+    g = split_head(out, 1)
+    assert g["indices"].tolist() == list(range(40))
+    np.testing.assert_allclose(np.exp(g["beta"]), np.ones(40), rtol=2e-4)
+
+
+@needs_cuda
+def test_plain_vs_batched_reading():
+    """(k, R) = (4, 2) and (8, 1) pick the same keys on the GPU too."""
+    heads = [W.structured_head(340, n=512, T=512)]
+    Q, K, _ = heads[0].f64()
+    sh = [shift_for(Q, K)]
+    a = run_gpu(heads, [30], 4, 2, sh)
+    b = run_gpu(heads, [30], 8, 1, sh)
+    assert torch.equal(a["indices"], b["indices"])
+
+
+@needs_cuda
+def test_deterministic_bitwise():
+    heads = [W.structured_head(350 + h, n=768, T=800) for h in range(2)]
+    a = run_gpu(heads, [17, 9], 4, 2)
+    b = run_gpu(heads, [17, 9], 4, 2)
+    for k in ("C_k", "beta", "C_v", "indices", "pick_order", "shift"):
+        assert torch.equal(a[k], b[k]), k
+
+
+@needs_cuda
+def test_device_shift_matches_max_logit():
+    heads = [W.structured_head(360 + h, n=300, T=260) for h in range(2)]
+    out = run_gpu(heads, [8, 8], 4, 2)
+    for h, hd in enumerate(heads):
+        Q, K, _ = hd.f64()
+        assert abs(float(out["shift"][h]) - O.max_logit(Q, K)) <= 1e-5 * max(1.0, abs(O.max_logit(Q, K)))
+
+
+@needs_cuda
+def test_qwen3_layer_full_size_sampled():
+    """The bench workload (8 heads, T = n = 8192, d = 128, t = 164, k = 4,
+    R = 2) run whole on the GPU; two heads checked against the oracle."""
+    wl = W.qwen3_4b_layer()
+    _, reps = check_all(wl.heads, wl.budgets, wl.topk, wl.refit_every, sample=[0, 5],
+                        label="qwen3 layer")
+    for r in reps:
+        assert r["out_rel"] <= 2e-3
