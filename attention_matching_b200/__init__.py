@@ -37,6 +37,12 @@ class AmError(RuntimeError):
         super().__init__(f"{where}: {STATUS.get(code, code)}")
 
 
+class AmWorkspaceView(ctypes.Structure):
+    """Mirror of am_workspace_view_t."""
+    _fields_ = [("phiT", ctypes.c_size_t), ("mass", ctypes.c_size_t), ("target", ctypes.c_size_t),
+                ("shift", ctypes.c_size_t), ("ldn", ctypes.c_int32), ("reserved", ctypes.c_int32)]
+
+
 class AmOpts(ctypes.Structure):
     """Mirror of am_opts_t (include/am_b200.h); field order and types match."""
     _fields_ = [
@@ -87,6 +93,9 @@ def lib() -> ctypes.CDLL:
         L.am_status_string.restype = ctypes.c_char_p
         L.am_version.argtypes = []
         L.am_version.restype = c_int
+        L.am_workspace_view.argtypes = [c_int, c_int, c_int, c_int, P_i32, ctypes.POINTER(AmOpts),
+                                        ctypes.POINTER(AmWorkspaceView)]
+        L.am_workspace_view.restype = c_int
         L.am_profile_enable.argtypes = [c_int]
         L.am_profile_enable.restype = c_int
         L.am_profile_collect.argtypes = [ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_int64)]
@@ -119,6 +128,33 @@ def workspace_size(n: int, T: int, d: int, budgets: Sequence[int], opts: AmOpts)
     if rc:
         raise AmError(rc, "am_workspace_size")
     return int(out.value)
+
+
+def features(out: Dict, n: int, T: int, d: int, budgets: Sequence[int], topk: int = 1,
+             refit_every: int = 1, dtype: int = BF16) -> Dict:
+    """Views of the intermediate features a finished call left in its
+    workspace: phiT [H, T, ldn] fp32, mass [H, ldn] fp64, target [H, n, d]
+    fp32, shift [H] fp32 (torch tensors sharing the workspace memory)."""
+    import torch
+    H = len(budgets)
+    opts = make_opts(dtype, topk, refit_every)
+    v = AmWorkspaceView()
+    rc = lib().am_workspace_view(n, T, d, H, _i32_array(budgets), ctypes.byref(opts), ctypes.byref(v))
+    if rc:
+        raise AmError(rc, "am_workspace_view")
+    ws = out["workspace"]
+
+    def view(off, count, dt):
+        nbytes = count * torch.empty((), dtype=dt).element_size()
+        return ws[off:off + nbytes].view(dt)
+
+    return {
+        "phiT": view(v.phiT, H * T * v.ldn, torch.float32).view(H, T, v.ldn),
+        "mass": view(v.mass, H * v.ldn, torch.float64).view(H, v.ldn),
+        "target": view(v.target, H * n * d, torch.float32).view(H, n, d),
+        "shift": view(v.shift, H, torch.float32),
+        "ldn": v.ldn,
+    }
 
 
 def _ptr(t) -> Optional[int]:

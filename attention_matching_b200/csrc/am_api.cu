@@ -208,6 +208,22 @@ am_status_t am_workspace_size(int32_t n, int32_t T, int32_t d, int32_t num_heads
   return AM_OK;
 }
 
+am_status_t am_workspace_view(int32_t n, int32_t T, int32_t d, int32_t num_heads, const int32_t* budgets,
+                              const am_opts_t* opts, am_workspace_view_t* view) {
+  if (!view) return AM_ERR_INVALID_ARG;
+  Tables tb;
+  am_status_t st = check_shape(n, T, d, num_heads, budgets, opts, &tb);
+  if (st != AM_OK) return st;
+  const Layout L = plan(n, T, d, num_heads, tb.sum_t, tb.sum_t2);
+  view->phiT = L.phiT;
+  view->mass = L.m;
+  view->target = L.Y;
+  view->shift = L.shift;
+  view->ldn = round_up(n, 32);
+  view->reserved = 0;
+  return AM_OK;
+}
+
 am_status_t am_compact_heads(const void* Q, const void* K, const void* V, int32_t n, int32_t T,
                              int32_t d, int32_t H, const int32_t* budgets, const am_opts_t* opts,
                              void* workspace, size_t workspace_bytes, const int64_t* out_offsets,

@@ -122,6 +122,26 @@ am_status_t am_compact_heads(const void* Q_ref, const void* K, const void* V,
                              void* C_k, float* beta, float* C_v, int32_t* indices,
                              void* stream);
 
+/* Where am_compact_heads leaves its intermediate features inside the
+ * caller's workspace (byte offsets from the workspace base), valid once the
+ * call has completed and until the workspace is reused:
+ *   phiT    fp32 [H][T][ldn]  Φᵀ_ji = exp(s_ij − c_h), key-major, rows padded
+ *                             with zeros from n to ldn
+ *   mass    fp64 [H][ldn]     m_i = Σ_j Φ_ij (exact sum of the stored fp32 Φ)
+ *   target  fp32 [H][n][d]    Y_i = Σ_j Φ_ij V_j / m_i
+ *   shift   fp32 [H]          c_h used
+ *   ldn     n rounded up to a multiple of 32
+ * Same argument rules as am_workspace_size. */
+typedef struct am_workspace_view {
+  size_t phiT, mass, target, shift;
+  int32_t ldn;
+  int32_t reserved;
+} am_workspace_view_t;
+
+am_status_t am_workspace_view(int32_t n, int32_t T, int32_t d, int32_t num_heads,
+                              const int32_t* budgets, const am_opts_t* opts,
+                              am_workspace_view_t* view);
+
 /* Synchronise `stream`, then copy the per-head device status words of the last
  * call that used `workspace` into host per_head[H] (may be NULL) and return the
  * most severe one (AM_OK if all heads succeeded). */

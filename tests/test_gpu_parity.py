@@ -117,3 +117,32 @@ def test_qwen3_layer_full_size_sampled():
                         label="qwen3 layer")
     for r in reps:
         assert r["out_rel"] <= 2e-3
+
+
+@needs_cuda
+@pytest.mark.parametrize("dtype,d,n,T", [("bf16", 128, 300, 333), ("bf16", 64, 200, 130), ("fp32", 64, 150, 100)])
+def test_features_elementwise(dtype, d, n, T):
+    """Φᵀ, m, Y and the device shift of the feature pass, element by element
+    against the oracle (tensor-core pass for bf16, CUDA-core pass for fp32)."""
+    import attention_matching_b200 as am
+    if dtype == "bf16":
+        heads = [W.structured_head(370 + h, n=n, T=T, d=d, rank=min(32, d // 2)) for h in range(2)]
+    else:
+        heads = [W.iid_head(380 + h, n=n, T=T, d=d) for h in range(2)]
+    out = run_gpu(heads, [5, 7], 4, 2)
+    f = am.features(out, n, T, d, [5, 7], 4, 2, am.BF16 if dtype == "bf16" else am.FP32)
+    for h, hd in enumerate(heads):
+        Q, K, V = hd.f64()
+        c = float(f["shift"][h])
+        assert abs(c - O.max_logit(Q, K)) <= 1e-5 * max(1.0, abs(c))
+        Phi, m, _ = O.mass_features(Q, K, shift=c)
+        P = f["phiT"][h, :, :n].double().cpu().numpy().T
+        assert torch.all(f["phiT"][h, :, n:] == 0)
+        rel = np.abs(P - Phi) / np.maximum(Phi, 1e-30)
+        assert rel.max() <= 3e-5, rel.max()
+        mg = f["mass"][h, :n].cpu().numpy()
+        np.testing.assert_allclose(mg, P.sum(axis=1), rtol=1e-12)      # exact sum of the stored values
+        np.testing.assert_allclose(mg, m, rtol=3e-5)
+        Y = O.target_outputs(Phi, V, m)
+        Yg = f["target"][h].double().cpu().numpy()
+        assert np.abs(Yg - Y).max() <= 1e-4 * np.abs(Y).max()
