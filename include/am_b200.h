@@ -142,6 +142,40 @@ am_status_t am_workspace_view(int32_t n, int32_t T, int32_t d, int32_t num_heads
                               const int32_t* budgets, const am_opts_t* opts,
                               am_workspace_view_t* view);
 
+/* Size of the fixed device scratch area behind am_compact_heads_noalloc. */
+#define AM_NOALLOC_SCRATCH_BYTES ((size_t)16 << 20)
+
+/* am_compact_heads without any device allocation (the paper has no
+ * counterpart; this is a library convenience).
+ *
+ * For callers that cannot call cudaMalloc: code running inside a runtime
+ * that owns every device allocation through its own pool and forbids
+ * others, code on a latency-critical path where an allocation would
+ * synchronise the device, or plugins handed only input and output buffers.
+ * The scratch memory this call needs lives in one file-scope device array of
+ * AM_NOALLOC_SCRATCH_BYTES (16 MiB) inside this library; every GPU that loads
+ * the library keeps that array until the process exits.
+ *
+ *   Arguments as for am_compact_heads, without workspace and size.
+ *   status_out  optional device int32 [H]: per-head status codes as
+ *               am_get_status reports them (AM_OK, AM_WARN_NOT_CONVERGED, ...),
+ *               written on `stream` when the call completes; NULL to skip.
+ * Returns AM_ERR_WORKSPACE, before touching the GPU, when the problem's
+ * workspace (am_workspace_size) exceeds AM_NOALLOC_SCRATCH_BYTES.
+ *
+ * The first call on a device looks up the array's device address with the
+ * CUDA runtime; make that first call outside any stream capture.  All calls
+ * share the one array and leave their contents in it: calls whose work
+ * overlaps on the GPU (on different streams, or from different threads)
+ * race on it and must be serialised by the caller.  The call allocates
+ * nothing: no cudaMalloc, no cudaFree, no allocating library routine. */
+am_status_t am_compact_heads_noalloc(const void* Q_ref, const void* K, const void* V,
+                                     int32_t n, int32_t T, int32_t d, int32_t num_heads,
+                                     const int32_t* budgets, const am_opts_t* opts,
+                                     const int64_t* out_offsets,
+                                     void* C_k, float* beta, float* C_v, int32_t* indices,
+                                     int32_t* status_out, void* stream);
+
 /* Synchronise `stream`, then copy the per-head device status words of the last
  * call that used `workspace` into host per_head[H] (may be NULL) and return the
  * most severe one (AM_OK if all heads succeeded). */
