@@ -40,20 +40,22 @@ LAYERS_QWEN3_4B = 36
 def parse_args():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="qwen3_4b_layer",
                     choices=["qwen3_4b_layer", "single_head_fp32", "qwen3_4b_model"])
+    ap.add_argument("--heads", type=int, default=None,
+                    help="heads per GPU for the layer workload (default 8); smaller for profiling")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     return ap.parse_args()
 
 
-def build_workload(name, rank):
+def build_workload(name, rank, heads=None):
     from attention_matching_b200 import workloads as W
     if name == "qwen3_4b_layer":
-        return W.qwen3_4b_layer(seed_base=2000 + 1000 * rank)
+        return W.qwen3_4b_layer(num_heads=heads or 8, seed_base=2000 + 1000 * rank)
     if name == "qwen3_4b_model":
         return W.qwen3_4b_model(seed_base=4000 + 1000 * rank)
     return W.single_head_fp32(seed=1000 + rank)
@@ -84,7 +86,7 @@ class ClockSampler:
         self.lines = []
 
     def start(self):
-        cmd = ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "200"]
+        cmd = ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "50"]
         if self.gpu_id is not None:
             cmd += ["-i", str(self.gpu_id)]
         try:
@@ -199,8 +201,8 @@ def roofline(stages, steps, models, peaks, clocks, traffic_info):
 
 
 def committed_traffic():
-    """DRAM bytes per launch from the committed ncu summary, valid only while
-    the kernel sources still hash to what was profiled."""
+    """DRAM bytes per launch from the committed ncu summary, used only while the
+    profiled kernel's source region still hashes to what was profiled."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
     try:
         with open(path) as f:
@@ -209,12 +211,12 @@ def committed_traffic():
         return {}
     out = {}
     for k, v in rec.items():
-        src = os.path.join(ROOT, v["source"])
         try:
-            h = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+            src = open(os.path.join(ROOT, v["source"])).read()
+            region = src[src.index(v["region_begin"]):src.index(v["region_end"])]
         except Exception:
             continue
-        if h == v["source_sha256_16"]:
+        if hashlib.sha256(region.encode()).hexdigest()[:16] == v["region_sha256_16"]:
             out[k] = v["dram_bytes_per_launch"]
     return out
 
@@ -256,7 +258,7 @@ def run_ours(args, rank, world, local_rank):
         import torch.distributed as dist
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=dev)
 
-    wl = build_workload(args.workload, rank)
+    wl = build_workload(args.workload, rank, args.heads)
     H = len(wl.heads)
     n, T, d = wl.heads[0].n, wl.heads[0].T, wl.heads[0].d
     Qh = torch.stack([h.Q for h in wl.heads]).contiguous()
