@@ -53,7 +53,7 @@ class AmOpts(ctypes.Structure):
         ("scale", ctypes.c_float),
         ("ridge", ctypes.c_float),
         ("w_floor_rel", ctypes.c_float),
-        ("reserved0", ctypes.c_float),
+        ("corr_dtype", ctypes.c_int32),
         ("shift", ctypes.c_void_p),
         ("key_bias", ctypes.c_void_p),
         ("pick_order", ctypes.c_void_p),
@@ -111,13 +111,15 @@ def _i32_array(vals: Sequence[int]):
 
 
 def make_opts(dtype: int = BF16, topk: int = 1, refit_every: int = 1, scale: float = 0.0,
-              ridge: float = 1e-6, w_floor_rel: float = 1e-12, nnls_max_iter: int = 0) -> AmOpts:
+              ridge: float = 1e-6, w_floor_rel: float = 1e-12, nnls_max_iter: int = 0,
+              corr_dtype: int = FP32) -> AmOpts:
     o = AmOpts()
     rc = lib().am_default_opts(ctypes.byref(o))
     if rc:
         raise AmError(rc, "am_default_opts")
     o.in_dtype, o.topk, o.refit_every, o.nnls_max_iter = dtype, topk, refit_every, nnls_max_iter
     o.scale, o.ridge, o.w_floor_rel = scale, ridge, w_floor_rel
+    o.corr_dtype = corr_dtype
     return o
 
 
@@ -164,7 +166,7 @@ def _ptr(t) -> Optional[int]:
 def compact_heads(Q, K, V, budgets: Sequence[int], topk: int = 1, refit_every: int = 1,
                   shift=None, key_bias=None, ridge: float = 1e-6, w_floor_rel: float = 1e-12,
                   scale: float = 0.0, nnls_max_iter: int = 0, workspace=None, trace: bool = False,
-                  stream=None, check: bool = True) -> Dict:
+                  stream=None, check: bool = True, corr_dtype: int = FP32) -> Dict:
     """Compact H heads on the GPU.
 
     Q [H, n, d], K [H, T, d], V [H, T, d]: contiguous tensors, bf16 or fp32,
@@ -194,7 +196,7 @@ def compact_heads(Q, K, V, budgets: Sequence[int], topk: int = 1, refit_every: i
             raise ValueError("inputs must be contiguous")
     dt = BF16 if Q.dtype == torch.bfloat16 else FP32
     dev = Q.device
-    opts = make_opts(dt, topk, refit_every, scale, ridge, w_floor_rel, nnls_max_iter)
+    opts = make_opts(dt, topk, refit_every, scale, ridge, w_floor_rel, nnls_max_iter, corr_dtype)
     if shift is not None:
         shift = shift.to(device=dev, dtype=torch.float32).contiguous()
         opts.shift = shift.data_ptr()

@@ -23,7 +23,7 @@ size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 struct Layout {
   // byte offsets from the workspace base
   size_t tables, status, shift, np, mm, rr_part;
-  size_t phiT, m, Y, r, corr, sel;
+  size_t phiT, phiT16, m, Y, r, corr, sel;
   size_t picks, pick_corr, plist, sorted_slot;
   size_t bvec, w, w_eff;
   size_t G, L, AtA, A, AtY;
@@ -40,7 +40,7 @@ struct Tables {
   int64_t sum_t = 0, sum_t2 = 0;
 };
 
-Layout plan(int n, int T, int d, int H, int64_t sum_t, int64_t sum_t2) {
+Layout plan(int n, int T, int d, int H, int64_t sum_t, int64_t sum_t2, bool corr_bf16) {
   Layout L{};
   const size_t ldn = (size_t)round_up(n, 32);
   size_t o = 0;
@@ -53,6 +53,7 @@ Layout plan(int n, int T, int d, int H, int64_t sum_t, int64_t sum_t2) {
   L.mm = take((size_t)H * 8);
   L.rr_part = take((size_t)H * kRedBlocks * 8);
   L.phiT = take((size_t)H * T * ldn * 4);
+  L.phiT16 = take(corr_bf16 ? (size_t)H * T * ldn * 2 : 0);
   L.m = take((size_t)H * ldn * 8);
   L.r = take((size_t)H * ldn * 4);
   L.Y = take((size_t)H * n * d * 4);
@@ -86,6 +87,7 @@ am_status_t check_shape(int n, int T, int d, int H, const int32_t* budgets, cons
   if (!(opts->ridge >= 0.f) || !isfinite(opts->ridge)) return AM_ERR_INVALID_ARG;
   if (!(opts->w_floor_rel > 0.f) || !(opts->w_floor_rel < 1.f)) return AM_ERR_INVALID_ARG;
   if (!isfinite(opts->scale)) return AM_ERR_INVALID_ARG;
+  if (opts->corr_dtype != AM_FP32 && opts->corr_dtype != AM_BF16) return AM_ERR_INVALID_ARG;
   if ((int64_t)n * d > (1ll << 31) || (int64_t)T * round_up(n, 32) > (1ll << 40))
     return AM_ERR_UNSUPPORTED;
   const int kR = opts->topk * opts->refit_every;
@@ -114,8 +116,9 @@ am_status_t check_shape(int n, int T, int d, int H, const int32_t* budgets, cons
   return AM_OK;
 }
 
-Work bind(const Layout& L, char* base) {
+Work bind(const Layout& L, char* base, bool corr_bf16) {
   Work w{};
+  w.phiT16 = corr_bf16 ? reinterpret_cast<__nv_bfloat16*>(base + L.phiT16) : nullptr;
   w.status = reinterpret_cast<int32_t*>(base + L.status);
   w.shift = reinterpret_cast<float*>(base + L.shift);
   w.np = reinterpret_cast<int32_t*>(base + L.np);
@@ -171,6 +174,7 @@ Problem make_problem(int n, int T, int d, int H, const am_opts_t* o, const Table
   p.w_floor_rel = o->w_floor_rel;
   p.max_t = tb.max_t;
   p.has_bias = o->key_bias != nullptr;
+  p.corr_bf16 = o->corr_dtype == AM_BF16;
   return p;
 }
 
@@ -195,6 +199,7 @@ am_status_t am_default_opts(am_opts_t* opts) {
   opts->scale = 0.f;
   opts->ridge = 1e-6f;
   opts->w_floor_rel = 1e-12f;
+  opts->corr_dtype = AM_FP32;
   return AM_OK;
 }
 
@@ -204,7 +209,7 @@ am_status_t am_workspace_size(int32_t n, int32_t T, int32_t d, int32_t num_heads
   Tables tb;
   am_status_t st = check_shape(n, T, d, num_heads, budgets, opts, &tb);
   if (st != AM_OK) return st;
-  *bytes = plan(n, T, d, num_heads, tb.sum_t, tb.sum_t2).total;
+  *bytes = plan(n, T, d, num_heads, tb.sum_t, tb.sum_t2, opts->corr_dtype == AM_BF16).total;
   return AM_OK;
 }
 
@@ -214,7 +219,7 @@ am_status_t am_workspace_view(int32_t n, int32_t T, int32_t d, int32_t num_heads
   Tables tb;
   am_status_t st = check_shape(n, T, d, num_heads, budgets, opts, &tb);
   if (st != AM_OK) return st;
-  const Layout L = plan(n, T, d, num_heads, tb.sum_t, tb.sum_t2);
+  const Layout L = plan(n, T, d, num_heads, tb.sum_t, tb.sum_t2, opts->corr_dtype == AM_BF16);
   view->phiT = L.phiT;
   view->mass = L.m;
   view->target = L.Y;
@@ -235,12 +240,12 @@ am_status_t am_compact_heads(const void* Q, const void* K, const void* V, int32_
   for (int h = 0; h <= H; ++h)
     if (out_offsets[h] != tb.cu_t[h]) return AM_ERR_INVALID_ARG;
   if (!workspace || ((uintptr_t)workspace % kAlign) != 0) return AM_ERR_WORKSPACE;
-  const Layout L = plan(n, T, d, H, tb.sum_t, tb.sum_t2);
+  const Layout L = plan(n, T, d, H, tb.sum_t, tb.sum_t2, opts->corr_dtype == AM_BF16);
   if (workspace_bytes < L.total) return AM_ERR_WORKSPACE;
 
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   char* base = reinterpret_cast<char*>(workspace);
-  Work w = bind(L, base);
+  Work w = bind(L, base, opts->corr_dtype == AM_BF16);
   std::vector<unsigned char> host_tables;
   pack_tables(tb, H, &host_tables, &w, base + L.tables);
   const Problem p = make_problem(n, T, d, H, opts, tb);

@@ -27,6 +27,7 @@ struct Problem {
   float ridge, w_floor_rel;
   int max_t;          // max_h t_h
   int has_bias;
+  int corr_bf16;      // the correlation pass streams a bf16 copy of Φᵀ
 };
 
 // Device pointers into the caller's workspace (see plan_workspace()).
@@ -38,6 +39,7 @@ struct Work {
   int32_t* order;       // [H] heads sorted by pass count, descending
   float* shift;         // [H]
   float* phiT;          // [H][T][ldn] key-major features Φᵀ
+  __nv_bfloat16* phiT16; // [H][T][ldn] bf16 copy for the correlation pass (or null)
   double* m;            // [H][ldn] mass: fp64 sum of the stored fp32 features
   float* Y;             // [H][n][d]
   float* r;             // [H][ldn] residual (fp32 copy read by the correlation pass)

@@ -46,10 +46,22 @@ __global__ void k_init(Problem p, Work w) {
 }
 
 // ----------------------------------------------------------- correlation --
-// One warp per 4 key rows; 128-bit streaming loads of Φᵀ, r from L1.
+// One warp per 4 key rows; 128-bit streaming loads of Φᵀ (4 fp32 or 8 bf16
+// features per load), r from L1.
 constexpr int kCorrRowsPerWarp = 4;
 constexpr int kCorrWarps = 8;
 constexpr int kCorrRowsPerBlock = kCorrRowsPerWarp * kCorrWarps;
+
+__device__ __forceinline__ float dot8_bf16(uint4 x, float4 ra, float4 rb, float acc) {
+  const __nv_bfloat162* e = reinterpret_cast<const __nv_bfloat162*>(&x);
+  float2 f0 = __bfloat1622float2(e[0]), f1 = __bfloat1622float2(e[1]);
+  float2 f2 = __bfloat1622float2(e[2]), f3 = __bfloat1622float2(e[3]);
+  acc = fmaf(f0.x, ra.x, acc); acc = fmaf(f0.y, ra.y, acc);
+  acc = fmaf(f1.x, ra.z, acc); acc = fmaf(f1.y, ra.w, acc);
+  acc = fmaf(f2.x, rb.x, acc); acc = fmaf(f2.y, rb.y, acc);
+  acc = fmaf(f3.x, rb.z, acc); acc = fmaf(f3.y, rb.w, acc);
+  return acc;
+}
 
 __global__ void __launch_bounds__(256) k_corr(Problem p, Work w, int pass) {
   const int h = w.order[blockIdx.y];
@@ -59,38 +71,69 @@ __global__ void __launch_bounds__(256) k_corr(Problem p, Work w, int pass) {
   const int j0 = blockIdx.x * kCorrRowsPerBlock + warp * kCorrRowsPerWarp;
   if (j0 >= p.T) return;
   const float4* r4 = reinterpret_cast<const float4*>(w.r + (int64_t)h * p.ldn);
-  const float4* rows[kCorrRowsPerWarp];
-#pragma unroll
-  for (int q = 0; q < kCorrRowsPerWarp; ++q) {
-    int j = min(j0 + q, p.T - 1);
-    rows[q] = reinterpret_cast<const float4*>(w.phiT + ((int64_t)h * p.T + j) * p.ldn);
-  }
   float acc[kCorrRowsPerWarp] = {0.f, 0.f, 0.f, 0.f};
-  const int n4 = p.ldn >> 2;
-  int i = lane;
-  for (; i + 32 < n4; i += 64) {
-    float4 ra = __ldg(r4 + i), rb = __ldg(r4 + i + 32);
-    float4 xa[kCorrRowsPerWarp], xb[kCorrRowsPerWarp];
+  if (w.phiT16) {
+    const uint4* rows[kCorrRowsPerWarp];
 #pragma unroll
     for (int q = 0; q < kCorrRowsPerWarp; ++q) {
-      xa[q] = __ldcs(rows[q] + i);
-      xb[q] = __ldcs(rows[q] + i + 32);
+      const int j = min(j0 + q, p.T - 1);
+      rows[q] = reinterpret_cast<const uint4*>(w.phiT16 + ((int64_t)h * p.T + j) * p.ldn);
     }
+    const int n8 = p.ldn >> 3;
+    int i = lane;
+    for (; i + 32 < n8; i += 64) {
+      const float4 ra0 = __ldg(r4 + 2 * i), rb0 = __ldg(r4 + 2 * i + 1);
+      const float4 ra1 = __ldg(r4 + 2 * (i + 32)), rb1 = __ldg(r4 + 2 * (i + 32) + 1);
+      uint4 xa[kCorrRowsPerWarp], xb[kCorrRowsPerWarp];
 #pragma unroll
-    for (int q = 0; q < kCorrRowsPerWarp; ++q) {
-      acc[q] = fmaf(xa[q].x, ra.x, acc[q]); acc[q] = fmaf(xa[q].y, ra.y, acc[q]);
-      acc[q] = fmaf(xa[q].z, ra.z, acc[q]); acc[q] = fmaf(xa[q].w, ra.w, acc[q]);
-      acc[q] = fmaf(xb[q].x, rb.x, acc[q]); acc[q] = fmaf(xb[q].y, rb.y, acc[q]);
-      acc[q] = fmaf(xb[q].z, rb.z, acc[q]); acc[q] = fmaf(xb[q].w, rb.w, acc[q]);
+      for (int q = 0; q < kCorrRowsPerWarp; ++q) {
+        xa[q] = __ldcs(rows[q] + i);
+        xb[q] = __ldcs(rows[q] + i + 32);
+      }
+#pragma unroll
+      for (int q = 0; q < kCorrRowsPerWarp; ++q) {
+        acc[q] = dot8_bf16(xa[q], ra0, rb0, acc[q]);
+        acc[q] = dot8_bf16(xb[q], ra1, rb1, acc[q]);
+      }
     }
-  }
-  for (; i < n4; i += 32) {
-    float4 ra = __ldg(r4 + i);
+    for (; i < n8; i += 32) {
+      const float4 ra = __ldg(r4 + 2 * i), rb = __ldg(r4 + 2 * i + 1);
+#pragma unroll
+      for (int q = 0; q < kCorrRowsPerWarp; ++q) acc[q] = dot8_bf16(__ldcs(rows[q] + i), ra, rb, acc[q]);
+    }
+  } else {
+    const float4* rows[kCorrRowsPerWarp];
 #pragma unroll
     for (int q = 0; q < kCorrRowsPerWarp; ++q) {
-      float4 x = __ldcs(rows[q] + i);
-      acc[q] = fmaf(x.x, ra.x, acc[q]); acc[q] = fmaf(x.y, ra.y, acc[q]);
-      acc[q] = fmaf(x.z, ra.z, acc[q]); acc[q] = fmaf(x.w, ra.w, acc[q]);
+      const int j = min(j0 + q, p.T - 1);
+      rows[q] = reinterpret_cast<const float4*>(w.phiT + ((int64_t)h * p.T + j) * p.ldn);
+    }
+    const int n4 = p.ldn >> 2;
+    int i = lane;
+    for (; i + 32 < n4; i += 64) {
+      const float4 ra = __ldg(r4 + i), rb = __ldg(r4 + i + 32);
+      float4 xa[kCorrRowsPerWarp], xb[kCorrRowsPerWarp];
+#pragma unroll
+      for (int q = 0; q < kCorrRowsPerWarp; ++q) {
+        xa[q] = __ldcs(rows[q] + i);
+        xb[q] = __ldcs(rows[q] + i + 32);
+      }
+#pragma unroll
+      for (int q = 0; q < kCorrRowsPerWarp; ++q) {
+        acc[q] = fmaf(xa[q].x, ra.x, acc[q]); acc[q] = fmaf(xa[q].y, ra.y, acc[q]);
+        acc[q] = fmaf(xa[q].z, ra.z, acc[q]); acc[q] = fmaf(xa[q].w, ra.w, acc[q]);
+        acc[q] = fmaf(xb[q].x, rb.x, acc[q]); acc[q] = fmaf(xb[q].y, rb.y, acc[q]);
+        acc[q] = fmaf(xb[q].z, rb.z, acc[q]); acc[q] = fmaf(xb[q].w, rb.w, acc[q]);
+      }
+    }
+    for (; i < n4; i += 32) {
+      const float4 ra = __ldg(r4 + i);
+#pragma unroll
+      for (int q = 0; q < kCorrRowsPerWarp; ++q) {
+        const float4 x = __ldcs(rows[q] + i);
+        acc[q] = fmaf(x.x, ra.x, acc[q]); acc[q] = fmaf(x.y, ra.y, acc[q]);
+        acc[q] = fmaf(x.z, ra.z, acc[q]); acc[q] = fmaf(x.w, ra.w, acc[q]);
+      }
     }
   }
 #pragma unroll
@@ -243,26 +286,44 @@ __global__ void __launch_bounds__(256) k_gram(Problem p, Work w, int pass) {
 
 // ---------------------------------------------------------------- NNLS ----
 // Lawson-Hanson active set on the normal equations G w = b in fp64, with
-// the Cholesky factor of G restricted to the passive set kept across refits
-// (appended to as variables enter; rebuilt when one leaves).  Entering
-// variables are added in blocks; if an entering block contains a variable
-// that will not grow, the refit continues one variable at a time.
-struct NnlsSmem {
-  double* x;      // [t] current weights (pick-slot indexed)
-  double* z;      // [t] solve buffer (factor-position indexed)
-  double* g;      // [t] gradient b − G x
-  int* P;         // [t] passive list, factor order
-  int* inP;       // [t] 1 if in P
-  int* blocked;   // [t]
-  int* add;       // [t] variables entering this outer iteration
-  double* L;      // packed factor (shared or global)
-};
-
+// the Cholesky factor of G restricted to the passive set kept across refits.
+// Entering variables are appended as a block: their forward solves against
+// the current factor run on separate warps, then a small Cholesky of their
+// Schur complement finishes the new rows.  If an entering block holds a
+// variable that will not grow, the refit continues one variable at a time.
+// Triangular solves multiply by stored reciprocal diagonals.
 __host__ __device__ inline size_t nnls_vec_bytes(int t) {
-  return (size_t)t * (3 * sizeof(double) + 4 * sizeof(int)) + 64 * sizeof(double) + 16 * sizeof(int);
+  // x, z, g, invd: 4t doubles; red: 64 doubles; ctl: 16 ints; P, inP, blocked, add, cand: 5t ints
+  size_t b = (size_t)t * 4 * sizeof(double) + 64 * sizeof(double) + 16 * sizeof(int) + (size_t)t * 5 * sizeof(int);
+  return (b + 15) & ~size_t(15);
 }
 __host__ __device__ inline size_t nnls_tri_bytes(int t) { return (size_t)t * (t + 1) / 2 * sizeof(double); }
 constexpr size_t kSmemCap = 227 * 1024;
+
+// v ← L⁻¹ v (one warp)
+__device__ __forceinline__ void warp_fwd(const double* L, const double* invd, double* v, int n) {
+  const int lane = threadIdx.x & 31;
+  for (int k = 0; k < n; ++k) {
+    const double yk = v[k] * invd[k];
+    __syncwarp();
+    if (lane == 0) v[k] = yk;
+    for (int i = k + 1 + lane; i < n; i += 32) v[i] -= L[tri(i, k)] * yk;
+    __syncwarp();
+  }
+}
+
+// v ← L⁻ᵀ v (one warp)
+__device__ __forceinline__ void warp_bwd(const double* L, const double* invd, double* v, int n) {
+  const int lane = threadIdx.x & 31;
+  for (int k = n - 1; k >= 0; --k) {
+    const double zk = v[k] * invd[k];
+    __syncwarp();
+    if (lane == 0) v[k] = zk;
+    const double* row = L + tri(k, 0);
+    for (int i = lane; i < k; i += 32) v[i] -= row[i] * zk;
+    __syncwarp();
+  }
+}
 
 __global__ void __launch_bounds__(kNnlsThreads) k_nnls(Problem p, Work w, int pass, int l_in_smem_max) {
   extern __shared__ __align__(16) unsigned char smem[];
@@ -271,189 +332,239 @@ __global__ void __launch_bounds__(kNnlsThreads) k_nnls(Problem p, Work w, int pa
   int s0, s1;
   pass_range(p, t, pass, s0, s1);
   if (s0 >= s1) return;
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nw = blockDim.x >> 5;
   const int np_old = w.np[h];
   const int64_t base = w.cu_t[h];
   const int64_t gbase = w.cu_t2[h];
   const double* G = w.G + gbase;
   const double* b = w.bvec + base;
 
-  NnlsSmem S;
-  S.x = reinterpret_cast<double*>(smem);
-  S.z = S.x + t;
-  S.g = S.z + t;
-  double* red = S.g + t;                       // 64 doubles
-  int* ints = reinterpret_cast<int*>(red + 64);
-  int* ctl = ints;                             // 16 ints of control
-  S.P = ints + 16;
-  S.inP = S.P + t;
-  S.blocked = S.inP + t;
-  S.add = S.blocked + t;
+  double* x = reinterpret_cast<double*>(smem);   // pick-slot indexed weights
+  double* z = x + t;                             // factor-position indexed solve buffer
+  double* g = z + t;                             // scaled gradient
+  double* invd = g + t;                          // 1 / L_qq
+  double* red = invd + t;                        // 64 doubles
+  int* ctl = reinterpret_cast<int*>(red + 64);   // 16 ints
+  int* P = ctl + 16;
+  int* inP = P + t;
+  int* blocked = inP + t;
+  int* add = blocked + t;
+  int* cand = add + t;
   const bool l_smem = t <= l_in_smem_max;
   double* Lg = w.L + gbase;
-  S.L = l_smem ? reinterpret_cast<double*>(S.add + t) : Lg;   // 64 + 16t bytes past red: 8-aligned
-  // ctl[0] = np, ctl[1] = nadd, ctl[2] = single_mode, ctl[3] = done/flags,
-  // ctl[4] = argmin, ctl[5] = nneg, ctl[6] = failed factor index, ctl[7] = scratch
+  double* L = l_smem ? reinterpret_cast<double*>(smem + nnls_vec_bytes(t)) : Lg;
+  // ctl: 0 np, 1 nadd, 2 single mode, 4 argmin, 5 nneg, 6 factor flag, 7 ncand, 8 append failures
   const int maxit = p.nnls_max_iter > 0 ? p.nnls_max_iter : 3 * t + 50;
   const double mnorm = sqrt(w.mm[h]);
+  auto diag = [&](int l) { return G[(int64_t)l * t + l]; };
 
   for (int l = tid; l < s1; l += blockDim.x) {
-    S.x[l] = l < s0 ? w.w[base + l] : 0.0;
-    S.inP[l] = 0;
-    S.blocked[l] = 0;
+    x[l] = l < s0 ? w.w[base + l] : 0.0;
+    inP[l] = 0;
+    blocked[l] = 0;
   }
-  for (int q = tid; q < np_old; q += blockDim.x) S.P[q] = w.plist[base + q];
+  for (int q = tid; q < np_old; q += blockDim.x) P[q] = w.plist[base + q];
   if (l_smem)
-    for (int64_t e = tid; e < tri(np_old, 0); e += blockDim.x) S.L[e] = Lg[e];
-  if (tid == 0) { ctl[0] = np_old; ctl[2] = 0; ctl[3] = 0; }
+    for (int64_t e = tid; e < tri(np_old, 0); e += blockDim.x) L[e] = Lg[e];
+  if (tid == 0) { ctl[0] = np_old; ctl[2] = 0; }
   __syncthreads();
-  for (int q = tid; q < np_old; q += blockDim.x) S.inP[S.P[q]] = 1;
+  for (int q = tid; q < np_old; q += blockDim.x) {
+    inP[P[q]] = 1;
+    invd[q] = 1.0 / L[tri(q, q)];
+  }
   __syncthreads();
-
-  auto diag = [&](int l) { return G[(int64_t)l * t + l]; };
-  int iter = 0;
-  bool converged = false;
 
   // Rebuild the factor of G[P, P] from scratch; drops dependent variables.
   auto refactor = [&]() {
     for (;;) {
       const int np = ctl[0];
-      for (int a = warp; a < np; a += blockDim.x >> 5)
-        for (int c = lane; c <= a; c += 32) S.L[tri(a, c)] = G[(int64_t)S.P[a] * t + S.P[c]];
+      for (int a = warp; a < np; a += nw)
+        for (int c = lane; c <= a; c += 32) L[tri(a, c)] = G[(int64_t)P[a] * t + P[c]];
       __syncthreads();
-      int badk = block_cholesky_packed(S.L, np, [&](int k) { return 1e-13 * diag(S.P[k]); }, &ctl[6]);
-      if (badk < 0) return;
+      int badk = block_cholesky_packed(L, np, [&](int k) { return 1e-13 * diag(P[k]); }, &ctl[6]);
+      if (badk < 0) {
+        for (int q = tid; q < np; q += blockDim.x) invd[q] = 1.0 / L[tri(q, q)];
+        __syncthreads();
+        return;
+      }
       if (tid == 0) {
-        int l = S.P[badk];
-        S.inP[l] = 0;
-        S.blocked[l] = 1;
-        S.x[l] = 0.0;
-        for (int q = badk; q + 1 < np; ++q) S.P[q] = S.P[q + 1];
+        const int l = P[badk];
+        inP[l] = 0;
+        blocked[l] = 1;
+        x[l] = 0.0;
+        for (int q = badk; q + 1 < np; ++q) P[q] = P[q + 1];
         ctl[0] = np - 1;
       }
       __syncthreads();
     }
   };
 
-  for (;;) {
-    // ---- gradient over non-passive variables, choose entering set ----
-    const int np = ctl[0];
-    for (int q = tid; q < np; q += blockDim.x) S.z[q] = S.x[S.P[q]];   // x gathered to factor order
-    __syncthreads();
-    for (int l = tid; l < s1; l += blockDim.x) {
-      double gl = -INFINITY;
-      if (!S.inP[l] && !S.blocked[l]) {
-        const double* Gl = G + (int64_t)l * t;
-        double acc = b[l];
-        for (int q = 0; q < np; ++q) acc -= Gl[S.P[q]] * S.z[q];
-        const double dl = diag(l);
-        gl = dl > 0.0 ? acc / (sqrt(dl) * mnorm) : -INFINITY;   // scale-free gradient
+  // Append add[0..nadd) to the factor as a block; variables whose Schur
+  // pivot is too small are blocked and the block is redone without them.
+  auto block_append = [&]() {
+    for (;;) {
+      const int np = ctl[0], k = ctl[1];
+      if (k == 0) return;
+      // right-hand sides G[add_e, P] into the new packed rows
+      for (int e = warp; e < k; e += nw) {
+        double* row = L + tri(np + e, 0);
+        const double* Ge = G + (int64_t)add[e] * t;
+        for (int q = lane; q < np; q += 32) row[q] = Ge[P[q]];
       }
-      S.g[l] = gl;
+      __syncthreads();
+      for (int e = warp; e < k; e += nw) warp_fwd(L, invd, L + tri(np + e, 0), np);
+      __syncthreads();
+      // Schur complement of the new block (lower triangle)
+      for (int pr = warp; pr < k * (k + 1) / 2; pr += nw) {
+        int e = 0;
+        while ((e + 1) * (e + 2) / 2 <= pr) ++e;
+        const int f = pr - e * (e + 1) / 2;
+        const double* re = L + tri(np + e, 0);
+        const double* rf = L + tri(np + f, 0);
+        double acc = 0.0;
+        for (int q = lane; q < np; q += 32) acc += re[q] * rf[q];
+        acc = warp_sum(acc);
+        if (lane == 0) L[tri(np + e, np + f)] = G[(int64_t)add[e] * t + add[f]] - acc;
+      }
+      __syncthreads();
+      if (tid == 0) {
+        int failed = 0;
+        for (int f = 0; f < k; ++f) {
+          const double piv = L[tri(np + f, np + f)];
+          if (!(piv > 1e-13 * diag(add[f]))) { blocked[add[f]] = 1; ++failed; break; }
+          const double lff = sqrt(piv);
+          L[tri(np + f, np + f)] = lff;
+          invd[np + f] = 1.0 / lff;
+          for (int e = f + 1; e < k; ++e) L[tri(np + e, np + f)] /= lff;
+          for (int e = f + 1; e < k; ++e)
+            for (int q = f + 1; q <= e; ++q) L[tri(np + e, np + q)] -= L[tri(np + e, np + f)] * L[tri(np + q, np + f)];
+        }
+        if (failed) {
+          int kk = 0;
+          for (int e = 0; e < k; ++e)
+            if (!blocked[add[e]]) add[kk++] = add[e];
+          ctl[1] = kk;
+        } else {
+          for (int e = 0; e < k; ++e) {
+            P[np + e] = add[e];
+            inP[add[e]] = 1;
+          }
+          ctl[0] = np + k;
+          ctl[1] = 0;
+        }
+      }
+      __syncthreads();
+      if (ctl[1] == 0) return;
+    }
+  };
+
+  int iter = 0;
+  bool converged = false;
+  for (int outer = 0; outer <= maxit; ++outer) {
+    // ---- candidates and their scaled gradients b_l − G[l, P] x_P ----
+    const int np = ctl[0];
+    for (int q = tid; q < np; q += blockDim.x) z[q] = x[P[q]];
+    if (warp == 0) {
+      int nc = 0;
+      for (int l0 = 0; l0 < s1; l0 += 32) {
+        const int l = l0 + lane;
+        const bool c = l < s1 && !inP[l] && !blocked[l];
+        const unsigned msk = __ballot_sync(0xffffffffu, c);
+        if (c) cand[nc + __popc(msk & ((1u << lane) - 1))] = l;
+        nc += __popc(msk);
+      }
+      if (lane == 0) ctl[7] = nc;
+    }
+    __syncthreads();
+    const int nc = ctl[7];
+    for (int ci = warp; ci < nc; ci += nw) {
+      const int l = cand[ci];
+      const double* Gl = G + (int64_t)l * t;
+      double acc = 0.0;
+      for (int q = lane; q < np; q += 32) acc += Gl[P[q]] * z[q];
+      acc = warp_sum(acc);
+      if (lane == 0) {
+        const double dl = diag(l);
+        g[l] = dl > 0.0 ? (b[l] - acc) / (sqrt(dl) * mnorm) : -INFINITY;
+      }
     }
     __syncthreads();
     if (warp == 0) {
       const double tol = 1e-11;
       int nadd = 0;
-      if (ctl[2]) {                         // single mode: argmax only
+      if (ctl[2]) {                                    // single mode: argmax only
         double bv = tol;
         int bi = -1;
-        for (int l = lane; l < s1; l += 32)
-          if (S.g[l] > bv) { bv = S.g[l]; bi = l; }
+        for (int ci = lane; ci < nc; ci += 32) {
+          const int l = cand[ci];
+          if (g[l] > bv || (g[l] == bv && bi >= 0 && l < bi)) { bv = g[l]; bi = l; }
+        }
         for (int o = 16; o; o >>= 1) {
-          double ov = __shfl_xor_sync(0xffffffffu, bv, o);
-          int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+          const double ov = __shfl_xor_sync(0xffffffffu, bv, o);
+          const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
           if (ov > bv || (ov == bv && oi >= 0 && (bi < 0 || oi < bi))) { bv = ov; bi = oi; }
         }
-        if (lane == 0 && bi >= 0) { S.add[0] = bi; nadd = 1; }
+        if (lane == 0 && bi >= 0) { add[0] = bi; nadd = 1; }
+        nadd = __shfl_sync(0xffffffffu, nadd, 0);
       } else {
-        for (int l0 = 0; l0 < s1; l0 += 32) {
-          int l = l0 + lane;
-          bool c = l < s1 && S.g[l] > tol;
-          unsigned msk = __ballot_sync(0xffffffffu, c);
-          if (c) S.add[nadd + __popc(msk & ((1u << lane) - 1))] = l;
+        for (int c0 = 0; c0 < nc; c0 += 32) {
+          const int ci = c0 + lane;
+          const bool c = ci < nc && g[cand[ci]] > tol;
+          const unsigned msk = __ballot_sync(0xffffffffu, c);
+          if (c) add[nadd + __popc(msk & ((1u << lane) - 1))] = cand[ci];
           nadd += __popc(msk);
         }
       }
-      nadd = __shfl_sync(0xffffffffu, nadd, 0);
       if (lane == 0) ctl[1] = nadd;
     }
     __syncthreads();
-    const int nadd = ctl[1];
-    if (nadd == 0) { converged = true; break; }
-
-    // ---- append entering variables to the factor (warp 0) ----
-    if (warp == 0) {
-      for (int e = 0; e < nadd; ++e) {
-        const int l = S.add[e];
-        const int npc = ctl[0];
-        double* row = S.L + tri(npc, 0);
-        const double* Gl = G + (int64_t)l * t;
-        for (int q = lane; q < npc; q += 32) row[q] = Gl[S.P[q]];
-        __syncwarp();
-        warp_forward_solve(S.L, row, npc);
-        double ss = 0.0;
-        for (int q = lane; q < npc; q += 32) ss += row[q] * row[q];
-        ss = warp_sum(ss);
-        const double delta = diag(l) - ss;
-        if (delta > 1e-13 * diag(l)) {
-          if (lane == 0) {
-            row[npc] = sqrt(delta);
-            S.P[npc] = l;
-            S.inP[l] = 1;
-            ctl[0] = npc + 1;
-          }
-        } else if (lane == 0) {
-          S.blocked[l] = 1;
-        }
-        __syncwarp();
-      }
-    }
-    __syncthreads();
+    if (ctl[1] == 0) { converged = true; break; }
+    block_append();
 
     // ---- inner loop: solve on P, step back toward feasibility ----
     bool abort = false;
     for (;;) {
       if (++iter > maxit) { abort = true; break; }
       const int npc = ctl[0];
-      for (int q = tid; q < npc; q += blockDim.x) S.z[q] = b[S.P[q]];
+      for (int q = tid; q < npc; q += blockDim.x) z[q] = b[P[q]];
       __syncthreads();
       if (warp == 0) {
-        warp_forward_solve(S.L, S.z, npc);
-        warp_backward_solve(S.L, S.z, npc);
+        warp_fwd(L, invd, z, npc);
+        warp_bwd(L, invd, z, npc);
       }
       __syncthreads();
-      // min step ratio over non-positive entries
       double best = INFINITY;
       int bq = -1, nneg = 0;
       for (int q = tid; q < npc; q += blockDim.x) {
-        const double zq = S.z[q];
+        const double zq = z[q];
         if (!(zq > 0.0)) {
           ++nneg;
-          const double xq = S.x[S.P[q]];
+          const double xq = x[P[q]];
           const double den = xq - zq;
           const double ratio = den > 0.0 ? xq / den : 0.0;
           if (ratio < best || (ratio == best && q < bq)) { best = ratio; bq = q; }
         }
       }
-      // block argmin
       for (int o = 16; o; o >>= 1) {
-        double ov = __shfl_xor_sync(0xffffffffu, best, o);
-        int oq = __shfl_xor_sync(0xffffffffu, bq, o);
-        int on = __shfl_xor_sync(0xffffffffu, nneg, o);
-        nneg += on;
+        const double ov = __shfl_xor_sync(0xffffffffu, best, o);
+        const int oq = __shfl_xor_sync(0xffffffffu, bq, o);
+        nneg += __shfl_xor_sync(0xffffffffu, nneg, o);
         if (ov < best || (ov == best && oq >= 0 && (bq < 0 || oq < bq))) { best = ov; bq = oq; }
       }
-      if (tid == 0) { ctl[5] = 0; }
+      if (tid == 0) ctl[5] = 0;
       __syncthreads();
-      if (lane == 0) { red[warp] = best; reinterpret_cast<int*>(red + 16)[warp] = bq; atomicAdd(&ctl[5], nneg); }
+      if (lane == 0) {
+        red[warp] = best;
+        reinterpret_cast<int*>(red + 16)[warp] = bq;
+        atomicAdd(&ctl[5], nneg);
+      }
       __syncthreads();
       if (tid == 0) {
         double bv = INFINITY;
         int bi = -1;
-        for (int k = 0; k < (int)(blockDim.x >> 5); ++k) {
-          double v = red[k];
-          int qi = reinterpret_cast<int*>(red + 16)[k];
+        for (int k = 0; k < nw; ++k) {
+          const double v = red[k];
+          const int qi = reinterpret_cast<int*>(red + 16)[k];
           if (qi >= 0 && (v < bv || (v == bv && qi < bi))) { bv = v; bi = qi; }
         }
         red[32] = bv;
@@ -461,7 +572,7 @@ __global__ void __launch_bounds__(kNnlsThreads) k_nnls(Problem p, Work w, int pa
       }
       __syncthreads();
       if (ctl[5] == 0) {   // all positive: accept
-        for (int q = tid; q < npc; q += blockDim.x) S.x[S.P[q]] = S.z[q];
+        for (int q = tid; q < npc; q += blockDim.x) x[P[q]] = z[q];
         __syncthreads();
         break;
       }
@@ -469,42 +580,41 @@ __global__ void __launch_bounds__(kNnlsThreads) k_nnls(Problem p, Work w, int pa
       if (alpha == 0.0) {
         // entering variables that will not grow: drop them
         if (tid == 0) {
-          int k = 0;
+          int kk = 0;
           const bool single = ctl[2];
           for (int q = 0; q < npc; ++q) {
-            const int l = S.P[q];
-            if (!(S.z[q] > 0.0) && S.x[l] == 0.0) {
-              S.inP[l] = 0;
-              if (single) S.blocked[l] = 1;
+            const int l = P[q];
+            if (!(z[q] > 0.0) && x[l] == 0.0) {
+              inP[l] = 0;
+              if (single) blocked[l] = 1;
             } else {
-              S.P[k++] = l;
+              P[kk++] = l;
             }
           }
-          ctl[0] = k;
+          ctl[0] = kk;
           ctl[2] = 1;
         }
       } else {
         const int qmin = ctl[4];
         for (int q = tid; q < npc; q += blockDim.x) {
-          const int l = S.P[q];
-          double v = S.x[l] + alpha * (S.z[q] - S.x[l]);
+          const int l = P[q];
+          double v = x[l] + alpha * (z[q] - x[l]);
           if (q == qmin) v = 0.0;
-          S.x[l] = v;
+          x[l] = v;
         }
         __syncthreads();
         if (tid == 0) {
-          int k = 0;
+          int kk = 0;
           for (int q = 0; q < npc; ++q) {
-            const int l = S.P[q];
-            if (S.x[l] <= 0.0) { S.inP[l] = 0; S.x[l] = 0.0; }
-            else S.P[k++] = l;
+            const int l = P[q];
+            if (x[l] <= 0.0) { inP[l] = 0; x[l] = 0.0; }
+            else P[kk++] = l;
           }
-          ctl[0] = k;
+          ctl[0] = kk;
         }
       }
       __syncthreads();
       refactor();
-      __syncthreads();
     }
     if (abort) break;
   }
@@ -512,10 +622,10 @@ __global__ void __launch_bounds__(kNnlsThreads) k_nnls(Problem p, Work w, int pa
 
   // ---- write back ----
   const int npf = ctl[0];
-  for (int l = tid; l < s1; l += blockDim.x) w.w[base + l] = S.inP[l] ? S.x[l] : 0.0;
-  for (int q = tid; q < npf; q += blockDim.x) w.plist[base + q] = S.P[q];
+  for (int l = tid; l < s1; l += blockDim.x) w.w[base + l] = inP[l] ? x[l] : 0.0;
+  for (int q = tid; q < npf; q += blockDim.x) w.plist[base + q] = P[q];
   if (l_smem)
-    for (int64_t e = tid; e < tri(npf, 0); e += blockDim.x) Lg[e] = S.L[e];
+    for (int64_t e = tid; e < tri(npf, 0); e += blockDim.x) Lg[e] = L[e];
   if (tid == 0) {
     w.np[h] = npf;
     if (!converged) record_status(w.status + h, AM_WARN_NOT_CONVERGED);

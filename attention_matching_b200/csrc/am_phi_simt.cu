@@ -118,7 +118,7 @@ __global__ void k_shift_copy(const float* src, float* dst, int H) {
 // Φᵀ[h][j][i] = exp(s_ij − c_h) for i < n, 0 in the padding n <= i < ldn.
 __global__ void __launch_bounds__(256) k_phi(Problem p, const void* Q, const void* K,
                                              const float* key_bias, const float* shift,
-                                             float* phiT) {
+                                             float* phiT, __nv_bfloat16* phiT16) {
   __shared__ __align__(16) float Qs[DK][TQ + 4];
   __shared__ __align__(16) float Ks[DK][TK + 4];
   const int h = blockIdx.z, i0 = blockIdx.x * TQ, j0 = blockIdx.y * TK;
@@ -140,6 +140,11 @@ __global__ void __launch_bounds__(256) k_phi(Problem p, const void* Q, const voi
       v[a] = (ibase + a < p.n) ? expf(fmaf(acc[a][b], p.scale, bmc)) : 0.f;
     *reinterpret_cast<float4*>(phiT + ((int64_t)h * p.T + j) * p.ldn + ibase) =
         make_float4(v[0], v[1], v[2], v[3]);
+    if (phiT16) {   // bf16 copy streamed by the correlation pass
+      __nv_bfloat162 lo = __floats2bfloat162_rn(v[0], v[1]), hi = __floats2bfloat162_rn(v[2], v[3]);
+      uint2 pk = make_uint2(*reinterpret_cast<uint32_t*>(&lo), *reinterpret_cast<uint32_t*>(&hi));
+      *reinterpret_cast<uint2*>(phiT16 + ((int64_t)h * p.T + j) * p.ldn + ibase) = pk;
+    }
   }
 }
 
@@ -229,7 +234,7 @@ cudaError_t launch_shift_max(const Problem& p, const void* Q, const void* K, con
 cudaError_t launch_phi(const Problem& p, const void* Q, const void* K, const float* key_bias,
                        const Work& w, cudaStream_t s) {
   dim3 grid((p.ldn + TQ - 1) / TQ, (p.T + TK - 1) / TK, p.H);
-  AM_LAUNCH(AM_STAGE_PHI, s, k_phi<<<grid, 256, 0, s>>>(p, Q, K, key_bias, w.shift, w.phiT));
+  AM_LAUNCH(AM_STAGE_PHI, s, k_phi<<<grid, 256, 0, s>>>(p, Q, K, key_bias, w.shift, w.phiT, w.phiT16));
   return cudaGetLastError();
 }
 

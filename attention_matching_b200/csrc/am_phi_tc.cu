@@ -13,11 +13,12 @@
 //            accumulators (kind::f16, bf16 in, fp32 out), then Y += P·V
 //            from the epilogue's P tiles (PHI mode)
 //   warp 2   TMEM allocation and release
-//   warps 4-7 epilogue: thread r owns query row r (TMEM lane r); per tile it
-//            reads 64 logits, forms p = exp(s·scale + b − c), adds p to the
-//            fp64 mass, writes Φᵀ (a warp writes 32 consecutive queries of one
-//            key: 128-byte coalesced), and stores p split as bf16 hi + lo
-//            (p = hi + lo to 16 bits) into a swizzled K-major operand for Y.
+//   warps 4-11 epilogue, two warpgroups: thread (half, r) owns query row r
+//            (TMEM lane r) and 32 of each tile's 64 keys; it reads its logits,
+//            forms p = exp(s·scale + b − c), adds p to the fp64 mass, writes Φᵀ
+//            (a warp writes 32 consecutive queries of one key: 128-byte
+//            coalesced), and stores p split as bf16 hi + lo (p = hi + lo to 16
+//            bits) into a swizzled K-major operand for Y.
 // MAX mode computes only max_ij (s·scale + b) per head (the shift).
 //
 // Every mbarrier wait is bounded by a clock budget; on expiry the CTA records
@@ -35,7 +36,7 @@ namespace {
 constexpr int BM = 128;        // queries per CTA (TMEM lanes)
 constexpr int BN = 64;         // keys per tile
 constexpr int STAGES = 3;      // key/value ring depth
-constexpr int kThreads = 256;
+constexpr int kThreads = 384;   // 4 control warps + 2 epilogue warpgroups
 constexpr int kEpiWarp0 = 4;   // first epilogue warp
 constexpr uint32_t kTmemCols = 256;
 constexpr long long kWaitBudgetCycles = 4000000000ll;   // ~2 s at 2 GHz
@@ -213,7 +214,8 @@ k_phi_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtens
   uint64_t* drain = s_full + 9;
   __shared__ uint32_t s_tmem;
   __shared__ int s_abort;
-  __shared__ float s_red[4];
+  __shared__ float s_red[8];
+  __shared__ double s_mass[256];
   __shared__ int s_stop[2];
   __shared__ int s_stop_y;
 
@@ -231,8 +233,8 @@ k_phi_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtens
     for (int s = 0; s < STAGES; ++s) { mbar_init(kv_full + s, 1); mbar_init(kv_empty + s, 1); }
     for (int b = 0; b < 2; ++b) {
       mbar_init(s_full + b, 1);
-      mbar_init(s_empty + b, 128);
-      mbar_init(p_full + b, 128);
+      mbar_init(s_empty + b, 256);
+      mbar_init(p_full + b, 256);
       mbar_init(p_empty + b, 1);
     }
     mbar_init(y_full, 1);
@@ -329,12 +331,21 @@ k_phi_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtens
     }
   } else if (warp >= kEpiWarp0) {
     // --------------------------------------------------- epilogue ----
-    const int et = threadIdx.x - kEpiWarp0 * 32;     // 0..127 = TMEM lane = query row
-    const int qd = warp - kEpiWarp0;                 // lane quadrant
+    // Two warpgroups: thread (half, et) owns query row et (TMEM lane et) and
+    // columns [32·half, 32·half + 32) of every 64-key tile.
+    const int ep = threadIdx.x - kEpiWarp0 * 32;     // 0..255
+    const int half = ep >> 7;
+    const int et = ep & 127;
+    const int qd = warp & 3;                         // TMEM lane quadrant of this warp
+    constexpr int HC = BN / 2;
     const int i = q0 + et;
     const bool row_live = i < p.n;
-    const float scale = p.scale;
     const float c = MODE == MODE_PHI ? w.shift[h] : 0.f;
+    // PHI: p = 2^(s·scale·log2e + (b − c)·log2e); any rounding of log2e or of
+    // c·log2e multiplies every feature of the head by one common factor,
+    // which no result depends on (the shift invariance).
+    const float kLog2e = 1.4426950408889634f;
+    const float scale = MODE == MODE_PHI ? p.scale * kLog2e : p.scale;
     double mrow = 0.0;
     float mx = -FLT_MAX;
     const uint32_t lane_addr = (uint32_t)(qd * 32) << 16;
@@ -343,68 +354,71 @@ k_phi_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtens
     for (int j = 0; j < NT; ++j) {
       const int b = j & 1, bu = j >> 1;
       // One thread waits (S tile ready; P buffer free again) and publishes a
-      // stop flag, so all 128 epilogue threads leave the loop together.
-      if (et == 0) {
+      // stop flag, so all 256 epilogue threads leave the loop together.
+      if (ep == 0) {
         bool good = mbar_wait(s_full + b, bu & 1, abort_flag, status);
         if (good && MODE == MODE_PHI && bu > 0) good = mbar_wait(p_empty + b, (bu - 1) & 1, abort_flag, status);
         s_stop[b] = good ? 0 : 1;
       }
-      // this tile's (bias − shift) per key, shared by the 128 rows
-      if (et < BN) {
-        const int jg = j * BN + et;
+      if (ep < BN) {   // this tile's per-key additive term, shared by all rows
+        const int jg = j * BN + ep;
         const float bj = (p.has_bias && jg < p.T) ? key_bias[(int64_t)h * p.T + jg] : 0.f;
-        sBias[b * BN + et] = MODE == MODE_PHI ? bj - c : bj;
+        sBias[b * BN + ep] = MODE == MODE_PHI ? (bj - c) * kLog2e : bj;
       }
-      asm volatile("bar.sync 1, 128;" ::: "memory");
+      asm volatile("bar.sync 1, 256;" ::: "memory");
       if (s_stop[b]) { ok = false; break; }
       tc_fence_after();
-      float v[BN];
-      tmem_ld32(tS[b] + lane_addr, *reinterpret_cast<float(*)[32]>(&v[0]));
-      tmem_ld32(tS[b] + lane_addr + 32, *reinterpret_cast<float(*)[32]>(&v[32]));
+      float v[HC];
+      tmem_ld32(tS[b] + lane_addr + half * HC, v);
       tmem_wait_ld();
       tc_fence_before();
       mbar_arrive(s_empty + b);
-      const int kvalid = min(BN, p.T - j * BN);
-      const float* bias_t = sBias + b * BN;
+      const int kvalid = min(BN, p.T - j * BN) - half * HC;   // valid columns of this half
+      const float* bias_t = sBias + b * BN + half * HC;
       if constexpr (MODE == MODE_MAX) {
         if (row_live) {
 #pragma unroll
-          for (int cc = 0; cc < BN; ++cc)
+          for (int cc = 0; cc < HC; ++cc)
             if (cc < kvalid) mx = fmaxf(mx, fmaf(v[cc], scale, bias_t[cc]));
         }
         continue;
       } else {
-      // p = exp(s·scale + b − c): one rounding of the argument
 #pragma unroll
-      for (int cc = 0; cc < BN; ++cc) {
+      for (int cc = 0; cc < HC; ++cc) {
         const float x = fmaf(v[cc], scale, bias_t[cc]);
-        v[cc] = (row_live && cc < kvalid) ? expf(x) : 0.f;
+        v[cc] = (row_live && cc < kvalid) ? exp2f(x) : 0.f;
       }
-      double part = 0.0;
+      double a4[4] = {0.0, 0.0, 0.0, 0.0};   // mass partials: short dependency chains
 #pragma unroll
-      for (int cc = 0; cc < BN; ++cc) part += (double)v[cc];
-      mrow += part;
+      for (int cc = 0; cc < HC; ++cc) a4[cc & 3] += (double)v[cc];
+      mrow += (a4[0] + a4[1]) + (a4[2] + a4[3]);
       if (i < p.ldn) {
-        float* col = phi_base + (int64_t)(j * BN) * p.ldn + i;
+        float* col = phi_base + (int64_t)(j * BN + half * HC) * p.ldn + i;
 #pragma unroll
-        for (int cc = 0; cc < BN; ++cc)
+        for (int cc = 0; cc < HC; ++cc)
           if (cc < kvalid) col[(int64_t)cc * p.ldn] = v[cc];
+        if (w.phiT16) {   // bf16 copy streamed by the correlation pass
+          __nv_bfloat16* col16 = w.phiT16 + ((int64_t)h * p.T + j * BN + half * HC) * p.ldn + i;
+#pragma unroll
+          for (int cc = 0; cc < HC; ++cc)
+            if (cc < kvalid) col16[(int64_t)cc * p.ldn] = __float2bfloat16_rn(v[cc]);
+        }
       }
       // P tile for Y += P·V: K-major, 128-byte rows, 16-byte chunks XOR-swizzled by row
       unsigned char* hi_row = sP + (b * 2 + 0) * P.p_bytes + et * 128;
       unsigned char* lo_row = sP + (b * 2 + 1) * P.p_bytes + et * 128;
 #pragma unroll
-      for (int ch = 0; ch < 8; ++ch) {
+      for (int c4 = 0; c4 < HC / 8; ++c4) {
         uint32_t hv[4], lv[4];
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-          const float a0 = v[ch * 8 + 2 * e], a1 = v[ch * 8 + 2 * e + 1];
-          const float h0 = __bfloat162float(__float2bfloat16_rn(a0));
-          const float h1 = __bfloat162float(__float2bfloat16_rn(a1));
-          hv[e] = pack_bf16x2(h0, h1);
-          lv[e] = pack_bf16x2(a0 - h0, a1 - h1);
+          const float a0 = v[c4 * 8 + 2 * e], a1 = v[c4 * 8 + 2 * e + 1];
+          const __nv_bfloat162 hb = __floats2bfloat162_rn(a0, a1);
+          const float2 hf = __bfloat1622float2(hb);
+          hv[e] = *reinterpret_cast<const uint32_t*>(&hb);
+          lv[e] = pack_bf16x2(a0 - hf.x, a1 - hf.y);
         }
-        const int pc = ch ^ (et & 7);
+        const int pc = (half * (HC / 8) + c4) ^ (et & 7);
         *reinterpret_cast<uint4*>(hi_row + pc * 16) = make_uint4(hv[0], hv[1], hv[2], hv[3]);
         *reinterpret_cast<uint4*>(lo_row + pc * 16) = make_uint4(lv[0], lv[1], lv[2], lv[3]);
       }
@@ -414,33 +428,40 @@ k_phi_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtens
     }
     if (MODE == MODE_MAX) {
       for (int o = 16; o; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-      if (lane == 0) s_red[qd] = mx;
-      asm volatile("bar.sync 1, 128;" ::: "memory");
-      if (et == 0) {
-        const float v = fmaxf(fmaxf(s_red[0], s_red[1]), fmaxf(s_red[2], s_red[3]));
+      if (lane == 0) s_red[warp - kEpiWarp0] = mx;
+      asm volatile("bar.sync 1, 256;" ::: "memory");
+      if (ep == 0) {
+        float v = s_red[0];
+        for (int k = 1; k < 8; ++k) v = fmaxf(v, s_red[k]);
         atomicMax(shift_ord + h, f2ord(v));
       }
     } else {
-      if (et == 0) s_stop_y = (ok && mbar_wait(y_full, 0, abort_flag, status)) ? 0 : 1;
-      asm volatile("bar.sync 1, 128;" ::: "memory");
+      // combine the two halves' mass partials (fixed order: half 0 + half 1)
+      if (half == 1) s_mass[et] = mrow;
+      if (ep == 0) s_stop_y = (ok && mbar_wait(y_full, 0, abort_flag, status)) ? 0 : 1;
+      asm volatile("bar.sync 1, 256;" ::: "memory");
+      if (half == 0) s_mass[128 + et] = mrow + s_mass[et];
+      asm volatile("bar.sync 1, 256;" ::: "memory");
+      const double mtot = s_mass[128 + et];
       if (!s_stop_y) {
         tc_fence_after();
         float* yrow = w.Y + ((int64_t)h * p.n + i) * p.d;
 #pragma unroll
-        for (int c0 = 0; c0 < D; c0 += 32) {
+        for (int c0 = 0; c0 < D / 2; c0 += 32) {
+          const int cb = half * (D / 2) + c0;
           float y[32];
-          tmem_ld32(tY + lane_addr + c0, y);
+          tmem_ld32(tY + lane_addr + cb, y);
           tmem_wait_ld();
           if (row_live) {
 #pragma unroll
             for (int cc = 0; cc < 32; cc += 4)
-              *reinterpret_cast<float4*>(yrow + c0 + cc) =
-                  make_float4((float)(y[cc] / mrow), (float)(y[cc + 1] / mrow), (float)(y[cc + 2] / mrow),
-                              (float)(y[cc + 3] / mrow));
+              *reinterpret_cast<float4*>(yrow + cb + cc) =
+                  make_float4((float)(y[cc] / mtot), (float)(y[cc + 1] / mtot), (float)(y[cc + 2] / mtot),
+                              (float)(y[cc + 3] / mtot));
           }
         }
-        if (i < p.ldn) {
-          const double mv = row_live ? mrow : 0.0;
+        if (half == 0 && i < p.ldn) {
+          const double mv = row_live ? mtot : 0.0;
           w.m[(int64_t)h * p.ldn + i] = mv;
           w.r[(int64_t)h * p.ldn + i] = (float)mv;
         }

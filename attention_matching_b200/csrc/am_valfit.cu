@@ -186,7 +186,9 @@ __global__ void __launch_bounds__(256) k_normal(Problem p, Work w) {
     }
 }
 
-__global__ void __launch_bounds__(kCholThreads) k_solve(Problem p, Work w, float* C_v, int l_smem_max) {
+// λ = ridge·tr(AᵀA)/t; packed Cholesky factor of AᵀA + λI and its
+// reciprocal diagonal, written to the workspace (one CTA per head).
+__global__ void __launch_bounds__(kCholThreads) k_chol(Problem p, Work w, int l_smem_max) {
   extern __shared__ __align__(16) unsigned char smem[];
   const int h = blockIdx.x;
   const int t = w.t[h];
@@ -199,47 +201,77 @@ __global__ void __launch_bounds__(kCholThreads) k_solve(Problem p, Work w, float
   for (int a = threadIdx.x; a < t; a += blockDim.x) tr += M[(int64_t)a * t + a];
   tr = block_sum(tr, scratch);
   const double lam = (double)p.ridge * tr / t;
-  double* L = t <= l_smem_max ? reinterpret_cast<double*>(smem) : w.L + gbase;
+  double* Lg = w.L + gbase;
+  double* L = t <= l_smem_max ? reinterpret_cast<double*>(smem) : Lg;
   for (int a = threadIdx.x >> 5; a < t; a += blockDim.x >> 5)
-    for (int c = threadIdx.x & 31; c <= a; c += 32)
-      L[tri(a, c)] = M[(int64_t)a * t + c] + (a == c ? lam : 0.0);
+    for (int c = threadIdx.x & 31; c <= a; c += 32) L[tri(a, c)] = M[(int64_t)a * t + c] + (a == c ? lam : 0.0);
   __syncthreads();
   const int bad = block_cholesky_packed(L, t, [](int) { return 0.0; }, &flag);
-  double* X = w.AtY + base * p.d;
   if (bad >= 0) {
     if (threadIdx.x == 0) record_status(w.status + h, AM_ERR_NOT_SPD);
-    for (int64_t e = threadIdx.x; e < (int64_t)t * p.d; e += blockDim.x) C_v[base * p.d + e] = 0.f;
+    for (int a = threadIdx.x; a < t; a += blockDim.x) w.w_eff[base + a] = 0.0;   // marks the head for k_trsm
     return;
   }
-  // one right-hand-side column per thread; four partial sums for ILP
-  for (int c = threadIdx.x; c < p.d; c += blockDim.x) {
-    for (int k = 0; k < t; ++k) {
-      const double* Lk = L + tri(k, 0);
-      double s0 = X[(int64_t)k * p.d + c], s1 = 0.0, s2 = 0.0, s3 = 0.0;
-      int j = 0;
-      for (; j + 3 < k; j += 4) {
-        s0 -= Lk[j] * X[(int64_t)j * p.d + c];
-        s1 -= Lk[j + 1] * X[(int64_t)(j + 1) * p.d + c];
-        s2 -= Lk[j + 2] * X[(int64_t)(j + 2) * p.d + c];
-        s3 -= Lk[j + 3] * X[(int64_t)(j + 3) * p.d + c];
-      }
-      for (; j < k; ++j) s0 -= Lk[j] * X[(int64_t)j * p.d + c];
-      X[(int64_t)k * p.d + c] = ((s0 + s1) + (s2 + s3)) / Lk[k];
+  if (L != Lg)
+    for (int64_t e = threadIdx.x; e < tri(t, 0); e += blockDim.x) Lg[e] = L[e];
+  // reciprocal diagonal in the NNLS vector slot (free after the bias is packed)
+  for (int a = threadIdx.x; a < t; a += blockDim.x) w.bvec[base + a] = 1.0 / L[tri(a, a)];
+}
+
+// C_v[:, c0:c0+CW] = L⁻ᵀ L⁻¹ AᵀY[:, c0:c0+CW]; 256 threads, 256/CW per column,
+// each row's dot product split across a column's threads.
+template <int CW>
+__global__ void __launch_bounds__(256) k_trsm(Problem p, Work w, float* C_v, int l_smem_max) {
+  extern __shared__ __align__(16) unsigned char smem[];
+  constexpr int TPC = 256 / CW;                 // threads per column (power of two)
+  const int h = blockIdx.x;
+  const int c0 = blockIdx.y * CW;
+  const int t = w.t[h];
+  const int64_t base = w.cu_t[h];
+  const int64_t gbase = w.cu_t2[h];
+  if (c0 >= p.d) return;
+  const double* invd = w.bvec + base;
+  const bool l_smem = t <= l_smem_max;
+  double* X = reinterpret_cast<double*>(smem);              // [t][CW]
+  double* Ls = X + (size_t)t * CW;
+  const double* L = l_smem ? Ls : w.L + gbase;
+  if (w.w_eff[base] == 0.0 && w.status[h] != 0) {           // factorization failed
+    for (int e = threadIdx.x; e < t * CW; e += blockDim.x) {
+      const int r = e / CW, c = c0 + e % CW;
+      if (c < p.d) C_v[(base + r) * p.d + c] = 0.f;
     }
-    for (int k = t - 1; k >= 0; --k) {
-      double s0 = X[(int64_t)k * p.d + c], s1 = 0.0, s2 = 0.0, s3 = 0.0;
-      int j = k + 1;
-      for (; j + 3 < t; j += 4) {
-        s0 -= L[tri(j, k)] * X[(int64_t)j * p.d + c];
-        s1 -= L[tri(j + 1, k)] * X[(int64_t)(j + 1) * p.d + c];
-        s2 -= L[tri(j + 2, k)] * X[(int64_t)(j + 2) * p.d + c];
-        s3 -= L[tri(j + 3, k)] * X[(int64_t)(j + 3) * p.d + c];
-      }
-      for (; j < t; ++j) s0 -= L[tri(j, k)] * X[(int64_t)j * p.d + c];
-      const double xk = ((s0 + s1) + (s2 + s3)) / L[tri(k, k)];
-      X[(int64_t)k * p.d + c] = xk;
-      C_v[(base + k) * p.d + c] = (float)xk;
-    }
+    return;
+  }
+  if (l_smem)
+    for (int64_t e = threadIdx.x; e < tri(t, 0); e += blockDim.x) Ls[e] = w.L[gbase + e];
+  for (int e = threadIdx.x; e < t * CW; e += blockDim.x) {
+    const int r = e / CW, c = c0 + e % CW;
+    X[e] = c < p.d ? w.AtY[(base + r) * p.d + c] : 0.0;
+  }
+  __syncthreads();
+  const int col = threadIdx.x / TPC, sub = threadIdx.x % TPC;
+  const unsigned gmask = (TPC == 32) ? 0xffffffffu : (((1u << TPC) - 1) << ((threadIdx.x & 31) / TPC * TPC));
+  // forward: y_k = (x_k − Σ_{j<k} L_kj y_j) / L_kk
+  for (int k = 0; k < t; ++k) {
+    const double* Lk = L + tri(k, 0);
+    double acc = 0.0;
+    for (int j = sub; j < k; j += TPC) acc += Lk[j] * X[j * CW + col];
+    for (int o = TPC / 2; o; o >>= 1) acc += __shfl_xor_sync(gmask, acc, o);
+    if (sub == 0) X[k * CW + col] = (X[k * CW + col] - acc) * invd[k];
+    __syncwarp(gmask);
+  }
+  // backward: z_k = (y_k − Σ_{j>k} L_jk z_j) / L_kk
+  for (int k = t - 1; k >= 0; --k) {
+    double acc = 0.0;
+    for (int j = k + 1 + sub; j < t; j += TPC) acc += L[tri(j, k)] * X[j * CW + col];
+    for (int o = TPC / 2; o; o >>= 1) acc += __shfl_xor_sync(gmask, acc, o);
+    if (sub == 0) X[k * CW + col] = (X[k * CW + col] - acc) * invd[k];
+    __syncwarp(gmask);
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < t * CW; e += blockDim.x) {
+    const int r = e / CW, c = c0 + e % CW;
+    if (c < p.d) C_v[(base + r) * p.d + c] = (float)X[e];
   }
 }
 
@@ -258,14 +290,28 @@ cudaError_t launch_value_fit(const Problem& p, const Work& w, float* C_v, cudaSt
   const int ta = (p.max_t + 31) / 32, td = (p.d + 31) / 32;
   dim3 gn(ta * (ta + 1) / 2 + ta * td, p.H);
   AM_LAUNCH(AM_STAGE_NORMAL, s, k_normal<<<gn, 256, 0, s>>>(p, w));
-  // heads with t <= tl keep the factor in shared memory, larger ones in the
-  // workspace; 1 KB is left for the kernel's static shared memory
+  // factor: heads with t <= tl keep it in shared memory while factoring
   const size_t cap = 226 * 1024;
   int tl = 0;
   while (tl < p.max_t && (size_t)(tl + 1) * (tl + 2) / 2 * sizeof(double) <= cap) ++tl;
   const size_t sm = (size_t)tl * (tl + 1) / 2 * sizeof(double);
-  cudaFuncSetAttribute(k_solve, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)cap);
-  AM_LAUNCH(AM_STAGE_SOLVE, s, k_solve<<<p.H, kCholThreads, sm, s>>>(p, w, C_v, tl));
+  cudaFuncSetAttribute(k_chol, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)cap);
+  AM_LAUNCH(AM_STAGE_SOLVE, s, k_chol<<<p.H, kCholThreads, sm, s>>>(p, w, tl));
+  // solves: a column slice of AᵀY plus (when it fits) the factor in shared memory
+  const bool wide = (size_t)p.max_t * 32 * 8 <= 120 * 1024;
+  const int CW = wide ? 32 : 8;
+  const size_t xbytes = (size_t)p.max_t * CW * 8;
+  int tl2 = 0;
+  while (tl2 < p.max_t && xbytes + (size_t)(tl2 + 1) * (tl2 + 2) / 2 * sizeof(double) <= cap) ++tl2;
+  const size_t sm2 = xbytes + (size_t)tl2 * (tl2 + 1) / 2 * sizeof(double);
+  dim3 g2(p.H, (p.d + CW - 1) / CW);
+  if (wide) {
+    cudaFuncSetAttribute(k_trsm<32>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)cap);
+    AM_LAUNCH(AM_STAGE_SOLVE, s, k_trsm<32><<<g2, 256, sm2, s>>>(p, w, C_v, tl2));
+  } else {
+    cudaFuncSetAttribute(k_trsm<8>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)cap);
+    AM_LAUNCH(AM_STAGE_SOLVE, s, k_trsm<8><<<g2, 256, sm2, s>>>(p, w, C_v, tl2));
+  }
   return cudaGetLastError();
 }
 

@@ -47,6 +47,8 @@ def parse_args():
                     choices=["qwen3_4b_layer", "single_head_fp32", "qwen3_4b_model"])
     ap.add_argument("--heads", type=int, default=None,
                     help="heads per GPU for the layer workload (default 8); smaller for profiling")
+    ap.add_argument("--corr-dtype", choices=["fp32", "bf16"], default="fp32",
+                    help="features streamed by the correlation pass")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     return ap.parse_args()
@@ -163,10 +165,10 @@ def cpu_baseline(wl, heads=1):
 
 
 # -------------------------------------------------------------- roofline ----
-def stage_models(wl, n, T, d, H, ldn, passes):
+def stage_models(wl, n, T, d, H, ldn, passes, corr_bytes=4):
     """Algorithmic bytes / flops of one launch of the main kernels."""
     return {
-        "corr": {"bound": "hbm", "bytes": H * (T * ldn * 4 + ldn * 4 + T * 4)},
+        "corr": {"bound": "hbm", "bytes": H * (T * ldn * corr_bytes + ldn * 4 + T * 4)},
         "phi": {"bound": "alu", "flops": 2.0 * H * n * T * d, "bytes": H * T * ldn * 4},
         "target": {"bound": "alu", "flops": 2.0 * H * n * T * d, "bytes": H * T * ldn * 4},
         "shift": {"bound": "alu", "flops": 2.0 * H * n * T * d},
@@ -265,8 +267,10 @@ def run_ours(args, rank, world, local_rank):
     Kh = torch.stack([h.K for h in wl.heads]).contiguous()
     Vh = torch.stack([h.V for h in wl.heads]).contiguous()
     Q, K, V = Qh.to(dev), Kh.to(dev), Vh.to(dev)
-    kw = dict(topk=wl.topk, refit_every=wl.refit_every)
-    opts = am.make_opts(am.BF16 if Q.dtype == torch.bfloat16 else am.FP32, wl.topk, wl.refit_every)
+    corr_dtype = am.BF16 if args.corr_dtype == "bf16" else am.FP32
+    kw = dict(topk=wl.topk, refit_every=wl.refit_every, corr_dtype=corr_dtype)
+    opts = am.make_opts(am.BF16 if Q.dtype == torch.bfloat16 else am.FP32, wl.topk, wl.refit_every,
+                        corr_dtype=corr_dtype)
     ws = torch.empty((am.workspace_size(n, T, d, wl.budgets, opts),), dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
     flush = torch.empty((256 << 20,), dtype=torch.uint8, device=dev)
@@ -344,13 +348,15 @@ def run_ours(args, rank, world, local_rank):
     ldn = (n + 31) // 32 * 32
     passes = max((t + wl.topk * wl.refit_every - 1) // (wl.topk * wl.refit_every) for t in wl.budgets)
     peaks = load_peaks()
-    rf = roofline(stages, args.steps, stage_models(wl, n, T, d, H, ldn, passes), peaks, clk,
-                  committed_traffic())
+    rf = roofline(stages, args.steps,
+                  stage_models(wl, n, T, d, H, ldn, passes, 2 if args.corr_dtype == "bf16" else 4),
+                  peaks, clk, committed_traffic() if args.corr_dtype == "fp32" else {})
     value = H * world / (ms * 1e-3)
     per_step_stage = {k: round(v["ms"] / args.steps, 4) for k, v in stages.items() if v["launches"]}
     cfg = {"workload": wl.name, "heads_per_gpu": H, "n": n, "T": T, "d": d,
            "budgets": wl.budgets if H <= 8 else f"{sum(wl.budgets)} total, min {min(wl.budgets)} max {max(wl.budgets)}",
-           "topk": wl.topk, "refit_every": wl.refit_every, "phi_storage": "fp32",
+           "topk": wl.topk, "refit_every": wl.refit_every,
+           "phi_storage": "fp32" + (" + bf16 copy for the correlation pass" if args.corr_dtype == "bf16" else ""),
            "l2": "256 MiB buffer written between timed steps",
            "stage_ms_per_step": per_step_stage, "device_status": worst}
     if args.workload == "qwen3_4b_layer":

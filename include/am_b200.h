@@ -69,7 +69,11 @@ typedef struct am_opts {
   float scale;             /* logit scale; <= 0 selects 1/sqrt(d)                */
   float ridge;             /* λ = ridge·tr(AᵀA)/t (default 1e-6); must be >= 0   */
   float w_floor_rel;       /* β floor: w >= w_floor_rel·max(w) (default 1e-12)   */
-  float reserved0;
+  int32_t corr_dtype;      /* features streamed by the correlation pass: AM_FP32
+                              (default) reads Φᵀ itself; AM_BF16 makes the feature
+                              pass also write a bf16 copy of Φᵀ, which the
+                              correlation pass reads at half the bytes (the mass,
+                              Gram, residual and value fit always use fp32 Φ)     */
   /* Optional device inputs */
   const float* shift;      /* [H] per-head shift c_h, or NULL: c_h = max_ij s_ij
                               computed on the device                              */
@@ -84,7 +88,8 @@ typedef struct am_opts {
 } am_opts_t;
 
 /* Fill *opts with defaults: bf16 inputs, k = 1, R = 1, scale = 1/sqrt(d),
- * ridge = 1e-6, w_floor_rel = 1e-12, every optional pointer NULL. */
+ * ridge = 1e-6, w_floor_rel = 1e-12, corr_dtype = AM_FP32, every optional
+ * pointer NULL. */
 am_status_t am_default_opts(am_opts_t* opts);
 
 /* Device workspace needed by am_compact_heads for this problem.
@@ -94,7 +99,8 @@ am_status_t am_default_opts(am_opts_t* opts);
  *   budgets          host int32 [H], 1 <= t_h <= T
  *   opts             as passed to am_compact_heads
  *   bytes            host out
- * The dominant term is H·T·round_up(n, 32)·4 bytes of stored features. */
+ * The dominant term is H·T·round_up(n, 32)·4 bytes of stored features
+ * (·6 with corr_dtype = AM_BF16). */
 am_status_t am_workspace_size(int32_t n, int32_t T, int32_t d, int32_t num_heads,
                               const int32_t* budgets, const am_opts_t* opts,
                               size_t* bytes);

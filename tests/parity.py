@@ -46,8 +46,13 @@ def split_head(out, h):
     return res
 
 
-def check_head(g, Q, K, V, t, topk, refit, shift, key_bias=None, oracle_res=None, label=""):
-    """Run every acceptance rule for one head; returns a dict of measurements."""
+def check_head(g, Q, K, V, t, topk, refit, shift, key_bias=None, oracle_res=None, label="",
+               exact_picks=True):
+    """Run every acceptance rule for one head; returns a dict of measurements.
+
+    ``exact_picks=False`` is for approximate correlation modes (bf16 feature
+    copy): picks are then only reported, and the remaining rules (residual,
+    β against the oracle on the GPU's own picks, output) still apply."""
     if oracle_res is None:
         oracle_res = O.compact_head(Q, K, V, t, topk, refit, shift=shift, key_bias=key_bias)
     o = oracle_res
@@ -68,7 +73,8 @@ def check_head(g, Q, K, V, t, topk, refit, shift, key_bias=None, oracle_res=None
                 continue
             slack = (rec["c_kth"] - rec["c"][j]) / scale
             worst_slack = max(worst_slack, slack)
-            assert slack <= GAP_TOL, f"{label}: pick {j} in round {rec['round']} trails by {slack:.3g}"
+            if exact_picks:
+                assert slack <= GAP_TOL, f"{label}: pick {j} in round {rec['round']} trails by {slack:.3g}"
     rep["pick_slack"] = worst_slack
 
     gaps = [(r["c_kth"] - r["c_next"]) / max(abs(r["c_max"]), 1e-300)
@@ -76,7 +82,7 @@ def check_head(g, Q, K, V, t, topk, refit, shift, key_bias=None, oracle_res=None
     rep["min_gap"] = min(gaps) if gaps else math.inf
     same = np.array_equal(idx, o["indices"])
     rep["same_set"] = bool(same)
-    if rep["min_gap"] > GAP_TOL:
+    if rep["min_gap"] > GAP_TOL and exact_picks:
         assert same, f"{label}: index sets differ although every gap > {GAP_TOL}"
 
     Phi, m, _ = O.mass_features(Q, K, shift, key_bias=key_bias)
