@@ -15,9 +15,11 @@ from typing import Dict, Optional, Sequence
 
 __all__ = ["AmError", "AmOpts", "lib", "library_path", "workspace_size", "compact_heads",
            "get_status", "profile_enable", "profile_collect", "kernel_launches", "STAGES",
-           "STATUS", "BF16", "FP32"]
+           "STATUS", "BF16", "FP32", "CORR_AUTO", "CORR_STORED_FP32", "CORR_STORED_BF16",
+           "CORR_RECOMPUTE"]
 
 BF16, FP32 = 0, 1
+CORR_AUTO, CORR_STORED_FP32, CORR_STORED_BF16, CORR_RECOMPUTE = 0, 1, 2, 3
 STATUS = {
     0: "AM_OK", 1: "AM_ERR_INVALID_ARG", 2: "AM_ERR_BUDGET", 3: "AM_ERR_WORKSPACE",
     4: "AM_ERR_NONFINITE", 5: "AM_ERR_CUDA", 6: "AM_ERR_TIMEOUT", 7: "AM_ERR_UNSUPPORTED",
@@ -53,7 +55,7 @@ class AmOpts(ctypes.Structure):
         ("scale", ctypes.c_float),
         ("ridge", ctypes.c_float),
         ("w_floor_rel", ctypes.c_float),
-        ("corr_dtype", ctypes.c_int32),
+        ("corr_mode", ctypes.c_int32),
         ("shift", ctypes.c_void_p),
         ("key_bias", ctypes.c_void_p),
         ("pick_order", ctypes.c_void_p),
@@ -112,14 +114,14 @@ def _i32_array(vals: Sequence[int]):
 
 def make_opts(dtype: int = BF16, topk: int = 1, refit_every: int = 1, scale: float = 0.0,
               ridge: float = 1e-6, w_floor_rel: float = 1e-12, nnls_max_iter: int = 0,
-              corr_dtype: int = FP32) -> AmOpts:
+              corr_mode: int = CORR_AUTO) -> AmOpts:
     o = AmOpts()
     rc = lib().am_default_opts(ctypes.byref(o))
     if rc:
         raise AmError(rc, "am_default_opts")
     o.in_dtype, o.topk, o.refit_every, o.nnls_max_iter = dtype, topk, refit_every, nnls_max_iter
     o.scale, o.ridge, o.w_floor_rel = scale, ridge, w_floor_rel
-    o.corr_dtype = corr_dtype
+    o.corr_mode = corr_mode
     return o
 
 
@@ -166,7 +168,7 @@ def _ptr(t) -> Optional[int]:
 def compact_heads(Q, K, V, budgets: Sequence[int], topk: int = 1, refit_every: int = 1,
                   shift=None, key_bias=None, ridge: float = 1e-6, w_floor_rel: float = 1e-12,
                   scale: float = 0.0, nnls_max_iter: int = 0, workspace=None, trace: bool = False,
-                  stream=None, check: bool = True, corr_dtype: int = FP32) -> Dict:
+                  stream=None, check: bool = True, corr_mode: int = CORR_AUTO) -> Dict:
     """Compact H heads on the GPU.
 
     Q [H, n, d], K [H, T, d], V [H, T, d]: contiguous tensors, bf16 or fp32,
@@ -196,7 +198,7 @@ def compact_heads(Q, K, V, budgets: Sequence[int], topk: int = 1, refit_every: i
             raise ValueError("inputs must be contiguous")
     dt = BF16 if Q.dtype == torch.bfloat16 else FP32
     dev = Q.device
-    opts = make_opts(dt, topk, refit_every, scale, ridge, w_floor_rel, nnls_max_iter, corr_dtype)
+    opts = make_opts(dt, topk, refit_every, scale, ridge, w_floor_rel, nnls_max_iter, corr_mode)
     if shift is not None:
         shift = shift.to(device=dev, dtype=torch.float32).contiguous()
         opts.shift = shift.data_ptr()

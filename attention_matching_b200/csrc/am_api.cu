@@ -26,7 +26,7 @@ struct Layout {
   size_t phiT, phiT16, m, Y, r, corr, sel;
   size_t picks, pick_corr, plist, sorted_slot;
   size_t bvec, w, w_eff;
-  size_t G, L, AtA, A, AtY;
+  size_t G, L, AtA, A, AtY, nrm_part;
   size_t total;
   size_t tables_bytes;
 };
@@ -71,6 +71,7 @@ Layout plan(int n, int T, int d, int H, int64_t sum_t, int64_t sum_t2, bool corr
   L.AtA = take((size_t)sum_t2 * 8);
   L.A = take((size_t)sum_t * ldn * 4);
   L.AtY = take((size_t)sum_t * d * 8);
+  L.nrm_part = take((size_t)kNormalMaxSplits * ((size_t)sum_t2 + (size_t)sum_t * d) * 8);
   L.total = o;
   return L;
 }
@@ -87,7 +88,9 @@ am_status_t check_shape(int n, int T, int d, int H, const int32_t* budgets, cons
   if (!(opts->ridge >= 0.f) || !isfinite(opts->ridge)) return AM_ERR_INVALID_ARG;
   if (!(opts->w_floor_rel > 0.f) || !(opts->w_floor_rel < 1.f)) return AM_ERR_INVALID_ARG;
   if (!isfinite(opts->scale)) return AM_ERR_INVALID_ARG;
-  if (opts->corr_dtype != AM_FP32 && opts->corr_dtype != AM_BF16) return AM_ERR_INVALID_ARG;
+  if (opts->corr_mode < AM_CORR_AUTO || opts->corr_mode > AM_CORR_RECOMPUTE) return AM_ERR_INVALID_ARG;
+  if (opts->corr_mode == AM_CORR_RECOMPUTE && !(opts->in_dtype == AM_BF16 && (d == 64 || d == 128)))
+    return AM_ERR_UNSUPPORTED;
   if ((int64_t)n * d > (1ll << 31) || (int64_t)T * round_up(n, 32) > (1ll << 40))
     return AM_ERR_UNSUPPORTED;
   const int kR = opts->topk * opts->refit_every;
@@ -142,6 +145,7 @@ Work bind(const Layout& L, char* base, bool corr_bf16) {
   w.AtA = reinterpret_cast<double*>(base + L.AtA);
   w.A = reinterpret_cast<float*>(base + L.A);
   w.AtY = reinterpret_cast<double*>(base + L.AtY);
+  w.nrm_part = reinterpret_cast<double*>(base + L.nrm_part);
   return w;
 }
 
@@ -174,7 +178,9 @@ Problem make_problem(int n, int T, int d, int H, const am_opts_t* o, const Table
   p.w_floor_rel = o->w_floor_rel;
   p.max_t = tb.max_t;
   p.has_bias = o->key_bias != nullptr;
-  p.corr_bf16 = o->corr_dtype == AM_BF16;
+  p.corr_bf16 = o->corr_mode == AM_CORR_STORED_BF16;
+  const bool tc = o->in_dtype == AM_BF16 && (d == 64 || d == 128);
+  p.corr_recompute = o->corr_mode == AM_CORR_RECOMPUTE || (o->corr_mode == AM_CORR_AUTO && tc);
   return p;
 }
 
@@ -199,7 +205,7 @@ am_status_t am_default_opts(am_opts_t* opts) {
   opts->scale = 0.f;
   opts->ridge = 1e-6f;
   opts->w_floor_rel = 1e-12f;
-  opts->corr_dtype = AM_FP32;
+  opts->corr_mode = AM_CORR_AUTO;
   return AM_OK;
 }
 
@@ -209,7 +215,7 @@ am_status_t am_workspace_size(int32_t n, int32_t T, int32_t d, int32_t num_heads
   Tables tb;
   am_status_t st = check_shape(n, T, d, num_heads, budgets, opts, &tb);
   if (st != AM_OK) return st;
-  *bytes = plan(n, T, d, num_heads, tb.sum_t, tb.sum_t2, opts->corr_dtype == AM_BF16).total;
+  *bytes = plan(n, T, d, num_heads, tb.sum_t, tb.sum_t2, opts->corr_mode == AM_CORR_STORED_BF16).total;
   return AM_OK;
 }
 
@@ -219,7 +225,7 @@ am_status_t am_workspace_view(int32_t n, int32_t T, int32_t d, int32_t num_heads
   Tables tb;
   am_status_t st = check_shape(n, T, d, num_heads, budgets, opts, &tb);
   if (st != AM_OK) return st;
-  const Layout L = plan(n, T, d, num_heads, tb.sum_t, tb.sum_t2, opts->corr_dtype == AM_BF16);
+  const Layout L = plan(n, T, d, num_heads, tb.sum_t, tb.sum_t2, opts->corr_mode == AM_CORR_STORED_BF16);
   view->phiT = L.phiT;
   view->mass = L.m;
   view->target = L.Y;
@@ -240,12 +246,14 @@ am_status_t am_compact_heads(const void* Q, const void* K, const void* V, int32_
   for (int h = 0; h <= H; ++h)
     if (out_offsets[h] != tb.cu_t[h]) return AM_ERR_INVALID_ARG;
   if (!workspace || ((uintptr_t)workspace % kAlign) != 0) return AM_ERR_WORKSPACE;
-  const Layout L = plan(n, T, d, H, tb.sum_t, tb.sum_t2, opts->corr_dtype == AM_BF16);
+  const Layout L = plan(n, T, d, H, tb.sum_t, tb.sum_t2, opts->corr_mode == AM_CORR_STORED_BF16);
   if (workspace_bytes < L.total) return AM_ERR_WORKSPACE;
 
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   char* base = reinterpret_cast<char*>(workspace);
-  Work w = bind(L, base, opts->corr_dtype == AM_BF16);
+  Work w = bind(L, base, opts->corr_mode == AM_CORR_STORED_BF16);
+  w.nrm_ata = tb.sum_t2;
+  w.nrm_stride = tb.sum_t2 + tb.sum_t * d;
   std::vector<unsigned char> host_tables;
   pack_tables(tb, H, &host_tables, &w, base + L.tables);
   const Problem p = make_problem(n, T, d, H, opts, tb);
@@ -279,7 +287,7 @@ am_status_t am_compact_heads(const void* Q, const void* K, const void* V, int32_
   }
   AM_TRY(launch_omp_init(p, w, s));
   for (int pass = 0; pass < (int)tb.active.size(); ++pass)
-    AM_TRY(launch_omp_pass(p, w, pass, tb.active[pass], s));
+    AM_TRY(launch_omp_pass(p, w, pass, tb.active[pass], CorrInputs{Q, K, opts->key_bias}, s));
   if (opts->residual_out) AM_TRY(launch_residual_norm(p, w, opts->residual_out, s));
   AM_TRY(launch_finalize(p, w, K, opts->key_bias, C_k, beta, indices, opts->w_out, opts->pick_order,
                          opts->pick_corr, s));

@@ -28,6 +28,7 @@ struct Problem {
   int max_t;          // max_h t_h
   int has_bias;
   int corr_bf16;      // the correlation pass streams a bf16 copy of Φᵀ
+  int corr_recompute; // the correlation pass recomputes Φ on the tensor cores
 };
 
 // Device pointers into the caller's workspace (see plan_workspace()).
@@ -60,9 +61,13 @@ struct Work {
   float* A;             // [Σt][ldn] design matrix, key-major
   double* AtA;          // [Σt²]
   double* AtY;          // [Σt][d]
+  double* nrm_part;     // [kNormalMaxSplits][Σt² + Σt·d] split partials of AᵀA, AᵀY
+  int64_t nrm_ata;      // Σt²
+  int64_t nrm_stride;   // Σt² + Σt·d
 };
 
 constexpr int kRedBlocks = 64;   // partial-sum slots per head for ‖r‖²
+constexpr int kNormalMaxSplits = 8;   // query splits of the normal-equation products
 
 // ---- launchers (each file defines its own) ----
 // feature pass (am_phi_simt.cu)
@@ -80,10 +85,18 @@ cudaError_t launch_shift_max_tc(const Problem& p, const void* Q, const void* K, 
                                 const Work& w, uint32_t* shift_ord, cudaStream_t s);
 cudaError_t launch_phi_tc(const Problem& p, const void* Q, const void* K, const void* V, const float* key_bias,
                           const Work& w, cudaStream_t s);
+cudaError_t launch_corr_tc(const Problem& p, const void* Q, const void* K, const float* key_bias, const Work& w,
+                           int pass, int active, cudaStream_t s);
 // OMP engine (am_omp.cu)
 cudaError_t launch_omp_init(const Problem& p, const Work& w, cudaStream_t s);
+// inputs the recomputing correlation pass needs
+struct CorrInputs {
+  const void* Q;
+  const void* K;
+  const float* key_bias;
+};
 cudaError_t launch_omp_pass(const Problem& p, const Work& w, int pass, int active_heads,
-                            cudaStream_t s);
+                            const CorrInputs& in, cudaStream_t s);
 cudaError_t launch_residual_norm(const Problem& p, const Work& w, double* residual_out,
                                  cudaStream_t s);
 // value fit and packing (am_valfit.cu)

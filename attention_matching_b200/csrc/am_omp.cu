@@ -718,10 +718,16 @@ cudaError_t launch_omp_init(const Problem& p, const Work& w, cudaStream_t s) {
   return cudaGetLastError();
 }
 
-cudaError_t launch_omp_pass(const Problem& p, const Work& w, int pass, int active, cudaStream_t s) {
+cudaError_t launch_omp_pass(const Problem& p, const Work& w, int pass, int active, const CorrInputs& in,
+                            cudaStream_t s) {
   if (active <= 0) return cudaSuccess;
-  dim3 gc((p.T + kCorrRowsPerBlock - 1) / kCorrRowsPerBlock, active);
-  AM_LAUNCH(AM_STAGE_CORR, s, k_corr<<<gc, 256, 0, s>>>(p, w, pass));
+  if (p.corr_recompute) {
+    cudaError_t e = launch_corr_tc(p, in.Q, in.K, in.key_bias, w, pass, active, s);
+    if (e != cudaSuccess) return e;
+  } else {
+    dim3 gc((p.T + kCorrRowsPerBlock - 1) / kCorrRowsPerBlock, active);
+    AM_LAUNCH(AM_STAGE_CORR, s, k_corr<<<gc, 256, 0, s>>>(p, w, pass));
+  }
   AM_LAUNCH(AM_STAGE_SELECT, s, k_select<<<active, 1024, 0, s>>>(p, w, pass));
   const int s1max = (pass + 1) * p.kR < p.max_t ? (pass + 1) * p.kR : p.max_t;
   dim3 gg(s1max, active);

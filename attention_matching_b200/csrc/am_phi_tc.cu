@@ -474,6 +474,162 @@ k_phi_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtens
   if (warp == 2) asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols));
 }
 
+// ---------------------------------------------------------------------------
+// Correlation by recomputation: c_j = Σ_i r_i exp(s_ij·scale + b_j − c_h) for
+// a block of 128 keys, with Φ recomputed from Q and K on the tensor cores
+// instead of re-read from HBM (the OMP correlation step, zhichai.net deep
+// dive §1.6: j* = argmax rᵀΦ_{:,j}).  Keys sit on the TMEM lanes (M = 128),
+// query tiles of 64 stream through a 4-stage ring (N = 64); two epilogue
+// warpgroups each fold 32 queries of every tile into their key's sum.
+constexpr int CQ = 64;          // queries per tile
+constexpr int CSTAGES = 4;
+
+__host__ __device__ inline uint32_t corr_smem_bytes(int d) {
+  return (uint32_t)(BM * d * 2 + CSTAGES * CQ * d * 2 + 2 * CQ * 4 + 32 * 8 + 1024);
+}
+
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1)
+k_corr_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK, Problem p, Work w,
+          const float* __restrict__ key_bias, int pass) {
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  constexpr int KB = D / 64;
+  const int hslot = blockIdx.y;
+  const int h = w.order[hslot];
+  if (pass * p.kR >= w.t[h]) return;          // head already finished (whole CTA leaves)
+  unsigned char* sm = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t k_bytes = BM * D * 2, q_bytes = CQ * D * 2;
+  unsigned char* sK = sm;
+  unsigned char* sQ = sm + k_bytes;
+  float* sR = reinterpret_cast<float*>(sQ + CSTAGES * q_bytes);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sR + 2 * CQ);
+  uint64_t* k_full = bars + 0;
+  uint64_t* q_full = bars + 1;                  // [CSTAGES]
+  uint64_t* q_empty = bars + 1 + CSTAGES;       // [CSTAGES]
+  uint64_t* s_full = bars + 1 + 2 * CSTAGES;    // [2]
+  uint64_t* s_empty = s_full + 2;               // [2]
+  uint64_t* drain = s_full + 4;
+  __shared__ uint32_t s_tmem;
+  __shared__ int s_abort;
+  __shared__ int s_stop[2];
+  __shared__ float s_part[128];
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int j0 = blockIdx.x * BM;
+  const int NQ = (p.n + CQ - 1) / CQ;
+  int32_t* status = w.status + h;
+  volatile int* abort_flag = &s_abort;
+
+  if (threadIdx.x == 0) {
+    s_abort = 0;
+    mbar_init(k_full, 1);
+    for (int s = 0; s < CSTAGES; ++s) { mbar_init(q_full + s, 1); mbar_init(q_empty + s, 1); }
+    for (int b = 0; b < 2; ++b) { mbar_init(s_full + b, 1); mbar_init(s_empty + b, 256); }
+    mbar_init(drain, 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 2) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(&s_tmem)),
+                 "r"(128));
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = s_tmem;
+  const uint32_t tS[2] = {tmem, tmem + CQ};
+
+  if (warp == 0) {
+    if (lane == 0) {
+      mbar_expect_tx(k_full, k_bytes);
+      for (int kb = 0; kb < KB; ++kb) tma_load_3d(sK + kb * BM * 128, &tmK, k_full, kb * 64, j0, h);
+      int issued[CSTAGES] = {};
+      for (int j = 0; j < NQ; ++j) {
+        const int s = j % CSTAGES, use = j / CSTAGES;
+        if (use > 0 && !mbar_wait(q_empty + s, (use - 1) & 1, abort_flag, status)) break;
+        mbar_expect_tx(q_full + s, q_bytes);
+        for (int kb = 0; kb < KB; ++kb)
+          tma_load_3d(sQ + s * q_bytes + kb * CQ * 128, &tmQ, q_full + s, kb * 64, j * CQ, h);
+        issued[s] = use + 1;
+      }
+      mbar_wait(k_full, 0, abort_flag, status);
+      for (int s = 0; s < CSTAGES; ++s)
+        if (issued[s] > 0) {
+          const long long t0 = clock64();
+          while (!mbar_try_wait(q_full + s, (issued[s] - 1) & 1) && clock64() - t0 < kWaitBudgetCycles) {}
+        }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      const uint32_t idesc = instr_desc(CQ, false);
+      bool ok = mbar_wait(k_full, 0, abort_flag, status);
+      tc_fence_after();
+      for (int j = 0; ok && j < NQ; ++j) {
+        const int s = j % CSTAGES, use = j / CSTAGES, b = j & 1, bu = j >> 1;
+        if (!mbar_wait(q_full + s, use & 1, abort_flag, status)) break;
+        if (bu > 0 && !mbar_wait(s_empty + b, (bu - 1) & 1, abort_flag, status)) break;
+        tc_fence_after();
+        const uint32_t kbase = smem_u32(sK), qbase = smem_u32(sQ + s * q_bytes);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t kblk = kk >> 2;
+          const uint64_t ad = smem_desc(kbase + kblk * BM * 128 + (kk & 3) * 32, 16, 1024);
+          const uint64_t bd = smem_desc(qbase + kblk * CQ * 128 + (kk & 3) * 32, 16, 1024);
+          tc_mma(tS[b], ad, bd, idesc, kk > 0 ? 1u : 0u);
+        }
+        tc_commit(s_full + b);
+        tc_commit(q_empty + s);
+      }
+      tc_commit(drain);
+      const long long t0 = clock64();
+      while (!mbar_try_wait(drain, 0) && clock64() - t0 < kWaitBudgetCycles) {}
+    }
+  } else if (warp >= kEpiWarp0) {
+    const int ep = threadIdx.x - kEpiWarp0 * 32;
+    const int half = ep >> 7;
+    const int et = ep & 127;
+    const int qd = warp & 3;
+    constexpr int HC = CQ / 2;
+    const int j = j0 + et;                       // this thread's key
+    const bool key_live = j < p.T;
+    const float kLog2e = 1.4426950408889634f;
+    const float scale = p.scale * kLog2e;
+    const float c = w.shift[h];
+    const float bj = (p.has_bias && key_live) ? key_bias[(int64_t)h * p.T + j] : 0.f;
+    const float bias2 = (bj - c) * kLog2e;
+    const float* rh = w.r + (int64_t)h * p.ldn;
+    const uint32_t lane_addr = (uint32_t)(qd * 32) << 16;
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+    for (int t = 0; t < NQ; ++t) {
+      const int b = t & 1, bu = t >> 1;
+      if (ep == 0) s_stop[b] = mbar_wait(s_full + b, bu & 1, abort_flag, status) ? 0 : 1;
+      if (ep < CQ) {   // this tile's residual entries (zero past n)
+        const int q = t * CQ + ep;
+        sR[b * CQ + ep] = q < p.n ? rh[q] : 0.f;
+      }
+      asm volatile("bar.sync 1, 256;" ::: "memory");
+      if (s_stop[b]) break;
+      tc_fence_after();
+      float v[HC];
+      tmem_ld32(tS[b] + lane_addr + half * HC, v);
+      tmem_wait_ld();
+      tc_fence_before();
+      mbar_arrive(s_empty + b);
+      const float* rr = sR + b * CQ + half * HC;
+#pragma unroll
+      for (int cc = 0; cc < HC; ++cc) acc[cc & 3] = fmaf(exp2f(fmaf(v[cc], scale, bias2)), rr[cc], acc[cc & 3]);
+    }
+    const float mine = (acc[0] + acc[1]) + (acc[2] + acc[3]);
+    if (half == 1) s_part[et] = mine;
+    asm volatile("bar.sync 1, 256;" ::: "memory");
+    if (half == 0 && key_live && !s_abort) w.corr[(int64_t)h * p.T + j] = mine + s_part[et];
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 2) asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(128));
+}
+
 // ---- host: tensor maps ----
 PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
   static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
@@ -518,7 +674,27 @@ cudaError_t launch_tc(const Problem& p, const void* Q, const void* K, const void
   return cudaGetLastError();
 }
 
+template <int D>
+cudaError_t launch_corr_tc_d(const Problem& p, const void* Q, const void* K, const float* key_bias, const Work& w,
+                             int pass, int active, cudaStream_t s) {
+  CUtensorMap mq, mk;
+  if (!make_map(&mq, Q, p.H, p.n, D, CQ) || !make_map(&mk, K, p.H, p.T, D, BM)) return cudaErrorInvalidValue;
+  const uint32_t bytes = corr_smem_bytes(D);
+  auto kern = k_corr_tc<D>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+  if (e != cudaSuccess) return e;
+  dim3 grid((p.T + BM - 1) / BM, active);
+  AM_LAUNCH(AM_STAGE_CORR, s, kern<<<grid, kThreads, bytes, s>>>(mq, mk, p, w, key_bias, pass));
+  return cudaGetLastError();
+}
+
 }  // namespace
+
+cudaError_t launch_corr_tc(const Problem& p, const void* Q, const void* K, const float* key_bias, const Work& w,
+                           int pass, int active, cudaStream_t s) {
+  return p.d == 64 ? launch_corr_tc_d<64>(p, Q, K, key_bias, w, pass, active, s)
+                   : launch_corr_tc_d<128>(p, Q, K, key_bias, w, pass, active, s);
+}
 
 bool phi_tc_supported(const Problem& p) { return p.in_dtype == AM_BF16 && (p.d == 64 || p.d == 128); }
 

@@ -115,16 +115,24 @@ __global__ void __launch_bounds__(kDesignThreads) k_design(Problem p, Work w) {
   }
 }
 
-// AᵀA (upper tile triangle, mirrored) and AᵀY; one 32×32 output tile per block.
-__global__ void __launch_bounds__(256) k_normal(Problem p, Work w) {
+// AᵀA (upper tile triangle, mirrored) and AᵀY; one 64×64 output tile per
+// block, 4×4 outputs per thread.  Operand tiles are converted to fp64 once,
+// when staged in shared memory, so the inner loop is pure fp64 FMA.
+constexpr int NT_ = 64;   // output tile edge
+constexpr int NK_ = 16;   // query chunk
+
+__global__ void __launch_bounds__(256) k_normal(Problem p, Work w, int splits, int64_t part_stride) {
   const int h = blockIdx.y;
+  const int z = blockIdx.z;   // query split: rows [i_begin, i_end)
+  const int chunk = ((p.n + splits - 1) / splits + NK_ - 1) / NK_ * NK_;
+  const int i_begin = z * chunk, i_end = min(p.n, i_begin + chunk);
   const int t = w.t[h];
-  const int ta = (t + 31) / 32, td = (p.d + 31) / 32;
+  const int ta = (t + NT_ - 1) / NT_, td = (p.d + NT_ - 1) / NT_;
   const int ntri = ta * (ta + 1) / 2;
   int tile = blockIdx.x;
   if (tile >= ntri + ta * td) return;
-  bool gram = tile < ntri;
-  int ta0, tb0;   // tile row/col
+  const bool gram = tile < ntri;
+  int ta0, tb0;
   if (gram) {
     int r = 0;
     while (tile >= ta - r) { tile -= ta - r; ++r; }
@@ -135,55 +143,72 @@ __global__ void __launch_bounds__(256) k_normal(Problem p, Work w) {
     ta0 = tile / td;
     tb0 = tile % td;
   }
-  const int a0 = ta0 * 32, b0 = tb0 * 32;
+  const int a0 = ta0 * NT_, b0 = tb0 * NT_;
   const int64_t base = w.cu_t[h];
-  __shared__ float As[32][33];
-  __shared__ float Bs[32][33];
+  __shared__ double As[NK_][NT_ + 1];
+  __shared__ double Bs[NK_][NT_ + 1];
   const int tx = threadIdx.x % 16, ty = threadIdx.x / 16;
-  double acc[2][2] = {{0.0, 0.0}, {0.0, 0.0}};
+  double acc[4][4] = {};
   const float* Yh = w.Y + (int64_t)h * p.n * p.d;
-  for (int i0 = 0; i0 < p.n; i0 += 32) {
+  for (int i0 = i_begin; i0 < i_end; i0 += NK_) {
     __syncthreads();
-    for (int e = threadIdx.x; e < 32 * 32; e += blockDim.x) {
-      const int rr = e / 32, ii = e % 32;
+    for (int e = threadIdx.x; e < NK_ * NT_; e += blockDim.x) {
+      const int rr = e / NK_, ii = e % NK_;          // A rows are contiguous along queries
       const int a = a0 + rr, i = i0 + ii;
-      As[ii][rr] = (a < t && i < p.n) ? w.A[(base + a) * p.ldn + i] : 0.f;
+      As[ii][rr] = (a < t && i < i_end) ? (double)w.A[(base + a) * p.ldn + i] : 0.0;
       if (gram) {
-        const int b = b0 + rr;
-        Bs[ii][rr] = (b < t && i < p.n) ? w.A[(base + b) * p.ldn + i] : 0.f;
+        const int bb = b0 + rr;
+        Bs[ii][rr] = (bb < t && i < i_end) ? (double)w.A[(base + bb) * p.ldn + i] : 0.0;
       }
     }
     if (!gram) {
-      for (int e = threadIdx.x; e < 32 * 32; e += blockDim.x) {
-        const int ii = e / 32, cc = e % 32;
+      for (int e = threadIdx.x; e < NK_ * NT_; e += blockDim.x) {
+        const int ii = e / NT_, cc = e % NT_;          // Y rows are contiguous along dims
         const int i = i0 + ii, c = b0 + cc;
-        Bs[ii][cc] = (i < p.n && c < p.d) ? Yh[(int64_t)i * p.d + c] : 0.f;
+        Bs[ii][cc] = (i < i_end && c < p.d) ? (double)Yh[(int64_t)i * p.d + c] : 0.0;
       }
     }
     __syncthreads();
-#pragma unroll 8
-    for (int ii = 0; ii < 32; ++ii) {
-      const double x0 = As[ii][ty * 2], x1 = As[ii][ty * 2 + 1];
-      const double y0 = Bs[ii][tx * 2], y1 = Bs[ii][tx * 2 + 1];
-      acc[0][0] += x0 * y0; acc[0][1] += x0 * y1;
-      acc[1][0] += x1 * y0; acc[1][1] += x1 * y1;
+#pragma unroll 4
+    for (int ii = 0; ii < NK_; ++ii) {
+      double x[4], y[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) { x[u] = As[ii][ty + 16 * u]; y[u] = Bs[ii][tx + 16 * u]; }
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+#pragma unroll
+        for (int v = 0; v < 4; ++v) acc[u][v] = fma(x[u], y[v], acc[u][v]);
     }
   }
+  // one split writes AᵀA / AᵀY directly; several write partials (reduced in order below)
+  double* AtA = splits == 1 ? w.AtA : w.nrm_part + z * part_stride;
+  double* AtY = splits == 1 ? w.AtY : w.nrm_part + z * part_stride + w.cu_t2[p.H];
   const int64_t gbase = w.cu_t2[h];
 #pragma unroll
-  for (int u = 0; u < 2; ++u)
+  for (int u = 0; u < 4; ++u)
 #pragma unroll
-    for (int v = 0; v < 2; ++v) {
-      const int a = a0 + ty * 2 + u, b = b0 + tx * 2 + v;
+    for (int v = 0; v < 4; ++v) {
+      const int a = a0 + ty + 16 * u, bb = b0 + tx + 16 * v;
       if (gram) {
-        if (a < t && b < t) {
-          w.AtA[gbase + (int64_t)a * t + b] = acc[u][v];
-          w.AtA[gbase + (int64_t)b * t + a] = acc[u][v];
+        if (a < t && bb < t) {
+          AtA[gbase + (int64_t)a * t + bb] = acc[u][v];
+          AtA[gbase + (int64_t)bb * t + a] = acc[u][v];
         }
-      } else if (a < t && b < p.d) {
-        w.AtY[(base + a) * p.d + b] = acc[u][v];
+      } else if (a < t && bb < p.d) {
+        AtY[(base + a) * p.d + bb] = acc[u][v];
       }
     }
+}
+
+// AᵀA and AᵀY = Σ over the query splits, added in split order.
+__global__ void k_normal_reduce(int64_t n_ata, int64_t n_aty, int splits, int64_t part_stride, Work w) {
+  const int64_t total = n_ata + n_aty;
+  for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < total; e += (int64_t)gridDim.x * blockDim.x) {
+    double acc = 0.0;
+    for (int z = 0; z < splits; ++z) acc += w.nrm_part[z * part_stride + e];
+    if (e < n_ata) w.AtA[e] = acc;
+    else w.AtY[e - n_ata] = acc;
+  }
 }
 
 // λ = ridge·tr(AᵀA)/t; packed Cholesky factor of AᵀA + λI and its
@@ -287,9 +312,17 @@ cudaError_t launch_finalize(const Problem& p, const Work& w, const void* K, cons
 cudaError_t launch_value_fit(const Problem& p, const Work& w, float* C_v, cudaStream_t s) {
   dim3 gd((p.ldn + kDesignThreads - 1) / kDesignThreads, p.H);
   AM_LAUNCH(AM_STAGE_DESIGN, s, k_design<<<gd, kDesignThreads, 0, s>>>(p, w));
-  const int ta = (p.max_t + 31) / 32, td = (p.d + 31) / 32;
-  dim3 gn(ta * (ta + 1) / 2 + ta * td, p.H);
-  AM_LAUNCH(AM_STAGE_NORMAL, s, k_normal<<<gn, 256, 0, s>>>(p, w));
+  const int ta = (p.max_t + NT_ - 1) / NT_, td = (p.d + NT_ - 1) / NT_;
+  const int blocks = (ta * (ta + 1) / 2 + ta * td) * p.H;
+  int splits = (2 * 148 + blocks - 1) / blocks;
+  splits = splits < 1 ? 1 : (splits > kNormalMaxSplits ? kNormalMaxSplits : splits);
+  if (splits > (p.n + NK_ - 1) / NK_) splits = (p.n + NK_ - 1) / NK_;
+  const int64_t part_stride = w.nrm_stride;
+  dim3 gn(ta * (ta + 1) / 2 + ta * td, p.H, splits);
+  AM_LAUNCH(AM_STAGE_NORMAL, s, k_normal<<<gn, 256, 0, s>>>(p, w, splits, part_stride));
+  if (splits > 1)
+    AM_LAUNCH(AM_STAGE_NORMAL, s,
+              k_normal_reduce<<<296, 256, 0, s>>>(w.nrm_ata, w.nrm_stride - w.nrm_ata, splits, part_stride, w));
   // factor: heads with t <= tl keep it in shared memory while factoring
   const size_t cap = 226 * 1024;
   int tl = 0;

@@ -47,8 +47,8 @@ def parse_args():
                     choices=["qwen3_4b_layer", "single_head_fp32", "qwen3_4b_model"])
     ap.add_argument("--heads", type=int, default=None,
                     help="heads per GPU for the layer workload (default 8); smaller for profiling")
-    ap.add_argument("--corr-dtype", choices=["fp32", "bf16"], default="fp32",
-                    help="features streamed by the correlation pass")
+    ap.add_argument("--corr", choices=["auto", "fp32", "bf16", "recompute"], default="auto",
+                    help="correlation pass: stored fp32 / stored bf16 copy / tensor-core recompute")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     return ap.parse_args()
@@ -165,10 +165,14 @@ def cpu_baseline(wl, heads=1):
 
 
 # -------------------------------------------------------------- roofline ----
-def stage_models(wl, n, T, d, H, ldn, passes, corr_bytes=4):
+def stage_models(wl, n, T, d, H, ldn, passes, corr_kind="fp32"):
     """Algorithmic bytes / flops of one launch of the main kernels."""
+    if corr_kind == "recompute":
+        corr = {"bound": "tensor", "flops": 2.0 * H * n * T * d, "exps": float(H) * n * T}
+    else:
+        corr = {"bound": "hbm", "bytes": H * (T * ldn * (2 if corr_kind == "bf16" else 4) + ldn * 4 + T * 4)}
     return {
-        "corr": {"bound": "hbm", "bytes": H * (T * ldn * corr_bytes + ldn * 4 + T * 4)},
+        "corr": corr,
         "phi": {"bound": "alu", "flops": 2.0 * H * n * T * d, "bytes": H * T * ldn * 4},
         "target": {"bound": "alu", "flops": 2.0 * H * n * T * d, "bytes": H * T * ldn * 4},
         "shift": {"bound": "alu", "flops": 2.0 * H * n * T * d},
@@ -190,6 +194,19 @@ def roofline(stages, steps, models, peaks, clocks, traffic_info):
         out.update({"bound": "hbm", "achieved": ach, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                     "frac": ach / peaks["hbm_gbs"], "peak_source": peaks["source"] + " hbm_gbs",
                     "algorithmic_bytes_per_launch": m["bytes"]})
+    elif m["bound"] == "tensor":
+        # dense bf16 MMA work of the launch against the sustained cuBLAS peak; the
+        # epilogue's exponentials (one per feature) are reported against the
+        # ex2 unit rate, 148 SMs x 16 per clock x median SM clock
+        ach = m["flops"] / (avg_ms * 1e-3) / 1e12
+        pk = peaks["bf16_tflops_sustained"]
+        mhz = (clocks or {}).get("sm_mhz") or peaks["sm_max_mhz"]
+        exp_peak = 148 * 16 * mhz * 1e6
+        out.update({"bound": "tensor", "achieved": ach, "peak": pk, "unit": "TFLOP/s", "frac": ach / pk,
+                    "peak_source": peaks["source"] + " bf16_tflops_sustained",
+                    "algorithmic_flops_per_launch": m["flops"],
+                    "exp_rate": {"achieved_per_s": m["exps"] / (avg_ms * 1e-3), "peak_per_s": exp_peak,
+                                 "frac": m["exps"] / (avg_ms * 1e-3) / exp_peak}})
     else:
         # fp32 FMA pipes: 148 SMs x 128 lanes x 2 flops x SM clock
         mhz = (clocks or {}).get("sm_mhz") or peaks["sm_max_mhz"]
@@ -267,10 +284,13 @@ def run_ours(args, rank, world, local_rank):
     Kh = torch.stack([h.K for h in wl.heads]).contiguous()
     Vh = torch.stack([h.V for h in wl.heads]).contiguous()
     Q, K, V = Qh.to(dev), Kh.to(dev), Vh.to(dev)
-    corr_dtype = am.BF16 if args.corr_dtype == "bf16" else am.FP32
-    kw = dict(topk=wl.topk, refit_every=wl.refit_every, corr_dtype=corr_dtype)
+    corr_mode = {"auto": am.CORR_AUTO, "fp32": am.CORR_STORED_FP32, "bf16": am.CORR_STORED_BF16,
+                 "recompute": am.CORR_RECOMPUTE}[args.corr]
+    kw = dict(topk=wl.topk, refit_every=wl.refit_every, corr_mode=corr_mode)
     opts = am.make_opts(am.BF16 if Q.dtype == torch.bfloat16 else am.FP32, wl.topk, wl.refit_every,
-                        corr_dtype=corr_dtype)
+                        corr_mode=corr_mode)
+    tc_ok = Q.dtype == torch.bfloat16 and d in (64, 128)
+    corr_kind = {"auto": "recompute" if tc_ok else "fp32"}.get(args.corr, args.corr)
     ws = torch.empty((am.workspace_size(n, T, d, wl.budgets, opts),), dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
     flush = torch.empty((256 << 20,), dtype=torch.uint8, device=dev)
@@ -348,15 +368,15 @@ def run_ours(args, rank, world, local_rank):
     ldn = (n + 31) // 32 * 32
     passes = max((t + wl.topk * wl.refit_every - 1) // (wl.topk * wl.refit_every) for t in wl.budgets)
     peaks = load_peaks()
-    rf = roofline(stages, args.steps,
-                  stage_models(wl, n, T, d, H, ldn, passes, 2 if args.corr_dtype == "bf16" else 4),
-                  peaks, clk, committed_traffic() if args.corr_dtype == "fp32" else {})
+    rf = roofline(stages, args.steps, stage_models(wl, n, T, d, H, ldn, passes, corr_kind),
+                  peaks, clk, committed_traffic() if corr_kind == "fp32" else {})
     value = H * world / (ms * 1e-3)
     per_step_stage = {k: round(v["ms"] / args.steps, 4) for k, v in stages.items() if v["launches"]}
     cfg = {"workload": wl.name, "heads_per_gpu": H, "n": n, "T": T, "d": d,
            "budgets": wl.budgets if H <= 8 else f"{sum(wl.budgets)} total, min {min(wl.budgets)} max {max(wl.budgets)}",
            "topk": wl.topk, "refit_every": wl.refit_every,
-           "phi_storage": "fp32" + (" + bf16 copy for the correlation pass" if args.corr_dtype == "bf16" else ""),
+           "correlation": {"fp32": "streams stored fp32 Phi^T", "bf16": "streams a bf16 copy of Phi^T",
+                           "recompute": "recomputes Phi on the tensor cores each pass"}[corr_kind],
            "l2": "256 MiB buffer written between timed steps",
            "stage_ms_per_step": per_step_stage, "device_status": worst}
     if args.workload == "qwen3_4b_layer":

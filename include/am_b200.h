@@ -60,6 +60,20 @@ typedef enum am_status {
 
 typedef enum am_dtype { AM_BF16 = 0, AM_FP32 = 1 } am_dtype_t;
 
+/* Where the correlation pass c = Φᵀ r reads the features from.  The mass,
+ * Gram, residual and value fit always use the stored fp32 Φ. */
+typedef enum am_corr_mode {
+  AM_CORR_AUTO = 0,         /* RECOMPUTE when the tensor-core path applies (bf16
+                               inputs, d in {64, 128}), else STORED_FP32          */
+  AM_CORR_STORED_FP32 = 1,  /* stream the stored fp32 Φᵀ (4 bytes per feature)    */
+  AM_CORR_STORED_BF16 = 2,  /* stream a bf16 copy of Φᵀ written by the feature
+                               pass (2 bytes per feature; picks may differ from
+                               exact arithmetic where correlations are closer
+                               than bf16 rounding)                                 */
+  AM_CORR_RECOMPUTE = 3     /* recompute Φ from Q and K on the tensor cores in
+                               every pass (no feature reads; bf16 inputs only)     */
+} am_corr_mode_t;
+
 /* Options.  Fill with am_default_opts() and override fields. */
 typedef struct am_opts {
   int32_t in_dtype;        /* am_dtype_t of Q_ref, K, V and of the C_k output   */
@@ -69,11 +83,7 @@ typedef struct am_opts {
   float scale;             /* logit scale; <= 0 selects 1/sqrt(d)                */
   float ridge;             /* λ = ridge·tr(AᵀA)/t (default 1e-6); must be >= 0   */
   float w_floor_rel;       /* β floor: w >= w_floor_rel·max(w) (default 1e-12)   */
-  int32_t corr_dtype;      /* features streamed by the correlation pass: AM_FP32
-                              (default) reads Φᵀ itself; AM_BF16 makes the feature
-                              pass also write a bf16 copy of Φᵀ, which the
-                              correlation pass reads at half the bytes (the mass,
-                              Gram, residual and value fit always use fp32 Φ)     */
+  int32_t corr_mode;       /* am_corr_mode_t: how the correlation pass gets Φ      */
   /* Optional device inputs */
   const float* shift;      /* [H] per-head shift c_h, or NULL: c_h = max_ij s_ij
                               computed on the device                              */
@@ -88,8 +98,8 @@ typedef struct am_opts {
 } am_opts_t;
 
 /* Fill *opts with defaults: bf16 inputs, k = 1, R = 1, scale = 1/sqrt(d),
- * ridge = 1e-6, w_floor_rel = 1e-12, corr_dtype = AM_FP32, every optional
- * pointer NULL. */
+ * ridge = 1e-6, w_floor_rel = 1e-12, corr_mode = AM_CORR_AUTO, every
+ * optional pointer NULL. */
 am_status_t am_default_opts(am_opts_t* opts);
 
 /* Device workspace needed by am_compact_heads for this problem.
@@ -100,7 +110,7 @@ am_status_t am_default_opts(am_opts_t* opts);
  *   opts             as passed to am_compact_heads
  *   bytes            host out
  * The dominant term is H·T·round_up(n, 32)·4 bytes of stored features
- * (·6 with corr_dtype = AM_BF16). */
+ * (·6 with AM_CORR_STORED_BF16). */
 am_status_t am_workspace_size(int32_t n, int32_t T, int32_t d, int32_t num_heads,
                               const int32_t* budgets, const am_opts_t* opts,
                               size_t* bytes);

@@ -128,7 +128,8 @@ def _ls_qr(A: np.ndarray, y: np.ndarray) -> np.ndarray:
     return solve_triangular(R, Qm.T @ y, lower=False)
 
 
-def nnls(A, y, tol: Optional[float] = None, max_iter: Optional[int] = None) -> np.ndarray:
+def nnls(A, y, tol: Optional[float] = None, max_iter: Optional[int] = None,
+         x0: Optional[np.ndarray] = None) -> np.ndarray:
     """argmin_{x ≥ 0} ‖A x − y‖₂ by the Lawson-Hanson active-set method.
 
     Outer loop: move the zero variable with the largest positive gradient
@@ -136,6 +137,10 @@ def nnls(A, y, tol: Optional[float] = None, max_iter: Optional[int] = None) -> n
     least squares on the passive set; if some passive value is not positive,
     step from x toward it until the first one hits zero, drop the zeros and
     resolve.  Stops when no zero variable has g_j > tol.
+
+    ``x0`` (optional, feasible) starts the method from that point with its
+    support as the passive set instead of from zero; the minimiser reached is
+    the same.
     """
     A = np.asarray(A, F64)
     y = np.asarray(y, F64)
@@ -148,14 +153,22 @@ def nnls(A, y, tol: Optional[float] = None, max_iter: Optional[int] = None) -> n
     passive = np.zeros(p, dtype=bool)
     blocked = np.zeros(p, dtype=bool)
     it = 0
+    j = -1
+    if x0 is not None:
+        x = np.maximum(np.asarray(x0, F64), 0.0)
+        passive = x > 0
+    first = x0 is not None and passive.any()
     g = A.T @ (y - A @ x)
     while True:
-        cand = (~passive) & (~blocked) & (g > tol)
-        if not cand.any():
-            break
-        idx = np.flatnonzero(cand)
-        j = int(idx[np.argmax(g[idx])])        # argmax returns the lowest index on ties
-        passive[j] = True
+        if first:
+            first = False     # a warm start begins with the inner loop on its support
+        else:
+            cand = (~passive) & (~blocked) & (g > tol)
+            if not cand.any():
+                break
+            idx = np.flatnonzero(cand)
+            j = int(idx[np.argmax(g[idx])])        # argmax returns the lowest index on ties
+            passive[j] = True
         while True:
             it += 1
             if it > max_iter:
@@ -174,7 +187,7 @@ def nnls(A, y, tol: Optional[float] = None, max_iter: Optional[int] = None) -> n
             x[neg[k]] = 0.0
             passive &= ~(passive & (x <= 0))
             x[~passive] = 0.0
-        if passive[j]:
+        if j < 0 or passive[j]:
             blocked[:] = False
         else:
             # round-off kept the entering variable from growing: leave it out
@@ -253,7 +266,8 @@ def omp_select(Phi, m, t: int, topk: int = 1, refit_every: int = 1,
         selected[picks] = True
         rnd += 1
         if rnd % refit_every == 0 or len(S) == t:
-            w = nnls(Phi[:, S], m)
+            # NNLS of the enlarged problem, started from the previous weights
+            w = nnls(Phi[:, S], m, x0=np.concatenate([w, np.zeros(len(S) - w.size)]))
             r = m - Phi[:, S] @ w
             rec["refit"] = True
         else:

@@ -139,6 +139,18 @@ def test_nnls_matches_enumeration_and_scipy(seed):
     assert kkt["min_x"] >= 0 and kkt["stationarity"] < 1e-9 and kkt["dual_feasibility"] < 1e-9
 
 
+@pytest.mark.parametrize("seed", range(4))
+def test_nnls_warm_start_reaches_the_same_minimiser(seed):
+    """A feasible warm start (as the OMP refits use) ends where a cold start does."""
+    rng = np.random.default_rng(200 + seed)
+    A = rng.random((40, 12)) + 0.1 * rng.standard_normal((40, 12))
+    y = rng.random(40)
+    cold = O.nnls(A, y)
+    for x0 in (np.zeros(12), rng.random(12), np.where(rng.random(12) < 0.5, rng.random(12), 0.0), cold):
+        np.testing.assert_allclose(O.nnls(A, y, x0=x0), cold, atol=1e-10)
+    np.testing.assert_allclose(cold, _nnls_by_enumeration(A, y), atol=1e-10)
+
+
 def test_nnls_single_column_closed_form():
     rng = np.random.default_rng(5)
     phi = rng.random(20)
