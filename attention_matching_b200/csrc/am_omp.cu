@@ -312,6 +312,21 @@ __device__ __forceinline__ void warp_fwd(const double* L, const double* invd, do
   }
 }
 
+// v ← L⁻¹ v (one warp), row form: y_k = (v_k − L[k, :k]·y[:k]) / L_kk.  Each
+// step reads one contiguous factor row (coalesced when the factor is in
+// global memory) and reduces across the warp.
+__device__ __forceinline__ void warp_fwd_rows(const double* L, const double* invd, double* v, int n) {
+  const int lane = threadIdx.x & 31;
+  for (int k = 0; k < n; ++k) {
+    const double* row = L + tri(k, 0);
+    double acc = 0.0;
+    for (int j = lane; j < k; j += 32) acc += row[j] * v[j];
+    acc = warp_sum(acc);
+    if (lane == 0) v[k] = (v[k] - acc) * invd[k];
+    __syncwarp();
+  }
+}
+
 // v ← L⁻ᵀ v (one warp)
 __device__ __forceinline__ void warp_bwd(const double* L, const double* invd, double* v, int n) {
   const int lane = threadIdx.x & 31;
@@ -412,7 +427,10 @@ __global__ void __launch_bounds__(kNnlsThreads) k_nnls(Problem p, Work w, int pa
         for (int q = lane; q < np; q += 32) row[q] = Ge[P[q]];
       }
       __syncthreads();
-      for (int e = warp; e < k; e += nw) warp_fwd(L, invd, L + tri(np + e, 0), np);
+      for (int e = warp; e < k; e += nw) {
+        if (l_smem) warp_fwd(L, invd, L + tri(np + e, 0), np);
+        else warp_fwd_rows(L, invd, L + tri(np + e, 0), np);
+      }
       __syncthreads();
       // Schur complement of the new block (lower triangle)
       for (int pr = warp; pr < k * (k + 1) / 2; pr += nw) {
@@ -529,7 +547,8 @@ __global__ void __launch_bounds__(kNnlsThreads) k_nnls(Problem p, Work w, int pa
       for (int q = tid; q < npc; q += blockDim.x) z[q] = b[P[q]];
       __syncthreads();
       if (warp == 0) {
-        warp_fwd(L, invd, z, npc);
+        if (l_smem) warp_fwd(L, invd, z, npc);
+        else warp_fwd_rows(L, invd, z, npc);
         warp_bwd(L, invd, z, npc);
       }
       __syncthreads();

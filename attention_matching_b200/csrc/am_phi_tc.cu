@@ -47,7 +47,7 @@ enum Mode { MODE_MAX = 0, MODE_PHI = 1 };
 struct Plan {
   int d;
   uint32_t q_bytes, k_bytes, v_bytes, p_bytes;
-  uint32_t off_q, off_k, off_v, off_p, off_bias, off_bar, total;
+  uint32_t off_q, off_k, off_v, off_p, off_bar, total;
 };
 
 __host__ __device__ inline Plan make_plan(int d, int mode) {
@@ -62,7 +62,6 @@ __host__ __device__ inline Plan make_plan(int d, int mode) {
   P.off_k = o; o += STAGES * P.k_bytes;
   P.off_v = o; o += STAGES * P.v_bytes;
   P.off_p = o; o += 2 * 2 * P.p_bytes;               // 2 buffers × (hi, lo)
-  P.off_bias = o; o += 2 * BN * 4;
   P.off_bar = o; o += 32 * 8;
   P.total = o + 1024;                                 // slack to align the base
   return P;
@@ -155,6 +154,9 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
   for (int k = 0; k < 32; ++k) v[k] = __uint_as_float(r[k]);
 }
 
+// TMEM address of lane quadrant q (lanes 32q..32q+31), column 0.
+__device__ __forceinline__ uint32_t lane_addr_base(int q) { return (uint32_t)(q * 32) << 16; }
+
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 
 // Shared-memory matrix descriptor, SWIZZLE_128B (sm_100 encoding 2), version 1.
@@ -201,7 +203,6 @@ k_phi_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtens
   unsigned char* sK = sm + P.off_k;
   unsigned char* sV = sm + P.off_v;
   unsigned char* sP = sm + P.off_p;
-  float* sBias = reinterpret_cast<float*>(sm + P.off_bias);
   uint64_t* bars = reinterpret_cast<uint64_t*>(sm + P.off_bar);
   uint64_t* q_full = bars + 0;
   uint64_t* kv_full = bars + 1;             // [STAGES]
@@ -216,7 +217,6 @@ k_phi_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtens
   __shared__ int s_abort;
   __shared__ float s_red[8];
   __shared__ double s_mass[256];
-  __shared__ int s_stop[2];
   __shared__ int s_stop_y;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -346,6 +346,7 @@ k_phi_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtens
     // which no result depends on (the shift invariance).
     const float kLog2e = 1.4426950408889634f;
     const float scale = MODE == MODE_PHI ? p.scale * kLog2e : p.scale;
+    const float bias_const = MODE == MODE_PHI ? -c * kLog2e : 0.f;
     double mrow = 0.0;
     float mx = -FLT_MAX;
     const uint32_t lane_addr = (uint32_t)(qd * 32) << 16;
@@ -353,20 +354,8 @@ k_phi_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtens
     bool ok = true;
     for (int j = 0; j < NT; ++j) {
       const int b = j & 1, bu = j >> 1;
-      // One thread waits (S tile ready; P buffer free again) and publishes a
-      // stop flag, so all 256 epilogue threads leave the loop together.
-      if (ep == 0) {
-        bool good = mbar_wait(s_full + b, bu & 1, abort_flag, status);
-        if (good && MODE == MODE_PHI && bu > 0) good = mbar_wait(p_empty + b, (bu - 1) & 1, abort_flag, status);
-        s_stop[b] = good ? 0 : 1;
-      }
-      if (ep < BN) {   // this tile's per-key additive term, shared by all rows
-        const int jg = j * BN + ep;
-        const float bj = (p.has_bias && jg < p.T) ? key_bias[(int64_t)h * p.T + jg] : 0.f;
-        sBias[b * BN + ep] = MODE == MODE_PHI ? (bj - c) * kLog2e : bj;
-      }
-      asm volatile("bar.sync 1, 256;" ::: "memory");
-      if (s_stop[b]) { ok = false; break; }
+      // every epilogue thread waits for the tile itself; no named barrier in the loop
+      if (!mbar_wait(s_full + b, bu & 1, abort_flag, status)) { ok = false; break; }
       tc_fence_after();
       float v[HC];
       tmem_ld32(tS[b] + lane_addr + half * HC, v);
@@ -374,18 +363,25 @@ k_phi_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtens
       tc_fence_before();
       mbar_arrive(s_empty + b);
       const int kvalid = min(BN, p.T - j * BN) - half * HC;   // valid columns of this half
-      const float* bias_t = sBias + b * BN + half * HC;
+      // per-key additive term: (b_j − c)·log2e (PHI) or b_j (MAX); a constant without a prior bias
+      const int jb = j * BN + half * HC;
+      auto bias_at = [&](int cc) -> float {
+        if (!p.has_bias) return bias_const;
+        const int jg = jb + cc;
+        const float bj = jg < p.T ? __ldg(key_bias + (int64_t)h * p.T + jg) : 0.f;
+        return MODE == MODE_PHI ? (bj - c) * kLog2e : bj;
+      };
       if constexpr (MODE == MODE_MAX) {
         if (row_live) {
 #pragma unroll
           for (int cc = 0; cc < HC; ++cc)
-            if (cc < kvalid) mx = fmaxf(mx, fmaf(v[cc], scale, bias_t[cc]));
+            if (cc < kvalid) mx = fmaxf(mx, fmaf(v[cc], scale, bias_at(cc)));
         }
         continue;
       } else {
 #pragma unroll
       for (int cc = 0; cc < HC; ++cc) {
-        const float x = fmaf(v[cc], scale, bias_t[cc]);
+        const float x = fmaf(v[cc], scale, bias_at(cc));
         v[cc] = (row_live && cc < kvalid) ? exp2f(x) : 0.f;
       }
       double a4[4] = {0.0, 0.0, 0.0, 0.0};   // mass partials: short dependency chains
@@ -404,7 +400,9 @@ k_phi_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtens
             if (cc < kvalid) col16[(int64_t)cc * p.ldn] = __float2bfloat16_rn(v[cc]);
         }
       }
-      // P tile for Y += P·V: K-major, 128-byte rows, 16-byte chunks XOR-swizzled by row
+      // P tile for Y += P·V: K-major, 128-byte rows, 16-byte chunks XOR-swizzled by row;
+      // the buffer is free once the MMA that read it two tiles ago has completed
+      if (bu > 0 && !mbar_wait(p_empty + b, (bu - 1) & 1, abort_flag, status)) { ok = false; break; }
       unsigned char* hi_row = sP + (b * 2 + 0) * P.p_bytes + et * 128;
       unsigned char* lo_row = sP + (b * 2 + 1) * P.p_bytes + et * 128;
 #pragma unroll
@@ -479,30 +477,38 @@ k_phi_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtens
 // a block of 128 keys, with Φ recomputed from Q and K on the tensor cores
 // instead of re-read from HBM (the OMP correlation step, zhichai.net deep
 // dive §1.6: j* = argmax rᵀΦ_{:,j}).  Keys sit on the TMEM lanes (M = 128),
-// query tiles of 64 stream through a 4-stage ring (N = 64); two epilogue
-// warpgroups each fold 32 queries of every tile into their key's sum.
-constexpr int CQ = 64;          // queries per tile
-constexpr int CSTAGES = 4;
+// query tiles of 128 stream through a 3-stage ring (N = 128); four epilogue
+// warpgroups each fold 32 queries of every tile into their key's sum.  Each
+// epilogue thread waits on the tile's barrier itself (no named barrier in
+// the loop) and reads the residual with broadcast vector loads.
+constexpr int CQ = 128;         // queries per tile
+constexpr int CSTAGES = 3;
+constexpr int kCorrThreads = 640;   // 4 control warps + 4 epilogue warpgroups
+constexpr uint32_t kCorrTmemCols = 256;
 
 __host__ __device__ inline uint32_t corr_smem_bytes(int d) {
-  return (uint32_t)(BM * d * 2 + CSTAGES * CQ * d * 2 + 2 * CQ * 4 + 32 * 8 + 1024);
+  return (uint32_t)(BM * d * 2 + CSTAGES * CQ * d * 2 + 32 * 8 + 1024);
+}
+
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
 }
 
 template <int D>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kCorrThreads, 1)
 k_corr_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK, Problem p, Work w,
           const float* __restrict__ key_bias, int pass) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   constexpr int KB = D / 64;
-  const int hslot = blockIdx.y;
-  const int h = w.order[hslot];
+  const int h = w.order[blockIdx.y];
   if (pass * p.kR >= w.t[h]) return;          // head already finished (whole CTA leaves)
   unsigned char* sm = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t k_bytes = BM * D * 2, q_bytes = CQ * D * 2;
   unsigned char* sK = sm;
   unsigned char* sQ = sm + k_bytes;
-  float* sR = reinterpret_cast<float*>(sQ + CSTAGES * q_bytes);
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sR + 2 * CQ);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sQ + CSTAGES * q_bytes);
   uint64_t* k_full = bars + 0;
   uint64_t* q_full = bars + 1;                  // [CSTAGES]
   uint64_t* q_empty = bars + 1 + CSTAGES;       // [CSTAGES]
@@ -511,8 +517,7 @@ k_corr_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
   uint64_t* drain = s_full + 4;
   __shared__ uint32_t s_tmem;
   __shared__ int s_abort;
-  __shared__ int s_stop[2];
-  __shared__ float s_part[128];
+  __shared__ float s_part[4][128];
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int j0 = blockIdx.x * BM;
@@ -524,13 +529,13 @@ k_corr_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
     s_abort = 0;
     mbar_init(k_full, 1);
     for (int s = 0; s < CSTAGES; ++s) { mbar_init(q_full + s, 1); mbar_init(q_empty + s, 1); }
-    for (int b = 0; b < 2; ++b) { mbar_init(s_full + b, 1); mbar_init(s_empty + b, 256); }
+    for (int b = 0; b < 2; ++b) { mbar_init(s_full + b, 1); mbar_init(s_empty + b, 512); }
     mbar_init(drain, 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   if (warp == 2) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(&s_tmem)),
-                 "r"(128));
+                 "r"(kCorrTmemCols));
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
   }
   tc_fence_before();
@@ -585,12 +590,10 @@ k_corr_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
       while (!mbar_try_wait(drain, 0) && clock64() - t0 < kWaitBudgetCycles) {}
     }
   } else if (warp >= kEpiWarp0) {
-    const int ep = threadIdx.x - kEpiWarp0 * 32;
-    const int half = ep >> 7;
-    const int et = ep & 127;
-    const int qd = warp & 3;
-    constexpr int HC = CQ / 2;
-    const int j = j0 + et;                       // this thread's key
+    const int wg = (warp - kEpiWarp0) >> 2;     // 32-query column group of each tile
+    const int qd = warp & 3;                    // TMEM lane quadrant
+    const int et = qd * 32 + lane;              // key row within the block
+    const int j = j0 + et;
     const bool key_live = j < p.T;
     const float kLog2e = 1.4426950408889634f;
     const float scale = p.scale * kLog2e;
@@ -598,36 +601,39 @@ k_corr_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
     const float bj = (p.has_bias && key_live) ? key_bias[(int64_t)h * p.T + j] : 0.f;
     const float bias2 = (bj - c) * kLog2e;
     const float* rh = w.r + (int64_t)h * p.ldn;
-    const uint32_t lane_addr = (uint32_t)(qd * 32) << 16;
+    const uint32_t tcol = lane_addr_base(qd) + wg * 32;
     float acc[4] = {0.f, 0.f, 0.f, 0.f};
     for (int t = 0; t < NQ; ++t) {
       const int b = t & 1, bu = t >> 1;
-      if (ep == 0) s_stop[b] = mbar_wait(s_full + b, bu & 1, abort_flag, status) ? 0 : 1;
-      if (ep < CQ) {   // this tile's residual entries (zero past n)
-        const int q = t * CQ + ep;
-        sR[b * CQ + ep] = q < p.n ? rh[q] : 0.f;
-      }
-      asm volatile("bar.sync 1, 256;" ::: "memory");
-      if (s_stop[b]) break;
+      if (!mbar_wait(s_full + b, bu & 1, abort_flag, status)) break;
       tc_fence_after();
-      float v[HC];
-      tmem_ld32(tS[b] + lane_addr + half * HC, v);
+      float v[32];
+      tmem_ld32(tS[b] + tcol, v);
       tmem_wait_ld();
       tc_fence_before();
       mbar_arrive(s_empty + b);
-      const float* rr = sR + b * CQ + half * HC;
+      const int q0 = t * CQ + wg * 32;
+      if (q0 < p.ldn) {   // r is zero from n to ldn; chunks of 32 lie wholly inside or outside
+        const float4* r4 = reinterpret_cast<const float4*>(rh + q0);
 #pragma unroll
-      for (int cc = 0; cc < HC; ++cc) acc[cc & 3] = fmaf(exp2f(fmaf(v[cc], scale, bias2)), rr[cc], acc[cc & 3]);
+        for (int k = 0; k < 8; ++k) {
+          const float4 rr = __ldg(r4 + k);
+          acc[0] = fmaf(ex2_approx(fmaf(v[4 * k + 0], scale, bias2)), rr.x, acc[0]);
+          acc[1] = fmaf(ex2_approx(fmaf(v[4 * k + 1], scale, bias2)), rr.y, acc[1]);
+          acc[2] = fmaf(ex2_approx(fmaf(v[4 * k + 2], scale, bias2)), rr.z, acc[2]);
+          acc[3] = fmaf(ex2_approx(fmaf(v[4 * k + 3], scale, bias2)), rr.w, acc[3]);
+        }
+      }
     }
-    const float mine = (acc[0] + acc[1]) + (acc[2] + acc[3]);
-    if (half == 1) s_part[et] = mine;
-    asm volatile("bar.sync 1, 256;" ::: "memory");
-    if (half == 0 && key_live && !s_abort) w.corr[(int64_t)h * p.T + j] = mine + s_part[et];
+    s_part[wg][et] = (acc[0] + acc[1]) + (acc[2] + acc[3]);
+    asm volatile("bar.sync 1, 512;" ::: "memory");
+    if (wg == 0 && key_live && !s_abort)
+      w.corr[(int64_t)h * p.T + j] = ((s_part[0][et] + s_part[1][et]) + s_part[2][et]) + s_part[3][et];
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (warp == 2) asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(128));
+  if (warp == 2) asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kCorrTmemCols));
 }
 
 // ---- host: tensor maps ----
@@ -684,7 +690,7 @@ cudaError_t launch_corr_tc_d(const Problem& p, const void* Q, const void* K, con
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
   if (e != cudaSuccess) return e;
   dim3 grid((p.T + BM - 1) / BM, active);
-  AM_LAUNCH(AM_STAGE_CORR, s, kern<<<grid, kThreads, bytes, s>>>(mq, mk, p, w, key_bias, pass));
+  AM_LAUNCH(AM_STAGE_CORR, s, kern<<<grid, kCorrThreads, bytes, s>>>(mq, mk, p, w, key_bias, pass));
   return cudaGetLastError();
 }
 

@@ -54,6 +54,21 @@ def parse_args():
     return ap.parse_args()
 
 
+def max_over_ranks(ms, dist, device):
+    """The step time of the job: the slowest rank's (identity for one process)."""
+    if dist is None:
+        return float(ms)
+    import torch
+    t = torch.tensor([ms], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(heads_per_rank, world, ms):
+    """Whole-job heads/s: every rank compacts its own heads in the same step time."""
+    return heads_per_rank * world / (ms * 1e-3)
+
+
 def build_workload(name, rank, heads=None):
     from attention_matching_b200 import workloads as W
     if name == "qwen3_4b_layer":
@@ -325,10 +340,7 @@ def run_ours(args, rank, world, local_rank):
     clk = clocks.stop()
     step_ms = [a.elapsed_time(b) for a, b in evs]
     ms = statistics.mean(step_ms)
-    ms_t = torch.tensor([ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(ms_t, op=dist.ReduceOp.MAX)
-    ms = float(ms_t.item())
+    ms = max_over_ranks(ms, dist if world > 1 else None, dev)
     _, worst = am.get_status(ws, H)
 
     # end to end through the public API with pinned host buffers
@@ -350,11 +362,8 @@ def run_ours(args, rank, world, local_rank):
             d2h = sum(o[k].numel() * o[k].element_size() for k in ("C_k", "beta", "C_v", "indices"))
         torch.cuda.synchronize()
         e_ms = statistics.mean(a.elapsed_time(b) for a, b in ev2)
-        e_t = torch.tensor([e_ms], dtype=torch.float64, device=dev)
-        if world > 1:
-            dist.all_reduce(e_t, op=dist.ReduceOp.MAX)
-        e_ms = float(e_t.item())
-        e2e = {"value": H * world / (e_ms * 1e-3), "unit": "heads/s",
+        e_ms = max_over_ranks(e_ms, dist if world > 1 else None, dev)
+        e2e = {"value": job_throughput(H, world, e_ms), "unit": "heads/s",
                "h2d_bytes_per_step": sum(x.numel() * x.element_size() for x in (Qh, Kh, Vh)),
                "d2h_bytes_per_step": d2h, "ms_per_step": e_ms}
 
@@ -370,7 +379,7 @@ def run_ours(args, rank, world, local_rank):
     peaks = load_peaks()
     rf = roofline(stages, args.steps, stage_models(wl, n, T, d, H, ldn, passes, corr_kind),
                   peaks, clk, committed_traffic() if corr_kind == "fp32" else {})
-    value = H * world / (ms * 1e-3)
+    value = job_throughput(H, world, ms)
     per_step_stage = {k: round(v["ms"] / args.steps, 4) for k, v in stages.items() if v["launches"]}
     cfg = {"workload": wl.name, "heads_per_gpu": H, "n": n, "T": T, "d": d,
            "budgets": wl.budgets if H <= 8 else f"{sum(wl.budgets)} total, min {min(wl.budgets)} max {max(wl.budgets)}",
