@@ -154,6 +154,12 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
   for (int k = 0; k < 32; ++k) v[k] = __uint_as_float(r[k]);
 }
 
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 // TMEM address of lane quadrant q (lanes 32q..32q+31), column 0.
 __device__ __forceinline__ uint32_t lane_addr_base(int q) { return (uint32_t)(q * 32) << 16; }
 
@@ -218,6 +224,7 @@ k_phi_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtens
   __shared__ float s_red[8];
   __shared__ double s_mass[256];
   __shared__ int s_stop_y;
+  __shared__ int s_stopm[2];
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int nqb = (p.n + BM - 1) / BM;
@@ -354,8 +361,15 @@ k_phi_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtens
     bool ok = true;
     for (int j = 0; j < NT; ++j) {
       const int b = j & 1, bu = j >> 1;
-      // every epilogue thread waits for the tile itself; no named barrier in the loop
-      if (!mbar_wait(s_full + b, bu & 1, abort_flag, status)) { ok = false; break; }
+      if constexpr (MODE == MODE_MAX) {
+        // light per-tile work: one thread waits and the group follows it
+        if (ep == 0) s_stopm[b] = mbar_wait(s_full + b, bu & 1, abort_flag, status) ? 0 : 1;
+        asm volatile("bar.sync 1, 256;" ::: "memory");
+        if (s_stopm[b]) { ok = false; break; }
+      } else {
+        // each epilogue thread waits for the tile itself; no named barrier in the loop
+        if (!mbar_wait(s_full + b, bu & 1, abort_flag, status)) { ok = false; break; }
+      }
       tc_fence_after();
       float v[HC];
       tmem_ld32(tS[b] + lane_addr + half * HC, v);
@@ -366,23 +380,31 @@ k_phi_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtens
       // per-key additive term: (b_j − c)·log2e (PHI) or b_j (MAX); a constant without a prior bias
       const int jb = j * BN + half * HC;
       auto bias_at = [&](int cc) -> float {
-        if (!p.has_bias) return bias_const;
         const int jg = jb + cc;
         const float bj = jg < p.T ? __ldg(key_bias + (int64_t)h * p.T + jg) : 0.f;
         return MODE == MODE_PHI ? (bj - c) * kLog2e : bj;
       };
+      const bool full = row_live && kvalid >= HC;
       if constexpr (MODE == MODE_MAX) {
-        if (row_live) {
+        if (full && !p.has_bias) {
+#pragma unroll
+          for (int cc = 0; cc < HC; ++cc) mx = fmaxf(mx, v[cc] * scale);
+        } else if (row_live) {
 #pragma unroll
           for (int cc = 0; cc < HC; ++cc)
-            if (cc < kvalid) mx = fmaxf(mx, fmaf(v[cc], scale, bias_at(cc)));
+            if (cc < kvalid) mx = fmaxf(mx, fmaf(v[cc], scale, p.has_bias ? bias_at(cc) : 0.f));
         }
         continue;
       } else {
+      if (full && !p.has_bias) {   // common case: whole tile, no prior bias
 #pragma unroll
-      for (int cc = 0; cc < HC; ++cc) {
-        const float x = fmaf(v[cc], scale, bias_at(cc));
-        v[cc] = (row_live && cc < kvalid) ? exp2f(x) : 0.f;
+        for (int cc = 0; cc < HC; ++cc) v[cc] = ex2_approx(fmaf(v[cc], scale, bias_const));
+      } else {
+#pragma unroll
+        for (int cc = 0; cc < HC; ++cc) {
+          const float x = fmaf(v[cc], scale, p.has_bias ? bias_at(cc) : bias_const);
+          v[cc] = (row_live && cc < kvalid) ? ex2_approx(x) : 0.f;
+        }
       }
       double a4[4] = {0.0, 0.0, 0.0, 0.0};   // mass partials: short dependency chains
 #pragma unroll
@@ -390,9 +412,14 @@ k_phi_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtens
       mrow += (a4[0] + a4[1]) + (a4[2] + a4[3]);
       if (i < p.ldn) {
         float* col = phi_base + (int64_t)(j * BN + half * HC) * p.ldn + i;
+        if (kvalid >= HC) {
 #pragma unroll
-        for (int cc = 0; cc < HC; ++cc)
-          if (cc < kvalid) col[(int64_t)cc * p.ldn] = v[cc];
+          for (int cc = 0; cc < HC; ++cc) col[(int64_t)cc * p.ldn] = v[cc];
+        } else {
+#pragma unroll
+          for (int cc = 0; cc < HC; ++cc)
+            if (cc < kvalid) col[(int64_t)cc * p.ldn] = v[cc];
+        }
         if (w.phiT16) {   // bf16 copy streamed by the correlation pass
           __nv_bfloat16* col16 = w.phiT16 + ((int64_t)h * p.T + j * BN + half * HC) * p.ldn + i;
 #pragma unroll
@@ -488,12 +515,6 @@ constexpr uint32_t kCorrTmemCols = 256;
 
 __host__ __device__ inline uint32_t corr_smem_bytes(int d) {
   return (uint32_t)(BM * d * 2 + CSTAGES * CQ * d * 2 + 32 * 8 + 1024);
-}
-
-__device__ __forceinline__ float ex2_approx(float x) {
-  float y;
-  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-  return y;
 }
 
 template <int D>
