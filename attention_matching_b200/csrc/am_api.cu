@@ -101,6 +101,7 @@ am_status_t check_shape(int n, int T, int d, int H, const int32_t* budgets, cons
   for (int h = 0; h < H; ++h) {
     const int t = budgets[h];
     if (t < 1 || t > T) return AM_ERR_BUDGET;
+    if (t > kMaxBudget) return AM_ERR_UNSUPPORTED;
     tb->cu_t[h + 1] = tb->cu_t[h] + t;
     tb->cu_t2[h + 1] = tb->cu_t2[h] + (int64_t)t * t;
     tb->max_t = std::max(tb->max_t, t);

@@ -13,6 +13,7 @@ namespace am {
 constexpr int kWsHeaderBytes = 256;      // magic + head count, then status words
 constexpr uint32_t kWsMagic = 0x414d4232u;  // "AMB2"
 constexpr int kMaxPicksPerPass = 64;     // k·R upper bound handled per pass
+constexpr int kMaxBudget = 2048;         // largest t_h the per-head solvers are sized for
 constexpr int kNnlsThreads = 256;
 constexpr int kCholThreads = 256;
 

@@ -396,7 +396,10 @@ __global__ void __launch_bounds__(kNnlsThreads) k_nnls(Problem p, Work w, int pa
       for (int a = warp; a < np; a += nw)
         for (int c = lane; c <= a; c += 32) L[tri(a, c)] = G[(int64_t)P[a] * t + P[c]];
       __syncthreads();
-      int badk = block_cholesky_packed(L, np, [&](int k) { return 1e-13 * diag(P[k]); }, &ctl[6]);
+      auto floor_k = [&](int k) { return 1e-13 * diag(P[k]); };
+      // a factor in the workspace is rebuilt tile by tile (shared memory as scratch)
+      int badk = l_smem ? block_cholesky_packed(L, np, floor_k, &ctl[6])
+                        : block_cholesky_tiled(L, np, floor_k, reinterpret_cast<double*>(smem + nnls_vec_bytes(t)), &ctl[6]);
       if (badk < 0) {
         for (int q = tid; q < np; q += blockDim.x) invd[q] = 1.0 / L[tri(q, q)];
         __syncthreads();

@@ -231,7 +231,9 @@ __global__ void __launch_bounds__(kCholThreads) k_chol(Problem p, Work w, int l_
   for (int a = threadIdx.x >> 5; a < t; a += blockDim.x >> 5)
     for (int c = threadIdx.x & 31; c <= a; c += 32) L[tri(a, c)] = M[(int64_t)a * t + c] + (a == c ? lam : 0.0);
   __syncthreads();
-  const int bad = block_cholesky_packed(L, t, [](int) { return 0.0; }, &flag);
+  // large heads: tiled factorization in the workspace, shared memory as tile scratch
+  const int bad = L != Lg ? block_cholesky_packed(L, t, [](int) { return 0.0; }, &flag)
+                          : block_cholesky_tiled(Lg, t, [](int) { return 0.0; }, reinterpret_cast<double*>(smem), &flag);
   if (bad >= 0) {
     if (threadIdx.x == 0) record_status(w.status + h, AM_ERR_NOT_SPD);
     for (int a = threadIdx.x; a < t; a += blockDim.x) w.w_eff[base + a] = 0.0;   // marks the head for k_trsm

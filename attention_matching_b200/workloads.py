@@ -216,3 +216,64 @@ def qwen3_4b_model(num_heads: int = 288, T: int = 8192, n: int = 8192, ratio: fl
     budgets = lognormal_budgets(seed_base + 999, num_heads, total)
     return Workload(f"qwen3_4b_model_H{num_heads}_T{T}_n{n}_d128_lognormal", heads,
                     budgets, 4, 2, "bf16")
+
+
+# ----------------------------------------------------------------------------
+# Online compaction rounds (xinfinite.net article §5 and Table 3: a fixed
+# physical cache; everything but the latest tokens is compacted by half,
+# repeatedly).  Each head keeps its rank-32 key basis across rounds; a round's
+# cache is [previous compacted keys (their β as prior key bias)] + [kept
+# latest tokens] + [fresh tokens], and reference queries are drawn against
+# the whole current cache.  The compacted values enter the next round rounded
+# to the storage dtype, as a cache would hold them.
+# ----------------------------------------------------------------------------
+
+class OnlineHeads:
+    def __init__(self, num_heads: int, cache: int = 2048, keep: int = 20, n: int = 2048, d: int = 128,
+                 rank: int = 32, seed: int = 3000, dtype: str = "bf16"):
+        self.H, self.cache, self.keep, self.n, self.d, self.rank = num_heads, cache, keep, n, d, rank
+        self.dtype = dtype
+        self.round = 0
+        self.rngs = [np.random.default_rng(seed + h) for h in range(num_heads)]
+        self.bases = [np.linalg.qr(r.standard_normal((d, rank)))[0] for r in self.rngs]
+        self.prev = None     # per head: (K f64, V f64, bias f64) of the uncompacted tail + compacted block
+
+    @property
+    def compact_len(self) -> int:
+        return self.cache - self.keep
+
+    @property
+    def budget(self) -> int:
+        return budget_for_ratio(self.compact_len, 2.0)
+
+    def _fresh(self, h: int, count: int, sinks: int):
+        rng = self.rngs[h]
+        K = _structured_keys(rng, count, self.d, self.rank, sinks, self.bases[h])
+        V = rng.standard_normal((count, self.d))
+        return upcast(round_to(K, self.dtype)), upcast(round_to(V, self.dtype))
+
+    def next_round(self, compacted=None) -> List[Head]:
+        """Heads of the next round.  `compacted` (after the first round) is a
+        per-head list of (C_k, beta, C_v) from the previous round's output."""
+        heads = []
+        for h in range(self.H):
+            if self.round == 0:
+                K, V = self._fresh(h, self.cache, sinks=4)
+                bias = np.zeros(self.cache)
+            else:
+                Ck, beta, Cv = compacted[h]
+                Kp, Vp, _ = self.prev[h]
+                kept_K, kept_V = Kp[self.compact_len:], Vp[self.compact_len:]
+                nf = self.cache - len(Ck) - self.keep
+                Kf, Vf = self._fresh(h, nf, sinks=0)
+                K = np.vstack([np.asarray(Ck, np.float64), kept_K, Kf])
+                V = np.vstack([upcast(round_to(np.asarray(Cv, np.float64), self.dtype)), kept_V, Vf])
+                bias = np.concatenate([np.asarray(beta, np.float64), np.zeros(self.keep + nf)])
+            Q = _mixture_queries(self.rngs[h], K, self.n, first=4 if self.round == 0 else 0)
+            self.prev = (self.prev or [None] * self.H)
+            self.prev[h] = (K, V, bias)
+            c = self.compact_len
+            heads.append(Head(round_to(Q, self.dtype), round_to(K[:c], self.dtype), round_to(V[:c], self.dtype),
+                              key_bias=np.float32(bias[:c])))
+        self.round += 1
+        return heads

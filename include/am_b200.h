@@ -106,7 +106,8 @@ am_status_t am_default_opts(am_opts_t* opts);
  *   n, T, d          reference queries, keys per head, head dim (d in {64, 128}
  *                    for bf16 inputs; any d in [1, 256] for fp32 inputs)
  *   num_heads        H
- *   budgets          host int32 [H], 1 <= t_h <= T
+ *   budgets          host int32 [H], 1 <= t_h <= T, and t_h <= 2048
+ *                    (larger budgets return AM_ERR_UNSUPPORTED)
  *   opts             as passed to am_compact_heads
  *   bytes            host out
  * The dominant term is H·T·round_up(n, 32)·4 bytes of stored features

@@ -51,6 +51,7 @@ def test_workspace_size_scales_with_features():
 @pytest.mark.parametrize("bad", [
     dict(budgets=[0]), dict(budgets=[301]), dict(topk=0), dict(refit_every=0),
     dict(topk=16, refit_every=8), dict(d=300), dict(ridge=-1.0), dict(w_floor_rel=0.0),
+    dict(T=4096, budgets=[2049]),
 ])
 def test_workspace_size_rejects(bad):
     args = dict(n=512, T=300, d=64, budgets=[16], topk=1, refit_every=1, ridge=1e-6, w_floor_rel=1e-12)

@@ -204,3 +204,23 @@ def test_recompute_and_stored_correlations_agree():
     b = run_gpu(heads, [6, 6], 4, 2, corr_mode=am.CORR_STORED_FP32)
     assert torch.equal(a["indices"], b["indices"])
     torch.testing.assert_close(a["pick_corr"], b["pick_corr"], rtol=2e-5, atol=0)
+
+
+@needs_cuda
+def test_online_rounds_chained():
+    """Online compaction (fixed cache, all but the latest 20 keys halved each
+    round): three rounds whose compacted blocks carry β as a prior key bias.
+    Rounds are chained through the oracle's outputs so both sides see the same
+    inputs; t = 246 also puts the solver factors in the workspace."""
+    on = W.OnlineHeads(2, cache=512, keep=20, n=512, d=128, seed=3100)
+    compacted = None
+    for rnd in range(3):
+        heads = on.next_round(compacted)
+        kb = [h.key_bias for h in heads]
+        check_all(heads, [on.budget] * 2, 4, 2, key_bias=kb, label=f"online round {rnd}")
+        compacted = []
+        for h in heads:
+            Q, K, V = h.f64()
+            b64 = np.asarray(h.key_bias, np.float64)
+            r = O.compact_head(Q, K, V, on.budget, 4, 2, shift=shift_for(Q, K, b64), key_bias=b64)
+            compacted.append((r["C_k"], np.float32(r["beta"]), r["C_v"]))
