@@ -132,11 +132,16 @@ def nnls(A, y, tol: Optional[float] = None, max_iter: Optional[int] = None,
          x0: Optional[np.ndarray] = None) -> np.ndarray:
     """argmin_{x ≥ 0} ‖A x − y‖₂ by the Lawson-Hanson active-set method.
 
-    Outer loop: move the zero variable with the largest positive gradient
-    g = Aᵀ(y − Ax) into the passive set.  Inner loop: solve the unconstrained
-    least squares on the passive set; if some passive value is not positive,
-    step from x toward it until the first one hits zero, drop the zeros and
-    resolve.  Stops when no zero variable has g_j > tol.
+    Outer loop: move the zero variable with the largest positive scaled
+    gradient g_j / ‖a_j‖, g = Aᵀ(y − Ax), into the passive set.  Inner loop:
+    solve the unconstrained least squares on the passive set; if some passive
+    value is not positive, step from x toward it until the first one hits
+    zero, drop the zeros and resolve.  Stops when no zero variable has
+    g_j > tol·‖a_j‖·‖y‖ (tol relative, default 1e-12).  The test is per
+    column and relative: an absolute threshold on g stops short of the
+    minimiser once ‖y − Ax‖ ≪ ‖y‖, where a variable with a tiny gradient can
+    still lower the residual by a large fraction when its column is nearly
+    dependent on the passive ones.
 
     ``x0`` (optional, feasible) starts the method from that point with its
     support as the passive set instead of from zero; the minimiser reached is
@@ -146,7 +151,10 @@ def nnls(A, y, tol: Optional[float] = None, max_iter: Optional[int] = None,
     y = np.asarray(y, F64)
     nrow, p = A.shape
     if tol is None:
-        tol = 1e-13 * np.linalg.norm(A) * np.linalg.norm(y)
+        tol = 1e-12
+    col = np.linalg.norm(A, axis=0)
+    thr = tol * col * np.linalg.norm(y)     # per-column threshold on g_j
+    col = np.where(col > 0, col, 1.0)
     if max_iter is None:
         max_iter = 3 * p + 50
     x = np.zeros(p)
@@ -163,11 +171,11 @@ def nnls(A, y, tol: Optional[float] = None, max_iter: Optional[int] = None,
         if first:
             first = False     # a warm start begins with the inner loop on its support
         else:
-            cand = (~passive) & (~blocked) & (g > tol)
+            cand = (~passive) & (~blocked) & (g > thr)
             if not cand.any():
                 break
             idx = np.flatnonzero(cand)
-            j = int(idx[np.argmax(g[idx])])        # argmax returns the lowest index on ties
+            j = int(idx[np.argmax(g[idx] / col[idx])])   # argmax returns the lowest index on ties
             passive[j] = True
         while True:
             it += 1

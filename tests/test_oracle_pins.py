@@ -151,6 +151,31 @@ def test_nnls_warm_start_reaches_the_same_minimiser(seed):
     np.testing.assert_allclose(cold, _nnls_by_enumeration(A, y), atol=1e-10)
 
 
+@pytest.mark.parametrize("seed", range(3))
+def test_nnls_reaches_the_minimiser_when_the_residual_is_tiny(seed):
+    """Brute force with columns of very different mass (one sink-like column
+    1e4 times the others, as attention features have): y = A[:, :5]x* + c·a_5
+    lies in the cone of A, and after the 5-column fit (also the warm start an
+    OMP refit begins from) a_5's gradient is ~1e-10·‖a_5‖‖y‖, far below
+    1e-13·‖A‖_F·‖y‖.  The minimiser (and the enumeration) reach residual ~0;
+    a stopping test on the raw gradient against ‖A‖_F·‖y‖ ends at ~1e-10·‖y‖."""
+    rng = np.random.default_rng(900 + seed)
+    n = 30
+    A = rng.random((n, 6)) + 0.2
+    A[:, 0] *= 1e4
+    x_true = rng.random(5) + 0.5
+    y = A[:, :5] @ x_true + 1e-5 * A[:, 5]
+    best = _nnls_by_enumeration(A, y)
+    rb = np.linalg.norm(A @ best - y)
+    assert rb < 1e-13 * np.linalg.norm(y)
+    x5 = np.linalg.lstsq(A[:, :5], y, rcond=None)[0]
+    for x0 in (None, np.concatenate([x5, [0.0]])):
+        x = O.nnls(A, y, x0=x0)
+        ry = np.linalg.norm(A @ x - y)
+        assert ry <= rb + 1e-13 * np.linalg.norm(y), (ry, rb)
+        assert x[5] > 0 and x.min() >= 0
+
+
 def test_nnls_single_column_closed_form():
     rng = np.random.default_rng(5)
     phi = rng.random(20)
