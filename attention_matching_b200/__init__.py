@@ -42,7 +42,8 @@ class AmError(RuntimeError):
 class AmWorkspaceView(ctypes.Structure):
     """Mirror of am_workspace_view_t."""
     _fields_ = [("phiT", ctypes.c_size_t), ("mass", ctypes.c_size_t), ("target", ctypes.c_size_t),
-                ("shift", ctypes.c_size_t), ("ldn", ctypes.c_int32), ("reserved", ctypes.c_int32)]
+                ("shift", ctypes.c_size_t), ("ldn", ctypes.c_int32), ("reserved", ctypes.c_int32),
+                ("weights", ctypes.c_size_t), ("resid", ctypes.c_size_t)]
 
 
 class AmOpts(ctypes.Structure):
@@ -135,13 +136,14 @@ def workspace_size(n: int, T: int, d: int, budgets: Sequence[int], opts: AmOpts)
 
 
 def features(out: Dict, n: int, T: int, d: int, budgets: Sequence[int], topk: int = 1,
-             refit_every: int = 1, dtype: int = BF16) -> Dict:
+             refit_every: int = 1, dtype: int = BF16, corr_mode: int = CORR_AUTO) -> Dict:
     """Views of the intermediate features a finished call left in its
     workspace: phiT [H, T, ldn] fp32, mass [H, ldn] fp64, target [H, n, d]
-    fp32, shift [H] fp32 (torch tensors sharing the workspace memory)."""
+    fp32, shift [H] fp32, weights [Σt] fp64 (last NNLS refit, pick order)
+    and resid [H, ldn] fp32 (torch tensors sharing the workspace memory)."""
     import torch
     H = len(budgets)
-    opts = make_opts(dtype, topk, refit_every)
+    opts = make_opts(dtype, topk, refit_every, corr_mode=corr_mode)
     v = AmWorkspaceView()
     rc = lib().am_workspace_view(n, T, d, H, _i32_array(budgets), ctypes.byref(opts), ctypes.byref(v))
     if rc:
@@ -157,6 +159,8 @@ def features(out: Dict, n: int, T: int, d: int, budgets: Sequence[int], topk: in
         "mass": view(v.mass, H * v.ldn, torch.float64).view(H, v.ldn),
         "target": view(v.target, H * n * d, torch.float32).view(H, n, d),
         "shift": view(v.shift, H, torch.float32),
+        "weights": view(v.weights, int(sum(budgets)), torch.float64),
+        "resid": view(v.resid, H * v.ldn, torch.float32).view(H, v.ldn),
         "ldn": v.ldn,
     }
 

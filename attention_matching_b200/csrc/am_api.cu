@@ -22,10 +22,10 @@ size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 
 struct Layout {
   // byte offsets from the workspace base
-  size_t tables, status, shift, np, mm, rr_part;
+  size_t tables, status, shift, np, ylen, mm, rr_part;
   size_t phiT, phiT16, m, Y, r, corr, sel;
   size_t picks, pick_corr, plist, sorted_slot;
-  size_t bvec, w, w_eff;
+  size_t bvec, w, w_eff, ycache;
   size_t G, L, AtA, A, AtY, nrm_part;
   size_t total;
   size_t tables_bytes;
@@ -50,6 +50,7 @@ Layout plan(int n, int T, int d, int H, int64_t sum_t, int64_t sum_t2, bool corr
   L.tables = take(L.tables_bytes);
   L.shift = take((size_t)H * 4);
   L.np = take((size_t)H * 4);
+  L.ylen = take((size_t)H * 4);
   L.mm = take((size_t)H * 8);
   L.rr_part = take((size_t)H * kRedBlocks * 8);
   L.phiT = take((size_t)H * T * ldn * 4);
@@ -66,6 +67,7 @@ Layout plan(int n, int T, int d, int H, int64_t sum_t, int64_t sum_t2, bool corr
   L.bvec = take((size_t)sum_t * 8);
   L.w = take((size_t)sum_t * 8);
   L.w_eff = take((size_t)sum_t * 8);
+  L.ycache = take((size_t)sum_t * 8);
   L.G = take((size_t)sum_t2 * 8);
   L.L = take((size_t)sum_t2 * 8);
   L.AtA = take((size_t)sum_t2 * 8);
@@ -126,6 +128,7 @@ Work bind(const Layout& L, char* base, bool corr_bf16) {
   w.status = reinterpret_cast<int32_t*>(base + L.status);
   w.shift = reinterpret_cast<float*>(base + L.shift);
   w.np = reinterpret_cast<int32_t*>(base + L.np);
+  w.ylen = reinterpret_cast<int32_t*>(base + L.ylen);
   w.mm = reinterpret_cast<double*>(base + L.mm);
   w.rr_part = reinterpret_cast<double*>(base + L.rr_part);
   w.phiT = reinterpret_cast<float*>(base + L.phiT);
@@ -141,6 +144,7 @@ Work bind(const Layout& L, char* base, bool corr_bf16) {
   w.bvec = reinterpret_cast<double*>(base + L.bvec);
   w.w = reinterpret_cast<double*>(base + L.w);
   w.w_eff = reinterpret_cast<double*>(base + L.w_eff);
+  w.ycache = reinterpret_cast<double*>(base + L.ycache);
   w.G = reinterpret_cast<double*>(base + L.G);
   w.L = reinterpret_cast<double*>(base + L.L);
   w.AtA = reinterpret_cast<double*>(base + L.AtA);
@@ -233,6 +237,8 @@ am_status_t am_workspace_view(int32_t n, int32_t T, int32_t d, int32_t num_heads
   view->shift = L.shift;
   view->ldn = round_up(n, 32);
   view->reserved = 0;
+  view->weights = L.w;
+  view->resid = L.r;
   return AM_OK;
 }
 

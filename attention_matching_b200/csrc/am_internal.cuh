@@ -55,10 +55,12 @@ struct Work {
   double* L;            // [Σt²] Cholesky factor scratch (global fallback)
   int32_t* plist;       // [Σt] NNLS passive list (factor order)
   int32_t* np;          // [H] passive count
+  int32_t* ylen;        // [H] leading length of ycache that is valid
   double* mm;           // [H] ‖m‖²
   double* rr_part;      // [H][kRedBlocks] partial ‖r‖²
   int32_t* sorted_slot; // [Σt] pick slot of each ascending-position output row
   double* w_eff;        // [Σt] floored weights, ascending-position order
+  double* ycache;       // [Σt] forward solve L⁻¹ b_P (factor order), kept across refits
   float* A;             // [Σt][ldn] design matrix, key-major
   double* AtA;          // [Σt²]
   double* AtY;          // [Σt][d]

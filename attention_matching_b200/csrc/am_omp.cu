@@ -39,6 +39,7 @@ __global__ void k_init(Problem p, Work w) {
   if (threadIdx.x == 0) {
     w.mm[h] = acc;
     w.np[h] = 0;
+    w.ylen[h] = 0;
     if (!(acc > 0.0) || !isfinite(acc)) record_status(w.status + h, AM_ERR_NONFINITE);
   }
   uint8_t* sel = w.sel + (int64_t)h * p.T;
@@ -291,53 +292,253 @@ __global__ void __launch_bounds__(256) k_gram(Problem p, Work w, int pass) {
 // the current factor run on separate warps, then a small Cholesky of their
 // Schur complement finishes the new rows.  If an entering block holds a
 // variable that will not grow, the refit continues one variable at a time.
+// A variable that leaves the passive set is deleted from the factor by a
+// rank-one update of the rows below it (no refactorisation), and the forward
+// solve y = L⁻¹ b_P is kept (also across refits) for every factor row above
+// the first one that changed, so each solve only extends it.
 // Triangular solves multiply by stored reciprocal diagonals.
+constexpr int kSB = 32;        // rows per block of the blocked triangular solves
+constexpr int kMaxRhs = 8;     // vectors one blocked forward solve carries
+constexpr size_t kDiagTileBytes = kSB * (kSB + 1) * sizeof(double);
+
 __host__ __device__ inline size_t nnls_vec_bytes(int t) {
-  // x, z, g, invd: 4t doubles; red: 64 doubles; ctl: 16 ints; P, inP, blocked, add, cand: 5t ints
-  size_t b = (size_t)t * 4 * sizeof(double) + 64 * sizeof(double) + 16 * sizeof(int) + (size_t)t * 5 * sizeof(int);
+  // x, z, g, invd, y: 5t doubles; red: 64 doubles; diagonal tile: 32×33 doubles;
+  // ctl: 16 ints; P, inP, blocked, add, cand: 5t ints
+  size_t b = (size_t)t * 5 * sizeof(double) + 64 * sizeof(double) + kDiagTileBytes + 16 * sizeof(int) +
+             (size_t)t * 5 * sizeof(int);
   return (b + 15) & ~size_t(15);
 }
 __host__ __device__ inline size_t nnls_tri_bytes(int t) { return (size_t)t * (t + 1) / 2 * sizeof(double); }
 constexpr size_t kSmemCap = 227 * 1024;
 
-// v ← L⁻¹ v (one warp)
-__device__ __forceinline__ void warp_fwd(const double* L, const double* invd, double* v, int n) {
-  const int lane = threadIdx.x & 31;
-  for (int k = 0; k < n; ++k) {
-    const double yk = v[k] * invd[k];
-    __syncwarp();
-    if (lane == 0) v[k] = yk;
-    for (int i = k + 1 + lane; i < n; i += 32) v[i] -= L[tri(i, k)] * yk;
-    __syncwarp();
+// Blocked triangular solves with the packed factor (shared or global
+// memory), run by all threads of the block, 32 rows at a time.  Each block of
+// rows takes the products with every solved entry in one parallel pass whose
+// factor reads are coalesced (lanes run along a factor row), then one warp per
+// vector sweeps the 32×32 diagonal block, staged in shared memory.
+typedef double DiagTile[kSB + 1];
+
+// dst[0..n) = src[0..n) by all threads, four loads per thread in flight.
+__device__ __forceinline__ void copy_doubles(double* dst, const double* src, int64_t n) {
+  for (int64_t e0 = threadIdx.x; e0 < n; e0 += 4 * (int64_t)blockDim.x) {
+    double v[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int64_t e = e0 + (int64_t)u * blockDim.x;
+      v[u] = e < n ? src[e] : 0.0;
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int64_t e = e0 + (int64_t)u * blockDim.x;
+      if (e < n) dst[e] = v[u];
+    }
   }
 }
 
-// v ← L⁻¹ v (one warp), row form: y_k = (v_k − L[k, :k]·y[:k]) / L_kk.  Each
-// step reads one contiguous factor row (coalesced when the factor is in
-// global memory) and reduces across the warp.
-__device__ __forceinline__ void warp_fwd_rows(const double* L, const double* invd, double* v, int n) {
-  const int lane = threadIdx.x & 31;
-  for (int k = 0; k < n; ++k) {
-    const double* row = L + tri(k, 0);
-    double acc = 0.0;
-    for (int j = lane; j < k; j += 32) acc += row[j] * v[j];
-    acc = warp_sum(acc);
-    if (lane == 0) v[k] = (v[k] - acc) * invd[k];
-    __syncwarp();
+// D[r][c] = L[r0 + r][r0 + c] for c <= r < bw, zero elsewhere.
+__device__ __forceinline__ void load_diag_tile(const double* L, int r0, int bw, DiagTile* D) {
+  for (int e = threadIdx.x; e < kSB * kSB; e += blockDim.x) {
+    const int r = e >> 5, c = e & 31;
+    D[r][c] = (r < bw && c <= r) ? L[tri(r0 + r, r0 + c)] : 0.0;
   }
 }
 
-// v ← L⁻ᵀ v (one warp)
-__device__ __forceinline__ void warp_bwd(const double* L, const double* invd, double* v, int n) {
-  const int lane = threadIdx.x & 31;
-  for (int k = n - 1; k >= 0; --k) {
-    const double zk = v[k] * invd[k];
-    __syncwarp();
-    if (lane == 0) v[k] = zk;
-    const double* row = L + tri(k, 0);
-    for (int i = lane; i < k; i += 32) v[i] -= row[i] * zk;
-    __syncwarp();
+// u_e ← L⁻¹ u_e on rows [k0, n) for the R <= 8 vectors U[0..R); entries
+// below k0 are already final.  Products: warp w takes rows r0 + 4w .. +3,
+// its lanes run across the solved columns.
+__device__ void block_forward(const double* L, const double* invd, double* const* U, int R, int k0, int n,
+                              DiagTile* D) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  for (int r0 = k0; r0 < n; r0 += kSB) {
+    const int bw = min(kSB, n - r0);
+    load_diag_tile(L, r0, bw, D);
+    const int rb = r0 + 4 * warp;
+    if (4 * warp < bw && r0 > 0) {
+      const double* lr[4];
+      bool live[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        live[i] = 4 * warp + i < bw;
+        lr[i] = L + tri(live[i] ? rb + i : rb, 0);
+      }
+      double acc[4][kMaxRhs];
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int e = 0; e < kMaxRhs; ++e) acc[i][e] = 0.0;
+      for (int j0 = lane; j0 < r0; j0 += 32 * 4) {   // four columns per lane in flight
+#pragma unroll
+        for (int s = 0; s < 4; ++s) {
+          const int j = j0 + 32 * s;
+          if (j < r0) {
+            double uj[kMaxRhs];
+#pragma unroll
+            for (int e = 0; e < kMaxRhs; ++e) uj[e] = e < R ? U[e][j] : 0.0;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              const double l = live[i] ? lr[i][j] : 0.0;
+#pragma unroll
+              for (int e = 0; e < kMaxRhs; ++e) acc[i][e] = fma(l, uj[e], acc[i][e]);
+            }
+          }
+        }
+      }
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int e = 0; e < kMaxRhs; ++e)
+          if (e < R) {
+            const double sum = warp_sum(acc[i][e]);
+            if (lane == 0 && live[i]) U[e][rb + i] -= sum;
+          }
+    }
+    __syncthreads();
+    if (warp < R) {
+      double* u = U[warp];
+      double v = lane < bw ? u[r0 + lane] : 0.0;
+      for (int c = 0; c < bw; ++c) {
+        if (lane == c) v *= invd[r0 + c];
+        const double vc = __shfl_sync(0xffffffffu, v, c);
+        if (lane > c) v -= D[lane][c] * vc;
+      }
+      if (lane < bw) u[r0 + lane] = v;
+    }
+    __syncthreads();
   }
+}
+
+// v ← L⁻ᵀ v on rows [0, n).  Blocks from the bottom: one warp sweeps the
+// diagonal block, then every row above takes that block's contribution
+// (threads across columns, each summing over the block's 32 factor rows).
+__device__ void block_backward(const double* L, const double* invd, double* v, int n, DiagTile* D) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  for (int b = (n + kSB - 1) / kSB - 1; b >= 0; --b) {
+    const int r0 = b * kSB, bw = min(kSB, n - r0);
+    load_diag_tile(L, r0, bw, D);
+    __syncthreads();
+    if (warp == 0) {
+      double x = lane < bw ? v[r0 + lane] : 0.0;
+      for (int c = bw - 1; c >= 0; --c) {
+        if (lane == c) x *= invd[r0 + c];
+        const double xc = __shfl_sync(0xffffffffu, x, c);
+        if (lane < c) x -= D[c][lane] * xc;
+      }
+      if (lane < bw) v[r0 + lane] = x;
+    }
+    __syncthreads();
+    for (int j = tid; j < r0; j += blockDim.x) {
+      const double* col = L + tri(r0, 0) + j;   // L[r0 + r][j] = col[r·r0 + r(r+1)/2]
+      double acc[4] = {0.0, 0.0, 0.0, 0.0};
+#pragma unroll
+      for (int r = 0; r < kSB; ++r)
+        if (r < bw) acc[r & 3] = fma(col[(int64_t)r * r0 + r * (r + 1) / 2], v[r0 + r], acc[r & 3]);
+      v[j] -= (acc[0] + acc[1]) + (acc[2] + acc[3]);
+    }
+    __syncthreads();
+  }
+}
+
+// Deletes position q from the packed factor L of an np×np matrix (all
+// threads of the block).  Writing L = [L11 · ·; l21ᵀ l22 ·; L31 l32 L33],
+// the matrix without row and column q has the factor [L11 ·; L31 L̃33] with
+// L̃33 L̃33ᵀ = L33 L33ᵀ + l32 l32ᵀ: the classic rank-one Cholesky update,
+// one plane rotation per column of L33.  The rotations are formed sixteen
+// columns at a time by one warp on the diagonal block, then applied by every
+// thread to one trailing row at a time.  Last, the rows below q move up one
+// slot and lose column q.  xv (m doubles) and rot (48 doubles) are scratch.
+constexpr int kRotBlock = 16;
+constexpr int kMoveRegs = 8;
+
+__device__ __forceinline__ int tri_row(int64_t e) {
+  // row of packed index e (e < 2^23: exact in fp32, then corrected)
+  int r = (int)((sqrtf(8.0f * (float)e + 1.0f) - 1.0f) * 0.5f);
+  while (tri(r + 1, 0) <= e) ++r;
+  while (tri(r, 0) > e) --r;
+  return r;
+}
+
+__device__ void factor_remove(double* L, double* invd, double* xv, double* rot, int q, int np) {
+  const int tid = threadIdx.x, nthr = blockDim.x, lane = tid & 31, warp = tid >> 5;
+  const int m = np - 1 - q;   // trailing rows: old indices o .. np-1
+  const int o = q + 1;
+  for (int a = tid; a < m; a += nthr) xv[a] = L[tri(o + a, q)];
+  __syncthreads();
+  for (int J = 0; J < m; J += kRotBlock) {
+    const int jw = min(kRotBlock, m - J);
+    if (warp == 0) {
+      // lane e holds trailing row J+e, columns J .. J+e
+      const bool mine = lane < jw;
+      double* row = L + tri(o + J + (mine ? lane : 0), o + J);
+      double v[kRotBlock];
+#pragma unroll
+      for (int c = 0; c < kRotBlock; ++c) v[c] = (mine && c <= lane) ? row[c] : 0.0;
+      double xr = mine ? xv[J + lane] : 0.0;
+#pragma unroll
+      for (int k = 0; k < kRotBlock; ++k) {
+        if (k < jw) {
+          const double lkk = __shfl_sync(0xffffffffu, v[k], k);
+          const double xk = __shfl_sync(0xffffffffu, xr, k);
+          const double r = hypot(lkk, xk);
+          const double c = r / lkk, sn = xk / lkk, ic = lkk / r;
+          if (lane == k) v[k] = r;
+          if (mine && lane > k) {
+            v[k] = (v[k] + sn * xr) * ic;
+            xr = c * xr - sn * v[k];
+          }
+          if (lane == 0) { rot[3 * k] = c; rot[3 * k + 1] = sn; rot[3 * k + 2] = ic; }
+        }
+      }
+      if (mine) {
+#pragma unroll
+        for (int c = 0; c < kRotBlock; ++c)
+          if (c <= lane) row[c] = v[c];
+      }
+    }
+    __syncthreads();
+    for (int a = J + jw + tid; a < m; a += nthr) {
+      double* row = L + tri(o + a, o + J);
+      double v[kRotBlock];
+#pragma unroll
+      for (int c = 0; c < kRotBlock; ++c) v[c] = c < jw ? row[c] : 0.0;
+      double xa = xv[a];
+#pragma unroll
+      for (int k = 0; k < kRotBlock; ++k) {
+        if (k < jw) {
+          v[k] = (v[k] + rot[3 * k + 1] * xa) * rot[3 * k + 2];
+          xa = rot[3 * k] * xa - rot[3 * k + 1] * v[k];
+        }
+      }
+#pragma unroll
+      for (int c = 0; c < kRotBlock; ++c)
+        if (c < jw) row[c] = v[c];
+      xv[a] = xa;
+    }
+    __syncthreads();
+  }
+  // New row r >= q is old row r+1 without column q; it fills exactly the
+  // slot of old row r, so the move runs in chunks, each read before written.
+  const int64_t f0 = tri(q, 0), f1 = tri(np - 1, 0);
+  for (int64_t e0 = f0; e0 < f1; e0 += (int64_t)nthr * kMoveRegs) {
+    double v[kMoveRegs];
+#pragma unroll
+    for (int u = 0; u < kMoveRegs; ++u) {
+      const int64_t e = e0 + (int64_t)u * nthr + tid;
+      if (e < f1) {
+        const int r = tri_row(e);
+        const int c = (int)(e - tri(r, 0));
+        v[u] = L[tri(r + 1, c + (c >= q))];
+      }
+    }
+    __syncthreads();
+#pragma unroll
+    for (int u = 0; u < kMoveRegs; ++u) {
+      const int64_t e = e0 + (int64_t)u * nthr + tid;
+      if (e < f1) L[e] = v[u];
+    }
+    __syncthreads();
+  }
+  for (int r = q + tid; r < np - 1; r += nthr) invd[r] = 1.0 / L[tri(r, r)];
+  __syncthreads();
 }
 
 __global__ void __launch_bounds__(kNnlsThreads) k_nnls(Problem p, Work w, int pass, int l_in_smem_max) {
@@ -358,8 +559,10 @@ __global__ void __launch_bounds__(kNnlsThreads) k_nnls(Problem p, Work w, int pa
   double* z = x + t;                             // factor-position indexed solve buffer
   double* g = z + t;                             // scaled gradient
   double* invd = g + t;                          // 1 / L_qq
-  double* red = invd + t;                        // 64 doubles
-  int* ctl = reinterpret_cast<int*>(red + 64);   // 16 ints
+  double* yv = invd + t;                         // forward solve L⁻¹ b_P, valid below ctl[10]
+  double* red = yv + t;                          // 64 doubles
+  DiagTile* D = reinterpret_cast<DiagTile*>(red + 64);              // solve scratch
+  int* ctl = reinterpret_cast<int*>(red + 64 + kSB * (kSB + 1));    // 16 ints
   int* P = ctl + 16;
   int* inP = P + t;
   int* blocked = inP + t;
@@ -368,7 +571,7 @@ __global__ void __launch_bounds__(kNnlsThreads) k_nnls(Problem p, Work w, int pa
   const bool l_smem = t <= l_in_smem_max;
   double* Lg = w.L + gbase;
   double* L = l_smem ? reinterpret_cast<double*>(smem + nnls_vec_bytes(t)) : Lg;
-  // ctl: 0 np, 1 nadd, 2 single mode, 4 argmin, 5 nneg, 6 factor flag, 7 ncand, 8 append failures
+  // ctl: 0 np, 1 nadd, 2 single mode, 4 argmin, 5 nneg, 7 ncand, 9 removed count, 10 valid y rows
   const int maxit = p.nnls_max_iter > 0 ? p.nnls_max_iter : 3 * t + 50;
   const double mnorm = sqrt(w.mm[h]);
   auto diag = [&](int l) { return G[(int64_t)l * t + l]; };
@@ -379,43 +582,16 @@ __global__ void __launch_bounds__(kNnlsThreads) k_nnls(Problem p, Work w, int pa
     blocked[l] = 0;
   }
   for (int q = tid; q < np_old; q += blockDim.x) P[q] = w.plist[base + q];
-  if (l_smem)
-    for (int64_t e = tid; e < tri(np_old, 0); e += blockDim.x) L[e] = Lg[e];
-  if (tid == 0) { ctl[0] = np_old; ctl[2] = 0; }
+  const int ylen0 = min(w.ylen[h], np_old);
+  for (int q = tid; q < ylen0; q += blockDim.x) yv[q] = w.ycache[base + q];
+  if (l_smem) copy_doubles(L, Lg, tri(np_old, 0));
+  if (tid == 0) { ctl[0] = np_old; ctl[2] = 0; ctl[10] = ylen0; }
   __syncthreads();
   for (int q = tid; q < np_old; q += blockDim.x) {
     inP[P[q]] = 1;
     invd[q] = 1.0 / L[tri(q, q)];
   }
   __syncthreads();
-
-  // Rebuild the factor of G[P, P] from scratch; drops dependent variables.
-  auto refactor = [&]() {
-    for (;;) {
-      const int np = ctl[0];
-      for (int a = warp; a < np; a += nw)
-        for (int c = lane; c <= a; c += 32) L[tri(a, c)] = G[(int64_t)P[a] * t + P[c]];
-      __syncthreads();
-      auto floor_k = [&](int k) { return 1e-13 * diag(P[k]); };
-      // a factor in the workspace is rebuilt tile by tile (shared memory as scratch)
-      int badk = l_smem ? block_cholesky_packed(L, np, floor_k, &ctl[6])
-                        : block_cholesky_tiled(L, np, floor_k, reinterpret_cast<double*>(smem + nnls_vec_bytes(t)), &ctl[6]);
-      if (badk < 0) {
-        for (int q = tid; q < np; q += blockDim.x) invd[q] = 1.0 / L[tri(q, q)];
-        __syncthreads();
-        return;
-      }
-      if (tid == 0) {
-        const int l = P[badk];
-        inP[l] = 0;
-        blocked[l] = 1;
-        x[l] = 0.0;
-        for (int q = badk; q + 1 < np; ++q) P[q] = P[q + 1];
-        ctl[0] = np - 1;
-      }
-      __syncthreads();
-    }
-  };
 
   // Append add[0..nadd) to the factor as a block; variables whose Schur
   // pivot is too small are blocked and the block is redone without them.
@@ -430,11 +606,13 @@ __global__ void __launch_bounds__(kNnlsThreads) k_nnls(Problem p, Work w, int pa
         for (int q = lane; q < np; q += 32) row[q] = Ge[P[q]];
       }
       __syncthreads();
-      for (int e = warp; e < k; e += nw) {
-        if (l_smem) warp_fwd(L, invd, L + tri(np + e, 0), np);
-        else warp_fwd_rows(L, invd, L + tri(np + e, 0), np);
+      for (int e0 = 0; e0 < k; e0 += kMaxRhs) {
+        const int R = min(kMaxRhs, k - e0);
+        double* U[kMaxRhs];
+#pragma unroll
+        for (int e = 0; e < kMaxRhs; ++e) U[e] = L + tri(np + e0 + min(e, R - 1), 0);
+        block_forward(L, invd, U, R, 0, np, D);
       }
-      __syncthreads();
       // Schur complement of the new block (lower triangle)
       for (int pr = warp; pr < k * (k + 1) / 2; pr += nw) {
         int e = 0;
@@ -448,30 +626,52 @@ __global__ void __launch_bounds__(kNnlsThreads) k_nnls(Problem p, Work w, int pa
         if (lane == 0) L[tri(np + e, np + f)] = G[(int64_t)add[e] * t + add[f]] - acc;
       }
       __syncthreads();
-      if (tid == 0) {
+      // Cholesky of the k×k Schur block: lane e owns new row e (lane 0 alone
+      // for k > 32); a pivot at or below 1e-13·G_ll blocks that variable
+      if (warp == 0) {
         int failed = 0;
+        const bool wide = k <= 32;
         for (int f = 0; f < k; ++f) {
           const double piv = L[tri(np + f, np + f)];
-          if (!(piv > 1e-13 * diag(add[f]))) { blocked[add[f]] = 1; ++failed; break; }
-          const double lff = sqrt(piv);
-          L[tri(np + f, np + f)] = lff;
-          invd[np + f] = 1.0 / lff;
-          for (int e = f + 1; e < k; ++e) L[tri(np + e, np + f)] /= lff;
-          for (int e = f + 1; e < k; ++e)
-            for (int q = f + 1; q <= e; ++q) L[tri(np + e, np + q)] -= L[tri(np + e, np + f)] * L[tri(np + q, np + f)];
-        }
-        if (failed) {
-          int kk = 0;
-          for (int e = 0; e < k; ++e)
-            if (!blocked[add[e]]) add[kk++] = add[e];
-          ctl[1] = kk;
-        } else {
-          for (int e = 0; e < k; ++e) {
-            P[np + e] = add[e];
-            inP[add[e]] = 1;
+          if (!(piv > 1e-13 * diag(add[f]))) {
+            if (lane == 0) blocked[add[f]] = 1;
+            failed = 1;
+            break;
           }
-          ctl[0] = np + k;
-          ctl[1] = 0;
+          const double lff = sqrt(piv), il = 1.0 / lff;
+          __syncwarp();
+          if (lane == 0) { L[tri(np + f, np + f)] = lff; invd[np + f] = il; }
+          if (wide) {
+            const int e = lane;
+            if (e > f && e < k) L[tri(np + e, np + f)] *= il;
+            __syncwarp();
+            if (e > f && e < k) {
+              const double lef = L[tri(np + e, np + f)];
+              for (int q = f + 1; q <= e; ++q) L[tri(np + e, np + q)] -= lef * L[tri(np + q, np + f)];
+            }
+          } else if (lane == 0) {
+            for (int e = f + 1; e < k; ++e) L[tri(np + e, np + f)] *= il;
+            for (int e = f + 1; e < k; ++e) {
+              const double lef = L[tri(np + e, np + f)];
+              for (int q = f + 1; q <= e; ++q) L[tri(np + e, np + q)] -= lef * L[tri(np + q, np + f)];
+            }
+          }
+          __syncwarp();
+        }
+        if (lane == 0) {
+          if (failed) {
+            int kk = 0;
+            for (int e = 0; e < k; ++e)
+              if (!blocked[add[e]]) add[kk++] = add[e];
+            ctl[1] = kk;
+          } else {
+            for (int e = 0; e < k; ++e) {
+              P[np + e] = add[e];
+              inP[add[e]] = 1;
+            }
+            ctl[0] = np + k;
+            ctl[1] = 0;
+          }
         }
       }
       __syncthreads();
@@ -501,9 +701,15 @@ __global__ void __launch_bounds__(kNnlsThreads) k_nnls(Problem p, Work w, int pa
     for (int ci = warp; ci < nc; ci += nw) {
       const int l = cand[ci];
       const double* Gl = G + (int64_t)l * t;
-      double acc = 0.0;
-      for (int q = lane; q < np; q += 32) acc += Gl[P[q]] * z[q];
-      acc = warp_sum(acc);
+      double a4[4] = {0.0, 0.0, 0.0, 0.0};
+      for (int q0 = lane; q0 < np; q0 += 128) {
+#pragma unroll
+        for (int s = 0; s < 4; ++s) {
+          const int q = q0 + 32 * s;
+          if (q < np) a4[s] = fma(Gl[P[q]], z[q], a4[s]);
+        }
+      }
+      const double acc = warp_sum((a4[0] + a4[1]) + (a4[2] + a4[3]));
       if (lane == 0) {
         const double dl = diag(l);
         g[l] = dl > 0.0 ? (b[l] - acc) / (sqrt(dl) * mnorm) : -INFINITY;
@@ -511,7 +717,9 @@ __global__ void __launch_bounds__(kNnlsThreads) k_nnls(Problem p, Work w, int pa
     }
     __syncthreads();
     if (warp == 0) {
-      const double tol = 1e-11;
+      // enter while g_l / (‖φ_l‖·‖m‖) > 1e-12; the rounding of b_l − G_l x
+      // in fp64 stays near 1e-14 on this scale
+      const double tol = 1e-12;
       int nadd = 0;
       if (ctl[2]) {                                    // single mode: argmax only
         double bv = tol;
@@ -546,15 +754,17 @@ __global__ void __launch_bounds__(kNnlsThreads) k_nnls(Problem p, Work w, int pa
     bool abort = false;
     for (;;) {
       if (++iter > maxit) { abort = true; break; }
-      const int npc = ctl[0];
-      for (int q = tid; q < npc; q += blockDim.x) z[q] = b[P[q]];
+      const int npc = ctl[0], y0 = ctl[10];
+      // z = y on the cached rows; the forward solve extends it over the rest
+      for (int q = tid; q < npc; q += blockDim.x) z[q] = q < y0 ? yv[q] : b[P[q]];
       __syncthreads();
-      if (warp == 0) {
-        if (l_smem) warp_fwd(L, invd, z, npc);
-        else warp_fwd_rows(L, invd, z, npc);
-        warp_bwd(L, invd, z, npc);
+      {
+        double* U[kMaxRhs] = {z, z, z, z, z, z, z, z};
+        block_forward(L, invd, U, 1, y0, npc, D);
       }
-      __syncthreads();
+      for (int q = y0 + tid; q < npc; q += blockDim.x) yv[q] = z[q];
+      if (tid == 0) ctl[10] = npc;
+      block_backward(L, invd, z, npc, D);
       double best = INFINITY;
       int bq = -1, nneg = 0;
       for (int q = tid; q < npc; q += blockDim.x) {
@@ -602,19 +812,21 @@ __global__ void __launch_bounds__(kNnlsThreads) k_nnls(Problem p, Work w, int pa
       if (alpha == 0.0) {
         // entering variables that will not grow: drop them
         if (tid == 0) {
-          int kk = 0;
+          int kk = 0, nrm = 0;
           const bool single = ctl[2];
           for (int q = 0; q < npc; ++q) {
             const int l = P[q];
             if (!(z[q] > 0.0) && x[l] == 0.0) {
               inP[l] = 0;
               if (single) blocked[l] = 1;
+              cand[nrm++] = q;
             } else {
               P[kk++] = l;
             }
           }
           ctl[0] = kk;
           ctl[2] = 1;
+          ctl[9] = nrm;
         }
       } else {
         const int qmin = ctl[4];
@@ -626,17 +838,22 @@ __global__ void __launch_bounds__(kNnlsThreads) k_nnls(Problem p, Work w, int pa
         }
         __syncthreads();
         if (tid == 0) {
-          int kk = 0;
+          int kk = 0, nrm = 0;
           for (int q = 0; q < npc; ++q) {
             const int l = P[q];
-            if (x[l] <= 0.0) { inP[l] = 0; x[l] = 0.0; }
+            if (x[l] <= 0.0) { inP[l] = 0; x[l] = 0.0; cand[nrm++] = q; }
             else P[kk++] = l;
           }
           ctl[0] = kk;
+          ctl[9] = nrm;
         }
       }
       __syncthreads();
-      refactor();
+      // delete the leavers from the factor, last position first
+      const int nrm = ctl[9];
+      for (int i = nrm - 1, npr = ctl[0] + nrm; i >= 0; --i, --npr) factor_remove(L, invd, g, red, cand[i], npr);
+      if (tid == 0 && nrm > 0) ctl[10] = min(ctl[10], cand[0]);
+      __syncthreads();
     }
     if (abort) break;
   }
@@ -646,10 +863,12 @@ __global__ void __launch_bounds__(kNnlsThreads) k_nnls(Problem p, Work w, int pa
   const int npf = ctl[0];
   for (int l = tid; l < s1; l += blockDim.x) w.w[base + l] = inP[l] ? x[l] : 0.0;
   for (int q = tid; q < npf; q += blockDim.x) w.plist[base + q] = P[q];
-  if (l_smem)
-    for (int64_t e = tid; e < tri(npf, 0); e += blockDim.x) Lg[e] = L[e];
+  const int yl = ctl[10];
+  for (int q = tid; q < yl; q += blockDim.x) w.ycache[base + q] = yv[q];
+  if (l_smem) copy_doubles(Lg, L, tri(npf, 0));
   if (tid == 0) {
     w.np[h] = npf;
+    w.ylen[h] = yl;
     if (!converged) record_status(w.status + h, AM_WARN_NOT_CONVERGED);
   }
 }

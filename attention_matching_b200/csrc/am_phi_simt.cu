@@ -204,11 +204,12 @@ __global__ void __launch_bounds__(256) k_y_m(Problem p, const void* V, const flo
   for (int a = 0; a < 4; ++a) {
     int i = i0 + tx * 4 + a;
     const double mi = msum[tx * 4 + a];
+    const double im = mi > 0.0 ? 1.0 / mi : 0.0;   // no mass (all features underflowed): zero target
     if (i < p.n) {
 #pragma unroll
       for (int c = 0; c < DPT; ++c) {
         int cc = ty * DPT + c;
-        if (cc < p.d) Y[((int64_t)h * p.n + i) * p.d + cc] = (float)((double)acc[a][c] / mi);
+        if (cc < p.d) Y[((int64_t)h * p.n + i) * p.d + cc] = (float)((double)acc[a][c] * im);
       }
     }
     if (ty == 0 && i < p.ldn) {

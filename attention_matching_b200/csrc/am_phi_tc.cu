@@ -478,11 +478,13 @@ k_phi_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtens
           tmem_ld32(tY + lane_addr + cb, y);
           tmem_wait_ld();
           if (row_live) {
+            // a query whose every feature underflowed has no mass: zero target
+            const double im = mtot > 0.0 ? 1.0 / mtot : 0.0;
 #pragma unroll
             for (int cc = 0; cc < 32; cc += 4)
               *reinterpret_cast<float4*>(yrow + cb + cc) =
-                  make_float4((float)(y[cc] / mtot), (float)(y[cc + 1] / mtot), (float)(y[cc + 2] / mtot),
-                              (float)(y[cc + 3] / mtot));
+                  make_float4((float)(y[cc] * im), (float)(y[cc + 1] * im), (float)(y[cc + 2] * im),
+                              (float)(y[cc + 3] * im));
           }
         }
         if (half == 0 && i < p.ldn) {

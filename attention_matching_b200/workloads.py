@@ -13,6 +13,10 @@ nor the weights are available, so heads shaped like those models stand in:
 * ``structured`` - per head a rank-32 key subspace: K = 2·U·Bᵀ + 0.3·E,
   four large-norm "sink" keys at positions 0-3, reference queries that are
   Dirichlet mixtures of four random keys plus 0.3·noise, V ~ N(0,1).
+* ``twin keys`` - a structured head whose every key is followed by a jittered
+  copy (repeated tokens); OMP then picks near-duplicate pairs and the NNLS
+  refits keep moving weight between them, so variables leave the passive set
+  often (a stress case for the refit rather than a page workload).
 
 All draws use ``numpy.random.default_rng(seed)`` (PCG64) in float64 and are
 then rounded once to the storage dtype (fp32, or bf16 round-to-nearest-even
@@ -116,6 +120,22 @@ def structured_head(seed: int, n: int, T: int, d: int = 128, rank: int = 32,
     Q = _mixture_queries(rng, Kr, n, first=min(sinks, T - 1))
     V = rng.standard_normal((T, d))
     return Head(round_to(Q, dtype), round_to(K, dtype), round_to(V, dtype))
+
+
+def twin_keys_head(seed: int, n: int, T: int, jitter: float = 0.3, d: int = 128,
+                   dtype: str = "bf16") -> Head:
+    """A structured head of T//2 keys (its own queries and values), each key
+    followed by a copy plus jitter·N(0,1) noise with a fresh N(0,1) value:
+    keys 2i and 2i+1 are near duplicates.  T must be even."""
+    base = structured_head(seed, n=n, T=T // 2, d=d, dtype=dtype)
+    rng = np.random.default_rng(seed + 7777)
+    K0, V0 = upcast(base.K), upcast(base.V)
+    K = np.empty((T, d))
+    V = np.empty((T, d))
+    K[0::2], V[0::2] = K0, V0
+    K[1::2] = K0 + jitter * rng.standard_normal(K0.shape)
+    V[1::2] = rng.standard_normal(V0.shape)
+    return Head(base.Q.clone(), round_to(K, dtype), round_to(V, dtype))
 
 
 def long_sequence_chunks(seed: int, T_total: int, chunk: int, n: int, d: int = 128,
@@ -269,7 +289,9 @@ class OnlineHeads:
                 K = np.vstack([np.asarray(Ck, np.float64), kept_K, Kf])
                 V = np.vstack([upcast(round_to(np.asarray(Cv, np.float64), self.dtype)), kept_V, Vf])
                 bias = np.concatenate([np.asarray(beta, np.float64), np.zeros(self.keep + nf)])
-            Q = _mixture_queries(self.rngs[h], K, self.n, first=4 if self.round == 0 else 0)
+            # the four sink keys lead the cache in the first round and, being
+            # selected first, lead every compacted block after it
+            Q = _mixture_queries(self.rngs[h], K, self.n, first=4)
             self.prev = (self.prev or [None] * self.H)
             self.prev[h] = (K, V, bias)
             c = self.compact_len

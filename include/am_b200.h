@@ -148,11 +148,15 @@ am_status_t am_compact_heads(const void* Q_ref, const void* K, const void* V,
  *   target  fp32 [H][n][d]    Y_i = Σ_j Φ_ij V_j / m_i
  *   shift   fp32 [H]          c_h used
  *   ldn     n rounded up to a multiple of 32
+ *   weights fp64 [Σt]         the last NNLS refit's w, packed per head at
+ *                             out_offsets[h] in PICK order (zero where w_l = 0)
+ *   resid   fp32 [H][ldn]     r = m − Φ_S w after the last refit
  * Same argument rules as am_workspace_size. */
 typedef struct am_workspace_view {
   size_t phiT, mass, target, shift;
   int32_t ldn;
   int32_t reserved;
+  size_t weights, resid;
 } am_workspace_view_t;
 
 am_status_t am_workspace_view(int32_t n, int32_t T, int32_t d, int32_t num_heads,

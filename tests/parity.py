@@ -119,3 +119,21 @@ def check_head(g, Q, K, V, t, topk, refit, shift, key_bias=None, oracle_res=None
 def shift_for(Q, K, key_bias=None):
     """The shared per-head shift: max logit in float64, rounded to fp32."""
     return float(np.float32(O.max_logit(Q, K, key_bias=key_bias)))
+
+
+def check_refit_kkt(out, feats, h, n, tol=1e-10):
+    """The last NNLS refit of head h, as the GPU holds it in fp64 (pick order),
+    satisfies the optimality conditions of min_{w>=0} ‖Φ_S w − m‖ on the GPU's
+    own stored features and mass: w >= 0, zero gradient on the support and no
+    descent direction off it, each relative to ‖φ_l‖·‖m‖.  With the refit's
+    unique minimising residual this pins the solver, independent of the
+    oracle's rounding."""
+    a, b = int(out["cu_t"][h]), int(out["cu_t"][h + 1])
+    picks = np.asarray(out["pick_order"][a:b].cpu().numpy(), np.int64)
+    w = feats["weights"][a:b].cpu().numpy()
+    Phi = feats["phiT"][h, :, :n].cpu().double().numpy().T
+    m = feats["mass"][h, :n].cpu().numpy()
+    kkt = O.nnls_kkt_residual(Phi[:, picks], m, w)
+    assert kkt["min_x"] >= 0.0, kkt
+    assert kkt["stationarity"] < tol and kkt["dual_feasibility"] < tol, kkt
+    return kkt

@@ -6,7 +6,7 @@ import torch
 
 from attention_matching_b200 import workloads as W
 from oracle import am_oracle as O
-from tests.parity import check_head, shift_for, split_head
+from tests.parity import check_refit_kkt, check_head, shift_for, split_head
 
 pytestmark = pytest.mark.gpu
 
@@ -204,6 +204,42 @@ def test_recompute_and_stored_correlations_agree():
     b = run_gpu(heads, [6, 6], 4, 2, corr_mode=am.CORR_STORED_FP32)
     assert torch.equal(a["indices"], b["indices"])
     torch.testing.assert_close(a["pick_corr"], b["pick_corr"], rtol=2e-5, atol=0)
+
+
+@needs_cuda
+def test_large_budget_global_factor():
+    """Budgets above what shared memory holds: the NNLS and value-fit
+    Cholesky factors live in the workspace instead (the regime of online
+    rounds and full-model schedules, t up to about 1000)."""
+    heads = [W.structured_head(390 + h, n=1536, T=1400) for h in range(2)]
+    check_all(heads, [300, 250], 4, 2, label="large t")
+
+
+@needs_cuda
+def test_kv_chunked_long_sequence():
+    """KV-based chunking: one long sequence cut into contiguous chunks that are
+    compacted independently (sinks only in the first chunk); chunks of equal
+    length share a call, the shorter last chunk gets its own."""
+    chunks = W.long_sequence_chunks(395, T_total=2500, chunk=1024, n=768)
+    assert [c.T for c in chunks] == [1024, 1024, 452]
+    check_all(chunks[:2], [103, 103], 8, 2, label="chunks 0-1")
+    check_all(chunks[2:], [46], 8, 2, label="last chunk")
+
+
+@needs_cuda
+def test_nnls_deletions_twin_keys():
+    """Near-duplicate key pairs make refits drop variables dozens of times
+    (several at once, deep inside the factor), in a factor held in shared
+    memory (t = 200) and one in the workspace (t = 300).  Besides the
+    acceptance rules, the last refit's fp64 weights, read from the workspace,
+    must satisfy the NNLS optimality conditions on the GPU's own features."""
+    import attention_matching_b200 as am
+    heads = [W.twin_keys_head(470 + h, n=512, T=800) for h in range(2)]
+    budgets = [300, 200]
+    out, _ = check_all(heads, budgets, 4, 2, label="twin keys")
+    f = am.features(out, 512, 800, 128, budgets, 4, 2, am.BF16)
+    for h in range(2):
+        check_refit_kkt(out, f, h, 512)
 
 
 @needs_cuda
