@@ -335,12 +335,39 @@ __device__ __forceinline__ void copy_doubles(double* dst, const double* src, int
   }
 }
 
-// D[r][c] = L[r0 + r][r0 + c] for c <= r < bw, zero elsewhere.
+// D[r][c] = L[r0 + r][r0 + c] for c <= r < bw, zero elsewhere (all loads
+// of a thread issued before its stores).
 __device__ __forceinline__ void load_diag_tile(const double* L, int r0, int bw, DiagTile* D) {
-  for (int e = threadIdx.x; e < kSB * kSB; e += blockDim.x) {
-    const int r = e >> 5, c = e & 31;
-    D[r][c] = (r < bw && c <= r) ? L[tri(r0 + r, r0 + c)] : 0.0;
+  for (int e0 = threadIdx.x; e0 < kSB * kSB; e0 += 4 * blockDim.x) {
+    double v[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int e = e0 + u * blockDim.x, r = e >> 5, c = e & 31;
+      v[u] = (e < kSB * kSB && r < bw && c <= r) ? L[tri(r0 + r, r0 + c)] : 0.0;
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int e = e0 + u * blockDim.x;
+      if (e < kSB * kSB) D[e >> 5][e & 31] = v[u];
+    }
   }
+}
+
+// Sums 32 per-lane values across the warp: afterwards lane l holds the
+// total of value l (31 shuffles: each step halves the values a lane keeps).
+__device__ __forceinline__ double warp_reduce32(double (&v)[32]) {
+  const int lane = threadIdx.x & 31;
+#pragma unroll
+  for (int s = 16; s >= 1; s >>= 1) {
+    const bool upper = (lane & s) != 0;
+#pragma unroll
+    for (int i = 0; i < s; ++i) {
+      const double send = upper ? v[i] : v[i + s];
+      const double keep = upper ? v[i + s] : v[i];
+      v[i] = keep + __shfl_xor_sync(0xffffffffu, send, s);
+    }
+  }
+  return v[0];
 }
 
 // u_e ← L⁻¹ u_e on rows [k0, n) for the R <= 8 vectors U[0..R); entries
@@ -383,14 +410,14 @@ __device__ void block_forward(const double* L, const double* invd, double* const
           }
         }
       }
+      double flat[32];   // value i·8 + e: row rb + i, vector e
 #pragma unroll
       for (int i = 0; i < 4; ++i)
 #pragma unroll
-        for (int e = 0; e < kMaxRhs; ++e)
-          if (e < R) {
-            const double sum = warp_sum(acc[i][e]);
-            if (lane == 0 && live[i]) U[e][rb + i] -= sum;
-          }
+        for (int e = 0; e < kMaxRhs; ++e) flat[i * kMaxRhs + e] = acc[i][e];
+      const double sum = warp_reduce32(flat);
+      const int li = lane / kMaxRhs, le = lane % kMaxRhs;
+      if (le < R && 4 * warp + li < bw) U[le][rb + li] -= sum;
     }
     __syncthreads();
     if (warp < R) {
