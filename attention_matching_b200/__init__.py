@@ -16,10 +16,10 @@ from typing import Dict, Optional, Sequence
 __all__ = ["AmError", "AmOpts", "lib", "library_path", "workspace_size", "compact_heads",
            "get_status", "profile_enable", "profile_collect", "kernel_launches", "STAGES",
            "STATUS", "BF16", "FP32", "CORR_AUTO", "CORR_STORED_FP32", "CORR_STORED_BF16",
-           "CORR_RECOMPUTE"]
+           "CORR_RECOMPUTE", "CORR_BOUNDED"]
 
 BF16, FP32 = 0, 1
-CORR_AUTO, CORR_STORED_FP32, CORR_STORED_BF16, CORR_RECOMPUTE = 0, 1, 2, 3
+CORR_AUTO, CORR_STORED_FP32, CORR_STORED_BF16, CORR_RECOMPUTE, CORR_BOUNDED = 0, 1, 2, 3, 4
 STATUS = {
     0: "AM_OK", 1: "AM_ERR_INVALID_ARG", 2: "AM_ERR_BUDGET", 3: "AM_ERR_WORKSPACE",
     4: "AM_ERR_NONFINITE", 5: "AM_ERR_CUDA", 6: "AM_ERR_TIMEOUT", 7: "AM_ERR_UNSUPPORTED",

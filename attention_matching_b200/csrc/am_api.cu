@@ -27,6 +27,7 @@ struct Layout {
   size_t picks, pick_corr, plist, sorted_slot;
   size_t bvec, w, w_eff, ycache;
   size_t G, L, AtA, A, AtY, nrm_part;
+  size_t cnorm, rnorm, corrd, clist, cstamp, ccount;
   size_t total;
   size_t tables_bytes;
 };
@@ -74,6 +75,12 @@ Layout plan(int n, int T, int d, int H, int64_t sum_t, int64_t sum_t2, bool corr
   L.A = take((size_t)sum_t * ldn * 4);
   L.AtY = take((size_t)sum_t * d * 8);
   L.nrm_part = take((size_t)kNormalMaxSplits * ((size_t)sum_t2 + (size_t)sum_t * d) * 8);
+  L.cnorm = take((size_t)H * T * 8);
+  L.rnorm = take((size_t)H * 8);
+  L.corrd = take((size_t)H * T * 8);
+  L.clist = take((size_t)H * T * 4);
+  L.cstamp = take((size_t)H * T * 4);
+  L.ccount = take((size_t)H * 2 * 4);
   L.total = o;
   return L;
 }
@@ -90,7 +97,7 @@ am_status_t check_shape(int n, int T, int d, int H, const int32_t* budgets, cons
   if (!(opts->ridge >= 0.f) || !isfinite(opts->ridge)) return AM_ERR_INVALID_ARG;
   if (!(opts->w_floor_rel > 0.f) || !(opts->w_floor_rel < 1.f)) return AM_ERR_INVALID_ARG;
   if (!isfinite(opts->scale)) return AM_ERR_INVALID_ARG;
-  if (opts->corr_mode < AM_CORR_AUTO || opts->corr_mode > AM_CORR_RECOMPUTE) return AM_ERR_INVALID_ARG;
+  if (opts->corr_mode < AM_CORR_AUTO || opts->corr_mode > AM_CORR_BOUNDED) return AM_ERR_INVALID_ARG;
   if (opts->corr_mode == AM_CORR_RECOMPUTE && !(opts->in_dtype == AM_BF16 && (d == 64 || d == 128)))
     return AM_ERR_UNSUPPORTED;
   if ((int64_t)n * d > (1ll << 31) || (int64_t)T * round_up(n, 32) > (1ll << 40))
@@ -151,6 +158,12 @@ Work bind(const Layout& L, char* base, bool corr_bf16) {
   w.A = reinterpret_cast<float*>(base + L.A);
   w.AtY = reinterpret_cast<double*>(base + L.AtY);
   w.nrm_part = reinterpret_cast<double*>(base + L.nrm_part);
+  w.cnorm = reinterpret_cast<double*>(base + L.cnorm);
+  w.rnorm = reinterpret_cast<double*>(base + L.rnorm);
+  w.corrd = reinterpret_cast<double*>(base + L.corrd);
+  w.clist = reinterpret_cast<int32_t*>(base + L.clist);
+  w.cstamp = reinterpret_cast<int32_t*>(base + L.cstamp);
+  w.ccount = reinterpret_cast<int32_t*>(base + L.ccount);
   return w;
 }
 
@@ -184,8 +197,8 @@ Problem make_problem(int n, int T, int d, int H, const am_opts_t* o, const Table
   p.max_t = tb.max_t;
   p.has_bias = o->key_bias != nullptr;
   p.corr_bf16 = o->corr_mode == AM_CORR_STORED_BF16;
-  const bool tc = o->in_dtype == AM_BF16 && (d == 64 || d == 128);
-  p.corr_recompute = o->corr_mode == AM_CORR_RECOMPUTE || (o->corr_mode == AM_CORR_AUTO && tc);
+  p.corr_recompute = o->corr_mode == AM_CORR_RECOMPUTE;
+  p.corr_bounded = o->corr_mode == AM_CORR_BOUNDED || o->corr_mode == AM_CORR_AUTO;
   return p;
 }
 
@@ -293,6 +306,8 @@ am_status_t am_compact_heads(const void* Q, const void* K, const void* V, int32_
     AM_TRY(launch_y_m(p, V, w, s));
   }
   AM_TRY(launch_omp_init(p, w, s));
+  if (p.corr_bounded) AM_TRY(launch_column_norms(p, w, s));
+  if (p.corr_bounded) AM_TRY(cudaMemsetAsync(w.cstamp, 0, (size_t)H * T * 4, s));
   for (int pass = 0; pass < (int)tb.active.size(); ++pass)
     AM_TRY(launch_omp_pass(p, w, pass, tb.active[pass], CorrInputs{Q, K, opts->key_bias}, s));
   if (opts->residual_out) AM_TRY(launch_residual_norm(p, w, opts->residual_out, s));

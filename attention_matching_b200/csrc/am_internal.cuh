@@ -30,6 +30,7 @@ struct Problem {
   int has_bias;
   int corr_bf16;      // the correlation pass streams a bf16 copy of Φᵀ
   int corr_recompute; // the correlation pass recomputes Φ on the tensor cores
+  int corr_bounded;   // the correlation pass computes only keys its bound cannot exclude
 };
 
 // Device pointers into the caller's workspace (see plan_workspace()).
@@ -65,6 +66,13 @@ struct Work {
   double* AtA;          // [Σt²]
   double* AtY;          // [Σt][d]
   double* nrm_part;     // [kNormalMaxSplits][Σt² + Σt·d] split partials of AᵀA, AᵀY
+  // bounded correlation pass
+  double* cnorm;        // [H][T] ‖Φ_{:,j}‖₂ (fp64, from the stored fp32 features)
+  double* rnorm;        // [H] ‖r‖₂ of the stored fp32 residual, this pass
+  double* corrd;        // [H][T] exact correlations of this pass's listed keys
+  int32_t* clist;       // [H][T] keys whose correlation this pass computes
+  int32_t* cstamp;      // [H][T] pass + 1 when the key is on this pass's list
+  int32_t* ccount;      // [H][2] probe count, total listed
   int64_t nrm_ata;      // Σt²
   int64_t nrm_stride;   // Σt² + Σt·d
 };
@@ -100,6 +108,10 @@ struct CorrInputs {
 };
 cudaError_t launch_omp_pass(const Problem& p, const Work& w, int pass, int active_heads,
                             const CorrInputs& in, cudaStream_t s);
+// bounded correlation pass (am_bounded.cu): column norms once, then per pass
+// probe, exact rows, extension, exact rows, selection
+cudaError_t launch_column_norms(const Problem& p, const Work& w, cudaStream_t s);
+cudaError_t launch_corr_bounded(const Problem& p, const Work& w, int pass, int active, cudaStream_t s);
 cudaError_t launch_residual_norm(const Problem& p, const Work& w, double* residual_out,
                                  cudaStream_t s);
 // value fit and packing (am_valfit.cu)
@@ -123,5 +135,11 @@ __device__ __forceinline__ void record_status(int32_t* status, int code) {
 
 // Number of OMP passes for budget t: one correlation pass per refit interval.
 __host__ __device__ inline int num_passes(int t, int kR) { return (t + kR - 1) / kR; }
+
+// Pick slots [s0, s1) that pass `pass` appends for a head of budget t.
+__device__ __forceinline__ void pass_range(const Problem& p, int t, int pass, int& s0, int& s1) {
+  s0 = min(pass * p.kR, t);
+  s1 = min(s0 + p.kR, t);
+}
 
 }  // namespace am

@@ -23,10 +23,6 @@
 namespace am {
 namespace {
 
-__device__ __forceinline__ void pass_range(const Problem& p, int t, int pass, int& s0, int& s1) {
-  s0 = min(pass * p.kR, t);
-  s1 = min(s0 + p.kR, t);
-}
 
 // ---------------------------------------------------------------- init ----
 __global__ void k_init(Problem p, Work w) {
@@ -989,14 +985,19 @@ cudaError_t launch_omp_init(const Problem& p, const Work& w, cudaStream_t s) {
 cudaError_t launch_omp_pass(const Problem& p, const Work& w, int pass, int active, const CorrInputs& in,
                             cudaStream_t s) {
   if (active <= 0) return cudaSuccess;
-  if (p.corr_recompute) {
-    cudaError_t e = launch_corr_tc(p, in.Q, in.K, in.key_bias, w, pass, active, s);
+  if (p.corr_bounded) {
+    cudaError_t e = launch_corr_bounded(p, w, pass, active, s);   // selects too
     if (e != cudaSuccess) return e;
   } else {
-    dim3 gc((p.T + kCorrRowsPerBlock - 1) / kCorrRowsPerBlock, active);
-    AM_LAUNCH(AM_STAGE_CORR, s, k_corr<<<gc, 256, 0, s>>>(p, w, pass));
+    if (p.corr_recompute) {
+      cudaError_t e = launch_corr_tc(p, in.Q, in.K, in.key_bias, w, pass, active, s);
+      if (e != cudaSuccess) return e;
+    } else {
+      dim3 gc((p.T + kCorrRowsPerBlock - 1) / kCorrRowsPerBlock, active);
+      AM_LAUNCH(AM_STAGE_CORR, s, k_corr<<<gc, 256, 0, s>>>(p, w, pass));
+    }
+    AM_LAUNCH(AM_STAGE_SELECT, s, k_select<<<active, 1024, 0, s>>>(p, w, pass));
   }
-  AM_LAUNCH(AM_STAGE_SELECT, s, k_select<<<active, 1024, 0, s>>>(p, w, pass));
   const int s1max = (pass + 1) * p.kR < p.max_t ? (pass + 1) * p.kR : p.max_t;
   dim3 gg(s1max, active);
   AM_LAUNCH(AM_STAGE_GRAM, s, k_gram<<<gg, 256, 0, s>>>(p, w, pass));

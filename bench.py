@@ -47,8 +47,9 @@ def parse_args():
                     choices=["qwen3_4b_layer", "single_head_fp32", "qwen3_4b_model", "online_rounds"])
     ap.add_argument("--heads", type=int, default=None,
                     help="heads per GPU for the layer workload (default 8); smaller for profiling")
-    ap.add_argument("--corr", choices=["auto", "fp32", "bf16", "recompute"], default="auto",
-                    help="correlation pass: stored fp32 / stored bf16 copy / tensor-core recompute")
+    ap.add_argument("--corr", choices=["auto", "fp32", "bf16", "recompute", "bounded"], default="auto",
+                    help="correlation pass: stored fp32 / stored bf16 copy / tensor-core recompute / "
+                         "bounded (exact values for the keys a Cauchy-Schwarz bound cannot exclude)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     return ap.parse_args()
@@ -300,12 +301,12 @@ def run_ours(args, rank, world, local_rank):
     Vh = torch.stack([h.V for h in wl.heads]).contiguous()
     Q, K, V = Qh.to(dev), Kh.to(dev), Vh.to(dev)
     corr_mode = {"auto": am.CORR_AUTO, "fp32": am.CORR_STORED_FP32, "bf16": am.CORR_STORED_BF16,
-                 "recompute": am.CORR_RECOMPUTE}[args.corr]
+                 "recompute": am.CORR_RECOMPUTE, "bounded": am.CORR_BOUNDED}[args.corr]
     kw = dict(topk=wl.topk, refit_every=wl.refit_every, corr_mode=corr_mode)
     opts = am.make_opts(am.BF16 if Q.dtype == torch.bfloat16 else am.FP32, wl.topk, wl.refit_every,
                         corr_mode=corr_mode)
     tc_ok = Q.dtype == torch.bfloat16 and d in (64, 128)
-    corr_kind = {"auto": "recompute" if tc_ok else "fp32"}.get(args.corr, args.corr)
+    corr_kind = {"auto": "bounded"}.get(args.corr, args.corr)
     ws = torch.empty((am.workspace_size(n, T, d, wl.budgets, opts),), dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
     flush = torch.empty((256 << 20,), dtype=torch.uint8, device=dev)
@@ -385,7 +386,9 @@ def run_ours(args, rank, world, local_rank):
            "budgets": wl.budgets if H <= 8 else f"{sum(wl.budgets)} total, min {min(wl.budgets)} max {max(wl.budgets)}",
            "topk": wl.topk, "refit_every": wl.refit_every,
            "correlation": {"fp32": "streams stored fp32 Phi^T", "bf16": "streams a bf16 copy of Phi^T",
-                           "recompute": "recomputes Phi on the tensor cores each pass"}[corr_kind],
+                           "recompute": "recomputes Phi on the tensor cores each pass",
+                           "bounded": "exact fp64 values for the keys whose Cauchy-Schwarz bound "
+                                      "reaches the pass's top k*R"}[corr_kind],
            "l2": "256 MiB buffer written between timed steps",
            "stage_ms_per_step": per_step_stage, "device_status": worst}
     if args.workload == "qwen3_4b_layer":

@@ -63,15 +63,19 @@ typedef enum am_dtype { AM_BF16 = 0, AM_FP32 = 1 } am_dtype_t;
 /* Where the correlation pass c = Φᵀ r reads the features from.  The mass,
  * Gram, residual and value fit always use the stored fp32 Φ. */
 typedef enum am_corr_mode {
-  AM_CORR_AUTO = 0,         /* RECOMPUTE when the tensor-core path applies (bf16
-                               inputs, d in {64, 128}), else STORED_FP32          */
+  AM_CORR_AUTO = 0,         /* BOUNDED                                           */
   AM_CORR_STORED_FP32 = 1,  /* stream the stored fp32 Φᵀ (4 bytes per feature)    */
   AM_CORR_STORED_BF16 = 2,  /* stream a bf16 copy of Φᵀ written by the feature
                                pass (2 bytes per feature; picks may differ from
                                exact arithmetic where correlations are closer
                                than bf16 rounding)                                 */
-  AM_CORR_RECOMPUTE = 3     /* recompute Φ from Q and K on the tensor cores in
+  AM_CORR_RECOMPUTE = 3,    /* recompute Φ from Q and K on the tensor cores in
                                every pass (no feature reads; bf16 inputs only)     */
+  AM_CORR_BOUNDED = 4       /* exact fp64 correlations, from the stored fp32 Φᵀ,
+                               for only the keys that can reach the pass's top
+                               k·R: |c_j| <= ‖r‖·‖Φ_{:,j}‖ (Cauchy-Schwarz) rules
+                               out every other key once k·R computed values exceed
+                               its bound; the picks are those of a full pass      */
 } am_corr_mode_t;
 
 /* Options.  Fill with am_default_opts() and override fields. */
