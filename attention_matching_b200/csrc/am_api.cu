@@ -27,7 +27,7 @@ struct Layout {
   size_t picks, pick_corr, plist, sorted_slot;
   size_t bvec, w, w_eff, ycache;
   size_t G, L, AtA, A, AtY, nrm_part;
-  size_t cnorm, rnorm, corrd, clist, cstamp, ccount;
+  size_t cnorm, rnorm, corrd, korder, knorm, ksort, cprefix;
   size_t total;
   size_t tables_bytes;
 };
@@ -78,9 +78,12 @@ Layout plan(int n, int T, int d, int H, int64_t sum_t, int64_t sum_t2, bool corr
   L.cnorm = take((size_t)H * T * 8);
   L.rnorm = take((size_t)H * 8);
   L.corrd = take((size_t)H * T * 8);
-  L.clist = take((size_t)H * T * 4);
-  L.cstamp = take((size_t)H * T * 4);
-  L.ccount = take((size_t)H * 2 * 4);
+  L.korder = take((size_t)H * T * 4);
+  L.knorm = take((size_t)H * T * 4);
+  size_t t2 = 1;
+  while (t2 < (size_t)T) t2 <<= 1;
+  L.ksort = take(T > kSortSmemKeys ? (size_t)H * t2 * 8 : 0);
+  L.cprefix = take((size_t)H * 4);
   L.total = o;
   return L;
 }
@@ -161,9 +164,10 @@ Work bind(const Layout& L, char* base, bool corr_bf16) {
   w.cnorm = reinterpret_cast<double*>(base + L.cnorm);
   w.rnorm = reinterpret_cast<double*>(base + L.rnorm);
   w.corrd = reinterpret_cast<double*>(base + L.corrd);
-  w.clist = reinterpret_cast<int32_t*>(base + L.clist);
-  w.cstamp = reinterpret_cast<int32_t*>(base + L.cstamp);
-  w.ccount = reinterpret_cast<int32_t*>(base + L.ccount);
+  w.korder = reinterpret_cast<int32_t*>(base + L.korder);
+  w.knorm = reinterpret_cast<float*>(base + L.knorm);
+  w.ksort = reinterpret_cast<uint64_t*>(base + L.ksort);
+  w.cprefix = reinterpret_cast<int32_t*>(base + L.cprefix);
   return w;
 }
 
@@ -307,7 +311,6 @@ am_status_t am_compact_heads(const void* Q, const void* K, const void* V, int32_
   }
   AM_TRY(launch_omp_init(p, w, s));
   if (p.corr_bounded) AM_TRY(launch_column_norms(p, w, s));
-  if (p.corr_bounded) AM_TRY(cudaMemsetAsync(w.cstamp, 0, (size_t)H * T * 4, s));
   for (int pass = 0; pass < (int)tb.active.size(); ++pass)
     AM_TRY(launch_omp_pass(p, w, pass, tb.active[pass], CorrInputs{Q, K, opts->key_bias}, s));
   if (opts->residual_out) AM_TRY(launch_residual_norm(p, w, opts->residual_out, s));

@@ -3,23 +3,27 @@
 // k·R keys per pass under top-k batching with lazy refit, xinfinite.net
 // article §3), evaluated exactly for only the keys that can win.
 //
-// For every key |c_j| = |rᵀΦ_{:,j}| <= ‖r‖₂·‖Φ_{:,j}‖₂ = B_j (Cauchy-Schwarz).
-// One pass of kk = s1 − s0 picks per head:
-//   1. k_probe   lists the unselected keys of largest bound: a histogram of B
-//                over 1/16-octave bins, cut where at least kProbe keys lie at
-//                or above;
-//   2. k_rows    computes their c_j exactly: fp64 sums of the stored fp32
-//                features times the stored fp32 residual;
-//   3. k_extend  takes θ = the kk-th largest of those values and lists every
-//                other unselected key with B_j·(1 + 1e-9) >= θ;
-//   4. k_rows    computes those;
-//   5. k_pick    appends the kk largest listed values (ties to the lower key).
-// A key left off the list has c_j < θ while kk listed keys reach θ, so it is
-// not among the kk largest: the picks are those of a full pass over all keys.
+// For every key |c_j| = |rᵀΦ_{:,j}| <= ‖r‖₂·‖Φ_{:,j}‖₂ (Cauchy-Schwarz).  The
+// column norms do not depend on r, so once per call the keys are sorted by
+// norm (k_colnorm, k_sortnorm); in every pass the keys a bound cannot exclude
+// then form a prefix of that order.  One pass of kk = s1 − s0 picks per head:
+//   1. k_rows    exact c_j for the unselected keys among the first
+//                P0 = kProbe + s0 sorted positions (so at least kProbe keys):
+//                fp64 sums of the stored fp32 features times the stored fp32
+//                residual;
+//   2. k_theta   θ = the kk-th largest of those values, and the prefix length
+//                L: every key with ‖Φ_{:,j}‖ >= θ / (‖r‖(1 + 1e-9)) lies in
+//                [0, L) (binary search in the sorted norms);
+//   3. k_rows    exact c_j for the unselected keys in [P0, L);
+//   4. k_pick    appends the kk largest values of [0, L) (ties to the lower
+//                key).
+// A key beyond L has c_j < θ while kk keys in the prefix reach θ, so it is not
+// among the kk largest: the picks are those of a full pass over all keys.
 // The margin 1e-9 covers the rounding of the fp64 sums and norms (relative
-// error below n·2^-53 for the sums, a few ulp for the norms).
-//
-// The column norms ‖Φ_{:,j}‖₂ are computed once per call (k_colnorm).
+// error below n·2^-53 for the sums, a few ulp for the norms); the fp32 copies
+// of the norms only move the cut outward (rounding to nearest is monotone).
+// The selections sort their candidates with a bitonic network in shared
+// memory (no serial merge, no atomics).
 #include "am_internal.cuh"
 #include "am_profile.cuh"
 #include "am_linalg.cuh"
@@ -29,26 +33,47 @@
 namespace am {
 namespace {
 
-constexpr int kProbe = 256;        // keys whose exact values set the first threshold
-constexpr int kHistBins = 4096;    // float bits 30..19 of the bound: 1/16 octave
+constexpr int kProbe = 256;        // unselected keys whose exact values set the threshold
 constexpr int kBoundThreads = 1024;
-constexpr int kStage = 4096;       // listed values staged in shared memory
-constexpr int kMaxKK = kMaxPicksPerPass;
+constexpr int kSelCap = 4096;      // candidates one selection sort holds
 constexpr double kBoundMargin = 1e-9;
 
-__device__ __forceinline__ int bound_bin(double b) {
-  return (int)(__float_as_uint((float)b) >> 19);   // b >= 0: monotone in b, < 4096
+// Order-preserving map of a double to uint64 (NaN ranks lowest).
+__device__ __forceinline__ uint64_t order_key(double v) {
+  if (v != v) return 0ull;
+  const uint64_t u = (uint64_t)__double_as_longlong(v);
+  return (u & 0x8000000000000000ull) ? ~u : (u | 0x8000000000000000ull);
 }
 
-// (v, j) precedes (v', j') in pick order: larger value first, then lower key.
-// A NaN value ranks below every number.
-__device__ __forceinline__ bool ahead(double v, int j, double v2, int j2) {
-  const bool n1 = v != v, n2 = v2 != v2;
-  if (n1 || n2) return !n1 && n2 ? true : (n1 && !n2 ? false : j < j2);
-  return v > v2 || (v == v2 && j < j2);
+// (a, ja) before (b, jb) in pick order: larger key first, then lower index.
+__device__ __forceinline__ bool before(uint64_t a, int ja, uint64_t b, int jb) {
+  return a > b || (a == b && ja < jb);
+}
+
+// Sorts the n2 (a power of two) pairs (key, idx) into pick order with a
+// bitonic network; all threads of the block.
+__device__ void bitonic_pairs(uint64_t* key, int* idx, int n2) {
+  for (int k = 2; k <= n2; k <<= 1) {
+    for (int jj = k >> 1; jj > 0; jj >>= 1) {
+      for (int i = threadIdx.x; i < n2; i += blockDim.x) {
+        const int l = i ^ jj;
+        if (l > i) {
+          const bool up = (i & k) == 0;   // this block in pick order, else reversed
+          const uint64_t a = key[i], b = key[l];
+          const int ia = idx[i], ib = idx[l];
+          if (up ? before(b, ib, a, ia) : before(a, ia, b, ib)) {
+            key[i] = b; key[l] = a;
+            idx[i] = ib; idx[l] = ia;
+          }
+        }
+      }
+      __syncthreads();
+    }
+  }
 }
 
 // ---------------------------------------------------------- column norms --
+// ‖Φ_{:,j}‖₂ in fp64 from the stored fp32 features: one warp per key.
 __global__ void __launch_bounds__(256) k_colnorm(Problem p, Work w) {
   const int h = blockIdx.y;
   const int j = blockIdx.x * 8 + (threadIdx.x >> 5);
@@ -68,88 +93,60 @@ __global__ void __launch_bounds__(256) k_colnorm(Problem p, Work w) {
   if (lane == 0) w.cnorm[(int64_t)h * p.T + j] = sqrt(s);
 }
 
-// ----------------------------------------------------------------- probe --
-__global__ void __launch_bounds__(kBoundThreads) k_probe(Problem p, Work w, int pass) {
-  const int h = w.order[blockIdx.x];
-  int s0, s1;
-  pass_range(p, w.t[h], pass, s0, s1);
-  if (s0 >= s1) return;
-  __shared__ int hist[kHistBins];
-  __shared__ int wsum[32];
-  __shared__ double red[33];
-  __shared__ int s_cut, s_n;
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const float* r = w.r + (int64_t)h * p.ldn;
-  double a = 0.0;
-  for (int i = tid; i < p.ldn; i += blockDim.x) {
-    const double v = r[i];
-    a = fma(v, v, a);
-  }
-  const double rn = sqrt(block_sum(a, red));
-  for (int b = tid; b < kHistBins; b += blockDim.x) hist[b] = 0;
-  if (tid == 0) {
-    w.rnorm[h] = rn;
-    s_n = 0;
-  }
-  __syncthreads();
+// Keys of each head by descending fp32 norm (ties: lower key first): one
+// block per head; 64-bit sort keys (norm bits, inverted key index) in shared
+// memory, or in the workspace when T exceeds kSortSmemKeys.
+__global__ void __launch_bounds__(kBoundThreads) k_sortnorm(Problem p, Work w) {
+  extern __shared__ __align__(16) unsigned char smem[];
+  const int h = blockIdx.x;
+  int n2 = 1;
+  while (n2 < p.T) n2 <<= 1;
+  uint64_t* key = p.T > kSortSmemKeys ? w.ksort + (int64_t)h * n2 : reinterpret_cast<uint64_t*>(smem);
   const double* cn = w.cnorm + (int64_t)h * p.T;
-  const uint8_t* sel = w.sel + (int64_t)h * p.T;
-  for (int j = tid; j < p.T; j += blockDim.x)
-    if (!sel[j]) atomicAdd(&hist[bound_bin(rn * cn[j])], 1);
+  for (int i = threadIdx.x; i < n2; i += blockDim.x)
+    key[i] = i < p.T ? ((uint64_t)__float_as_uint((float)cn[i]) << 32) | (uint32_t)(0xFFFFFFFFu - (uint32_t)i)
+                     : 0ull;
   __syncthreads();
-  // warp q sums bins [128q, 128q + 128); the cut is the highest bin with at
-  // least kProbe keys at or above it (bin 0 when fewer keys are left)
-  int cnt = 0;
-  for (int b = warp * 128 + lane; b < warp * 128 + 128; b += 32) cnt += hist[b];
-  for (int o = 16; o; o >>= 1) cnt += __shfl_xor_sync(0xffffffffu, cnt, o);
-  if (lane == 0) wsum[warp] = cnt;
-  __syncthreads();
-  if (tid == 0) {
-    int above = 0, cut = 0;
-    for (int q = 31; q >= 0; --q) {
-      if (above + wsum[q] >= kProbe) {
-        for (int b = q * 128 + 127; b >= q * 128; --b) {
-          above += hist[b];
-          if (above >= kProbe) { cut = b; break; }
+  for (int k = 2; k <= n2; k <<= 1) {
+    for (int jj = k >> 1; jj > 0; jj >>= 1) {
+      for (int i = threadIdx.x; i < n2; i += blockDim.x) {
+        const int l = i ^ jj;
+        if (l > i) {
+          const bool desc = (i & k) == 0;
+          const uint64_t a = key[i], b = key[l];
+          if (desc ? a < b : a > b) { key[i] = b; key[l] = a; }
         }
-        break;
       }
-      above += wsum[q];
+      __syncthreads();
     }
-    s_cut = cut;
   }
-  __syncthreads();
-  const int cut = s_cut;
-  int32_t* list = w.clist + (int64_t)h * p.T;
-  int32_t* stamp = w.cstamp + (int64_t)h * p.T;
-  for (int j = tid; j < p.T; j += blockDim.x)
-    if (!sel[j] && bound_bin(rn * cn[j]) >= cut) {
-      list[atomicAdd(&s_n, 1)] = j;
-      stamp[j] = pass + 1;
-    }
-  __syncthreads();
-  if (tid == 0) {
-    w.ccount[2 * h] = s_n;
-    w.ccount[2 * h + 1] = s_n;
+  for (int i = threadIdx.x; i < p.T; i += blockDim.x) {
+    const uint64_t k = key[i];
+    w.korder[(int64_t)h * p.T + i] = (int32_t)(0xFFFFFFFFu - (uint32_t)k);
+    w.knorm[(int64_t)h * p.T + i] = __uint_as_float((uint32_t)(k >> 32));
   }
 }
 
 // ------------------------------------------------------------ exact rows --
-// c_j = Σ_i r_i Φ_ij for the listed keys [lo, hi) of each head (probe list
-// when which = 0, its extension when which = 1): one warp per key, fp64 sums
-// of exact fp32 products, four float4 loads per lane in flight.
+// c_j = Σ_i r_i Φ_ij for the unselected keys at sorted positions [0, P0)
+// (which = 0) or [P0, L) (which = 1): one warp per key, fp64 sums of exact
+// fp32 products, four float4 loads per lane in flight.
 __global__ void __launch_bounds__(256) k_rows(Problem p, Work w, int pass, int which) {
   const int h = w.order[blockIdx.y];
   int s0, s1;
   pass_range(p, w.t[h], pass, s0, s1);
   if (s0 >= s1) return;
-  const int lo = which ? w.ccount[2 * h] : 0;
-  const int hi = which ? w.ccount[2 * h + 1] : w.ccount[2 * h];
+  const int p0 = min(p.T, kProbe + s0);
+  const int lo = which ? p0 : 0;
+  const int hi = which ? w.cprefix[h] : p0;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int32_t* ord = w.korder + (int64_t)h * p.T;
+  const uint8_t* sel = w.sel + (int64_t)h * p.T;
   const float4* r4 = reinterpret_cast<const float4*>(w.r + (int64_t)h * p.ldn);
   const int n4 = p.ldn >> 2;
   for (int q = lo + blockIdx.x * 8 + warp; q < hi; q += gridDim.x * 8) {
-    const int j = w.clist[(int64_t)h * p.T + q];
+    const int j = ord[q];
+    if (sel[j]) continue;
     const float4* row = reinterpret_cast<const float4*>(w.phiT + ((int64_t)h * p.T + j) * p.ldn);
     double a[4] = {0.0, 0.0, 0.0, 0.0};
     for (int i0 = lane; i0 < n4; i0 += 32 * 4) {
@@ -173,139 +170,114 @@ __global__ void __launch_bounds__(256) k_rows(Problem p, Work w, int pass, int w
   }
 }
 
-// ------------------------------------------------------------ top-kk -----
-// The kk <= 64 listed entries first in pick order, into ov/oi (shared).  Each
-// warp finds the top kk of its share by kk rounds of "best entry after the
-// previous one", then warp 0 does the same over the 32·kk warp winners.
-// Values of the first kStage entries are staged in shared memory.
-struct TopScratch {
-  double v[kStage];
-  int j[kStage];
-  double cv[32 * kMaxKK];
-  int cj[32 * kMaxKK];
+struct SelScratch {
+  uint64_t key[kSelCap];
+  int idx[kSelCap];
 };
 
-__device__ void block_topk(const Problem& p, const Work& w, int h, int cnt, int kk, TopScratch& S, double* ov,
-                           int* oi) {
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nw = blockDim.x >> 5;
-  const int32_t* list = w.clist + (int64_t)h * p.T;
+// Appends the unselected keys at sorted positions [lo, hi) to the candidate
+// slots from *count on (at most kSelCap in all); all threads.
+__device__ void stage_candidates(const Problem& p, const Work& w, int h, int lo, int hi, SelScratch& S,
+                                 int* count) {
+  const int32_t* ord = w.korder + (int64_t)h * p.T;
+  const uint8_t* sel = w.sel + (int64_t)h * p.T;
   const double* cd = w.corrd + (int64_t)h * p.T;
-  for (int q = tid; q < min(cnt, kStage); q += blockDim.x) {
-    const int j = list[q];
-    S.j[q] = j;
-    S.v[q] = cd[j];
-  }
-  __syncthreads();
-  auto entry = [&](int q, double& v, int& j) {
-    if (q < kStage) { v = S.v[q]; j = S.j[q]; }
-    else { j = list[q]; v = cd[j]; }
-  };
-  // per-warp winners over positions q ≡ warp (mod nw) ... strided by lanes
-  const int per = (cnt + nw - 1) / nw;
-  const int q0 = warp * per, q1 = min(cnt, q0 + per);
-  double pv = INFINITY;
-  int pj = -1;
-  for (int k = 0; k < kk; ++k) {
-    double bv = -INFINITY;
-    int bj = INT_MAX;
-    bool have = false;
-    for (int q = q0 + lane; q < q1; q += 32) {
-      double v;
-      int j;
-      entry(q, v, j);
-      const bool after = pj < 0 || ahead(pv, pj, v, j);
-      if (after && (!have || ahead(v, j, bv, bj))) { bv = v; bj = j; have = true; }
-    }
-    for (int o = 16; o; o >>= 1) {
-      const double v2 = __shfl_xor_sync(0xffffffffu, bv, o);
-      const int j2 = __shfl_xor_sync(0xffffffffu, bj, o);
-      const int h2 = __shfl_xor_sync(0xffffffffu, (int)have, o);
-      if (h2 && (!have || ahead(v2, j2, bv, bj))) { bv = v2; bj = j2; have = true; }
-    }
-    if (lane == 0) {
-      S.cv[warp * kMaxKK + k] = have ? bv : -INFINITY;
-      S.cj[warp * kMaxKK + k] = have ? bj : INT_MAX;
-    }
-    pv = bv;
-    pj = have ? bj : INT_MAX;
-  }
-  __syncthreads();
-  if (warp == 0) {
-    pv = INFINITY;
-    pj = -1;
-    for (int k = 0; k < kk; ++k) {
-      double bv = -INFINITY;
-      int bj = INT_MAX;
-      for (int e = lane; e < nw * kk; e += 32) {
-        const double v = S.cv[(e / kk) * kMaxKK + e % kk];
-        const int j = S.cj[(e / kk) * kMaxKK + e % kk];
-        if (j == INT_MAX) continue;
-        const bool after = pj < 0 || ahead(pv, pj, v, j);
-        if (after && (bj == INT_MAX || ahead(v, j, bv, bj))) { bv = v; bj = j; }
-      }
-      for (int o = 16; o; o >>= 1) {
-        const double v2 = __shfl_xor_sync(0xffffffffu, bv, o);
-        const int j2 = __shfl_xor_sync(0xffffffffu, bj, o);
-        if (j2 != INT_MAX && (bj == INT_MAX || ahead(v2, j2, bv, bj))) { bv = v2; bj = j2; }
-      }
-      if (lane == 0) { ov[k] = bv; oi[k] = bj; }
-      pv = bv;
-      pj = bj;
+  for (int q = lo + threadIdx.x; q < hi; q += blockDim.x) {
+    const int j = ord[q];
+    if (sel[j]) continue;
+    const int pos = atomicAdd(count, 1);
+    if (pos < kSelCap) {
+      S.key[pos] = order_key(cd[j]);
+      S.idx[pos] = j;
     }
   }
   __syncthreads();
 }
 
-// ------------------------------------------------------------- extension --
-__global__ void __launch_bounds__(kBoundThreads) k_extend(Problem p, Work w, int pass) {
+// Sorts the first n candidates into pick order (padding to a power of two).
+__device__ void sort_candidates(SelScratch& S, int n) {
+  int n2 = 1;
+  while (n2 < n) n2 <<= 1;
+  for (int i = n + threadIdx.x; i < n2; i += blockDim.x) {
+    S.key[i] = 0ull;
+    S.idx[i] = INT_MAX;
+  }
+  __syncthreads();
+  bitonic_pairs(S.key, S.idx, n2);
+}
+
+// ------------------------------------------------------ threshold, prefix --
+__global__ void __launch_bounds__(kBoundThreads) k_theta(Problem p, Work w, int pass) {
   extern __shared__ __align__(16) unsigned char smem[];
-  TopScratch& S = *reinterpret_cast<TopScratch*>(smem);
-  __shared__ double ov[kMaxKK];
-  __shared__ int oi[kMaxKK];
-  __shared__ int s_n;
+  SelScratch& S = *reinterpret_cast<SelScratch*>(smem);
+  __shared__ double red[33];
+  __shared__ int s_cnt;
   const int h = w.order[blockIdx.x];
   int s0, s1;
   pass_range(p, w.t[h], pass, s0, s1);
   if (s0 >= s1) return;
   const int kk = s1 - s0;
-  const int c0 = w.ccount[2 * h];
-  if (threadIdx.x == 0) s_n = 0;
-  block_topk(p, w, h, c0, kk, S, ov, oi);
-  const double theta = ov[kk - 1];
-  if (!(theta == theta)) return;   // NaN correlations: the pick stage reports them
-  const double rn = w.rnorm[h];
-  const double* cn = w.cnorm + (int64_t)h * p.T;
-  const uint8_t* sel = w.sel + (int64_t)h * p.T;
-  int32_t* list = w.clist + (int64_t)h * p.T;
-  int32_t* stamp = w.cstamp + (int64_t)h * p.T;
-  for (int j = threadIdx.x; j < p.T; j += blockDim.x)
-    if (!sel[j] && stamp[j] != pass + 1 && rn * cn[j] * (1.0 + kBoundMargin) >= theta) {
-      list[c0 + atomicAdd(&s_n, 1)] = j;
-      stamp[j] = pass + 1;
-    }
+  const int p0 = min(p.T, kProbe + s0);
+  const float* r = w.r + (int64_t)h * p.ldn;
+  double a = 0.0;
+  for (int i = threadIdx.x; i < p.ldn; i += blockDim.x) {
+    const double v = r[i];
+    a = fma(v, v, a);
+  }
+  const double rn = sqrt(block_sum(a, red));
+  if (threadIdx.x == 0) s_cnt = 0;
   __syncthreads();
-  if (threadIdx.x == 0) w.ccount[2 * h + 1] = c0 + s_n;
+  stage_candidates(p, w, h, 0, p0, S, &s_cnt);   // p0 <= kProbe + 2047 < kSelCap
+  const int n = min(s_cnt, kSelCap);
+  sort_candidates(S, n);
+  const double theta = kk <= n ? w.corrd[(int64_t)h * p.T + S.idx[kk - 1]] : -INFINITY;
+  // L = number of sorted norms not below θ / (‖r‖(1 + margin)); every key when
+  // the bound cannot help (θ <= 0, a zero or non-finite residual)
+  int count = 0;
+  const bool useful = theta > 0.0 && rn > 0.0 && rn < INFINITY;
+  const float thr = useful ? (float)(theta / (rn * (1.0 + kBoundMargin))) : 0.f;
+  const float* kn = w.knorm + (int64_t)h * p.T;
+  if (useful)
+    for (int q = threadIdx.x; q < p.T; q += blockDim.x) count += !(kn[q] < thr);
+  const double tot = block_sum((double)count, red);
+  if (threadIdx.x == 0) {
+    int L = useful ? (int)tot : p.T;
+    w.cprefix[h] = L > p0 ? L : p0;
+    w.rnorm[h] = rn;
+  }
 }
 
 // ------------------------------------------------------------------ pick --
+// The kk largest values among the unselected keys of [0, L), in chunks that
+// keep the best kk of what came before.
 __global__ void __launch_bounds__(kBoundThreads) k_pick(Problem p, Work w, int pass) {
   extern __shared__ __align__(16) unsigned char smem[];
-  TopScratch& S = *reinterpret_cast<TopScratch*>(smem);
-  __shared__ double ov[kMaxKK];
-  __shared__ int oi[kMaxKK];
+  SelScratch& S = *reinterpret_cast<SelScratch*>(smem);
+  __shared__ int s_cnt;
   const int h = w.order[blockIdx.x];
   int s0, s1;
   pass_range(p, w.t[h], pass, s0, s1);
   if (s0 >= s1) return;
   const int kk = s1 - s0;
-  block_topk(p, w, h, w.ccount[2 * h + 1], kk, S, ov, oi);
+  const int L = w.cprefix[h];
+  const int chunk = kSelCap - kMaxPicksPerPass;
+  int kept = 0;
+  for (int c = 0; c < L; c += chunk) {
+    if (threadIdx.x == 0) s_cnt = kept;
+    __syncthreads();
+    stage_candidates(p, w, h, c, min(L, c + chunk), S, &s_cnt);
+    const int n = min(s_cnt, kSelCap);
+    sort_candidates(S, n);
+    kept = min(kk, n);
+  }
   if (threadIdx.x == 0) {
     uint8_t* sel = w.sel + (int64_t)h * p.T;
+    const double* cd = w.corrd + (int64_t)h * p.T;
     bool bad = false;
     for (int k = 0; k < kk; ++k) {
-      int j = oi[k];
-      double v = ov[k];
-      if (j == INT_MAX || !(v == v)) {   // no finite value left: lowest free key
+      int j = k < kept ? S.idx[k] : INT_MAX;
+      double v = j != INT_MAX ? cd[j] : -INFINITY;
+      if (j == INT_MAX || !(v == v)) {   // no finite value: lowest free key
         bad = true;
         for (j = 0; j < p.T && sel[j]; ++j) {}
         v = -INFINITY;
@@ -329,19 +301,21 @@ int rows_ctas_per_head(int active) {
 cudaError_t launch_column_norms(const Problem& p, const Work& w, cudaStream_t s) {
   dim3 g((p.T + 7) / 8, p.H);
   AM_LAUNCH(AM_STAGE_PHI, s, k_colnorm<<<g, 256, 0, s>>>(p, w));
+  const int sort_smem = p.T > kSortSmemKeys ? 0 : (int)(sizeof(uint64_t) * kSortSmemKeys);
+  cudaFuncSetAttribute(k_sortnorm, cudaFuncAttributeMaxDynamicSharedMemorySize, sort_smem);
+  AM_LAUNCH(AM_STAGE_PHI, s, k_sortnorm<<<p.H, kBoundThreads, sort_smem, s>>>(p, w));
   return cudaGetLastError();
 }
 
 cudaError_t launch_corr_bounded(const Problem& p, const Work& w, int pass, int active, cudaStream_t s) {
-  const int top_smem = (int)sizeof(TopScratch);
-  cudaFuncSetAttribute(k_extend, cudaFuncAttributeMaxDynamicSharedMemorySize, top_smem);
-  cudaFuncSetAttribute(k_pick, cudaFuncAttributeMaxDynamicSharedMemorySize, top_smem);
+  const int sel_smem = (int)sizeof(SelScratch);
+  cudaFuncSetAttribute(k_theta, cudaFuncAttributeMaxDynamicSharedMemorySize, sel_smem);
+  cudaFuncSetAttribute(k_pick, cudaFuncAttributeMaxDynamicSharedMemorySize, sel_smem);
   dim3 gr(rows_ctas_per_head(active), active);
-  AM_LAUNCH(AM_STAGE_CORR, s, k_probe<<<active, kBoundThreads, 0, s>>>(p, w, pass));
   AM_LAUNCH(AM_STAGE_CORR, s, k_rows<<<gr, 256, 0, s>>>(p, w, pass, 0));
-  AM_LAUNCH(AM_STAGE_CORR, s, k_extend<<<active, kBoundThreads, top_smem, s>>>(p, w, pass));
+  AM_LAUNCH(AM_STAGE_CORR, s, k_theta<<<active, kBoundThreads, sel_smem, s>>>(p, w, pass));
   AM_LAUNCH(AM_STAGE_CORR, s, k_rows<<<gr, 256, 0, s>>>(p, w, pass, 1));
-  AM_LAUNCH(AM_STAGE_SELECT, s, k_pick<<<active, kBoundThreads, top_smem, s>>>(p, w, pass));
+  AM_LAUNCH(AM_STAGE_SELECT, s, k_pick<<<active, kBoundThreads, sel_smem, s>>>(p, w, pass));
   return cudaGetLastError();
 }
 

@@ -69,15 +69,17 @@ struct Work {
   // bounded correlation pass
   double* cnorm;        // [H][T] ‖Φ_{:,j}‖₂ (fp64, from the stored fp32 features)
   double* rnorm;        // [H] ‖r‖₂ of the stored fp32 residual, this pass
-  double* corrd;        // [H][T] exact correlations of this pass's listed keys
-  int32_t* clist;       // [H][T] keys whose correlation this pass computes
-  int32_t* cstamp;      // [H][T] pass + 1 when the key is on this pass's list
-  int32_t* ccount;      // [H][2] probe count, total listed
+  double* corrd;        // [H][T] exact correlations of this pass's evaluated keys
+  int32_t* korder;      // [H][T] keys by descending column norm
+  float* knorm;         // [H][T] those norms (fp32, descending)
+  uint64_t* ksort;      // [H][pow2 >= T] sort scratch when T exceeds the shared-memory sort
+  int32_t* cprefix;     // [H] this pass evaluates the keys at sorted positions [0, cprefix)
   int64_t nrm_ata;      // Σt²
   int64_t nrm_stride;   // Σt² + Σt·d
 };
 
 constexpr int kRedBlocks = 64;   // partial-sum slots per head for ‖r‖²
+constexpr int kSortSmemKeys = 16384;  // key counts the norm sort handles in shared memory
 constexpr int kNormalMaxSplits = 8;   // query splits of the normal-equation products
 
 // ---- launchers (each file defines its own) ----

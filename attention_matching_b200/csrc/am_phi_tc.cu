@@ -6,15 +6,15 @@
 // prior key bias and one per-head shift); xinfinite.net article §2 step 3:
 // the value fit targets the original local attention output Y = ΦV/m.
 //
-// One CTA per (head, 128-query block), 8 warps:
+// One CTA per (head, 128-query block), 20 warps:
 //   warp 0   TMA producer: the query block once, then (key, value) tiles of
 //            64 keys through a 3-stage ring
 //   warp 1   MMA issuer (one thread): S = Q·Kᵀ into one of two TMEM
 //            accumulators (kind::f16, bf16 in, fp32 out), then Y += P·V
 //            from the epilogue's P tiles (PHI mode)
 //   warp 2   TMEM allocation and release
-//   warps 4-11 epilogue, two warpgroups: thread (half, r) owns query row r
-//            (TMEM lane r) and 32 of each tile's 64 keys; it reads its logits,
+//   warps 4-19 epilogue, four warpgroups: thread (g, r) owns query row r
+//            (TMEM lane r) and 16 of each tile's 64 keys; it reads its logits,
 //            forms p = exp(s·scale + b − c), adds p to the fp64 mass, writes Φᵀ
 //            (a warp writes 32 consecutive queries of one key: 128-byte
 //            coalesced), and stores p split as bf16 hi + lo (p = hi + lo to 16
@@ -36,7 +36,9 @@ namespace {
 constexpr int BM = 128;        // queries per CTA (TMEM lanes)
 constexpr int BN = 64;         // keys per tile
 constexpr int STAGES = 3;      // key/value ring depth
-constexpr int kThreads = 384;   // 4 control warps + 2 epilogue warpgroups
+constexpr int kEpiGroups = 4;  // epilogue warpgroups; each takes BN / 4 columns of a tile
+constexpr int kEpiThreads = 128 * kEpiGroups;
+constexpr int kThreads = 128 + kEpiThreads;   // 4 control warps + the epilogue
 constexpr int kEpiWarp0 = 4;   // first epilogue warp
 constexpr uint32_t kTmemCols = 256;
 constexpr long long kWaitBudgetCycles = 4000000000ll;   // ~2 s at 2 GHz
@@ -154,6 +156,19 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
   for (int k = 0; k < 32; ++k) v[k] = __uint_as_float(r[k]);
 }
 
+// 32 lanes × 16 consecutive 32-bit columns.
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
+  uint32_t r[16];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
+#pragma unroll
+  for (int k = 0; k < 16; ++k) v[k] = __uint_as_float(r[k]);
+}
+
 __device__ __forceinline__ float ex2_approx(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
@@ -221,8 +236,8 @@ k_phi_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtens
   uint64_t* drain = s_full + 9;
   __shared__ uint32_t s_tmem;
   __shared__ int s_abort;
-  __shared__ float s_red[8];
-  __shared__ double s_mass[256];
+  __shared__ float s_red[4 * kEpiGroups];
+  __shared__ double s_mass[kEpiGroups + 1][BM];
   __shared__ int s_stop_y;
   __shared__ int s_stopm[2];
 
@@ -240,8 +255,8 @@ k_phi_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtens
     for (int s = 0; s < STAGES; ++s) { mbar_init(kv_full + s, 1); mbar_init(kv_empty + s, 1); }
     for (int b = 0; b < 2; ++b) {
       mbar_init(s_full + b, 1);
-      mbar_init(s_empty + b, 256);
-      mbar_init(p_full + b, 256);
+      mbar_init(s_empty + b, kEpiThreads);
+      mbar_init(p_full + b, kEpiThreads);
       mbar_init(p_empty + b, 1);
     }
     mbar_init(y_full, 1);
@@ -338,13 +353,13 @@ k_phi_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtens
     }
   } else if (warp >= kEpiWarp0) {
     // --------------------------------------------------- epilogue ----
-    // Two warpgroups: thread (half, et) owns query row et (TMEM lane et) and
-    // columns [32·half, 32·half + 32) of every 64-key tile.
-    const int ep = threadIdx.x - kEpiWarp0 * 32;     // 0..255
-    const int half = ep >> 7;
+    // Four warpgroups: thread (grp, et) owns query row et (TMEM lane et) and
+    // columns [16·grp, 16·grp + 16) of every 64-key tile.
+    const int ep = threadIdx.x - kEpiWarp0 * 32;     // 0..511
+    const int grp = ep >> 7;
     const int et = ep & 127;
     const int qd = warp & 3;                         // TMEM lane quadrant of this warp
-    constexpr int HC = BN / 2;
+    constexpr int HC = BN / kEpiGroups;
     const int i = q0 + et;
     const bool row_live = i < p.n;
     const float c = MODE == MODE_PHI ? w.shift[h] : 0.f;
@@ -364,7 +379,7 @@ k_phi_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtens
       if constexpr (MODE == MODE_MAX) {
         // light per-tile work: one thread waits and the group follows it
         if (ep == 0) s_stopm[b] = mbar_wait(s_full + b, bu & 1, abort_flag, status) ? 0 : 1;
-        asm volatile("bar.sync 1, 256;" ::: "memory");
+        asm volatile("bar.sync 1, %0;" ::"n"(kEpiThreads) : "memory");
         if (s_stopm[b]) { ok = false; break; }
       } else {
         // each epilogue thread waits for the tile itself; no named barrier in the loop
@@ -372,13 +387,13 @@ k_phi_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtens
       }
       tc_fence_after();
       float v[HC];
-      tmem_ld32(tS[b] + lane_addr + half * HC, v);
+      tmem_ld16(tS[b] + lane_addr + grp * HC, v);
       tmem_wait_ld();
       tc_fence_before();
       mbar_arrive(s_empty + b);
-      const int kvalid = min(BN, p.T - j * BN) - half * HC;   // valid columns of this half
+      const int kvalid = min(BN, p.T - j * BN) - grp * HC;   // valid columns of this group
       // per-key additive term: (b_j − c)·log2e (PHI) or b_j (MAX); a constant without a prior bias
-      const int jb = j * BN + half * HC;
+      const int jb = j * BN + grp * HC;
       auto bias_at = [&](int cc) -> float {
         const int jg = jb + cc;
         const float bj = jg < p.T ? __ldg(key_bias + (int64_t)h * p.T + jg) : 0.f;
@@ -411,7 +426,7 @@ k_phi_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtens
       for (int cc = 0; cc < HC; ++cc) a4[cc & 3] += (double)v[cc];
       mrow += (a4[0] + a4[1]) + (a4[2] + a4[3]);
       if (i < p.ldn) {
-        float* col = phi_base + (int64_t)(j * BN + half * HC) * p.ldn + i;
+        float* col = phi_base + (int64_t)(j * BN + grp * HC) * p.ldn + i;
         if (kvalid >= HC) {
 #pragma unroll
           for (int cc = 0; cc < HC; ++cc) col[(int64_t)cc * p.ldn] = v[cc];
@@ -421,7 +436,7 @@ k_phi_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtens
             if (cc < kvalid) col[(int64_t)cc * p.ldn] = v[cc];
         }
         if (w.phiT16) {   // bf16 copy streamed by the correlation pass
-          __nv_bfloat16* col16 = w.phiT16 + ((int64_t)h * p.T + j * BN + half * HC) * p.ldn + i;
+          __nv_bfloat16* col16 = w.phiT16 + ((int64_t)h * p.T + j * BN + grp * HC) * p.ldn + i;
 #pragma unroll
           for (int cc = 0; cc < HC; ++cc)
             if (cc < kvalid) col16[(int64_t)cc * p.ldn] = __float2bfloat16_rn(v[cc]);
@@ -443,7 +458,7 @@ k_phi_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtens
           hv[e] = *reinterpret_cast<const uint32_t*>(&hb);
           lv[e] = pack_bf16x2(a0 - hf.x, a1 - hf.y);
         }
-        const int pc = (half * (HC / 8) + c4) ^ (et & 7);
+        const int pc = (grp * (HC / 8) + c4) ^ (et & 7);
         *reinterpret_cast<uint4*>(hi_row + pc * 16) = make_uint4(hv[0], hv[1], hv[2], hv[3]);
         *reinterpret_cast<uint4*>(lo_row + pc * 16) = make_uint4(lv[0], lv[1], lv[2], lv[3]);
       }
@@ -454,40 +469,41 @@ k_phi_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtens
     if (MODE == MODE_MAX) {
       for (int o = 16; o; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
       if (lane == 0) s_red[warp - kEpiWarp0] = mx;
-      asm volatile("bar.sync 1, 256;" ::: "memory");
+      asm volatile("bar.sync 1, %0;" ::"n"(kEpiThreads) : "memory");
       if (ep == 0) {
         float v = s_red[0];
-        for (int k = 1; k < 8; ++k) v = fmaxf(v, s_red[k]);
+        for (int k = 1; k < 4 * kEpiGroups; ++k) v = fmaxf(v, s_red[k]);
         atomicMax(shift_ord + h, f2ord(v));
       }
     } else {
-      // combine the two halves' mass partials (fixed order: half 0 + half 1)
-      if (half == 1) s_mass[et] = mrow;
+      // combine the groups' mass partials in a fixed order: (0 + 1) + (2 + 3)
+      s_mass[grp][et] = mrow;
       if (ep == 0) s_stop_y = (ok && mbar_wait(y_full, 0, abort_flag, status)) ? 0 : 1;
-      asm volatile("bar.sync 1, 256;" ::: "memory");
-      if (half == 0) s_mass[128 + et] = mrow + s_mass[et];
-      asm volatile("bar.sync 1, 256;" ::: "memory");
-      const double mtot = s_mass[128 + et];
+      asm volatile("bar.sync 1, %0;" ::"n"(kEpiThreads) : "memory");
+      if (grp == 0) s_mass[kEpiGroups][et] = (s_mass[0][et] + s_mass[1][et]) + (s_mass[2][et] + s_mass[3][et]);
+      asm volatile("bar.sync 1, %0;" ::"n"(kEpiThreads) : "memory");
+      const double mtot = s_mass[kEpiGroups][et];
       if (!s_stop_y) {
         tc_fence_after();
         float* yrow = w.Y + ((int64_t)h * p.n + i) * p.d;
+        constexpr int YC = D / kEpiGroups;   // target columns of this group
 #pragma unroll
-        for (int c0 = 0; c0 < D / 2; c0 += 32) {
-          const int cb = half * (D / 2) + c0;
-          float y[32];
-          tmem_ld32(tY + lane_addr + cb, y);
+        for (int c0 = 0; c0 < YC; c0 += 16) {
+          const int cb = grp * YC + c0;
+          float y[16];
+          tmem_ld16(tY + lane_addr + cb, y);
           tmem_wait_ld();
           if (row_live) {
             // a query whose every feature underflowed has no mass: zero target
             const double im = mtot > 0.0 ? 1.0 / mtot : 0.0;
 #pragma unroll
-            for (int cc = 0; cc < 32; cc += 4)
+            for (int cc = 0; cc < 16; cc += 4)
               *reinterpret_cast<float4*>(yrow + cb + cc) =
                   make_float4((float)(y[cc] * im), (float)(y[cc + 1] * im), (float)(y[cc + 2] * im),
                               (float)(y[cc + 3] * im));
           }
         }
-        if (half == 0 && i < p.ldn) {
+        if (grp == 0 && i < p.ldn) {
           const double mv = row_live ? mtot : 0.0;
           w.m[(int64_t)h * p.ldn + i] = mv;
           w.r[(int64_t)h * p.ldn + i] = (float)mv;
