@@ -43,7 +43,8 @@ class AmWorkspaceView(ctypes.Structure):
     """Mirror of am_workspace_view_t."""
     _fields_ = [("phiT", ctypes.c_size_t), ("mass", ctypes.c_size_t), ("target", ctypes.c_size_t),
                 ("shift", ctypes.c_size_t), ("ldn", ctypes.c_int32), ("reserved", ctypes.c_int32),
-                ("weights", ctypes.c_size_t), ("resid", ctypes.c_size_t)]
+                ("weights", ctypes.c_size_t), ("resid", ctypes.c_size_t),
+                ("rows_evaluated", ctypes.c_size_t)]
 
 
 class AmOpts(ctypes.Structure):
@@ -161,6 +162,7 @@ def features(out: Dict, n: int, T: int, d: int, budgets: Sequence[int], topk: in
         "shift": view(v.shift, H, torch.float32),
         "weights": view(v.weights, int(sum(budgets)), torch.float64),
         "resid": view(v.resid, H * v.ldn, torch.float32).view(H, v.ldn),
+        "rows_evaluated": view(v.rows_evaluated, H, torch.int64),
         "ldn": v.ldn,
     }
 
@@ -258,7 +260,7 @@ def compact_heads(Q, K, V, budgets: Sequence[int], topk: int = 1, refit_every: i
 
 
 STAGES = ["shift", "phi", "target", "init", "corr", "select", "gram", "nnls", "resid",
-          "finalize", "design", "normal", "solve"]
+          "finalize", "design", "normal", "solve", "norms", "rows"]
 
 
 def profile_enable(on: bool = True) -> None:

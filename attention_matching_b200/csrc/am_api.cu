@@ -3,14 +3,18 @@
 // One call compacts H independent heads (the per-(layer, KV-head) problems of
 // "Fast KV Compaction via Attention Matching", zhichai.net deep dive §1.6;
 // varlen packing of non-uniform budgets per the zhichai.net/en summary,
-// "Engineering Practicality").  All work is enqueued on the caller's stream;
-// no device memory is allocated here.
+// "Engineering Practicality").  All work is ordered after the caller's stream
+// and the caller's stream waits for all of it; no device memory is allocated
+// here.  The OMP passes of different head groups run on internal streams of
+// their own (the heads are independent), so one group's latency-bound
+// refits overlap another group's bandwidth-bound passes.
 #include "am_internal.cuh"
 
 #include <math.h>
 #include <string.h>
 
 #include <algorithm>
+#include <mutex>
 #include <vector>
 
 namespace am {
@@ -27,7 +31,7 @@ struct Layout {
   size_t picks, pick_corr, plist, sorted_slot;
   size_t bvec, w, w_eff, ycache;
   size_t G, L, AtA, A, AtY, nrm_part;
-  size_t cnorm, rnorm, corrd, korder, knorm, ksort, cprefix;
+  size_t cnorm, rnorm, corrd, korder, knorm, ksort, cprefix, rows_eval;
   size_t total;
   size_t tables_bytes;
 };
@@ -37,6 +41,11 @@ struct Tables {
   std::vector<int64_t> cu_t, cu_t2;
   std::vector<int32_t> order;
   std::vector<int> active;   // active heads per pass
+  // head groups for concurrent pass chains: group g holds order[g], order[g + G], ...
+  std::vector<int32_t> gorder;                // groups' orders, concatenated
+  std::vector<int> gstart;                    // [G + 1] offsets into gorder
+  std::vector<std::vector<int>> gactive;      // per group: active heads per pass
+  std::vector<int> passes;                    // OMP passes per head
   int max_t = 0;
   int64_t sum_t = 0, sum_t2 = 0;
 };
@@ -47,7 +56,7 @@ Layout plan(int n, int T, int d, int H, int64_t sum_t, int64_t sum_t2, bool corr
   size_t o = 0;
   auto take = [&](size_t bytes) { size_t at = o; o = align_up(o + bytes); return at; };
   L.status = take(kWsHeaderBytes + (size_t)H * 4) + kWsHeaderBytes;   // header precedes status
-  L.tables_bytes = (size_t)H * 4 + (size_t)(H + 1) * 8 * 2 + (size_t)H * 4;
+  L.tables_bytes = (size_t)H * 4 + (size_t)(H + 1) * 8 * 2 + (size_t)H * 4 * 2;
   L.tables = take(L.tables_bytes);
   L.shift = take((size_t)H * 4);
   L.np = take((size_t)H * 4);
@@ -84,9 +93,12 @@ Layout plan(int n, int T, int d, int H, int64_t sum_t, int64_t sum_t2, bool corr
   while (t2 < (size_t)T) t2 <<= 1;
   L.ksort = take(T > kSortSmemKeys ? (size_t)H * t2 * 8 : 0);
   L.cprefix = take((size_t)H * 4);
+  L.rows_eval = take((size_t)H * 8);
   L.total = o;
   return L;
 }
+
+void set_groups(Tables* tb, const std::vector<int>& passes, int G);
 
 am_status_t check_shape(int n, int T, int d, int H, const int32_t* budgets, const am_opts_t* opts,
                         Tables* tb) {
@@ -129,7 +141,27 @@ am_status_t check_shape(int n, int T, int d, int H, const int32_t* budgets, cons
   tb->active.assign(maxp, 0);
   for (int q = 0; q < maxp; ++q)
     for (int h = 0; h < H; ++h) tb->active[q] += passes[h] > q;
+  tb->passes = passes;
+  set_groups(tb, passes, 1);
   return AM_OK;
+}
+
+// Splits the pass-ordered heads round-robin into G groups (each group's list
+// stays sorted by pass count, so a group's active heads are a prefix).
+void set_groups(Tables* tb, const std::vector<int>& passes, int G) {
+  const int H = (int)tb->order.size();
+  G = std::max(1, std::min(G, H));
+  tb->gorder.clear();
+  tb->gstart.assign(1, 0);
+  tb->gactive.assign(G, {});
+  for (int g = 0; g < G; ++g) {
+    for (int k = g; k < H; k += G) tb->gorder.push_back(tb->order[k]);
+    tb->gstart.push_back((int)tb->gorder.size());
+    const int maxp = passes[tb->gorder[tb->gstart[g]]];
+    tb->gactive[g].assign(maxp, 0);
+    for (int q = 0; q < maxp; ++q)
+      for (int k = tb->gstart[g]; k < tb->gstart[g + 1]; ++k) tb->gactive[g][q] += passes[tb->gorder[k]] > q;
+  }
 }
 
 Work bind(const Layout& L, char* base, bool corr_bf16) {
@@ -168,22 +200,40 @@ Work bind(const Layout& L, char* base, bool corr_bf16) {
   w.knorm = reinterpret_cast<float*>(base + L.knorm);
   w.ksort = reinterpret_cast<uint64_t*>(base + L.ksort);
   w.cprefix = reinterpret_cast<int32_t*>(base + L.cprefix);
+  w.rows_eval = reinterpret_cast<unsigned long long*>(base + L.rows_eval);
   return w;
 }
 
 // Packs the host tables in the device order cu_t | cu_t2 | t | order.
-void pack_tables(const Tables& tb, int H, std::vector<unsigned char>* out, Work* w, char* dev) {
+void pack_tables(const Tables& tb, int H, std::vector<unsigned char>* out, Work* w, char* dev,
+                 int32_t** gorder_dev) {
   const size_t b_cu = (size_t)(H + 1) * 8;
-  out->resize(2 * b_cu + 2 * (size_t)H * 4);
+  out->resize(2 * b_cu + 3 * (size_t)H * 4);
   unsigned char* o = out->data();
   memcpy(o, tb.cu_t.data(), b_cu);
   memcpy(o + b_cu, tb.cu_t2.data(), b_cu);
   memcpy(o + 2 * b_cu, tb.t.data(), (size_t)H * 4);
   memcpy(o + 2 * b_cu + (size_t)H * 4, tb.order.data(), (size_t)H * 4);
+  memcpy(o + 2 * b_cu + (size_t)H * 8, tb.gorder.data(), (size_t)H * 4);
   w->cu_t = reinterpret_cast<int64_t*>(dev);
   w->cu_t2 = reinterpret_cast<int64_t*>(dev + b_cu);
   w->t = reinterpret_cast<int32_t*>(dev + 2 * b_cu);
   w->order = reinterpret_cast<int32_t*>(dev + 2 * b_cu + (size_t)H * 4);
+  *gorder_dev = reinterpret_cast<int32_t*>(dev + 2 * b_cu + (size_t)H * 8);
+}
+
+// Internal streams for the head groups, created once per device.
+constexpr int kMaxGroups = 4;
+constexpr int kMaxDevices = 64;
+cudaStream_t group_stream(int g) {
+  static std::mutex mu;
+  static cudaStream_t streams[kMaxDevices][kMaxGroups] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  std::lock_guard<std::mutex> lock(mu);
+  if (!streams[dev][g] && cudaStreamCreateWithFlags(&streams[dev][g], cudaStreamNonBlocking) != cudaSuccess)
+    streams[dev][g] = nullptr;
+  return streams[dev][g];
 }
 
 Problem make_problem(int n, int T, int d, int H, const am_opts_t* o, const Tables& tb) {
@@ -256,6 +306,7 @@ am_status_t am_workspace_view(int32_t n, int32_t T, int32_t d, int32_t num_heads
   view->reserved = 0;
   view->weights = L.w;
   view->resid = L.r;
+  view->rows_evaluated = L.rows_eval;
   return AM_OK;
 }
 
@@ -263,10 +314,26 @@ am_status_t am_compact_heads(const void* Q, const void* K, const void* V, int32_
                              int32_t d, int32_t H, const int32_t* budgets, const am_opts_t* opts,
                              void* workspace, size_t workspace_bytes, const int64_t* out_offsets,
                              void* C_k, float* beta, float* C_v, int32_t* indices, void* stream) {
+  return am::compact_heads_impl(Q, K, V, n, T, d, H, budgets, opts, workspace, workspace_bytes, out_offsets, C_k,
+                                beta, C_v, indices, stream, am::kMaxGroups);
+}
+
+}  // extern "C"
+
+namespace am {
+am_status_t compact_heads_impl(const void* Q, const void* K, const void* V, int32_t n, int32_t T, int32_t d,
+                               int32_t H, const int32_t* budgets, const am_opts_t* opts, void* workspace,
+                               size_t workspace_bytes, const int64_t* out_offsets, void* C_k, float* beta,
+                               float* C_v, int32_t* indices, void* stream, int max_groups) {
   if (!Q || !K || !V || !C_k || !beta || !C_v || !indices || !out_offsets) return AM_ERR_INVALID_ARG;
   Tables tb;
   am_status_t st = check_shape(n, T, d, H, budgets, opts, &tb);
   if (st != AM_OK) return st;
+  // head groups on internal streams (one group: everything on the caller's stream)
+  int G = std::max(1, std::min(max_groups, H));
+  for (int g = 0; g < G && G > 1; ++g)
+    if (!group_stream(g)) G = 1;
+  set_groups(&tb, tb.passes, G);
   for (int h = 0; h <= H; ++h)
     if (out_offsets[h] != tb.cu_t[h]) return AM_ERR_INVALID_ARG;
   if (!workspace || ((uintptr_t)workspace % kAlign) != 0) return AM_ERR_WORKSPACE;
@@ -279,7 +346,8 @@ am_status_t am_compact_heads(const void* Q, const void* K, const void* V, int32_
   w.nrm_ata = tb.sum_t2;
   w.nrm_stride = tb.sum_t2 + tb.sum_t * d;
   std::vector<unsigned char> host_tables;
-  pack_tables(tb, H, &host_tables, &w, base + L.tables);
+  int32_t* gorder = nullptr;
+  pack_tables(tb, H, &host_tables, &w, base + L.tables, &gorder);
   const Problem p = make_problem(n, T, d, H, opts, tb);
 
   WsHeader hdr{kWsMagic, H};
@@ -311,8 +379,35 @@ am_status_t am_compact_heads(const void* Q, const void* K, const void* V, int32_
   }
   AM_TRY(launch_omp_init(p, w, s));
   if (p.corr_bounded) AM_TRY(launch_column_norms(p, w, s));
-  for (int pass = 0; pass < (int)tb.active.size(); ++pass)
-    AM_TRY(launch_omp_pass(p, w, pass, tb.active[pass], CorrInputs{Q, K, opts->key_bias}, s));
+  AM_TRY(cudaMemsetAsync(w.rows_eval, 0, (size_t)H * 8, s));
+  const CorrInputs cin{Q, K, opts->key_bias};
+  if (G == 1) {
+    for (int pass = 0; pass < (int)tb.active.size(); ++pass)
+      AM_TRY(launch_omp_pass(p, w, pass, tb.active[pass], cin, s));
+  } else {
+    // fork the groups off the caller's stream, issue their passes interleaved,
+    // and make the caller's stream wait for every group
+    cudaEvent_t fork, join[kMaxGroups];
+    AM_TRY(cudaEventCreateWithFlags(&fork, cudaEventDisableTiming));
+    AM_TRY(cudaEventRecord(fork, s));
+    std::vector<Work> wg(G, w);
+    for (int g = 0; g < G; ++g) {
+      wg[g].order = gorder + tb.gstart[g];
+      AM_TRY(cudaStreamWaitEvent(group_stream(g), fork, 0));
+    }
+    const int maxp = (int)tb.active.size();
+    for (int pass = 0; pass < maxp; ++pass)
+      for (int g = 0; g < G; ++g)
+        if (pass < (int)tb.gactive[g].size())
+          AM_TRY(launch_omp_pass(p, wg[g], pass, tb.gactive[g][pass], cin, group_stream(g)));
+    for (int g = 0; g < G; ++g) {
+      AM_TRY(cudaEventCreateWithFlags(&join[g], cudaEventDisableTiming));
+      AM_TRY(cudaEventRecord(join[g], group_stream(g)));
+      AM_TRY(cudaStreamWaitEvent(s, join[g], 0));
+      cudaEventDestroy(join[g]);   // released once the work it marks completes
+    }
+    cudaEventDestroy(fork);
+  }
   if (opts->residual_out) AM_TRY(launch_residual_norm(p, w, opts->residual_out, s));
   AM_TRY(launch_finalize(p, w, K, opts->key_bias, C_k, beta, indices, opts->w_out, opts->pick_order,
                          opts->pick_corr, s));
@@ -321,6 +416,9 @@ am_status_t am_compact_heads(const void* Q, const void* K, const void* V, int32_
 #undef AM_TRY
   return AM_OK;
 }
+}  // namespace am
+
+extern "C" {
 
 am_status_t am_get_status(const void* workspace, int32_t H, int32_t* per_head, void* stream) {
   if (!workspace || H < 1) return AM_ERR_INVALID_ARG;

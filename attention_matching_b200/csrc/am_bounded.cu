@@ -262,14 +262,17 @@ __global__ void __launch_bounds__(kBoundThreads) k_pick(Problem p, Work w, int p
   const int L = w.cprefix[h];
   const int chunk = kSelCap - kMaxPicksPerPass;
   int kept = 0;
+  unsigned long long evaluated = 0;
   for (int c = 0; c < L; c += chunk) {
     if (threadIdx.x == 0) s_cnt = kept;
     __syncthreads();
     stage_candidates(p, w, h, c, min(L, c + chunk), S, &s_cnt);
     const int n = min(s_cnt, kSelCap);
+    evaluated += (unsigned long long)(n - kept);
     sort_candidates(S, n);
     kept = min(kk, n);
   }
+  if (threadIdx.x == 0) w.rows_eval[h] += evaluated;
   if (threadIdx.x == 0) {
     uint8_t* sel = w.sel + (int64_t)h * p.T;
     const double* cd = w.corrd + (int64_t)h * p.T;
@@ -300,10 +303,10 @@ int rows_ctas_per_head(int active) {
 
 cudaError_t launch_column_norms(const Problem& p, const Work& w, cudaStream_t s) {
   dim3 g((p.T + 7) / 8, p.H);
-  AM_LAUNCH(AM_STAGE_PHI, s, k_colnorm<<<g, 256, 0, s>>>(p, w));
+  AM_LAUNCH(AM_STAGE_NORMS, s, k_colnorm<<<g, 256, 0, s>>>(p, w));
   const int sort_smem = p.T > kSortSmemKeys ? 0 : (int)(sizeof(uint64_t) * kSortSmemKeys);
   cudaFuncSetAttribute(k_sortnorm, cudaFuncAttributeMaxDynamicSharedMemorySize, sort_smem);
-  AM_LAUNCH(AM_STAGE_PHI, s, k_sortnorm<<<p.H, kBoundThreads, sort_smem, s>>>(p, w));
+  AM_LAUNCH(AM_STAGE_NORMS, s, k_sortnorm<<<p.H, kBoundThreads, sort_smem, s>>>(p, w));
   return cudaGetLastError();
 }
 
@@ -312,9 +315,9 @@ cudaError_t launch_corr_bounded(const Problem& p, const Work& w, int pass, int a
   cudaFuncSetAttribute(k_theta, cudaFuncAttributeMaxDynamicSharedMemorySize, sel_smem);
   cudaFuncSetAttribute(k_pick, cudaFuncAttributeMaxDynamicSharedMemorySize, sel_smem);
   dim3 gr(rows_ctas_per_head(active), active);
-  AM_LAUNCH(AM_STAGE_CORR, s, k_rows<<<gr, 256, 0, s>>>(p, w, pass, 0));
+  AM_LAUNCH(AM_STAGE_ROWS, s, k_rows<<<gr, 256, 0, s>>>(p, w, pass, 0));
   AM_LAUNCH(AM_STAGE_CORR, s, k_theta<<<active, kBoundThreads, sel_smem, s>>>(p, w, pass));
-  AM_LAUNCH(AM_STAGE_CORR, s, k_rows<<<gr, 256, 0, s>>>(p, w, pass, 1));
+  AM_LAUNCH(AM_STAGE_ROWS, s, k_rows<<<gr, 256, 0, s>>>(p, w, pass, 1));
   AM_LAUNCH(AM_STAGE_SELECT, s, k_pick<<<active, kBoundThreads, sel_smem, s>>>(p, w, pass));
   return cudaGetLastError();
 }

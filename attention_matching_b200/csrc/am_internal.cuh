@@ -74,6 +74,7 @@ struct Work {
   float* knorm;         // [H][T] those norms (fp32, descending)
   uint64_t* ksort;      // [H][pow2 >= T] sort scratch when T exceeds the shared-memory sort
   int32_t* cprefix;     // [H] this pass evaluates the keys at sorted positions [0, cprefix)
+  unsigned long long* rows_eval;   // [H] keys evaluated, summed over the passes
   int64_t nrm_ata;      // Σt²
   int64_t nrm_stride;   // Σt² + Σt·d
 };
@@ -121,6 +122,13 @@ cudaError_t launch_finalize(const Problem& p, const Work& w, const void* K, cons
                             void* C_k, float* beta, int32_t* indices, float* w_out,
                             int32_t* pick_order, float* pick_corr, cudaStream_t s);
 cudaError_t launch_value_fit(const Problem& p, const Work& w, float* C_v, cudaStream_t s);
+
+// The body of am_compact_heads; OMP passes of up to max_groups head groups run
+// concurrently on internal streams (1: everything on the caller's stream).
+am_status_t compact_heads_impl(const void* Q, const void* K, const void* V, int32_t n, int32_t T, int32_t d,
+                               int32_t H, const int32_t* budgets, const am_opts_t* opts, void* workspace,
+                               size_t workspace_bytes, const int64_t* out_offsets, void* C_k, float* beta,
+                               float* C_v, int32_t* indices, void* stream, int max_groups);
 
 // ---- small device helpers ----
 __host__ __device__ inline int round_up(int x, int a) { return (x + a - 1) / a * a; }

@@ -55,8 +55,9 @@ extern "C" am_status_t am_compact_heads_noalloc(const void* Q, const void* K, co
   if (need > AM_NOALLOC_SCRATCH_BYTES) return AM_ERR_WORKSPACE;
   void* scratch = nullptr;
   if (am::scratch_address(&scratch) != cudaSuccess) return AM_ERR_CUDA;
-  st = am_compact_heads(Q, K, V, n, T, d, H, budgets, opts, scratch, AM_NOALLOC_SCRATCH_BYTES, out_offsets, C_k,
-                        beta, C_v, indices, stream);
+  // one stream: this entry creates no stream or event either
+  st = am::compact_heads_impl(Q, K, V, n, T, d, H, budgets, opts, scratch, AM_NOALLOC_SCRATCH_BYTES, out_offsets,
+                              C_k, beta, C_v, indices, stream, 1);
   if (st != AM_OK) return st;
   if (status_out) {
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);

@@ -16,8 +16,9 @@ a device synchronize and the time is the max over ranks.
 
 Timing: per-step CUDA events on the compute stream; a 256 MiB buffer is
 written between timed steps to flush L2.  Stage times come from the
-library's own event brackets (am_profile_*), giving the live roofline of the
-dominant kernel.  `--impl reference` times the float64 CPU oracle on a
+library's own event brackets (am_profile_*) on separate untimed steps, giving
+the live roofline of the dominant stage (stages of different head groups
+overlap on the GPU, so stage times can add up to more than a step).  `--impl reference` times the float64 CPU oracle on a
 bounded sample of the same workload instead.
 """
 import argparse
@@ -181,57 +182,82 @@ def cpu_baseline(wl, heads=1):
 
 
 # -------------------------------------------------------------- roofline ----
-def stage_models(wl, n, T, d, H, ldn, passes, corr_kind="fp32"):
-    """Algorithmic bytes / flops of one launch of the main kernels."""
-    if corr_kind == "recompute":
-        corr = {"bound": "tensor", "flops": 2.0 * H * n * T * d, "exps": float(H) * n * T}
-    else:
-        corr = {"bound": "hbm", "bytes": H * (T * ldn * (2 if corr_kind == "bf16" else 4) + ldn * 4 + T * 4)}
-    return {
-        "corr": corr,
-        "phi": {"bound": "alu", "flops": 2.0 * H * n * T * d, "bytes": H * T * ldn * 4},
-        "target": {"bound": "alu", "flops": 2.0 * H * n * T * d, "bytes": H * T * ldn * 4},
-        "shift": {"bound": "alu", "flops": 2.0 * H * n * T * d},
+def stage_models(wl, n, T, d, H, ldn, corr_kind, rows_evaluated):
+    """Algorithmic work of one call (one step) per library stage: bytes that
+    must cross HBM for the memory-bound stages, dense flops for the GEMM and
+    the fp64 solver stages.  Summed over the stage's launches in the step."""
+    kR = wl.topk * wl.refit_every
+    s1 = [min((p + 1) * kR, t) for t in wl.budgets for p in range((t + kR - 1) // kR)]
+    row = ldn * 4                                   # one stored Φᵀ row (fp32)
+    m = {
+        "shift": {"bound": "tensor", "flops": 2.0 * H * n * T * d},
+        "phi": {"bound": "hbm", "bytes": H * (T * row + n * d * 2 + 2 * T * d * 2 + n * d * 4 + ldn * 12),
+                "flops": 4.0 * H * n * T * d},
+        "target": {"bound": "hbm", "bytes": H * (T * row + T * d * 4 + n * d * 4)},
+        "gram": {"bound": "hbm", "bytes": float(sum(s1)) * row},
+        "resid": {"bound": "hbm", "bytes": float(sum(s1)) * row + len(s1) * ldn * 12},
+        "nnls": {"bound": "hbm", "bytes": float(sum(2 * x * x * 8 for x in s1))},
+        "design": {"bound": "hbm", "bytes": float(sum(wl.budgets)) * row * 2},
+        "normal": {"bound": "fp64", "flops": float(sum(n * t * (t + 1) + 2 * n * t * d for t in wl.budgets))},
+        "solve": {"bound": "fp64", "flops": float(sum(t ** 3 / 3 + 2 * t * t * d for t in wl.budgets))},
     }
+    if corr_kind == "recompute":
+        m["corr"] = {"bound": "tensor", "flops": 2.0 * len(s1) * n * T * d, "exps": float(len(s1)) * n * T}
+    elif corr_kind == "bounded":
+        m["norms"] = {"bound": "hbm", "bytes": H * T * row}
+        m["rows"] = {"bound": "hbm", "bytes": float(rows_evaluated) * row}
+    else:
+        m["corr"] = {"bound": "hbm", "bytes": len(s1) * (T * ldn * (2 if corr_kind == "bf16" else 4) + row + T * 4)}
+    return m
+
+
+def stage_roofline(name, st, steps, model, peaks, clocks):
+    """Achieved rate of one stage against its roofline: the stage's algorithmic
+    work per step times the steps, over its measured device time."""
+    secs = st["ms"] * 1e-3
+    mhz = (clocks or {}).get("sm_mhz") or peaks["sm_max_mhz"]
+    out = {"kernel": name, "avg_launch_ms": st["ms"] / st["launches"], "launches_per_step": st["launches"] / steps}
+    if model is None:
+        out.update({"bound": None, "achieved": None, "peak": None, "unit": None, "frac": None})
+        return out
+    if model["bound"] == "hbm":
+        ach = model["bytes"] * steps / secs / 1e9
+        out.update({"bound": "hbm", "achieved": ach, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                    "frac": ach / peaks["hbm_gbs"], "peak_source": peaks["source"] + " hbm_gbs",
+                    "algorithmic_bytes_per_step": model["bytes"]})
+        if "flops" in model:
+            tf = model["flops"] * steps / secs / 1e12
+            out["tensor"] = {"achieved_tflops": tf, "frac_of_sustained_bf16": tf / peaks["bf16_tflops_sustained"]}
+    elif model["bound"] == "tensor":
+        ach = model["flops"] * steps / secs / 1e12
+        pk = peaks["bf16_tflops_sustained"]
+        out.update({"bound": "tensor", "achieved": ach, "peak": pk, "unit": "TFLOP/s", "frac": ach / pk,
+                    "peak_source": peaks["source"] + " bf16_tflops_sustained",
+                    "algorithmic_flops_per_step": model["flops"]})
+        if "exps" in model:
+            # one exponential per feature against the ex2 unit rate, 148 SMs x 16 per clock
+            exp_peak = 148 * 16 * mhz * 1e6
+            rate = model["exps"] * steps / secs
+            out["exp_rate"] = {"achieved_per_s": rate, "peak_per_s": exp_peak, "frac": rate / exp_peak}
+    else:
+        # fp64 FMA pipes: 148 SMs x 64 lanes x 2 flops x SM clock
+        peak = 148 * 64 * 2 * mhz * 1e6 / 1e12
+        ach = model["flops"] * steps / secs / 1e12
+        out.update({"bound": "alu", "achieved": ach, "peak": peak, "unit": "TFLOP/s", "frac": ach / peak,
+                    "peak_source": "fp64 FMA: 148 SMs x 64 lanes x 2 x median SM clock",
+                    "algorithmic_flops_per_step": model["flops"]})
+    return out
 
 
 def roofline(stages, steps, models, peaks, clocks, traffic_info):
+    """The dominant stage's roofline (the JSON contract), plus every stage's."""
     per = {k: v for k, v in stages.items() if v["launches"] > 0}
     dom = max(per, key=lambda k: per[k]["ms"])
-    launches = per[dom]["launches"]
-    avg_ms = per[dom]["ms"] / launches
-    m = models.get(dom)
-    out = {"kernel": dom, "avg_launch_ms": avg_ms, "launches_per_step": launches / steps}
-    if m is None:
-        out.update({"bound": None, "achieved": None, "peak": None, "unit": None, "frac": None, "traffic": None})
-        return out
-    if m["bound"] == "hbm":
-        ach = m["bytes"] / (avg_ms * 1e-3) / 1e9
-        out.update({"bound": "hbm", "achieved": ach, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                    "frac": ach / peaks["hbm_gbs"], "peak_source": peaks["source"] + " hbm_gbs",
-                    "algorithmic_bytes_per_launch": m["bytes"]})
-    elif m["bound"] == "tensor":
-        # dense bf16 MMA work of the launch against the sustained cuBLAS peak; the
-        # epilogue's exponentials (one per feature) are reported against the
-        # ex2 unit rate, 148 SMs x 16 per clock x median SM clock
-        ach = m["flops"] / (avg_ms * 1e-3) / 1e12
-        pk = peaks["bf16_tflops_sustained"]
-        mhz = (clocks or {}).get("sm_mhz") or peaks["sm_max_mhz"]
-        exp_peak = 148 * 16 * mhz * 1e6
-        out.update({"bound": "tensor", "achieved": ach, "peak": pk, "unit": "TFLOP/s", "frac": ach / pk,
-                    "peak_source": peaks["source"] + " bf16_tflops_sustained",
-                    "algorithmic_flops_per_launch": m["flops"],
-                    "exp_rate": {"achieved_per_s": m["exps"] / (avg_ms * 1e-3), "peak_per_s": exp_peak,
-                                 "frac": m["exps"] / (avg_ms * 1e-3) / exp_peak}})
-    else:
-        # fp32 FMA pipes: 148 SMs x 128 lanes x 2 flops x SM clock
-        mhz = (clocks or {}).get("sm_mhz") or peaks["sm_max_mhz"]
-        peak = 148 * 128 * 2 * mhz * 1e6 / 1e12
-        ach = m["flops"] / (avg_ms * 1e-3) / 1e12
-        out.update({"bound": "alu", "achieved": ach, "peak": peak, "unit": "TFLOP/s", "frac": ach / peak,
-                    "peak_source": "fp32 FMA: 148 SMs x 128 lanes x 2 x median SM clock",
-                    "algorithmic_flops_per_launch": m["flops"]})
+    out = stage_roofline(dom, per[dom], steps, models.get(dom), peaks, clocks)
     out["traffic"] = traffic_info.get(dom)
+    out["all_stages"] = {k: {kk: vv for kk, vv in stage_roofline(k, v, steps, models.get(k), peaks, clocks).items()
+                             if kk in ("bound", "achieved", "unit", "frac", "avg_launch_ms", "launches_per_step")}
+                         for k, v in sorted(per.items(), key=lambda kv: -kv[1]["ms"])}
     return out
 
 
@@ -321,7 +347,6 @@ def run_ours(args, rank, world, local_rank):
         dist.barrier()
     torch.cuda.synchronize()
     clocks.start()
-    am.profile_enable(True)
     l0 = am.kernel_launches()
     evs = []
     for _ in range(args.steps):
@@ -333,12 +358,18 @@ def run_ours(args, rank, world, local_rank):
         evs.append((a, b))
     torch.cuda.synchronize()
     launches = am.kernel_launches() - l0
-    am.profile_enable(False)
-    stages = am.profile_collect()
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
     clk = clocks.stop()
+    # stage times from separate, untimed steps with the library's event brackets
+    am.profile_enable(True)
+    for _ in range(args.steps):
+        flush.fill_(1)
+        am.compact_heads(Q, K, V, wl.budgets, workspace=ws, check=False, **kw)
+    torch.cuda.synchronize()
+    am.profile_enable(False)
+    stages = am.profile_collect()
     step_ms = [a.elapsed_time(b) for a, b in evs]
     ms = statistics.mean(step_ms)
     ms = max_over_ranks(ms, dist if world > 1 else None, dev)
@@ -376,10 +407,12 @@ def run_ours(args, rank, world, local_rank):
         return 0
 
     ldn = (n + 31) // 32 * 32
-    passes = max((t + wl.topk * wl.refit_every - 1) // (wl.topk * wl.refit_every) for t in wl.budgets)
     peaks = load_peaks()
-    rf = roofline(stages, args.steps, stage_models(wl, n, T, d, H, ldn, passes, corr_kind),
-                  peaks, clk, committed_traffic() if corr_kind == "fp32" else {})
+    rows_eval = int(am.features({"workspace": ws}, n, T, d, wl.budgets, wl.topk, wl.refit_every,
+                                am.BF16 if Q.dtype == torch.bfloat16 else am.FP32,
+                                corr_mode)["rows_evaluated"].sum().item())
+    rf = roofline(stages, args.steps, stage_models(wl, n, T, d, H, ldn, corr_kind, rows_eval),
+                  peaks, clk, committed_traffic())
     value = job_throughput(H, world, ms)
     per_step_stage = {k: round(v["ms"] / args.steps, 4) for k, v in stages.items() if v["launches"]}
     cfg = {"workload": wl.name, "heads_per_gpu": H, "n": n, "T": T, "d": d,
@@ -390,6 +423,7 @@ def run_ours(args, rank, world, local_rank):
                            "bounded": "exact fp64 values for the keys whose Cauchy-Schwarz bound "
                                       "reaches the pass's top k*R"}[corr_kind],
            "l2": "256 MiB buffer written between timed steps",
+           "correlation_rows_evaluated_per_step": rows_eval,
            "stage_ms_per_step": per_step_stage, "device_status": worst}
     if args.workload == "qwen3_4b_layer":
         cfg["s_per_model_extrapolated_x36_layers"] = LAYERS_QWEN3_4B * ms * 1e-3

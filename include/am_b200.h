@@ -155,12 +155,15 @@ am_status_t am_compact_heads(const void* Q_ref, const void* K, const void* V,
  *   weights fp64 [Σt]         the last NNLS refit's w, packed per head at
  *                             out_offsets[h] in PICK order (zero where w_l = 0)
  *   resid   fp32 [H][ldn]     r = m − Φ_S w after the last refit
+ *   rows_evaluated            see the field below
  * Same argument rules as am_workspace_size. */
 typedef struct am_workspace_view {
   size_t phiT, mass, target, shift;
   int32_t ldn;
   int32_t reserved;
   size_t weights, resid;
+  size_t rows_evaluated;   /* int64 [H]: keys whose correlation the bounded
+                              passes evaluated, summed over the call's passes */
 } am_workspace_view_t;
 
 am_status_t am_workspace_view(int32_t n, int32_t T, int32_t d, int32_t num_heads,
@@ -219,7 +222,7 @@ typedef enum am_stage {
   AM_STAGE_PHI = 1,      /* Φᵀ = exp(s − c_h)                        */
   AM_STAGE_TARGET = 2,   /* Y = ΦV/m and m                           */
   AM_STAGE_INIT = 3,     /* ‖m‖², selection flags                    */
-  AM_STAGE_CORR = 4,     /* c = Φᵀ r                                 */
+  AM_STAGE_CORR = 4,     /* c = Φᵀ r (bounded mode: the threshold)   */
   AM_STAGE_SELECT = 5,   /* top-k·R unselected keys                  */
   AM_STAGE_GRAM = 6,     /* Φ_SᵀΦ_S, Φ_Sᵀm updates                   */
   AM_STAGE_NNLS = 7,     /* active-set NNLS refit                    */
@@ -228,7 +231,9 @@ typedef enum am_stage {
   AM_STAGE_DESIGN = 10,  /* A = rownorm(Φ_S diag w)                  */
   AM_STAGE_NORMAL = 11,  /* AᵀA, AᵀY                                 */
   AM_STAGE_SOLVE = 12,   /* ridge Cholesky, C_v                      */
-  AM_STAGE_COUNT = 13
+  AM_STAGE_NORMS = 13,   /* bounded mode: ‖Φ_{:,j}‖, keys by norm    */
+  AM_STAGE_ROWS = 14,    /* bounded mode: exact c_j of listed keys   */
+  AM_STAGE_COUNT = 15
 } am_stage_t;
 
 am_status_t am_profile_enable(int32_t on);
