@@ -243,6 +243,14 @@ def test_nnls_deletions_twin_keys():
 
 
 @needs_cuda
+def test_bounded_correlation_long_key_axis():
+    """T = 20000 keys: the bounded correlation pass sorts the column norms in
+    workspace memory instead of shared memory (more than 16384 keys)."""
+    heads = [W.structured_head(480 + h, n=256, T=20000, d=64) for h in range(2)]
+    check_all(heads, [40, 24], 4, 2, label="T=20000")
+
+
+@needs_cuda
 def test_online_rounds_chained():
     """Online compaction (fixed cache, all but the latest 20 keys halved each
     round): three rounds whose compacted blocks carry β as a prior key bias.
