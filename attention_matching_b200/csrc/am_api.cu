@@ -31,7 +31,7 @@ struct Layout {
   size_t picks, pick_corr, plist, sorted_slot;
   size_t bvec, w, w_eff, ycache;
   size_t G, L, AtA, A, AtY, nrm_part;
-  size_t cnorm, rnorm, corrd, korder, knorm, ksort, cprefix, rows_eval;
+  size_t cnorm, rnorm, corrd, korder, knorm, ksort, cprefix, rows_eval, gpart, gcount;
   size_t total;
   size_t tables_bytes;
 };
@@ -94,6 +94,8 @@ Layout plan(int n, int T, int d, int H, int64_t sum_t, int64_t sum_t2, bool corr
   L.ksort = take(T > kSortSmemKeys ? (size_t)H * t2 * 8 : 0);
   L.cprefix = take((size_t)H * 4);
   L.rows_eval = take((size_t)H * 8);
+  L.gpart = take((size_t)kGramSplits * ((size_t)sum_t + H) * kGramMaxNew * 8);
+  L.gcount = take((size_t)H * 4);
   L.total = o;
   return L;
 }
@@ -201,6 +203,8 @@ Work bind(const Layout& L, char* base, bool corr_bf16) {
   w.ksort = reinterpret_cast<uint64_t*>(base + L.ksort);
   w.cprefix = reinterpret_cast<int32_t*>(base + L.cprefix);
   w.rows_eval = reinterpret_cast<unsigned long long*>(base + L.rows_eval);
+  w.gpart = reinterpret_cast<double*>(base + L.gpart);
+  w.gcount = reinterpret_cast<int32_t*>(base + L.gcount);
   return w;
 }
 
@@ -380,6 +384,7 @@ am_status_t compact_heads_impl(const void* Q, const void* K, const void* V, int3
   AM_TRY(launch_omp_init(p, w, s));
   if (p.corr_bounded) AM_TRY(launch_column_norms(p, w, s));
   AM_TRY(cudaMemsetAsync(w.rows_eval, 0, (size_t)H * 8, s));
+  AM_TRY(cudaMemsetAsync(w.gcount, 0, (size_t)H * 4, s));
   const CorrInputs cin{Q, K, opts->key_bias};
   if (G == 1) {
     for (int pass = 0; pass < (int)tb.active.size(); ++pass)

@@ -75,12 +75,16 @@ struct Work {
   uint64_t* ksort;      // [H][pow2 >= T] sort scratch when T exceeds the shared-memory sort
   int32_t* cprefix;     // [H] this pass evaluates the keys at sorted positions [0, cprefix)
   unsigned long long* rows_eval;   // [H] keys evaluated, summed over the passes
+  double* gpart;        // [kGramSplits·(Σt + H)·kGramMaxNew] Gram partial sums per query quarter
+  int32_t* gcount;      // [H] Gram blocks finished this pass
   int64_t nrm_ata;      // Σt²
   int64_t nrm_stride;   // Σt² + Σt·d
 };
 
 constexpr int kRedBlocks = 64;   // partial-sum slots per head for ‖r‖²
 constexpr int kSortSmemKeys = 16384;  // key counts the norm sort handles in shared memory
+constexpr int kGramSplits = 4;        // query quarters of the tiled Gram update
+constexpr int kGramMaxNew = 16;       // picks per pass the tiled Gram update takes
 constexpr int kNormalMaxSplits = 8;   // query splits of the normal-equation products
 
 // ---- launchers (each file defines its own) ----

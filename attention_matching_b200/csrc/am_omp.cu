@@ -281,6 +281,111 @@ __global__ void __launch_bounds__(256) k_gram(Problem p, Work w, int pass) {
   }
 }
 
+// Tiled form for passes of at most kGramMaxNew picks.  Block (tile, head,
+// split) takes four pick rows a (one warp each) against all new picks b of
+// the pass over a quarter of the queries; the new rows' columns are staged in
+// shared memory as fp64, once per block.  Products are exact (fp32 × fp32 in
+// fp64).  Each block writes its partial sums to the workspace; the last block
+// of a head to finish (counted with an atomic) adds the four quarters in a
+// fixed order and writes G (both triangles) and b, so the result does not
+// depend on block timing, and G[a][b], G[b][a] come out bitwise equal.
+constexpr int kGramTileRows = 4;
+constexpr int kGramChunk4 = 128;   // float4 columns per staged chunk
+
+__global__ void __launch_bounds__(kGramTileRows * 32) k_gram_tile(Problem p, Work w, int pass) {
+  extern __shared__ __align__(16) unsigned char smem[];
+  double4* stage = reinterpret_cast<double4*>(smem);   // [nb][kGramChunk4]
+  __shared__ int s_last;
+  const int h = w.order[blockIdx.y];
+  const int t = w.t[h];
+  int s0, s1;
+  pass_range(p, t, pass, s0, s1);
+  const int a0 = blockIdx.x * kGramTileRows;
+  if (s0 >= s1 || a0 >= s1) return;
+  const int nb = s1 - s0;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int a = a0 + warp;
+  const bool live = a < s1;
+  const int64_t base = w.cu_t[h];
+  const int64_t gbase = w.cu_t2[h];
+  const int n4 = p.ldn >> 2;
+  const int per = (n4 + kGramSplits - 1) / kGramSplits;
+  const int k0 = blockIdx.z * per, k1 = min(n4, k0 + per);
+  const float* P0 = w.phiT + (int64_t)h * p.T * p.ldn;
+  const float4* ra = reinterpret_cast<const float4*>(P0 + (int64_t)w.picks[base + (live ? a : s0)] * p.ldn);
+  const double2* m2 = reinterpret_cast<const double2*>(w.m + (int64_t)h * p.ldn);
+  double acc[kGramMaxNew];
+#pragma unroll
+  for (int b = 0; b < kGramMaxNew; ++b) acc[b] = 0.0;
+  double accm = 0.0;
+  for (int c0 = k0; c0 < k1; c0 += kGramChunk4) {
+    const int cw = min(kGramChunk4, k1 - c0);
+    for (int e = threadIdx.x; e < nb * cw; e += blockDim.x) {
+      const int b = e / cw, i = e - b * cw;
+      const float4 y = reinterpret_cast<const float4*>(P0 + (int64_t)w.picks[base + s0 + b] * p.ldn)[c0 + i];
+      stage[b * kGramChunk4 + i] = make_double4(y.x, y.y, y.z, y.w);
+    }
+    __syncthreads();
+    if (live) {
+      for (int i = lane; i < cw; i += 32) {
+        const float4 xf = ra[c0 + i];
+        const double4 x = make_double4(xf.x, xf.y, xf.z, xf.w);
+#pragma unroll
+        for (int b = 0; b < kGramMaxNew; ++b) {
+          if (b < nb) {
+            const double4 y = stage[b * kGramChunk4 + i];
+            acc[b] += x.x * y.x + x.y * y.y + x.z * y.z + x.w * y.w;
+          }
+        }
+        if (a >= s0) {
+          const double2 u = m2[2 * (c0 + i)], v = m2[2 * (c0 + i) + 1];
+          accm += x.x * u.x + x.y * u.y + x.z * v.x + x.w * v.y;
+        }
+      }
+    }
+    __syncthreads();
+  }
+  // partials: [split][row 0..t (row t: the new rows' b)][kR]
+  double* part = w.gpart + (int64_t)kGramSplits * (base + h) * p.kR;
+  const int64_t stride = (int64_t)(t + 1) * p.kR;
+  if (live) {
+#pragma unroll
+    for (int b = 0; b < kGramMaxNew; ++b) {
+      if (b < nb) {
+        const double v = warp_sum(acc[b]);
+        if (lane == 0) part[blockIdx.z * stride + (int64_t)a * p.kR + b] = v;
+      }
+    }
+    if (a >= s0) {
+      const double v = warp_sum(accm);
+      if (lane == 0) part[blockIdx.z * stride + (int64_t)t * p.kR + (a - s0)] = v;
+    }
+  }
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    const int blocks = (s1 + kGramTileRows - 1) / kGramTileRows * kGramSplits;
+    s_last = atomicAdd(w.gcount + h, 1) == blocks - 1;
+  }
+  __syncthreads();
+  if (!s_last) return;
+  __threadfence();
+  for (int e = threadIdx.x; e < (s1 + 1) * nb; e += blockDim.x) {
+    const int r = e / nb, b = e - r * nb;
+    const int row = r < s1 ? r : t;                  // the last entry row holds b
+    double v = 0.0;
+#pragma unroll
+    for (int z = 0; z < kGramSplits; ++z) v += part[z * stride + (int64_t)row * p.kR + b];
+    if (r < s1) {
+      w.G[gbase + (int64_t)r * t + s0 + b] = v;
+      if (r < s0) w.G[gbase + (int64_t)(s0 + b) * t + r] = v;
+    } else {
+      w.bvec[base + s0 + b] = v;
+    }
+  }
+  if (threadIdx.x == 0) w.gcount[h] = 0;   // ready for the next pass
+}
+
 // ---------------------------------------------------------------- NNLS ----
 // Lawson-Hanson active set on the normal equations G w = b in fp64, with
 // the Cholesky factor of G restricted to the passive set kept across refits.
@@ -898,7 +1003,12 @@ __global__ void __launch_bounds__(kNnlsThreads) k_nnls(Problem p, Work w, int pa
 
 // ------------------------------------------------------------ residual ----
 // r = m − Φ_S w over all current picks; fp64 sums, fp32 store; partial ‖r‖².
-constexpr int kResidThreads = 128;
+// A block covers 128 float4 positions (512 queries) with four thread groups,
+// group g taking picks g, g + 4, ...; the groups' sums are combined in a
+// fixed order, so the result is deterministic.
+constexpr int kResidPos = 128;     // float4 positions per block
+constexpr int kResidGroups = 4;    // pick groups per position
+constexpr int kResidThreads = kResidPos * kResidGroups;
 constexpr int kResidChunk = 512;   // picks staged in shared memory at a time
 
 __global__ void __launch_bounds__(kResidThreads) k_resid(Problem p, Work w, int pass) {
@@ -909,16 +1019,18 @@ __global__ void __launch_bounds__(kResidThreads) k_resid(Problem p, Work w, int 
   if (s0 >= s1) return;
   __shared__ int sj[kResidChunk];
   __shared__ double sw[kResidChunk];
+  __shared__ double4 part[kResidGroups - 1][kResidPos];
   __shared__ double scratch[33];
   const int64_t base = w.cu_t[h];
   const float* P0 = w.phiT + (int64_t)h * p.T * p.ldn;
   const int n4 = p.ldn >> 2;
+  const int g = threadIdx.x / kResidPos, li = threadIdx.x % kResidPos;
   double rr = 0.0;
-  for (int i4 = blockIdx.x * kResidThreads + threadIdx.x; i4 - (int)threadIdx.x < n4;
-       i4 += gridDim.x * kResidThreads) {
+  for (int b4 = blockIdx.x * kResidPos; b4 < n4; b4 += gridDim.x * kResidPos) {
+    const int i4 = b4 + li;
     const bool live = i4 < n4;
     double acc[4] = {0.0, 0.0, 0.0, 0.0};
-    if (live) {
+    if (live && g == 0) {
       const double2* m2 = reinterpret_cast<const double2*>(w.m + (int64_t)h * p.ldn);
       const double2 u = m2[2 * i4], v = m2[2 * i4 + 1];
       acc[0] = u.x; acc[1] = u.y; acc[2] = v.x; acc[3] = v.y;
@@ -932,15 +1044,31 @@ __global__ void __launch_bounds__(kResidThreads) k_resid(Problem p, Work w, int 
       }
       __syncthreads();
       if (live) {
-        for (int q = 0; q < cn; ++q) {
-          const double wl = sw[q];
-          if (wl == 0.0) continue;
-          float4 x = reinterpret_cast<const float4*>(P0 + (int64_t)sj[q] * p.ldn)[i4];
-          acc[0] -= x.x * wl; acc[1] -= x.y * wl; acc[2] -= x.z * wl; acc[3] -= x.w * wl;
+        for (int q0 = g; q0 < cn; q0 += 4 * kResidGroups) {   // four picks in flight
+          float4 x[4];
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const int q = q0 + u * kResidGroups;
+            x[u] = q < cn ? reinterpret_cast<const float4*>(P0 + (int64_t)sj[q] * p.ldn)[i4]
+                          : make_float4(0.f, 0.f, 0.f, 0.f);
+          }
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const int q = q0 + u * kResidGroups;
+            const double wl = q < cn ? sw[q] : 0.0;
+            acc[0] -= x[u].x * wl; acc[1] -= x[u].y * wl; acc[2] -= x[u].z * wl; acc[3] -= x[u].w * wl;
+          }
         }
       }
     }
-    if (live) {
+    if (g > 0) part[g - 1][li] = make_double4(acc[0], acc[1], acc[2], acc[3]);
+    __syncthreads();
+    if (g == 0 && live) {
+#pragma unroll
+      for (int k = 0; k < kResidGroups - 1; ++k) {
+        const double4 o = part[k][li];
+        acc[0] += o.x; acc[1] += o.y; acc[2] += o.z; acc[3] += o.w;
+      }
       float4 o = make_float4((float)acc[0], (float)acc[1], (float)acc[2], (float)acc[3]);
       reinterpret_cast<float4*>(w.r + (int64_t)h * p.ldn)[i4] = o;
       rr += acc[0] * acc[0] + acc[1] * acc[1] + acc[2] * acc[2] + acc[3] * acc[3];
@@ -960,7 +1088,7 @@ __global__ void k_residual_norm(Problem p, Work w, int nblk, double* out) {
 
 int resid_blocks(const Problem& p) {
   int n4 = p.ldn / 4;
-  int b = (n4 + kResidThreads - 1) / kResidThreads;
+  int b = (n4 + kResidPos - 1) / kResidPos;
   return b < kRedBlocks ? b : kRedBlocks;
 }
 
@@ -999,8 +1127,15 @@ cudaError_t launch_omp_pass(const Problem& p, const Work& w, int pass, int activ
     AM_LAUNCH(AM_STAGE_SELECT, s, k_select<<<active, 1024, 0, s>>>(p, w, pass));
   }
   const int s1max = (pass + 1) * p.kR < p.max_t ? (pass + 1) * p.kR : p.max_t;
-  dim3 gg(s1max, active);
-  AM_LAUNCH(AM_STAGE_GRAM, s, k_gram<<<gg, 256, 0, s>>>(p, w, pass));
+  if (p.kR <= kGramMaxNew) {
+    dim3 gg((s1max + kGramTileRows - 1) / kGramTileRows, active, kGramSplits);
+    const int gsm = p.kR * kGramChunk4 * (int)sizeof(double4);
+    cudaFuncSetAttribute(k_gram_tile, cudaFuncAttributeMaxDynamicSharedMemorySize, gsm);
+    AM_LAUNCH(AM_STAGE_GRAM, s, k_gram_tile<<<gg, kGramTileRows * 32, gsm, s>>>(p, w, pass));
+  } else {
+    dim3 gg(s1max, active);
+    AM_LAUNCH(AM_STAGE_GRAM, s, k_gram<<<gg, 256, 0, s>>>(p, w, pass));
+  }
   int lcap;
   size_t sm = nnls_smem_bytes(p.max_t, &lcap);
   cudaFuncSetAttribute(k_nnls, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemCap);
