@@ -129,9 +129,14 @@ __global__ void __launch_bounds__(kBoundThreads) k_sortnorm(Problem p, Work w) {
 
 // ------------------------------------------------------------ exact rows --
 // c_j = Σ_i r_i Φ_ij for the unselected keys at sorted positions [0, P0)
-// (which = 0) or [P0, L) (which = 1): one warp per key, fp64 sums of exact
-// fp32 products, four float4 loads per lane in flight.
+// (which = 0) or [P0, L) (which = 1), in fp64 sums of exact fp32 products.
+// Four warps share a key, each summing a quarter of the queries with four
+// columns per lane in flight; the quarters are added in a fixed order.
+constexpr int kRowSplit = 4;                 // warps per key
+constexpr int kRowsPerBlock = 8 / kRowSplit; // keys per 256-thread block
+
 __global__ void __launch_bounds__(256) k_rows(Problem p, Work w, int pass, int which) {
+  __shared__ double part[kRowsPerBlock][kRowSplit];
   const int h = w.order[blockIdx.y];
   int s0, s1;
   pass_range(p, w.t[h], pass, s0, s1);
@@ -140,33 +145,43 @@ __global__ void __launch_bounds__(256) k_rows(Problem p, Work w, int pass, int w
   const int lo = which ? p0 : 0;
   const int hi = which ? w.cprefix[h] : p0;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int slot = warp / kRowSplit, quarter = warp % kRowSplit;
   const int32_t* ord = w.korder + (int64_t)h * p.T;
   const uint8_t* sel = w.sel + (int64_t)h * p.T;
   const float4* r4 = reinterpret_cast<const float4*>(w.r + (int64_t)h * p.ldn);
   const int n4 = p.ldn >> 2;
-  for (int q = lo + blockIdx.x * 8 + warp; q < hi; q += gridDim.x * 8) {
-    const int j = ord[q];
-    if (sel[j]) continue;
-    const float4* row = reinterpret_cast<const float4*>(w.phiT + ((int64_t)h * p.T + j) * p.ldn);
+  const int per = (n4 + kRowSplit - 1) / kRowSplit;
+  const int c0 = quarter * per, c1 = min(n4, c0 + per);
+  for (int q0 = lo + blockIdx.x * kRowsPerBlock; q0 < hi; q0 += gridDim.x * kRowsPerBlock) {
+    const int q = q0 + slot;
+    const int j = q < hi ? ord[q] : 0;
+    const bool on = q < hi && !sel[j];
     double a[4] = {0.0, 0.0, 0.0, 0.0};
-    for (int i0 = lane; i0 < n4; i0 += 32 * 4) {
-      float4 x[4], y[4];
+    if (on) {
+      const float4* row = reinterpret_cast<const float4*>(w.phiT + ((int64_t)h * p.T + j) * p.ldn);
+      for (int i0 = c0 + lane; i0 < c1; i0 += 32 * 4) {
+        float4 x[4], y[4];
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int i = i0 + 32 * u;
-        x[u] = i < n4 ? __ldcs(row + i) : make_float4(0.f, 0.f, 0.f, 0.f);
-        y[u] = i < n4 ? __ldg(r4 + i) : make_float4(0.f, 0.f, 0.f, 0.f);
-      }
+        for (int u = 0; u < 4; ++u) {
+          const int i = i0 + 32 * u;
+          x[u] = i < c1 ? __ldcs(row + i) : make_float4(0.f, 0.f, 0.f, 0.f);
+          y[u] = i < c1 ? __ldg(r4 + i) : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        a[0] = fma((double)x[u].x, (double)y[u].x, a[0]);
-        a[1] = fma((double)x[u].y, (double)y[u].y, a[1]);
-        a[2] = fma((double)x[u].z, (double)y[u].z, a[2]);
-        a[3] = fma((double)x[u].w, (double)y[u].w, a[3]);
+        for (int u = 0; u < 4; ++u) {
+          a[0] = fma((double)x[u].x, (double)y[u].x, a[0]);
+          a[1] = fma((double)x[u].y, (double)y[u].y, a[1]);
+          a[2] = fma((double)x[u].z, (double)y[u].z, a[2]);
+          a[3] = fma((double)x[u].w, (double)y[u].w, a[3]);
+        }
       }
     }
     const double c = warp_sum((a[0] + a[1]) + (a[2] + a[3]));
-    if (lane == 0) w.corrd[(int64_t)h * p.T + j] = c;
+    if (lane == 0) part[slot][quarter] = c;
+    __syncthreads();
+    if (on && quarter == 0 && lane == 0)
+      w.corrd[(int64_t)h * p.T + j] = (part[slot][0] + part[slot][1]) + (part[slot][2] + part[slot][3]);
+    __syncthreads();
   }
 }
 
@@ -295,8 +310,8 @@ __global__ void __launch_bounds__(kBoundThreads) k_pick(Problem p, Work w, int p
 }
 
 int rows_ctas_per_head(int active) {
-  const int c = (2 * 148 + active - 1) / active;
-  return c < 1 ? 1 : (c > 64 ? 64 : c);
+  const int c = (8 * 148 + active - 1) / active;
+  return c < 1 ? 1 : (c > 256 ? 256 : c);
 }
 
 }  // namespace
