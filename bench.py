@@ -412,7 +412,7 @@ def run_ours(args, rank, world, local_rank):
                                 am.BF16 if Q.dtype == torch.bfloat16 else am.FP32,
                                 corr_mode)["rows_evaluated"].sum().item())
     rf = roofline(stages, args.steps, stage_models(wl, n, T, d, H, ldn, corr_kind, rows_eval),
-                  peaks, clk, committed_traffic())
+                  peaks, clk, committed_traffic() if corr_kind == "fp32" else {})
     value = job_throughput(H, world, ms)
     per_step_stage = {k: round(v["ms"] / args.steps, 4) for k, v in stages.items() if v["launches"]}
     cfg = {"workload": wl.name, "heads_per_gpu": H, "n": n, "T": T, "d": d,
