@@ -31,7 +31,7 @@ struct Layout {
   size_t picks, pick_corr, plist, sorted_slot;
   size_t bvec, w, w_eff, ycache;
   size_t G, L, AtA, A, AtY, nrm_part;
-  size_t cnorm, rnorm, corrd, korder, knorm, ksort, cprefix, rows_eval, gpart, gcount;
+  size_t cnorm, rnorm, corrd, korder, knorm, ksort, cprefix, rows_eval, gpart, gcount, rcount;
   size_t total;
   size_t tables_bytes;
 };
@@ -96,6 +96,7 @@ Layout plan(int n, int T, int d, int H, int64_t sum_t, int64_t sum_t2, bool corr
   L.rows_eval = take((size_t)H * 8);
   L.gpart = take((size_t)kGramSplits * ((size_t)sum_t + H) * kGramMaxNew * 8);
   L.gcount = take((size_t)H * 4);
+  L.rcount = take((size_t)H * 4);
   L.total = o;
   return L;
 }
@@ -205,6 +206,7 @@ Work bind(const Layout& L, char* base, bool corr_bf16) {
   w.rows_eval = reinterpret_cast<unsigned long long*>(base + L.rows_eval);
   w.gpart = reinterpret_cast<double*>(base + L.gpart);
   w.gcount = reinterpret_cast<int32_t*>(base + L.gcount);
+  w.rcount = reinterpret_cast<int32_t*>(base + L.rcount);
   return w;
 }
 
@@ -385,6 +387,7 @@ am_status_t compact_heads_impl(const void* Q, const void* K, const void* V, int3
   if (p.corr_bounded) AM_TRY(launch_column_norms(p, w, s));
   AM_TRY(cudaMemsetAsync(w.rows_eval, 0, (size_t)H * 8, s));
   AM_TRY(cudaMemsetAsync(w.gcount, 0, (size_t)H * 4, s));
+  AM_TRY(cudaMemsetAsync(w.rcount, 0, (size_t)H * 4, s));
   const CorrInputs cin{Q, K, opts->key_bias};
   if (G == 1) {
     for (int pass = 0; pass < (int)tb.active.size(); ++pass)

@@ -6,24 +6,23 @@
 // For every key |c_j| = |rᵀΦ_{:,j}| <= ‖r‖₂·‖Φ_{:,j}‖₂ (Cauchy-Schwarz).  The
 // column norms do not depend on r, so once per call the keys are sorted by
 // norm (k_colnorm, k_sortnorm); in every pass the keys a bound cannot exclude
-// then form a prefix of that order.  One pass of kk = s1 − s0 picks per head:
-//   1. k_rows    exact c_j for the unselected keys among the first
-//                P0 = kProbe + s0 sorted positions (so at least kProbe keys):
-//                fp64 sums of the stored fp32 features times the stored fp32
-//                residual;
-//   2. k_theta   θ = the kk-th largest of those values, and the prefix length
-//                L: every key with ‖Φ_{:,j}‖ >= θ / (‖r‖(1 + 1e-9)) lies in
-//                [0, L) (binary search in the sorted norms);
-//   3. k_rows    exact c_j for the unselected keys in [P0, L);
-//   4. k_pick    appends the kk largest values of [0, L) (ties to the lower
-//                key).
+// then form a prefix of that order.  One pass of kk = s1 − s0 picks per head
+// is two launches of k_rows:
+//   1. exact c_j for the unselected keys among the first P0 = kProbe + s0
+//      sorted positions (so at least kProbe keys): fp64 sums of the stored
+//      fp32 features times the stored fp32 residual; then the last block of
+//      the head takes θ = the kk-th largest of those values and the prefix
+//      length L: every key with ‖Φ_{:,j}‖ >= θ / (‖r‖(1 + 1e-9)) lies in
+//      [0, L) (a count over the sorted norms);
+//   2. exact c_j for the unselected keys in [P0, L); then the last block
+//      appends the kk largest values of [0, L) (ties to the lower key).
 // A key beyond L has c_j < θ while kk keys in the prefix reach θ, so it is not
 // among the kk largest: the picks are those of a full pass over all keys.
 // The margin 1e-9 covers the rounding of the fp64 sums and norms (relative
 // error below n·2^-53 for the sums, a few ulp for the norms); the fp32 copies
 // of the norms only move the cut outward (rounding to nearest is monotone).
-// The selections sort their candidates with a bitonic network in shared
-// memory (no serial merge, no atomics).
+// The selections take kk rounds of a block-wide argmax over candidates staged
+// in shared memory.
 #include "am_internal.cuh"
 #include "am_profile.cuh"
 #include "am_linalg.cuh"
@@ -35,7 +34,7 @@ namespace {
 
 constexpr int kProbe = 256;        // unselected keys whose exact values set the threshold
 constexpr int kBoundThreads = 1024;
-constexpr int kSelCap = 4096;      // candidates one selection sort holds
+constexpr int kSelCap = 2304;      // candidates one selection holds (>= kProbe + 2048)
 constexpr double kBoundMargin = 1e-9;
 
 // Order-preserving map of a double to uint64 (NaN ranks lowest).
@@ -48,28 +47,6 @@ __device__ __forceinline__ uint64_t order_key(double v) {
 // (a, ja) before (b, jb) in pick order: larger key first, then lower index.
 __device__ __forceinline__ bool before(uint64_t a, int ja, uint64_t b, int jb) {
   return a > b || (a == b && ja < jb);
-}
-
-// Sorts the n2 (a power of two) pairs (key, idx) into pick order with a
-// bitonic network; all threads of the block.
-__device__ void bitonic_pairs(uint64_t* key, int* idx, int n2) {
-  for (int k = 2; k <= n2; k <<= 1) {
-    for (int jj = k >> 1; jj > 0; jj >>= 1) {
-      for (int i = threadIdx.x; i < n2; i += blockDim.x) {
-        const int l = i ^ jj;
-        if (l > i) {
-          const bool up = (i & k) == 0;   // this block in pick order, else reversed
-          const uint64_t a = key[i], b = key[l];
-          const int ia = idx[i], ib = idx[l];
-          if (up ? before(b, ib, a, ia) : before(a, ia, b, ib)) {
-            key[i] = b; key[l] = a;
-            idx[i] = ib; idx[l] = ia;
-          }
-        }
-      }
-      __syncthreads();
-    }
-  }
 }
 
 // ---------------------------------------------------------- column norms --
@@ -127,20 +104,173 @@ __global__ void __launch_bounds__(kBoundThreads) k_sortnorm(Problem p, Work w) {
   }
 }
 
+// ------------------------------------------------------------ selection --
+constexpr int kSelThreads = 256;
+
+struct SelScratch {
+  uint64_t key[kSelCap];
+  int idx[kSelCap];
+  uint64_t wk[kSelThreads / 32];
+  int wj[kSelThreads / 32], wp[kSelThreads / 32];
+  uint64_t outk[kMaxPicksPerPass];
+  int outj[kMaxPicksPerPass];
+  double red[33];
+  int cnt;
+};
+
+// Appends the unselected keys at sorted positions [lo, hi) to the candidate
+// slots from S.cnt on (at most kSelCap in all); all threads.
+__device__ void stage_candidates(const Problem& p, const Work& w, int h, int lo, int hi, SelScratch& S) {
+  const int32_t* ord = w.korder + (int64_t)h * p.T;
+  const uint8_t* sel = w.sel + (int64_t)h * p.T;
+  const double* cd = w.corrd + (int64_t)h * p.T;
+  for (int q = lo + threadIdx.x; q < hi; q += blockDim.x) {
+    const int j = ord[q];
+    if (sel[j]) continue;
+    const int pos = atomicAdd(&S.cnt, 1);
+    if (pos < kSelCap) {
+      S.key[pos] = order_key(cd[j]);
+      S.idx[pos] = j;
+    }
+  }
+  __syncthreads();
+}
+
+// Keeps the better of (k, j, pos) and the lane `o` away, in pick order.
+__device__ __forceinline__ void shfl_best(uint64_t& k, int& j, int& pos, int o) {
+  const uint64_t k2 = __shfl_xor_sync(0xffffffffu, k, o);
+  const int j2 = __shfl_xor_sync(0xffffffffu, j, o);
+  const int p2 = __shfl_xor_sync(0xffffffffu, pos, o);
+  if (p2 >= 0 && (pos < 0 || before(k2, j2, k, j))) { k = k2; j = j2; pos = p2; }
+}
+
+// The kk candidates first in pick order, by kk rounds of a block-wide argmax
+// over slots [0, n): into S.outk / S.outj (index INT_MAX when none is left);
+// each winner's slot is cleared.  All threads.
+__device__ void select_rounds(SelScratch& S, int n, int kk) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nw = blockDim.x >> 5;
+  for (int k = 0; k < kk; ++k) {
+    uint64_t bk = 0ull;
+    int bj = INT_MAX, bp = -1;
+    for (int e = tid; e < n; e += blockDim.x) {
+      const int jv = S.idx[e];
+      if (jv == INT_MAX) continue;
+      const uint64_t kv = S.key[e];
+      if (bp < 0 || before(kv, jv, bk, bj)) { bk = kv; bj = jv; bp = e; }
+    }
+    for (int o = 16; o; o >>= 1) shfl_best(bk, bj, bp, o);
+    if (lane == 0) { S.wk[warp] = bk; S.wj[warp] = bj; S.wp[warp] = bp; }
+    __syncthreads();
+    if (warp == 0) {
+      bk = lane < nw ? S.wk[lane] : 0ull;
+      bj = lane < nw ? S.wj[lane] : INT_MAX;
+      bp = lane < nw ? S.wp[lane] : -1;
+      for (int o = 16; o; o >>= 1) shfl_best(bk, bj, bp, o);
+      if (lane == 0) {
+        S.outk[k] = bk;
+        S.outj[k] = bp >= 0 ? bj : INT_MAX;
+        if (bp >= 0) { S.key[bp] = 0ull; S.idx[bp] = INT_MAX; }
+      }
+    }
+    __syncthreads();
+  }
+}
+
+// θ and the prefix L (the last block of a head, after the probe rows).
+__device__ void theta_and_prefix(const Problem& p, const Work& w, int h, int p0, int kk, SelScratch& S) {
+  const float* r = w.r + (int64_t)h * p.ldn;
+  double a = 0.0;
+  for (int i = threadIdx.x; i < p.ldn; i += blockDim.x) {
+    const double v = r[i];
+    a = fma(v, v, a);
+  }
+  const double rn = sqrt(block_sum(a, S.red));
+  if (threadIdx.x == 0) S.cnt = 0;
+  __syncthreads();
+  stage_candidates(p, w, h, 0, p0, S);   // p0 <= kProbe + 2047 <= kSelCap unselected at most
+  select_rounds(S, min(S.cnt, kSelCap), kk);
+  const int jt = S.outj[kk - 1];
+  const double theta = jt != INT_MAX ? w.corrd[(int64_t)h * p.T + jt] : -INFINITY;
+  // L = number of sorted norms not below θ / (‖r‖(1 + margin)); every key when
+  // the bound cannot help (θ <= 0, a zero or non-finite residual)
+  const bool useful = theta > 0.0 && rn > 0.0 && rn < INFINITY;
+  const float thr = useful ? (float)(theta / (rn * (1.0 + kBoundMargin))) : 0.f;
+  const float* kn = w.knorm + (int64_t)h * p.T;
+  int count = 0;
+  if (useful)
+    for (int q = threadIdx.x; q < p.T; q += blockDim.x) count += !(kn[q] < thr);
+  const double tot = block_sum((double)count, S.red);
+  if (threadIdx.x == 0) {
+    const int L = useful ? (int)tot : p.T;
+    w.cprefix[h] = L > p0 ? L : p0;
+    w.rnorm[h] = rn;
+  }
+}
+
+// The kk largest values among the unselected keys of [0, L), in chunks that
+// carry the best kk of what came before (the last block of a head, after the
+// remaining rows).
+__device__ void pick_from_prefix(const Problem& p, const Work& w, int h, int s0, int kk, SelScratch& S) {
+  const int L = w.cprefix[h];
+  const int chunk = kSelCap - kMaxPicksPerPass;
+  int kept = 0;
+  unsigned long long evaluated = 0;
+  for (int c = 0; c < L; c += chunk) {
+    if (threadIdx.x < kept) {   // winners so far lead the next chunk
+      S.key[threadIdx.x] = S.outk[threadIdx.x];
+      S.idx[threadIdx.x] = S.outj[threadIdx.x];
+    }
+    if (threadIdx.x == 0) S.cnt = kept;
+    __syncthreads();
+    stage_candidates(p, w, h, c, min(L, c + chunk), S);
+    const int n = min(S.cnt, kSelCap);
+    evaluated += (unsigned long long)(n - kept);
+    select_rounds(S, n, kk);
+    kept = 0;
+    for (int k = 0; k < kk; ++k) kept += S.outj[k] != INT_MAX;
+  }
+  if (threadIdx.x == 0) {
+    w.rows_eval[h] += evaluated;
+    uint8_t* sel = w.sel + (int64_t)h * p.T;
+    const double* cd = w.corrd + (int64_t)h * p.T;
+    bool bad = false;
+    for (int k = 0; k < kk; ++k) {
+      int j = S.outj[k];
+      double v = j != INT_MAX ? cd[j] : -INFINITY;
+      if (j == INT_MAX || !(v == v)) {   // no finite value: lowest free key
+        bad = true;
+        for (j = 0; j < p.T && sel[j]; ++j) {}
+        v = -INFINITY;
+      }
+      const int64_t o = w.cu_t[h] + s0 + k;
+      w.picks[o] = j;
+      w.pick_corr[o] = (float)v;
+      sel[j] = 1;
+    }
+    if (bad) record_status(w.status + h, AM_ERR_NONFINITE);
+  }
+}
+
 // ------------------------------------------------------------ exact rows --
 // c_j = Σ_i r_i Φ_ij for the unselected keys at sorted positions [0, P0)
 // (which = 0) or [P0, L) (which = 1), in fp64 sums of exact fp32 products.
 // Four warps share a key, each summing a quarter of the queries with four
-// columns per lane in flight; the quarters are added in a fixed order.
-constexpr int kRowSplit = 4;                 // warps per key
-constexpr int kRowsPerBlock = 8 / kRowSplit; // keys per 256-thread block
+// columns per lane in flight; the quarters are added in a fixed order.  The
+// last block of a head to finish (counted with an atomic) then takes the
+// selection step: θ and L after the probe rows, the picks after the rest.
+constexpr int kRowSplit = 4;                           // warps per key
+constexpr int kRowsPerBlock = kSelThreads / 32 / kRowSplit;   // keys per block
 
-__global__ void __launch_bounds__(256) k_rows(Problem p, Work w, int pass, int which) {
+__global__ void __launch_bounds__(kSelThreads) k_rows(Problem p, Work w, int pass, int which) {
+  extern __shared__ __align__(16) unsigned char smem[];
+  SelScratch& S = *reinterpret_cast<SelScratch*>(smem);
   __shared__ double part[kRowsPerBlock][kRowSplit];
+  __shared__ int s_last;
   const int h = w.order[blockIdx.y];
   int s0, s1;
   pass_range(p, w.t[h], pass, s0, s1);
   if (s0 >= s1) return;
+  const int kk = s1 - s0;
   const int p0 = min(p.T, kProbe + s0);
   const int lo = which ? p0 : 0;
   const int hi = which ? w.cprefix[h] : p0;
@@ -183,130 +313,16 @@ __global__ void __launch_bounds__(256) k_rows(Problem p, Work w, int pass, int w
       w.corrd[(int64_t)h * p.T + j] = (part[slot][0] + part[slot][1]) + (part[slot][2] + part[slot][3]);
     __syncthreads();
   }
-}
-
-struct SelScratch {
-  uint64_t key[kSelCap];
-  int idx[kSelCap];
-};
-
-// Appends the unselected keys at sorted positions [lo, hi) to the candidate
-// slots from *count on (at most kSelCap in all); all threads.
-__device__ void stage_candidates(const Problem& p, const Work& w, int h, int lo, int hi, SelScratch& S,
-                                 int* count) {
-  const int32_t* ord = w.korder + (int64_t)h * p.T;
-  const uint8_t* sel = w.sel + (int64_t)h * p.T;
-  const double* cd = w.corrd + (int64_t)h * p.T;
-  for (int q = lo + threadIdx.x; q < hi; q += blockDim.x) {
-    const int j = ord[q];
-    if (sel[j]) continue;
-    const int pos = atomicAdd(count, 1);
-    if (pos < kSelCap) {
-      S.key[pos] = order_key(cd[j]);
-      S.idx[pos] = j;
-    }
-  }
+  // the last block of this head to get here takes the selection step
+  __threadfence();
   __syncthreads();
-}
-
-// Sorts the first n candidates into pick order (padding to a power of two).
-__device__ void sort_candidates(SelScratch& S, int n) {
-  int n2 = 1;
-  while (n2 < n) n2 <<= 1;
-  for (int i = n + threadIdx.x; i < n2; i += blockDim.x) {
-    S.key[i] = 0ull;
-    S.idx[i] = INT_MAX;
-  }
+  if (threadIdx.x == 0) s_last = atomicAdd(w.rcount + h, 1) == (int)gridDim.x - 1;
   __syncthreads();
-  bitonic_pairs(S.key, S.idx, n2);
-}
-
-// ------------------------------------------------------ threshold, prefix --
-__global__ void __launch_bounds__(kBoundThreads) k_theta(Problem p, Work w, int pass) {
-  extern __shared__ __align__(16) unsigned char smem[];
-  SelScratch& S = *reinterpret_cast<SelScratch*>(smem);
-  __shared__ double red[33];
-  __shared__ int s_cnt;
-  const int h = w.order[blockIdx.x];
-  int s0, s1;
-  pass_range(p, w.t[h], pass, s0, s1);
-  if (s0 >= s1) return;
-  const int kk = s1 - s0;
-  const int p0 = min(p.T, kProbe + s0);
-  const float* r = w.r + (int64_t)h * p.ldn;
-  double a = 0.0;
-  for (int i = threadIdx.x; i < p.ldn; i += blockDim.x) {
-    const double v = r[i];
-    a = fma(v, v, a);
-  }
-  const double rn = sqrt(block_sum(a, red));
-  if (threadIdx.x == 0) s_cnt = 0;
-  __syncthreads();
-  stage_candidates(p, w, h, 0, p0, S, &s_cnt);   // p0 <= kProbe + 2047 < kSelCap
-  const int n = min(s_cnt, kSelCap);
-  sort_candidates(S, n);
-  const double theta = kk <= n ? w.corrd[(int64_t)h * p.T + S.idx[kk - 1]] : -INFINITY;
-  // L = number of sorted norms not below θ / (‖r‖(1 + margin)); every key when
-  // the bound cannot help (θ <= 0, a zero or non-finite residual)
-  int count = 0;
-  const bool useful = theta > 0.0 && rn > 0.0 && rn < INFINITY;
-  const float thr = useful ? (float)(theta / (rn * (1.0 + kBoundMargin))) : 0.f;
-  const float* kn = w.knorm + (int64_t)h * p.T;
-  if (useful)
-    for (int q = threadIdx.x; q < p.T; q += blockDim.x) count += !(kn[q] < thr);
-  const double tot = block_sum((double)count, red);
-  if (threadIdx.x == 0) {
-    int L = useful ? (int)tot : p.T;
-    w.cprefix[h] = L > p0 ? L : p0;
-    w.rnorm[h] = rn;
-  }
-}
-
-// ------------------------------------------------------------------ pick --
-// The kk largest values among the unselected keys of [0, L), in chunks that
-// keep the best kk of what came before.
-__global__ void __launch_bounds__(kBoundThreads) k_pick(Problem p, Work w, int pass) {
-  extern __shared__ __align__(16) unsigned char smem[];
-  SelScratch& S = *reinterpret_cast<SelScratch*>(smem);
-  __shared__ int s_cnt;
-  const int h = w.order[blockIdx.x];
-  int s0, s1;
-  pass_range(p, w.t[h], pass, s0, s1);
-  if (s0 >= s1) return;
-  const int kk = s1 - s0;
-  const int L = w.cprefix[h];
-  const int chunk = kSelCap - kMaxPicksPerPass;
-  int kept = 0;
-  unsigned long long evaluated = 0;
-  for (int c = 0; c < L; c += chunk) {
-    if (threadIdx.x == 0) s_cnt = kept;
-    __syncthreads();
-    stage_candidates(p, w, h, c, min(L, c + chunk), S, &s_cnt);
-    const int n = min(s_cnt, kSelCap);
-    evaluated += (unsigned long long)(n - kept);
-    sort_candidates(S, n);
-    kept = min(kk, n);
-  }
-  if (threadIdx.x == 0) w.rows_eval[h] += evaluated;
-  if (threadIdx.x == 0) {
-    uint8_t* sel = w.sel + (int64_t)h * p.T;
-    const double* cd = w.corrd + (int64_t)h * p.T;
-    bool bad = false;
-    for (int k = 0; k < kk; ++k) {
-      int j = k < kept ? S.idx[k] : INT_MAX;
-      double v = j != INT_MAX ? cd[j] : -INFINITY;
-      if (j == INT_MAX || !(v == v)) {   // no finite value: lowest free key
-        bad = true;
-        for (j = 0; j < p.T && sel[j]; ++j) {}
-        v = -INFINITY;
-      }
-      const int64_t o = w.cu_t[h] + s0 + k;
-      w.picks[o] = j;
-      w.pick_corr[o] = (float)v;
-      sel[j] = 1;
-    }
-    if (bad) record_status(w.status + h, AM_ERR_NONFINITE);
-  }
+  if (!s_last) return;
+  __threadfence();
+  if (which == 0) theta_and_prefix(p, w, h, p0, kk, S);
+  else pick_from_prefix(p, w, h, s0, kk, S);
+  if (threadIdx.x == 0) w.rcount[h] = 0;
 }
 
 int rows_ctas_per_head(int active) {
@@ -327,13 +343,10 @@ cudaError_t launch_column_norms(const Problem& p, const Work& w, cudaStream_t s)
 
 cudaError_t launch_corr_bounded(const Problem& p, const Work& w, int pass, int active, cudaStream_t s) {
   const int sel_smem = (int)sizeof(SelScratch);
-  cudaFuncSetAttribute(k_theta, cudaFuncAttributeMaxDynamicSharedMemorySize, sel_smem);
-  cudaFuncSetAttribute(k_pick, cudaFuncAttributeMaxDynamicSharedMemorySize, sel_smem);
+  cudaFuncSetAttribute(k_rows, cudaFuncAttributeMaxDynamicSharedMemorySize, sel_smem);
   dim3 gr(rows_ctas_per_head(active), active);
-  AM_LAUNCH(AM_STAGE_ROWS, s, k_rows<<<gr, 256, 0, s>>>(p, w, pass, 0));
-  AM_LAUNCH(AM_STAGE_CORR, s, k_theta<<<active, kBoundThreads, sel_smem, s>>>(p, w, pass));
-  AM_LAUNCH(AM_STAGE_ROWS, s, k_rows<<<gr, 256, 0, s>>>(p, w, pass, 1));
-  AM_LAUNCH(AM_STAGE_SELECT, s, k_pick<<<active, kBoundThreads, sel_smem, s>>>(p, w, pass));
+  AM_LAUNCH(AM_STAGE_ROWS, s, k_rows<<<gr, kSelThreads, sel_smem, s>>>(p, w, pass, 0));
+  AM_LAUNCH(AM_STAGE_ROWS, s, k_rows<<<gr, kSelThreads, sel_smem, s>>>(p, w, pass, 1));
   return cudaGetLastError();
 }
 

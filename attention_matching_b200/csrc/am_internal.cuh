@@ -77,6 +77,7 @@ struct Work {
   unsigned long long* rows_eval;   // [H] keys evaluated, summed over the passes
   double* gpart;        // [kGramSplits·(Σt + H)·kGramMaxNew] Gram partial sums per query quarter
   int32_t* gcount;      // [H] Gram blocks finished this pass
+  int32_t* rcount;      // [H] bounded-correlation row blocks finished this launch
   int64_t nrm_ata;      // Σt²
   int64_t nrm_stride;   // Σt² + Σt·d
 };

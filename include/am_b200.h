@@ -222,7 +222,7 @@ typedef enum am_stage {
   AM_STAGE_PHI = 1,      /* Φᵀ = exp(s − c_h)                        */
   AM_STAGE_TARGET = 2,   /* Y = ΦV/m and m                           */
   AM_STAGE_INIT = 3,     /* ‖m‖², selection flags                    */
-  AM_STAGE_CORR = 4,     /* c = Φᵀ r (bounded mode: the threshold)   */
+  AM_STAGE_CORR = 4,     /* c = Φᵀ r (full-pass modes)                */
   AM_STAGE_SELECT = 5,   /* top-k·R unselected keys                  */
   AM_STAGE_GRAM = 6,     /* Φ_SᵀΦ_S, Φ_Sᵀm updates                   */
   AM_STAGE_NNLS = 7,     /* active-set NNLS refit                    */
@@ -232,7 +232,8 @@ typedef enum am_stage {
   AM_STAGE_NORMAL = 11,  /* AᵀA, AᵀY                                 */
   AM_STAGE_SOLVE = 12,   /* ridge Cholesky, C_v                      */
   AM_STAGE_NORMS = 13,   /* bounded mode: ‖Φ_{:,j}‖, keys by norm    */
-  AM_STAGE_ROWS = 14,    /* bounded mode: exact c_j of listed keys   */
+  AM_STAGE_ROWS = 14,    /* bounded mode: exact c_j of listed keys,
+                            threshold and picks                      */
   AM_STAGE_COUNT = 15
 } am_stage_t;
 
