@@ -227,13 +227,14 @@ __global__ void __launch_bounds__(kCholThreads) k_chol(Problem p, Work w, int l_
   tr = block_sum(tr, scratch);
   const double lam = (double)p.ridge * tr / t;
   double* Lg = w.L + gbase;
-  double* L = t <= l_smem_max ? reinterpret_cast<double*>(smem) : Lg;
+  // tile scratch first, then (when it fits) the packed matrix
+  double* scratch_t = reinterpret_cast<double*>(smem);
+  double* L = t <= l_smem_max ? scratch_t + kTiledScratchDoubles : Lg;
   for (int a = threadIdx.x >> 5; a < t; a += blockDim.x >> 5)
     for (int c = threadIdx.x & 31; c <= a; c += 32) L[tri(a, c)] = M[(int64_t)a * t + c] + (a == c ? lam : 0.0);
   __syncthreads();
-  // large heads: tiled factorization in the workspace, shared memory as tile scratch
-  const int bad = L != Lg ? block_cholesky_packed(L, t, [](int) { return 0.0; }, &flag)
-                          : block_cholesky_tiled(Lg, t, [](int) { return 0.0; }, reinterpret_cast<double*>(smem), &flag);
+  // tiled factorization (32×32 tiles), of the shared-memory copy or in the workspace
+  const int bad = block_cholesky_tiled(L, t, [](int) { return 0.0; }, scratch_t, &flag);
   if (bad >= 0) {
     if (threadIdx.x == 0) record_status(w.status + h, AM_ERR_NOT_SPD);
     for (int a = threadIdx.x; a < t; a += blockDim.x) w.w_eff[base + a] = 0.0;   // marks the head for k_trsm
@@ -245,60 +246,119 @@ __global__ void __launch_bounds__(kCholThreads) k_chol(Problem p, Work w, int l_
   for (int a = threadIdx.x; a < t; a += blockDim.x) w.bvec[base + a] = 1.0 / L[tri(a, a)];
 }
 
-// C_v[:, c0:c0+CW] = L⁻ᵀ L⁻¹ AᵀY[:, c0:c0+CW]; 256 threads, 256/CW per column,
-// each row's dot product split across a column's threads.
+// C_v[:, c0:c0+CW] = L⁻ᵀ L⁻¹ AᵀY[:, c0:c0+CW] (CW = 32, or 8 when 32 columns of
+// a large head do not fit in shared memory) for one head per block, by 32-row
+// blocks.  Forward, block [r0, r0+32): first every row of the block takes its
+// products with the solved rows above (thread = one row × four columns,
+// factor rows read along their length), then one warp (lane = column) sweeps
+// the 32×32 diagonal block.  Backward mirrors it from the bottom: the
+// diagonal sweep, then every row above takes the block's contribution.
+// X is [t][CW + 1] in shared memory (odd row stride: a warp's lanes and the
+// four-column groups land on distinct banks).
 template <int CW>
 __global__ void __launch_bounds__(256) k_trsm(Problem p, Work w, float* C_v, int l_smem_max) {
   extern __shared__ __align__(16) unsigned char smem[];
-  constexpr int TPC = 256 / CW;                 // threads per column (power of two)
+  constexpr int kTrsmCols = CW, kXs = CW + 1;
+  constexpr int kGroups = CW / 4;                 // four-column groups per row
   const int h = blockIdx.x;
-  const int c0 = blockIdx.y * CW;
+  const int c0 = blockIdx.y * kTrsmCols;
   const int t = w.t[h];
   const int64_t base = w.cu_t[h];
   const int64_t gbase = w.cu_t2[h];
   if (c0 >= p.d) return;
   const double* invd = w.bvec + base;
   const bool l_smem = t <= l_smem_max;
-  double* X = reinterpret_cast<double*>(smem);              // [t][CW]
-  double* Ls = X + (size_t)t * CW;
+  double* X = reinterpret_cast<double*>(smem);              // [t][kXs]
+  double* Ls = X + (size_t)t * kXs;
   const double* L = l_smem ? Ls : w.L + gbase;
   if (w.w_eff[base] == 0.0 && w.status[h] != 0) {           // factorization failed
-    for (int e = threadIdx.x; e < t * CW; e += blockDim.x) {
-      const int r = e / CW, c = c0 + e % CW;
+    for (int e = threadIdx.x; e < t * kTrsmCols; e += blockDim.x) {
+      const int r = e / kTrsmCols, c = c0 + e % kTrsmCols;
       if (c < p.d) C_v[(base + r) * p.d + c] = 0.f;
     }
     return;
   }
   if (l_smem)
     for (int64_t e = threadIdx.x; e < tri(t, 0); e += blockDim.x) Ls[e] = w.L[gbase + e];
-  for (int e = threadIdx.x; e < t * CW; e += blockDim.x) {
-    const int r = e / CW, c = c0 + e % CW;
-    X[e] = c < p.d ? w.AtY[(base + r) * p.d + c] : 0.0;
+  for (int e = threadIdx.x; e < t * kTrsmCols; e += blockDim.x) {
+    const int r = e / kTrsmCols, cc = e % kTrsmCols, c = c0 + cc;
+    X[r * kXs + cc] = c < p.d ? w.AtY[(base + r) * p.d + c] : 0.0;
   }
   __syncthreads();
-  const int col = threadIdx.x / TPC, sub = threadIdx.x % TPC;
-  const unsigned gmask = (TPC == 32) ? 0xffffffffu : (((1u << TPC) - 1) << ((threadIdx.x & 31) / TPC * TPC));
-  // forward: y_k = (x_k − Σ_{j<k} L_kj y_j) / L_kk
-  for (int k = 0; k < t; ++k) {
-    const double* Lk = L + tri(k, 0);
-    double acc = 0.0;
-    for (int j = sub; j < k; j += TPC) acc += Lk[j] * X[j * CW + col];
-    for (int o = TPC / 2; o; o >>= 1) acc += __shfl_xor_sync(gmask, acc, o);
-    if (sub == 0) X[k * CW + col] = (X[k * CW + col] - acc) * invd[k];
-    __syncwarp(gmask);
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  // products: row r0 + rr, columns cg .. cg+3, kKs threads splitting the sum
+  constexpr int kKs = 32 / CW;
+  const int ks = tid % kKs, rr = tid / kKs / kGroups, cg = (tid / kKs % kGroups) * 4;
+  const int nb = (t + 31) / 32;
+  // forward: y = L⁻¹ x
+  for (int b = 0; b < nb; ++b) {
+    const int r0 = b * 32, bw = min(32, t - r0);
+    if (r0 > 0) {
+      const bool live = rr < bw;
+      const double* Lr = L + tri(r0 + (live ? rr : 0), 0);
+      double a0 = 0.0, a1 = 0.0, a2 = 0.0, a3 = 0.0;
+      if (live)
+        for (int j = ks; j < r0; j += kKs) {
+          const double l = Lr[j];
+          const double* xj = X + j * kXs + cg;
+          a0 = fma(l, xj[0], a0); a1 = fma(l, xj[1], a1); a2 = fma(l, xj[2], a2); a3 = fma(l, xj[3], a3);
+        }
+#pragma unroll
+      for (int o = 1; o < kKs; o <<= 1) {   // the kKs partial sums are adjacent lanes
+        a0 += __shfl_xor_sync(0xffffffffu, a0, o);
+        a1 += __shfl_xor_sync(0xffffffffu, a1, o);
+        a2 += __shfl_xor_sync(0xffffffffu, a2, o);
+        a3 += __shfl_xor_sync(0xffffffffu, a3, o);
+      }
+      if (live && ks == 0) {
+        double* xr = X + (r0 + rr) * kXs + cg;
+        xr[0] -= a0; xr[1] -= a1; xr[2] -= a2; xr[3] -= a3;
+      }
+    }
+    __syncthreads();
+    if (warp == 0) {
+      for (int r = r0; r < r0 + bw; ++r) {
+        const double* Lr = L + tri(r, 0);
+        if (lane < CW) {
+          double acc = X[r * kXs + lane];
+          for (int j = r0; j < r; ++j) acc = fma(-Lr[j], X[j * kXs + lane], acc);
+          X[r * kXs + lane] = acc * invd[r];
+        }
+        __syncwarp();
+      }
+    }
+    __syncthreads();
   }
-  // backward: z_k = (y_k − Σ_{j>k} L_jk z_j) / L_kk
-  for (int k = t - 1; k >= 0; --k) {
-    double acc = 0.0;
-    for (int j = k + 1 + sub; j < t; j += TPC) acc += L[tri(j, k)] * X[j * CW + col];
-    for (int o = TPC / 2; o; o >>= 1) acc += __shfl_xor_sync(gmask, acc, o);
-    if (sub == 0) X[k * CW + col] = (X[k * CW + col] - acc) * invd[k];
-    __syncwarp(gmask);
+  // backward: z = L⁻ᵀ y
+  for (int b = nb - 1; b >= 0; --b) {
+    const int r0 = b * 32, bw = min(32, t - r0);
+    if (warp == 0) {
+      for (int r = r0 + bw - 1; r >= r0; --r) {
+        if (lane < CW) {
+          double acc = X[r * kXs + lane];
+          for (int j = r + 1; j < r0 + bw; ++j) acc = fma(-L[tri(j, r)], X[j * kXs + lane], acc);
+          X[r * kXs + lane] = acc * invd[r];
+        }
+        __syncwarp();
+      }
+    }
+    __syncthreads();
+    // rows above the block: x_j −= Σ_{r in block} L[r][j] z_r (thread = row j × four columns)
+    for (int j = tid / kGroups; j < r0; j += 256 / kGroups) {
+      double a0 = 0.0, a1 = 0.0, a2 = 0.0, a3 = 0.0;
+      for (int r = r0; r < r0 + bw; ++r) {
+        const double l = L[tri(r, j)];
+        const double* zr = X + r * kXs + cg;
+        a0 = fma(l, zr[0], a0); a1 = fma(l, zr[1], a1); a2 = fma(l, zr[2], a2); a3 = fma(l, zr[3], a3);
+      }
+      double* xj = X + j * kXs + cg;
+      xj[0] -= a0; xj[1] -= a1; xj[2] -= a2; xj[3] -= a3;
+    }
+    __syncthreads();
   }
-  __syncthreads();
-  for (int e = threadIdx.x; e < t * CW; e += blockDim.x) {
-    const int r = e / CW, c = c0 + e % CW;
-    if (c < p.d) C_v[(base + r) * p.d + c] = (float)X[e];
+  for (int e = threadIdx.x; e < t * kTrsmCols; e += blockDim.x) {
+    const int r = e / kTrsmCols, cc = e % kTrsmCols, c = c0 + cc;
+    if (c < p.d) C_v[(base + r) * p.d + c] = (float)X[r * kXs + cc];
   }
 }
 
@@ -325,17 +385,18 @@ cudaError_t launch_value_fit(const Problem& p, const Work& w, float* C_v, cudaSt
   if (splits > 1)
     AM_LAUNCH(AM_STAGE_NORMAL, s,
               k_normal_reduce<<<296, 256, 0, s>>>(w.nrm_ata, w.nrm_stride - w.nrm_ata, splits, part_stride, w));
-  // factor: heads with t <= tl keep it in shared memory while factoring
+  // factor: heads with t <= tl keep it in shared memory (beside the tile scratch) while factoring
   const size_t cap = 226 * 1024;
+  const size_t scr = kTiledScratchDoubles * sizeof(double);
   int tl = 0;
-  while (tl < p.max_t && (size_t)(tl + 1) * (tl + 2) / 2 * sizeof(double) <= cap) ++tl;
-  const size_t sm = (size_t)tl * (tl + 1) / 2 * sizeof(double);
+  while (tl < p.max_t && scr + (size_t)(tl + 1) * (tl + 2) / 2 * sizeof(double) <= cap) ++tl;
+  const size_t sm = scr + (size_t)tl * (tl + 1) / 2 * sizeof(double);
   cudaFuncSetAttribute(k_chol, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)cap);
   AM_LAUNCH(AM_STAGE_SOLVE, s, k_chol<<<p.H, kCholThreads, sm, s>>>(p, w, tl));
   // solves: a column slice of AᵀY plus (when it fits) the factor in shared memory
-  const bool wide = (size_t)p.max_t * 32 * 8 <= 120 * 1024;
+  const bool wide = (size_t)p.max_t * 33 * 8 <= 120 * 1024;
   const int CW = wide ? 32 : 8;
-  const size_t xbytes = (size_t)p.max_t * CW * 8;
+  const size_t xbytes = (size_t)p.max_t * (CW + 1) * 8;
   int tl2 = 0;
   while (tl2 < p.max_t && xbytes + (size_t)(tl2 + 1) * (tl2 + 2) / 2 * sizeof(double) <= cap) ++tl2;
   const size_t sm2 = xbytes + (size_t)tl2 * (tl2 + 1) / 2 * sizeof(double);
