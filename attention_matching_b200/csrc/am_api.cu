@@ -31,7 +31,7 @@ struct Layout {
   size_t picks, pick_corr, plist, sorted_slot;
   size_t bvec, w, w_eff, ycache;
   size_t G, L, AtA, A, AtY, nrm_part;
-  size_t cnorm, rnorm, corrd, korder, knorm, ksort, cprefix, rows_eval, gpart, gcount, rcount;
+  size_t cnorm, rnorm, corrd, korder, knorm, ksort, cprefix, rows_eval, gpart, gcount, rcount, dinv;
   size_t total;
   size_t tables_bytes;
 };
@@ -97,6 +97,7 @@ Layout plan(int n, int T, int d, int H, int64_t sum_t, int64_t sum_t2, bool corr
   L.gpart = take((size_t)kGramSplits * ((size_t)sum_t + H) * kGramMaxNew * 8);
   L.gcount = take((size_t)H * 4);
   L.rcount = take((size_t)H * 4);
+  L.dinv = take(((size_t)sum_t + 32 * (size_t)H) * 32 * 8);
   L.total = o;
   return L;
 }
@@ -207,6 +208,7 @@ Work bind(const Layout& L, char* base, bool corr_bf16) {
   w.gpart = reinterpret_cast<double*>(base + L.gpart);
   w.gcount = reinterpret_cast<int32_t*>(base + L.gcount);
   w.rcount = reinterpret_cast<int32_t*>(base + L.rcount);
+  w.dinv = reinterpret_cast<double*>(base + L.dinv);
   return w;
 }
 

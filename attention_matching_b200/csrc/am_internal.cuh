@@ -78,6 +78,7 @@ struct Work {
   double* gpart;        // [kGramSplits·(Σt + H)·kGramMaxNew] Gram partial sums per query quarter
   int32_t* gcount;      // [H] Gram blocks finished this pass
   int32_t* rcount;      // [H] bounded-correlation row blocks finished this launch
+  double* dinv;         // per head at 32·(cu_t[h] + 32h): inverses of the value-fit factor's 32×32 diagonal tiles
   int64_t nrm_ata;      // Σt²
   int64_t nrm_stride;   // Σt² + Σt·d
 };

@@ -103,12 +103,16 @@ namespace am {
 //      four 64-thread groups each taking one tile, 4×4 outputs per thread.
 // Each tile row is 32 consecutive doubles of the packed storage, so every
 // global access is coalesced.  Needs 4·3·32·33 + 32·33 doubles of shared
-// scratch (≈ 110 KB); all threads of the block (256) must call.
+// scratch (≈ 110 KB); all threads of the block (256) must call.  When dinv
+// is given, the inverse of each factored diagonal tile is stored there as a
+// zero-padded row-major 32×32 block (tile kb at dinv + kb·1024): one warp,
+// lane c solving D x = e_c by forward substitution.
 constexpr int kTile = 32;
 constexpr size_t kTiledScratchDoubles = 4 * 3 * kTile * (kTile + 1) + kTile * (kTile + 1);
 
 template <class Floor>
-__device__ int block_cholesky_tiled(double* M, int n, Floor pivot_floor, double* scratch, int* s_flag) {
+__device__ int block_cholesky_tiled(double* M, int n, Floor pivot_floor, double* scratch, int* s_flag,
+                                    double* dinv = nullptr) {
   const int tid = threadIdx.x;
   double (*D)[kTile + 1] = reinterpret_cast<double (*)[kTile + 1]>(scratch);
   double* grp_base = scratch + kTile * (kTile + 1);
@@ -143,6 +147,20 @@ __device__ int block_cholesky_tiled(double* M, int n, Floor pivot_floor, double*
     for (int e = tid; e < kTile * kTile; e += blockDim.x) {
       const int r = e / kTile, c = e % kTile;
       if (r < kw && c <= r) M[tri(k0 + r, k0 + c)] = D[r][c];
+    }
+    if (dinv && tid < 32) {   // lane c: column c of D⁻¹
+      const int c = tid;
+      double x[kTile];
+#pragma unroll
+      for (int r = 0; r < kTile; ++r) {
+        double acc = r == c ? 1.0 : 0.0;
+#pragma unroll
+        for (int j = 0; j < r; ++j) acc -= D[r][j] * x[j];
+        x[r] = (r < kw && r >= c) ? acc / D[r][r] : 0.0;
+      }
+      double* out = dinv + (int64_t)kb * kTile * kTile;
+#pragma unroll
+      for (int r = 0; r < kTile; ++r) out[r * kTile + c] = x[r];
     }
     // 2. panel: rows below the diagonal tile, X_r = M_r L_Dᵀ⁻¹ (one thread per row)
     for (int r = k0 + kw + tid; r < n; r += blockDim.x) {

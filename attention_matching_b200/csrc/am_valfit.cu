@@ -234,7 +234,8 @@ __global__ void __launch_bounds__(kCholThreads) k_chol(Problem p, Work w, int l_
     for (int c = threadIdx.x & 31; c <= a; c += 32) L[tri(a, c)] = M[(int64_t)a * t + c] + (a == c ? lam : 0.0);
   __syncthreads();
   // tiled factorization (32×32 tiles), of the shared-memory copy or in the workspace
-  const int bad = block_cholesky_tiled(L, t, [](int) { return 0.0; }, scratch_t, &flag);
+  const int bad = block_cholesky_tiled(L, t, [](int) { return 0.0; }, scratch_t, &flag,
+                                       w.dinv + (int64_t)32 * (base + 32 * h));
   if (bad >= 0) {
     if (threadIdx.x == 0) record_status(w.status + h, AM_ERR_NOT_SPD);
     for (int a = threadIdx.x; a < t; a += blockDim.x) w.w_eff[base + a] = 0.0;   // marks the head for k_trsm
@@ -248,11 +249,12 @@ __global__ void __launch_bounds__(kCholThreads) k_chol(Problem p, Work w, int l_
 
 // C_v[:, c0:c0+CW] = L⁻ᵀ L⁻¹ AᵀY[:, c0:c0+CW] (CW = 32, or 8 when 32 columns of
 // a large head do not fit in shared memory) for one head per block, by 32-row
-// blocks.  Forward, block [r0, r0+32): first every row of the block takes its
+// blocks.  Forward, block [r0, r0+32): every row of the block takes its
 // products with the solved rows above (thread = one row × four columns,
-// factor rows read along their length), then one warp (lane = column) sweeps
-// the 32×32 diagonal block.  Backward mirrors it from the bottom: the
-// diagonal sweep, then every row above takes the block's contribution.
+// factor rows read along their length), then the block is multiplied by the
+// inverse of its diagonal tile (stored by the factorization).  Backward
+// mirrors it from the bottom with the transposed tile inverse, then every
+// row above takes the block's contribution.  No step is a sequential sweep.
 // X is [t][CW + 1] in shared memory (odd row stride: a warp's lanes and the
 // four-column groups land on distinct banks).
 template <int CW>
@@ -266,10 +268,11 @@ __global__ void __launch_bounds__(256) k_trsm(Problem p, Work w, float* C_v, int
   const int64_t base = w.cu_t[h];
   const int64_t gbase = w.cu_t2[h];
   if (c0 >= p.d) return;
-  const double* invd = w.bvec + base;
   const bool l_smem = t <= l_smem_max;
-  double* X = reinterpret_cast<double*>(smem);              // [t][kXs]
+  double (*Dt)[33] = reinterpret_cast<double (*)[33]>(smem);   // a diagonal tile inverse
+  double* X = reinterpret_cast<double*>(smem) + 32 * 33;        // [t][kXs]
   double* Ls = X + (size_t)t * kXs;
+  const double* Dinv = w.dinv + (int64_t)32 * (base + 32 * h);
   const double* L = l_smem ? Ls : w.L + gbase;
   if (w.w_eff[base] == 0.0 && w.status[h] != 0) {           // factorization failed
     for (int e = threadIdx.x; e < t * kTrsmCols; e += blockDim.x) {
@@ -290,6 +293,31 @@ __global__ void __launch_bounds__(256) k_trsm(Problem p, Work w, float* C_v, int
   constexpr int kKs = 32 / CW;
   const int ks = tid % kKs, rr = tid / kKs / kGroups, cg = (tid / kKs % kGroups) * 4;
   const int nb = (t + 31) / 32;
+  // Xb[0..bw) ← D⁻¹ Xb (or D⁻ᵀ Xb), D⁻¹ in Dt; all threads, two barriers
+  auto diag_product = [&](double (*Di)[33], double* Xb, int bw, bool transposed, int rr, int cg, int ks) {
+    double a0 = 0.0, a1 = 0.0, a2 = 0.0, a3 = 0.0;
+    if (rr < bw) {
+      const int j0 = transposed ? rr : 0, j1 = transposed ? bw : rr + 1;
+      for (int j = j0 + ks; j < j1; j += kKs) {
+        const double dij = transposed ? Di[j][rr] : Di[rr][j];
+        const double* xj = Xb + j * kXs + cg;
+        a0 = fma(dij, xj[0], a0); a1 = fma(dij, xj[1], a1); a2 = fma(dij, xj[2], a2); a3 = fma(dij, xj[3], a3);
+      }
+    }
+#pragma unroll
+    for (int o = 1; o < kKs; o <<= 1) {
+      a0 += __shfl_xor_sync(0xffffffffu, a0, o);
+      a1 += __shfl_xor_sync(0xffffffffu, a1, o);
+      a2 += __shfl_xor_sync(0xffffffffu, a2, o);
+      a3 += __shfl_xor_sync(0xffffffffu, a3, o);
+    }
+    __syncthreads();
+    if (rr < bw && ks == 0) {
+      double* xr = Xb + rr * kXs + cg;
+      xr[0] = a0; xr[1] = a1; xr[2] = a2; xr[3] = a3;
+    }
+    __syncthreads();
+  };
   // forward: y = L⁻¹ x
   for (int b = 0; b < nb; ++b) {
     const int r0 = b * 32, bw = min(32, t - r0);
@@ -315,34 +343,16 @@ __global__ void __launch_bounds__(256) k_trsm(Problem p, Work w, float* C_v, int
         xr[0] -= a0; xr[1] -= a1; xr[2] -= a2; xr[3] -= a3;
       }
     }
+    for (int e = tid; e < 32 * 32; e += blockDim.x) Dt[e >> 5][e & 31] = Dinv[(int64_t)b * 1024 + e];
     __syncthreads();
-    if (warp == 0) {
-      for (int r = r0; r < r0 + bw; ++r) {
-        const double* Lr = L + tri(r, 0);
-        if (lane < CW) {
-          double acc = X[r * kXs + lane];
-          for (int j = r0; j < r; ++j) acc = fma(-Lr[j], X[j * kXs + lane], acc);
-          X[r * kXs + lane] = acc * invd[r];
-        }
-        __syncwarp();
-      }
-    }
-    __syncthreads();
+    diag_product(Dt, X + r0 * kXs, bw, false, rr, cg, ks);
   }
   // backward: z = L⁻ᵀ y
   for (int b = nb - 1; b >= 0; --b) {
     const int r0 = b * 32, bw = min(32, t - r0);
-    if (warp == 0) {
-      for (int r = r0 + bw - 1; r >= r0; --r) {
-        if (lane < CW) {
-          double acc = X[r * kXs + lane];
-          for (int j = r + 1; j < r0 + bw; ++j) acc = fma(-L[tri(j, r)], X[j * kXs + lane], acc);
-          X[r * kXs + lane] = acc * invd[r];
-        }
-        __syncwarp();
-      }
-    }
+    for (int e = tid; e < 32 * 32; e += blockDim.x) Dt[e >> 5][e & 31] = Dinv[(int64_t)b * 1024 + e];
     __syncthreads();
+    diag_product(Dt, X + r0 * kXs, bw, true, rr, cg, ks);
     // rows above the block: x_j −= Σ_{r in block} L[r][j] z_r (thread = row j × four columns)
     for (int j = tid / kGroups; j < r0; j += 256 / kGroups) {
       double a0 = 0.0, a1 = 0.0, a2 = 0.0, a3 = 0.0;
@@ -396,7 +406,7 @@ cudaError_t launch_value_fit(const Problem& p, const Work& w, float* C_v, cudaSt
   // solves: a column slice of AᵀY plus (when it fits) the factor in shared memory
   const bool wide = (size_t)p.max_t * 33 * 8 <= 120 * 1024;
   const int CW = wide ? 32 : 8;
-  const size_t xbytes = (size_t)p.max_t * (CW + 1) * 8;
+  const size_t xbytes = (size_t)p.max_t * (CW + 1) * 8 + 32 * 33 * 8;   // X and one tile inverse
   int tl2 = 0;
   while (tl2 < p.max_t && xbytes + (size_t)(tl2 + 1) * (tl2 + 2) / 2 * sizeof(double) <= cap) ++tl2;
   const size_t sm2 = xbytes + (size_t)tl2 * (tl2 + 1) / 2 * sizeof(double);
