@@ -314,16 +314,28 @@ __global__ void __launch_bounds__(kGramTileRows * 32) k_gram_tile(Problem p, Wor
   const float* P0 = w.phiT + (int64_t)h * p.T * p.ldn;
   const float4* ra = reinterpret_cast<const float4*>(P0 + (int64_t)w.picks[base + (live ? a : s0)] * p.ldn);
   const double2* m2 = reinterpret_cast<const double2*>(w.m + (int64_t)h * p.ldn);
+  __shared__ const float4* newrow[kGramMaxNew];
+  if (threadIdx.x < nb)
+    newrow[threadIdx.x] = reinterpret_cast<const float4*>(P0 + (int64_t)w.picks[base + s0 + threadIdx.x] * p.ldn);
+  __syncthreads();
   double acc[kGramMaxNew];
 #pragma unroll
   for (int b = 0; b < kGramMaxNew; ++b) acc[b] = 0.0;
   double accm = 0.0;
   for (int c0 = k0; c0 < k1; c0 += kGramChunk4) {
     const int cw = min(kGramChunk4, k1 - c0);
-    for (int e = threadIdx.x; e < nb * cw; e += blockDim.x) {
-      const int b = e / cw, i = e - b * cw;
-      const float4 y = reinterpret_cast<const float4*>(P0 + (int64_t)w.picks[base + s0 + b] * p.ldn)[c0 + i];
-      stage[b * kGramChunk4 + i] = make_double4(y.x, y.y, y.z, y.w);
+    for (int e0 = threadIdx.x; e0 < nb * cw; e0 += 4 * blockDim.x) {   // four loads in flight
+      float4 y[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int e = e0 + u * blockDim.x, b = e / cw, i = e - b * cw;
+        y[u] = e < nb * cw ? newrow[b][c0 + i] : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int e = e0 + u * blockDim.x, b = e / cw, i = e - b * cw;
+        if (e < nb * cw) stage[b * kGramChunk4 + i] = make_double4(y[u].x, y[u].y, y[u].z, y[u].w);
+      }
     }
     __syncthreads();
     if (live) {
@@ -1003,10 +1015,10 @@ __global__ void __launch_bounds__(kNnlsThreads) k_nnls(Problem p, Work w, int pa
 
 // ------------------------------------------------------------ residual ----
 // r = m − Φ_S w over all current picks; fp64 sums, fp32 store; partial ‖r‖².
-// A block covers 128 float4 positions (512 queries) with four thread groups,
+// A block covers 32 float4 positions (128 queries) with four thread groups,
 // group g taking picks g, g + 4, ...; the groups' sums are combined in a
 // fixed order, so the result is deterministic.
-constexpr int kResidPos = 128;     // float4 positions per block
+constexpr int kResidPos = 32;      // float4 positions per block
 constexpr int kResidGroups = 4;    // pick groups per position
 constexpr int kResidThreads = kResidPos * kResidGroups;
 constexpr int kResidChunk = 512;   // picks staged in shared memory at a time
@@ -1044,16 +1056,16 @@ __global__ void __launch_bounds__(kResidThreads) k_resid(Problem p, Work w, int 
       }
       __syncthreads();
       if (live) {
-        for (int q0 = g; q0 < cn; q0 += 4 * kResidGroups) {   // four picks in flight
-          float4 x[4];
+        for (int q0 = g; q0 < cn; q0 += 8 * kResidGroups) {   // eight picks in flight
+          float4 x[8];
 #pragma unroll
-          for (int u = 0; u < 4; ++u) {
+          for (int u = 0; u < 8; ++u) {
             const int q = q0 + u * kResidGroups;
             x[u] = q < cn ? reinterpret_cast<const float4*>(P0 + (int64_t)sj[q] * p.ldn)[i4]
                           : make_float4(0.f, 0.f, 0.f, 0.f);
           }
 #pragma unroll
-          for (int u = 0; u < 4; ++u) {
+          for (int u = 0; u < 8; ++u) {
             const int q = q0 + u * kResidGroups;
             const double wl = q < cn ? sw[q] : 0.0;
             acc[0] -= x[u].x * wl; acc[1] -= x[u].y * wl; acc[2] -= x[u].z * wl; acc[3] -= x[u].w * wl;
