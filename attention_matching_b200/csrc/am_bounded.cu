@@ -124,13 +124,28 @@ __device__ void stage_candidates(const Problem& p, const Work& w, int h, int lo,
   const int32_t* ord = w.korder + (int64_t)h * p.T;
   const uint8_t* sel = w.sel + (int64_t)h * p.T;
   const double* cd = w.corrd + (int64_t)h * p.T;
-  for (int q = lo + threadIdx.x; q < hi; q += blockDim.x) {
-    const int j = ord[q];
-    if (sel[j]) continue;
-    const int pos = atomicAdd(&S.cnt, 1);
-    if (pos < kSelCap) {
-      S.key[pos] = order_key(cd[j]);
-      S.idx[pos] = j;
+  for (int q0 = lo + threadIdx.x; q0 < hi; q0 += 4 * blockDim.x) {   // four keys in flight
+    int j[4];
+    bool s[4];
+    double v[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int q = q0 + u * blockDim.x;
+      j[u] = q < hi ? ord[q] : -1;
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      s[u] = j[u] < 0 || sel[j[u] < 0 ? 0 : j[u]];
+      v[u] = cd[j[u] < 0 ? 0 : j[u]];
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      if (s[u]) continue;
+      const int pos = atomicAdd(&S.cnt, 1);
+      if (pos < kSelCap) {
+        S.key[pos] = order_key(v[u]);
+        S.idx[pos] = j[u];
+      }
     }
   }
   __syncthreads();
@@ -176,15 +191,41 @@ __device__ void select_rounds(SelScratch& S, int n, int kk) {
   }
 }
 
+// Σ r_i² over [0, n) by all threads, eight loads per thread in flight.
+__device__ __forceinline__ double sum_squares(const float* r, int n) {
+  double a = 0.0;
+  for (int i0 = threadIdx.x; i0 < n; i0 += 8 * blockDim.x) {
+    float v[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int i = i0 + u * blockDim.x;
+      v[u] = i < n ? r[i] : 0.f;
+    }
+#pragma unroll
+    for (int u = 0; u < 8; ++u) a = fma((double)v[u], (double)v[u], a);
+  }
+  return a;
+}
+
+// Number of entries of kn[0, n) not below thr, by all threads (per-thread part).
+__device__ __forceinline__ int count_not_below(const float* kn, int n, float thr) {
+  int c = 0;
+  for (int i0 = threadIdx.x; i0 < n; i0 += 8 * blockDim.x) {
+    float v[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int i = i0 + u * blockDim.x;
+      v[u] = i < n ? kn[i] : thr;
+    }
+#pragma unroll
+    for (int u = 0; u < 8; ++u) c += (i0 + u * (int)blockDim.x < n) && !(v[u] < thr);
+  }
+  return c;
+}
+
 // θ and the prefix L (the last block of a head, after the probe rows).
 __device__ void theta_and_prefix(const Problem& p, const Work& w, int h, int p0, int kk, SelScratch& S) {
-  const float* r = w.r + (int64_t)h * p.ldn;
-  double a = 0.0;
-  for (int i = threadIdx.x; i < p.ldn; i += blockDim.x) {
-    const double v = r[i];
-    a = fma(v, v, a);
-  }
-  const double rn = sqrt(block_sum(a, S.red));
+  const double rn = sqrt(block_sum(sum_squares(w.r + (int64_t)h * p.ldn, p.ldn), S.red));
   if (threadIdx.x == 0) S.cnt = 0;
   __syncthreads();
   stage_candidates(p, w, h, 0, p0, S);   // p0 <= kProbe + 2047 <= kSelCap unselected at most
@@ -195,10 +236,7 @@ __device__ void theta_and_prefix(const Problem& p, const Work& w, int h, int p0,
   // the bound cannot help (θ <= 0, a zero or non-finite residual)
   const bool useful = theta > 0.0 && rn > 0.0 && rn < INFINITY;
   const float thr = useful ? (float)(theta / (rn * (1.0 + kBoundMargin))) : 0.f;
-  const float* kn = w.knorm + (int64_t)h * p.T;
-  int count = 0;
-  if (useful)
-    for (int q = threadIdx.x; q < p.T; q += blockDim.x) count += !(kn[q] < thr);
+  const int count = useful ? count_not_below(w.knorm + (int64_t)h * p.T, p.T, thr) : 0;
   const double tot = block_sum((double)count, S.red);
   if (threadIdx.x == 0) {
     const int L = useful ? (int)tot : p.T;
