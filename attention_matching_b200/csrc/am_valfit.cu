@@ -150,25 +150,37 @@ __global__ void __launch_bounds__(256) k_normal(Problem p, Work w, int splits, i
   const int tx = threadIdx.x % 16, ty = threadIdx.x / 16;
   double acc[4][4] = {};
   const float* Yh = w.Y + (int64_t)h * p.n * p.d;
-  for (int i0 = i_begin; i0 < i_end; i0 += NK_) {
-    __syncthreads();
-    for (int e = threadIdx.x; e < NK_ * NT_; e += blockDim.x) {
+  // the next chunk's operands travel in registers while this one is multiplied
+  constexpr int kPer = NK_ * NT_ / 256;   // elements per operand per thread (blockDim 256)
+  float ra[kPer], rb[kPer];
+  auto fetch = [&](int i0) {
+#pragma unroll
+    for (int u = 0; u < kPer; ++u) {
+      const int e = threadIdx.x + u * 256;
       const int rr = e / NK_, ii = e % NK_;          // A rows are contiguous along queries
       const int a = a0 + rr, i = i0 + ii;
-      As[ii][rr] = (a < t && i < i_end) ? (double)w.A[(base + a) * p.ldn + i] : 0.0;
+      ra[u] = (a < t && i < i_end) ? w.A[(base + a) * p.ldn + i] : 0.f;
       if (gram) {
         const int bb = b0 + rr;
-        Bs[ii][rr] = (bb < t && i < i_end) ? (double)w.A[(base + bb) * p.ldn + i] : 0.0;
+        rb[u] = (bb < t && i < i_end) ? w.A[(base + bb) * p.ldn + i] : 0.f;
+      } else {
+        const int i2 = i0 + e / NT_, c = b0 + e % NT_;   // Y rows are contiguous along dims
+        rb[u] = (i2 < i_end && c < p.d) ? Yh[(int64_t)i2 * p.d + c] : 0.f;
       }
     }
-    if (!gram) {
-      for (int e = threadIdx.x; e < NK_ * NT_; e += blockDim.x) {
-        const int ii = e / NT_, cc = e % NT_;          // Y rows are contiguous along dims
-        const int i = i0 + ii, c = b0 + cc;
-        Bs[ii][cc] = (i < i_end && c < p.d) ? (double)Yh[(int64_t)i * p.d + c] : 0.0;
-      }
+  };
+  fetch(i_begin);
+  for (int i0 = i_begin; i0 < i_end; i0 += NK_) {
+    __syncthreads();
+#pragma unroll
+    for (int u = 0; u < kPer; ++u) {
+      const int e = threadIdx.x + u * 256;
+      As[e % NK_][e / NK_] = (double)ra[u];
+      if (gram) Bs[e % NK_][e / NK_] = (double)rb[u];
+      else Bs[e / NT_][e % NT_] = (double)rb[u];
     }
     __syncthreads();
+    if (i0 + NK_ < i_end) fetch(i0 + NK_);
 #pragma unroll 4
     for (int ii = 0; ii < NK_; ++ii) {
       double x[4], y[4];
