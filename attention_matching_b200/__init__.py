@@ -44,7 +44,7 @@ class AmWorkspaceView(ctypes.Structure):
     _fields_ = [("phiT", ctypes.c_size_t), ("mass", ctypes.c_size_t), ("target", ctypes.c_size_t),
                 ("shift", ctypes.c_size_t), ("ldn", ctypes.c_int32), ("reserved", ctypes.c_int32),
                 ("weights", ctypes.c_size_t), ("resid", ctypes.c_size_t),
-                ("rows_evaluated", ctypes.c_size_t)]
+                ("rows_evaluated", ctypes.c_size_t), ("column_norms", ctypes.c_size_t)]
 
 
 class AmOpts(ctypes.Structure):
@@ -163,6 +163,7 @@ def features(out: Dict, n: int, T: int, d: int, budgets: Sequence[int], topk: in
         "weights": view(v.weights, int(sum(budgets)), torch.float64),
         "resid": view(v.resid, H * v.ldn, torch.float32).view(H, v.ldn),
         "rows_evaluated": view(v.rows_evaluated, H, torch.int64),
+        "column_norms": view(v.column_norms, H * T, torch.float64).view(H, T),
         "ldn": v.ldn,
     }
 

@@ -31,7 +31,7 @@ struct Layout {
   size_t picks, pick_corr, plist, sorted_slot;
   size_t bvec, w, w_eff, ycache;
   size_t G, L, AtA, A, AtY, nrm_part;
-  size_t cnorm, rnorm, corrd, korder, knorm, ksort, cprefix, rows_eval, gpart, gcount, rcount, dinv;
+  size_t cnorm, cnpart, rnorm, corrd, korder, knorm, ksort, cprefix, rows_eval, gpart, gcount, rcount, dinv;
   size_t total;
   size_t tables_bytes;
 };
@@ -85,6 +85,7 @@ Layout plan(int n, int T, int d, int H, int64_t sum_t, int64_t sum_t2, bool corr
   L.AtY = take((size_t)sum_t * d * 8);
   L.nrm_part = take((size_t)kNormalMaxSplits * ((size_t)sum_t2 + (size_t)sum_t * d) * 8);
   L.cnorm = take((size_t)H * T * 8);
+  L.cnpart = take((size_t)H * 4 * ((n + 127) / 128) * T * 4);
   L.rnorm = take((size_t)H * 8);
   L.corrd = take((size_t)H * T * 8);
   L.korder = take((size_t)H * T * 4);
@@ -198,6 +199,7 @@ Work bind(const Layout& L, char* base, bool corr_bf16) {
   w.AtY = reinterpret_cast<double*>(base + L.AtY);
   w.nrm_part = reinterpret_cast<double*>(base + L.nrm_part);
   w.cnorm = reinterpret_cast<double*>(base + L.cnorm);
+  w.cnpart = reinterpret_cast<float*>(base + L.cnpart);
   w.rnorm = reinterpret_cast<double*>(base + L.rnorm);
   w.corrd = reinterpret_cast<double*>(base + L.corrd);
   w.korder = reinterpret_cast<int32_t*>(base + L.korder);
@@ -315,6 +317,7 @@ am_status_t am_workspace_view(int32_t n, int32_t T, int32_t d, int32_t num_heads
   view->weights = L.w;
   view->resid = L.r;
   view->rows_evaluated = L.rows_eval;
+  view->column_norms = L.cnorm;
   return AM_OK;
 }
 
@@ -370,6 +373,7 @@ am_status_t compact_heads_impl(const void* Q, const void* K, const void* V, int3
   AM_TRY(cudaMemsetAsync(w.status, 0, (size_t)H * 4, s));
 
   const bool tc = phi_tc_supported(p);
+  if (!tc || !p.corr_bounded) w.cnpart = nullptr;   // column norms from the features instead
   if (opts->shift) {
     AM_TRY(launch_shift_copy(opts->shift, w.shift, H, s));
   } else if (tc) {

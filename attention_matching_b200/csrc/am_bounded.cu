@@ -70,6 +70,20 @@ __global__ void __launch_bounds__(256) k_colnorm(Problem p, Work w) {
   if (lane == 0) w.cnorm[(int64_t)h * p.T + j] = sqrt(s);
 }
 
+// ‖Φ_{:,j}‖₂ from the feature pass's per-warp partial sums (fp32 sums of 32
+// fp32 squares, relative error below 4e-7): their fp64 total, raised by the
+// factor 1 + 1e-6 so the result stays an upper bound of the exact norm.
+__global__ void __launch_bounds__(256) k_normsum(Problem p, Work w) {
+  const int h = blockIdx.y;
+  const int j = blockIdx.x * blockDim.x + threadIdx.x;
+  if (j >= p.T) return;
+  const int parts = 4 * ((p.n + 127) / 128);
+  const float* src = w.cnpart + (int64_t)h * parts * p.T + j;
+  double s = 0.0;
+  for (int k = 0; k < parts; ++k) s += (double)src[(int64_t)k * p.T];
+  w.cnorm[(int64_t)h * p.T + j] = sqrt(s) * (1.0 + 1e-6);
+}
+
 // Keys of each head by descending fp32 norm (ties: lower key first): one
 // block per head; 64-bit sort keys (norm bits, inverted key index) in shared
 // memory, or in the workspace when T exceeds kSortSmemKeys.
@@ -371,8 +385,13 @@ int rows_ctas_per_head(int active) {
 }  // namespace
 
 cudaError_t launch_column_norms(const Problem& p, const Work& w, cudaStream_t s) {
-  dim3 g((p.T + 7) / 8, p.H);
-  AM_LAUNCH(AM_STAGE_NORMS, s, k_colnorm<<<g, 256, 0, s>>>(p, w));
+  if (w.cnpart) {   // partial sums left by the tensor-core feature pass
+    dim3 g((p.T + 255) / 256, p.H);
+    AM_LAUNCH(AM_STAGE_NORMS, s, k_normsum<<<g, 256, 0, s>>>(p, w));
+  } else {
+    dim3 g((p.T + 7) / 8, p.H);
+    AM_LAUNCH(AM_STAGE_NORMS, s, k_colnorm<<<g, 256, 0, s>>>(p, w));
+  }
   const int sort_smem = p.T > kSortSmemKeys ? 0 : (int)(sizeof(uint64_t) * kSortSmemKeys);
   cudaFuncSetAttribute(k_sortnorm, cudaFuncAttributeMaxDynamicSharedMemorySize, sort_smem);
   AM_LAUNCH(AM_STAGE_NORMS, s, k_sortnorm<<<p.H, kBoundThreads, sort_smem, s>>>(p, w));

@@ -67,7 +67,8 @@ struct Work {
   double* AtY;          // [Σt][d]
   double* nrm_part;     // [kNormalMaxSplits][Σt² + Σt·d] split partials of AᵀA, AᵀY
   // bounded correlation pass
-  double* cnorm;        // [H][T] ‖Φ_{:,j}‖₂ (fp64, from the stored fp32 features)
+  double* cnorm;        // [H][T] ‖Φ_{:,j}‖₂ (fp64, an upper bound within 1e-6 when from cnpart)
+  float* cnpart;        // [H][⌈n/128⌉][4][T] per-warp partial Σ_i Φ_ij² from the feature pass, or null
   double* rnorm;        // [H] ‖r‖₂ of the stored fp32 residual, this pass
   double* corrd;        // [H][T] exact correlations of this pass's evaluated keys
   int32_t* korder;      // [H][T] keys by descending column norm

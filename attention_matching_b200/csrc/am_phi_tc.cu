@@ -382,8 +382,11 @@ k_phi_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtens
         asm volatile("bar.sync 1, %0;" ::"n"(kEpiThreads) : "memory");
         if (s_stopm[b]) { ok = false; break; }
       } else {
-        // each epilogue thread waits for the tile itself; no named barrier in the loop
-        if (!mbar_wait(s_full + b, bu & 1, abort_flag, status)) { ok = false; break; }
+        // each epilogue thread waits for the tile itself; no named barrier in the
+        // loop, but a warp leaves together (the loads and shuffles below are
+        // warp-collective)
+        const bool got = mbar_wait(s_full + b, bu & 1, abort_flag, status);
+        if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
       }
       tc_fence_after();
       float v[HC];
@@ -425,6 +428,27 @@ k_phi_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtens
 #pragma unroll
       for (int cc = 0; cc < HC; ++cc) a4[cc & 3] += (double)v[cc];
       mrow += (a4[0] + a4[1]) + (a4[2] + a4[3]);
+      if (w.cnpart) {
+        // this warp's 32 rows of Σ_i Φ_ij² for its 16 keys: a butterfly leaves
+        // key (lane >> 1) on lanes lane, lane ^ 1; even lanes store it
+        float q2[HC];
+#pragma unroll
+        for (int cc = 0; cc < HC; ++cc) q2[cc] = v[cc] * v[cc];
+#pragma unroll
+        for (int s = HC / 2, o = 16; s >= 1; s >>= 1, o >>= 1) {
+          const bool upper = (lane & o) != 0;
+#pragma unroll
+          for (int k = 0; k < s; ++k) {
+            const float send = upper ? q2[k] : q2[k + s];
+            const float keep = upper ? q2[k + s] : q2[k];
+            q2[k] = keep + __shfl_xor_sync(0xffffffffu, send, o);
+          }
+        }
+        q2[0] += __shfl_xor_sync(0xffffffffu, q2[0], 1);
+        const int key = jb + ((lane >> 1) & (HC - 1));
+        if (!(lane & 1) && key < p.T)
+          w.cnpart[(((int64_t)h * nqb + blockIdx.x % nqb) * 4 + qd) * p.T + key] = q2[0];
+      }
       if (i < p.ldn) {
         float* col = phi_base + (int64_t)(j * BN + grp * HC) * p.ldn + i;
         if (kvalid >= HC) {

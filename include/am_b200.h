@@ -164,6 +164,8 @@ typedef struct am_workspace_view {
   size_t weights, resid;
   size_t rows_evaluated;   /* int64 [H]: keys whose correlation the bounded
                               passes evaluated, summed over the call's passes */
+  size_t column_norms;     /* fp64 [H][T]: the bounded pass's ‖Φ_{:,j}‖₂, an upper
+                              bound within a relative 2e-6 of the exact norm */
 } am_workspace_view_t;
 
 am_status_t am_workspace_view(int32_t n, int32_t T, int32_t d, int32_t num_heads,

@@ -146,6 +146,12 @@ def test_features_elementwise(dtype, d, n, T):
         Y = O.target_outputs(Phi, V, m)
         Yg = f["target"][h].double().cpu().numpy()
         assert np.abs(Yg - Y).max() <= 1e-4 * np.abs(Y).max()
+        # the bounded correlation pass's column norms: upper bounds of the
+        # stored features' norms (to fp64 rounding) within a relative 2e-6
+        exact = np.sqrt((P * P).sum(axis=0))
+        cn = f["column_norms"][h].cpu().numpy()
+        assert np.all(cn >= exact * (1 - 1e-12)), np.min(cn / np.maximum(exact, 1e-300))
+        assert np.all(cn <= exact * (1 + 2e-6) + 1e-300), np.max(cn / np.maximum(exact, 1e-300))
 
 
 @needs_cuda
