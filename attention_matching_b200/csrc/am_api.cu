@@ -31,7 +31,8 @@ struct Layout {
   size_t picks, pick_corr, plist, sorted_slot;
   size_t bvec, w, w_eff, ycache;
   size_t G, L, AtA, A, AtY, nrm_part;
-  size_t cnorm, cnpart, rnorm, corrd, korder, knorm, ksort, cprefix, rows_eval, gpart, gcount, rcount, dinv;
+  size_t cnorm, cnpart, rnorm, corrd, korder, knorm, ksort, cprefix, cdone, cprobe, rows_eval, gpart, gcount, rcount,
+      dinv;
   size_t total;
   size_t tables_bytes;
 };
@@ -94,6 +95,8 @@ Layout plan(int n, int T, int d, int H, int64_t sum_t, int64_t sum_t2, bool corr
   while (t2 < (size_t)T) t2 <<= 1;
   L.ksort = take(T > kSortSmemKeys ? (size_t)H * t2 * 8 : 0);
   L.cprefix = take((size_t)H * 4);
+  L.cdone = take((size_t)H * 4);
+  L.cprobe = take((size_t)H * 4);
   L.rows_eval = take((size_t)H * 8);
   L.gpart = take((size_t)kGramSplits * ((size_t)sum_t + H) * kGramMaxNew * 8);
   L.gcount = take((size_t)H * 4);
@@ -206,6 +209,8 @@ Work bind(const Layout& L, char* base, bool corr_bf16) {
   w.knorm = reinterpret_cast<float*>(base + L.knorm);
   w.ksort = reinterpret_cast<uint64_t*>(base + L.ksort);
   w.cprefix = reinterpret_cast<int32_t*>(base + L.cprefix);
+  w.cdone = reinterpret_cast<int32_t*>(base + L.cdone);
+  w.cprobe = reinterpret_cast<int32_t*>(base + L.cprobe);
   w.rows_eval = reinterpret_cast<unsigned long long*>(base + L.rows_eval);
   w.gpart = reinterpret_cast<double*>(base + L.gpart);
   w.gcount = reinterpret_cast<int32_t*>(base + L.gcount);
@@ -394,6 +399,7 @@ am_status_t compact_heads_impl(const void* Q, const void* K, const void* V, int3
   AM_TRY(cudaMemsetAsync(w.rows_eval, 0, (size_t)H * 8, s));
   AM_TRY(cudaMemsetAsync(w.gcount, 0, (size_t)H * 4, s));
   AM_TRY(cudaMemsetAsync(w.rcount, 0, (size_t)H * 4, s));
+  AM_TRY(cudaMemsetAsync(w.cprefix, 0, (size_t)H * 4, s));
   const CorrInputs cin{Q, K, opts->key_bias};
   if (G == 1) {
     for (int pass = 0; pass < (int)tb.active.size(); ++pass)

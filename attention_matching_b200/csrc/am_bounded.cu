@@ -8,14 +8,16 @@
 // norm (k_colnorm, k_sortnorm); in every pass the keys a bound cannot exclude
 // then form a prefix of that order.  One pass of kk = s1 − s0 picks per head
 // is two launches of k_rows:
-//   1. exact c_j for the unselected keys among the first P0 = kProbe + s0
-//      sorted positions (so at least kProbe keys): fp64 sums of the stored
-//      fp32 features times the stored fp32 residual; then the last block of
-//      the head takes θ = the kk-th largest of those values and the prefix
-//      length L: every key with ‖Φ_{:,j}‖ >= θ / (‖r‖(1 + 1e-9)) lies in
-//      [0, L) (a count over the sorted norms);
-//   2. exact c_j for the unselected keys in [P0, L); then the last block
-//      appends the kk largest values of [0, L) (ties to the lower key).
+//   1. exact c_j for the unselected keys among the first P0 sorted positions,
+//      P0 = max(kProbe + s0, the previous pass's L) (so at least kProbe keys;
+//      L moves little from pass to pass): fp64 sums of the stored fp32
+//      features times the stored fp32 residual; then the last block of the
+//      head takes θ = the kk-th largest of those values and the prefix length
+//      L: every key with ‖Φ_{:,j}‖ >= θ / (‖r‖(1 + 1e-9)) lies in [0, L) (a
+//      count over the sorted norms).  When L <= P0 the kk largest values found
+//      are already the picks, and it appends them;
+//   2. otherwise exact c_j for the unselected keys in [P0, L); then the last
+//      block appends the kk largest values of [0, L) (ties to the lower key).
 // A key beyond L has c_j < θ while kk keys in the prefix reach θ, so it is not
 // among the kk largest: the picks are those of a full pass over all keys.
 // The margin 1e-9 covers the rounding of the fp64 sums and norms (relative
@@ -237,13 +239,17 @@ __device__ __forceinline__ int count_not_below(const float* kn, int n, float thr
   return c;
 }
 
-// θ and the prefix L (the last block of a head, after the probe rows).
-__device__ void theta_and_prefix(const Problem& p, const Work& w, int h, int p0, int kk, SelScratch& S) {
+__device__ void append_picks(const Problem& p, const Work& w, int h, int s0, int kk, SelScratch& S);
+
+// θ and the prefix L (the last block of a head, after the probe rows); the
+// picks too when the probe already covers L.
+__device__ void theta_and_prefix(const Problem& p, const Work& w, int h, int s0, int p0, int kk, SelScratch& S) {
   const double rn = sqrt(block_sum(sum_squares(w.r + (int64_t)h * p.ldn, p.ldn), S.red));
   if (threadIdx.x == 0) S.cnt = 0;
   __syncthreads();
-  stage_candidates(p, w, h, 0, p0, S);   // p0 <= kProbe + 2047 <= kSelCap unselected at most
-  select_rounds(S, min(S.cnt, kSelCap), kk);
+  stage_candidates(p, w, h, 0, p0, S);   // p0 <= kSelCap
+  const int staged = min(S.cnt, kSelCap);
+  select_rounds(S, staged, kk);
   const int jt = S.outj[kk - 1];
   const double theta = jt != INT_MAX ? w.corrd[(int64_t)h * p.T + jt] : -INFINITY;
   // L = number of sorted norms not below θ / (‖r‖(1 + margin)); every key when
@@ -252,11 +258,38 @@ __device__ void theta_and_prefix(const Problem& p, const Work& w, int h, int p0,
   const float thr = useful ? (float)(theta / (rn * (1.0 + kBoundMargin))) : 0.f;
   const int count = useful ? count_not_below(w.knorm + (int64_t)h * p.T, p.T, thr) : 0;
   const double tot = block_sum((double)count, S.red);
+  const int L = useful ? (int)tot : p.T;
+  const bool done = L <= p0;
   if (threadIdx.x == 0) {
-    const int L = useful ? (int)tot : p.T;
-    w.cprefix[h] = L > p0 ? L : p0;
+    w.cprefix[h] = L;   // the next pass sizes its probe by it
+    w.cprobe[h] = p0;
+    w.cdone[h] = done;
     w.rnorm[h] = rn;
+    if (done) w.rows_eval[h] += (unsigned long long)staged;
   }
+  if (done) append_picks(p, w, h, s0, kk, S);
+}
+
+// Appends S.outj[0, kk) as this pass's picks (thread 0).
+__device__ void append_picks(const Problem& p, const Work& w, int h, int s0, int kk, SelScratch& S) {
+  if (threadIdx.x != 0) return;
+  uint8_t* sel = w.sel + (int64_t)h * p.T;
+  const double* cd = w.corrd + (int64_t)h * p.T;
+  bool bad = false;
+  for (int k = 0; k < kk; ++k) {
+    int j = S.outj[k];
+    double v = j != INT_MAX ? cd[j] : -INFINITY;
+    if (j == INT_MAX || !(v == v)) {   // no finite value: lowest free key
+      bad = true;
+      for (j = 0; j < p.T && sel[j]; ++j) {}
+      v = -INFINITY;
+    }
+    const int64_t o = w.cu_t[h] + s0 + k;
+    w.picks[o] = j;
+    w.pick_corr[o] = (float)v;
+    sel[j] = 1;
+  }
+  if (bad) record_status(w.status + h, AM_ERR_NONFINITE);
 }
 
 // The kk largest values among the unselected keys of [0, L), in chunks that
@@ -281,26 +314,8 @@ __device__ void pick_from_prefix(const Problem& p, const Work& w, int h, int s0,
     kept = 0;
     for (int k = 0; k < kk; ++k) kept += S.outj[k] != INT_MAX;
   }
-  if (threadIdx.x == 0) {
-    w.rows_eval[h] += evaluated;
-    uint8_t* sel = w.sel + (int64_t)h * p.T;
-    const double* cd = w.corrd + (int64_t)h * p.T;
-    bool bad = false;
-    for (int k = 0; k < kk; ++k) {
-      int j = S.outj[k];
-      double v = j != INT_MAX ? cd[j] : -INFINITY;
-      if (j == INT_MAX || !(v == v)) {   // no finite value: lowest free key
-        bad = true;
-        for (j = 0; j < p.T && sel[j]; ++j) {}
-        v = -INFINITY;
-      }
-      const int64_t o = w.cu_t[h] + s0 + k;
-      w.picks[o] = j;
-      w.pick_corr[o] = (float)v;
-      sel[j] = 1;
-    }
-    if (bad) record_status(w.status + h, AM_ERR_NONFINITE);
-  }
+  if (threadIdx.x == 0) w.rows_eval[h] += evaluated;
+  append_picks(p, w, h, s0, kk, S);
 }
 
 // ------------------------------------------------------------ exact rows --
@@ -323,7 +338,10 @@ __global__ void __launch_bounds__(kSelThreads) k_rows(Problem p, Work w, int pas
   pass_range(p, w.t[h], pass, s0, s1);
   if (s0 >= s1) return;
   const int kk = s1 - s0;
-  const int p0 = min(p.T, kProbe + s0);
+  if (which && w.cdone[h]) return;                     // the probe step made the picks
+  // the probe reaches the previous pass's prefix (kept in cprefix until the
+  // probe's last block replaces it), at most kSelCap positions
+  const int p0 = which ? w.cprobe[h] : min(min(p.T, kSelCap), max(kProbe + s0, w.cprefix[h]));
   const int lo = which ? p0 : 0;
   const int hi = which ? w.cprefix[h] : p0;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -372,7 +390,7 @@ __global__ void __launch_bounds__(kSelThreads) k_rows(Problem p, Work w, int pas
   __syncthreads();
   if (!s_last) return;
   __threadfence();
-  if (which == 0) theta_and_prefix(p, w, h, p0, kk, S);
+  if (which == 0) theta_and_prefix(p, w, h, s0, p0, kk, S);
   else pick_from_prefix(p, w, h, s0, kk, S);
   if (threadIdx.x == 0) w.rcount[h] = 0;
 }

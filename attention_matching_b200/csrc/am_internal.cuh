@@ -75,6 +75,8 @@ struct Work {
   float* knorm;         // [H][T] those norms (fp32, descending)
   uint64_t* ksort;      // [H][pow2 >= T] sort scratch when T exceeds the shared-memory sort
   int32_t* cprefix;     // [H] this pass evaluates the keys at sorted positions [0, cprefix)
+  int32_t* cdone;       // [H] 1 when the probe step already made this pass's picks
+  int32_t* cprobe;      // [H] the probe length P0 of this pass
   unsigned long long* rows_eval;   // [H] keys evaluated, summed over the passes
   double* gpart;        // [kGramSplits·(Σt + H)·kGramMaxNew] Gram partial sums per query quarter
   int32_t* gcount;      // [H] Gram blocks finished this pass
