@@ -41,7 +41,7 @@ LAYERS_QWEN3_4B = 36
 def parse_args():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=100)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="qwen3_4b_layer",
@@ -119,6 +119,14 @@ class ClockSampler:
         for line in self.proc.stdout:
             self.lines.append(line.strip())
 
+    def wait_first(self, limit_s=10.0):
+        """Block until nvidia-smi has printed its first sample (it takes a
+        moment to start), so that the samples cover the timed region."""
+        t0 = time.time()
+        while self.proc is not None and not self.lines and time.time() - t0 < limit_s:
+            time.sleep(0.01)
+        self.lines.clear()
+
     def stop(self):
         if self.proc is None:
             return None
@@ -182,10 +190,12 @@ def cpu_baseline(wl, heads=1):
 
 
 # -------------------------------------------------------------- roofline ----
-def stage_models(wl, n, T, d, H, ldn, corr_kind, rows_evaluated):
+def stage_models(wl, n, T, d, H, ldn, corr_kind, rows_evaluated, tc=True):
     """Algorithmic work of one call (one step) per library stage: bytes that
     must cross HBM for the memory-bound stages, dense flops for the GEMM and
-    the fp64 solver stages.  Summed over the stage's launches in the step."""
+    the fp64 solver stages.  Summed over the stage's launches in the step.
+    With the tensor-core feature pass the column norms are summed from its
+    per-(query block, quarter) fp32 partials instead of re-reading Φᵀ."""
     kR = wl.topk * wl.refit_every
     s1 = [min((p + 1) * kR, t) for t in wl.budgets for p in range((t + kR - 1) // kR)]
     row = ldn * 4                                   # one stored Φᵀ row (fp32)
@@ -204,7 +214,10 @@ def stage_models(wl, n, T, d, H, ldn, corr_kind, rows_evaluated):
     if corr_kind == "recompute":
         m["corr"] = {"bound": "tensor", "flops": 2.0 * len(s1) * n * T * d, "exps": float(len(s1)) * n * T}
     elif corr_kind == "bounded":
-        m["norms"] = {"bound": "hbm", "bytes": H * T * row}
+        parts = 4 * ((n + 127) // 128)
+        # partials in, fp64 norms out and back in for the sort, sorted order and norms out
+        norms_in = parts * 4 if tc else row
+        m["norms"] = {"bound": "hbm", "bytes": float(H * T * (norms_in + 8 + 8 + 4 + 8))}
         m["rows"] = {"bound": "hbm", "bytes": float(rows_evaluated) * row}
     else:
         m["corr"] = {"bound": "hbm", "bytes": len(s1) * (T * ldn * (2 if corr_kind == "bf16" else 4) + row + T * 4)}
@@ -347,6 +360,7 @@ def run_ours(args, rank, world, local_rank):
         dist.barrier()
     torch.cuda.synchronize()
     clocks.start()
+    clocks.wait_first()
     l0 = am.kernel_launches()
     evs = []
     for _ in range(args.steps):
@@ -411,7 +425,7 @@ def run_ours(args, rank, world, local_rank):
     rows_eval = int(am.features({"workspace": ws}, n, T, d, wl.budgets, wl.topk, wl.refit_every,
                                 am.BF16 if Q.dtype == torch.bfloat16 else am.FP32,
                                 corr_mode)["rows_evaluated"].sum().item())
-    rf = roofline(stages, args.steps, stage_models(wl, n, T, d, H, ldn, corr_kind, rows_eval),
+    rf = roofline(stages, args.steps, stage_models(wl, n, T, d, H, ldn, corr_kind, rows_eval, tc_ok),
                   peaks, clk, committed_traffic() if corr_kind == "fp32" else {})
     value = job_throughput(H, world, ms)
     per_step_stage = {k: round(v["ms"] / args.steps, 4) for k, v in stages.items() if v["launches"]}

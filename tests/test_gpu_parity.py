@@ -249,6 +249,16 @@ def test_nnls_deletions_twin_keys():
 
 
 @needs_cuda
+def test_wide_passes_topk8_refit4():
+    """k·R = 32 picks per pass: the untiled Gram update (more than 16 new
+    picks) and 32 selection rounds per pass, on ragged heads and a prior bias."""
+    heads = [W.structured_head(490 + h, n=700, T=900) for h in range(2)]
+    rng = np.random.default_rng(491)
+    kb = [np.float32(rng.normal(0.0, 0.5, 900)) for _ in heads]
+    check_all(heads, [70, 45], 8, 4, key_bias=kb, label="k8 R4")
+
+
+@needs_cuda
 def test_bounded_correlation_long_key_axis():
     """T = 20000 keys: the bounded correlation pass sorts the column norms in
     workspace memory instead of shared memory (more than 16384 keys)."""
