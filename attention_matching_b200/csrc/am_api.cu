@@ -98,8 +98,8 @@ Layout plan(int n, int T, int d, int H, int64_t sum_t, int64_t sum_t2, bool corr
   L.cdone = take((size_t)H * 4);
   L.cprobe = take((size_t)H * 4);
   L.rows_eval = take((size_t)H * 8);
-  L.gpart = take((size_t)kGramSplits * ((size_t)sum_t + H) * kGramMaxNew * 8);
-  L.gcount = take((size_t)H * 4);
+  L.gpart = take((size_t)kGramMaxSlices * ((size_t)sum_t + H) * kGramMaxNew * 8);
+  L.gcount = take(((size_t)sum_t + H) * 4);
   L.rcount = take((size_t)H * 4);
   L.dinv = take(((size_t)sum_t + 32 * (size_t)H) * 32 * 8);
   L.total = o;
@@ -397,7 +397,7 @@ am_status_t compact_heads_impl(const void* Q, const void* K, const void* V, int3
   AM_TRY(launch_omp_init(p, w, s));
   if (p.corr_bounded) AM_TRY(launch_column_norms(p, w, s));
   AM_TRY(cudaMemsetAsync(w.rows_eval, 0, (size_t)H * 8, s));
-  AM_TRY(cudaMemsetAsync(w.gcount, 0, (size_t)H * 4, s));
+  AM_TRY(cudaMemsetAsync(w.gcount, 0, ((size_t)tb.sum_t + H) * 4, s));
   AM_TRY(cudaMemsetAsync(w.rcount, 0, (size_t)H * 4, s));
   AM_TRY(cudaMemsetAsync(w.cprefix, 0, (size_t)H * 4, s));
   const CorrInputs cin{Q, K, opts->key_bias};

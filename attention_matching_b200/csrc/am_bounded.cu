@@ -5,26 +5,28 @@
 //
 // For every key |c_j| = |rᵀΦ_{:,j}| <= ‖r‖₂·‖Φ_{:,j}‖₂ (Cauchy-Schwarz).  The
 // column norms do not depend on r, so once per call the keys are sorted by
-// norm (k_colnorm, k_sortnorm); in every pass the keys a bound cannot exclude
-// then form a prefix of that order.  One pass of kk = s1 − s0 picks per head
-// is two launches of k_rows:
+// norm (k_normsum or k_colnorm, then k_sortnorm); in every pass the keys a
+// bound cannot exclude then form a prefix of that order.  One pass of
+// kk = s1 − s0 picks per head is two launches of k_rows:
 //   1. exact c_j for the unselected keys among the first P0 sorted positions,
-//      P0 = max(kProbe + s0, the previous pass's L) (so at least kProbe keys;
-//      L moves little from pass to pass): fp64 sums of the stored fp32
-//      features times the stored fp32 residual; then the last block of the
-//      head takes θ = the kk-th largest of those values and the prefix length
-//      L: every key with ‖Φ_{:,j}‖ >= θ / (‖r‖(1 + 1e-9)) lies in [0, L) (a
-//      count over the sorted norms).  When L <= P0 the kk largest values found
-//      are already the picks, and it appends them;
+//      P0 = max(kProbe + s0, 5/4 of the previous pass's L plus 32) (L grows
+//      slowly from pass to pass, so the probe usually covers it): fp64 sums
+//      of the stored fp32 features times the stored fp32 residual; then the
+//      last block of the head takes θ = the kk-th largest of those values and
+//      the prefix length L: every key with ‖Φ_{:,j}‖ >= θ / (‖r‖(1 + 1e-7))
+//      lies in [0, L) (a sampled search over the sorted norms).  When L <= P0
+//      the kk largest values found are already the picks, and it appends them;
 //   2. otherwise exact c_j for the unselected keys in [P0, L); then the last
 //      block appends the kk largest values of [0, L) (ties to the lower key).
 // A key beyond L has c_j < θ while kk keys in the prefix reach θ, so it is not
 // among the kk largest: the picks are those of a full pass over all keys.
-// The margin 1e-9 covers the rounding of the fp64 sums and norms (relative
-// error below n·2^-53 for the sums, a few ulp for the norms); the fp32 copies
-// of the norms only move the cut outward (rounding to nearest is monotone).
-// The selections take kk rounds of a block-wide argmax over candidates staged
-// in shared memory.
+// The margin 1e-7 covers ‖r‖ being taken from the fp64 residual (the stored
+// fp32 one is larger by at most 2^-24 relative) and the rounding of the fp64
+// sums and norms (relative error below n·2^-53 for the sums, a few ulp for
+// the norms); the fp32 copies of the norms and of the cut only move it
+// outward (rounding to nearest is monotone).  A selection is a warp-level
+// top-kk (kk rounds of shuffle argmax per warp over shared-memory
+// candidates) followed by the same over the warps' winners.
 #include "am_internal.cuh"
 #include "am_profile.cuh"
 #include "am_linalg.cuh"
@@ -37,7 +39,7 @@ namespace {
 constexpr int kProbe = 256;        // unselected keys whose exact values set the threshold
 constexpr int kBoundThreads = 1024;
 constexpr int kSelCap = 2304;      // candidates one selection holds (>= kProbe + 2048)
-constexpr double kBoundMargin = 1e-9;
+constexpr double kBoundMargin = 1e-7;
 
 // Order-preserving map of a double to uint64 (NaN ranks lowest).
 __device__ __forceinline__ uint64_t order_key(double v) {
@@ -126,8 +128,8 @@ constexpr int kSelThreads = 256;
 struct SelScratch {
   uint64_t key[kSelCap];
   int idx[kSelCap];
-  uint64_t wk[kSelThreads / 32];
-  int wj[kSelThreads / 32], wp[kSelThreads / 32];
+  uint64_t ck[kSelThreads / 32][kMaxPicksPerPass];   // each warp's best, in pick order
+  int cj[kSelThreads / 32][kMaxPicksPerPass];
   uint64_t outk[kMaxPicksPerPass];
   int outj[kMaxPicksPerPass];
   double red[33];
@@ -175,90 +177,112 @@ __device__ __forceinline__ void shfl_best(uint64_t& k, int& j, int& pos, int o) 
   if (p2 >= 0 && (pos < 0 || before(k2, j2, k, j))) { k = k2; j = j2; pos = p2; }
 }
 
-// The kk candidates first in pick order, by kk rounds of a block-wide argmax
-// over slots [0, n): into S.outk / S.outj (index INT_MAX when none is left);
-// each winner's slot is cleared.  All threads.
-__device__ void select_rounds(SelScratch& S, int n, int kk) {
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nw = blockDim.x >> 5;
+// The best live entry (index not INT_MAX) of keys/idx at e = first, first +
+// stride, ... below n: (key, index, position), position -1 when none.
+__device__ __forceinline__ void lane_best(const uint64_t* keys, const int* idx, int first, int stride, int n,
+                                          uint64_t& bk, int& bj, int& bp) {
+  bk = 0ull; bj = INT_MAX; bp = -1;
+  for (int e = first; e < n; e += stride) {
+    const int jv = idx[e];
+    if (jv == INT_MAX) continue;
+    const uint64_t kv = keys[e];
+    if (bp < 0 || before(kv, jv, bk, bj)) { bk = kv; bj = jv; bp = e; }
+  }
+}
+
+// kk rounds of a warp argmax over one warp's entries (lane l owns positions
+// first + l·… as laid out by lane_best): round k's winner goes to outk[k] /
+// outj[k] (index INT_MAX once nothing is left) and its entry is marked used;
+// only the winning lane rescans.  One warp.
+__device__ __forceinline__ void warp_top(uint64_t* keys, int* idx, int first, int stride, int n, int kk,
+                                         uint64_t* outk, int* outj) {
+  const int lane = threadIdx.x & 31;
+  uint64_t bk;
+  int bj, bp;
+  lane_best(keys, idx, first, stride, n, bk, bj, bp);
   for (int k = 0; k < kk; ++k) {
-    uint64_t bk = 0ull;
-    int bj = INT_MAX, bp = -1;
-    for (int e = tid; e < n; e += blockDim.x) {
-      const int jv = S.idx[e];
-      if (jv == INT_MAX) continue;
-      const uint64_t kv = S.key[e];
-      if (bp < 0 || before(kv, jv, bk, bj)) { bk = kv; bj = jv; bp = e; }
+    uint64_t wk = bk;
+    int wj = bj, wp = bp;
+    for (int o = 16; o; o >>= 1) shfl_best(wk, wj, wp, o);
+    if (lane == 0) { outk[k] = wk; outj[k] = wp >= 0 ? wj : INT_MAX; }
+    if (wp >= 0 && wp == bp) {   // the owner of the winning entry takes its next best
+      idx[bp] = INT_MAX;
+      lane_best(keys, idx, first, stride, n, bk, bj, bp);
     }
-    for (int o = 16; o; o >>= 1) shfl_best(bk, bj, bp, o);
-    if (lane == 0) { S.wk[warp] = bk; S.wj[warp] = bj; S.wp[warp] = bp; }
-    __syncthreads();
-    if (warp == 0) {
-      bk = lane < nw ? S.wk[lane] : 0ull;
-      bj = lane < nw ? S.wj[lane] : INT_MAX;
-      bp = lane < nw ? S.wp[lane] : -1;
-      for (int o = 16; o; o >>= 1) shfl_best(bk, bj, bp, o);
-      if (lane == 0) {
-        S.outk[k] = bk;
-        S.outj[k] = bp >= 0 ? bj : INT_MAX;
-        if (bp >= 0) { S.key[bp] = 0ull; S.idx[bp] = INT_MAX; }
-      }
-    }
-    __syncthreads();
   }
+  __syncwarp();
 }
 
-// Σ r_i² over [0, n) by all threads, eight loads per thread in flight.
-__device__ __forceinline__ double sum_squares(const float* r, int n) {
-  double a = 0.0;
-  for (int i0 = threadIdx.x; i0 < n; i0 += 8 * blockDim.x) {
-    float v[8];
-#pragma unroll
-    for (int u = 0; u < 8; ++u) {
-      const int i = i0 + u * blockDim.x;
-      v[u] = i < n ? r[i] : 0.f;
-    }
-#pragma unroll
-    for (int u = 0; u < 8; ++u) a = fma((double)v[u], (double)v[u], a);
+// The kk candidates first in pick order among slots [0, n) (ties to the
+// lower key) into S.outk / S.outj, index INT_MAX when fewer are left: each
+// warp takes the kk best of its slots, then warp 0 the kk best of those.
+// The slots are consumed.  All threads.
+__device__ void select_top(SelScratch& S, int n, int kk) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
+  warp_top(S.key, S.idx, warp * 32 + lane, blockDim.x, n, kk, S.ck[warp], S.cj[warp]);
+  __syncthreads();
+  if (warp == 0) {
+    // candidates (w, k) at flat position w·kMaxPicksPerPass + k, k < kk
+    uint64_t* ck = &S.ck[0][0];
+    int* cj = &S.cj[0][0];
+    for (int e = lane; e < nw * kMaxPicksPerPass; e += 32)
+      if (e % kMaxPicksPerPass >= kk) cj[e] = INT_MAX;
+    __syncwarp();
+    warp_top(ck, cj, lane, 32, nw * kMaxPicksPerPass, kk, S.outk, S.outj);
   }
-  return a;
+  __syncthreads();
 }
 
-// Number of entries of kn[0, n) not below thr, by all threads (per-thread part).
-__device__ __forceinline__ int count_not_below(const float* kn, int n, float thr) {
-  int c = 0;
-  for (int i0 = threadIdx.x; i0 < n; i0 += 8 * blockDim.x) {
-    float v[8];
-#pragma unroll
-    for (int u = 0; u < 8; ++u) {
-      const int i = i0 + u * blockDim.x;
-      v[u] = i < n ? kn[i] : thr;
-    }
-#pragma unroll
-    for (int u = 0; u < 8; ++u) c += (i0 + u * (int)blockDim.x < n) && !(v[u] < thr);
+// The value behind an order key (NaN for key 0).
+__device__ __forceinline__ double key_value(uint64_t k) {
+  if (k == 0ull) return __longlong_as_double(0x7ff8000000000000ll);
+  return __longlong_as_double((long long)((k & 0x8000000000000000ull) ? (k & 0x7fffffffffffffffull) : ~k));
+}
+
+// Number of leading entries of kn[0, n) not below thr, the entries being in
+// descending order: a sampled search, one sample per thread and level (two
+// levels for n up to blockDim², one round trip each).  All threads.
+__device__ int prefix_not_below(const float* kn, int n, float thr) {
+  int lo = 0, hi = n;   // kn[i] >= thr known for i < lo, kn[i] < thr for i >= hi
+  while (lo < hi) {
+    const int span = hi - lo;
+    const int step = (span + (int)blockDim.x - 1) / (int)blockDim.x;
+    const int samples = (span + step - 1) / step;
+    const int i = lo + (int)threadIdx.x * step;
+    const bool ok = (int)threadIdx.x < samples && !(kn[i] < thr);
+    const int c = __syncthreads_count(ok);   // samples 0 .. c-1 pass
+    const int nlo = c > 0 ? lo + (c - 1) * step + 1 : lo;
+    hi = c < samples ? lo + c * step : hi;
+    lo = nlo;
   }
-  return c;
+  return lo;
 }
 
 __device__ void append_picks(const Problem& p, const Work& w, int h, int s0, int kk, SelScratch& S);
 
 // θ and the prefix L (the last block of a head, after the probe rows); the
-// picks too when the probe already covers L.
-__device__ void theta_and_prefix(const Problem& p, const Work& w, int h, int s0, int p0, int kk, SelScratch& S) {
-  const double rn = sqrt(block_sum(sum_squares(w.r + (int64_t)h * p.ldn, p.ldn), S.red));
+// picks too when the probe already covers L.  ‖r‖² is Σm² before the first
+// refit (r = m) and the residual update's per-block partials after it, added
+// in a fixed order; both are sums of the fp64 residual, whose stored fp32
+// copy (the one correlated) is larger by at most a factor 1 + 2^-24.
+__device__ void theta_and_prefix(const Problem& p, const Work& w, int h, int pass, int s0, int p0, int kk,
+                                 SelScratch& S) {
+  const int nrb = resid_blocks(p);
+  const double rr_mine = pass == 0 ? (threadIdx.x == 0 ? w.mm[h] : 0.0)
+                                   : ((int)threadIdx.x < nrb ? w.rr_part[(int64_t)h * kRedBlocks + threadIdx.x] : 0.0);
   if (threadIdx.x == 0) S.cnt = 0;
   __syncthreads();
   stage_candidates(p, w, h, 0, p0, S);   // p0 <= kSelCap
   const int staged = min(S.cnt, kSelCap);
-  select_rounds(S, staged, kk);
+  select_top(S, staged, kk);
+  const double rn = sqrt(block_sum(rr_mine, S.red));
   const int jt = S.outj[kk - 1];
-  const double theta = jt != INT_MAX ? w.corrd[(int64_t)h * p.T + jt] : -INFINITY;
+  const double theta = jt != INT_MAX ? key_value(S.outk[kk - 1]) : -INFINITY;
   // L = number of sorted norms not below θ / (‖r‖(1 + margin)); every key when
   // the bound cannot help (θ <= 0, a zero or non-finite residual)
   const bool useful = theta > 0.0 && rn > 0.0 && rn < INFINITY;
   const float thr = useful ? (float)(theta / (rn * (1.0 + kBoundMargin))) : 0.f;
-  const int count = useful ? count_not_below(w.knorm + (int64_t)h * p.T, p.T, thr) : 0;
-  const double tot = block_sum((double)count, S.red);
-  const int L = useful ? (int)tot : p.T;
+  const int L = useful ? prefix_not_below(w.knorm + (int64_t)h * p.T, p.T, thr) : p.T;
   const bool done = L <= p0;
   if (threadIdx.x == 0) {
     w.cprefix[h] = L;   // the next pass sizes its probe by it
@@ -270,26 +294,37 @@ __device__ void theta_and_prefix(const Problem& p, const Work& w, int h, int s0,
   if (done) append_picks(p, w, h, s0, kk, S);
 }
 
-// Appends S.outj[0, kk) as this pass's picks (thread 0).
+// Appends S.outj[0, kk) as this pass's picks, one thread each; a slot with no
+// finite value takes the lowest free key instead (thread 0, after the
+// others are marked) and flags the head.  All threads.
 __device__ void append_picks(const Problem& p, const Work& w, int h, int s0, int kk, SelScratch& S) {
-  if (threadIdx.x != 0) return;
   uint8_t* sel = w.sel + (int64_t)h * p.T;
-  const double* cd = w.corrd + (int64_t)h * p.T;
+  const int64_t o = w.cu_t[h] + s0;
+  const int k = threadIdx.x;
   bool bad = false;
-  for (int k = 0; k < kk; ++k) {
-    int j = S.outj[k];
-    double v = j != INT_MAX ? cd[j] : -INFINITY;
-    if (j == INT_MAX || !(v == v)) {   // no finite value: lowest free key
-      bad = true;
-      for (j = 0; j < p.T && sel[j]; ++j) {}
-      v = -INFINITY;
+  if (k < kk) {
+    const int j = S.outj[k];
+    const double v = j != INT_MAX ? key_value(S.outk[k]) : 0.0;
+    bad = j == INT_MAX || !(v == v);
+    if (!bad) {
+      w.picks[o + k] = j;
+      w.pick_corr[o + k] = (float)v;
+      sel[j] = 1;
     }
-    const int64_t o = w.cu_t[h] + s0 + k;
-    w.picks[o] = j;
-    w.pick_corr[o] = (float)v;
-    sel[j] = 1;
   }
-  if (bad) record_status(w.status + h, AM_ERR_NONFINITE);
+  if (__syncthreads_or(bad) && threadIdx.x == 0) {
+    for (int q = 0; q < kk; ++q) {
+      const double v = S.outj[q] != INT_MAX ? key_value(S.outk[q]) : 0.0;
+      if (S.outj[q] != INT_MAX && v == v) continue;
+      int j = 0;
+      while (j < p.T && sel[j]) ++j;
+      if (j >= p.T) break;   // cannot happen: t <= T leaves a free key per pick
+      w.picks[o + q] = j;
+      w.pick_corr[o + q] = -INFINITY;
+      sel[j] = 1;
+    }
+    record_status(w.status + h, AM_ERR_NONFINITE);
+  }
 }
 
 // The kk largest values among the unselected keys of [0, L), in chunks that
@@ -310,7 +345,7 @@ __device__ void pick_from_prefix(const Problem& p, const Work& w, int h, int s0,
     stage_candidates(p, w, h, c, min(L, c + chunk), S);
     const int n = min(S.cnt, kSelCap);
     evaluated += (unsigned long long)(n - kept);
-    select_rounds(S, n, kk);
+    select_top(S, n, kk);
     kept = 0;
     for (int k = 0; k < kk; ++k) kept += S.outj[k] != INT_MAX;
   }
@@ -339,9 +374,10 @@ __global__ void __launch_bounds__(kSelThreads) k_rows(Problem p, Work w, int pas
   if (s0 >= s1) return;
   const int kk = s1 - s0;
   if (which && w.cdone[h]) return;                     // the probe step made the picks
-  // the probe reaches the previous pass's prefix (kept in cprefix until the
-  // probe's last block replaces it), at most kSelCap positions
-  const int p0 = which ? w.cprobe[h] : min(min(p.T, kSelCap), max(kProbe + s0, w.cprefix[h]));
+  // the probe reaches 5/4 of the previous pass's prefix plus 32 (kept in
+  // cprefix until the probe's last block replaces it), at most kSelCap positions
+  const int lprev = w.cprefix[h];
+  const int p0 = which ? w.cprobe[h] : min(min(p.T, kSelCap), max(kProbe + s0, lprev + lprev / 4 + 32));
   const int lo = which ? p0 : 0;
   const int hi = which ? w.cprefix[h] : p0;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -390,7 +426,7 @@ __global__ void __launch_bounds__(kSelThreads) k_rows(Problem p, Work w, int pas
   __syncthreads();
   if (!s_last) return;
   __threadfence();
-  if (which == 0) theta_and_prefix(p, w, h, s0, p0, kk, S);
+  if (which == 0) theta_and_prefix(p, w, h, pass, s0, p0, kk, S);
   else pick_from_prefix(p, w, h, s0, kk, S);
   if (threadIdx.x == 0) w.rcount[h] = 0;
 }

@@ -78,8 +78,8 @@ struct Work {
   int32_t* cdone;       // [H] 1 when the probe step already made this pass's picks
   int32_t* cprobe;      // [H] the probe length P0 of this pass
   unsigned long long* rows_eval;   // [H] keys evaluated, summed over the passes
-  double* gpart;        // [kGramSplits·(Σt + H)·kGramMaxNew] Gram partial sums per query quarter
-  int32_t* gcount;      // [H] Gram blocks finished this pass
+  double* gpart;        // [kGramMaxSlices·(Σt + H)·kR] Gram partial sums per query slice
+  int32_t* gcount;      // [Σt + H] Gram blocks finished this pass, per head and row group
   int32_t* rcount;      // [H] bounded-correlation row blocks finished this launch
   double* dinv;         // per head at 32·(cu_t[h] + 32h): inverses of the value-fit factor's 32×32 diagonal tiles
   int64_t nrm_ata;      // Σt²
@@ -87,8 +87,15 @@ struct Work {
 };
 
 constexpr int kRedBlocks = 64;   // partial-sum slots per head for ‖r‖²
+constexpr int kResidPos = 32;    // float4 query positions per residual block
+
+// Blocks per head of the residual update, each leaving one partial ‖r‖².
+inline __host__ __device__ int resid_blocks(const Problem& p) {
+  const int b = (p.ldn / 4 + kResidPos - 1) / kResidPos;
+  return b < kRedBlocks ? b : kRedBlocks;
+}
 constexpr int kSortSmemKeys = 16384;  // key counts the norm sort handles in shared memory
-constexpr int kGramSplits = 4;        // query quarters of the tiled Gram update
+constexpr int kGramMaxSlices = 32;    // query slices of the tiled Gram update
 constexpr int kGramMaxNew = 16;       // picks per pass the tiled Gram update takes
 constexpr int kNormalMaxSplits = 8;   // query splits of the normal-equation products
 

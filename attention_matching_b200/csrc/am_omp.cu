@@ -281,121 +281,187 @@ __global__ void __launch_bounds__(256) k_gram(Problem p, Work w, int pass) {
   }
 }
 
-// Tiled form for passes of at most kGramMaxNew picks.  Block (tile, head,
-// split) takes four pick rows a (one warp each) against all new picks b of
-// the pass over a quarter of the queries; the new rows' columns are staged in
-// shared memory as fp64, once per block.  Products are exact (fp32 × fp32 in
-// fp64).  Each block writes its partial sums to the workspace; the last block
-// of a head to finish (counted with an atomic) adds the four quarters in a
-// fixed order and writes G (both triangles) and b, so the result does not
-// depend on block timing, and G[a][b], G[b][a] come out bitwise equal.
-constexpr int kGramTileRows = 4;
-constexpr int kGramChunk4 = 128;   // float4 columns per staged chunk
+// Sums 32 per-lane values across the warp: afterwards lane l holds the
+// total of value l (31 shuffles: each step halves the values a lane keeps).
+__device__ __forceinline__ double warp_reduce32(double (&v)[32]) {
+  const int lane = threadIdx.x & 31;
+#pragma unroll
+  for (int s = 16; s >= 1; s >>= 1) {
+    const bool upper = (lane & s) != 0;
+#pragma unroll
+    for (int i = 0; i < s; ++i) {
+      const double send = upper ? v[i] : v[i + s];
+      const double keep = upper ? v[i + s] : v[i];
+      v[i] = keep + __shfl_xor_sync(0xffffffffu, send, s);
+    }
+  }
+  return v[0];
+}
 
-__global__ void __launch_bounds__(kGramTileRows * 32) k_gram_tile(Problem p, Work w, int pass) {
-  extern __shared__ __align__(16) unsigned char smem[];
-  double4* stage = reinterpret_cast<double4*>(smem);   // [nb][kGramChunk4]
+// Sums N per-lane values (N a power of two, at most 32) across the warp:
+// afterwards lane l holds the total of value l mod N (N − 1 halving shuffles,
+// then one per remaining lane bit).
+template <int N>
+__device__ __forceinline__ double warp_reduce_n(double (&v)[N]) {
+  const int lane = threadIdx.x & 31;
+#pragma unroll
+  for (int s = N / 2; s >= 1; s >>= 1) {
+    const bool upper = (lane & s) != 0;
+#pragma unroll
+    for (int i = 0; i < s; ++i) {
+      const double send = upper ? v[i] : v[i + s];
+      const double keep = upper ? v[i + s] : v[i];
+      v[i] = keep + __shfl_xor_sync(0xffffffffu, send, s);
+    }
+  }
+  double r = v[0];
+#pragma unroll
+  for (int s = N; s < 32; s <<= 1) r += __shfl_xor_sync(0xffffffffu, r, s);
+  return r;
+}
+
+// Tiled form for passes of at most kGramMaxNew picks, NB >= the pass's new
+// picks.  Block (row group, query slice, head): warp k takes row a0 + k of
+// the rows 0 .. s1 (rows below s1 are the picks' feature columns, row s1 is
+// m, giving b_new = Σ_i m_i Φ_{i,new}) against the new picks over one slice of
+// 512 queries (grid-stride over slices when there are more than gridDim.y).
+// The new picks' slice is staged in shared memory and every lane loads its
+// row's 16 queries before any is used; lane l then holds the partial of new
+// pick l mod NB after one butterfly across the warp.  Products of features
+// are exact (fp32 × fp32 in fp64).  The last block of a (head, row group) to
+// finish (counted with an atomic) adds the slices' partials in a fixed order
+// and writes each unordered pair of G once into both triangles, so G is
+// exactly symmetric and the result does not depend on block timing.
+constexpr int kGramWarps = 8;        // rows per block
+constexpr int kGramSlice4 = 128;     // float4 positions per query slice
+constexpr int kGramPos = kGramSlice4 / 32;   // float4 positions per lane
+
+template <int NB>
+__global__ void __launch_bounds__(kGramWarps * 32, 2) k_gram_tile(Problem p, Work w, int pass) {
+  __shared__ __align__(16) float4 stage[NB][kGramSlice4];
+  __shared__ const float4* newrow[NB];
   __shared__ int s_last;
-  const int h = w.order[blockIdx.y];
+  const int h = w.order[blockIdx.z];
   const int t = w.t[h];
   int s0, s1;
   pass_range(p, t, pass, s0, s1);
-  const int a0 = blockIdx.x * kGramTileRows;
-  if (s0 >= s1 || a0 >= s1) return;
+  const int a0 = blockIdx.x * kGramWarps;
+  if (s0 >= s1 || a0 > s1) return;
   const int nb = s1 - s0;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int a = a0 + warp;
-  const bool live = a < s1;
+  const int a = a0 + warp;                     // warp-uniform
+  const bool is_m = a == s1, live = a <= s1;
   const int64_t base = w.cu_t[h];
   const int64_t gbase = w.cu_t2[h];
   const int n4 = p.ldn >> 2;
-  const int per = (n4 + kGramSplits - 1) / kGramSplits;
-  const int k0 = blockIdx.z * per, k1 = min(n4, k0 + per);
+  const int nslices = (n4 + kGramSlice4 - 1) / kGramSlice4;
   const float* P0 = w.phiT + (int64_t)h * p.T * p.ldn;
-  const float4* ra = reinterpret_cast<const float4*>(P0 + (int64_t)w.picks[base + (live ? a : s0)] * p.ldn);
   const double2* m2 = reinterpret_cast<const double2*>(w.m + (int64_t)h * p.ldn);
-  __shared__ const float4* newrow[kGramMaxNew];
-  if (threadIdx.x < nb)
-    newrow[threadIdx.x] = reinterpret_cast<const float4*>(P0 + (int64_t)w.picks[base + s0 + threadIdx.x] * p.ldn);
+  if (threadIdx.x < NB)
+    newrow[threadIdx.x] = reinterpret_cast<const float4*>(
+        P0 + (int64_t)w.picks[base + s0 + min((int)threadIdx.x, nb - 1)] * p.ldn);
+  const float4* row = reinterpret_cast<const float4*>(P0 + (int64_t)w.picks[base + min(a, s1 - 1)] * p.ldn);
   __syncthreads();
-  double acc[kGramMaxNew];
+  double acc[NB];
 #pragma unroll
-  for (int b = 0; b < kGramMaxNew; ++b) acc[b] = 0.0;
-  double accm = 0.0;
-  for (int c0 = k0; c0 < k1; c0 += kGramChunk4) {
-    const int cw = min(kGramChunk4, k1 - c0);
-    for (int e0 = threadIdx.x; e0 < nb * cw; e0 += 4 * blockDim.x) {   // four loads in flight
-      float4 y[4];
+  for (int b = 0; b < NB; ++b) acc[b] = 0.0;
+  for (int sl = blockIdx.y; sl < nslices; sl += gridDim.y) {
+    const int c0 = sl * kGramSlice4;
+    const int cw = min(kGramSlice4, n4 - c0);
+    // every load of the slice first: the new picks' columns, then this warp's row
+    constexpr int kStage = (NB * kGramSlice4 + kGramWarps * 32 - 1) / (kGramWarps * 32);
+    float4 sv[kStage];
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int e = e0 + u * blockDim.x, b = e / cw, i = e - b * cw;
-        y[u] = e < nb * cw ? newrow[b][c0 + i] : make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int u = 0; u < kStage; ++u) {
+      const int e = threadIdx.x + u * kGramWarps * 32, b = e / kGramSlice4, i = e % kGramSlice4;
+      sv[u] = e < NB * kGramSlice4 && b < nb && i < cw ? newrow[b][c0 + i] : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+    float4 xf[kGramPos];
+    double2 xm[kGramPos][2];
+    if (is_m) {
+#pragma unroll
+      for (int k = 0; k < kGramPos; ++k) {
+        const int i = lane + 32 * k;
+        xm[k][0] = i < cw ? m2[2 * (c0 + i)] : make_double2(0.0, 0.0);
+        xm[k][1] = i < cw ? m2[2 * (c0 + i) + 1] : make_double2(0.0, 0.0);
       }
+    } else {
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int e = e0 + u * blockDim.x, b = e / cw, i = e - b * cw;
-        if (e < nb * cw) stage[b * kGramChunk4 + i] = make_double4(y[u].x, y[u].y, y[u].z, y[u].w);
+      for (int k = 0; k < kGramPos; ++k) {
+        const int i = lane + 32 * k;
+        xf[k] = live && i < cw ? row[c0 + i] : make_float4(0.f, 0.f, 0.f, 0.f);
       }
     }
-    __syncthreads();
-    if (live) {
-      for (int i = lane; i < cw; i += 32) {
-        const float4 xf = ra[c0 + i];
-        const double4 x = make_double4(xf.x, xf.y, xf.z, xf.w);
 #pragma unroll
-        for (int b = 0; b < kGramMaxNew; ++b) {
-          if (b < nb) {
-            const double4 y = stage[b * kGramChunk4 + i];
-            acc[b] += x.x * y.x + x.y * y.y + x.z * y.z + x.w * y.w;
-          }
+    for (int u = 0; u < kStage; ++u) {
+      const int e = threadIdx.x + u * kGramWarps * 32;
+      if (e < NB * kGramSlice4) stage[e / kGramSlice4][e % kGramSlice4] = sv[u];
+    }
+    __syncthreads();
+    if (is_m) {
+#pragma unroll
+      for (int b = 0; b < NB; ++b) {
+#pragma unroll
+        for (int k = 0; k < kGramPos; ++k) {
+          const float4 y = stage[b][lane + 32 * k];
+          acc[b] = fma(xm[k][0].x, (double)y.x, acc[b]);
+          acc[b] = fma(xm[k][0].y, (double)y.y, acc[b]);
+          acc[b] = fma(xm[k][1].x, (double)y.z, acc[b]);
+          acc[b] = fma(xm[k][1].y, (double)y.w, acc[b]);
         }
-        if (a >= s0) {
-          const double2 u = m2[2 * (c0 + i)], v = m2[2 * (c0 + i) + 1];
-          accm += x.x * u.x + x.y * u.y + x.z * v.x + x.w * v.y;
+      }
+    } else {
+#pragma unroll
+      for (int b = 0; b < NB; ++b) {
+#pragma unroll
+        for (int k = 0; k < kGramPos; ++k) {
+          const float4 y = stage[b][lane + 32 * k];
+          acc[b] = fma((double)xf[k].x, (double)y.x, acc[b]);
+          acc[b] = fma((double)xf[k].y, (double)y.y, acc[b]);
+          acc[b] = fma((double)xf[k].z, (double)y.z, acc[b]);
+          acc[b] = fma((double)xf[k].w, (double)y.w, acc[b]);
         }
       }
     }
     __syncthreads();
   }
-  // partials: [split][row 0..t (row t: the new rows' b)][kR]
-  double* part = w.gpart + (int64_t)kGramSplits * (base + h) * p.kR;
-  const int64_t stride = (int64_t)(t + 1) * p.kR;
-  if (live) {
-#pragma unroll
-    for (int b = 0; b < kGramMaxNew; ++b) {
-      if (b < nb) {
-        const double v = warp_sum(acc[b]);
-        if (lane == 0) part[blockIdx.z * stride + (int64_t)a * p.kR + b] = v;
-      }
-    }
-    if (a >= s0) {
-      const double v = warp_sum(accm);
-      if (lane == 0) part[blockIdx.z * stride + (int64_t)t * p.kR + (a - s0)] = v;
-    }
+  // partials: [slice][row 0..t (row t: b_new)][kR]
+  double* part = w.gpart + (int64_t)kGramMaxSlices * (base + h) * p.kR;
+  const int64_t zstride = (int64_t)(t + 1) * p.kR;
+  {
+    const double tot = warp_reduce_n<NB>(acc);
+    const int prow = is_m ? t : a;
+    if (live && lane < nb) part[blockIdx.y * zstride + (int64_t)prow * p.kR + lane] = tot;
   }
   __threadfence();
   __syncthreads();
-  if (threadIdx.x == 0) {
-    const int blocks = (s1 + kGramTileRows - 1) / kGramTileRows * kGramSplits;
-    s_last = atomicAdd(w.gcount + h, 1) == blocks - 1;
-  }
+  int32_t* counter = w.gcount + base + h + blockIdx.x;
+  if (threadIdx.x == 0) s_last = atomicAdd(counter, 1) == (int)gridDim.y - 1;
   __syncthreads();
   if (!s_last) return;
   __threadfence();
-  for (int e = threadIdx.x; e < (s1 + 1) * nb; e += blockDim.x) {
-    const int r = e / nb, b = e - r * nb;
-    const int row = r < s1 ? r : t;                  // the last entry row holds b
+  const int rows_here = min(kGramWarps, s1 + 1 - a0);
+  for (int e = threadIdx.x; e < rows_here * nb; e += blockDim.x) {
+    const int ri = e / nb, b = e - ri * nb;
+    const int r = a0 + ri;
+    const int prow = r == s1 ? t : r;
     double v = 0.0;
+    for (int q0 = 0; q0 < (int)gridDim.y; q0 += 8) {   // eight slices' partials in flight
+      double z[8];
 #pragma unroll
-    for (int z = 0; z < kGramSplits; ++z) v += part[z * stride + (int64_t)row * p.kR + b];
-    if (r < s1) {
-      w.G[gbase + (int64_t)r * t + s0 + b] = v;
-      if (r < s0) w.G[gbase + (int64_t)(s0 + b) * t + r] = v;
-    } else {
+      for (int q = 0; q < 8; ++q)
+        z[q] = q0 + q < (int)gridDim.y ? __ldcg(part + (q0 + q) * zstride + (int64_t)prow * p.kR + b) : 0.0;
+#pragma unroll
+      for (int q = 0; q < 8; ++q) v += z[q];
+    }
+    if (r == s1) {
       w.bvec[base + s0 + b] = v;
+    } else if (r < s0 || s0 + b <= r) {   // each unordered pair once, both triangles
+      w.G[gbase + (int64_t)r * t + s0 + b] = v;
+      w.G[gbase + (int64_t)(s0 + b) * t + r] = v;
     }
   }
-  if (threadIdx.x == 0) w.gcount[h] = 0;   // ready for the next pass
+  if (threadIdx.x == 0) *counter = 0;   // ready for the next pass
 }
 
 // ---------------------------------------------------------------- NNLS ----
@@ -464,23 +530,6 @@ __device__ __forceinline__ void load_diag_tile(const double* L, int r0, int bw, 
       if (e < kSB * kSB) D[e >> 5][e & 31] = v[u];
     }
   }
-}
-
-// Sums 32 per-lane values across the warp: afterwards lane l holds the
-// total of value l (31 shuffles: each step halves the values a lane keeps).
-__device__ __forceinline__ double warp_reduce32(double (&v)[32]) {
-  const int lane = threadIdx.x & 31;
-#pragma unroll
-  for (int s = 16; s >= 1; s >>= 1) {
-    const bool upper = (lane & s) != 0;
-#pragma unroll
-    for (int i = 0; i < s; ++i) {
-      const double send = upper ? v[i] : v[i + s];
-      const double keep = upper ? v[i + s] : v[i];
-      v[i] = keep + __shfl_xor_sync(0xffffffffu, send, s);
-    }
-  }
-  return v[0];
 }
 
 // u_e ← L⁻¹ u_e on rows [k0, n) for the R <= 8 vectors U[0..R); entries
@@ -1018,7 +1067,6 @@ __global__ void __launch_bounds__(kNnlsThreads) k_nnls(Problem p, Work w, int pa
 // A block covers 32 float4 positions (128 queries) with four thread groups,
 // group g taking picks g, g + 4, ...; the groups' sums are combined in a
 // fixed order, so the result is deterministic.
-constexpr int kResidPos = 32;      // float4 positions per block
 constexpr int kResidGroups = 4;    // pick groups per position
 constexpr int kResidThreads = kResidPos * kResidGroups;
 constexpr int kResidChunk = 512;   // picks staged in shared memory at a time
@@ -1098,11 +1146,6 @@ __global__ void k_residual_norm(Problem p, Work w, int nblk, double* out) {
   out[h] = sqrt(s / w.mm[h]);
 }
 
-int resid_blocks(const Problem& p) {
-  int n4 = p.ldn / 4;
-  int b = (n4 + kResidPos - 1) / kResidPos;
-  return b < kRedBlocks ? b : kRedBlocks;
-}
 
 }  // namespace
 
@@ -1140,10 +1183,18 @@ cudaError_t launch_omp_pass(const Problem& p, const Work& w, int pass, int activ
   }
   const int s1max = (pass + 1) * p.kR < p.max_t ? (pass + 1) * p.kR : p.max_t;
   if (p.kR <= kGramMaxNew) {
-    dim3 gg((s1max + kGramTileRows - 1) / kGramTileRows, active, kGramSplits);
-    const int gsm = p.kR * kGramChunk4 * (int)sizeof(double4);
-    cudaFuncSetAttribute(k_gram_tile, cudaFuncAttributeMaxDynamicSharedMemorySize, gsm);
-    AM_LAUNCH(AM_STAGE_GRAM, s, k_gram_tile<<<gg, kGramTileRows * 32, gsm, s>>>(p, w, pass));
+    const int nslices = (p.ldn / 4 + kGramSlice4 - 1) / kGramSlice4;
+    const int Z = nslices < kGramMaxSlices ? nslices : kGramMaxSlices;
+    const int nb = p.kR <= 1 ? 1 : p.kR <= 2 ? 2 : p.kR <= 4 ? 4 : p.kR <= 8 ? 8 : 16;
+    dim3 gg((s1max + 1 + kGramWarps - 1) / kGramWarps, Z, active);
+    const int th = kGramWarps * 32;
+    switch (nb) {
+      case 1: AM_LAUNCH(AM_STAGE_GRAM, s, k_gram_tile<1><<<gg, th, 0, s>>>(p, w, pass)); break;
+      case 2: AM_LAUNCH(AM_STAGE_GRAM, s, k_gram_tile<2><<<gg, th, 0, s>>>(p, w, pass)); break;
+      case 4: AM_LAUNCH(AM_STAGE_GRAM, s, k_gram_tile<4><<<gg, th, 0, s>>>(p, w, pass)); break;
+      case 8: AM_LAUNCH(AM_STAGE_GRAM, s, k_gram_tile<8><<<gg, th, 0, s>>>(p, w, pass)); break;
+      default: AM_LAUNCH(AM_STAGE_GRAM, s, k_gram_tile<16><<<gg, th, 0, s>>>(p, w, pass)); break;
+    }
   } else {
     dim3 gg(s1max, active);
     AM_LAUNCH(AM_STAGE_GRAM, s, k_gram<<<gg, 256, 0, s>>>(p, w, pass));
