@@ -135,7 +135,8 @@ am_status_t check_shape(int n, int T, int d, int H, const int32_t* budgets, cons
     if (t < 1 || t > T) return AM_ERR_BUDGET;
     if (t > kMaxBudget) return AM_ERR_UNSUPPORTED;
     tb->cu_t[h + 1] = tb->cu_t[h] + t;
-    tb->cu_t2[h + 1] = tb->cu_t2[h] + (int64_t)t * t;
+    // t² rounded up to even: every head's t×t regions start 16-byte aligned
+    tb->cu_t2[h + 1] = tb->cu_t2[h] + (((int64_t)t * t + 1) & ~(int64_t)1);
     tb->max_t = std::max(tb->max_t, t);
     passes[h] = num_passes(t, kR);
   }

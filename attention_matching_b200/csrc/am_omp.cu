@@ -15,6 +15,7 @@
 //   k_nnls    active-set NNLS on (G, b), warm-started from the last refit
 //   k_resid   r = m − Φ_S w (fp64 sums, stored fp32)
 #include "am_internal.cuh"
+#include "am_async.cuh"
 #include "am_profile.cuh"
 #include "am_linalg.cuh"
 
@@ -482,13 +483,15 @@ constexpr size_t kDiagTileBytes = kSB * (kSB + 1) * sizeof(double);
 
 __host__ __device__ inline size_t nnls_vec_bytes(int t) {
   // x, z, g, invd, y: 5t doubles; red: 64 doubles; diagonal tile: 32×33 doubles;
-  // ctl: 16 ints; P, inP, blocked, add, cand: 5t ints
-  size_t b = (size_t)t * 5 * sizeof(double) + 64 * sizeof(double) + kDiagTileBytes + 16 * sizeof(int) +
+  // ctl: 16 ints; the factor copy's barrier: 16 bytes; P, inP, blocked, add, cand: 5t ints
+  size_t b = (size_t)t * 5 * sizeof(double) + 64 * sizeof(double) + kDiagTileBytes + 16 * sizeof(int) + 16 +
              (size_t)t * 5 * sizeof(int);
   return (b + 15) & ~size_t(15);
 }
 __host__ __device__ inline size_t nnls_tri_bytes(int t) { return (size_t)t * (t + 1) / 2 * sizeof(double); }
 constexpr size_t kSmemCap = 227 * 1024;
+constexpr uint32_t kBulkChunk = 32768;               // bytes per bulk copy instruction
+constexpr long long kBulkWaitCycles = 4000000000ll;  // ~2 s at 2 GHz
 
 // Blocked triangular solves with the packed factor (shared or global
 // memory), run by all threads of the block, 32 rows at a time.  Each block of
@@ -752,7 +755,8 @@ __global__ void __launch_bounds__(kNnlsThreads) k_nnls(Problem p, Work w, int pa
   double* red = yv + t;                          // 64 doubles
   DiagTile* D = reinterpret_cast<DiagTile*>(red + 64);              // solve scratch
   int* ctl = reinterpret_cast<int*>(red + 64 + kSB * (kSB + 1));    // 16 ints
-  int* P = ctl + 16;
+  uint64_t* lbar = reinterpret_cast<uint64_t*>(ctl + 16);            // 16 bytes
+  int* P = ctl + 20;
   int* inP = P + t;
   int* blocked = inP + t;
   int* add = blocked + t;
@@ -760,7 +764,12 @@ __global__ void __launch_bounds__(kNnlsThreads) k_nnls(Problem p, Work w, int pa
   const bool l_smem = t <= l_in_smem_max;
   double* Lg = w.L + gbase;
   double* L = l_smem ? reinterpret_cast<double*>(smem + nnls_vec_bytes(t)) : Lg;
-  // ctl: 0 np, 1 nadd, 2 single mode, 4 argmin, 5 nneg, 7 ncand, 9 removed count, 10 valid y rows
+  // the factor kept in shared memory arrives by one bulk copy (16-byte
+  // aligned at both ends; rounding the size up reads at most one double past
+  // the factor, still inside the head's t×t region and the shared buffer)
+  const uint32_t lbytes = l_smem ? (uint32_t)((tri(np_old, 0) * 8 + 15) & ~(int64_t)15) : 0u;
+  // ctl: 0 np, 1 nadd, 2 single mode, 4 argmin, 5 nneg, 7 ncand, 9 removed count, 10 valid y rows,
+  //      11 first factor row that differs from the stored factor
   const int maxit = p.nnls_max_iter > 0 ? p.nnls_max_iter : 3 * t + 50;
   const double mnorm = sqrt(w.mm[h]);
   auto diag = [&](int l) { return G[(int64_t)l * t + l]; };
@@ -770,12 +779,26 @@ __global__ void __launch_bounds__(kNnlsThreads) k_nnls(Problem p, Work w, int pa
     inP[l] = 0;
     blocked[l] = 0;
   }
+  if (lbytes > 0 && tid == 0) {
+    mbar_init(lbar, 1);
+    mbar_init_fence();
+    mbar_expect_tx(lbar, lbytes);
+    for (uint32_t o = 0; o < lbytes; o += kBulkChunk)
+      bulk_load(reinterpret_cast<char*>(L) + o, reinterpret_cast<const char*>(Lg) + o,
+                lbytes - o < kBulkChunk ? lbytes - o : kBulkChunk, lbar);
+  }
   for (int q = tid; q < np_old; q += blockDim.x) P[q] = w.plist[base + q];
   const int ylen0 = min(w.ylen[h], np_old);
   for (int q = tid; q < ylen0; q += blockDim.x) yv[q] = w.ycache[base + q];
-  if (l_smem) copy_doubles(L, Lg, tri(np_old, 0));
-  if (tid == 0) { ctl[0] = np_old; ctl[2] = 0; ctl[10] = ylen0; }
-  __syncthreads();
+  if (tid == 0) { ctl[0] = np_old; ctl[2] = 0; ctl[10] = ylen0; ctl[11] = np_old; }
+  __syncthreads();   // the barrier is initialised before anyone waits on it
+  const bool landed = lbytes == 0 || mbar_wait_bounded(lbar, 0, kBulkWaitCycles);
+  if (__syncthreads_or(!landed)) {
+    // the copy did not land: flag the head, let it drain, leave everything as it was
+    if (tid == 0) record_status(w.status + h, AM_ERR_TIMEOUT);
+    mbar_wait_bounded(lbar, 0, kBulkWaitCycles);
+    return;
+  }
   for (int q = tid; q < np_old; q += blockDim.x) {
     inP[P[q]] = 1;
     invd[q] = 1.0 / L[tri(q, q)];
@@ -1041,7 +1064,10 @@ __global__ void __launch_bounds__(kNnlsThreads) k_nnls(Problem p, Work w, int pa
       // delete the leavers from the factor, last position first
       const int nrm = ctl[9];
       for (int i = nrm - 1, npr = ctl[0] + nrm; i >= 0; --i, --npr) factor_remove(L, invd, g, red, cand[i], npr);
-      if (tid == 0 && nrm > 0) ctl[10] = min(ctl[10], cand[0]);
+      if (tid == 0 && nrm > 0) {
+        ctl[10] = min(ctl[10], cand[0]);
+        ctl[11] = min(ctl[11], cand[0]);
+      }
       __syncthreads();
     }
     if (abort) break;
@@ -1054,7 +1080,10 @@ __global__ void __launch_bounds__(kNnlsThreads) k_nnls(Problem p, Work w, int pa
   for (int q = tid; q < npf; q += blockDim.x) w.plist[base + q] = P[q];
   const int yl = ctl[10];
   for (int q = tid; q < yl; q += blockDim.x) w.ycache[base + q] = yv[q];
-  if (l_smem) copy_doubles(Lg, L, tri(npf, 0));
+  if (l_smem) {   // rows above ctl[11] are unchanged since the load
+    const int64_t e0 = tri(ctl[11], 0);
+    copy_doubles(Lg + e0, L + e0, tri(npf, 0) - e0);
+  }
   if (tid == 0) {
     w.np[h] = npf;
     w.ylen[h] = yl;

@@ -24,6 +24,7 @@
 // Every mbarrier wait is bounded by a clock budget; on expiry the CTA records
 // AM_ERR_TIMEOUT, stops issuing work, drains what it issued and releases TMEM.
 #include "am_internal.cuh"
+#include "am_async.cuh"
 #include "am_profile.cuh"
 
 #include <cuda.h>
@@ -69,36 +70,7 @@ __host__ __device__ inline Plan make_plan(int d, int mode) {
   return P;
 }
 
-// ---- PTX wrappers ----
-__device__ __forceinline__ uint32_t smem_u32(const void* p) {
-  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
-}
-
-__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
-  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count));
-}
-
-__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
-  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
-               : "memory");
-}
-
-__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
-  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
-}
-
-__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok)
-      : "r"(smem_u32(bar)), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
-
+// ---- PTX wrappers (mbarriers: am_async.cuh) ----
 // Bounded wait: false if the CTA aborted (here or elsewhere) before completion.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
                                           int32_t* status) {
@@ -261,7 +233,7 @@ k_phi_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtens
     }
     mbar_init(y_full, 1);
     mbar_init(drain, 1);
-    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    mbar_init_fence();
   }
   if (warp == 2) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(&s_tmem)),
@@ -594,7 +566,7 @@ k_corr_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
     for (int s = 0; s < CSTAGES; ++s) { mbar_init(q_full + s, 1); mbar_init(q_empty + s, 1); }
     for (int b = 0; b < 2; ++b) { mbar_init(s_full + b, 1); mbar_init(s_empty + b, 512); }
     mbar_init(drain, 1);
-    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    mbar_init_fence();
   }
   if (warp == 2) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(&s_tmem)),
