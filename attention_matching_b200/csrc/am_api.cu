@@ -31,7 +31,7 @@ struct Layout {
   size_t picks, pick_corr, plist, sorted_slot;
   size_t bvec, w, w_eff, ycache;
   size_t G, L, AtA, A, AtY, nrm_part;
-  size_t cnorm, cnpart, rnorm, corrd, korder, knorm, ksort, cprefix, cdone, cprobe, rows_eval, gpart, gcount, rcount,
+  size_t cnorm, cnpart, rnorm, clist, clj, ccount, korder, knorm, ksort, cprefix, cdone, cprobe, rows_eval, gpart, gcount, rcount,
       dinv;
   size_t total;
   size_t tables_bytes;
@@ -88,7 +88,9 @@ Layout plan(int n, int T, int d, int H, int64_t sum_t, int64_t sum_t2, bool corr
   L.cnorm = take((size_t)H * T * 8);
   L.cnpart = take((size_t)H * 4 * ((n + 127) / 128) * T * 4);
   L.rnorm = take((size_t)H * 8);
-  L.corrd = take((size_t)H * T * 8);
+  L.clist = take((size_t)H * T * 8);
+  L.clj = take((size_t)H * T * 4);
+  L.ccount = take((size_t)H * 4);
   L.korder = take((size_t)H * T * 4);
   L.knorm = take((size_t)H * T * 4);
   size_t t2 = 1;
@@ -205,7 +207,9 @@ Work bind(const Layout& L, char* base, bool corr_bf16) {
   w.cnorm = reinterpret_cast<double*>(base + L.cnorm);
   w.cnpart = reinterpret_cast<float*>(base + L.cnpart);
   w.rnorm = reinterpret_cast<double*>(base + L.rnorm);
-  w.corrd = reinterpret_cast<double*>(base + L.corrd);
+  w.clist = reinterpret_cast<uint64_t*>(base + L.clist);
+  w.clj = reinterpret_cast<int32_t*>(base + L.clj);
+  w.ccount = reinterpret_cast<int32_t*>(base + L.ccount);
   w.korder = reinterpret_cast<int32_t*>(base + L.korder);
   w.knorm = reinterpret_cast<float*>(base + L.knorm);
   w.ksort = reinterpret_cast<uint64_t*>(base + L.ksort);
@@ -401,6 +405,7 @@ am_status_t compact_heads_impl(const void* Q, const void* K, const void* V, int3
   AM_TRY(cudaMemsetAsync(w.gcount, 0, ((size_t)tb.sum_t + H) * 4, s));
   AM_TRY(cudaMemsetAsync(w.rcount, 0, (size_t)H * 4, s));
   AM_TRY(cudaMemsetAsync(w.cprefix, 0, (size_t)H * 4, s));
+  AM_TRY(cudaMemsetAsync(w.ccount, 0, (size_t)H * 4, s));
   const CorrInputs cin{Q, K, opts->key_bias};
   if (G == 1) {
     for (int pass = 0; pass < (int)tb.active.size(); ++pass)

@@ -128,41 +128,34 @@ constexpr int kSelThreads = 256;
 struct SelScratch {
   uint64_t key[kSelCap];
   int idx[kSelCap];
-  uint64_t ck[kSelThreads / 32][kMaxPicksPerPass];   // each warp's best, in pick order
-  int cj[kSelThreads / 32][kMaxPicksPerPass];
+  uint64_t ck[kSelThreads / 32 * kMaxPicksPerPass];   // warp w's kk best at [w·kk, (w+1)·kk)
+  int cj[kSelThreads / 32 * kMaxPicksPerPass];
   uint64_t outk[kMaxPicksPerPass];
   int outj[kMaxPicksPerPass];
   double red[33];
-  int cnt;
 };
 
-// Appends the unselected keys at sorted positions [lo, hi) to the candidate
-// slots from S.cnt on (at most kSelCap in all); all threads.
-__device__ void stage_candidates(const Problem& p, const Work& w, int h, int lo, int hi, SelScratch& S) {
-  const int32_t* ord = w.korder + (int64_t)h * p.T;
-  const uint8_t* sel = w.sel + (int64_t)h * p.T;
-  const double* cd = w.corrd + (int64_t)h * p.T;
-  for (int q0 = lo + threadIdx.x; q0 < hi; q0 += 4 * blockDim.x) {   // four keys in flight
+// Copies entries [lo, hi) of the head's list of evaluated keys (order key of
+// c_j, key index) to candidate slots from `at` on; all threads, four loads
+// per thread in flight.
+__device__ void stage_list(const Problem& p, const Work& w, int h, int lo, int hi, int at, SelScratch& S) {
+  const uint64_t* lk = w.clist + (int64_t)h * p.T;
+  const int32_t* lj = w.clj + (int64_t)h * p.T;
+  for (int q0 = lo + threadIdx.x; q0 < hi; q0 += 4 * blockDim.x) {
+    uint64_t k[4];
     int j[4];
-    bool s[4];
-    double v[4];
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
       const int q = q0 + u * blockDim.x;
-      j[u] = q < hi ? ord[q] : -1;
+      k[u] = q < hi ? __ldcg(lk + q) : 0ull;
+      j[u] = q < hi ? __ldcg(lj + q) : 0;
     }
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
-      s[u] = j[u] < 0 || sel[j[u] < 0 ? 0 : j[u]];
-      v[u] = cd[j[u] < 0 ? 0 : j[u]];
-    }
-#pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      if (s[u]) continue;
-      const int pos = atomicAdd(&S.cnt, 1);
-      if (pos < kSelCap) {
-        S.key[pos] = order_key(v[u]);
-        S.idx[pos] = j[u];
+      const int q = q0 + u * blockDim.x;
+      if (q < hi) {
+        S.key[at + q - lo] = k[u];
+        S.idx[at + q - lo] = j[u];
       }
     }
   }
@@ -219,17 +212,9 @@ __device__ __forceinline__ void warp_top(uint64_t* keys, int* idx, int first, in
 // The slots are consumed.  All threads.
 __device__ void select_top(SelScratch& S, int n, int kk) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
-  warp_top(S.key, S.idx, warp * 32 + lane, blockDim.x, n, kk, S.ck[warp], S.cj[warp]);
+  warp_top(S.key, S.idx, warp * 32 + lane, blockDim.x, n, kk, S.ck + warp * kk, S.cj + warp * kk);
   __syncthreads();
-  if (warp == 0) {
-    // candidates (w, k) at flat position w·kMaxPicksPerPass + k, k < kk
-    uint64_t* ck = &S.ck[0][0];
-    int* cj = &S.cj[0][0];
-    for (int e = lane; e < nw * kMaxPicksPerPass; e += 32)
-      if (e % kMaxPicksPerPass >= kk) cj[e] = INT_MAX;
-    __syncwarp();
-    warp_top(ck, cj, lane, 32, nw * kMaxPicksPerPass, kk, S.outk, S.outj);
-  }
+  if (warp == 0) warp_top(S.ck, S.cj, lane, 32, nw * kk, kk, S.outk, S.outj);
   __syncthreads();
 }
 
@@ -270,10 +255,8 @@ __device__ void theta_and_prefix(const Problem& p, const Work& w, int h, int pas
   const int nrb = resid_blocks(p);
   const double rr_mine = pass == 0 ? (threadIdx.x == 0 ? w.mm[h] : 0.0)
                                    : ((int)threadIdx.x < nrb ? w.rr_part[(int64_t)h * kRedBlocks + threadIdx.x] : 0.0);
-  if (threadIdx.x == 0) S.cnt = 0;
-  __syncthreads();
-  stage_candidates(p, w, h, 0, p0, S);   // p0 <= kSelCap
-  const int staged = min(S.cnt, kSelCap);
+  const int staged = __ldcg(w.ccount + h);   // <= p0 <= kSelCap: the probe's unselected keys
+  stage_list(p, w, h, 0, staged, 0, S);
   select_top(S, staged, kk);
   const double rn = sqrt(block_sum(rr_mine, S.red));
   const int jt = S.outj[kk - 1];
@@ -289,7 +272,10 @@ __device__ void theta_and_prefix(const Problem& p, const Work& w, int h, int pas
     w.cprobe[h] = p0;
     w.cdone[h] = done;
     w.rnorm[h] = rn;
-    if (done) w.rows_eval[h] += (unsigned long long)staged;
+    if (done) {
+      w.rows_eval[h] += (unsigned long long)staged;
+      w.ccount[h] = 0;   // the list is consumed; otherwise the second launch extends it
+    }
   }
   if (done) append_picks(p, w, h, s0, kk, S);
 }
@@ -327,29 +313,28 @@ __device__ void append_picks(const Problem& p, const Work& w, int h, int s0, int
   }
 }
 
-// The kk largest values among the unselected keys of [0, L), in chunks that
-// carry the best kk of what came before (the last block of a head, after the
-// remaining rows).
+// The kk largest values in the head's list of evaluated keys (the unselected
+// keys of [0, L)), in chunks that carry the best kk of what came before (the
+// last block of a head, after the remaining rows).
 __device__ void pick_from_prefix(const Problem& p, const Work& w, int h, int s0, int kk, SelScratch& S) {
-  const int L = w.cprefix[h];
+  const int n = __ldcg(w.ccount + h);
   const int chunk = kSelCap - kMaxPicksPerPass;
   int kept = 0;
-  unsigned long long evaluated = 0;
-  for (int c = 0; c < L; c += chunk) {
+  for (int c = 0; c < n; c += chunk) {
     if (threadIdx.x < kept) {   // winners so far lead the next chunk
       S.key[threadIdx.x] = S.outk[threadIdx.x];
       S.idx[threadIdx.x] = S.outj[threadIdx.x];
     }
-    if (threadIdx.x == 0) S.cnt = kept;
-    __syncthreads();
-    stage_candidates(p, w, h, c, min(L, c + chunk), S);
-    const int n = min(S.cnt, kSelCap);
-    evaluated += (unsigned long long)(n - kept);
-    select_top(S, n, kk);
+    const int m = min(n, c + chunk) - c;
+    stage_list(p, w, h, c, c + m, kept, S);
+    select_top(S, kept + m, kk);
     kept = 0;
     for (int k = 0; k < kk; ++k) kept += S.outj[k] != INT_MAX;
   }
-  if (threadIdx.x == 0) w.rows_eval[h] += evaluated;
+  if (threadIdx.x == 0) {
+    w.rows_eval[h] += (unsigned long long)n;
+    w.ccount[h] = 0;
+  }
   append_picks(p, w, h, s0, kk, S);
 }
 
@@ -364,6 +349,7 @@ constexpr int kRowSplit = 4;                           // warps per key
 constexpr int kRowsPerBlock = kSelThreads / 32 / kRowSplit;   // keys per block
 
 __global__ void __launch_bounds__(kSelThreads) k_rows(Problem p, Work w, int pass, int which) {
+  chain_wait();
   extern __shared__ __align__(16) unsigned char smem[];
   SelScratch& S = *reinterpret_cast<SelScratch*>(smem);
   __shared__ double part[kRowsPerBlock][kRowSplit];
@@ -415,10 +401,15 @@ __global__ void __launch_bounds__(kSelThreads) k_rows(Problem p, Work w, int pas
     const double c = warp_sum((a[0] + a[1]) + (a[2] + a[3]));
     if (lane == 0) part[slot][quarter] = c;
     __syncthreads();
-    if (on && quarter == 0 && lane == 0)
-      w.corrd[(int64_t)h * p.T + j] = (part[slot][0] + part[slot][1]) + (part[slot][2] + part[slot][3]);
+    if (on && quarter == 0 && lane == 0) {   // onto the head's list of evaluated keys
+      const double cj = (part[slot][0] + part[slot][1]) + (part[slot][2] + part[slot][3]);
+      const int at = atomicAdd(w.ccount + h, 1);
+      w.clist[(int64_t)h * p.T + at] = order_key(cj);
+      w.clj[(int64_t)h * p.T + at] = j;
+    }
     __syncthreads();
   }
+  chain_release();
   // the last block of this head to get here takes the selection step
   __threadfence();
   __syncthreads();
@@ -456,8 +447,8 @@ cudaError_t launch_corr_bounded(const Problem& p, const Work& w, int pass, int a
   const int sel_smem = (int)sizeof(SelScratch);
   cudaFuncSetAttribute(k_rows, cudaFuncAttributeMaxDynamicSharedMemorySize, sel_smem);
   dim3 gr(rows_ctas_per_head(active), active);
-  AM_LAUNCH(AM_STAGE_ROWS, s, k_rows<<<gr, kSelThreads, sel_smem, s>>>(p, w, pass, 0));
-  AM_LAUNCH(AM_STAGE_ROWS, s, k_rows<<<gr, kSelThreads, sel_smem, s>>>(p, w, pass, 1));
+  AM_LAUNCH(AM_STAGE_ROWS, s, launch_chained(k_rows, gr, dim3(kSelThreads), sel_smem, s, p, w, pass, 0));
+  AM_LAUNCH(AM_STAGE_ROWS, s, launch_chained(k_rows, gr, dim3(kSelThreads), sel_smem, s, p, w, pass, 1));
   return cudaGetLastError();
 }
 

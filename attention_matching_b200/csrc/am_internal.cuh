@@ -70,7 +70,9 @@ struct Work {
   double* cnorm;        // [H][T] ‖Φ_{:,j}‖₂ (fp64, an upper bound within 1e-6 when from cnpart)
   float* cnpart;        // [H][⌈n/128⌉][4][T] per-warp partial Σ_i Φ_ij² from the feature pass, or null
   double* rnorm;        // [H] ‖r‖₂ of the stored fp32 residual, this pass
-  double* corrd;        // [H][T] exact correlations of this pass's evaluated keys
+  uint64_t* clist;      // [H][T] this pass's evaluated keys: order keys of their exact c_j
+  int32_t* clj;         // [H][T] and the key indices, in completion order
+  int32_t* ccount;      // [H] entries in that list
   int32_t* korder;      // [H][T] keys by descending column norm
   float* knorm;         // [H][T] those norms (fp32, descending)
   uint64_t* ksort;      // [H][pow2 >= T] sort scratch when T exceeds the shared-memory sort
@@ -166,6 +168,32 @@ __host__ __device__ inline int num_passes(int t, int kR) { return (t + kR - 1) /
 __device__ __forceinline__ void pass_range(const Problem& p, int t, int pass, int& s0, int& s1) {
   s0 = min(pass * p.kR, t);
   s1 = min(s0 + p.kR, t);
+}
+
+// ---- programmatic dependent launch (the per-pass kernel chain) ----
+// A kernel launched with launch_chained may start while its stream
+// predecessor drains: it must call chain_wait() before touching anything,
+// which returns once the predecessor grid has completed and its writes are
+// visible (a no-op for an ordinary launch).  chain_release() lets the next
+// chained kernel begin launching; a kernel calls it once its block is past
+// the main parallel work.
+__device__ __forceinline__ void chain_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void chain_release() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_chained(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                                  Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
 }
 
 }  // namespace am

@@ -339,6 +339,7 @@ constexpr int kGramPos = kGramSlice4 / 32;   // float4 positions per lane
 
 template <int NB>
 __global__ void __launch_bounds__(kGramWarps * 32, 2) k_gram_tile(Problem p, Work w, int pass) {
+  chain_wait();
   __shared__ __align__(16) float4 stage[NB][kGramSlice4];
   __shared__ const float4* newrow[NB];
   __shared__ int s_last;
@@ -434,6 +435,7 @@ __global__ void __launch_bounds__(kGramWarps * 32, 2) k_gram_tile(Problem p, Wor
     const int prow = is_m ? t : a;
     if (live && lane < nb) part[blockIdx.y * zstride + (int64_t)prow * p.kR + lane] = tot;
   }
+  chain_release();
   __threadfence();
   __syncthreads();
   int32_t* counter = w.gcount + base + h + blockIdx.x;
@@ -734,6 +736,7 @@ __device__ void factor_remove(double* L, double* invd, double* xv, double* rot, 
 }
 
 __global__ void __launch_bounds__(kNnlsThreads) k_nnls(Problem p, Work w, int pass, int l_in_smem_max) {
+  chain_wait();
   extern __shared__ __align__(16) unsigned char smem[];
   const int h = w.order[blockIdx.x];
   const int t = w.t[h];
@@ -1075,6 +1078,7 @@ __global__ void __launch_bounds__(kNnlsThreads) k_nnls(Problem p, Work w, int pa
   __syncthreads();
 
   // ---- write back ----
+  chain_release();
   const int npf = ctl[0];
   for (int l = tid; l < s1; l += blockDim.x) w.w[base + l] = inP[l] ? x[l] : 0.0;
   for (int q = tid; q < npf; q += blockDim.x) w.plist[base + q] = P[q];
@@ -1101,6 +1105,7 @@ constexpr int kResidThreads = kResidPos * kResidGroups;
 constexpr int kResidChunk = 512;   // picks staged in shared memory at a time
 
 __global__ void __launch_bounds__(kResidThreads) k_resid(Problem p, Work w, int pass) {
+  chain_wait();
   const int h = w.order[blockIdx.y];
   const int t = w.t[h];
   int s0, s1;
@@ -1163,6 +1168,7 @@ __global__ void __launch_bounds__(kResidThreads) k_resid(Problem p, Work w, int 
       rr += acc[0] * acc[0] + acc[1] * acc[1] + acc[2] * acc[2] + acc[3] * acc[3];
     }
   }
+  chain_release();
   rr = block_sum(rr, scratch);
   if (threadIdx.x == 0) w.rr_part[(int64_t)h * kRedBlocks + blockIdx.x] = rr;
 }
@@ -1218,11 +1224,11 @@ cudaError_t launch_omp_pass(const Problem& p, const Work& w, int pass, int activ
     dim3 gg((s1max + 1 + kGramWarps - 1) / kGramWarps, Z, active);
     const int th = kGramWarps * 32;
     switch (nb) {
-      case 1: AM_LAUNCH(AM_STAGE_GRAM, s, k_gram_tile<1><<<gg, th, 0, s>>>(p, w, pass)); break;
-      case 2: AM_LAUNCH(AM_STAGE_GRAM, s, k_gram_tile<2><<<gg, th, 0, s>>>(p, w, pass)); break;
-      case 4: AM_LAUNCH(AM_STAGE_GRAM, s, k_gram_tile<4><<<gg, th, 0, s>>>(p, w, pass)); break;
-      case 8: AM_LAUNCH(AM_STAGE_GRAM, s, k_gram_tile<8><<<gg, th, 0, s>>>(p, w, pass)); break;
-      default: AM_LAUNCH(AM_STAGE_GRAM, s, k_gram_tile<16><<<gg, th, 0, s>>>(p, w, pass)); break;
+      case 1: AM_LAUNCH(AM_STAGE_GRAM, s, launch_chained(k_gram_tile<1>, gg, dim3(th), 0, s, p, w, pass)); break;
+      case 2: AM_LAUNCH(AM_STAGE_GRAM, s, launch_chained(k_gram_tile<2>, gg, dim3(th), 0, s, p, w, pass)); break;
+      case 4: AM_LAUNCH(AM_STAGE_GRAM, s, launch_chained(k_gram_tile<4>, gg, dim3(th), 0, s, p, w, pass)); break;
+      case 8: AM_LAUNCH(AM_STAGE_GRAM, s, launch_chained(k_gram_tile<8>, gg, dim3(th), 0, s, p, w, pass)); break;
+      default: AM_LAUNCH(AM_STAGE_GRAM, s, launch_chained(k_gram_tile<16>, gg, dim3(th), 0, s, p, w, pass)); break;
     }
   } else {
     dim3 gg(s1max, active);
@@ -1231,9 +1237,9 @@ cudaError_t launch_omp_pass(const Problem& p, const Work& w, int pass, int activ
   int lcap;
   size_t sm = nnls_smem_bytes(p.max_t, &lcap);
   cudaFuncSetAttribute(k_nnls, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemCap);
-  AM_LAUNCH(AM_STAGE_NNLS, s, k_nnls<<<active, kNnlsThreads, sm, s>>>(p, w, pass, lcap));
+  AM_LAUNCH(AM_STAGE_NNLS, s, launch_chained(k_nnls, dim3(active), dim3(kNnlsThreads), sm, s, p, w, pass, lcap));
   dim3 gr(resid_blocks(p), active);
-  AM_LAUNCH(AM_STAGE_RESID, s, k_resid<<<gr, kResidThreads, 0, s>>>(p, w, pass));
+  AM_LAUNCH(AM_STAGE_RESID, s, launch_chained(k_resid, gr, dim3(kResidThreads), 0, s, p, w, pass));
   return cudaGetLastError();
 }
 
