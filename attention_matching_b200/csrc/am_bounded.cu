@@ -162,14 +162,6 @@ __device__ void stage_list(const Problem& p, const Work& w, int h, int lo, int h
   __syncthreads();
 }
 
-// Keeps the better of (k, j, pos) and the lane `o` away, in pick order.
-__device__ __forceinline__ void shfl_best(uint64_t& k, int& j, int& pos, int o) {
-  const uint64_t k2 = __shfl_xor_sync(0xffffffffu, k, o);
-  const int j2 = __shfl_xor_sync(0xffffffffu, j, o);
-  const int p2 = __shfl_xor_sync(0xffffffffu, pos, o);
-  if (p2 >= 0 && (pos < 0 || before(k2, j2, k, j))) { k = k2; j = j2; pos = p2; }
-}
-
 // The best live entry (index not INT_MAX) of keys/idx at e = first, first +
 // stride, ... below n: (key, index, position), position -1 when none.
 __device__ __forceinline__ void lane_best(const uint64_t* keys, const int* idx, int first, int stride, int n,
@@ -186,7 +178,9 @@ __device__ __forceinline__ void lane_best(const uint64_t* keys, const int* idx, 
 // kk rounds of a warp argmax over one warp's entries (lane l owns positions
 // first + l·… as laid out by lane_best): round k's winner goes to outk[k] /
 // outj[k] (index INT_MAX once nothing is left) and its entry is marked used;
-// only the winning lane rescans.  One warp.
+// only the winning lane rescans.  A round is three warp reductions in pick
+// order: the largest high word of the key, the largest low word among those,
+// the lowest key index among those (entries carry distinct indices).  One warp.
 __device__ __forceinline__ void warp_top(uint64_t* keys, int* idx, int first, int stride, int n, int kk,
                                          uint64_t* outk, int* outj) {
   const int lane = threadIdx.x & 31;
@@ -194,11 +188,19 @@ __device__ __forceinline__ void warp_top(uint64_t* keys, int* idx, int first, in
   int bj, bp;
   lane_best(keys, idx, first, stride, n, bk, bj, bp);
   for (int k = 0; k < kk; ++k) {
-    uint64_t wk = bk;
-    int wj = bj, wp = bp;
-    for (int o = 16; o; o >>= 1) shfl_best(wk, wj, wp, o);
-    if (lane == 0) { outk[k] = wk; outj[k] = wp >= 0 ? wj : INT_MAX; }
-    if (wp >= 0 && wp == bp) {   // the owner of the winning entry takes its next best
+    const bool live = bp >= 0;
+    const unsigned kh = live ? (unsigned)(bk >> 32) : 0u;
+    const unsigned kl = live ? (unsigned)bk : 0u;
+    const unsigned jj = live ? (unsigned)bj : 0x7fffffffu;
+    const unsigned m1 = __reduce_max_sync(0xffffffffu, kh);
+    const unsigned m2 = __reduce_max_sync(0xffffffffu, kh == m1 ? kl : 0u);
+    const bool top = kh == m1 && kl == m2;
+    const unsigned m3 = __reduce_min_sync(0xffffffffu, top ? jj : 0xffffffffu);
+    if (lane == 0) {
+      outk[k] = ((uint64_t)m1 << 32) | m2;
+      outj[k] = (int)m3;   // INT_MAX when no lane had an entry left
+    }
+    if (live && top && jj == m3) {   // the owner of the winning entry takes its next best
       idx[bp] = INT_MAX;
       lane_best(keys, idx, first, stride, n, bk, bj, bp);
     }
@@ -226,15 +228,26 @@ __device__ __forceinline__ double key_value(uint64_t k) {
 
 // Number of leading entries of kn[0, n) not below thr, the entries being in
 // descending order: a sampled search, one sample per thread and level (two
-// levels for n up to blockDim², one round trip each).  All threads.
-__device__ int prefix_not_below(const float* kn, int n, float thr) {
+// levels for n up to blockDim², one round trip each).  The first level's
+// sample, kn[min(tid·step0, n − 1)] with step0 = ceil(n / blockDim), does not
+// depend on thr: the caller loads it ahead (first_sample) and passes it in.
+// All threads.
+__device__ __forceinline__ float first_sample(const float* kn, int n) {
+  const int step = (n + (int)blockDim.x - 1) / (int)blockDim.x;
+  return kn[min((int)threadIdx.x * step, n - 1)];
+}
+
+__device__ int prefix_not_below(const float* kn, int n, float thr, float sample0) {
   int lo = 0, hi = n;   // kn[i] >= thr known for i < lo, kn[i] < thr for i >= hi
+  bool first = true;
   while (lo < hi) {
     const int span = hi - lo;
     const int step = (span + (int)blockDim.x - 1) / (int)blockDim.x;
     const int samples = (span + step - 1) / step;
     const int i = lo + (int)threadIdx.x * step;
-    const bool ok = (int)threadIdx.x < samples && !(kn[i] < thr);
+    const bool in = (int)threadIdx.x < samples;
+    const bool ok = in && !((first ? sample0 : kn[i]) < thr);
+    first = false;
     const int c = __syncthreads_count(ok);   // samples 0 .. c-1 pass
     const int nlo = c > 0 ? lo + (c - 1) * step + 1 : lo;
     hi = c < samples ? lo + c * step : hi;
@@ -255,8 +268,12 @@ __device__ void theta_and_prefix(const Problem& p, const Work& w, int h, int pas
   const int nrb = resid_blocks(p);
   const double rr_mine = pass == 0 ? (threadIdx.x == 0 ? w.mm[h] : 0.0)
                                    : ((int)threadIdx.x < nrb ? w.rr_part[(int64_t)h * kRedBlocks + threadIdx.x] : 0.0);
+  // every load that does not depend on θ goes out first: the list count, the
+  // list itself up to p0 (entries past the count are left over and ignored),
+  // the first level of the prefix search
   const int staged = __ldcg(w.ccount + h);   // <= p0 <= kSelCap: the probe's unselected keys
-  stage_list(p, w, h, 0, staged, 0, S);
+  const float sample0 = first_sample(w.knorm + (int64_t)h * p.T, p.T);
+  stage_list(p, w, h, 0, p0, 0, S);
   select_top(S, staged, kk);
   const double rn = sqrt(block_sum(rr_mine, S.red));
   const int jt = S.outj[kk - 1];
@@ -265,7 +282,7 @@ __device__ void theta_and_prefix(const Problem& p, const Work& w, int h, int pas
   // the bound cannot help (θ <= 0, a zero or non-finite residual)
   const bool useful = theta > 0.0 && rn > 0.0 && rn < INFINITY;
   const float thr = useful ? (float)(theta / (rn * (1.0 + kBoundMargin))) : 0.f;
-  const int L = useful ? prefix_not_below(w.knorm + (int64_t)h * p.T, p.T, thr) : p.T;
+  const int L = useful ? prefix_not_below(w.knorm + (int64_t)h * p.T, p.T, thr, sample0) : p.T;
   const bool done = L <= p0;
   if (threadIdx.x == 0) {
     w.cprefix[h] = L;   // the next pass sizes its probe by it
@@ -341,12 +358,13 @@ __device__ void pick_from_prefix(const Problem& p, const Work& w, int h, int s0,
 // ------------------------------------------------------------ exact rows --
 // c_j = Σ_i r_i Φ_ij for the unselected keys at sorted positions [0, P0)
 // (which = 0) or [P0, L) (which = 1), in fp64 sums of exact fp32 products.
-// Four warps share a key, each summing a quarter of the queries with four
+// Four warps share a key, each summing a quarter of the queries with eight
 // columns per lane in flight; the quarters are added in a fixed order.  The
 // last block of a head to finish (counted with an atomic) then takes the
 // selection step: θ and L after the probe rows, the picks after the rest.
 constexpr int kRowSplit = 4;                           // warps per key
 constexpr int kRowsPerBlock = kSelThreads / 32 / kRowSplit;   // keys per block
+constexpr int kRowLoads = 8;                           // float4 columns per lane in flight
 
 __global__ void __launch_bounds__(kSelThreads) k_rows(Problem p, Work w, int pass, int which) {
   chain_wait();
@@ -381,16 +399,16 @@ __global__ void __launch_bounds__(kSelThreads) k_rows(Problem p, Work w, int pas
     double a[4] = {0.0, 0.0, 0.0, 0.0};
     if (on) {
       const float4* row = reinterpret_cast<const float4*>(w.phiT + ((int64_t)h * p.T + j) * p.ldn);
-      for (int i0 = c0 + lane; i0 < c1; i0 += 32 * 4) {
-        float4 x[4], y[4];
+      for (int i0 = c0 + lane; i0 < c1; i0 += 32 * kRowLoads) {
+        float4 x[kRowLoads], y[kRowLoads];
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
+        for (int u = 0; u < kRowLoads; ++u) {
           const int i = i0 + 32 * u;
           x[u] = i < c1 ? __ldcs(row + i) : make_float4(0.f, 0.f, 0.f, 0.f);
           y[u] = i < c1 ? __ldg(r4 + i) : make_float4(0.f, 0.f, 0.f, 0.f);
         }
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
+        for (int u = 0; u < kRowLoads; ++u) {
           a[0] = fma((double)x[u].x, (double)y[u].x, a[0]);
           a[1] = fma((double)x[u].y, (double)y[u].y, a[1]);
           a[2] = fma((double)x[u].z, (double)y[u].z, a[2]);
