@@ -846,9 +846,11 @@ __global__ void __launch_bounds__(kNnlsThreads) k_nnls(Problem p, Work w, int pa
       if (warp == 0) {
         int failed = 0;
         const bool wide = k <= 32;
+        const double dg = wide && lane < k ? diag(add[lane]) : 0.0;   // G_ll of new row `lane`
         for (int f = 0; f < k; ++f) {
           const double piv = L[tri(np + f, np + f)];
-          if (!(piv > 1e-13 * diag(add[f]))) {
+          const double gff = wide ? __shfl_sync(0xffffffffu, dg, f) : diag(add[f]);
+          if (!(piv > 1e-13 * gff)) {
             if (lane == 0) blocked[add[f]] = 1;
             failed = 1;
             break;
@@ -916,6 +918,7 @@ __global__ void __launch_bounds__(kNnlsThreads) k_nnls(Problem p, Work w, int pa
     for (int ci = warp; ci < nc; ci += nw) {
       const int l = cand[ci];
       const double* Gl = G + (int64_t)l * t;
+      const double dl = lane == 0 ? diag(l) : 0.0, bl = lane == 0 ? b[l] : 0.0;   // in flight with the row
       double a4[4] = {0.0, 0.0, 0.0, 0.0};
       for (int q0 = lane; q0 < np; q0 += 128) {
 #pragma unroll
@@ -925,10 +928,7 @@ __global__ void __launch_bounds__(kNnlsThreads) k_nnls(Problem p, Work w, int pa
         }
       }
       const double acc = warp_sum((a4[0] + a4[1]) + (a4[2] + a4[3]));
-      if (lane == 0) {
-        const double dl = diag(l);
-        g[l] = dl > 0.0 ? (b[l] - acc) / (sqrt(dl) * mnorm) : -INFINITY;
-      }
+      if (lane == 0) g[l] = dl > 0.0 ? (bl - acc) / (sqrt(dl) * mnorm) : -INFINITY;
     }
     __syncthreads();
     if (warp == 0) {
@@ -1097,10 +1097,10 @@ __global__ void __launch_bounds__(kNnlsThreads) k_nnls(Problem p, Work w, int pa
 
 // ------------------------------------------------------------ residual ----
 // r = m − Φ_S w over all current picks; fp64 sums, fp32 store; partial ‖r‖².
-// A block covers 32 float4 positions (128 queries) with four thread groups,
-// group g taking picks g, g + 4, ...; the groups' sums are combined in a
-// fixed order, so the result is deterministic.
-constexpr int kResidGroups = 4;    // pick groups per position
+// A block covers 32 float4 positions (128 queries) with sixteen thread
+// groups, group g taking picks g, g + 16, ... (eight in flight); the groups'
+// sums are combined in a fixed order, so the result is deterministic.
+constexpr int kResidGroups = 16;   // pick groups per position
 constexpr int kResidThreads = kResidPos * kResidGroups;
 constexpr int kResidChunk = 512;   // picks staged in shared memory at a time
 
