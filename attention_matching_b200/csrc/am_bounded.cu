@@ -24,9 +24,11 @@
 // fp32 one is larger by at most 2^-24 relative) and the rounding of the fp64
 // sums and norms (relative error below n·2^-53 for the sums, a few ulp for
 // the norms); the fp32 copies of the norms and of the cut only move it
-// outward (rounding to nearest is monotone).  A selection is a warp-level
-// top-kk (kk rounds of shuffle argmax per warp over shared-memory
-// candidates) followed by the same over the warps' winners.
+// outward (rounding to nearest is monotone).  The row blocks append every
+// evaluated key (order key of c_j, key index) to a per-head list; a
+// selection stages that list in shared memory and takes a warp-level top-kk
+// (kk rounds of three warp reductions per warp) followed by the same over the
+// warps' winners.
 #include "am_internal.cuh"
 #include "am_profile.cuh"
 #include "am_linalg.cuh"

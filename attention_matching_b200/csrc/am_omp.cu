@@ -8,12 +8,16 @@
 //
 // One "pass" covers R rounds of k picks: the residual does not change
 // between refits, so those R rounds take the next k·R keys of one
-// correlation vector.  A pass is five launches over the active heads:
-//   k_corr    c = Φᵀ r                 (HBM-bound GEMV over key-major Φᵀ)
-//   k_select  top-(k·R) unselected keys, ties to the lowest index
-//   k_gram    new rows/columns of G = Φ_SᵀΦ_S and b = Φ_Sᵀm (fp64 sums)
+// correlation vector.  A pass is four or five launches over the active heads:
+//   correlation and selection of the top-(k·R) unselected keys (ties to the
+//             lowest index): k_rows twice (the default bounded mode,
+//             am_bounded.cu), or k_corr / k_corr_tc (c = Φᵀ r streamed or
+//             recomputed) then k_select
+//   k_gram_tile (k_gram past 16 picks per pass)  new rows/columns of
+//             G = Φ_SᵀΦ_S and b = Φ_Sᵀm (fp64 sums)
 //   k_nnls    active-set NNLS on (G, b), warm-started from the last refit
-//   k_resid   r = m − Φ_S w (fp64 sums, stored fp32)
+//   k_resid   r = m − Φ_S w (fp64 sums, stored fp32) and partials of ‖r‖²
+// The pass kernels are chained with programmatic dependent launch.
 #include "am_internal.cuh"
 #include "am_async.cuh"
 #include "am_profile.cuh"

@@ -10,7 +10,9 @@
 //               packed indices, β and C_k = K[S]
 //   k_design    A_il = Φ_{i,S_l} w_l / Σ_l' Φ_{i,S_l'} w_l'  (key-major [t][ldn])
 //   k_normal    AᵀA and AᵀY with fp64 sums of fp32 products
-//   k_solve     λ = ridge·tr(AᵀA)/t, Cholesky of AᵀA + λI, C_v = (AᵀA + λI)⁻¹AᵀY
+//   k_chol      λ = ridge·tr(AᵀA)/t, tiled Cholesky of AᵀA + λI (inverses of the
+//               32×32 diagonal tiles kept)
+//   k_trsm      C_v = (AᵀA + λI)⁻¹AᵀY by blocked forward and backward solves
 #include "am_internal.cuh"
 #include "am_profile.cuh"
 #include "am_linalg.cuh"
