@@ -20,6 +20,7 @@ __all__ = ["AmError", "AmOpts", "lib", "library_path", "workspace_size", "compac
 
 BF16, FP32 = 0, 1
 CORR_AUTO, CORR_STORED_FP32, CORR_STORED_BF16, CORR_RECOMPUTE, CORR_BOUNDED = 0, 1, 2, 3, 4
+SELECT_OMP, SELECT_HIGHEST = 0, 1   # am_select_mode_t
 STATUS = {
     0: "AM_OK", 1: "AM_ERR_INVALID_ARG", 2: "AM_ERR_BUDGET", 3: "AM_ERR_WORKSPACE",
     4: "AM_ERR_NONFINITE", 5: "AM_ERR_CUDA", 6: "AM_ERR_TIMEOUT", 7: "AM_ERR_UNSUPPORTED",
@@ -65,6 +66,7 @@ class AmOpts(ctypes.Structure):
         ("shift_out", ctypes.c_void_p),
         ("residual_out", ctypes.c_void_p),
         ("w_out", ctypes.c_void_p),
+        ("select_mode", ctypes.c_int32),
     ]
 
 
@@ -116,7 +118,7 @@ def _i32_array(vals: Sequence[int]):
 
 def make_opts(dtype: int = BF16, topk: int = 1, refit_every: int = 1, scale: float = 0.0,
               ridge: float = 1e-6, w_floor_rel: float = 1e-12, nnls_max_iter: int = 0,
-              corr_mode: int = CORR_AUTO) -> AmOpts:
+              corr_mode: int = CORR_AUTO, select_mode: int = 0) -> AmOpts:
     o = AmOpts()
     rc = lib().am_default_opts(ctypes.byref(o))
     if rc:
@@ -124,6 +126,7 @@ def make_opts(dtype: int = BF16, topk: int = 1, refit_every: int = 1, scale: flo
     o.in_dtype, o.topk, o.refit_every, o.nnls_max_iter = dtype, topk, refit_every, nnls_max_iter
     o.scale, o.ridge, o.w_floor_rel = scale, ridge, w_floor_rel
     o.corr_mode = corr_mode
+    o.select_mode = select_mode
     return o
 
 
@@ -137,14 +140,15 @@ def workspace_size(n: int, T: int, d: int, budgets: Sequence[int], opts: AmOpts)
 
 
 def features(out: Dict, n: int, T: int, d: int, budgets: Sequence[int], topk: int = 1,
-             refit_every: int = 1, dtype: int = BF16, corr_mode: int = CORR_AUTO) -> Dict:
+             refit_every: int = 1, dtype: int = BF16, corr_mode: int = CORR_AUTO,
+             select_mode: int = SELECT_OMP) -> Dict:
     """Views of the intermediate features a finished call left in its
     workspace: phiT [H, T, ldn] fp32, mass [H, ldn] fp64, target [H, n, d]
     fp32, shift [H] fp32, weights [Σt] fp64 (last NNLS refit, pick order)
     and resid [H, ldn] fp32 (torch tensors sharing the workspace memory)."""
     import torch
     H = len(budgets)
-    opts = make_opts(dtype, topk, refit_every, corr_mode=corr_mode)
+    opts = make_opts(dtype, topk, refit_every, corr_mode=corr_mode, select_mode=select_mode)
     v = AmWorkspaceView()
     rc = lib().am_workspace_view(n, T, d, H, _i32_array(budgets), ctypes.byref(opts), ctypes.byref(v))
     if rc:
@@ -175,14 +179,17 @@ def _ptr(t) -> Optional[int]:
 def compact_heads(Q, K, V, budgets: Sequence[int], topk: int = 1, refit_every: int = 1,
                   shift=None, key_bias=None, ridge: float = 1e-6, w_floor_rel: float = 1e-12,
                   scale: float = 0.0, nnls_max_iter: int = 0, workspace=None, trace: bool = False,
-                  stream=None, check: bool = True, corr_mode: int = CORR_AUTO) -> Dict:
+                  stream=None, check: bool = True, corr_mode: int = CORR_AUTO,
+                  select_mode: int = SELECT_OMP) -> Dict:
     """Compact H heads on the GPU.
 
     Q [H, n, d], K [H, T, d], V [H, T, d]: contiguous tensors, bf16 or fp32,
     all on the current CUDA device or all on the host (then copied in, and the
     outputs copied back to the host).
     budgets: H ints in [1, T].  shift [H] fp32 and key_bias [H, T] fp32 are
-    optional CUDA tensors.  Returns a dict of CUDA tensors in the packed
+    optional CUDA tensors.  select_mode SELECT_HIGHEST keeps each head's t
+    keys of largest total attention instead of the OMP picks (topk,
+    refit_every and corr_mode are then ignored).  Returns a dict of CUDA tensors in the packed
     varlen layout (C_k, beta, C_v, indices, cu_t) plus, with ``trace``, the
     pick order, pick correlations, shift used, mass residual and weights.
     """
@@ -205,7 +212,7 @@ def compact_heads(Q, K, V, budgets: Sequence[int], topk: int = 1, refit_every: i
             raise ValueError("inputs must be contiguous")
     dt = BF16 if Q.dtype == torch.bfloat16 else FP32
     dev = Q.device
-    opts = make_opts(dt, topk, refit_every, scale, ridge, w_floor_rel, nnls_max_iter, corr_mode)
+    opts = make_opts(dt, topk, refit_every, scale, ridge, w_floor_rel, nnls_max_iter, corr_mode, select_mode)
     if shift is not None:
         shift = shift.to(device=dev, dtype=torch.float32).contiguous()
         opts.shift = shift.data_ptr()

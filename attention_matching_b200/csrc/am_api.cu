@@ -31,7 +31,7 @@ struct Layout {
   size_t picks, pick_corr, plist, sorted_slot;
   size_t bvec, w, w_eff, ycache;
   size_t G, L, AtA, A, AtY, nrm_part;
-  size_t cnorm, cnpart, rnorm, clist, clj, ccount, korder, knorm, ksort, cprefix, cdone, cprobe, rows_eval, gpart, gcount, rcount,
+  size_t cnorm, cnpart, rnorm, clist, clj, ccount, inv_m, korder, knorm, ksort, cprefix, cdone, cprobe, rows_eval, gpart, gcount, rcount,
       dinv;
   size_t total;
   size_t tables_bytes;
@@ -50,6 +50,11 @@ struct Tables {
   int max_t = 0;
   int64_t sum_t = 0, sum_t2 = 0;
 };
+
+// The feature pass also writes a bf16 copy of Φᵀ for the bf16 correlation mode.
+bool bf16_copy(const am_opts_t* o) {
+  return o->corr_mode == AM_CORR_STORED_BF16 && o->select_mode == AM_SELECT_OMP;
+}
 
 Layout plan(int n, int T, int d, int H, int64_t sum_t, int64_t sum_t2, bool corr_bf16) {
   Layout L{};
@@ -91,6 +96,7 @@ Layout plan(int n, int T, int d, int H, int64_t sum_t, int64_t sum_t2, bool corr
   L.clist = take((size_t)H * T * 8);
   L.clj = take((size_t)H * T * 4);
   L.ccount = take((size_t)H * 4);
+  L.inv_m = take((size_t)H * ldn * 8);
   L.korder = take((size_t)H * T * 4);
   L.knorm = take((size_t)H * T * 4);
   size_t t2 = 1;
@@ -116,18 +122,21 @@ am_status_t check_shape(int n, int T, int d, int H, const int32_t* budgets, cons
   if (n < 1 || T < 1 || d < 1 || H < 1) return AM_ERR_INVALID_ARG;
   if (opts->in_dtype != AM_BF16 && opts->in_dtype != AM_FP32) return AM_ERR_INVALID_ARG;
   if (d > 256) return AM_ERR_UNSUPPORTED;
-  if (opts->topk < 1 || opts->refit_every < 1) return AM_ERR_INVALID_ARG;
-  if ((int64_t)opts->topk * opts->refit_every > kMaxPicksPerPass) return AM_ERR_UNSUPPORTED;
+  if (opts->select_mode != AM_SELECT_OMP && opts->select_mode != AM_SELECT_HIGHEST) return AM_ERR_INVALID_ARG;
+  const bool highest = opts->select_mode == AM_SELECT_HIGHEST;
+  if (!highest && (opts->topk < 1 || opts->refit_every < 1)) return AM_ERR_INVALID_ARG;
+  if (!highest && (int64_t)opts->topk * opts->refit_every > kMaxPicksPerPass) return AM_ERR_UNSUPPORTED;
+  if (highest && T > kSortSmemKeys) return AM_ERR_UNSUPPORTED;
   if (opts->nnls_max_iter < 0) return AM_ERR_INVALID_ARG;
   if (!(opts->ridge >= 0.f) || !isfinite(opts->ridge)) return AM_ERR_INVALID_ARG;
   if (!(opts->w_floor_rel > 0.f) || !(opts->w_floor_rel < 1.f)) return AM_ERR_INVALID_ARG;
   if (!isfinite(opts->scale)) return AM_ERR_INVALID_ARG;
   if (opts->corr_mode < AM_CORR_AUTO || opts->corr_mode > AM_CORR_BOUNDED) return AM_ERR_INVALID_ARG;
-  if (opts->corr_mode == AM_CORR_RECOMPUTE && !(opts->in_dtype == AM_BF16 && (d == 64 || d == 128)))
+  if (!highest && opts->corr_mode == AM_CORR_RECOMPUTE && !(opts->in_dtype == AM_BF16 && (d == 64 || d == 128)))
     return AM_ERR_UNSUPPORTED;
   if ((int64_t)n * d > (1ll << 31) || (int64_t)T * round_up(n, 32) > (1ll << 40))
     return AM_ERR_UNSUPPORTED;
-  const int kR = opts->topk * opts->refit_every;
+  const int kR = highest ? kHighestChunk : opts->topk * opts->refit_every;
   tb->t.assign(budgets, budgets + H);
   tb->cu_t.assign(H + 1, 0);
   tb->cu_t2.assign(H + 1, 0);
@@ -210,6 +219,7 @@ Work bind(const Layout& L, char* base, bool corr_bf16) {
   w.clist = reinterpret_cast<uint64_t*>(base + L.clist);
   w.clj = reinterpret_cast<int32_t*>(base + L.clj);
   w.ccount = reinterpret_cast<int32_t*>(base + L.ccount);
+  w.inv_m = reinterpret_cast<double*>(base + L.inv_m);
   w.korder = reinterpret_cast<int32_t*>(base + L.korder);
   w.knorm = reinterpret_cast<float*>(base + L.knorm);
   w.ksort = reinterpret_cast<uint64_t*>(base + L.ksort);
@@ -262,17 +272,19 @@ Problem make_problem(int n, int T, int d, int H, const am_opts_t* o, const Table
   p.ldn = round_up(n, 32);
   p.in_dtype = o->in_dtype;
   p.scale = o->scale > 0.f ? o->scale : (float)(1.0 / sqrt((double)d));
-  p.topk = o->topk;
-  p.refit_every = o->refit_every;
-  p.kR = o->topk * o->refit_every;
+  p.select_highest = o->select_mode == AM_SELECT_HIGHEST;
+  p.topk = p.select_highest ? kHighestChunk : o->topk;
+  p.refit_every = p.select_highest ? 1 : o->refit_every;
+  p.kR = p.topk * p.refit_every;
   p.nnls_max_iter = o->nnls_max_iter;
   p.ridge = o->ridge;
   p.w_floor_rel = o->w_floor_rel;
   p.max_t = tb.max_t;
   p.has_bias = o->key_bias != nullptr;
-  p.corr_bf16 = o->corr_mode == AM_CORR_STORED_BF16;
+  p.corr_bf16 = bf16_copy(o);
   p.corr_recompute = o->corr_mode == AM_CORR_RECOMPUTE;
-  p.corr_bounded = o->corr_mode == AM_CORR_BOUNDED || o->corr_mode == AM_CORR_AUTO;
+  p.corr_bounded = !p.select_highest && (o->corr_mode == AM_CORR_BOUNDED || o->corr_mode == AM_CORR_AUTO);
+  if (p.select_highest) p.corr_recompute = false;
   return p;
 }
 
@@ -307,7 +319,7 @@ am_status_t am_workspace_size(int32_t n, int32_t T, int32_t d, int32_t num_heads
   Tables tb;
   am_status_t st = check_shape(n, T, d, num_heads, budgets, opts, &tb);
   if (st != AM_OK) return st;
-  *bytes = plan(n, T, d, num_heads, tb.sum_t, tb.sum_t2, opts->corr_mode == AM_CORR_STORED_BF16).total;
+  *bytes = plan(n, T, d, num_heads, tb.sum_t, tb.sum_t2, bf16_copy(opts)).total;
   return AM_OK;
 }
 
@@ -317,7 +329,7 @@ am_status_t am_workspace_view(int32_t n, int32_t T, int32_t d, int32_t num_heads
   Tables tb;
   am_status_t st = check_shape(n, T, d, num_heads, budgets, opts, &tb);
   if (st != AM_OK) return st;
-  const Layout L = plan(n, T, d, num_heads, tb.sum_t, tb.sum_t2, opts->corr_mode == AM_CORR_STORED_BF16);
+  const Layout L = plan(n, T, d, num_heads, tb.sum_t, tb.sum_t2, bf16_copy(opts));
   view->phiT = L.phiT;
   view->mass = L.m;
   view->target = L.Y;
@@ -358,12 +370,12 @@ am_status_t compact_heads_impl(const void* Q, const void* K, const void* V, int3
   for (int h = 0; h <= H; ++h)
     if (out_offsets[h] != tb.cu_t[h]) return AM_ERR_INVALID_ARG;
   if (!workspace || ((uintptr_t)workspace % kAlign) != 0) return AM_ERR_WORKSPACE;
-  const Layout L = plan(n, T, d, H, tb.sum_t, tb.sum_t2, opts->corr_mode == AM_CORR_STORED_BF16);
+  const Layout L = plan(n, T, d, H, tb.sum_t, tb.sum_t2, bf16_copy(opts));
   if (workspace_bytes < L.total) return AM_ERR_WORKSPACE;
 
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   char* base = reinterpret_cast<char*>(workspace);
-  Work w = bind(L, base, opts->corr_mode == AM_CORR_STORED_BF16);
+  Work w = bind(L, base, bf16_copy(opts));
   w.nrm_ata = tb.sum_t2;
   w.nrm_stride = tb.sum_t2 + tb.sum_t * d;
   std::vector<unsigned char> host_tables;
@@ -406,6 +418,7 @@ am_status_t compact_heads_impl(const void* Q, const void* K, const void* V, int3
   AM_TRY(cudaMemsetAsync(w.rcount, 0, (size_t)H * 4, s));
   AM_TRY(cudaMemsetAsync(w.cprefix, 0, (size_t)H * 4, s));
   AM_TRY(cudaMemsetAsync(w.ccount, 0, (size_t)H * 4, s));
+  if (p.select_highest) AM_TRY(launch_select_highest(p, w, s));
   const CorrInputs cin{Q, K, opts->key_bias};
   if (G == 1) {
     for (int pass = 0; pass < (int)tb.active.size(); ++pass)

@@ -442,6 +442,115 @@ __global__ void __launch_bounds__(kSelThreads) k_rows(Problem p, Work w, int pas
   if (threadIdx.x == 0) w.rcount[h] = 0;
 }
 
+// ------------------------------------------------- highest attention --
+// AM-Highest ("Fast KV Compaction via Attention Matching": zhichai.net/en
+// summary, "Method Family and Trade-offs"; youleyou.com rewrite, the
+// highest-attention keys): each head keeps the t keys with the largest total
+// attention over its reference queries, score_j = Σ_i Φ_ij / m_i (query i's
+// softmax probability of key j; the shift cancels), ties to the lower key.
+
+// 1 / m_i per query in fp64, 0 for a query without mass or past n.
+__global__ void __launch_bounds__(256) k_inv_m(Problem p, Work w) {
+  const int h = blockIdx.y;
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= p.ldn) return;
+  const double m = w.m[(int64_t)h * p.ldn + i];
+  w.inv_m[(int64_t)h * p.ldn + i] = (i < p.n && m > 0.0) ? 1.0 / m : 0.0;
+}
+
+// score_j for every key, into w.cnorm [H][T]: fp64 sums of the stored fp32
+// features times 1 / m_i; four warps per key, a quarter of the queries each,
+// eight float4 columns per lane in flight, the quarters added in a fixed order.
+__global__ void __launch_bounds__(kSelThreads) k_score(Problem p, Work w) {
+  __shared__ double part[kRowsPerBlock][kRowSplit];
+  const int h = blockIdx.y;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int slot = warp / kRowSplit, quarter = warp % kRowSplit;
+  const double2* im2 = reinterpret_cast<const double2*>(w.inv_m + (int64_t)h * p.ldn);
+  const int n4 = p.ldn >> 2;
+  const int per = (n4 + kRowSplit - 1) / kRowSplit;
+  const int c0 = quarter * per, c1 = min(n4, c0 + per);
+  for (int j0 = blockIdx.x * kRowsPerBlock; j0 < p.T; j0 += gridDim.x * kRowsPerBlock) {
+    const int j = j0 + slot;
+    const bool on = j < p.T;
+    double a[4] = {0.0, 0.0, 0.0, 0.0};
+    if (on) {
+      const float4* row = reinterpret_cast<const float4*>(w.phiT + ((int64_t)h * p.T + j) * p.ldn);
+      for (int i0 = c0 + lane; i0 < c1; i0 += 32 * kRowLoads) {
+        float4 x[kRowLoads];
+#pragma unroll
+        for (int u = 0; u < kRowLoads; ++u) {
+          const int i = i0 + 32 * u;
+          x[u] = i < c1 ? __ldcs(row + i) : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+#pragma unroll
+        for (int u = 0; u < kRowLoads; ++u) {
+          const int i = i0 + 32 * u;
+          if (i < c1) {
+            const double2 lo = __ldg(im2 + 2 * i), hi = __ldg(im2 + 2 * i + 1);
+            a[0] = fma((double)x[u].x, lo.x, a[0]);
+            a[1] = fma((double)x[u].y, lo.y, a[1]);
+            a[2] = fma((double)x[u].z, hi.x, a[2]);
+            a[3] = fma((double)x[u].w, hi.y, a[3]);
+          }
+        }
+      }
+    }
+    const double c = warp_sum((a[0] + a[1]) + (a[2] + a[3]));
+    if (lane == 0) part[slot][quarter] = c;
+    __syncthreads();
+    if (on && quarter == 0 && lane == 0)
+      w.cnorm[(int64_t)h * p.T + j] = (part[slot][0] + part[slot][1]) + (part[slot][2] + part[slot][3]);
+    __syncthreads();
+  }
+}
+
+// Each head's keys in pick order (larger score first, ties to the lower key):
+// a bitonic sort of (order key, key index) pairs in shared memory, one block
+// per head; the first t become the head's picks, in that order.
+__global__ void __launch_bounds__(kBoundThreads) k_pick_highest(Problem p, Work w) {
+  extern __shared__ __align__(16) unsigned char smem[];
+  const int h = blockIdx.x;
+  int n2 = 1;
+  while (n2 < p.T) n2 <<= 1;
+  uint64_t* key = reinterpret_cast<uint64_t*>(smem);
+  int* idx = reinterpret_cast<int*>(key + n2);
+  const double* sc = w.cnorm + (int64_t)h * p.T;
+  for (int i = threadIdx.x; i < n2; i += blockDim.x) {
+    key[i] = i < p.T ? order_key(sc[i]) : 0ull;
+    idx[i] = i < p.T ? i : INT_MAX;
+  }
+  __syncthreads();
+  for (int k = 2; k <= n2; k <<= 1) {
+    for (int jj = k >> 1; jj > 0; jj >>= 1) {
+      for (int i = threadIdx.x; i < n2; i += blockDim.x) {
+        const int l = i ^ jj;
+        if (l > i) {
+          const uint64_t a = key[i], b = key[l];
+          const int ja = idx[i], jb = idx[l];
+          // segments with bit k clear end in pick order, the others reversed
+          const bool swap = (i & k) == 0 ? before(b, jb, a, ja) : before(a, ja, b, jb);
+          if (swap) {
+            key[i] = b; key[l] = a;
+            idx[i] = jb; idx[l] = ja;
+          }
+        }
+      }
+      __syncthreads();
+    }
+  }
+  const int t = w.t[h];
+  const int64_t base = w.cu_t[h];
+  uint8_t* sel = w.sel + (int64_t)h * p.T;
+  for (int l = threadIdx.x; l < t; l += blockDim.x) {
+    const int j = idx[l];   // t <= T: a real key
+    w.picks[base + l] = j;
+    w.pick_corr[base + l] = (float)key_value(key[l]);
+    sel[j] = 1;
+  }
+  if (threadIdx.x == 0) w.rows_eval[h] = (unsigned long long)p.T;
+}
+
 int rows_ctas_per_head(int active) {
   const int c = (8 * 148 + active - 1) / active;
   return c < 1 ? 1 : (c > 256 ? 256 : c);
@@ -469,6 +578,20 @@ cudaError_t launch_corr_bounded(const Problem& p, const Work& w, int pass, int a
   dim3 gr(rows_ctas_per_head(active), active);
   AM_LAUNCH(AM_STAGE_ROWS, s, launch_chained(k_rows, gr, dim3(kSelThreads), sel_smem, s, p, w, pass, 0));
   AM_LAUNCH(AM_STAGE_ROWS, s, launch_chained(k_rows, gr, dim3(kSelThreads), sel_smem, s, p, w, pass, 1));
+  return cudaGetLastError();
+}
+
+cudaError_t launch_select_highest(const Problem& p, const Work& w, cudaStream_t s) {
+  dim3 gi((p.ldn + 255) / 256, p.H);
+  AM_LAUNCH(AM_STAGE_CORR, s, k_inv_m<<<gi, 256, 0, s>>>(p, w));
+  const int per_head = (8 * 148 + p.H - 1) / p.H;
+  dim3 gs(min((p.T + kRowsPerBlock - 1) / kRowsPerBlock, per_head < 1 ? 1 : per_head), p.H);
+  AM_LAUNCH(AM_STAGE_CORR, s, k_score<<<gs, kSelThreads, 0, s>>>(p, w));
+  int n2 = 1;
+  while (n2 < p.T) n2 <<= 1;
+  const int sm = n2 * (int)(sizeof(uint64_t) + sizeof(int));   // T <= kSortSmemKeys: at most 192 KiB
+  cudaFuncSetAttribute(k_pick_highest, cudaFuncAttributeMaxDynamicSharedMemorySize, sm);
+  AM_LAUNCH(AM_STAGE_SELECT, s, k_pick_highest<<<p.H, kBoundThreads, sm, s>>>(p, w));
   return cudaGetLastError();
 }
 

@@ -13,6 +13,7 @@ namespace am {
 constexpr int kWsHeaderBytes = 256;      // magic + head count, then status words
 constexpr uint32_t kWsMagic = 0x414d4232u;  // "AMB2"
 constexpr int kMaxPicksPerPass = 64;     // k·R upper bound handled per pass
+constexpr int kHighestChunk = 8;         // pre-selected keys appended per refit (AM_SELECT_HIGHEST)
 constexpr int kMaxBudget = 2048;         // largest t_h the per-head solvers are sized for
 constexpr int kNnlsThreads = 256;
 constexpr int kCholThreads = 256;
@@ -31,6 +32,7 @@ struct Problem {
   int corr_bf16;      // the correlation pass streams a bf16 copy of Φᵀ
   int corr_recompute; // the correlation pass recomputes Φ on the tensor cores
   int corr_bounded;   // the correlation pass computes only keys its bound cannot exclude
+  int select_highest; // keys chosen up front by total attention, fed to the refits kR at a time
 };
 
 // Device pointers into the caller's workspace (see plan_workspace()).
@@ -47,6 +49,7 @@ struct Work {
   float* Y;             // [H][n][d]
   float* r;             // [H][ldn] residual (fp32 copy read by the correlation pass)
   float* corr;          // [H][T]
+  double* inv_m;        // [H][ldn] 1 / m_i (0 for a query without mass), highest-attention scores
   uint8_t* sel;         // [H][T] selected flags
   int32_t* picks;       // [Σt] pick order
   float* pick_corr;     // [Σt]
@@ -133,6 +136,8 @@ cudaError_t launch_omp_pass(const Problem& p, const Work& w, int pass, int activ
 // probe, exact rows, extension, exact rows, selection
 cudaError_t launch_column_norms(const Problem& p, const Work& w, cudaStream_t s);
 cudaError_t launch_corr_bounded(const Problem& p, const Work& w, int pass, int active, cudaStream_t s);
+// highest-attention selection: scores, then each head's t best keys as its picks (am_bounded.cu)
+cudaError_t launch_select_highest(const Problem& p, const Work& w, cudaStream_t s);
 cudaError_t launch_residual_norm(const Problem& p, const Work& w, double* residual_out,
                                  cudaStream_t s);
 // value fit and packing (am_valfit.cu)

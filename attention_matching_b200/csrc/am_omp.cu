@@ -1207,7 +1207,9 @@ cudaError_t launch_omp_init(const Problem& p, const Work& w, cudaStream_t s) {
 cudaError_t launch_omp_pass(const Problem& p, const Work& w, int pass, int active, const CorrInputs& in,
                             cudaStream_t s) {
   if (active <= 0) return cudaSuccess;
-  if (p.corr_bounded) {
+  if (p.select_highest) {
+    // the picks were made up front; this pass feeds the next kR of them to the refit
+  } else if (p.corr_bounded) {
     cudaError_t e = launch_corr_bounded(p, w, pass, active, s);   // selects too
     if (e != cudaSuccess) return e;
   } else {

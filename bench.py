@@ -51,6 +51,8 @@ def parse_args():
     ap.add_argument("--corr", choices=["auto", "fp32", "bf16", "recompute", "bounded"], default="auto",
                     help="correlation pass: stored fp32 / stored bf16 copy / tensor-core recompute / "
                          "bounded (exact values for the keys a Cauchy-Schwarz bound cannot exclude)")
+    ap.add_argument("--select", choices=["omp", "highest"], default="omp",
+                    help="key selection: greedy OMP (the method) or the t keys of highest total attention")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     return ap.parse_args()
@@ -190,13 +192,16 @@ def cpu_baseline(wl, heads=1):
 
 
 # -------------------------------------------------------------- roofline ----
+HIGHEST_CHUNK = 8   # pre-selected keys the library appends per refit in highest-attention mode
+
+
 def stage_models(wl, n, T, d, H, ldn, corr_kind, rows_evaluated, tc=True):
     """Algorithmic work of one call (one step) per library stage: bytes that
     must cross HBM for the memory-bound stages, dense flops for the GEMM and
     the fp64 solver stages.  Summed over the stage's launches in the step.
     With the tensor-core feature pass the column norms are summed from its
     per-(query block, quarter) fp32 partials instead of re-reading Φᵀ."""
-    kR = wl.topk * wl.refit_every
+    kR = HIGHEST_CHUNK if corr_kind == "highest" else wl.topk * wl.refit_every
     s1 = [min((p + 1) * kR, t) for t in wl.budgets for p in range((t + kR - 1) // kR)]
     row = ldn * 4                                   # one stored Φᵀ row (fp32)
     m = {
@@ -211,7 +216,10 @@ def stage_models(wl, n, T, d, H, ldn, corr_kind, rows_evaluated, tc=True):
         "normal": {"bound": "fp64", "flops": float(sum(n * t * (t + 1) + 2 * n * t * d for t in wl.budgets))},
         "solve": {"bound": "fp64", "flops": float(sum(t ** 3 / 3 + 2 * t * t * d for t in wl.budgets))},
     }
-    if corr_kind == "recompute":
+    if corr_kind == "highest":
+        # one fp64 pass over the stored features for the scores, then a per-head sort
+        m["corr"] = {"bound": "hbm", "bytes": float(H * (T * row + ldn * 8))}
+    elif corr_kind == "recompute":
         m["corr"] = {"bound": "tensor", "flops": 2.0 * len(s1) * n * T * d, "exps": float(len(s1)) * n * T}
     elif corr_kind == "bounded":
         parts = 4 * ((n + 127) // 128)
@@ -341,11 +349,12 @@ def run_ours(args, rank, world, local_rank):
     Q, K, V = Qh.to(dev), Kh.to(dev), Vh.to(dev)
     corr_mode = {"auto": am.CORR_AUTO, "fp32": am.CORR_STORED_FP32, "bf16": am.CORR_STORED_BF16,
                  "recompute": am.CORR_RECOMPUTE, "bounded": am.CORR_BOUNDED}[args.corr]
-    kw = dict(topk=wl.topk, refit_every=wl.refit_every, corr_mode=corr_mode)
+    select_mode = am.SELECT_HIGHEST if args.select == "highest" else am.SELECT_OMP
+    kw = dict(topk=wl.topk, refit_every=wl.refit_every, corr_mode=corr_mode, select_mode=select_mode)
     opts = am.make_opts(am.BF16 if Q.dtype == torch.bfloat16 else am.FP32, wl.topk, wl.refit_every,
-                        corr_mode=corr_mode)
+                        corr_mode=corr_mode, select_mode=select_mode)
     tc_ok = Q.dtype == torch.bfloat16 and d in (64, 128)
-    corr_kind = {"auto": "bounded"}.get(args.corr, args.corr)
+    corr_kind = "highest" if args.select == "highest" else {"auto": "bounded"}.get(args.corr, args.corr)
     ws = torch.empty((am.workspace_size(n, T, d, wl.budgets, opts),), dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
     flush = torch.empty((256 << 20,), dtype=torch.uint8, device=dev)
@@ -424,7 +433,7 @@ def run_ours(args, rank, world, local_rank):
     peaks = load_peaks()
     rows_eval = int(am.features({"workspace": ws}, n, T, d, wl.budgets, wl.topk, wl.refit_every,
                                 am.BF16 if Q.dtype == torch.bfloat16 else am.FP32,
-                                corr_mode)["rows_evaluated"].sum().item())
+                                corr_mode, select_mode)["rows_evaluated"].sum().item())
     rf = roofline(stages, args.steps, stage_models(wl, n, T, d, H, ldn, corr_kind, rows_eval, tc_ok),
                   peaks, clk, committed_traffic() if corr_kind == "fp32" else {})
     value = job_throughput(H, world, ms)
@@ -432,7 +441,10 @@ def run_ours(args, rank, world, local_rank):
     cfg = {"workload": wl.name, "heads_per_gpu": H, "n": n, "T": T, "d": d,
            "budgets": wl.budgets if H <= 8 else f"{sum(wl.budgets)} total, min {min(wl.budgets)} max {max(wl.budgets)}",
            "topk": wl.topk, "refit_every": wl.refit_every,
+           "selection": "greedy OMP with NNLS refits" if args.select == "omp" else
+                        "the t keys of highest total attention, NNLS beta fit",
            "correlation": {"fp32": "streams stored fp32 Phi^T", "bf16": "streams a bf16 copy of Phi^T",
+                           "highest": "fp64 total-attention score of every key, one pass over Phi^T",
                            "recompute": "recomputes Phi on the tensor cores each pass",
                            "bounded": "exact fp64 values for the keys whose Cauchy-Schwarz bound "
                                       "reaches the pass's top k*R"}[corr_kind],

@@ -78,6 +78,21 @@ typedef enum am_corr_mode {
                                its bound; the picks are those of a full pass      */
 } am_corr_mode_t;
 
+/* How the t keys of each head are chosen.  Either way β is fit by NNLS on
+ * the chosen keys and C_v by the ridge least-squares fit.
+ *   AM_SELECT_OMP      greedy Orthogonal Matching Pursuit on the attention
+ *                      mass ("Fast KV Compaction via Attention Matching":
+ *                      zhichai.net deep dive §1.6; top-k batching with lazy
+ *                      refit, xinfinite.net article §3)
+ *   AM_SELECT_HIGHEST  the t keys with the largest total attention over the
+ *                      reference queries, score_j = Σ_i Φ_ij / m_i (each
+ *                      query's softmax probability of key j), ties to the
+ *                      lower key (AM-Highest: zhichai.net/en summary, "Method
+ *                      Family and Trade-offs"; the youleyou.com rewrite's
+ *                      highest-attention keys).  topk, refit_every and
+ *                      corr_mode are ignored; requires T <= 16384. */
+typedef enum am_select_mode { AM_SELECT_OMP = 0, AM_SELECT_HIGHEST = 1 } am_select_mode_t;
+
 /* Options.  Fill with am_default_opts() and override fields. */
 typedef struct am_opts {
   int32_t in_dtype;        /* am_dtype_t of Q_ref, K, V and of the C_k output   */
@@ -95,15 +110,17 @@ typedef struct am_opts {
                               block's β), or NULL for b = 0                       */
   /* Optional device outputs (NULL = not written) */
   int32_t* pick_order;     /* [Σt] keys in greedy pick order, packed like indices */
-  float* pick_corr;        /* [Σt] correlation c_j of each pick when it was made  */
+  float* pick_corr;        /* [Σt] correlation c_j of each pick when it was made
+                              (AM_SELECT_HIGHEST: its score)                     */
   float* shift_out;        /* [H] shift used                                     */
   double* residual_out;    /* [H] ‖m − Φ_S w‖ / ‖m‖ after the last refit          */
   float* w_out;            /* [Σt] NNLS weights, aligned with indices            */
+  int32_t select_mode;     /* am_select_mode_t (default AM_SELECT_OMP)           */
 } am_opts_t;
 
 /* Fill *opts with defaults: bf16 inputs, k = 1, R = 1, scale = 1/sqrt(d),
  * ridge = 1e-6, w_floor_rel = 1e-12, corr_mode = AM_CORR_AUTO, every
- * optional pointer NULL. */
+ * optional pointer NULL, select_mode = AM_SELECT_OMP. */
 am_status_t am_default_opts(am_opts_t* opts);
 
 /* Device workspace needed by am_compact_heads for this problem.

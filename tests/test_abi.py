@@ -26,9 +26,27 @@ def test_library_exports_every_declared_symbol():
         assert hasattr(L, n), n
 
 
-def test_opts_struct_layout_matches_header():
-    # 8 four-byte fields then 7 pointers
-    assert ctypes.sizeof(am.AmOpts) == 8 * 4 + 7 * 8
+def test_opts_struct_layout_matches_header(tmp_path):
+    """The ctypes mirror of am_opts_t has the size and field offsets a C
+    compiler gives the header's struct."""
+    import shutil
+    import subprocess
+    cc = shutil.which("gcc") or shutil.which("cc")
+    if cc is None:
+        pytest.skip("no C compiler")
+    fields = [f[0] for f in am.AmOpts._fields_]
+    src = tmp_path / "layout.c"
+    src.write_text("#include <stdio.h>\n#include <stddef.h>\n#include \"am_b200.h\"\n"
+                   "int main(void) {\n  printf(\"%zu\\n\", sizeof(am_opts_t));\n"
+                   + "".join(f"  printf(\"%zu\\n\", offsetof(am_opts_t, {f}));\n" for f in fields)
+                   + "  return 0;\n}\n")
+    exe = tmp_path / "layout"
+    include = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include")
+    subprocess.run([cc, "-std=c99", "-I", include, str(src), "-o", str(exe)], check=True)
+    got = [int(x) for x in subprocess.run([str(exe)], check=True, capture_output=True,
+                                          text=True).stdout.split()]
+    assert got[0] == ctypes.sizeof(am.AmOpts)
+    assert got[1:] == [getattr(am.AmOpts, f).offset for f in fields]
 
 
 def test_defaults_and_status_strings():

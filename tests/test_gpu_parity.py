@@ -258,6 +258,57 @@ def test_wide_passes_topk8_refit4():
     check_all(heads, [70, 45], 8, 4, key_bias=kb, label="k8 R4")
 
 
+def _attention_scores(Q, K, key_bias=None):
+    """Σ_i softmax_i(s)_j in float64: the total attention each key receives."""
+    s = O.logits(Q, K, key_bias=key_bias)
+    p = np.exp(s - s.max(axis=1, keepdims=True))
+    p /= p.sum(axis=1, keepdims=True)
+    return p.sum(axis=0)
+
+
+def check_highest(heads, budgets, key_bias=None, label=""):
+    """AM-Highest on the GPU against the oracle: the pick order is the
+    oracle's highest-attention order (a swap only where two scores agree to
+    1e-6 of the largest: the GPU's scores come from the stored fp32 features,
+    whose exponentials carry a few 1e-7 of relative error), and β, residual
+    and output match the oracle's one-round compaction on those picks under
+    the rules of tests/parity.py."""
+    import attention_matching_b200 as am
+    shifts = [shift_for(*h.f64()[:2], key_bias=None if key_bias is None else key_bias[i])
+              for i, h in enumerate(heads)]
+    out = run_gpu(heads, budgets, 1, 1, shifts, key_bias, select_mode=am.SELECT_HIGHEST)
+    assert all(s in (0, 8) for s in out["status"]), out["status"]
+    for h, t in enumerate(budgets):
+        Q, K, V = heads[h].f64()
+        kb = None if key_bias is None else np.asarray(key_bias[h], np.float64)
+        g = split_head(out, h)
+        score = _attention_scores(Q, K, kb)
+        want = O.highest_attention_select(Q, K, t, key_bias=kb)
+        got = g["pick_order"]
+        for a, b in zip(got, want):
+            if a != b:
+                assert abs(score[a] - score[b]) <= 1e-6 * score.max(), f"{label} head {h}: pick {a} vs {b}"
+        ref = O.compact_head(Q, K, V, t, t, 1, shift=shifts[h], key_bias=kb, forced_picks=want)
+        rep = check_head(g, Q, K, V, t, t, 1, shifts[h], kb, oracle_res=ref, label=f"{label} head {h}",
+                         exact_picks=False)
+        if list(got) == list(want):
+            assert rep["same_set"], rep
+
+
+@needs_cuda
+def test_highest_attention_selection_bf16():
+    heads = [W.structured_head(520 + h, n=512, T=700) for h in range(2)]
+    check_highest(heads, [40, 25], label="highest bf16")
+
+
+@needs_cuda
+def test_highest_attention_selection_fp32_prior_bias():
+    wl = W.single_head_fp32()
+    rng = np.random.default_rng(531)
+    kb = [np.float32(rng.normal(0.0, 0.5, wl.heads[0].K.shape[0]))]
+    check_highest(wl.heads, [16], key_bias=kb, label="highest fp32 bias")
+
+
 @needs_cuda
 def test_bounded_correlation_long_key_axis():
     """T = 20000 keys: the bounded correlation pass sorts the column norms in
