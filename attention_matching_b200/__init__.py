@@ -16,7 +16,7 @@ from typing import Dict, Optional, Sequence
 __all__ = ["AmError", "AmOpts", "lib", "library_path", "workspace_size", "compact_heads",
            "get_status", "profile_enable", "profile_collect", "kernel_launches", "STAGES",
            "STATUS", "BF16", "FP32", "CORR_AUTO", "CORR_STORED_FP32", "CORR_STORED_BF16",
-           "CORR_RECOMPUTE", "CORR_BOUNDED"]
+           "CORR_RECOMPUTE", "CORR_BOUNDED", "SELECT_OMP", "SELECT_HIGHEST", "attend_packed"]
 
 BF16, FP32 = 0, 1
 CORR_AUTO, CORR_STORED_FP32, CORR_STORED_BF16, CORR_RECOMPUTE, CORR_BOUNDED = 0, 1, 2, 3, 4
@@ -108,6 +108,10 @@ def lib() -> ctypes.CDLL:
         L.am_profile_collect.restype = c_int
         L.am_kernel_launches.argtypes = []
         L.am_kernel_launches.restype = ctypes.c_int64
+        L.am_attend_packed.argtypes = [c_void_p, c_int, c_int, c_int, c_int, c_void_p, c_void_p, c_void_p,
+                                       c_void_p, c_void_p, c_void_p, c_int, ctypes.c_float, c_void_p,
+                                       c_void_p]
+        L.am_attend_packed.restype = c_int
         _lib = L
     return _lib
 
@@ -268,7 +272,7 @@ def compact_heads(Q, K, V, budgets: Sequence[int], topk: int = 1, refit_every: i
 
 
 STAGES = ["shift", "phi", "target", "init", "corr", "select", "gram", "nnls", "resid",
-          "finalize", "design", "normal", "solve", "norms", "rows"]
+          "finalize", "design", "normal", "solve", "norms", "rows", "attend"]
 
 
 def profile_enable(on: bool = True) -> None:
@@ -288,6 +292,38 @@ def profile_collect() -> Dict[str, Dict[str, float]]:
 
 def kernel_launches() -> int:
     return int(lib().am_kernel_launches())
+
+
+def attend_packed(Q, packed: Dict, K_new=None, V_new=None, scale: float = 0.0, stream=None):
+    """Attention of Q [H, nq, d] over each head's compacted segment (the
+    packed C_k, beta, C_v, cu_t that compact_heads returned) followed by
+    fresh keys K_new, V_new [H, T_new, d] (optional).  Q, C_k, K_new and
+    V_new share a dtype (bf16 or fp32), all on the GPU; returns out
+    [H, nq, d] fp32."""
+    import torch
+    if not Q.is_cuda or Q.dim() != 3 or not Q.is_contiguous():
+        raise ValueError("Q must be a contiguous CUDA tensor [H, nq, d]")
+    H, nq, d = Q.shape
+    dt = BF16 if Q.dtype == torch.bfloat16 else FP32
+    C_k, beta, C_v = packed["C_k"], packed["beta"], packed["C_v"]
+    if C_k.dtype != Q.dtype:
+        raise ValueError("C_k and Q must share a dtype")
+    cu = packed["cu_t"].to(device=Q.device, dtype=torch.int64).contiguous()
+    Tn = 0
+    if K_new is not None:
+        if K_new.shape[:1] != (H,) or K_new.shape != V_new.shape or K_new.dtype != Q.dtype:
+            raise ValueError("K_new and V_new must be [H, T_new, d] in Q's dtype")
+        K_new, V_new = K_new.contiguous(), V_new.contiguous()
+        Tn = K_new.shape[1]
+    out = torch.empty((H, nq, d), dtype=torch.float32, device=Q.device)
+    if stream is None:
+        stream = torch.cuda.current_stream(Q.device).cuda_stream
+    rc = lib().am_attend_packed(Q.data_ptr(), nq, d, H, dt, C_k.data_ptr(), beta.data_ptr(), C_v.data_ptr(),
+                                cu.data_ptr(), _ptr(K_new), _ptr(V_new), Tn, scale, out.data_ptr(),
+                                ctypes.c_void_p(stream))
+    if rc:
+        raise AmError(rc, "am_attend_packed")
+    return out
 
 
 def get_status(workspace, H: int, stream=None):

@@ -223,6 +223,31 @@ am_status_t am_compact_heads_noalloc(const void* Q_ref, const void* K, const voi
                                      void* C_k, float* beta, float* C_v, int32_t* indices,
                                      int32_t* status_out, void* stream);
 
+/* Attention that consumes a compacted cache: for head h and query i,
+ *   out[h][i] = Σ_j softmax_j(q_i·k_j·scale + b_j) v_j
+ * over head h's compacted segment (k = C_k, v = C_v, b = β, rows cu_t[h] ..
+ * cu_t[h+1] of the packed outputs of am_compact_heads) followed by T_new
+ * fresh keys (k = K_new, v = V_new, b = 0).  The compacted block stands in
+ * for the keys it replaced through its additive per-key bias, and the
+ * result equals the mass-weighted mixture of the two blocks' local outputs
+ * (the attention mixing identity: "Fast KV Compaction via Attention
+ * Matching", zhichai.net deep dive §4.1-4.2 on bias-capable attention
+ * kernels and varlen per-head segments; zhichai.net/en summary,
+ * "Engineering Practicality").
+ *   Q            device [H][nq][d], dtype in_dtype
+ *   C_k          device [Σt][d], dtype in_dtype; beta device [Σt] fp32;
+ *   C_v          device [Σt][d] fp32 (as am_compact_heads writes them)
+ *   cu_t         device int64 [H+1], the segment offsets
+ *   K_new, V_new device [H][T_new][d], dtype in_dtype (NULL when T_new = 0)
+ *   scale        logit scale; <= 0 selects 1/sqrt(d)
+ *   out          device [H][nq][d] fp32
+ * fp32 arithmetic with an online softmax; 1 <= d <= 256, num_heads <= 65535.
+ * Asynchronous on stream; argument errors return synchronously. */
+am_status_t am_attend_packed(const void* Q, int32_t nq, int32_t d, int32_t num_heads, int32_t in_dtype,
+                             const void* C_k, const float* beta, const float* C_v, const int64_t* cu_t,
+                             const void* K_new, const void* V_new, int32_t T_new, float scale,
+                             float* out, void* stream);
+
 /* Synchronise `stream`, then copy the per-head device status words of the last
  * call that used `workspace` into host per_head[H] (may be NULL) and return the
  * most severe one (AM_OK if all heads succeeded). */
@@ -253,7 +278,8 @@ typedef enum am_stage {
   AM_STAGE_NORMS = 13,   /* bounded mode: ‖Φ_{:,j}‖, keys by norm    */
   AM_STAGE_ROWS = 14,    /* bounded mode: exact c_j of listed keys,
                             threshold and picks                      */
-  AM_STAGE_COUNT = 15
+  AM_STAGE_ATTEND = 15,  /* am_attend_packed                         */
+  AM_STAGE_COUNT = 16
 } am_stage_t;
 
 am_status_t am_profile_enable(int32_t on);

@@ -104,3 +104,24 @@ def test_compact_heads_argument_errors_are_synchronous():
     assert _call(ws=None) == 3                      # no workspace
     assert _call(ws=4096 + 8, ws_bytes=1 << 30) == 3  # misaligned workspace
     assert _call(ws=4096, ws_bytes=16) == 3          # too small
+
+
+def test_attend_packed_argument_errors():
+    """am_attend_packed rejects missing buffers and unsupported sizes before
+    any GPU work."""
+    L = am.lib()
+    v = ctypes.c_void_p(16)
+    args = dict(Q=v, nq=4, d=64, H=2, dt=am.BF16, Ck=v, beta=v, Cv=v, cu=v, Kn=None, Vn=None, Tn=0,
+                scale=ctypes.c_float(0.0), out=v, stream=None)
+
+    def call(**kw):
+        a = dict(args, **kw)
+        return L.am_attend_packed(a["Q"], a["nq"], a["d"], a["H"], a["dt"], a["Ck"], a["beta"], a["Cv"],
+                                  a["cu"], a["Kn"], a["Vn"], a["Tn"], a["scale"], a["out"], a["stream"])
+
+    code = {v: k for k, v in am.STATUS.items()}
+    assert call(Q=None) == code["AM_ERR_INVALID_ARG"]
+    assert call(Tn=5) == code["AM_ERR_INVALID_ARG"]          # fresh keys without buffers
+    assert call(d=300) == code["AM_ERR_UNSUPPORTED"]
+    assert call(dt=7) == code["AM_ERR_INVALID_ARG"]
+    assert call(nq=0) == code["AM_ERR_INVALID_ARG"]

@@ -309,6 +309,47 @@ def test_highest_attention_selection_fp32_prior_bias():
     check_highest(wl.heads, [16], key_bias=kb, label="highest fp32 bias")
 
 
+def check_attend(heads, budgets, topk, refit, Tn, nq, seed, label):
+    """attend_packed over each head's compacted segment (the GPU's own C_k, β,
+    C_v) and Tn fresh keys, against float64 attention over the concatenated
+    keys with bias [β, 0]; that reference also equals the mass-weighted mixture
+    of the two blocks' local outputs (the mixing identity)."""
+    import attention_matching_b200 as am
+    out = run_gpu(heads, budgets, topk, refit)
+    H = len(heads)
+    d = heads[0].Q.shape[1]
+    dt = heads[0].Q.dtype
+    rng = np.random.default_rng(seed)
+    Kn = torch.tensor(rng.normal(0.0, 1.0, (H, Tn, d)), dtype=torch.float32).to(dt)
+    Vn = torch.tensor(rng.normal(0.0, 1.0, (H, Tn, d)), dtype=torch.float32).to(dt)
+    Qt = torch.stack([h.Q[:nq] for h in heads]).contiguous()
+    got = am.attend_packed(Qt.cuda(), out, Kn.cuda(), Vn.cuda()).cpu().double().numpy()
+    got0 = am.attend_packed(Qt.cuda(), out).cpu().double().numpy()
+    for h in range(H):
+        g = split_head(out, h)
+        Qh, Kh, Vh = Qt[h].double().numpy(), Kn[h].double().numpy(), Vn[h].double().numpy()
+        want = O.attention_output(Qh, np.concatenate([g["C_k"], Kh]), np.concatenate([g["C_v"], Vh]),
+                                  key_bias=np.concatenate([g["beta"], np.zeros(Tn)]))
+        o1, l1 = O.local_attention(Qh, g["C_k"], g["C_v"], key_bias=g["beta"])
+        o2, l2 = O.local_attention(Qh, Kh, Vh)
+        np.testing.assert_allclose(O.mix_blocks([o1, o2], [l1, l2]), want, rtol=1e-9, atol=1e-12)
+        rel = np.linalg.norm(got[h] - want) / np.linalg.norm(want)
+        rel0 = np.linalg.norm(got0[h] - o1) / np.linalg.norm(o1)
+        assert rel < 1e-5 and rel0 < 1e-5, f"{label} head {h}: {rel} {rel0}"
+
+
+@needs_cuda
+def test_attend_packed_bf16_with_fresh_keys():
+    heads = [W.structured_head(540 + h, n=512, T=700) for h in range(2)]
+    check_attend(heads, [40, 30], 4, 2, Tn=50, nq=37, seed=541, label="attend bf16")
+
+
+@needs_cuda
+def test_attend_packed_fp32_d64():
+    wl = W.single_head_fp32()
+    check_attend(wl.heads, [16], 1, 1, Tn=9, nq=20, seed=551, label="attend fp32 d64")
+
+
 @needs_cuda
 def test_bounded_correlation_long_key_axis():
     """T = 20000 keys: the bounded correlation pass sorts the column norms in
