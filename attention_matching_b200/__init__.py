@@ -16,7 +16,8 @@ from typing import Dict, Optional, Sequence
 __all__ = ["AmError", "AmOpts", "lib", "library_path", "workspace_size", "compact_heads",
            "get_status", "profile_enable", "profile_collect", "kernel_launches", "STAGES",
            "STATUS", "BF16", "FP32", "CORR_AUTO", "CORR_STORED_FP32", "CORR_STORED_BF16",
-           "CORR_RECOMPUTE", "CORR_BOUNDED", "SELECT_OMP", "SELECT_HIGHEST", "attend_packed"]
+           "CORR_RECOMPUTE", "CORR_BOUNDED", "SELECT_OMP", "SELECT_HIGHEST", "attend_packed",
+           "assign_budgets"]
 
 BF16, FP32 = 0, 1
 CORR_AUTO, CORR_STORED_FP32, CORR_STORED_BF16, CORR_RECOMPUTE, CORR_BOUNDED = 0, 1, 2, 3, 4
@@ -112,6 +113,9 @@ def lib() -> ctypes.CDLL:
                                        c_void_p, c_void_p, c_void_p, c_int, ctypes.c_float, c_void_p,
                                        c_void_p]
         L.am_attend_packed.restype = c_int
+        L.am_assign_budgets.argtypes = [ctypes.POINTER(ctypes.c_double), c_int, c_int, c_int, c_int,
+                                        ctypes.c_int64, c_int, P_i32, P_i32]
+        L.am_assign_budgets.restype = c_int
         _lib = L
     return _lib
 
@@ -324,6 +328,24 @@ def attend_packed(Q, packed: Dict, K_new=None, V_new=None, scale: float = 0.0, s
     if rc:
         raise AmError(rc, "am_attend_packed")
     return out
+
+
+def assign_budgets(loss, t_min: int, quantum: int, total: int, max_swaps: Optional[int] = None):
+    """Per-head budgets from sensitivity curves loss [H, G] (head h's loss at
+    budget t_min + g·quantum) by the library's greedy swaps (host code).
+    Returns (budgets, swaps)."""
+    import numpy as np
+    L = np.ascontiguousarray(loss, dtype=np.float64)
+    if L.ndim != 2:
+        raise ValueError("loss must be [num_heads, levels]")
+    H, G = L.shape
+    out = (ctypes.c_int32 * H)()
+    sw = ctypes.c_int32(0)
+    rc = lib().am_assign_budgets(L.ctypes.data_as(ctypes.POINTER(ctypes.c_double)), H, G, t_min, quantum,
+                                 total, -1 if max_swaps is None else max_swaps, out, ctypes.byref(sw))
+    if rc:
+        raise AmError(rc, "am_assign_budgets")
+    return list(out), sw.value
 
 
 def get_status(workspace, H: int, stream=None):

@@ -299,3 +299,24 @@ class OnlineHeads:
                               key_bias=np.float32(bias[:c])))
         self.round += 1
         return heads
+
+
+def sensitivity_curves(seed: int, num_heads: int, levels: int, t_min: int = 4, quantum: int = 16,
+                       convex: bool = True) -> np.ndarray:
+    """Synthetic per-head sensitivity curves [num_heads][levels]: head h's loss
+    at budget t = t_min + g·quantum is a_h·exp(−(t − t_min)/τ_h) + c_h, with
+    a_h = exp(N(0, 1)), τ_h = 64·exp(0.7·N(0, 1)) and c_h ~ U(0, 0.1):
+    decreasing with diminishing returns, heads differing in scale and in how
+    fast they saturate (the pages' curves need models and data).  With
+    convex=False each head also gets a bump of height 0.3·a_h at a random
+    level, so that some gains grow before they shrink."""
+    rng = np.random.default_rng(seed)
+    a = np.exp(rng.standard_normal(num_heads))
+    tau = 64.0 * np.exp(0.7 * rng.standard_normal(num_heads))
+    c = rng.uniform(0.0, 0.1, num_heads)
+    t = t_min + quantum * np.arange(levels, dtype=np.float64)
+    L = a[:, None] * np.exp(-(t[None, :] - t_min) / tau[:, None]) + c[:, None]
+    if not convex:
+        at = rng.integers(0, levels, num_heads)
+        L[np.arange(num_heads), at] += 0.3 * a
+    return L

@@ -248,6 +248,25 @@ am_status_t am_attend_packed(const void* Q, int32_t nq, int32_t d, int32_t num_h
                              const void* K_new, const void* V_new, int32_t T_new, float scale,
                              float* out, void* stream);
 
+/* Non-uniform per-head budgets from sensitivity curves by greedy swaps
+ * ("Fast KV Compaction via Attention Matching": zhichai.net/en summary,
+ * "Engineering Practicality"; zhichai.net deep dive §4.2).  Host-only: no
+ * GPU work, every pointer is a host pointer.
+ *   loss        [num_heads][levels]: head h's loss at budget t_min + g·quantum
+ *   total       Σ budgets; total − num_heads·t_min must be a multiple of
+ *               quantum and at most num_heads·(levels − 1)·quantum
+ *               (otherwise AM_ERR_BUDGET)
+ *   max_swaps   cap on swaps, < 0 for none
+ *   budgets_out [num_heads]; swaps_out (optional) the swaps made
+ * The levels start as even as the total allows (the first heads take the
+ * remainder); each swap moves one quantum to the head whose loss falls most
+ * from the head, other than that one, whose loss rises least, ties to the
+ * lower head, while the fall exceeds the rise.  Non-finite losses return
+ * AM_ERR_NONFINITE. */
+am_status_t am_assign_budgets(const double* loss, int32_t num_heads, int32_t levels, int32_t t_min,
+                              int32_t quantum, int64_t total, int32_t max_swaps,
+                              int32_t* budgets_out, int32_t* swaps_out);
+
 /* Synchronise `stream`, then copy the per-head device status words of the last
  * call that used `workspace` into host per_head[H] (may be NULL) and return the
  * most severe one (AM_OK if all heads succeeded). */

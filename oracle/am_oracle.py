@@ -407,3 +407,55 @@ def highest_attention_select(Q, K, t: int, scale=None, key_bias=None) -> List[in
     T = score.size
     order = np.lexsort((np.arange(T), -score))
     return [int(j) for j in order[:t]]
+
+
+# ---------------------------------------------------------------------------
+# Non-uniform head budgets by greedy swaps ([Summary] "Engineering
+# Practicality": sensitivity curves rank head importance once, a greedy-swap
+# algorithm assigns per-head ratios; [DeepDive] §4.2 steps 1-2; [News]
+# "non-uniform compaction").  The pages name the algorithm only; the reading
+# taken: one quantum at a time moves from the head that loses least by
+# giving it up to the head that gains most by receiving it, while that
+# lowers the summed loss, starting from the most even split.
+# ---------------------------------------------------------------------------
+
+def greedy_swap_budgets(loss, t_min: int, quantum: int, total: int,
+                        max_swaps: Optional[int] = None):
+    """Per-head budgets from sensitivity curves.
+
+    loss[h][g] is head h's loss at budget t_min + g·quantum.  The levels
+    start as even as the total allows (every head at units // H, one more
+    for the first units % H heads, units = (total − H·t_min) / quantum).
+    Each swap: the receiver b is the head with the largest gain
+    loss[b][l_b] − loss[b][l_b + 1] (lowest index on ties, a head already at
+    the top level excluded); the donor a is the head other than b with the
+    smallest cost loss[a][l_a − 1] − loss[a][l_a] (lowest index on ties, a
+    head at level 0 excluded); the quantum moves when gain > cost.  Returns
+    (budgets, swaps)."""
+    L = np.asarray(loss, F64)
+    H, G = L.shape
+    rest = total - H * t_min
+    if rest < 0 or rest % quantum or rest // quantum > H * (G - 1):
+        raise ValueError("total is not reachable on this budget grid")
+    units = rest // quantum
+    lev = [units // H + (1 if h < units % H else 0) for h in range(H)]
+    swaps = 0
+    while max_swaps is None or swaps < max_swaps:
+        b, gain = -1, -math.inf
+        for h in range(H):
+            if lev[h] < G - 1:
+                gh = L[h, lev[h]] - L[h, lev[h] + 1]
+                if gh > gain:
+                    b, gain = h, gh
+        a, cost = -1, math.inf
+        for h in range(H):
+            if h != b and lev[h] > 0:
+                ch = L[h, lev[h] - 1] - L[h, lev[h]]
+                if ch < cost:
+                    a, cost = h, ch
+        if a < 0 or b < 0 or not gain > cost:
+            break
+        lev[a] -= 1
+        lev[b] += 1
+        swaps += 1
+    return [t_min + quantum * x for x in lev], swaps
