@@ -182,7 +182,9 @@ typedef struct am_workspace_view {
   size_t rows_evaluated;   /* int64 [H]: keys whose correlation the bounded
                               passes evaluated, summed over the call's passes */
   size_t column_norms;     /* fp64 [H][T]: the bounded pass's ‖Φ_{:,j}‖₂, an upper
-                              bound within a relative 2e-6 of the exact norm */
+                              bound within a relative 2e-6 of the exact norm
+                              (AM_SELECT_HIGHEST: each key's total-attention
+                              score Σ_i Φ_ij / m_i instead) */
 } am_workspace_view_t;
 
 am_status_t am_workspace_view(int32_t n, int32_t T, int32_t d, int32_t num_heads,

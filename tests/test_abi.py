@@ -26,27 +26,29 @@ def test_library_exports_every_declared_symbol():
         assert hasattr(L, n), n
 
 
-def test_opts_struct_layout_matches_header(tmp_path):
-    """The ctypes mirror of am_opts_t has the size and field offsets a C
-    compiler gives the header's struct."""
+@pytest.mark.parametrize("cname,mirror", [("am_opts_t", "AmOpts"), ("am_workspace_view_t", "AmWorkspaceView")])
+def test_struct_layout_matches_header(tmp_path, cname, mirror):
+    """Each ctypes mirror has the size and field offsets a C compiler gives
+    the header's struct."""
     import shutil
     import subprocess
     cc = shutil.which("gcc") or shutil.which("cc")
     if cc is None:
         pytest.skip("no C compiler")
-    fields = [f[0] for f in am.AmOpts._fields_]
+    cls = getattr(am, mirror)
+    fields = [f[0] for f in cls._fields_]
     src = tmp_path / "layout.c"
     src.write_text("#include <stdio.h>\n#include <stddef.h>\n#include \"am_b200.h\"\n"
-                   "int main(void) {\n  printf(\"%zu\\n\", sizeof(am_opts_t));\n"
-                   + "".join(f"  printf(\"%zu\\n\", offsetof(am_opts_t, {f}));\n" for f in fields)
+                   f"int main(void) {{\n  printf(\"%zu\\n\", sizeof({cname}));\n"
+                   + "".join(f"  printf(\"%zu\\n\", offsetof({cname}, {f}));\n" for f in fields)
                    + "  return 0;\n}\n")
     exe = tmp_path / "layout"
     include = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include")
     subprocess.run([cc, "-std=c99", "-I", include, str(src), "-o", str(exe)], check=True)
     got = [int(x) for x in subprocess.run([str(exe)], check=True, capture_output=True,
                                           text=True).stdout.split()]
-    assert got[0] == ctypes.sizeof(am.AmOpts)
-    assert got[1:] == [getattr(am.AmOpts, f).offset for f in fields]
+    assert got[0] == ctypes.sizeof(cls)
+    assert got[1:] == [getattr(cls, f).offset for f in fields]
 
 
 def test_defaults_and_status_strings():
@@ -125,3 +127,29 @@ def test_attend_packed_argument_errors():
     assert call(d=300) == code["AM_ERR_UNSUPPORTED"]
     assert call(dt=7) == code["AM_ERR_INVALID_ARG"]
     assert call(nq=0) == code["AM_ERR_INVALID_ARG"]
+
+
+@pytest.mark.parametrize("n,T,d,budgets,select", [
+    (512, 256, 64, [16], 0), (1000, 1100, 128, [13, 22, 8], 0), (8192, 8192, 128, [164] * 8, 0),
+    (700, 900, 128, [70, 45], 1), (33, 1, 16, [1], 0),
+])
+def test_workspace_view_regions_fit_align_and_do_not_overlap(n, T, d, budgets, select):
+    """The feature regions am_workspace_view reports lie inside the size
+    am_workspace_size asks for, start 16-byte aligned and are disjoint."""
+    dt = am.BF16 if d in (64, 128) else am.FP32
+    o = am.make_opts(dt, 4, 2, select_mode=select)
+    size = am.workspace_size(n, T, d, budgets, o)
+    v = am.AmWorkspaceView()
+    H, S = len(budgets), sum(budgets)
+    arr = (ctypes.c_int32 * H)(*budgets)
+    assert am.lib().am_workspace_view(n, T, d, H, arr, ctypes.byref(o), ctypes.byref(v)) == 0
+    ldn = v.ldn
+    assert ldn % 32 == 0 and ldn >= n
+    regions = [(v.phiT, H * T * ldn * 4), (v.mass, H * ldn * 8), (v.target, H * n * d * 4), (v.shift, H * 4),
+               (v.weights, S * 8), (v.resid, H * ldn * 4), (v.rows_evaluated, H * 8),
+               (v.column_norms, H * T * 8)]
+    for off, sz in regions:
+        assert off % 16 == 0 and off + sz <= size, (off, sz, size)
+    spans = sorted(regions)
+    for (a, sa), (b, _) in zip(spans, spans[1:]):
+        assert a + sa <= b, (a, sa, b)
