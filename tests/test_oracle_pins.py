@@ -362,6 +362,16 @@ def test_highest_attention_select():
     score = torch.softmax(torch.from_numpy(Q @ K.T / math.sqrt(d)), dim=1).sum(0).numpy()
     sel = O.highest_attention_select(Q, K, 5)
     assert sorted(sel) == sorted(np.argsort(-score, kind="stable")[:5].tolist())
+    assert sel == np.argsort(-score, kind="stable")[:5].tolist()      # pick order: largest first
+    # with a prior per-key bias, the softmax takes it as an additive logit term
+    b = rng.standard_normal(T)
+    score_b = torch.softmax(torch.from_numpy(Q @ K.T / math.sqrt(d) + b[None, :]), dim=1).sum(0).numpy()
+    assert O.highest_attention_select(Q, K, 7, key_bias=b) == np.argsort(-score_b, kind="stable")[:7].tolist()
+    # exact ties go to the lower key: duplicated keys share a score
+    K2 = np.concatenate([K[:3], K[:3]])
+    sel2 = O.highest_attention_select(Q, K2, 6)
+    for j in range(3):
+        assert sel2.index(j) < sel2.index(j + 3)
 
 
 # --------------------------------------------------------------------------
