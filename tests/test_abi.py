@@ -153,3 +153,20 @@ def test_workspace_view_regions_fit_align_and_do_not_overlap(n, T, d, budgets, s
     spans = sorted(regions)
     for (a, sa), (b, _) in zip(spans, spans[1:]):
         assert a + sa <= b, (a, sa, b)
+
+
+def test_highest_attention_mode_argument_rules():
+    """Highest-attention selection ignores topk and refit_every (a k·R the
+    OMP path rejects is accepted) and needs T <= 16384 for its per-head sort."""
+    code = {v: k for k, v in am.STATUS.items()}
+    ok = am.make_opts(am.BF16, 64, 64, select_mode=am.SELECT_HIGHEST)
+    assert am.workspace_size(512, 4096, 128, [100, 200], ok) > 0
+    with pytest.raises(am.AmError) as e:
+        am.workspace_size(512, 4096, 128, [100], am.make_opts(am.BF16, 64, 64))
+    assert e.value.code == code["AM_ERR_UNSUPPORTED"]
+    with pytest.raises(am.AmError) as e:
+        am.workspace_size(512, 20000, 128, [100], ok)
+    assert e.value.code == code["AM_ERR_UNSUPPORTED"]
+    with pytest.raises(am.AmError) as e:
+        am.workspace_size(512, 4096, 128, [100], am.make_opts(am.BF16, 4, 2, select_mode=5))
+    assert e.value.code == code["AM_ERR_INVALID_ARG"]
