@@ -213,11 +213,16 @@ am_status_t am_workspace_view(int32_t n, int32_t T, int32_t d, int32_t num_heads
  * workspace (am_workspace_size) exceeds AM_NOALLOC_SCRATCH_BYTES.
  *
  * The first call on a device looks up the array's device address with the
- * CUDA runtime; make that first call outside any stream capture.  All calls
- * share the one array and leave their contents in it: calls whose work
- * overlaps on the GPU (on different streams, or from different threads)
+ * CUDA runtime.  Every call also copies a small header and the per-head
+ * tables from pageable host memory with cudaMemcpyAsync, so the call cannot
+ * be recorded into a CUDA graph: make every call outside stream capture.
+ * All calls share the one array and leave their contents in it: calls whose
+ * work overlaps on the GPU (on different streams, or from different threads)
  * race on it and must be serialised by the caller.  The call allocates
- * nothing: no cudaMalloc, no cudaFree, no allocating library routine. */
+ * nothing: no cudaMalloc, no cudaFree, no allocating library routine.  It
+ * creates no stream or event, except that while stage timing is switched on
+ * (am_profile_enable) each launch is bracketed by CUDA events as described
+ * there. */
 am_status_t am_compact_heads_noalloc(const void* Q_ref, const void* K, const void* V,
                                      int32_t n, int32_t T, int32_t d, int32_t num_heads,
                                      const int32_t* budgets, const am_opts_t* opts,
@@ -276,8 +281,9 @@ am_status_t am_get_status(const void* workspace, int32_t num_heads,
                           int32_t* per_head, void* stream);
 
 /* Stage timing.  While enabled, every kernel launch made by
- * am_compact_heads is bracketed by CUDA events recorded on the call's stream
- * (event creation is the only host-side cost; no device memory is used).
+ * am_compact_heads (and am_compact_heads_noalloc) is bracketed by CUDA events
+ * that the library creates and records on the launch's stream (event
+ * creation is the only host-side cost; no device memory is used).
  * am_profile_collect() waits for the recorded events, adds up the device time
  * and the launch count per stage into ms[AM_STAGE_COUNT] and
  * launches[AM_STAGE_COUNT] (host arrays, either may be NULL), and clears the

@@ -191,7 +191,9 @@ def test_bf16_correlation_copy_full_size_sampled():
 
 @needs_cuda
 def test_stored_fp32_correlation_ragged_and_full_size():
-    """AM_CORR_STORED_FP32 (the default for bf16 inputs recomputes Φ instead)."""
+    """AM_CORR_STORED_FP32: the correlation pass streams every stored fp32 feature
+    row (the default, AM_CORR_BOUNDED, evaluates only the keys its bound cannot
+    exclude)."""
     import attention_matching_b200 as am
     heads = [W.structured_head(300 + h, n=1000, T=1100) for h in range(3)]
     check_all(heads, [13, 22, 8], 4, 2, label="stored fp32 ragged", corr_mode=am.CORR_STORED_FP32)

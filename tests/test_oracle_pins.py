@@ -184,6 +184,46 @@ def test_nnls_single_column_closed_form():
     assert O.nnls(phi[:, None], -y)[0] == 0.0
 
 
+def test_kkt_checker_flags_points_that_are_not_optimal():
+    """The KKT checker that accepts the GPU's fp64 weights must reject points
+    that are not minimisers.  Closed form first: with A = I and y = (1, -1)
+    the minimiser is x = (1, 0) with gradient g = x - y = (0, 1); at x = 0
+    the first variable has g_0 = -1 off the support (a descent direction),
+    at x = (1.5, 0) it has g_0 = 0.5 on the support, and a negative entry is
+    reported as min_x.  Then perturbations of scipy's minimiser of a random
+    problem: scaling one positive weight, zeroing one, and making a zero one
+    positive each break one condition by far more than the 1e-10 bar."""
+    A = np.eye(2)
+    y = np.array([1.0, -1.0])
+    ok = O.nnls_kkt_residual(A, y, np.array([1.0, 0.0]))
+    assert ok["min_x"] == 0.0 and ok["stationarity"] == 0.0 and ok["dual_feasibility"] == 0.0
+    at0 = O.nnls_kkt_residual(A, y, np.zeros(2))
+    assert abs(at0["dual_feasibility"] - 1.0 / math.sqrt(2.0)) < 1e-15
+    over = O.nnls_kkt_residual(A, y, np.array([1.5, 0.0]))
+    assert abs(over["stationarity"] - 0.5 / math.sqrt(2.0)) < 1e-15
+    assert O.nnls_kkt_residual(A, y, np.array([1.0, -0.25]))["min_x"] == -0.25
+
+    rng = np.random.default_rng(61)
+    A = rng.random((60, 14)) + 0.05 * rng.standard_normal((60, 14))
+    y = A[:, :4] @ rng.uniform(0.5, 2.0, 4) - 0.3 * A[:, 9] + 0.01 * rng.standard_normal(60)
+    x = scipy_nnls(A, y)[0]
+    on, off = np.flatnonzero(x > 0), np.flatnonzero(x == 0)
+    assert on.size and off.size
+    base = O.nnls_kkt_residual(A, y, x)
+    assert base["stationarity"] < 1e-10 and base["dual_feasibility"] < 1e-10
+    bad = x.copy()
+    bad[on[0]] *= 1.01
+    assert O.nnls_kkt_residual(A, y, bad)["stationarity"] > 1e-6
+    bad = x.copy()
+    bad[on[0]] = 0.0
+    assert O.nnls_kkt_residual(A, y, bad)["dual_feasibility"] > 1e-6
+    bad = x.copy()
+    g = A.T @ (A @ x - y)
+    j = off[np.argmax(g[off])]          # the zero weight whose gradient is most positive
+    bad[j] = 0.1
+    assert O.nnls_kkt_residual(A, y, bad)["stationarity"] > 1e-6
+
+
 def test_nnls_kkt_on_exp_features():
     """Mass-fit-shaped problem (positive, correlated columns)."""
     h = W.iid_head(7, n=128, T=40, d=16, dtype="fp32")
@@ -290,6 +330,32 @@ def test_omp_lazy_refit_reading():
     S81, w81, _ = O.omp_select(Phi, m, 30, 8, 1)
     assert S42 == S81
     np.testing.assert_allclose(w42, w81, rtol=1e-12)
+
+
+def test_best_subset_sixteen_keys_known_optimum():
+    """Exhaustive search over T = 16 keys on a problem whose optimum is known
+    by construction: m is an exact positive combination of three columns of a
+    positive Φ, so that subset fits with zero residual while no other subset
+    of three generic columns can.  The search must return it, and its
+    residual must equal the minimum over all subsets computed independently
+    with scipy's NNLS; OMP's residual is never below it."""
+    rng = np.random.default_rng(77)
+    n, T, t = 40, 16, 3
+    Phi = rng.uniform(0.05, 1.0, (n, T))
+    S_true = [2, 9, 13]
+    m = Phi[:, S_true] @ np.array([0.7, 1.9, 0.4])
+    res, S = O.best_subset(Phi, m, t)
+    assert S == S_true and res < 1e-12
+    indep = min(np.linalg.norm(m - Phi[:, list(c)] @ scipy_nnls(Phi[:, list(c)], m)[0])
+                for c in itertools.combinations(range(T), t)) / np.linalg.norm(m)
+    assert abs(res - indep) < 1e-12
+    for k in (1, 2):
+        res_k, S_k = O.best_subset(Phi, m, k)
+        indep_k = min(np.linalg.norm(m - Phi[:, list(c)] @ scipy_nnls(Phi[:, list(c)], m)[0])
+                      for c in itertools.combinations(range(T), k)) / np.linalg.norm(m)
+        assert abs(res_k - indep_k) < 1e-12
+        Somp, w, _ = O.omp_select(Phi, m, k, 1, 1)
+        assert res_k <= O.mass_residual(Phi, m, Somp, w) + 1e-12
 
 
 def test_omp_greedy_never_beats_best_subset():

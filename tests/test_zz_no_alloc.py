@@ -80,7 +80,7 @@ def test_noalloc_matches_ordinary_entry_point_twice(label, make, budgets, topk, 
         ref = am.compact_heads(Q, K, V, budgets, topk=topk, refit_every=refit)
         assert torch.equal(out["indices"], ref["indices"]), label
         assert torch.equal(out["C_k"], ref["C_k"]), label
-        torch.testing.assert_close(out["beta"], ref["beta"], rtol=0, atol=1e-3)
+        assert torch.equal(out["beta"], ref["beta"]), label
         torch.testing.assert_close(out["C_v"], ref["C_v"], rtol=1e-5, atol=1e-6)
 
 
@@ -92,6 +92,8 @@ def test_noalloc_rejects_problems_beyond_the_scratch():
     H, n, T, d = 1, 2048, 2048, 128
     b = (ctypes.c_int32 * 1)(40)
     offs = (ctypes.c_int64 * 2)(0, 40)
-    rc = _noalloc()(1 << 20, 1 << 21, 1 << 22, n, T, d, H, b, ctypes.byref(opts), offs,
-                    1 << 23, 1 << 24, 1 << 25, 1 << 26, None, None)
+    # every device pointer is null: the size check answers first, and were it
+    # ever skipped the null-argument check would stop the call before any launch
+    rc = _noalloc()(None, None, None, n, T, d, H, b, ctypes.byref(opts), offs,
+                    None, None, None, None, None, None)
     assert rc == 3   # AM_ERR_WORKSPACE, returned before any GPU work
