@@ -68,6 +68,8 @@ class AmOpts(ctypes.Structure):
         ("residual_out", ctypes.c_void_p),
         ("w_out", ctypes.c_void_p),
         ("select_mode", ctypes.c_int32),
+        ("reserved0", ctypes.c_int32),
+        ("key_offsets", ctypes.c_void_p),
     ]
 
 
@@ -90,6 +92,9 @@ def lib() -> ctypes.CDLL:
         L.am_workspace_size.argtypes = [c_int, c_int, c_int, c_int, P_i32, ctypes.POINTER(AmOpts),
                                         ctypes.POINTER(c_size_t)]
         L.am_workspace_size.restype = c_int
+        L.am_workspace_size_waves.argtypes = [c_int, c_int, c_int, c_int, P_i32, ctypes.POINTER(AmOpts), c_int,
+                                              ctypes.POINTER(c_size_t)]
+        L.am_workspace_size_waves.restype = c_int
         L.am_compact_heads.argtypes = [c_void_p, c_void_p, c_void_p, c_int, c_int, c_int, c_int, P_i32,
                                        ctypes.POINTER(AmOpts), c_void_p, c_size_t, P_i64,
                                        c_void_p, c_void_p, c_void_p, c_void_p, c_void_p]
@@ -138,10 +143,17 @@ def make_opts(dtype: int = BF16, topk: int = 1, refit_every: int = 1, scale: flo
     return o
 
 
-def workspace_size(n: int, T: int, d: int, budgets: Sequence[int], opts: AmOpts) -> int:
+def workspace_size(n: int, T: int, d: int, budgets: Sequence[int], opts: AmOpts,
+                   wave_heads: Optional[int] = None) -> int:
+    """Workspace bytes for one call: every head in one wave, or (wave_heads)
+    waves of at most that many consecutive heads through the same memory."""
     out = ctypes.c_size_t(0)
-    rc = lib().am_workspace_size(n, T, d, len(budgets), _i32_array(budgets), ctypes.byref(opts),
-                                 ctypes.byref(out))
+    if wave_heads is None:
+        rc = lib().am_workspace_size(n, T, d, len(budgets), _i32_array(budgets), ctypes.byref(opts),
+                                     ctypes.byref(out))
+    else:
+        rc = lib().am_workspace_size_waves(n, T, d, len(budgets), _i32_array(budgets), ctypes.byref(opts),
+                                           int(wave_heads), ctypes.byref(out))
     if rc:
         raise AmError(rc, "am_workspace_size")
     return int(out.value)
@@ -188,18 +200,24 @@ def compact_heads(Q, K, V, budgets: Sequence[int], topk: int = 1, refit_every: i
                   shift=None, key_bias=None, ridge: float = 1e-6, w_floor_rel: float = 1e-12,
                   scale: float = 0.0, nnls_max_iter: int = 0, workspace=None, trace: bool = False,
                   stream=None, check: bool = True, corr_mode: int = CORR_AUTO,
-                  select_mode: int = SELECT_OMP) -> Dict:
+                  select_mode: int = SELECT_OMP, key_offsets: Optional[Sequence[int]] = None,
+                  wave_heads: Optional[int] = None) -> Dict:
     """Compact H heads on the GPU.
 
     Q [H, n, d], K [H, T, d], V [H, T, d]: contiguous tensors, bf16 or fp32,
     all on the current CUDA device or all on the host (then copied in, and the
-    outputs copied back to the host).
-    budgets: H ints in [1, T].  shift [H] fp32 and key_bias [H, T] fp32 are
+    outputs copied back to the host).  With ``key_offsets`` (H + 1 ints,
+    starting at 0) head h has T_h = key_offsets[h+1] − key_offsets[h] keys and
+    K, V are packed [Σ T_h, d] (key_bias packed [Σ T_h]).
+    budgets: H ints in [1, T_h].  shift [H] fp32 and key_bias [H, T] fp32 are
     optional CUDA tensors.  select_mode SELECT_HIGHEST keeps each head's t
     keys of largest total attention instead of the OMP picks (topk,
-    refit_every and corr_mode are then ignored).  Returns a dict of CUDA tensors in the packed
-    varlen layout (C_k, beta, C_v, indices, cu_t) plus, with ``trace``, the
-    pick order, pick correlations, shift used, mass residual and weights.
+    refit_every and corr_mode are then ignored).  ``wave_heads`` sizes an
+    allocated workspace for waves of at most that many heads (a workspace
+    passed in decides the waves by its own size).  Returns a dict of CUDA
+    tensors in the packed varlen layout (C_k, beta, C_v, indices, cu_t) plus,
+    with ``trace``, the pick order, pick correlations, shift used, mass
+    residual and weights.
     """
     import torch
     host = not (Q.is_cuda or K.is_cuda or V.is_cuda)
@@ -210,9 +228,19 @@ def compact_heads(Q, K, V, budgets: Sequence[int], topk: int = 1, refit_every: i
     if not (Q.is_cuda and K.is_cuda and V.is_cuda):
         raise ValueError("Q, K, V must all be CUDA tensors or all host tensors")
     H, n, d = Q.shape
-    T = K.shape[1]
-    if K.shape != (H, T, d) or V.shape != (H, T, d) or len(budgets) != H:
-        raise ValueError("shape mismatch")
+    if key_offsets is None:
+        T = K.shape[1]
+        if K.shape != (H, T, d) or V.shape != (H, T, d) or len(budgets) != H:
+            raise ValueError("shape mismatch")
+        koffs = None
+    else:
+        ko = [int(x) for x in key_offsets]
+        if len(ko) != H + 1 or ko[0] != 0 or len(budgets) != H:
+            raise ValueError("key_offsets must hold H + 1 offsets starting at 0")
+        T = max(ko[h + 1] - ko[h] for h in range(H))
+        if K.shape != (ko[-1], d) or V.shape != (ko[-1], d):
+            raise ValueError("with key_offsets, K and V are packed [sum T_h, d]")
+        koffs = (ctypes.c_int64 * (H + 1))(*ko)
     if Q.dtype != K.dtype or Q.dtype != V.dtype or Q.dtype not in (torch.bfloat16, torch.float32):
         raise ValueError("Q, K, V must share dtype bf16 or fp32")
     for t in (Q, K, V):
@@ -221,6 +249,8 @@ def compact_heads(Q, K, V, budgets: Sequence[int], topk: int = 1, refit_every: i
     dt = BF16 if Q.dtype == torch.bfloat16 else FP32
     dev = Q.device
     opts = make_opts(dt, topk, refit_every, scale, ridge, w_floor_rel, nnls_max_iter, corr_mode, select_mode)
+    if koffs is not None:
+        opts.key_offsets = ctypes.cast(koffs, ctypes.c_void_p)
     if shift is not None:
         shift = shift.to(device=dev, dtype=torch.float32).contiguous()
         opts.shift = shift.data_ptr()
@@ -249,9 +279,9 @@ def compact_heads(Q, K, V, budgets: Sequence[int], topk: int = 1, refit_every: i
         opts.shift_out = out["shift"].data_ptr()
         opts.residual_out = out["residual"].data_ptr()
         opts.w_out = out["w"].data_ptr()
-    need = workspace_size(n, T, d, budgets, opts)
-    if workspace is None or workspace.numel() * workspace.element_size() < need:
-        workspace = torch.empty((need,), dtype=torch.uint8, device=dev)
+    if workspace is None:
+        workspace = torch.empty((workspace_size(n, T, d, budgets, opts, wave_heads),), dtype=torch.uint8,
+                                device=dev)
     offs = (ctypes.c_int64 * (H + 1))(*cu)
     if stream is None:
         stream = torch.cuda.current_stream(dev).cuda_stream

@@ -3,11 +3,17 @@
 // One call compacts H independent heads (the per-(layer, KV-head) problems of
 // "Fast KV Compaction via Attention Matching", zhichai.net deep dive §1.6;
 // varlen packing of non-uniform budgets per the zhichai.net/en summary,
-// "Engineering Practicality").  All work is ordered after the caller's stream
-// and the caller's stream waits for all of it; no device memory is allocated
-// here.  The OMP passes of different head groups run on internal streams of
-// their own (the heads are independent), so one group's latency-bound
-// refits overlap another group's bandwidth-bound passes.
+// "Engineering Practicality"; per-head key counts for KV-based chunking of a
+// long context, xinfinite.net article §3).  All work is ordered after the
+// caller's stream and the caller's stream waits for all of it; no device
+// memory is allocated here.  The OMP passes of different head groups run on
+// internal streams of their own (the heads are independent), so one group's
+// latency-bound refits overlap another group's bandwidth-bound passes.
+//
+// Workspace: a prefix (header, every head's status word, the device tables
+// of every wave), then one wave's region.  When the caller's workspace holds
+// fewer heads than the call has, the heads run in waves of consecutive heads
+// through that one region, each wave as many heads as fit.
 #include "am_internal.cuh"
 
 #include <math.h>
@@ -39,6 +45,8 @@ struct Layout {
 
 struct Tables {
   std::vector<int32_t> t;
+  std::vector<int32_t> Th;        // key count per head
+  std::vector<int64_t> koff;      // [H+1] first key row per head (relative to the first head's)
   std::vector<int64_t> cu_t, cu_t2;
   std::vector<int32_t> order;
   std::vector<int> active;   // active heads per pass
@@ -56,14 +64,22 @@ bool bf16_copy(const am_opts_t* o) {
   return o->corr_mode == AM_CORR_STORED_BF16 && o->select_mode == AM_SELECT_OMP;
 }
 
-Layout plan(int n, int T, int d, int H, int64_t sum_t, int64_t sum_t2, bool corr_bf16) {
+// Bytes of one wave's device tables: cu_t, cu_t2, koff [H+1] int64 and
+// t, Th, order, group order [H] int32 (a multiple of 8).
+size_t table_bytes(int H) { return (size_t)(H + 1) * 8 * 3 + (size_t)H * 4 * 4; }
+
+// The workspace prefix for a call of H heads: header, H status words, and a
+// tables region that holds every wave's tables (Σ over waves of
+// table_bytes(H_w) <= 64·H bytes for any split into waves).
+size_t prefix_bytes(int H) { return align_up(kWsHeaderBytes + (size_t)H * 4) + align_up((size_t)H * 64 + 256); }
+
+// One wave's region, from byte `o0` (the end of the prefix) on.
+Layout plan(int n, int T, int d, int H, int64_t sum_t, int64_t sum_t2, bool corr_bf16, size_t o0) {
   Layout L{};
   const size_t ldn = (size_t)round_up(n, 32);
-  size_t o = 0;
+  size_t o = o0;
   auto take = [&](size_t bytes) { size_t at = o; o = align_up(o + bytes); return at; };
-  L.status = take(kWsHeaderBytes + (size_t)H * 4) + kWsHeaderBytes;   // header precedes status
-  L.tables_bytes = (size_t)H * 4 + (size_t)(H + 1) * 8 * 2 + (size_t)H * 4 * 2;
-  L.tables = take(L.tables_bytes);
+  L.tables_bytes = table_bytes(H);
   L.shift = take((size_t)H * 4);
   L.np = take((size_t)H * 4);
   L.ylen = take((size_t)H * 4);
@@ -115,6 +131,12 @@ Layout plan(int n, int T, int d, int H, int64_t sum_t, int64_t sum_t2, bool corr
 }
 
 void set_groups(Tables* tb, const std::vector<int>& passes, int G);
+void finish_tables(Tables* tb, int kR);
+
+// Key rows per pass of greedy selection (or per refit of pre-selected keys).
+int picks_per_pass(const am_opts_t* o) {
+  return o->select_mode == AM_SELECT_HIGHEST ? kHighestChunk : o->topk * o->refit_every;
+}
 
 am_status_t check_shape(int n, int T, int d, int H, const int32_t* budgets, const am_opts_t* opts,
                         Tables* tb) {
@@ -136,15 +158,47 @@ am_status_t check_shape(int n, int T, int d, int H, const int32_t* budgets, cons
     return AM_ERR_UNSUPPORTED;
   if ((int64_t)n * d > (1ll << 31) || (int64_t)T * round_up(n, 32) > (1ll << 40))
     return AM_ERR_UNSUPPORTED;
+  if (opts->reserved0 != 0) return AM_ERR_INVALID_ARG;
   const int kR = highest ? kHighestChunk : opts->topk * opts->refit_every;
   tb->t.assign(budgets, budgets + H);
-  tb->cu_t.assign(H + 1, 0);
-  tb->cu_t2.assign(H + 1, 0);
-  std::vector<int> passes(H);
+  tb->Th.assign(H, T);
+  tb->koff.assign(H + 1, 0);
+  if (opts->key_offsets) {
+    const int64_t* ko = opts->key_offsets;
+    if (ko[0] != 0) return AM_ERR_INVALID_ARG;
+    int tmax = 0;
+    for (int h = 0; h < H; ++h) {
+      const int64_t th = ko[h + 1] - ko[h];
+      if (th < 1 || th > T) return AM_ERR_INVALID_ARG;
+      tb->Th[h] = (int)th;
+      tmax = std::max(tmax, (int)th);
+    }
+    if (tmax != T) return AM_ERR_INVALID_ARG;
+    for (int h = 0; h <= H; ++h) tb->koff[h] = ko[h];
+  } else {
+    for (int h = 0; h <= H; ++h) tb->koff[h] = (int64_t)h * T;
+  }
+  // the feature passes address key rows with 32-bit tensor-map coordinates
+  if (tb->koff[H] > (int64_t)INT32_MAX - 256) return AM_ERR_UNSUPPORTED;
   for (int h = 0; h < H; ++h) {
     const int t = budgets[h];
-    if (t < 1 || t > T) return AM_ERR_BUDGET;
+    if (t < 1 || t > tb->Th[h]) return AM_ERR_BUDGET;
     if (t > kMaxBudget) return AM_ERR_UNSUPPORTED;
+  }
+  finish_tables(tb, kR);
+  return AM_OK;
+}
+
+// From t, Th and koff: the packed offsets, pass counts, the pass order of the
+// heads and the active heads per pass (one group).
+void finish_tables(Tables* tb, int kR) {
+  const int H = (int)tb->t.size();
+  tb->cu_t.assign(H + 1, 0);
+  tb->cu_t2.assign(H + 1, 0);
+  tb->max_t = 0;
+  std::vector<int> passes(H);
+  for (int h = 0; h < H; ++h) {
+    const int t = tb->t[h];
     tb->cu_t[h + 1] = tb->cu_t[h] + t;
     // t² rounded up to even: every head's t×t regions start 16-byte aligned
     tb->cu_t2[h + 1] = tb->cu_t2[h] + (((int64_t)t * t + 1) & ~(int64_t)1);
@@ -163,7 +217,16 @@ am_status_t check_shape(int n, int T, int d, int H, const int32_t* budgets, cons
     for (int h = 0; h < H; ++h) tb->active[q] += passes[h] > q;
   tb->passes = passes;
   set_groups(tb, passes, 1);
-  return AM_OK;
+}
+
+// Heads [h0, h1) of `all` as a problem of their own (key rows relative to
+// head h0's first row).
+void sub_tables(const Tables& all, int h0, int h1, int kR, Tables* tw) {
+  tw->t.assign(all.t.begin() + h0, all.t.begin() + h1);
+  tw->Th.assign(all.Th.begin() + h0, all.Th.begin() + h1);
+  tw->koff.resize(h1 - h0 + 1);
+  for (int h = h0; h <= h1; ++h) tw->koff[h - h0] = all.koff[h] - all.koff[h0];
+  finish_tables(tw, kR);
 }
 
 // Splits the pass-ordered heads round-robin into G groups (each group's list
@@ -187,7 +250,6 @@ void set_groups(Tables* tb, const std::vector<int>& passes, int G) {
 Work bind(const Layout& L, char* base, bool corr_bf16) {
   Work w{};
   w.phiT16 = corr_bf16 ? reinterpret_cast<__nv_bfloat16*>(base + L.phiT16) : nullptr;
-  w.status = reinterpret_cast<int32_t*>(base + L.status);
   w.shift = reinterpret_cast<float*>(base + L.shift);
   w.np = reinterpret_cast<int32_t*>(base + L.np);
   w.ylen = reinterpret_cast<int32_t*>(base + L.ylen);
@@ -234,22 +296,30 @@ Work bind(const Layout& L, char* base, bool corr_bf16) {
   return w;
 }
 
-// Packs the host tables in the device order cu_t | cu_t2 | t | order.
+// Appends one wave's tables to `out` in the device order
+// cu_t | cu_t2 | koff | t | Th | order | group order, and points the Work
+// (and *gorder_dev) at where they will sit on the device: `dev` is the
+// device address of the block's first byte.
 void pack_tables(const Tables& tb, int H, std::vector<unsigned char>* out, Work* w, char* dev,
                  int32_t** gorder_dev) {
-  const size_t b_cu = (size_t)(H + 1) * 8;
-  out->resize(2 * b_cu + 3 * (size_t)H * 4);
-  unsigned char* o = out->data();
+  const size_t b_cu = (size_t)(H + 1) * 8, b_h = (size_t)H * 4;
+  const size_t at = out->size();
+  out->resize(at + table_bytes(H));
+  unsigned char* o = out->data() + at;
   memcpy(o, tb.cu_t.data(), b_cu);
   memcpy(o + b_cu, tb.cu_t2.data(), b_cu);
-  memcpy(o + 2 * b_cu, tb.t.data(), (size_t)H * 4);
-  memcpy(o + 2 * b_cu + (size_t)H * 4, tb.order.data(), (size_t)H * 4);
-  memcpy(o + 2 * b_cu + (size_t)H * 8, tb.gorder.data(), (size_t)H * 4);
+  memcpy(o + 2 * b_cu, tb.koff.data(), b_cu);
+  memcpy(o + 3 * b_cu, tb.t.data(), b_h);
+  memcpy(o + 3 * b_cu + b_h, tb.Th.data(), b_h);
+  memcpy(o + 3 * b_cu + 2 * b_h, tb.order.data(), b_h);
+  memcpy(o + 3 * b_cu + 3 * b_h, tb.gorder.data(), b_h);
   w->cu_t = reinterpret_cast<int64_t*>(dev);
   w->cu_t2 = reinterpret_cast<int64_t*>(dev + b_cu);
-  w->t = reinterpret_cast<int32_t*>(dev + 2 * b_cu);
-  w->order = reinterpret_cast<int32_t*>(dev + 2 * b_cu + (size_t)H * 4);
-  *gorder_dev = reinterpret_cast<int32_t*>(dev + 2 * b_cu + (size_t)H * 8);
+  w->koff = reinterpret_cast<int64_t*>(dev + 2 * b_cu);
+  w->t = reinterpret_cast<int32_t*>(dev + 3 * b_cu);
+  w->Th = reinterpret_cast<int32_t*>(dev + 3 * b_cu + b_h);
+  w->order = reinterpret_cast<int32_t*>(dev + 3 * b_cu + 2 * b_h);
+  *gorder_dev = reinterpret_cast<int32_t*>(dev + 3 * b_cu + 3 * b_h);
 }
 
 // Internal streams for the head groups, created once per device.
@@ -285,6 +355,7 @@ Problem make_problem(int n, int T, int d, int H, const am_opts_t* o, const Table
   p.corr_recompute = o->corr_mode == AM_CORR_RECOMPUTE;
   p.corr_bounded = !p.select_highest && (o->corr_mode == AM_CORR_BOUNDED || o->corr_mode == AM_CORR_AUTO);
   if (p.select_highest) p.corr_recompute = false;
+  p.key_rows = tb.koff[H];
   return p;
 }
 
@@ -292,6 +363,31 @@ struct WsHeader {
   uint32_t magic;
   int32_t H;
 };
+
+// Size of the wave region for heads [h0, h1) of `tb`.
+size_t wave_bytes(const Tables& tb, int n, int T, int d, int h0, int h1, bool corr_bf16) {
+  const int64_t st = tb.cu_t[h1] - tb.cu_t[h0], st2 = tb.cu_t2[h1] - tb.cu_t2[h0];
+  return plan(n, T, d, h1 - h0, st, st2, corr_bf16, 0).total;
+}
+
+// Waves of consecutive heads: each takes as many heads as fit in `region`
+// bytes.  Empty when one head does not fit.
+std::vector<std::pair<int, int>> plan_waves(const Tables& tb, int n, int T, int d, bool corr_bf16, size_t region) {
+  const int H = (int)tb.t.size();
+  std::vector<std::pair<int, int>> waves;
+  int h0 = 0;
+  while (h0 < H) {
+    int h1 = h0;
+    while (h1 < H && wave_bytes(tb, n, T, d, h0, h1 + 1, corr_bf16) <= region) ++h1;
+    if (h1 == h0) return {};
+    waves.emplace_back(h0, h1);
+    h0 = h1;
+  }
+  return waves;
+}
+
+const char* cbyte(const void* p, int64_t off) { return reinterpret_cast<const char*>(p) + off; }
+char* mbyte(void* p, int64_t off) { return reinterpret_cast<char*>(p) + off; }
 
 }  // namespace
 }  // namespace am
@@ -315,11 +411,23 @@ am_status_t am_default_opts(am_opts_t* opts) {
 
 am_status_t am_workspace_size(int32_t n, int32_t T, int32_t d, int32_t num_heads,
                               const int32_t* budgets, const am_opts_t* opts, size_t* bytes) {
-  if (!bytes) return AM_ERR_INVALID_ARG;
+  return am_workspace_size_waves(n, T, d, num_heads, budgets, opts, num_heads, bytes);
+}
+
+am_status_t am_workspace_size_waves(int32_t n, int32_t T, int32_t d, int32_t num_heads,
+                                    const int32_t* budgets, const am_opts_t* opts, int32_t wave_heads,
+                                    size_t* bytes) {
+  if (!bytes || wave_heads < 1) return AM_ERR_INVALID_ARG;
   Tables tb;
   am_status_t st = check_shape(n, T, d, num_heads, budgets, opts, &tb);
   if (st != AM_OK) return st;
-  *bytes = plan(n, T, d, num_heads, tb.sum_t, tb.sum_t2, bf16_copy(opts)).total;
+  // the largest region over every window of wave_heads consecutive heads, so
+  // that the call's waves (each as many heads as fit) hold wave_heads heads
+  const int W = std::min(wave_heads, num_heads);
+  size_t region = 0;
+  for (int h0 = 0; h0 + W <= num_heads; ++h0)
+    region = std::max(region, wave_bytes(tb, n, T, d, h0, h0 + W, bf16_copy(opts)));
+  *bytes = prefix_bytes(num_heads) + region;
   return AM_OK;
 }
 
@@ -329,7 +437,7 @@ am_status_t am_workspace_view(int32_t n, int32_t T, int32_t d, int32_t num_heads
   Tables tb;
   am_status_t st = check_shape(n, T, d, num_heads, budgets, opts, &tb);
   if (st != AM_OK) return st;
-  const Layout L = plan(n, T, d, num_heads, tb.sum_t, tb.sum_t2, bf16_copy(opts));
+  const Layout L = plan(n, T, d, num_heads, tb.sum_t, tb.sum_t2, bf16_copy(opts), prefix_bytes(num_heads));
   view->phiT = L.phiT;
   view->mass = L.m;
   view->target = L.Y;
@@ -354,62 +462,46 @@ am_status_t am_compact_heads(const void* Q, const void* K, const void* V, int32_
 }  // extern "C"
 
 namespace am {
-am_status_t compact_heads_impl(const void* Q, const void* K, const void* V, int32_t n, int32_t T, int32_t d,
-                               int32_t H, const int32_t* budgets, const am_opts_t* opts, void* workspace,
-                               size_t workspace_bytes, const int64_t* out_offsets, void* C_k, float* beta,
-                               float* C_v, int32_t* indices, void* stream, int max_groups) {
-  if (!Q || !K || !V || !C_k || !beta || !C_v || !indices || !out_offsets) return AM_ERR_INVALID_ARG;
-  Tables tb;
-  am_status_t st = check_shape(n, T, d, H, budgets, opts, &tb);
-  if (st != AM_OK) return st;
-  // head groups on internal streams (one group: everything on the caller's stream)
-  int G = std::max(1, std::min(max_groups, H));
-  for (int g = 0; g < G && G > 1; ++g)
-    if (!group_stream(g)) G = 1;
-  set_groups(&tb, tb.passes, G);
-  for (int h = 0; h <= H; ++h)
-    if (out_offsets[h] != tb.cu_t[h]) return AM_ERR_INVALID_ARG;
-  if (!workspace || ((uintptr_t)workspace % kAlign) != 0) return AM_ERR_WORKSPACE;
-  const Layout L = plan(n, T, d, H, tb.sum_t, tb.sum_t2, bf16_copy(opts));
-  if (workspace_bytes < L.total) return AM_ERR_WORKSPACE;
 
-  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  char* base = reinterpret_cast<char*>(workspace);
-  Work w = bind(L, base, bf16_copy(opts));
-  w.nrm_ata = tb.sum_t2;
-  w.nrm_stride = tb.sum_t2 + tb.sum_t * d;
-  std::vector<unsigned char> host_tables;
-  int32_t* gorder = nullptr;
-  pack_tables(tb, H, &host_tables, &w, base + L.tables, &gorder);
-  const Problem p = make_problem(n, T, d, H, opts, tb);
-
-  WsHeader hdr{kWsMagic, H};
 #define AM_TRY(x)                      \
   do {                                 \
     if ((x) != cudaSuccess) return AM_ERR_CUDA; \
   } while (0)
-  // Pageable sources: both copies are staged before cudaMemcpyAsync returns.
-  AM_TRY(cudaMemcpyAsync(base, &hdr, sizeof(hdr), cudaMemcpyHostToDevice, s));
-  AM_TRY(cudaMemcpyAsync(base + L.tables, host_tables.data(), host_tables.size(),
-                         cudaMemcpyHostToDevice, s));
-  AM_TRY(cudaMemsetAsync(w.status, 0, (size_t)H * 4, s));
 
+// Outputs and optional inputs of one wave, already offset to its first head.
+struct WaveIO {
+  const void *Q, *K, *V;
+  const float* key_bias;
+  const float* shift_in;
+  void* C_k;
+  float *beta, *C_v;
+  int32_t* indices;
+  int32_t* pick_order;
+  float *pick_corr, *w_out, *shift_out;
+  double* residual_out;
+};
+
+// The compaction of one wave of heads, on stream s (internal group streams
+// forked from and joined back into s).
+am_status_t run_wave(const Problem& p, Work w, const Tables& tb, int G, int32_t* gorder, const WaveIO& io,
+                     cudaStream_t s) {
+  const int H = p.H;
   const bool tc = phi_tc_supported(p);
   if (!tc || !p.corr_bounded) w.cnpart = nullptr;   // column norms from the features instead
-  if (opts->shift) {
-    AM_TRY(launch_shift_copy(opts->shift, w.shift, H, s));
+  if (io.shift_in) {
+    AM_TRY(launch_shift_copy(io.shift_in, w.shift, H, s));
   } else if (tc) {
     AM_TRY(launch_shift_init(w.shift, H, s));
-    AM_TRY(launch_shift_max_tc(p, Q, K, opts->key_bias, w, reinterpret_cast<uint32_t*>(w.shift), s));
+    AM_TRY(launch_shift_max_tc(p, io.Q, io.K, io.key_bias, w, reinterpret_cast<uint32_t*>(w.shift), s));
     AM_TRY(launch_shift_decode(w.shift, H, s));
   } else {
-    AM_TRY(launch_shift_max(p, Q, K, opts->key_bias, w.shift, s));
+    AM_TRY(launch_shift_max(p, w, io.Q, io.K, io.key_bias, w.shift, s));
   }
   if (tc) {
-    AM_TRY(launch_phi_tc(p, Q, K, V, opts->key_bias, w, s));
+    AM_TRY(launch_phi_tc(p, io.Q, io.K, io.V, io.key_bias, w, s));
   } else {
-    AM_TRY(launch_phi(p, Q, K, opts->key_bias, w, s));
-    AM_TRY(launch_y_m(p, V, w, s));
+    AM_TRY(launch_phi(p, io.Q, io.K, io.key_bias, w, s));
+    AM_TRY(launch_y_m(p, io.V, w, s));
   }
   AM_TRY(launch_omp_init(p, w, s));
   if (p.corr_bounded) AM_TRY(launch_column_norms(p, w, s));
@@ -419,7 +511,7 @@ am_status_t compact_heads_impl(const void* Q, const void* K, const void* V, int3
   AM_TRY(cudaMemsetAsync(w.cprefix, 0, (size_t)H * 4, s));
   AM_TRY(cudaMemsetAsync(w.ccount, 0, (size_t)H * 4, s));
   if (p.select_highest) AM_TRY(launch_select_highest(p, w, s));
-  const CorrInputs cin{Q, K, opts->key_bias};
+  const CorrInputs cin{io.Q, io.K, io.key_bias};
   if (G == 1) {
     for (int pass = 0; pass < (int)tb.active.size(); ++pass)
       AM_TRY(launch_omp_pass(p, w, pass, tb.active[pass], cin, s));
@@ -447,14 +539,89 @@ am_status_t compact_heads_impl(const void* Q, const void* K, const void* V, int3
     }
     cudaEventDestroy(fork);
   }
-  if (opts->residual_out) AM_TRY(launch_residual_norm(p, w, opts->residual_out, s));
-  AM_TRY(launch_finalize(p, w, K, opts->key_bias, C_k, beta, indices, opts->w_out, opts->pick_order,
-                         opts->pick_corr, s));
-  AM_TRY(launch_value_fit(p, w, C_v, s));
-  if (opts->shift_out) AM_TRY(launch_shift_copy(w.shift, opts->shift_out, H, s));
-#undef AM_TRY
+  if (io.residual_out) AM_TRY(launch_residual_norm(p, w, io.residual_out, s));
+  AM_TRY(launch_finalize(p, w, io.K, io.key_bias, io.C_k, io.beta, io.indices, io.w_out, io.pick_order,
+                         io.pick_corr, s));
+  AM_TRY(launch_value_fit(p, w, io.C_v, s));
+  if (io.shift_out) AM_TRY(launch_shift_copy(w.shift, io.shift_out, H, s));
   return AM_OK;
 }
+
+am_status_t compact_heads_impl(const void* Q, const void* K, const void* V, int32_t n, int32_t T, int32_t d,
+                               int32_t H, const int32_t* budgets, const am_opts_t* opts, void* workspace,
+                               size_t workspace_bytes, const int64_t* out_offsets, void* C_k, float* beta,
+                               float* C_v, int32_t* indices, void* stream, int max_groups) {
+  if (!Q || !K || !V || !C_k || !beta || !C_v || !indices || !out_offsets) return AM_ERR_INVALID_ARG;
+  Tables tb;
+  am_status_t st = check_shape(n, T, d, H, budgets, opts, &tb);
+  if (st != AM_OK) return st;
+  for (int h = 0; h <= H; ++h)
+    if (out_offsets[h] != tb.cu_t[h]) return AM_ERR_INVALID_ARG;
+  if (!workspace || ((uintptr_t)workspace % kAlign) != 0) return AM_ERR_WORKSPACE;
+  const bool bf16 = bf16_copy(opts);
+  const size_t pre = prefix_bytes(H);
+  if (workspace_bytes <= pre) return AM_ERR_WORKSPACE;
+  const std::vector<std::pair<int, int>> waves = plan_waves(tb, n, T, d, bf16, workspace_bytes - pre);
+  if (waves.empty()) return AM_ERR_WORKSPACE;
+  // head groups on internal streams (one group: everything on the caller's stream)
+  int G = std::max(1, std::min(max_groups, H));
+  for (int g = 0; g < G && G > 1; ++g)
+    if (!group_stream(g)) G = 1;
+
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  char* base = reinterpret_cast<char*>(workspace);
+  const int kR = picks_per_pass(opts);
+  const size_t esz = opts->in_dtype == AM_BF16 ? 2 : 4;
+  // every wave's tables, packed into one host block and copied once
+  const size_t tables_at = align_up(kWsHeaderBytes + (size_t)H * 4);
+  std::vector<unsigned char> host_tables;
+  std::vector<Tables> wt(waves.size());
+  std::vector<Work> ww(waves.size());
+  std::vector<int32_t*> wgorder(waves.size());
+  for (size_t k = 0; k < waves.size(); ++k) {
+    const int h0 = waves[k].first, h1 = waves[k].second, Hw = h1 - h0;
+    sub_tables(tb, h0, h1, kR, &wt[k]);
+    set_groups(&wt[k], wt[k].passes, std::min(G, Hw));
+    const Layout L = plan(n, T, d, Hw, wt[k].sum_t, wt[k].sum_t2, bf16, pre);
+    ww[k] = bind(L, base, bf16);
+    ww[k].status = reinterpret_cast<int32_t*>(base + kWsHeaderBytes) + h0;
+    ww[k].nrm_ata = wt[k].sum_t2;
+    ww[k].nrm_stride = wt[k].sum_t2 + wt[k].sum_t * d;
+    pack_tables(wt[k], Hw, &host_tables, &ww[k], base + tables_at + host_tables.size(), &wgorder[k]);
+  }
+  if (host_tables.size() > pre - tables_at) return AM_ERR_WORKSPACE;   // cannot happen: 64 bytes per head
+
+  WsHeader hdr{kWsMagic, H};
+  // Pageable sources: both copies are staged before cudaMemcpyAsync returns.
+  AM_TRY(cudaMemcpyAsync(base, &hdr, sizeof(hdr), cudaMemcpyHostToDevice, s));
+  AM_TRY(cudaMemcpyAsync(base + tables_at, host_tables.data(), host_tables.size(), cudaMemcpyHostToDevice, s));
+  AM_TRY(cudaMemsetAsync(base + kWsHeaderBytes, 0, (size_t)H * 4, s));
+
+  for (size_t k = 0; k < waves.size(); ++k) {
+    const int h0 = waves[k].first, h1 = waves[k].second, Hw = h1 - h0;
+    const Problem p = make_problem(n, T, d, Hw, opts, wt[k]);
+    const int64_t krow = tb.koff[h0], orow = tb.cu_t[h0];
+    WaveIO io{};
+    io.Q = cbyte(Q, (int64_t)h0 * n * d * (int64_t)esz);
+    io.K = cbyte(K, krow * d * (int64_t)esz);
+    io.V = cbyte(V, krow * d * (int64_t)esz);
+    io.key_bias = opts->key_bias ? opts->key_bias + krow : nullptr;
+    io.shift_in = opts->shift ? opts->shift + h0 : nullptr;
+    io.C_k = mbyte(C_k, orow * d * (int64_t)esz);
+    io.beta = beta + orow;
+    io.C_v = C_v + orow * d;
+    io.indices = indices + orow;
+    io.pick_order = opts->pick_order ? opts->pick_order + orow : nullptr;
+    io.pick_corr = opts->pick_corr ? opts->pick_corr + orow : nullptr;
+    io.w_out = opts->w_out ? opts->w_out + orow : nullptr;
+    io.shift_out = opts->shift_out ? opts->shift_out + h0 : nullptr;
+    io.residual_out = opts->residual_out ? opts->residual_out + h0 : nullptr;
+    st = run_wave(p, ww[k], wt[k], std::min(G, Hw), wgorder[k], io, s);
+    if (st != AM_OK) return st;
+  }
+  return AM_OK;
+}
+#undef AM_TRY
 }  // namespace am
 
 extern "C" {

@@ -62,6 +62,10 @@ __global__ void __launch_bounds__(256) k_colnorm(Problem p, Work w) {
   const int j = blockIdx.x * 8 + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (j >= p.T) return;
+  if (j >= w.Th[h]) {   // no such key in this head: norm 0, sorted last, never evaluated
+    if (lane == 0) w.cnorm[(int64_t)h * p.T + j] = 0.0;
+    return;
+  }
   const float4* row = reinterpret_cast<const float4*>(w.phiT + ((int64_t)h * p.T + j) * p.ldn);
   const int n4 = p.ldn >> 2;
   double a0 = 0.0, a1 = 0.0;
@@ -83,6 +87,10 @@ __global__ void __launch_bounds__(256) k_normsum(Problem p, Work w) {
   const int h = blockIdx.y;
   const int j = blockIdx.x * blockDim.x + threadIdx.x;
   if (j >= p.T) return;
+  if (j >= w.Th[h]) {   // no such key in this head: norm 0, sorted last, never evaluated
+    w.cnorm[(int64_t)h * p.T + j] = 0.0;
+    return;
+  }
   const int parts = 4 * ((p.n + 127) / 128);
   const float* src = w.cnpart + (int64_t)h * parts * p.T + j;
   double s = 0.0;
@@ -470,9 +478,10 @@ __global__ void __launch_bounds__(kSelThreads) k_score(Problem p, Work w) {
   const int n4 = p.ldn >> 2;
   const int per = (n4 + kRowSplit - 1) / kRowSplit;
   const int c0 = quarter * per, c1 = min(n4, c0 + per);
+  const int Th = w.Th[h];
   for (int j0 = blockIdx.x * kRowsPerBlock; j0 < p.T; j0 += gridDim.x * kRowsPerBlock) {
     const int j = j0 + slot;
-    const bool on = j < p.T;
+    const bool on = j < Th;
     double a[4] = {0.0, 0.0, 0.0, 0.0};
     if (on) {
       const float4* row = reinterpret_cast<const float4*>(w.phiT + ((int64_t)h * p.T + j) * p.ldn);
@@ -499,8 +508,9 @@ __global__ void __launch_bounds__(kSelThreads) k_score(Problem p, Work w) {
     const double c = warp_sum((a[0] + a[1]) + (a[2] + a[3]));
     if (lane == 0) part[slot][quarter] = c;
     __syncthreads();
-    if (on && quarter == 0 && lane == 0)
-      w.cnorm[(int64_t)h * p.T + j] = (part[slot][0] + part[slot][1]) + (part[slot][2] + part[slot][3]);
+    // a key past the head's own (j >= Th) scores −1, below every real key's score
+    if (j < p.T && quarter == 0 && lane == 0)
+      w.cnorm[(int64_t)h * p.T + j] = on ? (part[slot][0] + part[slot][1]) + (part[slot][2] + part[slot][3]) : -1.0;
     __syncthreads();
   }
 }
@@ -548,7 +558,7 @@ __global__ void __launch_bounds__(kBoundThreads) k_pick_highest(Problem p, Work 
     w.pick_corr[base + l] = (float)key_value(key[l]);
     sel[j] = 1;
   }
-  if (threadIdx.x == 0) w.rows_eval[h] = (unsigned long long)p.T;
+  if (threadIdx.x == 0) w.rows_eval[h] = (unsigned long long)w.Th[h];
 }
 
 int rows_ctas_per_head(int active) {

@@ -20,7 +20,7 @@ constexpr int kCholThreads = 256;
 
 // Problem-wide constants, passed by value to every kernel.
 struct Problem {
-  int H, n, T, d;
+  int H, n, T, d;     // T: the largest key count of a head (the padded per-head stride)
   int ldn;            // leading dimension of per-query rows, n rounded up to 32
   int in_dtype;       // AM_BF16 / AM_FP32
   float scale;        // logit scale
@@ -33,6 +33,7 @@ struct Problem {
   int corr_recompute; // the correlation pass recomputes Φ on the tensor cores
   int corr_bounded;   // the correlation pass computes only keys its bound cannot exclude
   int select_highest; // keys chosen up front by total attention, fed to the refits kR at a time
+  int64_t key_rows;   // rows of K and V (and entries of key_bias) this launch reads: Σ_h Th[h]
 };
 
 // Device pointers into the caller's workspace (see plan_workspace()).
@@ -42,6 +43,8 @@ struct Work {
   int64_t* cu_t;        // [H+1] packed output offsets
   int64_t* cu_t2;       // [H+1] offsets of per-head t×t blocks
   int32_t* order;       // [H] heads sorted by pass count, descending
+  int64_t* koff;        // [H+1] first input key row of each head (K, V, key_bias rows)
+  int32_t* Th;          // [H] key count of each head (<= T); keys j >= Th[h] do not exist
   float* shift;         // [H]
   float* phiT;          // [H][T][ldn] key-major features Φᵀ
   __nv_bfloat16* phiT16; // [H][T][ldn] bf16 copy for the correlation pass (or null)
@@ -106,7 +109,7 @@ constexpr int kNormalMaxSplits = 8;   // query splits of the normal-equation pro
 
 // ---- launchers (each file defines its own) ----
 // feature pass (am_phi_simt.cu)
-cudaError_t launch_shift_max(const Problem& p, const void* Q, const void* K, const float* key_bias,
+cudaError_t launch_shift_max(const Problem& p, const Work& w, const void* Q, const void* K, const float* key_bias,
                              float* shift, cudaStream_t s);
 cudaError_t launch_phi(const Problem& p, const void* Q, const void* K, const float* key_bias,
                        const Work& w, cudaStream_t s);

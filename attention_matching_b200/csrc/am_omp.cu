@@ -43,8 +43,10 @@ __global__ void k_init(Problem p, Work w) {
     w.ylen[h] = 0;
     if (!(acc > 0.0) || !isfinite(acc)) record_status(w.status + h, AM_ERR_NONFINITE);
   }
+  // keys past the head's own count are marked as taken: never candidates
   uint8_t* sel = w.sel + (int64_t)h * p.T;
-  for (int j = threadIdx.x; j < p.T; j += blockDim.x) sel[j] = 0;
+  const int Th = w.Th[h];
+  for (int j = threadIdx.x; j < p.T; j += blockDim.x) sel[j] = j >= Th;
 }
 
 // ----------------------------------------------------------- correlation --
@@ -71,14 +73,15 @@ __global__ void __launch_bounds__(256) k_corr(Problem p, Work w, int pass) {
   if (pass * p.kR >= t) return;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int j0 = blockIdx.x * kCorrRowsPerBlock + warp * kCorrRowsPerWarp;
-  if (j0 >= p.T) return;
+  const int Th = w.Th[h];   // rows past the head's keys are never read
+  if (j0 >= Th) return;
   const float4* r4 = reinterpret_cast<const float4*>(w.r + (int64_t)h * p.ldn);
   float acc[kCorrRowsPerWarp] = {0.f, 0.f, 0.f, 0.f};
   if (w.phiT16) {
     const uint4* rows[kCorrRowsPerWarp];
 #pragma unroll
     for (int q = 0; q < kCorrRowsPerWarp; ++q) {
-      const int j = min(j0 + q, p.T - 1);
+      const int j = min(j0 + q, Th - 1);
       rows[q] = reinterpret_cast<const uint4*>(w.phiT16 + ((int64_t)h * p.T + j) * p.ldn);
     }
     const int n8 = p.ldn >> 3;
@@ -107,7 +110,7 @@ __global__ void __launch_bounds__(256) k_corr(Problem p, Work w, int pass) {
     const float4* rows[kCorrRowsPerWarp];
 #pragma unroll
     for (int q = 0; q < kCorrRowsPerWarp; ++q) {
-      const int j = min(j0 + q, p.T - 1);
+      const int j = min(j0 + q, Th - 1);
       rows[q] = reinterpret_cast<const float4*>(w.phiT + ((int64_t)h * p.T + j) * p.ldn);
     }
     const int n4 = p.ldn >> 2;
@@ -142,7 +145,7 @@ __global__ void __launch_bounds__(256) k_corr(Problem p, Work w, int pass) {
   for (int q = 0; q < kCorrRowsPerWarp; ++q) {
     float v = acc[q];
     for (int o = 16; o; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-    if (lane == 0 && j0 + q < p.T) w.corr[(int64_t)h * p.T + j0 + q] = v;
+    if (lane == 0 && j0 + q < Th) w.corr[(int64_t)h * p.T + j0 + q] = v;
   }
 }
 

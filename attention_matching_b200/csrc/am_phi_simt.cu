@@ -43,18 +43,18 @@ __device__ __forceinline__ void load_tile_T(float (*dst)[TQ + 4], const void* sr
 // One 64×64 tile of s = Q Kᵀ·scale (+ bias): thread (tx, ty) owns queries
 // i0 + 4tx .. +3 and keys j0 + 4ty .. +3.
 __device__ __forceinline__ void tile_logits(const Problem& p, const void* Q, const void* K, int h,
-                                            int i0, int j0, float (*Qs)[TQ + 4],
+                                            int64_t krow0, int Th, int i0, int j0, float (*Qs)[TQ + 4],
                                             float (*Ks)[TK + 4], float acc[4][4]) {
   const int tx = threadIdx.x % 16, ty = threadIdx.x / 16;
 #pragma unroll
   for (int a = 0; a < 4; ++a)
 #pragma unroll
     for (int b = 0; b < 4; ++b) acc[a][b] = 0.f;
-  const int64_t qbase = (int64_t)h * p.n * p.d, kbase = (int64_t)h * p.T * p.d;
+  const int64_t qbase = (int64_t)h * p.n * p.d, kbase = krow0 * p.d;
   for (int k0 = 0; k0 < p.d; k0 += DK) {
     __syncthreads();
     load_tile_T(Qs, Q, qbase, p.n, i0, k0, p.d, p.in_dtype);
-    load_tile_T(Ks, K, kbase, p.T, j0, k0, p.d, p.in_dtype);
+    load_tile_T(Ks, K, kbase, Th, j0, k0, p.d, p.in_dtype);
     __syncthreads();
 #pragma unroll 8
     for (int k = 0; k < DK; ++k) {
@@ -69,21 +69,24 @@ __device__ __forceinline__ void tile_logits(const Problem& p, const void* Q, con
   }
 }
 
-__global__ void __launch_bounds__(256) k_shift_max(Problem p, const void* Q, const void* K,
+__global__ void __launch_bounds__(256) k_shift_max(Problem p, Work w, const void* Q, const void* K,
                                                    const float* key_bias, uint32_t* out) {
   __shared__ __align__(16) float Qs[DK][TQ + 4];
   __shared__ __align__(16) float Ks[DK][TK + 4];
   __shared__ float red[8];
   const int h = blockIdx.z, i0 = blockIdx.x * TQ, j0 = blockIdx.y * TK;
+  const int Th = w.Th[h];
+  const int64_t krow0 = w.koff[h];
+  if (j0 >= Th) return;   // the whole block: no key of this head here
   float acc[4][4];
-  tile_logits(p, Q, K, h, i0, j0, Qs, Ks, acc);
+  tile_logits(p, Q, K, h, krow0, Th, i0, j0, Qs, Ks, acc);
   const int tx = threadIdx.x % 16, ty = threadIdx.x / 16;
   float mx = -FLT_MAX;
 #pragma unroll
   for (int b = 0; b < 4; ++b) {
     int j = j0 + ty * 4 + b;
-    if (j >= p.T) continue;
-    float bj = p.has_bias ? key_bias[(int64_t)h * p.T + j] : 0.f;
+    if (j >= Th) continue;
+    float bj = p.has_bias ? key_bias[krow0 + j] : 0.f;
 #pragma unroll
     for (int a = 0; a < 4; ++a) {
       int i = i0 + tx * 4 + a;
@@ -116,14 +119,17 @@ __global__ void k_shift_copy(const float* src, float* dst, int H) {
 }
 
 // Φᵀ[h][j][i] = exp(s_ij − c_h) for i < n, 0 in the padding n <= i < ldn.
-__global__ void __launch_bounds__(256) k_phi(Problem p, const void* Q, const void* K,
+__global__ void __launch_bounds__(256) k_phi(Problem p, Work w, const void* Q, const void* K,
                                              const float* key_bias, const float* shift,
                                              float* phiT, __nv_bfloat16* phiT16) {
   __shared__ __align__(16) float Qs[DK][TQ + 4];
   __shared__ __align__(16) float Ks[DK][TK + 4];
   const int h = blockIdx.z, i0 = blockIdx.x * TQ, j0 = blockIdx.y * TK;
+  const int Th = w.Th[h];
+  const int64_t krow0 = w.koff[h];
+  if (j0 >= Th) return;   // the whole block: keys past the head's own are never read
   float acc[4][4];
-  tile_logits(p, Q, K, h, i0, j0, Qs, Ks, acc);
+  tile_logits(p, Q, K, h, krow0, Th, i0, j0, Qs, Ks, acc);
   const int tx = threadIdx.x % 16, ty = threadIdx.x / 16;
   const float c = shift[h];
   const int ibase = i0 + tx * 4;
@@ -131,9 +137,9 @@ __global__ void __launch_bounds__(256) k_phi(Problem p, const void* Q, const voi
 #pragma unroll
   for (int b = 0; b < 4; ++b) {
     int j = j0 + ty * 4 + b;
-    if (j >= p.T) continue;
+    if (j >= Th) continue;
     // one rounding of s·scale + b − c (no intermediate rounding of s, |s| ≈ c)
-    const float bmc = p.has_bias ? key_bias[(int64_t)h * p.T + j] - c : -c;
+    const float bmc = p.has_bias ? key_bias[krow0 + j] - c : -c;
     float v[4];
 #pragma unroll
     for (int a = 0; a < 4; ++a)
@@ -151,7 +157,7 @@ __global__ void __launch_bounds__(256) k_phi(Problem p, const void* Q, const voi
 // Y[i][:] = Σ_j Φᵀ[j][i] V[j][:] / m_i and m_i = Σ_j Φᵀ[j][i]; also r = m.
 // Thread (tx, ty): queries i0 + 4tx .. +3, value dims ty·DPT .. +DPT-1.
 template <int DPT>
-__global__ void __launch_bounds__(256) k_y_m(Problem p, const void* V, const float* phiT,
+__global__ void __launch_bounds__(256) k_y_m(Problem p, Work w, const void* V, const float* phiT,
                                              float* Y, double* m, float* r) {
   constexpr int DT = 16 * DPT;
   __shared__ __align__(16) float Ps[DK][TQ + 4];
@@ -166,18 +172,19 @@ __global__ void __launch_bounds__(256) k_y_m(Problem p, const void* V, const flo
 #pragma unroll
     for (int c = 0; c < DPT; ++c) acc[a][c] = 0.f;
   const float* P = phiT + (int64_t)h * p.T * p.ldn;
-  const int64_t vbase = (int64_t)h * p.T * p.d;
-  for (int j0 = 0; j0 < p.T; j0 += DK) {
+  const int Th = w.Th[h];
+  const int64_t vbase = w.koff[h] * p.d;
+  for (int j0 = 0; j0 < Th; j0 += DK) {
     __syncthreads();
     for (int e = threadIdx.x; e < DK * TQ; e += blockDim.x) {
       int jj = e / TQ, ii = e % TQ;
       int j = j0 + jj, i = i0 + ii;
-      Ps[jj][ii] = (j < p.T && i < p.ldn) ? P[(int64_t)j * p.ldn + i] : 0.f;
+      Ps[jj][ii] = (j < Th && i < p.ldn) ? P[(int64_t)j * p.ldn + i] : 0.f;
     }
     for (int e = threadIdx.x; e < DK * DT; e += blockDim.x) {
       int jj = e / DT, c = e % DT;
       int j = j0 + jj;
-      Vs[jj][c] = (j < p.T && c < p.d) ? load_in(V, vbase + (int64_t)j * p.d + c, p.in_dtype) : 0.f;
+      Vs[jj][c] = (j < Th && c < p.d) ? load_in(V, vbase + (int64_t)j * p.d + c, p.in_dtype) : 0.f;
     }
     __syncthreads();
 #pragma unroll 4
@@ -222,12 +229,12 @@ __global__ void __launch_bounds__(256) k_y_m(Problem p, const void* V, const flo
 
 }  // namespace
 
-cudaError_t launch_shift_max(const Problem& p, const void* Q, const void* K, const float* key_bias,
+cudaError_t launch_shift_max(const Problem& p, const Work& w, const void* Q, const void* K, const float* key_bias,
                              float* shift, cudaStream_t s) {
   uint32_t* u = reinterpret_cast<uint32_t*>(shift);
   AM_LAUNCH(AM_STAGE_SHIFT, s, k_shift_init<<<(p.H + 127) / 128, 128, 0, s>>>(u, p.H));
   dim3 grid((p.n + TQ - 1) / TQ, (p.T + TK - 1) / TK, p.H);
-  AM_LAUNCH(AM_STAGE_SHIFT, s, k_shift_max<<<grid, 256, 0, s>>>(p, Q, K, key_bias, u));
+  AM_LAUNCH(AM_STAGE_SHIFT, s, k_shift_max<<<grid, 256, 0, s>>>(p, w, Q, K, key_bias, u));
   AM_LAUNCH(AM_STAGE_SHIFT, s, k_shift_decode<<<(p.H + 127) / 128, 128, 0, s>>>(u, p.H));
   return cudaGetLastError();
 }
@@ -235,17 +242,17 @@ cudaError_t launch_shift_max(const Problem& p, const void* Q, const void* K, con
 cudaError_t launch_phi(const Problem& p, const void* Q, const void* K, const float* key_bias,
                        const Work& w, cudaStream_t s) {
   dim3 grid((p.ldn + TQ - 1) / TQ, (p.T + TK - 1) / TK, p.H);
-  AM_LAUNCH(AM_STAGE_PHI, s, k_phi<<<grid, 256, 0, s>>>(p, Q, K, key_bias, w.shift, w.phiT, w.phiT16));
+  AM_LAUNCH(AM_STAGE_PHI, s, k_phi<<<grid, 256, 0, s>>>(p, w, Q, K, key_bias, w.shift, w.phiT, w.phiT16));
   return cudaGetLastError();
 }
 
 cudaError_t launch_y_m(const Problem& p, const void* V, const Work& w, cudaStream_t s) {
   dim3 grid((p.ldn + TQ - 1) / TQ, p.H);
-  if (p.d <= 16) AM_LAUNCH(AM_STAGE_TARGET, s, k_y_m<1><<<grid, 256, 0, s>>>(p, V, w.phiT, w.Y, w.m, w.r));
-  else if (p.d <= 32) AM_LAUNCH(AM_STAGE_TARGET, s, k_y_m<2><<<grid, 256, 0, s>>>(p, V, w.phiT, w.Y, w.m, w.r));
-  else if (p.d <= 64) AM_LAUNCH(AM_STAGE_TARGET, s, k_y_m<4><<<grid, 256, 0, s>>>(p, V, w.phiT, w.Y, w.m, w.r));
-  else if (p.d <= 128) AM_LAUNCH(AM_STAGE_TARGET, s, k_y_m<8><<<grid, 256, 0, s>>>(p, V, w.phiT, w.Y, w.m, w.r));
-  else AM_LAUNCH(AM_STAGE_TARGET, s, k_y_m<16><<<grid, 256, 0, s>>>(p, V, w.phiT, w.Y, w.m, w.r));
+  if (p.d <= 16) AM_LAUNCH(AM_STAGE_TARGET, s, k_y_m<1><<<grid, 256, 0, s>>>(p, w, V, w.phiT, w.Y, w.m, w.r));
+  else if (p.d <= 32) AM_LAUNCH(AM_STAGE_TARGET, s, k_y_m<2><<<grid, 256, 0, s>>>(p, w, V, w.phiT, w.Y, w.m, w.r));
+  else if (p.d <= 64) AM_LAUNCH(AM_STAGE_TARGET, s, k_y_m<4><<<grid, 256, 0, s>>>(p, w, V, w.phiT, w.Y, w.m, w.r));
+  else if (p.d <= 128) AM_LAUNCH(AM_STAGE_TARGET, s, k_y_m<8><<<grid, 256, 0, s>>>(p, w, V, w.phiT, w.Y, w.m, w.r));
+  else AM_LAUNCH(AM_STAGE_TARGET, s, k_y_m<16><<<grid, 256, 0, s>>>(p, w, V, w.phiT, w.Y, w.m, w.r));
   return cudaGetLastError();
 }
 

@@ -94,6 +94,13 @@ __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, u
       : "memory");
 }
 
+__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, uint64_t* bar, int x, int y) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cta.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], [%2];"
+      ::"r"(smem_u32(dst)), "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x), "r"(y)
+      : "memory");
+}
+
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
 
@@ -217,7 +224,12 @@ k_phi_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtens
   const int nqb = (p.n + BM - 1) / BM;
   const int h = blockIdx.x / nqb;
   const int q0 = (blockIdx.x % nqb) * BM;
-  const int NT = (p.T + BN - 1) / BN;
+  // this head's keys are rows krow0 .. krow0 + Th − 1 of the packed K and V
+  // (the 2-D tensor maps): a tile reaching past Th reads the next head's
+  // rows (or zeros past the end), and the epilogue masks those columns
+  const int Th = w.Th[h];
+  const int krow0 = (int)w.koff[h];
+  const int NT = (Th + BN - 1) / BN;
   int32_t* status = w.status + h;
   volatile int* abort_flag = &s_abort;
 
@@ -258,10 +270,10 @@ k_phi_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtens
         if (use > 0 && !mbar_wait(kv_empty + s, (use - 1) & 1, abort_flag, status)) break;
         mbar_expect_tx(kv_full + s, P.k_bytes + P.v_bytes);
         for (int kb = 0; kb < KB; ++kb)
-          tma_load_3d(sK + s * P.k_bytes + kb * BN * 128, &tmK, kv_full + s, kb * 64, j * BN, h);
+          tma_load_2d(sK + s * P.k_bytes + kb * BN * 128, &tmK, kv_full + s, kb * 64, krow0 + j * BN);
         if (MODE == MODE_PHI)
           for (int kb = 0; kb < KB; ++kb)
-            tma_load_3d(sV + s * P.v_bytes + kb * BN * 128, &tmV, kv_full + s, kb * 64, j * BN, h);
+            tma_load_2d(sV + s * P.v_bytes + kb * BN * 128, &tmV, kv_full + s, kb * 64, krow0 + j * BN);
         issued[s] = use + 1;
       }
       // copies still in flight must land before the CTA releases its memory
@@ -366,12 +378,12 @@ k_phi_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtens
       tmem_wait_ld();
       tc_fence_before();
       mbar_arrive(s_empty + b);
-      const int kvalid = min(BN, p.T - j * BN) - grp * HC;   // valid columns of this group
+      const int kvalid = min(BN, Th - j * BN) - grp * HC;    // valid columns of this group
       // per-key additive term: (b_j − c)·log2e (PHI) or b_j (MAX); a constant without a prior bias
       const int jb = j * BN + grp * HC;
       auto bias_at = [&](int cc) -> float {
         const int jg = jb + cc;
-        const float bj = jg < p.T ? __ldg(key_bias + (int64_t)h * p.T + jg) : 0.f;
+        const float bj = jg < Th ? __ldg(key_bias + krow0 + jg) : 0.f;
         return MODE == MODE_PHI ? (bj - c) * kLog2e : bj;
       };
       const bool full = row_live && kvalid >= HC;
@@ -418,7 +430,7 @@ k_phi_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtens
         }
         q2[0] += __shfl_xor_sync(0xffffffffu, q2[0], 1);
         const int key = jb + ((lane >> 1) & (HC - 1));
-        if (!(lane & 1) && key < p.T)
+        if (!(lane & 1) && key < Th)
           w.cnpart[(((int64_t)h * nqb + blockIdx.x % nqb) * 4 + qd) * p.T + key] = q2[0];
       }
       if (i < p.ldn) {
@@ -538,7 +550,10 @@ k_corr_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   constexpr int KB = D / 64;
   const int h = w.order[blockIdx.y];
-  if (pass * p.kR >= w.t[h]) return;          // head already finished (whole CTA leaves)
+  const int Th = w.Th[h];
+  // the whole CTA leaves when the head is finished or has no key in this block
+  if (pass * p.kR >= w.t[h] || (int)blockIdx.x * BM >= Th) return;
+  const int krow0 = (int)w.koff[h];
   unsigned char* sm = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t k_bytes = BM * D * 2, q_bytes = CQ * D * 2;
   unsigned char* sK = sm;
@@ -582,7 +597,7 @@ k_corr_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
   if (warp == 0) {
     if (lane == 0) {
       mbar_expect_tx(k_full, k_bytes);
-      for (int kb = 0; kb < KB; ++kb) tma_load_3d(sK + kb * BM * 128, &tmK, k_full, kb * 64, j0, h);
+      for (int kb = 0; kb < KB; ++kb) tma_load_2d(sK + kb * BM * 128, &tmK, k_full, kb * 64, krow0 + j0);
       int issued[CSTAGES] = {};
       for (int j = 0; j < NQ; ++j) {
         const int s = j % CSTAGES, use = j / CSTAGES;
@@ -629,11 +644,11 @@ k_corr_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
     const int qd = warp & 3;                    // TMEM lane quadrant
     const int et = qd * 32 + lane;              // key row within the block
     const int j = j0 + et;
-    const bool key_live = j < p.T;
+    const bool key_live = j < Th;
     const float kLog2e = 1.4426950408889634f;
     const float scale = p.scale * kLog2e;
     const float c = w.shift[h];
-    const float bj = (p.has_bias && key_live) ? key_bias[(int64_t)h * p.T + j] : 0.f;
+    const float bj = (p.has_bias && key_live) ? key_bias[krow0 + j] : 0.f;
     const float bias2 = (bj - c) * kLog2e;
     const float* rh = w.r + (int64_t)h * p.ldn;
     const uint32_t tcol = lane_addr_base(qd) + wg * 32;
@@ -684,6 +699,21 @@ PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
   return fn;
 }
 
+// [rows][d] bf16 (the packed keys or values of every head), box = 64
+// elements (128 B) × box_rows, 128-byte swizzle; rows past the end read zeros.
+bool make_map_2d(CUtensorMap* map, const void* base, int64_t rows, int d, int box_rows) {
+  auto enc = get_encode();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)d, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)d * 2};
+  cuuint32_t box[2] = {64, (cuuint32_t)box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 // [H][rows][d] bf16, box = 64 elements (128 B) × box_rows × 1, 128-byte swizzle.
 bool make_map(CUtensorMap* map, const void* base, int H, int rows, int d, int box_rows) {
   auto enc = get_encode();
@@ -702,8 +732,8 @@ template <int D, int MODE>
 cudaError_t launch_tc(const Problem& p, const void* Q, const void* K, const void* V, const float* key_bias,
                       const Work& w, uint32_t* shift_ord, cudaStream_t s) {
   CUtensorMap mq, mk, mv;
-  if (!make_map(&mq, Q, p.H, p.n, D, BM) || !make_map(&mk, K, p.H, p.T, D, BN) ||
-      !make_map(&mv, MODE == MODE_PHI ? V : K, p.H, p.T, D, BN))
+  if (!make_map(&mq, Q, p.H, p.n, D, BM) || !make_map_2d(&mk, K, p.key_rows, D, BN) ||
+      !make_map_2d(&mv, MODE == MODE_PHI ? V : K, p.key_rows, D, BN))
     return cudaErrorInvalidValue;
   const Plan P = make_plan(D, MODE);
   auto kern = k_phi_tc<D, MODE>;
@@ -719,7 +749,7 @@ template <int D>
 cudaError_t launch_corr_tc_d(const Problem& p, const void* Q, const void* K, const float* key_bias, const Work& w,
                              int pass, int active, cudaStream_t s) {
   CUtensorMap mq, mk;
-  if (!make_map(&mq, Q, p.H, p.n, D, CQ) || !make_map(&mk, K, p.H, p.T, D, BM)) return cudaErrorInvalidValue;
+  if (!make_map(&mq, Q, p.H, p.n, D, CQ) || !make_map_2d(&mk, K, p.key_rows, D, BM)) return cudaErrorInvalidValue;
   const uint32_t bytes = corr_smem_bytes(D);
   auto kern = k_corr_tc<D>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);

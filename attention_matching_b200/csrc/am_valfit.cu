@@ -55,7 +55,7 @@ __global__ void __launch_bounds__(256) k_finalize(Problem p, Work w, const void*
     const double wl = w.w[base + l];
     const double we = fmax(wl, floor_w);
     w.w_eff[base + q] = we;
-    const double bj = p.has_bias ? (double)key_bias[(int64_t)h * p.T + j] : 0.0;
+    const double bj = p.has_bias ? (double)key_bias[w.koff[h] + j] : 0.0;
     beta[base + q] = (float)(bj + log(we));
     if (w_out) w_out[base + q] = (float)wl;
     if (pick_order) pick_order[base + l] = j;
@@ -67,7 +67,7 @@ __global__ void __launch_bounds__(256) k_finalize(Problem p, Work w, const void*
   for (int64_t e = threadIdx.x; e < total; e += blockDim.x) {
     const int q = (int)(e / p.d), c = (int)(e % p.d);
     const int j = indices[base + q];
-    const int64_t src = ((int64_t)h * p.T + j) * p.d + c;
+    const int64_t src = (w.koff[h] + j) * p.d + c;
     const int64_t dst = (base + q) * p.d + c;
     if (p.in_dtype == AM_BF16)
       reinterpret_cast<__nv_bfloat16*>(C_k)[dst] = reinterpret_cast<const __nv_bfloat16*>(K)[src];

@@ -209,6 +209,16 @@ class Workload:
     refit_every: int
     dtype: str
     note: str = ""
+    key_offsets: Optional[List[int]] = None   # set when the heads' key counts differ
+
+
+def key_offsets_of(heads: List[Head]) -> List[int]:
+    """Row offsets of each head's keys when the heads' K (and V) are stacked
+    end to end: [0, T_0, T_0 + T_1, ...]."""
+    out = [0]
+    for h in heads:
+        out.append(out[-1] + h.T)
+    return out
 
 
 def single_head_fp32(seed: int = 1000) -> Workload:
@@ -236,6 +246,26 @@ def qwen3_4b_model(num_heads: int = 288, T: int = 8192, n: int = 8192, ratio: fl
     budgets = lognormal_budgets(seed_base + 999, num_heads, total)
     return Workload(f"qwen3_4b_model_H{num_heads}_T{T}_n{n}_d128_lognormal", heads,
                     budgets, 4, 2, "bf16")
+
+
+def llama31_8b_longctx(num_layers: int = 32, kv_heads: int = 8, T_total: int = 60000, chunk: int = 8192,
+                       n: int = 8192, ratio: float = 10.0, seed_base: int = 5000,
+                       max_sequences: Optional[int] = None) -> Workload:
+    """Llama-3.1-8B-shaped long context at 10×: per (layer, KV head) one
+    structured sequence of T_total keys cut KV-based into chunks of `chunk`
+    keys (the last one shorter: 60000 = 7·8192 + 2656), each chunk with its
+    own n reference queries; every chunk is an independent problem with budget
+    round-half-up(T_c / ratio) (819 and 266), top-k 8 with a refit every 2
+    rounds.  Heads are ordered (layer, KV head, chunk); their key counts
+    differ, so the workload carries key offsets.  ``max_sequences`` keeps only
+    the first sequences (a smaller sample of the same workload)."""
+    seqs = num_layers * kv_heads if max_sequences is None else min(max_sequences, num_layers * kv_heads)
+    heads: List[Head] = []
+    for q in range(seqs):
+        heads.extend(long_sequence_chunks(seed_base + q, T_total, chunk, n))
+    budgets = [budget_for_ratio(h.T, ratio) for h in heads]
+    name = f"llama31_8b_longctx_{seqs}seq_T{T_total}_chunk{chunk}_n{n}_d128_x{int(ratio)}"
+    return Workload(name, heads, budgets, 8, 2, "bf16", key_offsets=key_offsets_of(heads))
 
 
 # ----------------------------------------------------------------------------

@@ -116,11 +116,24 @@ typedef struct am_opts {
   double* residual_out;    /* [H] ‖m − Φ_S w‖ / ‖m‖ after the last refit          */
   float* w_out;            /* [Σt] NNLS weights, aligned with indices            */
   int32_t select_mode;     /* am_select_mode_t (default AM_SELECT_OMP)           */
+  int32_t reserved0;       /* must be 0                                          */
+  /* Optional HOST input: variable key counts per head (KV-based chunking of a
+   * long context, "Fast KV Compaction via Attention Matching": xinfinite.net
+   * article §3, where each chunk is compacted independently and the last
+   * chunk is shorter; per-head varlen segments, zhichai.net deep dive §4.2).
+   * NULL: every head has T keys, K/V are [H][T][d] and key_bias [H][T].
+   * Otherwise int64 [H+1], key_offsets[0] = 0, T_h = key_offsets[h+1] −
+   * key_offsets[h] >= 1, and max_h T_h must equal the T argument: K and V
+   * are packed [Σ T_h][d] (head h's keys are rows key_offsets[h] ..
+   * key_offsets[h+1] − 1), key_bias is packed [Σ T_h], and each budget
+   * satisfies 1 <= t_h <= T_h.  Read during the call only. */
+  const int64_t* key_offsets;
 } am_opts_t;
 
 /* Fill *opts with defaults: bf16 inputs, k = 1, R = 1, scale = 1/sqrt(d),
  * ridge = 1e-6, w_floor_rel = 1e-12, corr_mode = AM_CORR_AUTO, every
- * optional pointer NULL, select_mode = AM_SELECT_OMP. */
+ * optional pointer NULL (key_offsets NULL: T keys per head),
+ * select_mode = AM_SELECT_OMP. */
 am_status_t am_default_opts(am_opts_t* opts);
 
 /* Device workspace needed by am_compact_heads for this problem.
@@ -137,12 +150,27 @@ am_status_t am_workspace_size(int32_t n, int32_t T, int32_t d, int32_t num_heads
                               const int32_t* budgets, const am_opts_t* opts,
                               size_t* bytes);
 
+/* Workspace with which am_compact_heads processes the heads in waves of at
+ * most `wave_heads` consecutive heads (head order), one wave after the other
+ * through the same memory.  Problems whose stored features do not fit in
+ * HBM at once (2048 chunk-heads of 8192 keys × 8192 queries hold 512 GiB of
+ * fp32 Φᵀ) run this way.  wave_heads >= 1; values >= num_heads give
+ * am_workspace_size().  Same argument rules otherwise. */
+am_status_t am_workspace_size_waves(int32_t n, int32_t T, int32_t d, int32_t num_heads,
+                                    const int32_t* budgets, const am_opts_t* opts,
+                                    int32_t wave_heads, size_t* bytes);
+
 /* Compact H independent heads.
  *   Q_ref   [H][n][d], K [H][T][d], V [H][T][d], row-major, dtype opts->in_dtype
+ *           (K, V packed [Σ T_h][d] when opts->key_offsets is set)
  *   budgets host int32 [H]
  *   out_offsets host int64 [H+1]: out_offsets[0] = 0,
  *           out_offsets[h+1] = out_offsets[h] + budgets[h] (checked)
- *   workspace   device, 256-byte aligned, >= am_workspace_size() bytes
+ *   workspace   device, 256-byte aligned.  With >= am_workspace_size() bytes
+ *               all heads run in one wave; with less, the call runs the heads
+ *               in waves of consecutive heads, each as many as the workspace
+ *               holds (am_workspace_size_waves() gives the size for a chosen
+ *               wave size).  AM_ERR_WORKSPACE if one head does not fit.
  *   Outputs, packed per head at out_offsets[h] (the varlen layout), rows in
  *   ascending original key position:
  *     C_k      [Σt][d]  dtype opts->in_dtype (exact copies of the chosen keys)
@@ -161,10 +189,12 @@ am_status_t am_compact_heads(const void* Q_ref, const void* K, const void* V,
                              void* stream);
 
 /* Where am_compact_heads leaves its intermediate features inside the
- * caller's workspace (byte offsets from the workspace base), valid once the
- * call has completed and until the workspace is reused:
+ * caller's workspace (byte offsets from the workspace base), valid once a
+ * call that ran all heads in one wave (workspace >= am_workspace_size())
+ * has completed, and until the workspace is reused:
  *   phiT    fp32 [H][T][ldn]  Φᵀ_ji = exp(s_ij − c_h), key-major, rows padded
- *                             with zeros from n to ldn
+ *                             with zeros from n to ldn (with key_offsets:
+ *                             rows T_h .. T−1 of head h are not written)
  *   mass    fp64 [H][ldn]     m_i = Σ_j Φ_ij (exact sum of the stored fp32 Φ)
  *   target  fp32 [H][n][d]    Y_i = Σ_j Φ_ij V_j / m_i
  *   shift   fp32 [H]          c_h used

@@ -170,3 +170,54 @@ def test_highest_attention_mode_argument_rules():
     with pytest.raises(am.AmError) as e:
         am.workspace_size(512, 4096, 128, [100], am.make_opts(am.BF16, 4, 2, select_mode=5))
     assert e.value.code == code["AM_ERR_INVALID_ARG"]
+
+
+def _opts_with_offsets(offsets, dtype=None):
+    o = am.make_opts(am.BF16 if dtype is None else dtype, 8, 2)
+    arr = (ctypes.c_int64 * len(offsets))(*offsets)
+    o.key_offsets = ctypes.cast(arr, ctypes.c_void_p)
+    return o, arr
+
+
+def test_key_offsets_argument_rules():
+    """Per-head key counts: offsets start at 0 and grow by at least one key,
+    the largest count equals T, and each budget fits its own head."""
+    code = {v: k for k, v in am.STATUS.items()}
+    o, keep = _opts_with_offsets([0, 1024, 2048, 2500])
+    assert am.workspace_size(768, 1024, 128, [103, 103, 46], o) > 0
+    for offs, T, budgets, want in [
+        ([1, 1024, 2048, 2500], 1024, [10, 10, 10], "AM_ERR_INVALID_ARG"),    # does not start at 0
+        ([0, 1024, 1024, 2500], 1476, [10, 10, 10], "AM_ERR_INVALID_ARG"),    # an empty head
+        ([0, 1024, 2048, 2500], 2048, [10, 10, 10], "AM_ERR_INVALID_ARG"),    # T is not the largest count
+        ([0, 1024, 2048, 2500], 1024, [10, 10, 453], "AM_ERR_BUDGET"),        # t above the head's 452 keys
+    ]:
+        o, keep = _opts_with_offsets(offs)
+        with pytest.raises(am.AmError) as e:
+            am.workspace_size(768, T, 128, budgets, o)
+        assert e.value.code == code[want], (offs, T, budgets)
+
+
+def test_wave_workspace_sizes():
+    """Waves of consecutive heads: one wave of every head is the ordinary
+    workspace; smaller waves need less, never less than the largest single
+    head, and the size grows with the wave."""
+    o = am.make_opts(am.BF16, 8, 2)
+    budgets = [819] * 7 + [266]
+    offs = [0]
+    for h in range(8):
+        offs.append(offs[-1] + (8192 if h < 7 else 2656))
+    o, keep = _opts_with_offsets(offs)
+    full = am.workspace_size(8192, 8192, 128, budgets, o)
+    assert am.workspace_size(8192, 8192, 128, budgets, o, wave_heads=8) == full
+    assert am.workspace_size(8192, 8192, 128, budgets, o, wave_heads=100) == full
+    sizes = [am.workspace_size(8192, 8192, 128, budgets, o, wave_heads=w) for w in (1, 2, 4, 8)]
+    assert sizes == sorted(sizes) and sizes[0] < sizes[1] < sizes[3]
+    assert sizes[0] >= 8192 * 8192 * 4        # one head's stored features
+    assert sizes[1] < 3 * 8192 * 8192 * 4     # two heads' worth, not eight
+
+
+def test_workspace_below_one_head_is_rejected_before_any_work():
+    """A workspace that cannot hold one head's wave is refused synchronously."""
+    o = am.make_opts(am.FP32)
+    one = am.workspace_size(64, 32, 16, [4], o)
+    assert _call(ws=4096, ws_bytes=one - 4096) == 3

@@ -1,5 +1,7 @@
 """GPU parity: the CUDA path, called through the C ABI, against the float64
 oracle on the same seeded inputs (rules in tests/parity.py)."""
+import ctypes
+
 import numpy as np
 import pytest
 import torch
@@ -26,10 +28,24 @@ def run_gpu(heads, budgets, topk, refit, shifts=None, key_bias=None, **kw):
                             trace=True, **kw)
 
 
-def check_all(heads, budgets, topk, refit, key_bias=None, sample=None, label="", exact_picks=True, **kw):
+def run_gpu_varlen(heads, budgets, topk, refit, shifts=None, key_bias=None, **kw):
+    """One call over heads of different key counts: K, V (and the prior bias)
+    packed end to end with their key offsets."""
+    import attention_matching_b200 as am
+    Q = _stack(heads, "Q")
+    K = torch.cat([h.K for h in heads]).contiguous().cuda()
+    V = torch.cat([h.V for h in heads]).contiguous().cuda()
+    sh = None if shifts is None else torch.tensor(shifts, dtype=torch.float32).cuda()
+    kb = None if key_bias is None else torch.tensor(np.concatenate(key_bias), dtype=torch.float32).cuda()
+    return am.compact_heads(Q, K, V, budgets, topk=topk, refit_every=refit, shift=sh, key_bias=kb,
+                            trace=True, key_offsets=W.key_offsets_of(heads), **kw)
+
+
+def check_all(heads, budgets, topk, refit, key_bias=None, sample=None, label="", exact_picks=True,
+              varlen=False, **kw):
     shifts = [shift_for(*h.f64()[:2], key_bias=None if key_bias is None else key_bias[i])
               for i, h in enumerate(heads)]
-    out = run_gpu(heads, budgets, topk, refit, shifts, key_bias, **kw)
+    out = (run_gpu_varlen if varlen else run_gpu)(heads, budgets, topk, refit, shifts, key_bias, **kw)
     assert all(s in (0, 8) for s in out["status"]), out["status"]
     reps = []
     for h in (range(len(heads)) if sample is None else sample):
@@ -109,14 +125,12 @@ def test_device_shift_matches_max_logit():
 
 
 @needs_cuda
-def test_qwen3_layer_full_size_sampled():
-    """The bench workload (8 heads, T = n = 8192, d = 128, t = 164, k = 4,
-    R = 2) run whole on the GPU; two heads checked against the oracle."""
+def test_qwen3_layer_full_size_all_heads():
+    """The Qwen3-4B layer (8 heads, T = n = 8192, d = 128, t = 164, k = 4,
+    R = 2) run whole on the GPU; every head checked against the oracle."""
     wl = W.qwen3_4b_layer()
-    _, reps = check_all(wl.heads, wl.budgets, wl.topk, wl.refit_every, sample=[0, 5],
-                        label="qwen3 layer")
-    for r in reps:
-        assert r["out_rel"] <= 2e-3
+    _, reps = check_all(wl.heads, wl.budgets, wl.topk, wl.refit_every, label="qwen3 layer")
+    assert len(reps) == 8
 
 
 @needs_cuda
@@ -226,12 +240,74 @@ def test_large_budget_global_factor():
 @needs_cuda
 def test_kv_chunked_long_sequence():
     """KV-based chunking: one long sequence cut into contiguous chunks that are
-    compacted independently (sinks only in the first chunk); chunks of equal
-    length share a call, the shorter last chunk gets its own."""
+    compacted independently (sinks only in the first chunk); the full chunks
+    and the shorter last chunk share one call through per-head key offsets."""
     chunks = W.long_sequence_chunks(395, T_total=2500, chunk=1024, n=768)
     assert [c.T for c in chunks] == [1024, 1024, 452]
-    check_all(chunks[:2], [103, 103], 8, 2, label="chunks 0-1")
-    check_all(chunks[2:], [46], 8, 2, label="last chunk")
+    check_all(chunks, [103, 103, 46], 8, 2, varlen=True, label="chunks")
+
+
+@needs_cuda
+def test_varlen_keys_fp32_prior_bias():
+    """Per-head key counts on the CUDA-core feature pass (fp32, d = 64), with a
+    packed prior key bias and the shift computed on the device."""
+    heads = [W.iid_head(560 + h, n=200, T=T, d=64) for h, T in enumerate((130, 257, 64))]
+    rng = np.random.default_rng(561)
+    kb = [np.float32(rng.normal(0.0, 0.5, h.T)) for h in heads]
+    out, _ = check_all(heads, [9, 20, 5], 4, 2, key_bias=kb, varlen=True, label="varlen fp32")
+    for h, hd in enumerate(heads):
+        Q, K, _ = hd.f64()
+        want = O.max_logit(Q, K, key_bias=np.float64(kb[h]))
+        assert abs(float(out["shift"][h]) - float(np.float32(want))) <= 1e-5 * max(1.0, abs(want))
+
+
+@needs_cuda
+def test_varlen_keys_recompute_and_stored_and_highest():
+    """Per-head key counts through the other selection paths: the tensor-core
+    recompute of Φ (key blocks past a head's own keys leave no values), the
+    stored-feature GEMV, and highest-attention selection."""
+    import attention_matching_b200 as am
+    heads = [W.structured_head(570 + h, n=520, T=T) for h, T in enumerate((700, 333, 129))]
+    for mode in (am.CORR_RECOMPUTE, am.CORR_STORED_FP32):
+        check_all(heads, [30, 17, 8], 4, 2, varlen=True, corr_mode=mode, label=f"varlen corr {mode}")
+    shifts = [shift_for(*h.f64()[:2]) for h in heads]
+    out = run_gpu_varlen(heads, [25, 14, 9], 1, 1, shifts, select_mode=am.SELECT_HIGHEST)
+    for h, t in enumerate([25, 14, 9]):
+        Q, K, V = heads[h].f64()
+        got = split_head(out, h)["pick_order"]
+        want = O.highest_attention_select(Q, K, t)
+        score = _attention_scores(Q, K)
+        for a, b in zip(got, want):
+            if a != b:
+                assert abs(score[a] - score[b]) <= 1e-6 * score.max(), f"highest varlen head {h}"
+
+
+@needs_cuda
+def test_waves_give_the_one_wave_result():
+    """A workspace smaller than the whole problem: the heads run in waves of
+    consecutive heads through the same memory, with the one-wave result
+    (ragged key counts, non-uniform budgets, a prior bias): picks, β and
+    residuals bit for bit; C_v to fp32 rounding, since the value fit splits
+    its fp64 sums over the queries by the number of heads in a launch."""
+    import attention_matching_b200 as am
+    heads = [W.structured_head(580 + h, n=600, T=T) for h, T in enumerate((640, 512, 777, 300, 640))]
+    budgets = [40, 12, 66, 30, 25]
+    rng = np.random.default_rng(581)
+    kb = [np.float32(rng.normal(0.0, 0.3, h.T)) for h in heads]
+    one = run_gpu_varlen(heads, budgets, 4, 2, key_bias=kb)
+    offs = W.key_offsets_of(heads)
+    opts = am.make_opts(am.BF16, 4, 2)
+    arr = (ctypes.c_int64 * len(offs))(*offs)
+    opts.key_offsets = ctypes.cast(arr, ctypes.c_void_p)
+    for wave in (1, 2, 3):
+        need = am.workspace_size(600, 777, 128, budgets, opts, wave_heads=wave)
+        assert need < am.workspace_size(600, 777, 128, budgets, opts)
+        ws = torch.empty((need,), dtype=torch.uint8, device="cuda")
+        got = run_gpu_varlen(heads, budgets, 4, 2, key_bias=kb, workspace=ws)
+        assert all(s in (0, 8) for s in got["status"]), got["status"]
+        for k in ("indices", "C_k", "beta", "pick_order", "shift", "residual"):
+            assert torch.equal(got[k], one[k]), (wave, k)
+        torch.testing.assert_close(got["C_v"], one["C_v"], rtol=1e-5, atol=1e-6)
 
 
 @needs_cuda
