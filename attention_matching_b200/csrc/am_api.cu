@@ -158,7 +158,7 @@ am_status_t check_shape(int n, int T, int d, int H, const int32_t* budgets, cons
     return AM_ERR_UNSUPPORTED;
   if ((int64_t)n * d > (1ll << 31) || (int64_t)T * round_up(n, 32) > (1ll << 40))
     return AM_ERR_UNSUPPORTED;
-  if (opts->reserved0 != 0) return AM_ERR_INVALID_ARG;
+  if (opts->reserved0 != 0 || opts->wait_cycles < 0) return AM_ERR_INVALID_ARG;
   const int kR = highest ? kHighestChunk : opts->topk * opts->refit_every;
   tb->t.assign(budgets, budgets + H);
   tb->Th.assign(H, T);
@@ -356,6 +356,7 @@ Problem make_problem(int n, int T, int d, int H, const am_opts_t* o, const Table
   p.corr_bounded = !p.select_highest && (o->corr_mode == AM_CORR_BOUNDED || o->corr_mode == AM_CORR_AUTO);
   if (p.select_highest) p.corr_recompute = false;
   p.key_rows = tb.koff[H];
+  p.wait_cycles = o->wait_cycles > 0 ? (long long)o->wait_cycles : kDefaultWaitCycles;
   return p;
 }
 
@@ -658,6 +659,7 @@ const char* am_status_string(am_status_t s) {
     case AM_ERR_UNSUPPORTED: return "unsupported shape or dtype";
     case AM_WARN_NOT_CONVERGED: return "NNLS stopped at its iteration cap";
     case AM_ERR_NOT_SPD: return "value-fit matrix not positive definite";
+    case AM_WARN_MASS_UNDERFLOW: return "a reference query's features all underflowed in fp32";
   }
   return "unknown status";
 }

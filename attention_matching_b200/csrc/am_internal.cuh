@@ -34,7 +34,10 @@ struct Problem {
   int corr_bounded;   // the correlation pass computes only keys its bound cannot exclude
   int select_highest; // keys chosen up front by total attention, fed to the refits kR at a time
   int64_t key_rows;   // rows of K and V (and entries of key_bias) this launch reads: Σ_h Th[h]
+  long long wait_cycles;   // budget of a bounded device wait that does not drain issued work
 };
+
+constexpr long long kDefaultWaitCycles = 4000000000ll;   // ~2 s at 2 GHz
 
 // Device pointers into the caller's workspace (see plan_workspace()).
 struct Work {
@@ -164,9 +167,13 @@ __device__ __forceinline__ float load_in(const void* base, int64_t idx, int dtyp
   return reinterpret_cast<const float*>(base)[idx];
 }
 
+__device__ __forceinline__ bool is_warning(int code) {
+  return code == AM_WARN_NOT_CONVERGED || code == AM_WARN_MASS_UNDERFLOW;
+}
+
 __device__ __forceinline__ void record_status(int32_t* status, int code) {
-  // keep the most severe (largest) code; errors outrank the warning
-  atomicMax(status, code == AM_WARN_NOT_CONVERGED ? 1000 + code : 2000 + code);
+  // keep the most severe (largest) code; errors outrank the warnings
+  atomicMax(status, is_warning(code) ? 1000 + code : 2000 + code);
 }
 
 // Number of OMP passes for budget t: one correlation pass per refit interval.

@@ -802,9 +802,10 @@ __global__ void __launch_bounds__(kNnlsThreads) k_nnls(Problem p, Work w, int pa
   for (int q = tid; q < ylen0; q += blockDim.x) yv[q] = w.ycache[base + q];
   if (tid == 0) { ctl[0] = np_old; ctl[2] = 0; ctl[10] = ylen0; ctl[11] = np_old; }
   __syncthreads();   // the barrier is initialised before anyone waits on it
-  const bool landed = lbytes == 0 || mbar_wait_bounded(lbar, 0, kBulkWaitCycles);
+  const bool landed = lbytes == 0 || mbar_wait_bounded(lbar, 0, p.wait_cycles);
   if (__syncthreads_or(!landed)) {
-    // the copy did not land: flag the head, let it drain, leave everything as it was
+    // the copy did not land: flag the head, let it drain (full budget), leave
+    // everything as it was; the head's outputs are not valid (AM_ERR_TIMEOUT)
     if (tid == 0) record_status(w.status + h, AM_ERR_TIMEOUT);
     mbar_wait_bounded(lbar, 0, kBulkWaitCycles);
     return;

@@ -219,6 +219,8 @@ __global__ void __launch_bounds__(256) k_y_m(Problem p, Work w, const void* V, c
         if (cc < p.d) Y[((int64_t)h * p.n + i) * p.d + cc] = (float)((double)acc[a][c] * im);
       }
     }
+    // every feature of this reference query underflowed: it carries no mass
+    if (ty == 0 && i < p.n && !(mi > 0.0)) record_status(w.status + h, AM_WARN_MASS_UNDERFLOW);
     if (ty == 0 && i < p.ldn) {
       const double v = (i < p.n) ? mi : 0.0;
       m[(int64_t)h * p.ldn + i] = v;

@@ -42,6 +42,8 @@ constexpr int kEpiThreads = 128 * kEpiGroups;
 constexpr int kThreads = 128 + kEpiThreads;   // 4 control warps + the epilogue
 constexpr int kEpiWarp0 = 4;   // first epilogue warp
 constexpr uint32_t kTmemCols = 256;
+// Waits that drain work already issued (before the CTA releases TMEM and
+// shared memory) always get the full budget; the others get p.wait_cycles.
 constexpr long long kWaitBudgetCycles = 4000000000ll;   // ~2 s at 2 GHz
 
 enum Mode { MODE_MAX = 0, MODE_PHI = 1 };
@@ -73,11 +75,11 @@ __host__ __device__ inline Plan make_plan(int d, int mode) {
 // ---- PTX wrappers (mbarriers: am_async.cuh) ----
 // Bounded wait: false if the CTA aborted (here or elsewhere) before completion.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
-                                          int32_t* status) {
+                                          int32_t* status, long long budget) {
   const long long t0 = clock64();
   while (!mbar_try_wait(bar, parity)) {
     if (*abort_flag) return false;
-    if (clock64() - t0 > kWaitBudgetCycles) {
+    if (clock64() - t0 > budget) {
       *abort_flag = 1;
       record_status(status, AM_ERR_TIMEOUT);
       return false;
@@ -267,7 +269,7 @@ k_phi_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtens
       int issued[STAGES] = {};
       for (int j = 0; j < NT; ++j) {
         const int s = j % STAGES, use = j / STAGES;
-        if (use > 0 && !mbar_wait(kv_empty + s, (use - 1) & 1, abort_flag, status)) break;
+        if (use > 0 && !mbar_wait(kv_empty + s, (use - 1) & 1, abort_flag, status, p.wait_cycles)) break;
         mbar_expect_tx(kv_full + s, P.k_bytes + P.v_bytes);
         for (int kb = 0; kb < KB; ++kb)
           tma_load_2d(sK + s * P.k_bytes + kb * BN * 128, &tmK, kv_full + s, kb * 64, krow0 + j * BN);
@@ -277,7 +279,10 @@ k_phi_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtens
         issued[s] = use + 1;
       }
       // copies still in flight must land before the CTA releases its memory
-      mbar_wait(q_full, 0, abort_flag, status);
+      {
+        const long long t0 = clock64();
+        while (!mbar_try_wait(q_full, 0) && clock64() - t0 < kWaitBudgetCycles) {}
+      }
       for (int s = 0; s < STAGES; ++s)
         if (issued[s] > 0) {
           const long long t0 = clock64();
@@ -289,11 +294,11 @@ k_phi_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtens
     if (lane == 0) {
       const uint32_t idesc1 = instr_desc(BN, false);
       const uint32_t idesc2 = instr_desc(D, true);
-      bool ok = mbar_wait(q_full, 0, abort_flag, status);
+      bool ok = mbar_wait(q_full, 0, abort_flag, status, p.wait_cycles);
       tc_fence_after();
       auto gemm2 = [&](int jj) -> bool {
         const int b = jj & 1, bu = jj >> 1, s = jj % STAGES;
-        if (!mbar_wait(p_full + b, bu & 1, abort_flag, status)) return false;
+        if (!mbar_wait(p_full + b, bu & 1, abort_flag, status, p.wait_cycles)) return false;
         tc_fence_after();
         const uint32_t vbase = smem_u32(sV + s * P.v_bytes);
 #pragma unroll
@@ -313,8 +318,8 @@ k_phi_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtens
       int j = 0;
       for (; ok && j < NT; ++j) {
         const int s = j % STAGES, use = j / STAGES, b = j & 1, bu = j >> 1;
-        if (!mbar_wait(kv_full + s, use & 1, abort_flag, status)) { ok = false; break; }
-        if (bu > 0 && !mbar_wait(s_empty + b, (bu - 1) & 1, abort_flag, status)) { ok = false; break; }
+        if (!mbar_wait(kv_full + s, use & 1, abort_flag, status, p.wait_cycles)) { ok = false; break; }
+        if (bu > 0 && !mbar_wait(s_empty + b, (bu - 1) & 1, abort_flag, status, p.wait_cycles)) { ok = false; break; }
         tc_fence_after();
         const uint32_t qbase = smem_u32(sQ), kbase = smem_u32(sK + s * P.k_bytes);
 #pragma unroll
@@ -362,14 +367,14 @@ k_phi_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtens
       const int b = j & 1, bu = j >> 1;
       if constexpr (MODE == MODE_MAX) {
         // light per-tile work: one thread waits and the group follows it
-        if (ep == 0) s_stopm[b] = mbar_wait(s_full + b, bu & 1, abort_flag, status) ? 0 : 1;
+        if (ep == 0) s_stopm[b] = mbar_wait(s_full + b, bu & 1, abort_flag, status, p.wait_cycles) ? 0 : 1;
         asm volatile("bar.sync 1, %0;" ::"n"(kEpiThreads) : "memory");
         if (s_stopm[b]) { ok = false; break; }
       } else {
         // each epilogue thread waits for the tile itself; no named barrier in the
         // loop, but a warp leaves together (the loads and shuffles below are
         // warp-collective)
-        const bool got = mbar_wait(s_full + b, bu & 1, abort_flag, status);
+        const bool got = mbar_wait(s_full + b, bu & 1, abort_flag, status, p.wait_cycles);
         if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
       }
       tc_fence_after();
@@ -452,7 +457,7 @@ k_phi_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtens
       }
       // P tile for Y += P·V: K-major, 128-byte rows, 16-byte chunks XOR-swizzled by row;
       // the buffer is free once the MMA that read it two tiles ago has completed
-      if (bu > 0 && !mbar_wait(p_empty + b, (bu - 1) & 1, abort_flag, status)) { ok = false; break; }
+      if (bu > 0 && !mbar_wait(p_empty + b, (bu - 1) & 1, abort_flag, status, p.wait_cycles)) { ok = false; break; }
       unsigned char* hi_row = sP + (b * 2 + 0) * P.p_bytes + et * 128;
       unsigned char* lo_row = sP + (b * 2 + 1) * P.p_bytes + et * 128;
 #pragma unroll
@@ -486,7 +491,7 @@ k_phi_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtens
     } else {
       // combine the groups' mass partials in a fixed order: (0 + 1) + (2 + 3)
       s_mass[grp][et] = mrow;
-      if (ep == 0) s_stop_y = (ok && mbar_wait(y_full, 0, abort_flag, status)) ? 0 : 1;
+      if (ep == 0) s_stop_y = (ok && mbar_wait(y_full, 0, abort_flag, status, p.wait_cycles)) ? 0 : 1;
       asm volatile("bar.sync 1, %0;" ::"n"(kEpiThreads) : "memory");
       if (grp == 0) s_mass[kEpiGroups][et] = (s_mass[0][et] + s_mass[1][et]) + (s_mass[2][et] + s_mass[3][et]);
       asm volatile("bar.sync 1, %0;" ::"n"(kEpiThreads) : "memory");
@@ -511,6 +516,8 @@ k_phi_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtens
                               (float)(y[cc + 3] * im));
           }
         }
+        // every feature of this reference query underflowed: it carries no mass
+        if (grp == 0 && row_live && !(mtot > 0.0)) record_status(status, AM_WARN_MASS_UNDERFLOW);
         if (grp == 0 && i < p.ldn) {
           const double mv = row_live ? mtot : 0.0;
           w.m[(int64_t)h * p.ldn + i] = mv;
@@ -601,13 +608,16 @@ k_corr_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
       int issued[CSTAGES] = {};
       for (int j = 0; j < NQ; ++j) {
         const int s = j % CSTAGES, use = j / CSTAGES;
-        if (use > 0 && !mbar_wait(q_empty + s, (use - 1) & 1, abort_flag, status)) break;
+        if (use > 0 && !mbar_wait(q_empty + s, (use - 1) & 1, abort_flag, status, p.wait_cycles)) break;
         mbar_expect_tx(q_full + s, q_bytes);
         for (int kb = 0; kb < KB; ++kb)
           tma_load_3d(sQ + s * q_bytes + kb * CQ * 128, &tmQ, q_full + s, kb * 64, j * CQ, h);
         issued[s] = use + 1;
       }
-      mbar_wait(k_full, 0, abort_flag, status);
+      {   // the key block's copy must land before the CTA releases its memory
+        const long long t0 = clock64();
+        while (!mbar_try_wait(k_full, 0) && clock64() - t0 < kWaitBudgetCycles) {}
+      }
       for (int s = 0; s < CSTAGES; ++s)
         if (issued[s] > 0) {
           const long long t0 = clock64();
@@ -617,12 +627,12 @@ k_corr_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
   } else if (warp == 1) {
     if (lane == 0) {
       const uint32_t idesc = instr_desc(CQ, false);
-      bool ok = mbar_wait(k_full, 0, abort_flag, status);
+      bool ok = mbar_wait(k_full, 0, abort_flag, status, p.wait_cycles);
       tc_fence_after();
       for (int j = 0; ok && j < NQ; ++j) {
         const int s = j % CSTAGES, use = j / CSTAGES, b = j & 1, bu = j >> 1;
-        if (!mbar_wait(q_full + s, use & 1, abort_flag, status)) break;
-        if (bu > 0 && !mbar_wait(s_empty + b, (bu - 1) & 1, abort_flag, status)) break;
+        if (!mbar_wait(q_full + s, use & 1, abort_flag, status, p.wait_cycles)) break;
+        if (bu > 0 && !mbar_wait(s_empty + b, (bu - 1) & 1, abort_flag, status, p.wait_cycles)) break;
         tc_fence_after();
         const uint32_t kbase = smem_u32(sK), qbase = smem_u32(sQ + s * q_bytes);
 #pragma unroll
@@ -655,7 +665,7 @@ k_corr_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
     float acc[4] = {0.f, 0.f, 0.f, 0.f};
     for (int t = 0; t < NQ; ++t) {
       const int b = t & 1, bu = t >> 1;
-      if (!mbar_wait(s_full + b, bu & 1, abort_flag, status)) break;
+      if (!mbar_wait(s_full + b, bu & 1, abort_flag, status, p.wait_cycles)) break;
       tc_fence_after();
       float v[32];
       tmem_ld32(tS[b] + tcol, v);

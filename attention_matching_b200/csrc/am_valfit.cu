@@ -367,15 +367,18 @@ __global__ void __launch_bounds__(256) k_trsm(Problem p, Work w, float* C_v, int
     for (int e = tid; e < 32 * 32; e += blockDim.x) Dt[e >> 5][e & 31] = Dinv[(int64_t)b * 1024 + e];
     __syncthreads();
     diag_product(Dt, X + r0 * kXs, bw, true, rr, cg, ks);
-    // rows above the block: x_j −= Σ_{r in block} L[r][j] z_r (thread = row j × four columns)
+    // rows above the block: x_j −= Σ_{r in block} L[r][j] z_r (thread = row j × four
+    // columns: thread tid takes row tid / kGroups and column group tid % kGroups,
+    // so every (row, column group) pair above the block has exactly one owner)
+    const int cga = (tid % kGroups) * 4;
     for (int j = tid / kGroups; j < r0; j += 256 / kGroups) {
       double a0 = 0.0, a1 = 0.0, a2 = 0.0, a3 = 0.0;
       for (int r = r0; r < r0 + bw; ++r) {
         const double l = L[tri(r, j)];
-        const double* zr = X + r * kXs + cg;
+        const double* zr = X + r * kXs + cga;
         a0 = fma(l, zr[0], a0); a1 = fma(l, zr[1], a1); a2 = fma(l, zr[2], a2); a3 = fma(l, zr[3], a3);
       }
-      double* xj = X + j * kXs + cg;
+      double* xj = X + j * kXs + cga;
       xj[0] -= a0; xj[1] -= a1; xj[2] -= a2; xj[3] -= a3;
     }
     __syncthreads();

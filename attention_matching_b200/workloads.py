@@ -106,18 +106,20 @@ def _mixture_queries(rng: np.random.Generator, K: np.ndarray, n: int,
 
 
 def structured_head(seed: int, n: int, T: int, d: int = 128, rank: int = 32,
-                    sinks: int = 4, dtype: str = "bf16") -> Head:
+                    sinks: int = 4, dtype: str = "bf16", sink_queries: bool = False) -> Head:
     """Structured head (rank-32 keys + noise, sink keys, mixture queries).
 
     Draw order: basis B (QR of an N(0,1) d×rank matrix), U, E, one unit vector
     per sink, then the query mixture indices, Dirichlet weights and noise,
-    then V.
+    then V.  ``sink_queries`` lets the sink keys be mixture components too
+    (the mixture indices then range over every key): a query that mixes a
+    sink in reaches logits near 130, far above the other queries' best ones.
     """
     rng = np.random.default_rng(seed)
     B, _ = np.linalg.qr(rng.standard_normal((d, rank)))
     K = _structured_keys(rng, T, d, rank, sinks, B)
     Kr = upcast(round_to(K, dtype))
-    Q = _mixture_queries(rng, Kr, n, first=min(sinks, T - 1))
+    Q = _mixture_queries(rng, Kr, n, first=0 if sink_queries else min(sinks, T - 1))
     V = rng.standard_normal((T, d))
     return Head(round_to(Q, dtype), round_to(K, dtype), round_to(V, dtype))
 
@@ -238,14 +240,18 @@ def qwen3_4b_layer(num_heads: int = 8, T: int = 8192, n: int = 8192, ratio: floa
 
 
 def qwen3_4b_model(num_heads: int = 288, T: int = 8192, n: int = 8192, ratio: float = 50.0,
-                   seed_base: int = 4000) -> Workload:
+                   seed_base: int = 4000, only: Optional[List[int]] = None) -> Workload:
     """Full Qwen3-4B-shaped model (36 layers × 8 KV heads) with log-normal
-    non-uniform budgets summing to T·H/ratio, clipped to [4, 1024]."""
-    heads = [structured_head(seed_base + h, n=n, T=T) for h in range(num_heads)]
+    non-uniform budgets summing to T·H/ratio, clipped to [4, 1024].  ``only``
+    keeps the listed heads (their own seeds and budgets), in that order."""
     total = int(math.floor(T * num_heads / ratio + 0.5))
     budgets = lognormal_budgets(seed_base + 999, num_heads, total)
-    return Workload(f"qwen3_4b_model_H{num_heads}_T{T}_n{n}_d128_lognormal", heads,
-                    budgets, 4, 2, "bf16")
+    keep = list(range(num_heads)) if only is None else [int(h) for h in only]
+    heads = [structured_head(seed_base + h, n=n, T=T) for h in keep]
+    name = f"qwen3_4b_model_H{num_heads}_T{T}_n{n}_d128_lognormal"
+    if only is not None:
+        name += f"_{len(keep)}of{num_heads}heads"
+    return Workload(name, heads, [budgets[h] for h in keep], 4, 2, "bf16")
 
 
 def llama31_8b_longctx(num_layers: int = 32, kv_heads: int = 8, T_total: int = 60000, chunk: int = 8192,

@@ -24,6 +24,9 @@
  *   Y_i = Σ_j Φ_ij V_j / m_i,  A_il = softmax_l(Q C_kᵀ·scale + β)_i,
  *   C_v = (AᵀA + λI)⁻¹ AᵀY with λ = ridge·tr(AᵀA)/t_h.
  *
+ * Status codes 8 and 10 are warnings (the results are valid as described);
+ * the others above 0 are errors.
+ *
  * Conventions shared by every entry point
  *   - All tensor pointers are DEVICE pointers unless marked "host".
  *   - The caller owns every buffer; nothing is allocated inside a call.
@@ -55,7 +58,12 @@ typedef enum am_status {
   AM_ERR_TIMEOUT = 6,         /* (device) a bounded wait ran out            */
   AM_ERR_UNSUPPORTED = 7,     /* shape or dtype this build does not handle  */
   AM_WARN_NOT_CONVERGED = 8,  /* (device) NNLS stopped at its iteration cap */
-  AM_ERR_NOT_SPD = 9          /* (device) value-fit matrix not positive definite */
+  AM_ERR_NOT_SPD = 9,         /* (device) value-fit matrix not positive definite */
+  AM_WARN_MASS_UNDERFLOW = 10 /* (device) every fp32 feature of some reference
+                                 query underflowed to 0 (its best logit lies more
+                                 than ~87 below the head's shift): that query has
+                                 no mass, and it drops out of the NNLS and the
+                                 value fit (zero target, zero design row) */
 } am_status_t;
 
 typedef enum am_dtype { AM_BF16 = 0, AM_FP32 = 1 } am_dtype_t;
@@ -128,6 +136,12 @@ typedef struct am_opts {
    * key_offsets[h+1] − 1), key_bias is packed [Σ T_h], and each budget
    * satisfies 1 <= t_h <= T_h.  Read during the call only. */
   const int64_t* key_offsets;
+  /* Clock-cycle budget of each bounded device wait on an asynchronous copy
+   * or tensor-core step (0: 4e9 cycles, about 2 s).  A wait that runs out
+   * records AM_ERR_TIMEOUT for its head; the kernel then stops issuing
+   * work, waits (with the full budget) for what it already issued, releases
+   * its tensor memory and returns, so the context stays usable.  >= 0. */
+  int64_t wait_cycles;
 } am_opts_t;
 
 /* Fill *opts with defaults: bf16 inputs, k = 1, R = 1, scale = 1/sqrt(d),

@@ -56,7 +56,7 @@ def test_defaults_and_status_strings():
     assert (o.in_dtype, o.topk, o.refit_every) == (am.BF16, 1, 1)
     assert abs(o.ridge - 1e-6) < 1e-12 and abs(o.w_floor_rel - 1e-12) < 1e-18
     L = am.lib()
-    for code in range(10):
+    for code in range(11):
         assert L.am_status_string(code)
     assert L.am_version() >= 100
 

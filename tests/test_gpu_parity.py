@@ -454,3 +454,12 @@ def test_online_rounds_chained():
             b64 = np.asarray(h.key_bias, np.float64)
             r = O.compact_head(Q, K, V, on.budget, 4, 2, shift=shift_for(Q, K, b64), key_bias=b64)
             compacted.append((r["C_k"], np.float32(r["beta"]), r["C_v"]))
+
+
+@needs_cuda
+def test_value_fit_narrow_column_slices():
+    """A budget above 465 makes the value-fit solve take eight columns of C_v
+    per block (32 columns of X no longer fit in shared memory) for every head
+    of the call; a small head shares the launch."""
+    heads = [W.structured_head(590 + h, n=1024, T=1100) for h in range(2)]
+    check_all(heads, [480, 8], 4, 2, label="narrow solve")
