@@ -36,11 +36,12 @@ struct Layout {
   size_t phiT, phiT16, m, Y, r, corr, sel;
   size_t picks, pick_corr, plist, sorted_slot;
   size_t bvec, w, w_eff, ycache;
-  size_t G, L, AtA, A, AtY, nrm_part;
+  size_t G, L, AtA, A, Apl, Ypl, AtY, nrm_part;
   size_t cnorm, cnpart, rnorm, clist, clj, ccount, inv_m, korder, knorm, ksort, cprefix, cdone, cprobe, rows_eval, gpart, gcount, rcount,
       dinv;
   size_t total;
   size_t tables_bytes;
+  bool tc_normal;   // the value fit's normal equations run on the tensor cores (bf16 planes)
 };
 
 struct Tables {
@@ -64,6 +65,10 @@ bool bf16_copy(const am_opts_t* o) {
   return o->corr_mode == AM_CORR_STORED_BF16 && o->select_mode == AM_SELECT_OMP;
 }
 
+// The value fit forms its normal equations on the tensor cores (bf16 inputs,
+// d in {64, 128}); otherwise on CUDA cores in fp64.
+bool tc_normal(const am_opts_t* o, int d) { return o->in_dtype == AM_BF16 && (d == 64 || d == 128); }
+
 // Bytes of one wave's device tables: cu_t, cu_t2, koff [H+1] int64 and
 // t, Th, order, group order [H] int32 (a multiple of 8).
 size_t table_bytes(int H) { return (size_t)(H + 1) * 8 * 3 + (size_t)H * 4 * 4; }
@@ -74,12 +79,13 @@ size_t table_bytes(int H) { return (size_t)(H + 1) * 8 * 3 + (size_t)H * 4 * 4; 
 size_t prefix_bytes(int H) { return align_up(kWsHeaderBytes + (size_t)H * 4) + align_up((size_t)H * 64 + 256); }
 
 // One wave's region, from byte `o0` (the end of the prefix) on.
-Layout plan(int n, int T, int d, int H, int64_t sum_t, int64_t sum_t2, bool corr_bf16, size_t o0) {
+Layout plan(int n, int T, int d, int H, int64_t sum_t, int64_t sum_t2, bool corr_bf16, size_t o0, bool tc_normal) {
   Layout L{};
   const size_t ldn = (size_t)round_up(n, 32);
   size_t o = o0;
   auto take = [&](size_t bytes) { size_t at = o; o = align_up(o + bytes); return at; };
   L.tables_bytes = table_bytes(H);
+  L.tc_normal = tc_normal;
   L.shift = take((size_t)H * 4);
   L.np = take((size_t)H * 4);
   L.ylen = take((size_t)H * 4);
@@ -103,7 +109,11 @@ Layout plan(int n, int T, int d, int H, int64_t sum_t, int64_t sum_t2, bool corr
   L.G = take((size_t)sum_t2 * 8);
   L.L = take((size_t)sum_t2 * 8);
   L.AtA = take((size_t)sum_t2 * 8);
-  L.A = take((size_t)sum_t * ldn * 4);
+  // the design matrix: fp32 for the CUDA-core normal equations, or three bf16
+  // planes (and the targets' planes) for the tensor-core ones
+  L.A = take(tc_normal ? 0 : (size_t)sum_t * ldn * 4);
+  L.Apl = take(tc_normal ? (size_t)3 * sum_t * ldn * 2 : 0);
+  L.Ypl = take(tc_normal ? (size_t)3 * H * n * d * 2 : 0);
   L.AtY = take((size_t)sum_t * d * 8);
   L.nrm_part = take((size_t)kNormalMaxSplits * ((size_t)sum_t2 + (size_t)sum_t * d) * 8);
   L.cnorm = take((size_t)H * T * 8);
@@ -273,6 +283,8 @@ Work bind(const Layout& L, char* base, bool corr_bf16) {
   w.L = reinterpret_cast<double*>(base + L.L);
   w.AtA = reinterpret_cast<double*>(base + L.AtA);
   w.A = reinterpret_cast<float*>(base + L.A);
+  w.Apl = L.tc_normal ? reinterpret_cast<__nv_bfloat16*>(base + L.Apl) : nullptr;
+  w.Ypl = L.tc_normal ? reinterpret_cast<__nv_bfloat16*>(base + L.Ypl) : nullptr;
   w.AtY = reinterpret_cast<double*>(base + L.AtY);
   w.nrm_part = reinterpret_cast<double*>(base + L.nrm_part);
   w.cnorm = reinterpret_cast<double*>(base + L.cnorm);
@@ -366,20 +378,21 @@ struct WsHeader {
 };
 
 // Size of the wave region for heads [h0, h1) of `tb`.
-size_t wave_bytes(const Tables& tb, int n, int T, int d, int h0, int h1, bool corr_bf16) {
+size_t wave_bytes(const Tables& tb, int n, int T, int d, int h0, int h1, bool corr_bf16, bool tcn) {
   const int64_t st = tb.cu_t[h1] - tb.cu_t[h0], st2 = tb.cu_t2[h1] - tb.cu_t2[h0];
-  return plan(n, T, d, h1 - h0, st, st2, corr_bf16, 0).total;
+  return plan(n, T, d, h1 - h0, st, st2, corr_bf16, 0, tcn).total;
 }
 
 // Waves of consecutive heads: each takes as many heads as fit in `region`
 // bytes.  Empty when one head does not fit.
-std::vector<std::pair<int, int>> plan_waves(const Tables& tb, int n, int T, int d, bool corr_bf16, size_t region) {
+std::vector<std::pair<int, int>> plan_waves(const Tables& tb, int n, int T, int d, bool corr_bf16, bool tcn,
+                                            size_t region) {
   const int H = (int)tb.t.size();
   std::vector<std::pair<int, int>> waves;
   int h0 = 0;
   while (h0 < H) {
     int h1 = h0;
-    while (h1 < H && wave_bytes(tb, n, T, d, h0, h1 + 1, corr_bf16) <= region) ++h1;
+    while (h1 < H && wave_bytes(tb, n, T, d, h0, h1 + 1, corr_bf16, tcn) <= region) ++h1;
     if (h1 == h0) return {};
     waves.emplace_back(h0, h1);
     h0 = h1;
@@ -427,7 +440,7 @@ am_status_t am_workspace_size_waves(int32_t n, int32_t T, int32_t d, int32_t num
   const int W = std::min(wave_heads, num_heads);
   size_t region = 0;
   for (int h0 = 0; h0 + W <= num_heads; ++h0)
-    region = std::max(region, wave_bytes(tb, n, T, d, h0, h0 + W, bf16_copy(opts)));
+    region = std::max(region, wave_bytes(tb, n, T, d, h0, h0 + W, bf16_copy(opts), tc_normal(opts, d)));
   *bytes = prefix_bytes(num_heads) + region;
   return AM_OK;
 }
@@ -438,7 +451,8 @@ am_status_t am_workspace_view(int32_t n, int32_t T, int32_t d, int32_t num_heads
   Tables tb;
   am_status_t st = check_shape(n, T, d, num_heads, budgets, opts, &tb);
   if (st != AM_OK) return st;
-  const Layout L = plan(n, T, d, num_heads, tb.sum_t, tb.sum_t2, bf16_copy(opts), prefix_bytes(num_heads));
+  const Layout L = plan(n, T, d, num_heads, tb.sum_t, tb.sum_t2, bf16_copy(opts), prefix_bytes(num_heads),
+                        tc_normal(opts, d));
   view->phiT = L.phiT;
   view->mass = L.m;
   view->target = L.Y;
@@ -562,7 +576,8 @@ am_status_t compact_heads_impl(const void* Q, const void* K, const void* V, int3
   const bool bf16 = bf16_copy(opts);
   const size_t pre = prefix_bytes(H);
   if (workspace_bytes <= pre) return AM_ERR_WORKSPACE;
-  const std::vector<std::pair<int, int>> waves = plan_waves(tb, n, T, d, bf16, workspace_bytes - pre);
+  const bool tcn = tc_normal(opts, d);
+  const std::vector<std::pair<int, int>> waves = plan_waves(tb, n, T, d, bf16, tcn, workspace_bytes - pre);
   if (waves.empty()) return AM_ERR_WORKSPACE;
   // head groups on internal streams (one group: everything on the caller's stream)
   int G = std::max(1, std::min(max_groups, H));
@@ -583,11 +598,12 @@ am_status_t compact_heads_impl(const void* Q, const void* K, const void* V, int3
     const int h0 = waves[k].first, h1 = waves[k].second, Hw = h1 - h0;
     sub_tables(tb, h0, h1, kR, &wt[k]);
     set_groups(&wt[k], wt[k].passes, std::min(G, Hw));
-    const Layout L = plan(n, T, d, Hw, wt[k].sum_t, wt[k].sum_t2, bf16, pre);
+    const Layout L = plan(n, T, d, Hw, wt[k].sum_t, wt[k].sum_t2, bf16, pre, tcn);
     ww[k] = bind(L, base, bf16);
     ww[k].status = reinterpret_cast<int32_t*>(base + kWsHeaderBytes) + h0;
     ww[k].nrm_ata = wt[k].sum_t2;
     ww[k].nrm_stride = wt[k].sum_t2 + wt[k].sum_t * d;
+    ww[k].sum_t = wt[k].sum_t;
     pack_tables(wt[k], Hw, &host_tables, &ww[k], base + tables_at + host_tables.size(), &wgorder[k]);
   }
   if (host_tables.size() > pre - tables_at) return AM_ERR_WORKSPACE;   // cannot happen: 64 bytes per head

@@ -71,7 +71,9 @@ struct Work {
   int32_t* sorted_slot; // [Σt] pick slot of each ascending-position output row
   double* w_eff;        // [Σt] floored weights, ascending-position order
   double* ycache;       // [Σt] forward solve L⁻¹ b_P (factor order), kept across refits
-  float* A;             // [Σt][ldn] design matrix, key-major
+  float* A;             // [Σt][ldn] design matrix, key-major (CUDA-core normal equations)
+  __nv_bfloat16* Apl;   // [3][Σt][ldn] the design matrix as bf16 planes hi, mid, lo (tensor-core path)
+  __nv_bfloat16* Ypl;   // [3][H][n][d] the targets Y as bf16 planes hi, mid, lo (tensor-core path)
   double* AtA;          // [Σt²]
   double* AtY;          // [Σt][d]
   double* nrm_part;     // [kNormalMaxSplits][Σt² + Σt·d] split partials of AᵀA, AᵀY
@@ -95,6 +97,7 @@ struct Work {
   double* dinv;         // per head at 32·(cu_t[h] + 32h): inverses of the value-fit factor's 32×32 diagonal tiles
   int64_t nrm_ata;      // Σt²
   int64_t nrm_stride;   // Σt² + Σt·d
+  int64_t sum_t;        // Σt
 };
 
 constexpr int kRedBlocks = 64;   // partial-sum slots per head for ‖r‖²
@@ -109,6 +112,7 @@ constexpr int kSortSmemKeys = 16384;  // key counts the norm sort handles in sha
 constexpr int kGramMaxSlices = 32;    // query slices of the tiled Gram update
 constexpr int kGramMaxNew = 16;       // picks per pass the tiled Gram update takes
 constexpr int kNormalMaxSplits = 8;   // query splits of the normal-equation products
+constexpr int kQuerySplit = 2048;     // queries one tensor-core normal-equation CTA sums in fp32
 
 // ---- launchers (each file defines its own) ----
 // feature pass (am_phi_simt.cu)
@@ -151,6 +155,10 @@ cudaError_t launch_finalize(const Problem& p, const Work& w, const void* K, cons
                             void* C_k, float* beta, int32_t* indices, float* w_out,
                             int32_t* pick_order, float* pick_corr, cudaStream_t s);
 cudaError_t launch_value_fit(const Problem& p, const Work& w, float* C_v, cudaStream_t s);
+cudaError_t launch_normal_reduce(const Work& w, int splits, cudaStream_t s);
+// tensor-core normal equations (am_normal_tc.cu): bf16 inputs, d in {64, 128}
+bool normal_tc_supported(const Problem& p);
+cudaError_t launch_normal_tc(const Problem& p, const Work& w, cudaStream_t s);
 
 // The body of am_compact_heads; OMP passes of up to max_groups head groups run
 // concurrently on internal streams (1: everything on the caller's stream).
@@ -167,13 +175,24 @@ __device__ __forceinline__ float load_in(const void* base, int64_t idx, int dtyp
   return reinterpret_cast<const float*>(base)[idx];
 }
 
-__device__ __forceinline__ bool is_warning(int code) {
-  return code == AM_WARN_NOT_CONVERGED || code == AM_WARN_MASS_UNDERFLOW;
+// Severity of a device condition: a head keeps the most severe one it met.
+// A timeout leaves the head's work unfinished; non-finite values are the
+// cause of whatever else failed downstream (a value-fit matrix that is not
+// positive definite, an iteration cap); warnings rank below every error.
+__device__ __forceinline__ int severity(int code) {
+  switch (code) {
+    case AM_WARN_NOT_CONVERGED: return 1;
+    case AM_WARN_MASS_UNDERFLOW: return 2;
+    case AM_ERR_NOT_SPD: return 3;
+    case AM_ERR_NONFINITE: return 4;
+    default: return 5;   // AM_ERR_TIMEOUT
+  }
 }
 
+// Status words hold 1000·severity + code (0 for none), so the largest word is
+// the most severe condition and word % 1000 its code.
 __device__ __forceinline__ void record_status(int32_t* status, int code) {
-  // keep the most severe (largest) code; errors outrank the warnings
-  atomicMax(status, is_warning(code) ? 1000 + code : 2000 + code);
+  atomicMax(status, 1000 * severity(code) + code);
 }
 
 // Number of OMP passes for budget t: one correlation pass per refit interval.

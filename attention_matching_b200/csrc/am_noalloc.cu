@@ -34,8 +34,8 @@ cudaError_t scratch_address(void** out) {
   return cudaSuccess;
 }
 
-// Status words are stored most-severe-wins as 1000 + code (warning) or
-// 2000 + code (error); report the plain code.
+// Status words are stored most-severe-wins as 1000·severity + code; report
+// the plain code.
 __global__ void k_status_codes(const int32_t* words, int32_t* out, int H) {
   const int h = blockIdx.x * blockDim.x + threadIdx.x;
   if (h < H) out[h] = words[h] % 1000;

@@ -112,7 +112,20 @@ __global__ void __launch_bounds__(kDesignThreads) k_design(Problem p, Work w) {
     if (i < p.ldn)
       for (int q = 0; q < cn; ++q) {
         const double a = live ? (double)P0[(int64_t)sj[q] * p.ldn + i] * sw[q] * invD : 0.0;
-        w.A[(base + c0 + q) * p.ldn + i] = (float)a;
+        const int64_t at = (base + c0 + q) * p.ldn + i;
+        if (w.Apl) {
+          // fp32 value as three bf16 planes, af = hi + mid + lo exactly
+          const float af = (float)a;
+          const __nv_bfloat16 hi = __float2bfloat16_rn(af);
+          const float r1 = af - __bfloat162float(hi);
+          const __nv_bfloat16 mid = __float2bfloat16_rn(r1);
+          const int64_t plane = w.cu_t[p.H] * p.ldn;
+          w.Apl[at] = hi;
+          w.Apl[plane + at] = mid;
+          w.Apl[2 * plane + at] = __float2bfloat16_rn(r1 - __bfloat162float(mid));
+        } else {
+          w.A[at] = (float)a;
+        }
       }
   }
 }
@@ -398,6 +411,12 @@ cudaError_t launch_finalize(const Problem& p, const Work& w, const void* K, cons
   return cudaGetLastError();
 }
 
+cudaError_t launch_normal_reduce(const Work& w, int splits, cudaStream_t s) {
+  AM_LAUNCH(AM_STAGE_NORMAL, s,
+            k_normal_reduce<<<296, 256, 0, s>>>(w.nrm_ata, w.nrm_stride - w.nrm_ata, splits, w.nrm_stride, w));
+  return cudaGetLastError();
+}
+
 cudaError_t launch_value_fit(const Problem& p, const Work& w, float* C_v, cudaStream_t s) {
   dim3 gd((p.ldn + kDesignThreads - 1) / kDesignThreads, p.H);
   AM_LAUNCH(AM_STAGE_DESIGN, s, k_design<<<gd, kDesignThreads, 0, s>>>(p, w));
@@ -407,11 +426,14 @@ cudaError_t launch_value_fit(const Problem& p, const Work& w, float* C_v, cudaSt
   splits = splits < 1 ? 1 : (splits > kNormalMaxSplits ? kNormalMaxSplits : splits);
   if (splits > (p.n + NK_ - 1) / NK_) splits = (p.n + NK_ - 1) / NK_;
   const int64_t part_stride = w.nrm_stride;
-  dim3 gn(ta * (ta + 1) / 2 + ta * td, p.H, splits);
-  AM_LAUNCH(AM_STAGE_NORMAL, s, k_normal<<<gn, 256, 0, s>>>(p, w, splits, part_stride));
-  if (splits > 1)
-    AM_LAUNCH(AM_STAGE_NORMAL, s,
-              k_normal_reduce<<<296, 256, 0, s>>>(w.nrm_ata, w.nrm_stride - w.nrm_ata, splits, part_stride, w));
+  if (w.Apl) {
+    cudaError_t e = launch_normal_tc(p, w, s);
+    if (e != cudaSuccess) return e;
+  } else {
+    dim3 gn(ta * (ta + 1) / 2 + ta * td, p.H, splits);
+    AM_LAUNCH(AM_STAGE_NORMAL, s, k_normal<<<gn, 256, 0, s>>>(p, w, splits, part_stride));
+    if (splits > 1) launch_normal_reduce(w, splits, s);
+  }
   // factor: heads with t <= tl keep it in shared memory (beside the tile scratch) while factoring
   const size_t cap = 226 * 1024;
   const size_t scr = kTiledScratchDoubles * sizeof(double);

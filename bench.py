@@ -317,7 +317,10 @@ def stage_models(wl, n, key_counts, d, ldn, corr_kind, rows_evaluated, tc=True):
         "resid": {"bound": "hbm", "bytes": float(sum(s1)) * row + len(s1) * ldn * 12},
         "nnls": {"bound": "hbm", "bytes": float(sum(2 * x * x * 8 for x in s1))},
         "design": {"bound": "hbm", "bytes": float(sum(wl.budgets)) * row * 2},
-        "normal": {"bound": "fp64", "flops": float(sum(n * t * (t + 1) + 2 * n * t * d for t in wl.budgets))},
+        # AᵀA and AᵀY as a dense GEMM (2·n·t·(t + d) flops): on the tensor cores for bf16
+        # inputs with d in {64, 128} (six bf16 products per fp32 product), else fp64 FMA
+        "normal": ({"bound": "tensor", "flops": float(sum(2 * n * t * (t + d) for t in wl.budgets))} if tc else
+                   {"bound": "fp64", "flops": float(sum(n * t * (t + 1) + 2 * n * t * d for t in wl.budgets))}),
         "solve": {"bound": "fp64", "flops": float(sum(t ** 3 / 3 + 2 * t * t * d for t in wl.budgets))},
     }
     if corr_kind == "highest":

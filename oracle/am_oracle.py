@@ -258,7 +258,7 @@ def omp_select(Phi, m, t: int, topk: int = 1, refit_every: int = 1,
         order = cand[np.lexsort((cand, -c[cand]))]
         own = [int(j) for j in order[:kk]]
         rec = {
-            "round": rnd, "kk": kk, "c": c, "own": own,
+            "round": rnd, "kk": kk, "c": c, "own": own, "r_norm": float(np.linalg.norm(r)),
             "c_max": float(c[order[0]]),
             "c_kth": float(c[order[kk - 1]]),
             "c_next": float(c[order[kk]]) if order.size > kk else None,

@@ -5,7 +5,9 @@ replay because near-ties may legitimately go either way):
 
 * picks: the oracle replays the GPU's pick order; each GPU pick must be one
   of the oracle's own top-kk for that round, or have a correlation within
-  1e-4·|c_max| of the oracle's kk-th best;
+  tol·|c_max| of the oracle's kk-th best, tol = max(1e-4, U_FEAT·‖m‖/‖r‖)
+  (see U_FEAT below: the fp32 storage of Φ bounds the GPU's correlation
+  accuracy once the residual is small);
 * index sets: identical whenever every round of the oracle's own run
   separates its kk-th and (kk+1)-th correlations by more than 1e-4·|c_max|;
 * mass residual ‖m − Φ_S w‖/‖m‖ (both evaluated in float64 by the harness):
@@ -24,9 +26,23 @@ from oracle import am_oracle as O
 
 GAP_TOL = 1e-4
 RES_TOL = 1e-3
+# The GPU stores Φ in fp32 (each feature from the ex2 unit, a few ulp of
+# 2^-24) and forms r = m − Φ_S w from those stored values, so its residual
+# differs from the float64 one by about U_FEAT·‖m‖ and a correlation
+# c_j = φ_jᵀr by about U_FEAT·‖φ_j‖‖m‖: relative to the round's largest
+# correlation that is U_FEAT·‖m‖/‖r‖, which late in a long run (‖r‖ below
+# 1e-3·‖m‖) exceeds 1e-4.  The teacher-forced pick rule allows the larger of
+# 1e-4 and that bound, with U_FEAT = 8·2^-24 (four ulp of the exponential,
+# twice for the two terms of r).
+U_FEAT = 8.0 * 2.0 ** -24
 BETA_TOL = 1e-3
 OUT_TOL = 2e-3
 W_CMP_REL = 1e-6
+
+
+def pick_tolerance(m_norm, r_norm):
+    """Allowed pick slack in a round whose residual has norm r_norm."""
+    return max(GAP_TOL, U_FEAT * m_norm / max(r_norm, 1e-300))
 
 
 def split_head(out, h):
@@ -71,15 +87,17 @@ def check_head(g, Q, K, V, t, topk, refit, shift, key_bias=None, oracle_res=None
             oracle_res = O.compact_head(Q, K, V, t, topk, refit, shift=shift, key_bias=key_bias)
     o = oracle_res
     worst_slack = 0.0
+    m_norm = forced["rounds"][0]["r_norm"]          # r = m before the first refit
     for rec in forced["rounds"]:
         scale = max(abs(rec["c_max"]), 1e-300)
+        tol = pick_tolerance(m_norm, rec["r_norm"])
         for j in rec["picks"]:
             if j in rec["own"]:
                 continue
             slack = (rec["c_kth"] - rec["c"][j]) / scale
             worst_slack = max(worst_slack, slack)
             if exact_picks:
-                assert slack <= GAP_TOL, f"{label}: pick {j} in round {rec['round']} trails by {slack:.3g}"
+                assert slack <= tol, f"{label}: pick {j} in round {rec['round']} trails by {slack:.3g} (allowed {tol:.3g})"
     rep["pick_slack"] = worst_slack
 
     gaps = [(r["c_kth"] - r["c_next"]) / max(abs(r["c_max"]), 1e-300)
@@ -169,13 +187,16 @@ def check_head_prefix(g, Q, K, V, t, topk, refit, shift, key_bias=None, prefix=2
     forced = O.compact_head(Q, K, V, prefix, topk, refit, shift=shift, key_bias=key_bias,
                             forced_picks=g["pick_order"][:prefix])
     worst = 0.0
+    m_norm = forced["rounds"][0]["r_norm"]
     for rec in forced["rounds"]:
         sc = max(abs(rec["c_max"]), 1e-300)
+        tol = pick_tolerance(m_norm, rec["r_norm"])
         for j in rec["picks"]:
             if j not in rec["own"]:
-                worst = max(worst, (rec["c_kth"] - rec["c"][j]) / sc)
+                slack = (rec["c_kth"] - rec["c"][j]) / sc
+                worst = max(worst, slack)
+                assert slack <= tol, f"{label}: prefix pick {j} trails by {slack:.3g} (allowed {tol:.3g})"
     rep["pick_slack"] = worst
-    assert worst <= GAP_TOL, f"{label}: a prefix pick trails by {worst:.3g}"
     if all(set(r["picks"]) == set(r["own"]) for r in forced["rounds"]):
         own = forced
     else:
