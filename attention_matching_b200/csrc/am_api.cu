@@ -38,7 +38,7 @@ struct Layout {
   size_t bvec, w, w_eff, ycache;
   size_t G, L, AtA, A, Apl, Ypl, AtY, nrm_part;
   size_t cnorm, cnpart, rnorm, clist, clj, ccount, inv_m, korder, knorm, ksort, cprefix, cdone, cprobe, rows_eval, gpart, gcount, rcount,
-      dinv;
+      dinv, vinv;
   size_t total;
   size_t tables_bytes;
   bool tc_normal;   // the value fit's normal equations run on the tensor cores (bf16 planes)
@@ -136,6 +136,7 @@ Layout plan(int n, int T, int d, int H, int64_t sum_t, int64_t sum_t2, bool corr
   L.gcount = take(((size_t)sum_t + H) * 4);
   L.rcount = take((size_t)H * 4);
   L.dinv = take(((size_t)sum_t + 32 * (size_t)H) * 32 * 8);
+  L.vinv = take(((size_t)sum_t + 64 * (size_t)H) * 64 * 8);
   L.total = o;
   return L;
 }
@@ -305,6 +306,7 @@ Work bind(const Layout& L, char* base, bool corr_bf16) {
   w.gcount = reinterpret_cast<int32_t*>(base + L.gcount);
   w.rcount = reinterpret_cast<int32_t*>(base + L.rcount);
   w.dinv = reinterpret_cast<double*>(base + L.dinv);
+  w.vinv = reinterpret_cast<double*>(base + L.vinv);
   return w;
 }
 

@@ -8,12 +8,16 @@
 // they replaced, so attention over [compacted block, fresh keys] is the
 // mass-weighted mixture of the two blocks' local outputs.
 //
-//   k_attend   one block per (head, 8 queries): 32-key tiles of the
-//              concatenated key list (the compacted segment with bias β, then
-//              the fresh keys with bias 0) are staged in shared memory and
-//              shared by the block's 8 warps; in a warp, lane r scores key r
-//              of the tile against the warp's query, and each lane keeps d/32
-//              output dimensions of the online-softmax value sum, in fp32.
+//   k_attend   one block per (head, 8 queries), up to four key splits of 8
+//              warps: split s takes every nsplit-th 32-key tile of the concatenated key
+//              list (the compacted segment with bias β, then the fresh keys
+//              with bias 0), staged in its own shared memory and shared by its
+//              8 warps; in a warp, lane r scores key r of the tile against the
+//              warp's query, and each lane keeps d/32 output dimensions of the
+//              online-softmax value sum, in fp32.  The four splits' partial
+//              softmaxes (running maximum, weight sum, weighted values) are
+//              merged in shared memory at the end (split-key decoding inside
+//              one block: no global scratch).
 #include "am_internal.cuh"
 #include "am_profile.cuh"
 
@@ -23,36 +27,45 @@ namespace am {
 namespace {
 
 constexpr int kAttWarps = 8;       // queries per block
+constexpr int kAttMaxSplit = 4;    // key splits per block (fewer when shared memory is short)
 constexpr int kAttTile = 32;       // keys per staged tile (one per lane)
 constexpr int kAttPerLane = 8;     // d <= 32·8
 
 __device__ __forceinline__ float to_f(float x) { return x; }
 __device__ __forceinline__ float to_f(__nv_bfloat16 x) { return __bfloat162float(x); }
 
-// Shared memory of k_attend for head dim d: K tile [32][d + 1], V tile
-// [32][d], the warps' queries [8][d], tile biases [32], warps' weights [8][32].
-__host__ __device__ inline size_t attend_smem_bytes(int d) {
-  return sizeof(float) * ((size_t)kAttTile * (d + 1) + (size_t)kAttTile * d + (size_t)kAttWarps * d + kAttTile +
-                          (size_t)kAttWarps * kAttTile);
+// Shared memory of one key split for head dim d: K tile [32][d + 1], V tile
+// [32][d], tile biases [32], warps' weights [8][32]; then the block's queries
+// [8][d].  The merge reuses the splits' tiles.
+__host__ __device__ inline size_t attend_split_floats(int d) {
+  return (size_t)kAttTile * (d + 1) + (size_t)kAttTile * d + kAttTile + (size_t)kAttWarps * kAttTile;
+}
+__host__ __device__ inline size_t attend_smem_bytes(int d, int nsplit) {
+  return sizeof(float) * (nsplit * attend_split_floats(d) + (size_t)kAttWarps * d);
 }
 
 template <typename TK>
-__global__ void __launch_bounds__(kAttWarps * 32) k_attend(const TK* Q, int nq, int d, const TK* Ck,
-                                                           const float* beta, const float* Cv,
-                                                           const int64_t* cu_t, const TK* Kn, const TK* Vn,
-                                                           int Tn, float scale, float* out) {
+__global__ void __launch_bounds__(kAttWarps * kAttMaxSplit * 32) k_attend(const TK* Q, int nq, int d, const TK* Ck,
+                                                                          const float* beta, const float* Cv,
+                                                                          const int64_t* cu_t, const TK* Kn,
+                                                                          const TK* Vn, int Tn, float scale,
+                                                                          float* out, int nsplit) {
   extern __shared__ __align__(16) float sm[];
-  float* Ks = sm;                                  // [32][d + 1]
-  float* Vs = Ks + kAttTile * (d + 1);             // [32][d]
-  float* qs = Vs + kAttTile * d;                   // [8][d]
-  float* bs = qs + kAttWarps * d;                  // [32]
-  float* ps = bs + kAttTile;                       // [8][32]
+  const int lane = threadIdx.x & 31;
+  const int warp_all = threadIdx.x >> 5;
+  const int split = warp_all / kAttWarps, warp = warp_all % kAttWarps;
+  const int sthreads = kAttWarps * 32, stid = threadIdx.x % sthreads;   // threads of this split
+  float* Ks = sm + split * attend_split_floats(d);   // [32][d + 1]
+  float* Vs = Ks + kAttTile * (d + 1);               // [32][d]
+  float* bs = Vs + kAttTile * d;                     // [32]
+  float* ps = bs + kAttTile;                         // [8][32]
+  float* qs = sm + nsplit * attend_split_floats(d);   // [8][d], shared by the splits
   const int h = blockIdx.y;
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int i = blockIdx.x * kAttWarps + warp;
   const bool qlive = i < nq;
-  for (int e = lane; e < d; e += 32)
-    qs[warp * d + e] = qlive ? to_f(Q[((int64_t)h * nq + i) * d + e]) : 0.f;
+  if (split == 0)
+    for (int e = lane; e < d; e += 32) qs[warp * d + e] = qlive ? to_f(Q[((int64_t)h * nq + i) * d + e]) : 0.f;
+  __syncthreads();
   const int64_t c0 = cu_t[h];
   const int nc = (int)(cu_t[h + 1] - c0);
   const int ntot = nc + Tn;
@@ -60,9 +73,12 @@ __global__ void __launch_bounds__(kAttWarps * 32) k_attend(const TK* Q, int nq, 
 #pragma unroll
   for (int u = 0; u < kAttPerLane; ++u) acc[u] = 0.f;
   float mrun = -INFINITY, l = 0.f;
-  for (int k0 = 0; k0 < ntot; k0 += kAttTile) {
+  const int ntiles = (ntot + kAttTile - 1) / kAttTile;
+  // every split runs the same number of iterations (barriers are block-wide)
+  for (int it = 0; it < (ntiles + nsplit - 1) / nsplit; ++it) {
+    const int k0 = (it * nsplit + split) * kAttTile;
     __syncthreads();   // the previous tile is no longer read
-    for (int f = threadIdx.x; f < kAttTile * d; f += blockDim.x) {
+    for (int f = stid; f < kAttTile * d; f += sthreads) {
       const int r = f / d, e = f - r * d, g = k0 + r;
       float kv = 0.f, vv = 0.f;
       if (g < nc) {
@@ -76,9 +92,9 @@ __global__ void __launch_bounds__(kAttWarps * 32) k_attend(const TK* Q, int nq, 
       Ks[r * (d + 1) + e] = kv;
       Vs[r * d + e] = vv;
     }
-    if (threadIdx.x < kAttTile) {
-      const int g = k0 + threadIdx.x;
-      bs[threadIdx.x] = g < nc ? beta[c0 + g] : (g < ntot ? 0.f : -INFINITY);
+    if (stid < kAttTile) {
+      const int g = k0 + stid;
+      bs[stid] = g < nc ? beta[c0 + g] : (g < ntot ? 0.f : -INFINITY);
     }
     __syncthreads();
     // lane r: the logit of key r of the tile for this warp's query
@@ -87,14 +103,14 @@ __global__ void __launch_bounds__(kAttWarps * 32) k_attend(const TK* Q, int nq, 
     const float* qw = qs + warp * d;
     for (int e = 0; e < d; ++e) dot = fmaf(qw[e], kr[e], dot);
     const float b = bs[lane];
-    const float s = b == -INFINITY ? -INFINITY : fmaf(dot, scale, b);
-    float mt = s;
+    const float sc = b == -INFINITY ? -INFINITY : fmaf(dot, scale, b);
+    float mt = sc;
 #pragma unroll
     for (int o = 16; o; o >>= 1) mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, o));
     const float mnew = fmaxf(mrun, mt);
     if (mnew == -INFINITY) continue;   // warp-uniform: nothing finite yet
     const float a = expf(mrun - mnew);
-    const float pj = s == -INFINITY ? 0.f : expf(s - mnew);
+    const float pj = sc == -INFINITY ? 0.f : expf(sc - mnew);
     float psum = pj;
 #pragma unroll
     for (int o = 16; o; o >>= 1) psum += __shfl_xor_sync(0xffffffffu, psum, o);
@@ -114,13 +130,39 @@ __global__ void __launch_bounds__(kAttWarps * 32) k_attend(const TK* Q, int nq, 
     __syncwarp();
     mrun = mnew;
   }
-  if (!qlive) return;
-  const float il = l > 0.f ? 1.f / l : 0.f;
-  float* orow = out + ((int64_t)h * nq + i) * d;
+  // merge the splits' partial softmaxes: o = Σ_s e^{m_s − M} acc_s / Σ_s e^{m_s − M} l_s
+  __syncthreads();   // the tiles are free
+  float* part = sm;                                       // [split][warp][d] weighted values
+  float* pm = sm + (size_t)nsplit * kAttWarps * d;     // [split][warp] running maxima
+  float* pl = pm + nsplit * kAttWarps;                 // [split][warp] weight sums
 #pragma unroll
   for (int u = 0; u < kAttPerLane; ++u) {
     const int e = lane + 32 * u;
-    if (e < d) orow[e] = acc[u] * il;
+    if (e < d) part[(split * kAttWarps + warp) * d + e] = acc[u];
+  }
+  if (lane == 0) {
+    pm[split * kAttWarps + warp] = mrun;
+    pl[split * kAttWarps + warp] = l;
+  }
+  __syncthreads();
+  if (split != 0 || !qlive) return;
+  float M = -INFINITY;
+  for (int q = 0; q < nsplit; ++q) M = fmaxf(M, pm[q * kAttWarps + warp]);
+  float wsum = 0.f, wq[kAttMaxSplit];
+#pragma unroll
+  for (int q = 0; q < kAttMaxSplit; ++q) {
+    const float mq = q < nsplit ? pm[q * kAttWarps + warp] : -INFINITY;
+    wq[q] = mq == -INFINITY ? 0.f : expf(mq - M);
+    if (q < nsplit) wsum = fmaf(wq[q], pl[q * kAttWarps + warp], wsum);
+  }
+  const float il = wsum > 0.f ? 1.f / wsum : 0.f;
+  float* orow = out + ((int64_t)h * nq + i) * d;
+  for (int e = lane; e < d; e += 32) {
+    float o = 0.f;
+#pragma unroll
+    for (int q = 0; q < kAttMaxSplit; ++q)
+      if (q < nsplit) o = fmaf(wq[q], part[(q * kAttWarps + warp) * d + e], o);
+    orow[e] = o * il;
   }
 }
 
@@ -142,20 +184,23 @@ extern "C" am_status_t am_attend_packed(const void* Q, int32_t nq, int32_t d, in
   const float sc = scale > 0.f ? scale : (float)(1.0 / sqrt((double)d));
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   dim3 grid((nq + kAttWarps - 1) / kAttWarps, num_heads);
-  const size_t sm = attend_smem_bytes(d);   // d <= 256: at most 74 KiB
+  int nsplit = kAttMaxSplit;   // d <= 256: two splits always fit (at most 139 KiB)
+  while (nsplit > 1 && attend_smem_bytes(d, nsplit) > 227 * 1024) nsplit >>= 1;
+  const size_t sm = attend_smem_bytes(d, nsplit);
+  const int threads = kAttWarps * 32 * nsplit;
   if (in_dtype == AM_BF16) {
     cudaFuncSetAttribute(k_attend<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
     AM_LAUNCH(AM_STAGE_ATTEND, s,
-              k_attend<__nv_bfloat16><<<grid, kAttWarps * 32, sm, s>>>(
+              k_attend<__nv_bfloat16><<<grid, threads, sm, s>>>(
                   static_cast<const __nv_bfloat16*>(Q), nq, d, static_cast<const __nv_bfloat16*>(C_k), beta, C_v,
                   cu_t, static_cast<const __nv_bfloat16*>(K_new), static_cast<const __nv_bfloat16*>(V_new), T_new,
-                  sc, out));
+                  sc, out, nsplit));
   } else {
     cudaFuncSetAttribute(k_attend<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
     AM_LAUNCH(AM_STAGE_ATTEND, s,
-              k_attend<float><<<grid, kAttWarps * 32, sm, s>>>(
+              k_attend<float><<<grid, threads, sm, s>>>(
                   static_cast<const float*>(Q), nq, d, static_cast<const float*>(C_k), beta, C_v, cu_t,
-                  static_cast<const float*>(K_new), static_cast<const float*>(V_new), T_new, sc, out));
+                  static_cast<const float*>(K_new), static_cast<const float*>(V_new), T_new, sc, out, nsplit));
   }
   return cudaGetLastError() == cudaSuccess ? AM_OK : AM_ERR_CUDA;
 }

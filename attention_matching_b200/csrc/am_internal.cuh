@@ -95,6 +95,7 @@ struct Work {
   int32_t* gcount;      // [Σt + H] Gram blocks finished this pass, per head and row group
   int32_t* rcount;      // [H] bounded-correlation row blocks finished this launch
   double* dinv;         // per head at 32·(cu_t[h] + 32h): inverses of the value-fit factor's 32×32 diagonal tiles
+  double* vinv;         // per head at 64·(cu_t[h] + 64h): inverses of the 64×64 diagonal tiles (tiled solve)
   int64_t nrm_ata;      // Σt²
   int64_t nrm_stride;   // Σt² + Σt·d
   int64_t sum_t;        // Σt
@@ -156,6 +157,9 @@ cudaError_t launch_finalize(const Problem& p, const Work& w, const void* K, cons
                             int32_t* pick_order, float* pick_corr, cudaStream_t s);
 cudaError_t launch_value_fit(const Problem& p, const Work& w, float* C_v, cudaStream_t s);
 cudaError_t launch_normal_reduce(const Work& w, int splits, cudaStream_t s);
+// the value-fit solve for large budgets, tiled over many CTAs (am_valsolve.cu)
+cudaError_t launch_value_solve_tiled(const Problem& p, const Work& w, float* C_v, cudaStream_t s);
+constexpr int kTiledSolveMinT = 97;   // budgets from which a call uses the tiled solve
 // tensor-core normal equations (am_normal_tc.cu): bf16 inputs, d in {64, 128}
 bool normal_tc_supported(const Problem& p);
 cudaError_t launch_normal_tc(const Problem& p, const Work& w, cudaStream_t s);

@@ -434,6 +434,7 @@ cudaError_t launch_value_fit(const Problem& p, const Work& w, float* C_v, cudaSt
     AM_LAUNCH(AM_STAGE_NORMAL, s, k_normal<<<gn, 256, 0, s>>>(p, w, splits, part_stride));
     if (splits > 1) launch_normal_reduce(w, splits, s);
   }
+  if (p.max_t >= kTiledSolveMinT) return launch_value_solve_tiled(p, w, C_v, s);
   // factor: heads with t <= tl keep it in shared memory (beside the tile scratch) while factoring
   const size_t cap = 226 * 1024;
   const size_t scr = kTiledScratchDoubles * sizeof(double);

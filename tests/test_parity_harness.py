@@ -53,3 +53,20 @@ def test_harness_rejects_planted_mistakes(head, check):
     g["C_k"] = K[g["indices"]]
     with pytest.raises(AssertionError):
         run(g)
+
+
+def test_undetermined_weights_flags_only_ill_posed_splits():
+    """On well-separated columns every weight is fixed by the data; when a
+    column is repeated with a relative jitter far below fp32 precision the
+    split of weight between the twins is not, and only those twins are
+    flagged."""
+    from tests.parity import undetermined_weights
+    rng = np.random.default_rng(71)
+    A = rng.uniform(0.1, 1.0, (200, 6))
+    y = A @ np.array([1.0, 0.5, 2.0, 0.7, 1.3, 0.9])
+    w = O.nnls(A, y)
+    assert not undetermined_weights(A, y, w).any()
+    B = np.concatenate([A, A[:, :1] * (1.0 + 1e-9 * rng.standard_normal((200, 1)))], axis=1)
+    wb = O.nnls(B, y)
+    flags = undetermined_weights(B, y, wb)
+    assert set(np.flatnonzero(flags)) <= {0, 6}
