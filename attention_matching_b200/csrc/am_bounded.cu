@@ -56,45 +56,80 @@ __device__ __forceinline__ bool before(uint64_t a, int ja, uint64_t b, int jb) {
 }
 
 // ---------------------------------------------------------- column norms --
-// ‖Φ_{:,j}‖₂ in fp64 from the stored fp32 features: one warp per key.
+// Besides ‖Φ_{:,j}‖₂, every key gets an upper bound of its norm over each
+// residual query group g (the queries i with (i / 128) mod G == g, G =
+// resid_blocks(p): the groups whose ‖r_g‖² the residual update leaves), so
+// that |c_j| <= Σ_g ‖r_g‖·‖Φ_{g,j}‖ (Cauchy-Schwarz on each group) can skip
+// keys the global bound ‖r‖·‖Φ_{:,j}‖ keeps.  Group norms are raised by the
+// factor 1 + 2e-6 (covering fp32 partial sums and the fp32 store).
+constexpr double kBlockNormInflate = 1.0 + 2e-6;
+
+// ‖Φ_{:,j}‖₂ in fp64 from the stored fp32 features, and the group norms: one
+// warp per key; lane l takes float4 l of each 128-query segment.
 __global__ void __launch_bounds__(256) k_colnorm(Problem p, Work w) {
+  __shared__ double gsum[8][kRedBlocks];
   const int h = blockIdx.y;
-  const int j = blockIdx.x * 8 + (threadIdx.x >> 5);
+  const int wib = threadIdx.x >> 5;
+  const int j = blockIdx.x * 8 + wib;
   const int lane = threadIdx.x & 31;
   if (j >= p.T) return;
   if (j >= w.Th[h]) {   // no such key in this head: norm 0, sorted last, never evaluated
     if (lane == 0) w.cnorm[(int64_t)h * p.T + j] = 0.0;
+    for (int g = lane; g < kRedBlocks; g += 32) w.cnblk[((int64_t)h * p.T + j) * kRedBlocks + g] = 0.f;
     return;
   }
+  const int G = resid_blocks(p);
+  for (int g = lane; g < kRedBlocks; g += 32) gsum[wib][g] = 0.0;
+  __syncwarp();
   const float4* row = reinterpret_cast<const float4*>(w.phiT + ((int64_t)h * p.T + j) * p.ldn);
   const int n4 = p.ldn >> 2;
-  double a0 = 0.0, a1 = 0.0;
-  for (int i = lane; i < n4; i += 32) {
-    const float4 x = __ldcs(row + i);
-    a0 = fma((double)x.x, (double)x.x, a0);
-    a1 = fma((double)x.y, (double)x.y, a1);
-    a0 = fma((double)x.z, (double)x.z, a0);
-    a1 = fma((double)x.w, (double)x.w, a1);
+  double tot = 0.0;
+  for (int seg = 0; seg * 32 < n4; ++seg) {
+    const int i = seg * 32 + lane;
+    double a = 0.0;
+    if (i < n4) {
+      const float4 x = __ldcs(row + i);
+      a = fma((double)x.x, (double)x.x, a);
+      a = fma((double)x.y, (double)x.y, a);
+      a = fma((double)x.z, (double)x.z, a);
+      a = fma((double)x.w, (double)x.w, a);
+    }
+    a = warp_sum(a);
+    tot += a;
+    if (lane == 0) gsum[wib][seg % G] += a;
   }
-  const double s = warp_sum(a0 + a1);
-  if (lane == 0) w.cnorm[(int64_t)h * p.T + j] = sqrt(s);
+  __syncwarp();
+  if (lane == 0) w.cnorm[(int64_t)h * p.T + j] = sqrt(tot);
+  for (int g = lane; g < kRedBlocks; g += 32)
+    w.cnblk[((int64_t)h * p.T + j) * kRedBlocks + g] = g < G ? (float)(sqrt(gsum[wib][g]) * kBlockNormInflate) : 0.f;
 }
 
 // ‖Φ_{:,j}‖₂ from the feature pass's per-warp partial sums (fp32 sums of 32
 // fp32 squares, relative error below 4e-7): their fp64 total, raised by the
-// factor 1 + 1e-6 so the result stays an upper bound of the exact norm.
+// factor 1 + 1e-6 so the result stays an upper bound of the exact norm; and
+// the group norms from the same partials (a 128-query block is one segment).
 __global__ void __launch_bounds__(256) k_normsum(Problem p, Work w) {
   const int h = blockIdx.y;
   const int j = blockIdx.x * blockDim.x + threadIdx.x;
   if (j >= p.T) return;
+  float* blk = w.cnblk + ((int64_t)h * p.T + j) * kRedBlocks;
   if (j >= w.Th[h]) {   // no such key in this head: norm 0, sorted last, never evaluated
     w.cnorm[(int64_t)h * p.T + j] = 0.0;
+    for (int g = 0; g < kRedBlocks; ++g) blk[g] = 0.f;
     return;
   }
-  const int parts = 4 * ((p.n + 127) / 128);
-  const float* src = w.cnpart + (int64_t)h * parts * p.T + j;
+  const int nqb = (p.n + 127) / 128;
+  const int G = resid_blocks(p);
+  const float* src = w.cnpart + (int64_t)h * 4 * nqb * p.T + j;
   double s = 0.0;
-  for (int k = 0; k < parts; ++k) s += (double)src[(int64_t)k * p.T];
+  for (int g = 0; g < kRedBlocks; ++g) {
+    double sg = 0.0;
+    if (g < G)
+      for (int qb = g; qb < nqb; qb += G)
+        for (int k = 0; k < 4; ++k) sg += (double)src[(int64_t)(qb * 4 + k) * p.T];
+    s += sg;
+    blk[g] = g < G ? (float)(sqrt(sg) * kBlockNormInflate) : 0.f;
+  }
   w.cnorm[(int64_t)h * p.T + j] = sqrt(s) * (1.0 + 1e-6);
 }
 
@@ -295,12 +330,14 @@ __device__ void theta_and_prefix(const Problem& p, const Work& w, int h, int pas
   const int L = useful ? prefix_not_below(w.knorm + (int64_t)h * p.T, p.T, thr, sample0) : p.T;
   const bool done = L <= p0;
   if (threadIdx.x == 0) {
-    w.cprefix[h] = L;   // the next pass sizes its probe by it
+    w.cprefix[h] = L;
     w.cprobe[h] = p0;
     w.cdone[h] = done;
     w.rnorm[h] = rn;
+    w.ctheta[h] = theta;   // the second launch skips keys whose group bound is below it
     if (done) {
       w.rows_eval[h] += (unsigned long long)staged;
+      w.cpassed[h] = staged;   // the next pass sizes its probe by it
       w.ccount[h] = 0;   // the list is consumed; otherwise the second launch extends it
     }
   }
@@ -360,6 +397,7 @@ __device__ void pick_from_prefix(const Problem& p, const Work& w, int h, int s0,
   }
   if (threadIdx.x == 0) {
     w.rows_eval[h] += (unsigned long long)n;
+    w.cpassed[h] = n;   // the next pass sizes its probe by it
     w.ccount[h] = 0;
   }
   append_picks(p, w, h, s0, kk, S);
@@ -368,6 +406,11 @@ __device__ void pick_from_prefix(const Problem& p, const Work& w, int h, int s0,
 // ------------------------------------------------------------ exact rows --
 // c_j = Σ_i r_i Φ_ij for the unselected keys at sorted positions [0, P0)
 // (which = 0) or [P0, L) (which = 1), in fp64 sums of exact fp32 products.
+// In the second launch a key is first tested against the group bound
+// Σ_g ‖r_g‖·‖Φ_{g,j}‖ (1 + 1e-6): below θ it cannot reach the picks and its
+// row is not read.  ‖r_g‖ comes from the fp64 residual's per-group sums
+// (k_init before the first refit, k_resid after); the fp32 copy the rows
+// are correlated with is larger by at most 2^-24 relative, inside the margin.
 // Four warps share a key, each summing a quarter of the queries with eight
 // columns per lane in flight; the quarters are added in a fixed order.  The
 // last block of a head to finish (counted with an atomic) then takes the
@@ -388,9 +431,9 @@ __global__ void __launch_bounds__(kSelThreads) k_rows(Problem p, Work w, int pas
   if (s0 >= s1) return;
   const int kk = s1 - s0;
   if (which && w.cdone[h]) return;                     // the probe step made the picks
-  // the probe reaches 5/4 of the previous pass's prefix plus 32 (kept in
-  // cprefix until the probe's last block replaces it), at most kSelCap positions
-  const int lprev = w.cprefix[h];
+  // the probe reaches 5/4 of the keys the previous pass evaluated plus 32, at
+  // most kSelCap positions
+  const int lprev = w.cpassed[h];
   const int p0 = which ? w.cprobe[h] : min(min(p.T, kSelCap), max(kProbe + s0, lprev + lprev / 4 + 32));
   const int lo = which ? p0 : 0;
   const int hi = which ? w.cprefix[h] : p0;
@@ -402,10 +445,28 @@ __global__ void __launch_bounds__(kSelThreads) k_rows(Problem p, Work w, int pas
   const int n4 = p.ldn >> 2;
   const int per = (n4 + kRowSplit - 1) / kRowSplit;
   const int c0 = quarter * per, c1 = min(n4, c0 + per);
+  // the second launch's key filter: ‖r_g‖ per group, and θ
+  __shared__ double rg[kRedBlocks];
+  const bool filter = which && w.cnblk != nullptr;
+  const int G = resid_blocks(p);
+  double theta = 0.0;
+  if (filter) {
+    for (int g = threadIdx.x; g < kRedBlocks; g += blockDim.x)
+      rg[g] = g < G ? sqrt(w.rr_part[(int64_t)h * kRedBlocks + g]) : 0.0;
+    theta = w.ctheta[h];
+    __syncthreads();
+  }
   for (int q0 = lo + blockIdx.x * kRowsPerBlock; q0 < hi; q0 += gridDim.x * kRowsPerBlock) {
     const int q = q0 + slot;
     const int j = q < hi ? ord[q] : 0;
-    const bool on = q < hi && !sel[j];
+    bool on = q < hi && !sel[j];
+    if (filter && on) {
+      // every warp of the key forms the same bound (same order of operations)
+      const float* bj = w.cnblk + ((int64_t)h * p.T + j) * kRedBlocks;
+      double b = (double)bj[lane] * rg[lane] + (double)bj[lane + 32] * rg[lane + 32];
+      b = warp_sum(b) * (1.0 + 1e-6);
+      on = !(b < theta);
+    }
     double a[4] = {0.0, 0.0, 0.0, 0.0};
     if (on) {
       const float4* row = reinterpret_cast<const float4*>(w.phiT + ((int64_t)h * p.T + j) * p.ldn);

@@ -90,6 +90,10 @@ struct Work {
   int32_t* cprefix;     // [H] this pass evaluates the keys at sorted positions [0, cprefix)
   int32_t* cdone;       // [H] 1 when the probe step already made this pass's picks
   int32_t* cprobe;      // [H] the probe length P0 of this pass
+  float* cnblk;         // [H][T][kRedBlocks] per residual query group g, an upper bound of ‖Φ_{i∈g, j}‖₂
+                        // (group g: queries i with (i / 128) mod resid_blocks == g), or null
+  double* ctheta;       // [H] this pass's threshold θ, the kk-th largest value the probe found
+  int32_t* cpassed;     // [H] keys whose correlation the last pass evaluated (sizes the next probe)
   unsigned long long* rows_eval;   // [H] keys evaluated, summed over the passes
   double* gpart;        // [kGramMaxSlices·(Σt + H)·kR] Gram partial sums per query slice
   int32_t* gcount;      // [Σt + H] Gram blocks finished this pass, per head and row group

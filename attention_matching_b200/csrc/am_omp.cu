@@ -37,6 +37,19 @@ __global__ void k_init(Problem p, Work w) {
   double acc = 0.0;
   for (int i = threadIdx.x; i < p.n; i += blockDim.x) acc += m[i] * m[i];
   acc = block_sum(acc, scratch);
+  // Σ m² per residual query group (the groups of k_resid's ‖r‖² partials):
+  // r = m until the first refit; warp w takes groups w, w + 8, ...
+  {
+    const int G = resid_blocks(p), lane = threadIdx.x & 31, nw = blockDim.x >> 5;
+    const int nseg = p.ldn / 128 + (p.ldn % 128 ? 1 : 0);
+    for (int g = threadIdx.x >> 5; g < G; g += nw) {
+      double sg = 0.0;
+      for (int seg = g; seg < nseg; seg += G)
+        for (int i = seg * 128 + lane; i < min(p.ldn, seg * 128 + 128); i += 32) sg += m[i] * m[i];
+      sg = warp_sum(sg);
+      if (lane == 0) w.rr_part[(int64_t)h * kRedBlocks + g] = sg;
+    }
+  }
   if (threadIdx.x == 0) {
     w.mm[h] = acc;
     w.np[h] = 0;

@@ -260,7 +260,8 @@ def oracle_sample(wl, seconds, order):
 def cpu_baseline(wl, seconds):
     """The oracle (as it stands) on a bounded sample of the workload's heads:
     a seeded random order over the heads whose budget is at most the median
-    (so that no single head exceeds the time budget).  The whole workload's
+    and at most 300 (so that no single head exceeds the time budget; when no
+    head qualifies, the smallest budgets).  The whole workload's
     oracle time is extrapolated with per-head time = a + b·cost_h, cost_h =
     t_h·⌈t_h/(k·R)⌉, a and b >= 0 fitted to the sampled heads by least squares
     (with one sampled head or one distinct cost: proportional to cost).  The
@@ -271,8 +272,11 @@ def cpu_baseline(wl, seconds):
     from attention_matching_b200.sharding import head_cost
     kR = wl.topk * wl.refit_every
     cost = np.array([head_cost(t, kR) for t in wl.budgets], dtype=np.float64)
-    med = float(np.median(wl.budgets))
-    order = [h for h in range(len(wl.heads)) if wl.budgets[h] <= med]
+    cap = min(float(np.median(wl.budgets)), 300.0)
+    order = [h for h in range(len(wl.heads)) if wl.budgets[h] <= cap]
+    if not order:
+        lo = min(wl.budgets)
+        order = [h for h in range(len(wl.heads)) if wl.budgets[h] == lo]
     random.Random(12345).shuffle(order)
     done, each, cores = oracle_sample(wl, seconds, order)
     c, tm = cost[done], np.array(each)
@@ -287,7 +291,7 @@ def cpu_baseline(wl, seconds):
     return {"value": len(wl.heads) / whole, "unit": "heads/s", "cores": cores, "kind": "oracle",
             "s_per_workload_extrapolated": whole,
             "sample": f"{len(done)} of {len(wl.heads)} heads of {wl.name} (seeded random order over budgets "
-                      f"<= the median; sampled budgets {sorted(wl.budgets[h] for h in done)}), float64 "
+                      f"<= min(median, 300); sampled budgets {sorted(wl.budgets[h] for h in done)}), float64 "
                       f"NumPy/SciPy oracle, {dt:.1f} s wall; workload time extrapolated as "
                       f"sum(a + b*t*ceil(t/(k*R))) with a = {a:.3g} s, b = {b:.3g} s fitted to the sample"}
 

@@ -13,8 +13,9 @@ replay because near-ties may legitimately go either way):
 * mass residual ‖m − Φ_S w‖/‖m‖ (both evaluated in float64 by the harness):
   within 1e-3 of the oracle's;
 * β: within 1e-3 absolute where the oracle's w >= 1e-6·max(w) and the data
-  fix w to that precision (undetermined_weights: an fp32-sized perturbation
-  of the features does not move the oracle's own β by more than 5e-4);
+  fix w to that precision (undetermined_weights: the first-order
+  componentwise least-squares bound for fp32-sized errors in Φ and m keeps
+  the oracle's own β within 5e-4);
   elsewhere both sides' β − b_S at most log(1e-6·max w) + 1e-3; compared
   against the oracle re-run on the GPU's own picks when the index sets differ;
 * reconstructed output softmax(Q C_kᵀ/√d + β) C_v, in float64: relative
@@ -42,28 +43,35 @@ OUT_TOL = 2e-3
 W_CMP_REL = 1e-6
 
 
-def undetermined_weights(Phi_S, m, w, draws=2, seed=0):
-    """Keys whose NNLS weight the data does not fix to the β tolerance at the
-    precision the GPU stores its features in: the oracle re-solves the NNLS
-    on Φ_S and m perturbed entry by entry by ±U_FEAT (relative, random signs;
-    the size of the fp32 storage error), started from its own weights, and a
-    key counts as undetermined when its β = log w moves by more than
-    BETA_TOL / 2 in any draw.  On ill-conditioned subsets (near-collinear
-    exp features late in a long selection) the minimiser's residual is
-    unique but w is not fixed by fp32 data, so β is compared only where it
-    is determined; the mass residual and the output are still compared in
-    full.  Returns a boolean mask aligned with w."""
-    rng = np.random.default_rng(seed)
-    wmax = float(w.max())
-    floor = 1e-12 * wmax
-    base = np.log(np.maximum(w, floor))
-    moved = np.zeros(w.shape, dtype=bool)
-    for _ in range(draws):
-        P = Phi_S * (1.0 + U_FEAT * rng.choice([-1.0, 1.0], size=Phi_S.shape))
-        m2 = m * (1.0 + U_FEAT * rng.choice([-1.0, 1.0], size=m.shape))
-        w2 = O.nnls(P, m2, x0=w)
-        moved |= np.abs(np.log(np.maximum(w2, floor)) - base) > BETA_TOL / 2
-    return moved
+def undetermined_weights(Phi_S, m, w):
+    """Keys whose NNLS weight the data do not fix to the β tolerance at the
+    precision the GPU stores its features in.  On the oracle's passive set P
+    (w > 0) the minimiser is the least-squares solution of Φ_P w_P = m, and the
+    first-order componentwise perturbation bound for least squares (for
+    |δΦ| <= u|Φ| and |δm| <= u|m| entrywise) is
+        |δw_P| <= u·( |Φ_P⁺|·(|m| + |Φ_P| w_P) + |(Φ_PᵀΦ_P)⁻¹|·|Φ_P|ᵀ|r| ),
+    with u = U_FEAT (the fp32 storage error of Φ and m) and r = m − Φ_P w_P.
+    A key counts as undetermined when that bound exceeds BETA_TOL/2 of its
+    weight (β = log w then moves by more than 5e-4).  On ill-conditioned
+    subsets (near-collinear exp features late in a long selection) the
+    minimising residual is unique but w is not fixed by fp32 data, so β is
+    compared only where it is determined; the mass residual and the output
+    are still compared in full.  Returns a boolean mask aligned with w."""
+    from scipy.linalg import solve_triangular
+    w = np.asarray(w, np.float64)
+    P = np.flatnonzero(w > 0)
+    out = np.zeros(w.shape, dtype=bool)
+    if P.size == 0:
+        return out
+    A = np.asarray(Phi_S, np.float64)[:, P]
+    Qm, R = np.linalg.qr(A, mode="reduced")
+    Apinv = solve_triangular(R, Qm.T, lower=False)              # Φ_P⁺ = R⁻¹Qᵀ
+    Rinv = solve_triangular(R, np.eye(P.size), lower=False)
+    GinvAbs = np.abs(Rinv @ Rinv.T)                              # |(Φ_PᵀΦ_P)⁻¹|
+    r = m - A @ w[P]
+    dw = U_FEAT * (np.abs(Apinv) @ (np.abs(m) + A @ w[P]) + GinvAbs @ (A.T @ np.abs(r)))
+    out[P] = dw > (BETA_TOL / 2) * w[P]
+    return out
 
 
 def pick_tolerance(m_norm, r_norm):

@@ -62,3 +62,64 @@ def test_tight_cauchy_schwarz_cases(seed):
     for kk in (1, 4, 8):
         for probe in (kk, 64, 256):
             check(Phi32, r64, probe, kk)
+
+
+# ---------------------------------------------------------------------------
+# The group bound of the second launch: |c_j| <= Σ_g ‖r_g‖·‖Φ_{g,j}‖, with the
+# queries split into groups g = (i / 128) mod G (the residual update's
+# partial sums), group norms from fp32 partial sums of 32 squares raised by
+# 1 + 2e-6 and stored in fp32, and the sum raised by 1 + 1e-6.  A key whose
+# bound is below θ is skipped: its c_j must be below θ too.
+# ---------------------------------------------------------------------------
+
+def group_bound(Phi32, r64, G):
+    n, T = Phi32.shape
+    seg = np.arange(n) // 128
+    g_of = seg % G
+    # fp32 partial sums of 32 squares (one warp's rows), then fp64 over partials
+    sq = (Phi32.astype(np.float32) ** 2)
+    pad = (-n) % 32
+    sqp = np.concatenate([sq, np.zeros((pad, T), np.float32)]) if pad else sq
+    part = sqp.reshape(-1, 32, T).sum(axis=1, dtype=np.float32).astype(np.float64)   # [n/32, T]
+    part_g = (np.arange(part.shape[0]) * 32 // 128) % G
+    gn = np.zeros((G, T))
+    for g in range(G):
+        gn[g] = np.sqrt(part[part_g == g].sum(axis=0))
+    gn32 = (gn * (1.0 + 2e-6)).astype(np.float32).astype(np.float64)
+    rg = np.sqrt(np.array([(r64[g_of == g] ** 2).sum() for g in range(G)]))
+    return (rg[:, None] * gn32).sum(axis=0) * (1.0 + 1e-6)
+
+
+@pytest.mark.parametrize("seed", range(20))
+def test_group_bound_never_excludes_a_key_that_reaches_theta(seed):
+    rng = np.random.default_rng(300 + seed)
+    n, T = int(rng.integers(130, 1200)), int(rng.integers(200, 900))
+    G = min((n + 127) // 128, 64)
+    # features concentrated on a few queries per key, as attention mass is
+    Phi = np.exp(rng.standard_normal((n, T)) * 1.5 - 4.0)
+    Phi32 = Phi.astype(np.float32)
+    w = np.abs(rng.standard_normal(T)) * (rng.random(T) < 0.05)
+    r64 = Phi32.astype(np.float64).sum(axis=1) - Phi32.astype(np.float64) @ w
+    c = Phi32.astype(np.float64).T @ r64.astype(np.float32).astype(np.float64)
+    bound = group_bound(Phi32, r64, G)
+    assert np.all(np.abs(c) <= bound), np.max(np.abs(c) / bound)
+    # tighter than the global bound, and usually much tighter
+    glob = np.sqrt((r64 ** 2).sum()) * np.sqrt((Phi32.astype(np.float64) ** 2).sum(axis=0))
+    assert np.all(bound <= glob * (1 + 1e-5))
+    for kk in (1, 4, 16):
+        theta = np.sort(c)[::-1][kk - 1]
+        skipped = bound < theta
+        assert np.all(c[skipped] < theta)
+
+
+def test_group_bound_is_tight_when_the_residual_sits_in_one_group():
+    """r supported on one group and parallel to one key's features there:
+    that key's bound equals its correlation to within the margins."""
+    rng = np.random.default_rng(7)
+    n, T, G = 512, 50, 4
+    Phi32 = np.exp(rng.standard_normal((n, T))).astype(np.float32)
+    r64 = np.zeros(n)
+    r64[128:256] = Phi32[128:256, 3].astype(np.float64) * 0.7
+    c = Phi32.astype(np.float64).T @ r64.astype(np.float32).astype(np.float64)
+    bound = group_bound(Phi32, r64, G)
+    assert c[3] <= bound[3] <= c[3] * (1 + 1e-5)

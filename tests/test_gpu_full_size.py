@@ -71,6 +71,11 @@ def test_online_round_full_size_with_prior_bias():
     out = _run(heads, [t] * H, 4, 2, shifts, key_bias=kb)
     res = out["residual"].cpu().numpy()
     pick = sorted({0, int(np.argmax(res)), int(np.argmin(res))})
+    # the GPU's own fp64 weights solve the NNLS of its own stored features
+    import attention_matching_b200 as am
+    f = am.features(out, n, T, 128, [t] * H, 4, 2, am.BF16)
+    for h in pick:
+        check_refit_kkt(out, f, h, n)
     reps = check_heads_parallel([_job("full", out, heads, h, t, 4, 2, shifts[h], kb[h], f"online head {h}")
                                  for h in pick])
     for r in reps:
