@@ -223,8 +223,11 @@ void finish_tables(Tables* tb, int kR) {
   tb->sum_t2 = tb->cu_t2[H];
   tb->order.resize(H);
   for (int h = 0; h < H; ++h) tb->order[h] = h;
-  std::stable_sort(tb->order.begin(), tb->order.end(),
-                   [&](int a, int b) { return passes[a] > passes[b]; });
+  // by pass count, then budget, descending: the heads whose NNLS factor
+  // lives in the workspace (the largest budgets) lead every group's order
+  std::stable_sort(tb->order.begin(), tb->order.end(), [&](int a, int b) {
+    return passes[a] != passes[b] ? passes[a] > passes[b] : tb->t[a] > tb->t[b];
+  });
   const int maxp = passes[tb->order[0]];
   tb->active.assign(maxp, 0);
   for (int q = 0; q < maxp; ++q)
@@ -536,9 +539,21 @@ am_status_t run_wave(const Problem& p, Work w, const Tables& tb, int G, int32_t*
   AM_TRY(cudaMemsetAsync(w.ccount, 0, (size_t)H * 4, s));
   if (p.select_highest) AM_TRY(launch_select_highest(p, w, s));
   const CorrInputs cin{io.Q, io.K, io.key_bias};
+  // the NNLS refit keeps a head's factor in shared memory when its budget is
+  // at most lcap; per pass, the active heads above it (a prefix of the order)
+  // get a launch of their own with a small shared-memory footprint
+  const int lcap = nnls_smem_cap(p.max_t);
+  // (count of those, largest budget among the rest)
+  auto big_heads = [&](const int32_t* ord, int active) {
+    int nb = 0;
+    while (nb < active && tb.t[ord[nb]] > lcap) ++nb;
+    return std::make_pair(nb, nb < active ? (int)tb.t[ord[nb]] : 0);
+  };
   if (G == 1) {
-    for (int pass = 0; pass < (int)tb.active.size(); ++pass)
-      AM_TRY(launch_omp_pass(p, w, pass, tb.active[pass], cin, s));
+    for (int pass = 0; pass < (int)tb.active.size(); ++pass) {
+      const auto bh = big_heads(tb.order.data(), tb.active[pass]);
+      AM_TRY(launch_omp_pass(p, w, pass, tb.active[pass], bh.first, bh.second, cin, s));
+    }
   } else {
     // fork the groups off the caller's stream, issue their passes interleaved,
     // and make the caller's stream wait for every group
@@ -553,8 +568,10 @@ am_status_t run_wave(const Problem& p, Work w, const Tables& tb, int G, int32_t*
     const int maxp = (int)tb.active.size();
     for (int pass = 0; pass < maxp; ++pass)
       for (int g = 0; g < G; ++g)
-        if (pass < (int)tb.gactive[g].size())
-          AM_TRY(launch_omp_pass(p, wg[g], pass, tb.gactive[g][pass], cin, group_stream(g)));
+        if (pass < (int)tb.gactive[g].size()) {
+          const auto bh = big_heads(tb.gorder.data() + tb.gstart[g], tb.gactive[g][pass]);
+          AM_TRY(launch_omp_pass(p, wg[g], pass, tb.gactive[g][pass], bh.first, bh.second, cin, group_stream(g)));
+        }
     for (int g = 0; g < G; ++g) {
       AM_TRY(cudaEventCreateWithFlags(&join[g], cudaEventDisableTiming));
       AM_TRY(cudaEventRecord(join[g], group_stream(g)));

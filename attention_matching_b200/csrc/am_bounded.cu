@@ -431,10 +431,10 @@ __global__ void __launch_bounds__(kSelThreads) k_rows(Problem p, Work w, int pas
   if (s0 >= s1) return;
   const int kk = s1 - s0;
   if (which && w.cdone[h]) return;                     // the probe step made the picks
-  // the probe reaches 5/4 of the keys the previous pass evaluated plus 32, at
-  // most kSelCap positions
-  const int lprev = w.cpassed[h];
-  const int p0 = which ? w.cprobe[h] : min(min(p.T, kSelCap), max(kProbe + s0, lprev + lprev / 4 + 32));
+  // the probe: the first kProbe + s0 positions of the norm order (s0 keys are
+  // already selected), at most kSelCap; the rest of the prefix is filtered
+  // by the group bound in the second launch
+  const int p0 = which ? w.cprobe[h] : min(min(p.T, kSelCap), kProbe + s0);
   const int lo = which ? p0 : 0;
   const int hi = which ? w.cprefix[h] : p0;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;

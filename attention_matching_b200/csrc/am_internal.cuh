@@ -145,8 +145,12 @@ struct CorrInputs {
   const void* K;
   const float* key_bias;
 };
-cudaError_t launch_omp_pass(const Problem& p, const Work& w, int pass, int active_heads,
-                            const CorrInputs& in, cudaStream_t s);
+// big_heads: how many of the first active heads of w.order keep their NNLS
+// factor in the workspace (budget above nnls_smem_cap(max_t)); small_tmax:
+// the largest budget among the other active heads
+cudaError_t launch_omp_pass(const Problem& p, const Work& w, int pass, int active_heads, int big_heads,
+                            int small_tmax, const CorrInputs& in, cudaStream_t s);
+int nnls_smem_cap(int max_t);
 // bounded correlation pass (am_bounded.cu): column norms once, then per pass
 // probe, exact rows, extension, exact rows, selection
 cudaError_t launch_column_norms(const Problem& p, const Work& w, cudaStream_t s);

@@ -1221,8 +1221,14 @@ cudaError_t launch_omp_init(const Problem& p, const Work& w, cudaStream_t s) {
   return cudaGetLastError();
 }
 
-cudaError_t launch_omp_pass(const Problem& p, const Work& w, int pass, int active, const CorrInputs& in,
-                            cudaStream_t s) {
+int nnls_smem_cap(int max_t) {
+  int lcap = 0;
+  nnls_smem_bytes(max_t, &lcap);
+  return lcap;
+}
+
+cudaError_t launch_omp_pass(const Problem& p, const Work& w, int pass, int active, int big, int small_tmax,
+                            const CorrInputs& in, cudaStream_t s) {
   if (active <= 0) return cudaSuccess;
   if (p.select_highest) {
     // the picks were made up front; this pass feeds the next kR of them to the refit
@@ -1260,7 +1266,20 @@ cudaError_t launch_omp_pass(const Problem& p, const Work& w, int pass, int activ
   int lcap;
   size_t sm = nnls_smem_bytes(p.max_t, &lcap);
   cudaFuncSetAttribute(k_nnls, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemCap);
-  AM_LAUNCH(AM_STAGE_NNLS, s, launch_chained(k_nnls, dim3(active), dim3(kNnlsThreads), sm, s, p, w, pass, lcap));
+  // heads whose factor lives in the workspace: the vectors alone in shared
+  // memory, so several CTAs share an SM; then the others with the factor
+  if (big > 0)
+    AM_LAUNCH(AM_STAGE_NNLS, s,
+              launch_chained(k_nnls, dim3(big), dim3(kNnlsThreads), nnls_vec_bytes(p.max_t), s, p, w, pass, 0));
+  if (active > big) {
+    Work ws = w;
+    ws.order = w.order + big;
+    // shared memory for the largest factor of this launch, not of the whole call
+    const size_t sm_small = nnls_vec_bytes(p.max_t) + nnls_tri_bytes(small_tmax < lcap ? small_tmax : lcap);
+    AM_LAUNCH(AM_STAGE_NNLS, s,
+              launch_chained(k_nnls, dim3(active - big), dim3(kNnlsThreads), sm_small < sm ? sm_small : sm, s, p,
+                             ws, pass, lcap));
+  }
   dim3 gr(resid_blocks(p), active);
   AM_LAUNCH(AM_STAGE_RESID, s, launch_chained(k_resid, gr, dim3(kResidThreads), 0, s, p, w, pass));
   return cudaGetLastError();

@@ -19,7 +19,10 @@ replay because near-ties may legitimately go either way):
   elsewhere both sides' β − b_S at most log(1e-6·max w) + 1e-3; compared
   against the oracle re-run on the GPU's own picks when the index sets differ;
 * reconstructed output softmax(Q C_kᵀ/√d + β) C_v, in float64: relative
-  Frobenius distance to the oracle's at most 2e-3.
+  Frobenius distance to the oracle's at most 2e-3; where some weights are
+  undetermined (previous rule) the output is a different, equally valid
+  compaction, and its fit to the original attention output Y must be within
+  2e-3 of the oracle's fit instead.
 """
 import math
 
@@ -173,9 +176,16 @@ def check_head(g, Q, K, V, t, topk, refit, shift, key_bias=None, oracle_res=None
     O_ref = O.reconstructed_output(Q, o["C_k"], o["beta"], o["C_v"])
     rel = np.linalg.norm(O_gpu - O_ref) / np.linalg.norm(O_ref)
     rep["out_rel"] = float(rel)
-    assert rel <= OUT_TOL, f"{label}: output relative error {rel}"
     rep["fit_err_gpu"] = float(np.linalg.norm(O_gpu - o["Y"]) / np.linalg.norm(o["Y"]))
     rep["fit_err_oracle"] = float(np.linalg.norm(O_ref - o["Y"]) / np.linalg.norm(o["Y"]))
+    if rep.get("beta_undetermined"):
+        # weights the data do not fix: a different, equally valid weighting gives
+        # a different output; it must fit the original attention output as well
+        # as the oracle's does, to the same tolerance
+        assert rep["fit_err_gpu"] <= rep["fit_err_oracle"] + OUT_TOL, \
+            f"{label}: fit {rep['fit_err_gpu']} vs oracle {rep['fit_err_oracle']}"
+    else:
+        assert rel <= OUT_TOL, f"{label}: output relative error {rel}"
     return rep
 
 
@@ -273,7 +283,12 @@ def check_head_prefix(g, Q, K, V, t, topk, refit, shift, key_bias=None, prefix=2
     O_ref = O.reconstructed_output(Q, K[idx], beta_o, C_v)
     O_gpu = O.reconstructed_output(Q, g["C_k"], g["beta"], g["C_v"])
     rep["out_rel"] = float(np.linalg.norm(O_gpu - O_ref) / np.linalg.norm(O_ref))
-    assert rep["out_rel"] <= OUT_TOL, f"{label}: output relative error {rep['out_rel']}"
+    if rep.get("beta_undetermined"):
+        rep["fit_err_gpu"] = float(np.linalg.norm(O_gpu - Y) / np.linalg.norm(Y))
+        rep["fit_err_oracle"] = float(np.linalg.norm(O_ref - Y) / np.linalg.norm(Y))
+        assert rep["fit_err_gpu"] <= rep["fit_err_oracle"] + OUT_TOL, label
+    else:
+        assert rep["out_rel"] <= OUT_TOL, f"{label}: output relative error {rep['out_rel']}"
     return rep
 
 
