@@ -79,7 +79,7 @@ def test_online_round_full_size_with_prior_bias():
     reps = check_heads_parallel([_job("full", out, heads, h, t, 4, 2, shifts[h], kb[h], f"online head {h}")
                                  for h in pick])
     for r in reps:
-        assert r["out_rel"] <= 2e-3 and r["beta_maxdiff"] <= 1e-3
+        assert r["beta_maxdiff"] <= 1e-3   # output (or fit) checked in check_head
 
 
 @needs_cuda
