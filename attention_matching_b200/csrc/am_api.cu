@@ -37,7 +37,8 @@ struct Layout {
   size_t picks, pick_corr, plist, sorted_slot;
   size_t bvec, w, w_eff, ycache;
   size_t G, L, AtA, A, Apl, Ypl, AtY, nrm_part;
-  size_t cnorm, cnpart, rnorm, clist, clj, ccount, inv_m, korder, knorm, ksort, cprefix, cdone, cprobe, cnblk, ctheta, cpassed, rows_eval, gpart, gcount, rcount,
+  size_t cnorm, cnpart, rnorm, clist, clj, ccount, inv_m, gb, ghist, gtau, gcnt, cdone, cnblk, ctheta, rows_eval, gpart, gcount,
+      rcount,
       dinv, vinv;
   size_t total;
   size_t tables_bytes;
@@ -123,17 +124,13 @@ Layout plan(int n, int T, int d, int H, int64_t sum_t, int64_t sum_t2, bool corr
   L.clj = take((size_t)H * T * 4);
   L.ccount = take((size_t)H * 4);
   L.inv_m = take((size_t)H * ldn * 8);
-  L.korder = take((size_t)H * T * 4);
-  L.knorm = take((size_t)H * T * 4);
-  size_t t2 = 1;
-  while (t2 < (size_t)T) t2 <<= 1;
-  L.ksort = take(T > kSortSmemKeys ? (size_t)H * t2 * 8 : 0);
-  L.cprefix = take((size_t)H * 4);
+  L.gb = take((size_t)H * T * 4);
+  L.ghist = take((size_t)H * 1024 * 4);
+  L.gtau = take((size_t)H * 4);
+  L.gcnt = take((size_t)H * 4);
   L.cdone = take((size_t)H * 4);
-  L.cprobe = take((size_t)H * 4);
   L.cnblk = take((size_t)H * T * kRedBlocks * 4);
   L.ctheta = take((size_t)H * 8);
-  L.cpassed = take((size_t)H * 4);
   L.rows_eval = take((size_t)H * 8);
   L.gpart = take((size_t)kGramMaxSlices * ((size_t)sum_t + H) * kGramMaxNew * 8);
   L.gcount = take(((size_t)sum_t + H) * 4);
@@ -301,15 +298,13 @@ Work bind(const Layout& L, char* base, bool corr_bf16) {
   w.clj = reinterpret_cast<int32_t*>(base + L.clj);
   w.ccount = reinterpret_cast<int32_t*>(base + L.ccount);
   w.inv_m = reinterpret_cast<double*>(base + L.inv_m);
-  w.korder = reinterpret_cast<int32_t*>(base + L.korder);
-  w.knorm = reinterpret_cast<float*>(base + L.knorm);
-  w.ksort = reinterpret_cast<uint64_t*>(base + L.ksort);
-  w.cprefix = reinterpret_cast<int32_t*>(base + L.cprefix);
+  w.gb = reinterpret_cast<float*>(base + L.gb);
+  w.ghist = reinterpret_cast<int32_t*>(base + L.ghist);
+  w.gtau = reinterpret_cast<float*>(base + L.gtau);
+  w.gcnt = reinterpret_cast<int32_t*>(base + L.gcnt);
   w.cdone = reinterpret_cast<int32_t*>(base + L.cdone);
-  w.cprobe = reinterpret_cast<int32_t*>(base + L.cprobe);
   w.cnblk = reinterpret_cast<float*>(base + L.cnblk);
   w.ctheta = reinterpret_cast<double*>(base + L.ctheta);
-  w.cpassed = reinterpret_cast<int32_t*>(base + L.cpassed);
   w.rows_eval = reinterpret_cast<unsigned long long*>(base + L.rows_eval);
   w.gpart = reinterpret_cast<double*>(base + L.gpart);
   w.gcount = reinterpret_cast<int32_t*>(base + L.gcount);
@@ -534,8 +529,8 @@ am_status_t run_wave(const Problem& p, Work w, const Tables& tb, int G, int32_t*
   AM_TRY(cudaMemsetAsync(w.rows_eval, 0, (size_t)H * 8, s));
   AM_TRY(cudaMemsetAsync(w.gcount, 0, ((size_t)tb.sum_t + H) * 4, s));
   AM_TRY(cudaMemsetAsync(w.rcount, 0, (size_t)H * 4, s));
-  AM_TRY(cudaMemsetAsync(w.cprefix, 0, (size_t)H * 4, s));
-  AM_TRY(cudaMemsetAsync(w.cpassed, 0, (size_t)H * 4, s));
+  AM_TRY(cudaMemsetAsync(w.ghist, 0, (size_t)H * 1024 * 4, s));
+  AM_TRY(cudaMemsetAsync(w.gcnt, 0, (size_t)H * 4, s));
   AM_TRY(cudaMemsetAsync(w.ccount, 0, (size_t)H * 4, s));
   if (p.select_highest) AM_TRY(launch_select_highest(p, w, s));
   const CorrInputs cin{io.Q, io.K, io.key_bias};

@@ -3,32 +3,34 @@
 // k·R keys per pass under top-k batching with lazy refit, xinfinite.net
 // article §3), evaluated exactly for only the keys that can win.
 //
-// For every key |c_j| = |rᵀΦ_{:,j}| <= ‖r‖₂·‖Φ_{:,j}‖₂ (Cauchy-Schwarz).  The
-// column norms do not depend on r, so once per call the keys are sorted by
-// norm (k_normsum or k_colnorm, then k_sortnorm); in every pass the keys a
-// bound cannot exclude then form a prefix of that order.  One pass of
-// kk = s1 − s0 picks per head is two launches of k_rows:
-//   1. exact c_j for the unselected keys among the first P0 sorted positions,
-//      P0 = max(kProbe + s0, 5/4 of the previous pass's L plus 32) (L grows
-//      slowly from pass to pass, so the probe usually covers it): fp64 sums
-//      of the stored fp32 features times the stored fp32 residual; then the
-//      last block of the head takes θ = the kk-th largest of those values and
-//      the prefix length L: every key with ‖Φ_{:,j}‖ >= θ / (‖r‖(1 + 1e-7))
-//      lies in [0, L) (a sampled search over the sorted norms).  When L <= P0
-//      the kk largest values found are already the picks, and it appends them;
-//   2. otherwise exact c_j for the unselected keys in [P0, L); then the last
-//      block appends the kk largest values of [0, L) (ties to the lower key).
-// A key beyond L has c_j < θ while kk keys in the prefix reach θ, so it is not
-// among the kk largest: the picks are those of a full pass over all keys.
-// The margin 1e-7 covers ‖r‖ being taken from the fp64 residual (the stored
-// fp32 one is larger by at most 2^-24 relative) and the rounding of the fp64
-// sums and norms (relative error below n·2^-53 for the sums, a few ulp for
-// the norms); the fp32 copies of the norms and of the cut only move it
-// outward (rounding to nearest is monotone).  The row blocks append every
-// evaluated key (order key of c_j, key index) to a per-head list; a
-// selection stages that list in shared memory and takes a warp-level top-kk
-// (kk rounds of three warp reductions per warp) followed by the same over the
-// warps' winners.
+// Split the queries into the residual update's groups g (queries i with
+// (i / 128) mod G == g).  For every key, by Cauchy-Schwarz on each group,
+//   |c_j| = |Σ_i r_i Φ_ij| <= Σ_g ‖r_g‖·‖Φ_{g,j}‖ =: b_j.
+// The group norms ‖Φ_{g,j}‖ do not depend on r: they come once per call from
+// the feature pass's partial sums (k_normsum, or k_colnorm from the stored
+// features).  One pass of kk = s1 − s0 picks per head is three launches:
+//   1. k_gbound: b_j for every unselected key (fp64 sum of the group terms,
+//      stored fp32) and a histogram of the bounds; the head's last block sets
+//      τ, the lower edge of the histogram bin at which 2·kk + 32 keys are
+//      reached counting from the top;
+//   2. k_rows (probe): exact c_j (fp64 sums of the stored fp32 features times
+//      the stored fp32 residual) for the keys with b_j >= τ; the head's last
+//      block takes θ = the kk-th largest value; when θ >= τ·(1 + 1e-6) every
+//      key left out has c_j <= b_j < θ, and it appends the kk largest as the
+//      picks (ties to the lower key);
+//   3. k_rows (rest): otherwise exact c_j for the keys with b_j < τ and
+//      b_j·(1 + 1e-6) >= θ; then the kk largest of everything evaluated.
+// A key left out has c_j < θ while kk evaluated keys reach θ, so the picks are
+// those of a full pass over all keys.  The margins cover the rounding of the
+// fp64 sums, the fp32 store of b_j (both below 1e-7 relative), the group
+// norms (raised by 2e-6 over their fp32 partial sums) and ‖r_g‖ being taken
+// from the fp64 residual while the rows are correlated with its fp32 copy
+// (larger by at most 2^-24 relative).  The row blocks append every evaluated
+// key (order key of c_j, key index) to a per-head list; a selection stages
+// that list in shared memory and takes a warp-level top-kk (kk rounds of
+// three warp reductions per warp) followed by the same over the warps'
+// winners.  The global column norms ‖Φ_{:,j}‖ are kept as well (the
+// workspace view reports them).
 #include "am_internal.cuh"
 #include "am_profile.cuh"
 #include "am_linalg.cuh"
@@ -38,10 +40,8 @@
 namespace am {
 namespace {
 
-constexpr int kProbe = 256;        // unselected keys whose exact values set the threshold
 constexpr int kBoundThreads = 1024;
-constexpr int kSelCap = 2304;      // candidates one selection holds (>= kProbe + 2048)
-constexpr double kBoundMargin = 1e-7;
+constexpr int kSelCap = 2304;      // list entries one selection stage holds
 
 // Order-preserving map of a double to uint64 (NaN ranks lowest).
 __device__ __forceinline__ uint64_t order_key(double v) {
@@ -73,9 +73,9 @@ __global__ void __launch_bounds__(256) k_colnorm(Problem p, Work w) {
   const int j = blockIdx.x * 8 + wib;
   const int lane = threadIdx.x & 31;
   if (j >= p.T) return;
-  if (j >= w.Th[h]) {   // no such key in this head: norm 0, sorted last, never evaluated
+  if (j >= w.Th[h]) {   // no such key in this head: norm 0, never evaluated
     if (lane == 0) w.cnorm[(int64_t)h * p.T + j] = 0.0;
-    for (int g = lane; g < kRedBlocks; g += 32) w.cnblk[((int64_t)h * p.T + j) * kRedBlocks + g] = 0.f;
+    for (int g = lane; g < kRedBlocks; g += 32) w.cnblk[((int64_t)h * kRedBlocks + g) * p.T + j] = 0.f;
     return;
   }
   const int G = resid_blocks(p);
@@ -101,7 +101,7 @@ __global__ void __launch_bounds__(256) k_colnorm(Problem p, Work w) {
   __syncwarp();
   if (lane == 0) w.cnorm[(int64_t)h * p.T + j] = sqrt(tot);
   for (int g = lane; g < kRedBlocks; g += 32)
-    w.cnblk[((int64_t)h * p.T + j) * kRedBlocks + g] = g < G ? (float)(sqrt(gsum[wib][g]) * kBlockNormInflate) : 0.f;
+    w.cnblk[((int64_t)h * kRedBlocks + g) * p.T + j] = g < G ? (float)(sqrt(gsum[wib][g]) * kBlockNormInflate) : 0.f;
 }
 
 // ‖Φ_{:,j}‖₂ from the feature pass's per-warp partial sums (fp32 sums of 32
@@ -112,10 +112,10 @@ __global__ void __launch_bounds__(256) k_normsum(Problem p, Work w) {
   const int h = blockIdx.y;
   const int j = blockIdx.x * blockDim.x + threadIdx.x;
   if (j >= p.T) return;
-  float* blk = w.cnblk + ((int64_t)h * p.T + j) * kRedBlocks;
-  if (j >= w.Th[h]) {   // no such key in this head: norm 0, sorted last, never evaluated
+  float* blk = w.cnblk + (int64_t)h * kRedBlocks * p.T + j;   // group g at blk[g·T]
+  if (j >= w.Th[h]) {   // no such key in this head: norm 0, never evaluated
     w.cnorm[(int64_t)h * p.T + j] = 0.0;
-    for (int g = 0; g < kRedBlocks; ++g) blk[g] = 0.f;
+    for (int g = 0; g < kRedBlocks; ++g) blk[(int64_t)g * p.T] = 0.f;
     return;
   }
   const int nqb = (p.n + 127) / 128;
@@ -128,43 +128,9 @@ __global__ void __launch_bounds__(256) k_normsum(Problem p, Work w) {
       for (int qb = g; qb < nqb; qb += G)
         for (int k = 0; k < 4; ++k) sg += (double)src[(int64_t)(qb * 4 + k) * p.T];
     s += sg;
-    blk[g] = g < G ? (float)(sqrt(sg) * kBlockNormInflate) : 0.f;
+    blk[(int64_t)g * p.T] = g < G ? (float)(sqrt(sg) * kBlockNormInflate) : 0.f;
   }
   w.cnorm[(int64_t)h * p.T + j] = sqrt(s) * (1.0 + 1e-6);
-}
-
-// Keys of each head by descending fp32 norm (ties: lower key first): one
-// block per head; 64-bit sort keys (norm bits, inverted key index) in shared
-// memory, or in the workspace when T exceeds kSortSmemKeys.
-__global__ void __launch_bounds__(kBoundThreads) k_sortnorm(Problem p, Work w) {
-  extern __shared__ __align__(16) unsigned char smem[];
-  const int h = blockIdx.x;
-  int n2 = 1;
-  while (n2 < p.T) n2 <<= 1;
-  uint64_t* key = p.T > kSortSmemKeys ? w.ksort + (int64_t)h * n2 : reinterpret_cast<uint64_t*>(smem);
-  const double* cn = w.cnorm + (int64_t)h * p.T;
-  for (int i = threadIdx.x; i < n2; i += blockDim.x)
-    key[i] = i < p.T ? ((uint64_t)__float_as_uint((float)cn[i]) << 32) | (uint32_t)(0xFFFFFFFFu - (uint32_t)i)
-                     : 0ull;
-  __syncthreads();
-  for (int k = 2; k <= n2; k <<= 1) {
-    for (int jj = k >> 1; jj > 0; jj >>= 1) {
-      for (int i = threadIdx.x; i < n2; i += blockDim.x) {
-        const int l = i ^ jj;
-        if (l > i) {
-          const bool desc = (i & k) == 0;
-          const uint64_t a = key[i], b = key[l];
-          if (desc ? a < b : a > b) { key[i] = b; key[l] = a; }
-        }
-      }
-      __syncthreads();
-    }
-  }
-  for (int i = threadIdx.x; i < p.T; i += blockDim.x) {
-    const uint64_t k = key[i];
-    w.korder[(int64_t)h * p.T + i] = (int32_t)(0xFFFFFFFFu - (uint32_t)k);
-    w.knorm[(int64_t)h * p.T + i] = __uint_as_float((uint32_t)(k >> 32));
-  }
 }
 
 // ------------------------------------------------------------ selection --
@@ -271,78 +237,7 @@ __device__ __forceinline__ double key_value(uint64_t k) {
   return __longlong_as_double((long long)((k & 0x8000000000000000ull) ? (k & 0x7fffffffffffffffull) : ~k));
 }
 
-// Number of leading entries of kn[0, n) not below thr, the entries being in
-// descending order: a sampled search, one sample per thread and level (two
-// levels for n up to blockDim², one round trip each).  The first level's
-// sample, kn[min(tid·step0, n − 1)] with step0 = ceil(n / blockDim), does not
-// depend on thr: the caller loads it ahead (first_sample) and passes it in.
-// All threads.
-__device__ __forceinline__ float first_sample(const float* kn, int n) {
-  const int step = (n + (int)blockDim.x - 1) / (int)blockDim.x;
-  return kn[min((int)threadIdx.x * step, n - 1)];
-}
-
-__device__ int prefix_not_below(const float* kn, int n, float thr, float sample0) {
-  int lo = 0, hi = n;   // kn[i] >= thr known for i < lo, kn[i] < thr for i >= hi
-  bool first = true;
-  while (lo < hi) {
-    const int span = hi - lo;
-    const int step = (span + (int)blockDim.x - 1) / (int)blockDim.x;
-    const int samples = (span + step - 1) / step;
-    const int i = lo + (int)threadIdx.x * step;
-    const bool in = (int)threadIdx.x < samples;
-    const bool ok = in && !((first ? sample0 : kn[i]) < thr);
-    first = false;
-    const int c = __syncthreads_count(ok);   // samples 0 .. c-1 pass
-    const int nlo = c > 0 ? lo + (c - 1) * step + 1 : lo;
-    hi = c < samples ? lo + c * step : hi;
-    lo = nlo;
-  }
-  return lo;
-}
-
 __device__ void append_picks(const Problem& p, const Work& w, int h, int s0, int kk, SelScratch& S);
-
-// θ and the prefix L (the last block of a head, after the probe rows); the
-// picks too when the probe already covers L.  ‖r‖² is Σm² before the first
-// refit (r = m) and the residual update's per-block partials after it, added
-// in a fixed order; both are sums of the fp64 residual, whose stored fp32
-// copy (the one correlated) is larger by at most a factor 1 + 2^-24.
-__device__ void theta_and_prefix(const Problem& p, const Work& w, int h, int pass, int s0, int p0, int kk,
-                                 SelScratch& S) {
-  const int nrb = resid_blocks(p);
-  const double rr_mine = pass == 0 ? (threadIdx.x == 0 ? w.mm[h] : 0.0)
-                                   : ((int)threadIdx.x < nrb ? w.rr_part[(int64_t)h * kRedBlocks + threadIdx.x] : 0.0);
-  // every load that does not depend on θ goes out first: the list count, the
-  // list itself up to p0 (entries past the count are left over and ignored),
-  // the first level of the prefix search
-  const int staged = __ldcg(w.ccount + h);   // <= p0 <= kSelCap: the probe's unselected keys
-  const float sample0 = first_sample(w.knorm + (int64_t)h * p.T, p.T);
-  stage_list(p, w, h, 0, p0, 0, S);
-  select_top(S, staged, kk);
-  const double rn = sqrt(block_sum(rr_mine, S.red));
-  const int jt = S.outj[kk - 1];
-  const double theta = jt != INT_MAX ? key_value(S.outk[kk - 1]) : -INFINITY;
-  // L = number of sorted norms not below θ / (‖r‖(1 + margin)); every key when
-  // the bound cannot help (θ <= 0, a zero or non-finite residual)
-  const bool useful = theta > 0.0 && rn > 0.0 && rn < INFINITY;
-  const float thr = useful ? (float)(theta / (rn * (1.0 + kBoundMargin))) : 0.f;
-  const int L = useful ? prefix_not_below(w.knorm + (int64_t)h * p.T, p.T, thr, sample0) : p.T;
-  const bool done = L <= p0;
-  if (threadIdx.x == 0) {
-    w.cprefix[h] = L;
-    w.cprobe[h] = p0;
-    w.cdone[h] = done;
-    w.rnorm[h] = rn;
-    w.ctheta[h] = theta;   // the second launch skips keys whose group bound is below it
-    if (done) {
-      w.rows_eval[h] += (unsigned long long)staged;
-      w.cpassed[h] = staged;   // the next pass sizes its probe by it
-      w.ccount[h] = 0;   // the list is consumed; otherwise the second launch extends it
-    }
-  }
-  if (done) append_picks(p, w, h, s0, kk, S);
-}
 
 // Appends S.outj[0, kk) as this pass's picks, one thread each; a slot with no
 // finite value takes the lowest free key instead (thread 0, after the
@@ -377,13 +272,17 @@ __device__ void append_picks(const Problem& p, const Work& w, int h, int s0, int
   }
 }
 
-// The kk largest values in the head's list of evaluated keys (the unselected
-// keys of [0, L)), in chunks that carry the best kk of what came before (the
-// last block of a head, after the remaining rows).
-__device__ void pick_from_prefix(const Problem& p, const Work& w, int h, int s0, int kk, SelScratch& S) {
+// The kk largest values in the head's list of evaluated keys into
+// S.outk / S.outj (index INT_MAX when fewer), in chunks that carry the best kk
+// of what came before; returns the list length.  All threads.
+__device__ int top_of_list(const Problem& p, const Work& w, int h, int kk, SelScratch& S) {
   const int n = __ldcg(w.ccount + h);
   const int chunk = kSelCap - kMaxPicksPerPass;
   int kept = 0;
+  if (n == 0) {
+    if (threadIdx.x < kk) { S.outk[threadIdx.x] = 0ull; S.outj[threadIdx.x] = INT_MAX; }
+    __syncthreads();
+  }
   for (int c = 0; c < n; c += chunk) {
     if (threadIdx.x < kept) {   // winners so far lead the next chunk
       S.key[threadIdx.x] = S.outk[threadIdx.x];
@@ -395,29 +294,121 @@ __device__ void pick_from_prefix(const Problem& p, const Work& w, int h, int s0,
     kept = 0;
     for (int k = 0; k < kk; ++k) kept += S.outj[k] != INT_MAX;
   }
+  return n;
+}
+
+// The picks from everything evaluated this pass (the last block of a head).
+__device__ void pick_from_list(const Problem& p, const Work& w, int h, int s0, int kk, SelScratch& S) {
+  const int n = top_of_list(p, w, h, kk, S);
   if (threadIdx.x == 0) {
     w.rows_eval[h] += (unsigned long long)n;
-    w.cpassed[h] = n;   // the next pass sizes its probe by it
     w.ccount[h] = 0;
   }
   append_picks(p, w, h, s0, kk, S);
 }
 
+// ------------------------------------------------------------ group bound --
+constexpr int kHistBins = 1024;   // bins of positive fp32 bounds: exponent and two mantissa bits
+constexpr int kProbeExtra = 32;   // the probe aims at 2·kk + 32 keys
+constexpr double kBoundMargin = 1.0 + 1e-6;
+
+__device__ __forceinline__ int bound_bin(float b) { return (int)(__float_as_uint(b) >> 21); }   // b > 0
+__device__ __forceinline__ float bin_floor(int bin) { return __uint_as_float((uint32_t)bin << 21); }
+
+// b_j for every key of the head (−1 for a selected key or one past T_h), and
+// the histogram of the positive ones; the head's last block turns the
+// histogram into τ and clears it for the next pass.
+__global__ void __launch_bounds__(256) k_gbound(Problem p, Work w, int pass) {
+  chain_wait();
+  __shared__ double rg[kRedBlocks];
+  __shared__ int hist[kHistBins];
+  __shared__ int s_last;
+  __shared__ int csum[32];
+  const int h = w.order[blockIdx.y];
+  int s0, s1;
+  pass_range(p, w.t[h], pass, s0, s1);
+  if (s0 >= s1) return;
+  const int kk = s1 - s0;
+  const int G = resid_blocks(p);
+  for (int g = threadIdx.x; g < kRedBlocks; g += blockDim.x)
+    rg[g] = g < G ? sqrt(w.rr_part[(int64_t)h * kRedBlocks + g]) : 0.0;
+  for (int i = threadIdx.x; i < kHistBins; i += blockDim.x) hist[i] = 0;
+  __syncthreads();
+  const int j = blockIdx.x * blockDim.x + threadIdx.x;
+  if (j < p.T) {
+    float b = -1.f;
+    if (!w.sel[(int64_t)h * p.T + j]) {
+      const float* cb = w.cnblk + (int64_t)h * kRedBlocks * p.T + j;
+      double acc = 0.0;
+      for (int g = 0; g < G; ++g) acc = fma(rg[g], (double)__ldg(cb + (int64_t)g * p.T), acc);
+      b = (float)acc;
+      if (b > 0.f) atomicAdd(&hist[bound_bin(b)], 1);
+    }
+    w.gb[(int64_t)h * p.T + j] = b;
+  }
+  __syncthreads();
+  for (int i = threadIdx.x; i < kHistBins; i += blockDim.x)
+    if (hist[i]) atomicAdd(w.ghist + (int64_t)h * kHistBins + i, hist[i]);
+  chain_release();
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0) s_last = atomicAdd(w.gcnt + h, 1) == (int)gridDim.x - 1;
+  __syncthreads();
+  if (!s_last) return;
+  __threadfence();
+  // τ: counting bins from the top, the first at which 2·kk + 32 keys are reached
+  int* gh = w.ghist + (int64_t)h * kHistBins;
+  for (int i = threadIdx.x; i < kHistBins; i += blockDim.x) {
+    hist[i] = __ldcg(gh + i);
+    gh[i] = 0;   // ready for the next pass
+  }
+  __syncthreads();
+  if (threadIdx.x < 32) {
+    const int lane = threadIdx.x;
+    const int top = kHistBins - 1 - 32 * lane;   // this lane's bins: top .. top − 31
+    int sum = 0;
+    for (int k = 0; k < 32; ++k) sum += hist[top - k];
+    int incl = sum;
+    for (int o = 1; o < 32; o <<= 1) {
+      const int v = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += v;
+    }
+    csum[lane] = incl;
+    __syncwarp();
+    const int target = 2 * kk + kProbeExtra;
+    const unsigned reach = __ballot_sync(0xffffffffu, incl >= target);
+    float tau = 0.f;   // fewer keys than the target: the probe takes every unselected key
+    if (reach) {
+      const int l = __ffs(reach) - 1;
+      if (lane == l) {
+        int cum = l > 0 ? csum[l - 1] : 0;
+        int bin = top;
+        for (int k = 0; k < 32; ++k) {
+          cum += hist[top - k];
+          if (cum >= target) { bin = top - k; break; }
+        }
+        w.gtau[h] = bin_floor(bin);
+      }
+    } else if (lane == 0) {
+      w.gtau[h] = tau;
+    }
+    if (lane == 0) w.gcnt[h] = 0;
+  }
+}
+
 // ------------------------------------------------------------ exact rows --
-// c_j = Σ_i r_i Φ_ij for the unselected keys at sorted positions [0, P0)
-// (which = 0) or [P0, L) (which = 1), in fp64 sums of exact fp32 products.
-// In the second launch a key is first tested against the group bound
-// Σ_g ‖r_g‖·‖Φ_{g,j}‖ (1 + 1e-6): below θ it cannot reach the picks and its
-// row is not read.  ‖r_g‖ comes from the fp64 residual's per-group sums
-// (k_init before the first refit, k_resid after); the fp32 copy the rows
-// are correlated with is larger by at most 2^-24 relative, inside the margin.
-// Four warps share a key, each summing a quarter of the queries with eight
-// columns per lane in flight; the quarters are added in a fixed order.  The
-// last block of a head to finish (counted with an atomic) then takes the
-// selection step: θ and L after the probe rows, the picks after the rest.
+// c_j = Σ_i r_i Φ_ij in fp64 sums of exact fp32 products for the keys the
+// launch takes: b_j >= τ (which = 0, the probe) or b_j < τ with
+// b_j·(1 + 1e-6) >= θ (which = 1, the rest).  Each CTA scans a slice of the
+// head's keys in chunks, gathers the keys it takes in shared memory, and
+// evaluates them two at a time: four warps share a key, each summing a
+// quarter of the queries with eight columns per lane in flight; the quarters
+// are added in a fixed order.  The last block of a head to finish (counted
+// with an atomic) then takes the selection step.
 constexpr int kRowSplit = 4;                           // warps per key
 constexpr int kRowsPerBlock = kSelThreads / 32 / kRowSplit;   // keys per block
 constexpr int kRowLoads = 8;                           // float4 columns per lane in flight
+constexpr int kScanChunk = 2048;                       // keys scanned per chunk of a CTA's slice
 
 __global__ void __launch_bounds__(kSelThreads) k_rows(Problem p, Work w, int pass, int which) {
   chain_wait();
@@ -425,78 +416,73 @@ __global__ void __launch_bounds__(kSelThreads) k_rows(Problem p, Work w, int pas
   SelScratch& S = *reinterpret_cast<SelScratch*>(smem);
   __shared__ double part[kRowsPerBlock][kRowSplit];
   __shared__ int s_last;
+  __shared__ int cand[kScanChunk];
+  __shared__ int ncand;
   const int h = w.order[blockIdx.y];
   int s0, s1;
   pass_range(p, w.t[h], pass, s0, s1);
   if (s0 >= s1) return;
   const int kk = s1 - s0;
   if (which && w.cdone[h]) return;                     // the probe step made the picks
-  // the probe: the first kProbe + s0 positions of the norm order (s0 keys are
-  // already selected), at most kSelCap; the rest of the prefix is filtered
-  // by the group bound in the second launch
-  const int p0 = which ? w.cprobe[h] : min(min(p.T, kSelCap), kProbe + s0);
-  const int lo = which ? p0 : 0;
-  const int hi = which ? w.cprefix[h] : p0;
+  const float tau = w.gtau[h];
+  const double theta = which ? w.ctheta[h] : 0.0;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int slot = warp / kRowSplit, quarter = warp % kRowSplit;
-  const int32_t* ord = w.korder + (int64_t)h * p.T;
   const uint8_t* sel = w.sel + (int64_t)h * p.T;
+  const float* gb = w.gb + (int64_t)h * p.T;
   const float4* r4 = reinterpret_cast<const float4*>(w.r + (int64_t)h * p.ldn);
   const int n4 = p.ldn >> 2;
   const int per = (n4 + kRowSplit - 1) / kRowSplit;
   const int c0 = quarter * per, c1 = min(n4, c0 + per);
-  // the second launch's key filter: ‖r_g‖ per group, and θ
-  __shared__ double rg[kRedBlocks];
-  const bool filter = which && w.cnblk != nullptr;
-  const int G = resid_blocks(p);
-  double theta = 0.0;
-  if (filter) {
-    for (int g = threadIdx.x; g < kRedBlocks; g += blockDim.x)
-      rg[g] = g < G ? sqrt(w.rr_part[(int64_t)h * kRedBlocks + g]) : 0.0;
-    theta = w.ctheta[h];
+  const int slice = (p.T + gridDim.x - 1) / gridDim.x;
+  const int j_lo = blockIdx.x * slice, j_hi = min(p.T, j_lo + slice);
+  for (int k0 = j_lo; k0 < j_hi; k0 += kScanChunk) {
+    const int k1 = min(j_hi, k0 + kScanChunk);
+    if (threadIdx.x == 0) ncand = 0;
     __syncthreads();
-  }
-  for (int q0 = lo + blockIdx.x * kRowsPerBlock; q0 < hi; q0 += gridDim.x * kRowsPerBlock) {
-    const int q = q0 + slot;
-    const int j = q < hi ? ord[q] : 0;
-    bool on = q < hi && !sel[j];
-    if (filter && on) {
-      // every warp of the key forms the same bound (same order of operations)
-      const float* bj = w.cnblk + ((int64_t)h * p.T + j) * kRedBlocks;
-      double b = (double)bj[lane] * rg[lane] + (double)bj[lane + 32] * rg[lane + 32];
-      b = warp_sum(b) * (1.0 + 1e-6);
-      on = !(b < theta);
+    for (int j = k0 + threadIdx.x; j < k1; j += blockDim.x) {
+      const float b = gb[j];
+      bool take = false;
+      if (!sel[j]) take = which == 0 ? b >= tau : (b < tau && (double)b * kBoundMargin >= theta);
+      if (take) cand[atomicAdd(&ncand, 1)] = j;
     }
-    double a[4] = {0.0, 0.0, 0.0, 0.0};
-    if (on) {
-      const float4* row = reinterpret_cast<const float4*>(w.phiT + ((int64_t)h * p.T + j) * p.ldn);
-      for (int i0 = c0 + lane; i0 < c1; i0 += 32 * kRowLoads) {
-        float4 x[kRowLoads], y[kRowLoads];
+    __syncthreads();
+    const int nc = ncand;
+    for (int q0 = 0; q0 < nc; q0 += kRowsPerBlock) {
+      const int q = q0 + slot;
+      const bool on = q < nc;
+      const int j = on ? cand[q] : 0;
+      double a[4] = {0.0, 0.0, 0.0, 0.0};
+      if (on) {
+        const float4* row = reinterpret_cast<const float4*>(w.phiT + ((int64_t)h * p.T + j) * p.ldn);
+        for (int i0 = c0 + lane; i0 < c1; i0 += 32 * kRowLoads) {
+          float4 x[kRowLoads], y[kRowLoads];
 #pragma unroll
-        for (int u = 0; u < kRowLoads; ++u) {
-          const int i = i0 + 32 * u;
-          x[u] = i < c1 ? __ldcs(row + i) : make_float4(0.f, 0.f, 0.f, 0.f);
-          y[u] = i < c1 ? __ldg(r4 + i) : make_float4(0.f, 0.f, 0.f, 0.f);
-        }
+          for (int u = 0; u < kRowLoads; ++u) {
+            const int i = i0 + 32 * u;
+            x[u] = i < c1 ? __ldcs(row + i) : make_float4(0.f, 0.f, 0.f, 0.f);
+            y[u] = i < c1 ? __ldg(r4 + i) : make_float4(0.f, 0.f, 0.f, 0.f);
+          }
 #pragma unroll
-        for (int u = 0; u < kRowLoads; ++u) {
-          a[0] = fma((double)x[u].x, (double)y[u].x, a[0]);
-          a[1] = fma((double)x[u].y, (double)y[u].y, a[1]);
-          a[2] = fma((double)x[u].z, (double)y[u].z, a[2]);
-          a[3] = fma((double)x[u].w, (double)y[u].w, a[3]);
+          for (int u = 0; u < kRowLoads; ++u) {
+            a[0] = fma((double)x[u].x, (double)y[u].x, a[0]);
+            a[1] = fma((double)x[u].y, (double)y[u].y, a[1]);
+            a[2] = fma((double)x[u].z, (double)y[u].z, a[2]);
+            a[3] = fma((double)x[u].w, (double)y[u].w, a[3]);
+          }
         }
       }
+      const double c = warp_sum((a[0] + a[1]) + (a[2] + a[3]));
+      if (lane == 0) part[slot][quarter] = c;
+      __syncthreads();
+      if (on && quarter == 0 && lane == 0) {   // onto the head's list of evaluated keys
+        const double cj = (part[slot][0] + part[slot][1]) + (part[slot][2] + part[slot][3]);
+        const int at = atomicAdd(w.ccount + h, 1);
+        w.clist[(int64_t)h * p.T + at] = order_key(cj);
+        w.clj[(int64_t)h * p.T + at] = j;
+      }
+      __syncthreads();
     }
-    const double c = warp_sum((a[0] + a[1]) + (a[2] + a[3]));
-    if (lane == 0) part[slot][quarter] = c;
-    __syncthreads();
-    if (on && quarter == 0 && lane == 0) {   // onto the head's list of evaluated keys
-      const double cj = (part[slot][0] + part[slot][1]) + (part[slot][2] + part[slot][3]);
-      const int at = atomicAdd(w.ccount + h, 1);
-      w.clist[(int64_t)h * p.T + at] = order_key(cj);
-      w.clj[(int64_t)h * p.T + at] = j;
-    }
-    __syncthreads();
   }
   chain_release();
   // the last block of this head to get here takes the selection step
@@ -506,8 +492,24 @@ __global__ void __launch_bounds__(kSelThreads) k_rows(Problem p, Work w, int pas
   __syncthreads();
   if (!s_last) return;
   __threadfence();
-  if (which == 0) theta_and_prefix(p, w, h, pass, s0, p0, kk, S);
-  else pick_from_prefix(p, w, h, s0, kk, S);
+  if (which == 0) {
+    // θ from the probe; done when every key left out is below it
+    const int n = top_of_list(p, w, h, kk, S);
+    const int jt = S.outj[kk - 1];
+    const double th = jt != INT_MAX ? key_value(S.outk[kk - 1]) : -INFINITY;
+    const bool done = !(tau > 0.f) || (jt != INT_MAX && th >= (double)tau * kBoundMargin);
+    if (threadIdx.x == 0) {
+      w.cdone[h] = done;
+      w.ctheta[h] = th;
+      if (done) {
+        w.rows_eval[h] += (unsigned long long)n;
+        w.ccount[h] = 0;   // the list is consumed; otherwise the second launch extends it
+      }
+    }
+    if (done) append_picks(p, w, h, s0, kk, S);
+  } else {
+    pick_from_list(p, w, h, s0, kk, S);
+  }
   if (threadIdx.x == 0) w.rcount[h] = 0;
 }
 
@@ -637,13 +639,12 @@ cudaError_t launch_column_norms(const Problem& p, const Work& w, cudaStream_t s)
     dim3 g((p.T + 7) / 8, p.H);
     AM_LAUNCH(AM_STAGE_NORMS, s, k_colnorm<<<g, 256, 0, s>>>(p, w));
   }
-  const int sort_smem = p.T > kSortSmemKeys ? 0 : (int)(sizeof(uint64_t) * kSortSmemKeys);
-  cudaFuncSetAttribute(k_sortnorm, cudaFuncAttributeMaxDynamicSharedMemorySize, sort_smem);
-  AM_LAUNCH(AM_STAGE_NORMS, s, k_sortnorm<<<p.H, kBoundThreads, sort_smem, s>>>(p, w));
   return cudaGetLastError();
 }
 
 cudaError_t launch_corr_bounded(const Problem& p, const Work& w, int pass, int active, cudaStream_t s) {
+  dim3 gb((p.T + 255) / 256, active);
+  AM_LAUNCH(AM_STAGE_ROWS, s, launch_chained(k_gbound, gb, dim3(256), 0, s, p, w, pass));
   const int sel_smem = (int)sizeof(SelScratch);
   cudaFuncSetAttribute(k_rows, cudaFuncAttributeMaxDynamicSharedMemorySize, sel_smem);
   dim3 gr(rows_ctas_per_head(active), active);

@@ -84,16 +84,14 @@ struct Work {
   uint64_t* clist;      // [H][T] this pass's evaluated keys: order keys of their exact c_j
   int32_t* clj;         // [H][T] and the key indices, in completion order
   int32_t* ccount;      // [H] entries in that list
-  int32_t* korder;      // [H][T] keys by descending column norm
-  float* knorm;         // [H][T] those norms (fp32, descending)
-  uint64_t* ksort;      // [H][pow2 >= T] sort scratch when T exceeds the shared-memory sort
-  int32_t* cprefix;     // [H] this pass evaluates the keys at sorted positions [0, cprefix)
+  float* gb;            // [H][T] this pass's group bound b_j of every key (−1: selected or past T_h)
+  int32_t* ghist;       // [H][1024] histogram of the positive bounds (cleared after each use)
+  float* gtau;          // [H] this pass's probe threshold τ
+  int32_t* gcnt;        // [H] group-bound blocks finished this pass
   int32_t* cdone;       // [H] 1 when the probe step already made this pass's picks
-  int32_t* cprobe;      // [H] the probe length P0 of this pass
-  float* cnblk;         // [H][T][kRedBlocks] per residual query group g, an upper bound of ‖Φ_{i∈g, j}‖₂
-                        // (group g: queries i with (i / 128) mod resid_blocks == g), or null
+  float* cnblk;         // [H][64][T] per residual query group g, an upper bound of ‖Φ_{i∈g, j}‖₂
+                        // (group g: queries i with (i / 128) mod resid_blocks == g)
   double* ctheta;       // [H] this pass's threshold θ, the kk-th largest value the probe found
-  int32_t* cpassed;     // [H] keys whose correlation the last pass evaluated (sizes the next probe)
   unsigned long long* rows_eval;   // [H] keys evaluated, summed over the passes
   double* gpart;        // [kGramMaxSlices·(Σt + H)·kR] Gram partial sums per query slice
   int32_t* gcount;      // [Σt + H] Gram blocks finished this pass, per head and row group
@@ -113,7 +111,7 @@ inline __host__ __device__ int resid_blocks(const Problem& p) {
   const int b = (p.ldn / 4 + kResidPos - 1) / kResidPos;
   return b < kRedBlocks ? b : kRedBlocks;
 }
-constexpr int kSortSmemKeys = 16384;  // key counts the norm sort handles in shared memory
+constexpr int kSortSmemKeys = 16384;  // key counts the highest-attention sort handles in shared memory
 constexpr int kGramMaxSlices = 32;    // query slices of the tiled Gram update
 constexpr int kGramMaxNew = 16;       // picks per pass the tiled Gram update takes
 constexpr int kNormalMaxSplits = 8;   // query splits of the normal-equation products

@@ -336,10 +336,15 @@ def stage_models(wl, n, key_counts, d, ldn, corr_kind, rows_evaluated, tc=True):
         m["corr"] = {"bound": "tensor", "flops": 2.0 * work * n * d, "exps": work * n}
     elif corr_kind == "bounded":
         parts = 4 * ((n + 127) // 128)
-        # partials in, fp64 norms out and back in for the sort, sorted order and norms out
+        G = min((ldn // 4 + 31) // 32, 64)
+        # partials in (or the stored features on the CUDA-core path), fp64 norms and the
+        # per-group fp32 norms out
         norms_in = parts * 4 if tc else row
-        m["norms"] = {"bound": "hbm", "bytes": sT * (norms_in + 8 + 8 + 4 + 8)}
-        m["rows"] = {"bound": "hbm", "bytes": float(rows_evaluated) * row}
+        m["norms"] = {"bound": "hbm", "bytes": sT * (norms_in + 8 + 64 * 4)}
+        # per pass and head: every key's group norms read and its bound written, then the
+        # evaluated rows of the stored features
+        heads_passes = float(sum(((t + kR - 1) // kR) * T for t, T in zip(wl.budgets, key_counts)))
+        m["rows"] = {"bound": "hbm", "bytes": float(rows_evaluated) * row + heads_passes * (G * 4 + 4 + 4)}
     else:
         passes = [(t + kR - 1) // kR for t in wl.budgets]
         b = 2 if corr_kind == "bf16" else 4
