@@ -652,6 +652,241 @@ __device__ void block_backward(const double* L, const double* invd, double* v, i
   }
 }
 
+// ---------------------------------------------- streamed factor solves ----
+// For a head whose factor lives in the workspace, a triangular solve reads
+// the whole factor once, in order.  The reads go through a ring of kRing
+// shared-memory stages filled by asynchronous 8-byte copies issued kRing − 1
+// pieces ahead, so the copies of later rows are in flight while a diagonal
+// block is swept.  A piece is up to 32 factor rows × 64 columns (row stride
+// 65: a warp reading down a column meets distinct banks); a row block's
+// pieces are its off-diagonal column chunks and its diagonal block.
+constexpr int kRing = 4;
+constexpr int kPieceCols = 64;
+constexpr int kPieceLd = kPieceCols + 1;
+constexpr int kStageDoubles = kSB * kPieceLd;
+constexpr size_t kRingBytes = (size_t)kRing * kStageDoubles * sizeof(double);
+constexpr int kStreamRhs = 8;    // vectors one streamed forward solve carries
+constexpr int kAppendRows = 32;  // most new rows the append keeps in shared memory
+
+struct Piece {
+  int r0, bw, c0, cw;
+  bool diag;
+};
+
+// Copies piece pc of the packed factor L into a stage (the diagonal block's
+// lower triangle only) and commits the copies as one group.
+__device__ __forceinline__ void issue_piece(const double* L, double* stage, const Piece& pc) {
+#pragma unroll
+  for (int u = 0; u < kSB * kPieceCols / kNnlsThreads; ++u) {
+    const int e = threadIdx.x + u * kNnlsThreads, r = e / kPieceCols, c = e % kPieceCols;
+    if (r < pc.bw && c < pc.cw && (!pc.diag || c <= r))
+      cp_async8(stage + r * kPieceLd + c, L + tri(pc.r0 + r, pc.c0 + c));
+  }
+  cp_async_commit();
+}
+
+__device__ __forceinline__ int off_chunks(int r0) { return (r0 + kPieceCols - 1) / kPieceCols; }
+
+// Forward order over rows [k0, n): row blocks top down, each its column
+// chunks of [0, r0) then its diagonal block.
+struct ForwardPieces {
+  int r0, c, n;
+  __device__ bool done() const { return r0 >= n; }
+  __device__ Piece piece() const {
+    Piece d;
+    d.r0 = r0;
+    d.bw = min(kSB, n - r0);
+    d.diag = c == off_chunks(r0);
+    d.c0 = d.diag ? r0 : c * kPieceCols;
+    d.cw = d.diag ? d.bw : min(kPieceCols, r0 - d.c0);
+    return d;
+  }
+  __device__ void next() {
+    if (++c > off_chunks(r0)) { c = 0; r0 += kSB; }
+  }
+};
+
+// Backward order over rows [0, n): row blocks bottom up (at multiples of 32),
+// each its diagonal block then its column chunks of [0, r0).
+struct BackwardPieces {
+  int r0, c, n;
+  __device__ bool done() const { return r0 < 0; }
+  __device__ Piece piece() const {
+    Piece d;
+    d.r0 = r0;
+    d.bw = min(kSB, n - r0);
+    d.diag = c == 0;
+    d.c0 = d.diag ? r0 : (c - 1) * kPieceCols;
+    d.cw = d.diag ? d.bw : min(kPieceCols, r0 - d.c0);
+    return d;
+  }
+  __device__ void next() {
+    if (++c > off_chunks(r0)) { c = 0; r0 -= kSB; }
+  }
+};
+
+// Runs consume(piece, stage) over the pieces of `it` in order, with the
+// stages kRing − 1 pieces ahead in flight.  Every thread of the block calls
+// it; consume may synchronise the block.  Ends with the block synchronised.
+template <class Pieces, class Consume>
+__device__ __forceinline__ void stream_pieces(const double* L, double* ring, Pieces it, Consume&& consume) {
+  Pieces ahead = it;
+#pragma unroll
+  for (int s = 0; s < kRing - 1; ++s) {
+    if (!ahead.done()) {
+      issue_piece(L, ring + s * kStageDoubles, ahead.piece());
+      ahead.next();
+    } else {
+      cp_async_commit();
+    }
+  }
+  for (int p = 0; !it.done(); ++p) {
+    cp_async_wait<kRing - 2>();
+    __syncthreads();   // piece p is in; the stage of piece p − 1 is free
+    if (!ahead.done()) {
+      issue_piece(L, ring + ((p + kRing - 1) % kRing) * kStageDoubles, ahead.piece());
+      ahead.next();
+    } else {
+      cp_async_commit();
+    }
+    consume(it.piece(), static_cast<const double*>(ring + (p % kRing) * kStageDoubles));
+    it.next();
+  }
+  cp_async_wait<0>();
+  __syncthreads();
+}
+
+// u_e ← L⁻¹ u_e on rows [k0, n) for the R <= RMAX vectors u_e = U0 + e·ldu
+// (shared memory); entries below k0 are already final.  Products: warp w
+// takes rows 4w .. 4w+3 of the row block, its lanes run across the piece's
+// columns; the sums close at the diagonal block, whose sweep runs one warp
+// per vector.
+template <int RMAX>
+__device__ void stream_forward(const double* L, const double* invd, double* U0, int ldu, int R, int k0, int n,
+                               double* ring) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, rl = 4 * warp;
+  double acc[4][RMAX];
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int e = 0; e < RMAX; ++e) acc[i][e] = 0.0;
+  stream_pieces(L, ring, ForwardPieces{k0, 0, n}, [&](const Piece& pc, const double* S) {
+    if (!pc.diag) {
+      if (rl < pc.bw) {
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+          const int j = lane + 32 * half;
+          if (j < pc.cw) {
+            double u[RMAX];
+#pragma unroll
+            for (int e = 0; e < RMAX; ++e) u[e] = e < R ? U0[e * ldu + pc.c0 + j] : 0.0;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              const double l = rl + i < pc.bw ? S[(rl + i) * kPieceLd + j] : 0.0;
+#pragma unroll
+              for (int e = 0; e < RMAX; ++e) acc[i][e] = fma(l, u[e], acc[i][e]);
+            }
+          }
+        }
+      }
+      return;
+    }
+    if (pc.r0 > 0 && rl < pc.bw) {
+      if constexpr (RMAX == 1) {
+        double flat[4] = {acc[0][0], acc[1][0], acc[2][0], acc[3][0]};
+        const double sum = warp_reduce_n<4>(flat);   // lane l: row rl + l mod 4
+        if (lane < 4 && rl + lane < pc.bw) U0[pc.r0 + rl + lane] -= sum;
+      } else {
+        static_assert(RMAX == 8, "four rows × eight vectors fill the 32 lanes");
+        double flat[32];   // value i·8 + e: row rl + i, vector e
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+#pragma unroll
+          for (int e = 0; e < 8; ++e) flat[i * 8 + e] = acc[i][e];
+        const double sum = warp_reduce32(flat);
+        const int li = lane / 8, le = lane % 8;
+        if (le < R && rl + li < pc.bw) U0[le * ldu + pc.r0 + rl + li] -= sum;
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int e = 0; e < RMAX; ++e) acc[i][e] = 0.0;
+    __syncthreads();
+    if (warp < R) {
+      double* u = U0 + warp * ldu;
+      double v = lane < pc.bw ? u[pc.r0 + lane] : 0.0;
+      for (int c = 0; c < pc.bw; ++c) {
+        if (lane == c) v *= invd[pc.r0 + c];
+        const double vc = __shfl_sync(0xffffffffu, v, c);
+        if (lane > c && lane < pc.bw) v -= S[lane * kPieceLd + c] * vc;
+      }
+      if (lane < pc.bw) u[pc.r0 + lane] = v;
+    }
+  });
+}
+
+// v ← L⁻ᵀ v on rows [0, n), v in shared memory.  Per row block from the
+// bottom: warp 0 sweeps the diagonal block, then each column chunk takes the
+// block's contribution, warp w on columns 8w .. 8w+7 with the four lane
+// quarters on eight factor rows each (summed by two shuffles).
+__device__ void stream_backward(const double* L, const double* invd, double* v, int n, double* ring) {
+  if (n <= 0) return;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  stream_pieces(L, ring, BackwardPieces{((n - 1) / kSB) * kSB, 0, n}, [&](const Piece& pc, const double* S) {
+    if (pc.diag) {
+      if (warp == 0) {
+        double x = lane < pc.bw ? v[pc.r0 + lane] : 0.0;
+        for (int c = pc.bw - 1; c >= 0; --c) {
+          if (lane == c) x *= invd[pc.r0 + c];
+          const double xc = __shfl_sync(0xffffffffu, x, c);
+          if (lane < c) x -= S[c * kPieceLd + lane] * xc;
+        }
+        if (lane < pc.bw) v[pc.r0 + lane] = x;
+      }
+      return;
+    }
+    const int j = 8 * warp + (lane & 7), q = lane >> 3;
+    double s = 0.0;
+    if (j < pc.cw) {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const int r = 8 * q + i;
+        if (r < pc.bw) s = fma(S[r * kPieceLd + j], v[pc.r0 + r], s);
+      }
+    }
+    s += __shfl_xor_sync(0xffffffffu, s, 8);
+    s += __shfl_xor_sync(0xffffffffu, s, 16);
+    if (q == 0 && j < pc.cw) v[pc.c0 + j] -= s;
+  });
+}
+
+// Us[e·ldu + q] = G[add_e, P_q] for e < R, q < np (all loads of a thread
+// issued before its stores, eight at a time).
+__device__ __forceinline__ void gather_new_rows(double* Us, int ldu, const double* G, int t, const int* addl, int R,
+                                                const int* P, int np) {
+  const int total = R * np;
+  for (int i0 = threadIdx.x; i0 < total; i0 += 8 * blockDim.x) {
+    double v[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int i = i0 + u * blockDim.x;
+      if (i < total) {
+        const int e = i / np, q = i - e * np;
+        v[u] = G[(int64_t)addl[e] * t + P[q]];
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int i = i0 + u * blockDim.x;
+      if (i < total) {
+        const int e = i / np, q = i - e * np;
+        Us[e * ldu + q] = v[u];
+      }
+    }
+  }
+}
+
 // Deletes position q from the packed factor L of an np×np matrix (all
 // threads of the block).  Writing L = [L11 · ·; l21ᵀ l22 ·; L31 l32 L33],
 // the matrix without row and column q has the factor [L11 ·; L31 L̃33] with
@@ -755,7 +990,11 @@ __device__ void factor_remove(double* L, double* invd, double* xv, double* rot, 
   __syncthreads();
 }
 
-__global__ void __launch_bounds__(kNnlsThreads) k_nnls(Problem p, Work w, int pass, int l_in_smem_max) {
+// l_in_smem_max: heads with t at or below it keep the factor in shared
+// memory.  ucap > 0: the others stream their solves (ring and up to ucap new
+// rows of t doubles in shared memory after the vectors); 0: they read the
+// factor in place.
+__global__ void __launch_bounds__(kNnlsThreads) k_nnls(Problem p, Work w, int pass, int l_in_smem_max, int ucap) {
   chain_wait();
   extern __shared__ __align__(16) unsigned char smem[];
   const int h = w.order[blockIdx.x];
@@ -787,6 +1026,9 @@ __global__ void __launch_bounds__(kNnlsThreads) k_nnls(Problem p, Work w, int pa
   const bool l_smem = t <= l_in_smem_max;
   double* Lg = w.L + gbase;
   double* L = l_smem ? reinterpret_cast<double*>(smem + nnls_vec_bytes(t)) : Lg;
+  const bool streamed = !l_smem && ucap > 0;
+  double* ring = reinterpret_cast<double*>(smem + nnls_vec_bytes(t));   // streamed heads only
+  double* Us = ring + kRing * kStageDoubles;                              // ucap rows of t
   // the factor kept in shared memory arrives by one bulk copy (16-byte
   // aligned at both ends; rounding the size up reads at most one double past
   // the factor, still inside the head's t×t region and the shared buffer)
@@ -917,6 +1159,140 @@ __global__ void __launch_bounds__(kNnlsThreads) k_nnls(Problem p, Work w, int pa
     }
   };
 
+  // Streamed heads: the same block append with the forward solves of the new
+  // rows streamed (kStreamRhs vectors per read of the factor), and, for at
+  // most ucap new rows, the rows, their Schur block and its Cholesky in
+  // shared memory until the block is accepted.
+  auto append_streamed = [&]() {
+    for (;;) {
+      const int np = ctl[0], k = ctl[1];
+      if (k == 0) return;
+      const bool one = k <= ucap;
+      const int chunk = one ? k : ucap;
+      for (int e0 = 0; e0 < k; e0 += chunk) {
+        const int rows = min(chunk, k - e0);
+        gather_new_rows(Us, t, G, t, add + e0, rows, P, np);
+        for (int c0 = 0; c0 < rows; c0 += kStreamRhs) {
+          const int R = min(kStreamRhs, rows - c0);
+          if (R == 1)
+            stream_forward<1>(Lg, invd, Us + c0 * t, t, 1, 0, np, ring);
+          else
+            stream_forward<kStreamRhs>(Lg, invd, Us + c0 * t, t, R, 0, np, ring);
+        }
+        if (!one) {
+          for (int i = tid; i < rows * np; i += blockDim.x) {
+            const int e = i / np, q = i - e * np;
+            Lg[tri(np + e0 + e, q)] = Us[e * t + q];
+          }
+          __syncthreads();
+        }
+      }
+      // Schur complement of the new block: in the diagonal tile for k <= 32,
+      // else in the factor
+      const bool small = k <= kSB;
+      for (int pr = warp; pr < k * (k + 1) / 2; pr += nw) {
+        int e = 0;
+        while ((e + 1) * (e + 2) / 2 <= pr) ++e;
+        const int f = pr - e * (e + 1) / 2;
+        const double* re = one ? Us + e * t : Lg + tri(np + e, 0);
+        const double* rf = one ? Us + f * t : Lg + tri(np + f, 0);
+        double a4[4] = {0.0, 0.0, 0.0, 0.0};
+        for (int q0 = lane; q0 < np; q0 += 128) {
+#pragma unroll
+          for (int s = 0; s < 4; ++s) {
+            const int q = q0 + 32 * s;
+            if (q < np) a4[s] = fma(re[q], rf[q], a4[s]);
+          }
+        }
+        const double acc = warp_sum((a4[0] + a4[1]) + (a4[2] + a4[3]));
+        if (lane == 0) {
+          const double sv = G[(int64_t)add[e] * t + add[f]] - acc;
+          if (small)
+            D[e][f] = sv;
+          else
+            Lg[tri(np + e, np + f)] = sv;
+        }
+      }
+      __syncthreads();
+      // Cholesky of the Schur block (lane e owns new row e; lane 0 alone past
+      // 32 rows); a pivot at or below 1e-13·G_ll blocks that variable
+      if (warp == 0) {
+        int failed = 0;
+        if (small) {
+          const double dg = lane < k ? diag(add[lane]) : 0.0;
+          for (int f = 0; f < k; ++f) {
+            const double piv = D[f][f];
+            const double gff = __shfl_sync(0xffffffffu, dg, f);
+            if (!(piv > 1e-13 * gff)) {
+              if (lane == 0) blocked[add[f]] = 1;
+              failed = 1;
+              break;
+            }
+            const double lff = sqrt(piv), il = 1.0 / lff;
+            __syncwarp();
+            if (lane == f) D[f][f] = lff;
+            if (lane > f && lane < k) D[lane][f] *= il;
+            __syncwarp();
+            if (lane > f && lane < k) {
+              const double lef = D[lane][f];
+              for (int q = f + 1; q <= lane; ++q) D[lane][q] -= lef * D[q][f];
+            }
+            __syncwarp();
+          }
+        } else if (lane == 0) {
+          for (int f = 0; f < k; ++f) {
+            const double piv = Lg[tri(np + f, np + f)];
+            if (!(piv > 1e-13 * diag(add[f]))) {
+              blocked[add[f]] = 1;
+              failed = 1;
+              break;
+            }
+            const double lff = sqrt(piv), il = 1.0 / lff;
+            Lg[tri(np + f, np + f)] = lff;
+            invd[np + f] = il;
+            for (int e = f + 1; e < k; ++e) Lg[tri(np + e, np + f)] *= il;
+            for (int e = f + 1; e < k; ++e) {
+              const double lef = Lg[tri(np + e, np + f)];
+              for (int q = f + 1; q <= e; ++q) Lg[tri(np + e, np + q)] -= lef * Lg[tri(np + q, np + f)];
+            }
+          }
+        }
+        failed = __shfl_sync(0xffffffffu, failed, 0);
+        if (lane == 0) {
+          if (failed) {
+            int kk = 0;
+            for (int e = 0; e < k; ++e)
+              if (!blocked[add[e]]) add[kk++] = add[e];
+            ctl[1] = kk;
+          } else {
+            for (int e = 0; e < k; ++e) {
+              P[np + e] = add[e];
+              inP[add[e]] = 1;
+            }
+            ctl[0] = np + k;
+            ctl[1] = 0;
+          }
+        }
+      }
+      __syncthreads();
+      const bool ok = ctl[0] != np;
+      if (ok && small) {   // the accepted block goes into the factor
+        if (one)
+          for (int i = tid; i < k * np; i += blockDim.x) {
+            const int e = i / np, q = i - e * np;
+            Lg[tri(np + e, q)] = Us[e * t + q];
+          }
+        for (int i = tid; i < k * k; i += blockDim.x) {
+          const int e = i / k, f = i - e * k;
+          if (f <= e) Lg[tri(np + e, np + f)] = D[e][f];
+        }
+        for (int e = tid; e < k; e += blockDim.x) invd[np + e] = 1.0 / D[e][e];
+      }
+      __syncthreads();
+      if (ok || ctl[1] == 0) return;
+    }
+  };
+
   int iter = 0;
   bool converged = false;
   for (int outer = 0; outer <= maxit; ++outer) {
@@ -984,7 +1360,10 @@ __global__ void __launch_bounds__(kNnlsThreads) k_nnls(Problem p, Work w, int pa
     }
     __syncthreads();
     if (ctl[1] == 0) { converged = true; break; }
-    block_append();
+    if (streamed)
+      append_streamed();
+    else
+      block_append();
 
     // ---- inner loop: solve on P, step back toward feasibility ----
     bool abort = false;
@@ -994,13 +1373,18 @@ __global__ void __launch_bounds__(kNnlsThreads) k_nnls(Problem p, Work w, int pa
       // z = y on the cached rows; the forward solve extends it over the rest
       for (int q = tid; q < npc; q += blockDim.x) z[q] = q < y0 ? yv[q] : b[P[q]];
       __syncthreads();
-      {
+      if (streamed) {
+        stream_forward<1>(Lg, invd, z, 0, 1, y0, npc, ring);
+      } else {
         double* U[kMaxRhs] = {z, z, z, z, z, z, z, z};
         block_forward(L, invd, U, 1, y0, npc, D);
       }
       for (int q = y0 + tid; q < npc; q += blockDim.x) yv[q] = z[q];
       if (tid == 0) ctl[10] = npc;
-      block_backward(L, invd, z, npc, D);
+      if (streamed)
+        stream_backward(Lg, invd, z, npc, ring);
+      else
+        block_backward(L, invd, z, npc, D);
       double best = INFINITY;
       int bq = -1, nneg = 0;
       for (int q = tid; q < npc; q += blockDim.x) {
@@ -1221,6 +1605,15 @@ cudaError_t launch_omp_init(const Problem& p, const Work& w, cudaStream_t s) {
   return cudaGetLastError();
 }
 
+// New rows the streamed append keeps in shared memory next to the vectors
+// for max_t and the ring (0: the factor does not stream).
+int nnls_stream_rows(int max_t) {
+  const size_t fixed = nnls_vec_bytes(max_t) + kRingBytes, row = (size_t)max_t * sizeof(double);
+  if (fixed + row > kSmemCap) return 0;
+  const size_t r = (kSmemCap - fixed) / row;
+  return r < (size_t)kAppendRows ? (int)r : kAppendRows;
+}
+
 int nnls_smem_cap(int max_t) {
   int lcap = 0;
   nnls_smem_bytes(max_t, &lcap);
@@ -1266,11 +1659,15 @@ cudaError_t launch_omp_pass(const Problem& p, const Work& w, int pass, int activ
   int lcap;
   size_t sm = nnls_smem_bytes(p.max_t, &lcap);
   cudaFuncSetAttribute(k_nnls, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemCap);
-  // heads whose factor lives in the workspace: the vectors alone in shared
-  // memory, so several CTAs share an SM; then the others with the factor
-  if (big > 0)
+  // heads whose factor lives in the workspace (the vectors, the copy ring and
+  // the new rows in shared memory); then the others with the factor
+  if (big > 0) {
+    const int ucap = nnls_stream_rows(p.max_t);
+    const size_t sm_big =
+        nnls_vec_bytes(p.max_t) + (ucap > 0 ? kRingBytes + (size_t)ucap * p.max_t * sizeof(double) : 0);
     AM_LAUNCH(AM_STAGE_NNLS, s,
-              launch_chained(k_nnls, dim3(big), dim3(kNnlsThreads), nnls_vec_bytes(p.max_t), s, p, w, pass, 0));
+              launch_chained(k_nnls, dim3(big), dim3(kNnlsThreads), sm_big, s, p, w, pass, 0, ucap));
+  }
   if (active > big) {
     Work ws = w;
     ws.order = w.order + big;
@@ -1278,7 +1675,7 @@ cudaError_t launch_omp_pass(const Problem& p, const Work& w, int pass, int activ
     const size_t sm_small = nnls_vec_bytes(p.max_t) + nnls_tri_bytes(small_tmax < lcap ? small_tmax : lcap);
     AM_LAUNCH(AM_STAGE_NNLS, s,
               launch_chained(k_nnls, dim3(active - big), dim3(kNnlsThreads), sm_small < sm ? sm_small : sm, s, p,
-                             ws, pass, lcap));
+                             ws, pass, lcap, 0));
   }
   dim3 gr(resid_blocks(p), active);
   AM_LAUNCH(AM_STAGE_RESID, s, launch_chained(k_resid, gr, dim3(kResidThreads), 0, s, p, w, pass));
