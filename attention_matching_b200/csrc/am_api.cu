@@ -39,7 +39,7 @@ struct Layout {
   size_t G, L, AtA, A, Apl, Ypl, AtY, nrm_part;
   size_t cnorm, cnpart, rnorm, clist, clj, ccount, inv_m, gb, ghist, gtau, gcnt, cdone, cnblk, ctheta, rows_eval, gpart, gcount,
       rcount,
-      dinv, vinv;
+      dinv, vinv, ndinv, dvalid;
   size_t total;
   size_t tables_bytes;
   bool tc_normal;   // the value fit's normal equations run on the tensor cores (bf16 planes)
@@ -137,6 +137,8 @@ Layout plan(int n, int T, int d, int H, int64_t sum_t, int64_t sum_t2, bool corr
   L.rcount = take((size_t)H * 4);
   L.dinv = take(((size_t)sum_t + 32 * (size_t)H) * 32 * 8);
   L.vinv = take(((size_t)sum_t + 64 * (size_t)H) * 64 * 8);
+  L.ndinv = take(((size_t)sum_t + 32 * (size_t)H) * 64 * 8);
+  L.dvalid = take((size_t)H * 4);
   L.total = o;
   return L;
 }
@@ -311,6 +313,8 @@ Work bind(const Layout& L, char* base, bool corr_bf16) {
   w.rcount = reinterpret_cast<int32_t*>(base + L.rcount);
   w.dinv = reinterpret_cast<double*>(base + L.dinv);
   w.vinv = reinterpret_cast<double*>(base + L.vinv);
+  w.ndinv = reinterpret_cast<double*>(base + L.ndinv);
+  w.dvalid = reinterpret_cast<int32_t*>(base + L.dvalid);
   return w;
 }
 

@@ -67,11 +67,12 @@ __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t b
 
 namespace am {
 
-// Asynchronous 8-byte copy from global to this thread block's shared memory
-// (cp.async, cached in L1).  A thread's copies complete in the groups it
-// commits; cp_async_wait<N> returns once at most N of its groups are pending.
-__device__ __forceinline__ void cp_async8(void* dst, const void* src) {
-  asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
+// Asynchronous 16-byte copy from global to this thread block's shared memory
+// (cp.async, cached in L2 only); both addresses 16-byte aligned.  A thread's
+// copies complete in the groups it commits; cp_async_wait<N> returns once at
+// most N of its groups are pending.
+__device__ __forceinline__ void cp_async16(void* dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
 }
 
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }

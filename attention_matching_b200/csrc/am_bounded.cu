@@ -399,8 +399,8 @@ __global__ void __launch_bounds__(256) k_gbound(Problem p, Work w, int pass) {
 // ------------------------------------------------------------ exact rows --
 // c_j = Σ_i r_i Φ_ij in fp64 sums of exact fp32 products for the keys the
 // launch takes: b_j >= τ (which = 0, the probe) or b_j < τ with
-// b_j·(1 + 1e-6) >= θ (which = 1, the rest).  Each CTA scans a slice of the
-// head's keys in chunks, gathers the keys it takes in shared memory, and
+// b_j·(1 + 1e-6) >= θ (which = 1, the rest).  Each CTA scans every
+// gridDim.x-th key of the head in chunks, gathers the keys it takes in shared memory, and
 // evaluates them two at a time: four warps share a key, each summing a
 // quarter of the queries with eight columns per lane in flight; the quarters
 // are added in a fixed order.  The last block of a head to finish (counted
@@ -434,13 +434,15 @@ __global__ void __launch_bounds__(kSelThreads) k_rows(Problem p, Work w, int pas
   const int n4 = p.ldn >> 2;
   const int per = (n4 + kRowSplit - 1) / kRowSplit;
   const int c0 = quarter * per, c1 = min(n4, c0 + per);
-  const int slice = (p.T + gridDim.x - 1) / gridDim.x;
-  const int j_lo = blockIdx.x * slice, j_hi = min(p.T, j_lo + slice);
-  for (int k0 = j_lo; k0 < j_hi; k0 += kScanChunk) {
-    const int k1 = min(j_hi, k0 + kScanChunk);
+  // this CTA's keys: j ≡ blockIdx.x (mod gridDim.x), so keys the bound keeps,
+  // which cluster by index, spread evenly over the head's CTAs
+  const int nkeys = (p.T - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x;
+  for (int i0 = 0; i0 < nkeys; i0 += kScanChunk) {
+    const int i1 = min(nkeys, i0 + kScanChunk);
     if (threadIdx.x == 0) ncand = 0;
     __syncthreads();
-    for (int j = k0 + threadIdx.x; j < k1; j += blockDim.x) {
+    for (int i = i0 + threadIdx.x; i < i1; i += blockDim.x) {
+      const int j = (int)blockIdx.x + i * (int)gridDim.x;
       const float b = gb[j];
       bool take = false;
       if (!sel[j]) take = which == 0 ? b >= tau : (b < tau && (double)b * kBoundMargin >= theta);

@@ -98,6 +98,8 @@ struct Work {
   int32_t* rcount;      // [H] bounded-correlation row blocks finished this launch
   double* dinv;         // per head at 32·(cu_t[h] + 32h): inverses of the value-fit factor's 32×32 diagonal tiles
   double* vinv;         // per head at 64·(cu_t[h] + 64h): inverses of the 64×64 diagonal tiles (tiled solve)
+  double* ndinv;        // per head at 64·(cu_t[h] + 32h): the NNLS factor's diagonal-tile inverses and their transposes
+  int32_t* dvalid;      // [H] leading row blocks of the NNLS factor whose cached inverse is valid
   int64_t nrm_ata;      // Σt²
   int64_t nrm_stride;   // Σt² + Σt·d
   int64_t sum_t;        // Σt

@@ -54,6 +54,7 @@ __global__ void k_init(Problem p, Work w) {
     w.mm[h] = acc;
     w.np[h] = 0;
     w.ylen[h] = 0;
+    w.dvalid[h] = 0;
     if (!(acc > 0.0) || !isfinite(acc)) record_status(w.status + h, AM_ERR_NONFINITE);
   }
   // keys past the head's own count are marked as taken: never candidates
@@ -652,150 +653,201 @@ __device__ void block_backward(const double* L, const double* invd, double* v, i
   }
 }
 
-// ---------------------------------------------- streamed factor solves ----
-// For a head whose factor lives in the workspace, a triangular solve reads
-// the whole factor once, in order.  The reads go through a ring of kRing
-// shared-memory stages filled by asynchronous 8-byte copies issued kRing − 1
-// pieces ahead, so the copies of later rows are in flight while a diagonal
-// block is swept.  A piece is up to 32 factor rows × 64 columns (row stride
-// 65: a warp reading down a column meets distinct banks); a row block's
-// pieces are its off-diagonal column chunks and its diagonal block.
-constexpr int kRing = 4;
-constexpr int kPieceCols = 64;
-constexpr int kPieceLd = kPieceCols + 1;
-constexpr int kStageDoubles = kSB * kPieceLd;
-constexpr size_t kRingBytes = (size_t)kRing * kStageDoubles * sizeof(double);
-constexpr int kStreamRhs = 8;    // vectors one streamed forward solve carries
+// ------------------------------------------------- tiled factor solves ----
+// A head whose factor lives in the workspace keeps it in 32×32 tiles: tile
+// (I, J), J <= I, holds rows 32I .. 32I+31 and columns 32J .. 32J+31
+// row-major at offset (I(I+1)/2 + J)·1024, so the off-diagonal tiles of a
+// row block are one contiguous range.  Beside the factor the head keeps the
+// inverses of its diagonal tiles, D_I = L_II⁻¹ and D_Iᵀ, valid for its first
+// `dvalid` row blocks; a triangular solve then takes each diagonal block as
+// one 32×32 matrix-vector product instead of 32 dependent steps, and a block
+// whose inverse is stale is inverted (one warp, a column per lane) when the
+// solve reaches it.  A solve reads the factor once, in order: steps of up to
+// kSlotTiles tiles go through a ring of kSlots shared-memory slots filled by
+// 16-byte asynchronous copies (cp.async) one step ahead of their use.
+constexpr int kTileElems = kSB * kSB;
+constexpr int kSlotTiles = 3;
+constexpr int kSlots = 3;
+constexpr int kSlotDoubles = kSlotTiles * kTileElems;
+constexpr size_t kRingBytes = (size_t)kSlots * kSlotDoubles * sizeof(double);
+constexpr int kStreamRhs = 8;    // vectors one forward solve carries
 constexpr int kAppendRows = 32;  // most new rows the append keeps in shared memory
 
-struct Piece {
-  int r0, bw, c0, cw;
+__host__ __device__ __forceinline__ int64_t tile_at(int I, int J) {
+  return ((int64_t)I * (I + 1) / 2 + J) * kTileElems;
+}
+// element (r, c), c <= r, of a tiled factor
+__device__ __forceinline__ int64_t tl(int r, int c) { return tile_at(r >> 5, c >> 5) + (r & 31) * kSB + (c & 31); }
+// doubles a tiled factor of order t takes, plus one for the 16-byte alignment
+__host__ __device__ inline int64_t tiled_doubles(int t) { return tile_at((t + kSB - 1) / kSB, 0) + 1; }
+// the cached inverses of head h: block I at 2·1024·I (D_I) and + 1024 (D_Iᵀ)
+__device__ __forceinline__ double* dinv_cache(const Work& w, int h) {
+  return w.ndinv + 64 * (w.cu_t[h] + 32 * (int64_t)h);
+}
+
+struct Step {
+  int I, J0, nt;
   bool diag;
 };
 
-// Copies piece pc of the packed factor L into a stage (the diagonal block's
-// lower triangle only) and commits the copies as one group.
-__device__ __forceinline__ void issue_piece(const double* L, double* stage, const Piece& pc) {
+// Forward order over row blocks I0 .. I1: each block's off-diagonal tiles in
+// steps of up to kSlotTiles, then its diagonal step.
+struct ForwardSteps {
+  int I, J, I1;
+  __device__ bool done() const { return I > I1; }
+  __device__ Step step() const {
+    Step s;
+    s.I = I;
+    s.diag = J >= I;
+    s.J0 = s.diag ? I : J;
+    s.nt = s.diag ? 1 : min(kSlotTiles, I - J);
+    return s;
+  }
+  __device__ void next() {
+    if (J >= I) { ++I; J = 0; } else { J += kSlotTiles; }
+  }
+};
+
+// Backward order over row blocks I1 .. 0: each block's diagonal step, then
+// its off-diagonal tiles in steps of up to kSlotTiles.
+struct BackwardSteps {
+  int I, J;   // J < 0: the diagonal step
+  __device__ bool done() const { return I < 0; }
+  __device__ Step step() const {
+    Step s;
+    s.I = I;
+    s.diag = J < 0;
+    s.J0 = s.diag ? I : J;
+    s.nt = s.diag ? 1 : min(kSlotTiles, I - J);
+    return s;
+  }
+  __device__ void next() {
+    J = J < 0 ? 0 : J + kSlotTiles;
+    if (J >= I) { --I; J = -1; }
+  }
+};
+
+// Copies step s into a slot and commits the copies as one group: its
+// off-diagonal tiles, or for a diagonal step the cached inverse (D_Iᵀ for a
+// forward solve, D_I for a backward one) when block I is below dvalid, else
+// the factor's diagonal tile.
+__device__ __forceinline__ void issue_step(const double* Lt, const double* dc, int dvalid, bool fwd, double* slot,
+                                           const Step& s) {
+  const double* src = s.diag ? (s.I < dvalid ? dc + (int64_t)s.I * 2 * kTileElems + (fwd ? kTileElems : 0)
+                                             : Lt + tile_at(s.I, s.I))
+                             : Lt + tile_at(s.I, s.J0);
+  const int chunks = s.nt * kTileElems / 2;   // 16-byte chunks
 #pragma unroll
-  for (int u = 0; u < kSB * kPieceCols / kNnlsThreads; ++u) {
-    const int e = threadIdx.x + u * kNnlsThreads, r = e / kPieceCols, c = e % kPieceCols;
-    if (r < pc.bw && c < pc.cw && (!pc.diag || c <= r))
-      cp_async8(stage + r * kPieceLd + c, L + tri(pc.r0 + r, pc.c0 + c));
+  for (int u = 0; u < kSlotDoubles / 2 / kNnlsThreads; ++u) {
+    const int e = threadIdx.x + u * kNnlsThreads;
+    if (e < chunks) cp_async16(slot + 2 * e, src + 2 * e);
   }
   cp_async_commit();
 }
 
-__device__ __forceinline__ int off_chunks(int r0) { return (r0 + kPieceCols - 1) / kPieceCols; }
-
-// Forward order over rows [k0, n): row blocks top down, each its column
-// chunks of [0, r0) then its diagonal block.
-struct ForwardPieces {
-  int r0, c, n;
-  __device__ bool done() const { return r0 >= n; }
-  __device__ Piece piece() const {
-    Piece d;
-    d.r0 = r0;
-    d.bw = min(kSB, n - r0);
-    d.diag = c == off_chunks(r0);
-    d.c0 = d.diag ? r0 : c * kPieceCols;
-    d.cw = d.diag ? d.bw : min(kPieceCols, r0 - d.c0);
-    return d;
-  }
-  __device__ void next() {
-    if (++c > off_chunks(r0)) { c = 0; r0 += kSB; }
-  }
-};
-
-// Backward order over rows [0, n): row blocks bottom up (at multiples of 32),
-// each its diagonal block then its column chunks of [0, r0).
-struct BackwardPieces {
-  int r0, c, n;
-  __device__ bool done() const { return r0 < 0; }
-  __device__ Piece piece() const {
-    Piece d;
-    d.r0 = r0;
-    d.bw = min(kSB, n - r0);
-    d.diag = c == 0;
-    d.c0 = d.diag ? r0 : (c - 1) * kPieceCols;
-    d.cw = d.diag ? d.bw : min(kPieceCols, r0 - d.c0);
-    return d;
-  }
-  __device__ void next() {
-    if (++c > off_chunks(r0)) { c = 0; r0 -= kSB; }
-  }
-};
-
-// Runs consume(piece, stage) over the pieces of `it` in order, with the
-// stages kRing − 1 pieces ahead in flight.  Every thread of the block calls
-// it; consume may synchronise the block.  Ends with the block synchronised.
-template <class Pieces, class Consume>
-__device__ __forceinline__ void stream_pieces(const double* L, double* ring, Pieces it, Consume&& consume) {
-  Pieces ahead = it;
+// Runs consume(step, slot) over the steps of `it` in order, with the next
+// kSlots − 1 steps' copies in flight.  Every thread of the block calls it;
+// consume may synchronise the block.  Ends with the block synchronised.
+template <class Steps, class Consume>
+__device__ __forceinline__ void stream_steps(const double* Lt, const double* dc, int dvalid, bool fwd, double* ring,
+                                             Steps it, Consume&& consume) {
+  Steps ahead = it;
 #pragma unroll
-  for (int s = 0; s < kRing - 1; ++s) {
+  for (int s = 0; s < kSlots - 1; ++s) {
     if (!ahead.done()) {
-      issue_piece(L, ring + s * kStageDoubles, ahead.piece());
+      issue_step(Lt, dc, dvalid, fwd, ring + s * kSlotDoubles, ahead.step());
       ahead.next();
     } else {
       cp_async_commit();
     }
   }
   for (int p = 0; !it.done(); ++p) {
-    cp_async_wait<kRing - 2>();
-    __syncthreads();   // piece p is in; the stage of piece p − 1 is free
+    cp_async_wait<kSlots - 2>();
+    __syncthreads();   // step p is in; the slot of step p − 1 is free
     if (!ahead.done()) {
-      issue_piece(L, ring + ((p + kRing - 1) % kRing) * kStageDoubles, ahead.piece());
+      issue_step(Lt, dc, dvalid, fwd, ring + ((p + kSlots - 1) % kSlots) * kSlotDoubles, ahead.step());
       ahead.next();
     } else {
       cp_async_commit();
     }
-    consume(it.piece(), static_cast<const double*>(ring + (p % kRing) * kStageDoubles));
+    consume(it.step(), static_cast<const double*>(ring + (p % kSlots) * kSlotDoubles));
     it.next();
   }
   cp_async_wait<0>();
   __syncthreads();
 }
 
-// u_e ← L⁻¹ u_e on rows [k0, n) for the R <= RMAX vectors u_e = U0 + e·ldu
-// (shared memory); entries below k0 are already final.  Products: warp w
-// takes rows 4w .. 4w+3 of the row block, its lanes run across the piece's
-// columns; the sums close at the diagonal block, whose sweep runs one warp
-// per vector.
+// X = S⁻¹ for the 32×32 lower-triangular tile S (row-major) with reciprocal
+// diagonal id[0..32), by one warp: lane c computes column c, each entry as
+// soon as its sum is complete, then adds its terms to every later row's sum
+// (independent products, not one chain); rows past the block's last hold
+// whatever their entries give.  X goes to D with zeros above the diagonal.
+__device__ __noinline__ void invert_tile(const double* S, const double* id, DiagTile* D) {
+  const int c = threadIdx.x & 31;
+  double a[kSB];
+#pragma unroll
+  for (int r = 0; r < kSB; ++r) a[r] = 0.0;
+#pragma unroll
+  for (int m = 0; m < kSB; ++m) {
+    const double d = id[m];
+    a[m] = m < c ? 0.0 : (m == c ? d : -a[m] * d);
+#pragma unroll
+    for (int r = m + 1; r < kSB; ++r) a[r] = fma(S[r * kSB + m], a[m], a[r]);
+  }
+#pragma unroll
+  for (int r = 0; r < kSB; ++r) D[r][c] = a[r];
+}
+
+// After invert_tile and a block barrier: D_I and D_Iᵀ of block I into the cache.
+__device__ __forceinline__ void store_inverse(const DiagTile* D, double* dc, int I) {
+  double* di = dc + (int64_t)I * 2 * kTileElems;
+  for (int e = threadIdx.x; e < kTileElems; e += blockDim.x) {
+    const int a = e >> 5, b = e & 31;
+    di[e] = D[a][b];                // D_I[a][b]
+    di[kTileElems + e] = D[b][a];   // D_Iᵀ[a][b]
+  }
+}
+
+// u_e ← L⁻¹ u_e on rows [32·I0, n) for the R <= RMAX vectors u_e = U0 + e·ldu
+// (shared memory); entries below 32·I0 are final.  Products: warp w takes
+// rows 4w .. 4w+3 of the row block, its lanes a column of each tile; the sums
+// close at the diagonal step, which multiplies by D_I, one warp per vector.
+// *dvalid is raised past the blocks this solve inverted.
 template <int RMAX>
-__device__ void stream_forward(const double* L, const double* invd, double* U0, int ldu, int R, int k0, int n,
-                               double* ring) {
+__device__ void stream_forward(const double* Lt, double* dc, int* dvalid, const double* invd, double* U0, int ldu,
+                               int R, int I0, int n, double* ring, DiagTile* D) {
+  if (32 * I0 >= n) return;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, rl = 4 * warp;
+  const int dv = *dvalid;
   double acc[4][RMAX];
 #pragma unroll
   for (int i = 0; i < 4; ++i)
 #pragma unroll
     for (int e = 0; e < RMAX; ++e) acc[i][e] = 0.0;
-  stream_pieces(L, ring, ForwardPieces{k0, 0, n}, [&](const Piece& pc, const double* S) {
-    if (!pc.diag) {
-      if (rl < pc.bw) {
+  stream_steps(Lt, dc, dv, true, ring, ForwardSteps{I0, 0, (n - 1) / kSB}, [&](const Step& st, const double* S) {
+    const int r0 = kSB * st.I, bw = min(kSB, n - r0);
+    if (!st.diag) {
+      if (rl < bw) {
+        for (int j = 0; j < st.nt; ++j) {
+          const int col = kSB * (st.J0 + j) + lane;
+          double u[RMAX];
 #pragma unroll
-        for (int half = 0; half < 2; ++half) {
-          const int j = lane + 32 * half;
-          if (j < pc.cw) {
-            double u[RMAX];
+          for (int e = 0; e < RMAX; ++e) u[e] = e < R ? U0[e * ldu + col] : 0.0;
 #pragma unroll
-            for (int e = 0; e < RMAX; ++e) u[e] = e < R ? U0[e * ldu + pc.c0 + j] : 0.0;
+          for (int i = 0; i < 4; ++i) {
+            const double l = rl + i < bw ? S[j * kTileElems + (rl + i) * kSB + lane] : 0.0;
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-              const double l = rl + i < pc.bw ? S[(rl + i) * kPieceLd + j] : 0.0;
-#pragma unroll
-              for (int e = 0; e < RMAX; ++e) acc[i][e] = fma(l, u[e], acc[i][e]);
-            }
+            for (int e = 0; e < RMAX; ++e) acc[i][e] = fma(l, u[e], acc[i][e]);
           }
         }
       }
       return;
     }
-    if (pc.r0 > 0 && rl < pc.bw) {
+    if (st.I > 0 && rl < bw) {
       if constexpr (RMAX == 1) {
         double flat[4] = {acc[0][0], acc[1][0], acc[2][0], acc[3][0]};
         const double sum = warp_reduce_n<4>(flat);   // lane l: row rl + l mod 4
-        if (lane < 4 && rl + lane < pc.bw) U0[pc.r0 + rl + lane] -= sum;
+        if (lane < 4 && rl + lane < bw) U0[r0 + rl + lane] -= sum;
       } else {
         static_assert(RMAX == 8, "four rows × eight vectors fill the 32 lanes");
         double flat[32];   // value i·8 + e: row rl + i, vector e
@@ -805,60 +857,90 @@ __device__ void stream_forward(const double* L, const double* invd, double* U0, 
           for (int e = 0; e < 8; ++e) flat[i * 8 + e] = acc[i][e];
         const double sum = warp_reduce32(flat);
         const int li = lane / 8, le = lane % 8;
-        if (le < R && rl + li < pc.bw) U0[le * ldu + pc.r0 + rl + li] -= sum;
+        if (le < R && rl + li < bw) U0[le * ldu + r0 + rl + li] -= sum;
       }
     }
 #pragma unroll
     for (int i = 0; i < 4; ++i)
 #pragma unroll
       for (int e = 0; e < RMAX; ++e) acc[i][e] = 0.0;
+    const bool cached = st.I < dv;
+    if (!cached && warp == 0) invert_tile(S, invd + r0, D);
     __syncthreads();
-    if (warp < R) {
-      double* u = U0 + warp * ldu;
-      double v = lane < pc.bw ? u[pc.r0 + lane] : 0.0;
-      for (int c = 0; c < pc.bw; ++c) {
-        if (lane == c) v *= invd[pc.r0 + c];
-        const double vc = __shfl_sync(0xffffffffu, v, c);
-        if (lane > c && lane < pc.bw) v -= S[lane * kPieceLd + c] * vc;
+    if (!cached) store_inverse(D, dc, st.I);
+    if (warp < R) {   // u ← D_I w, lane r one row (D_I[r][c] from D_Iᵀ or D)
+      double* u = U0 + warp * ldu + r0;
+      double a[4] = {0.0, 0.0, 0.0, 0.0};
+      if (cached) {
+#pragma unroll
+        for (int c = 0; c < kSB; ++c)
+          if (c < bw) a[c & 3] = fma(S[c * kSB + lane], u[c], a[c & 3]);
+      } else {
+#pragma unroll
+        for (int c = 0; c < kSB; ++c)
+          if (c < bw) a[c & 3] = fma(D[lane][c], u[c], a[c & 3]);
       }
-      if (lane < pc.bw) u[pc.r0 + lane] = v;
+      __syncwarp();
+      if (lane < bw) u[lane] = (a[0] + a[1]) + (a[2] + a[3]);
     }
   });
+  if (threadIdx.x == 0 && dv >= I0) *dvalid = max(dv, (n - 1) / kSB + 1);
+  __syncthreads();
 }
 
 // v ← L⁻ᵀ v on rows [0, n), v in shared memory.  Per row block from the
-// bottom: warp 0 sweeps the diagonal block, then each column chunk takes the
-// block's contribution, warp w on columns 8w .. 8w+7 with the four lane
-// quarters on eight factor rows each (summed by two shuffles).
-__device__ void stream_backward(const double* L, const double* invd, double* v, int n, double* ring) {
+// bottom: warp 0 multiplies the block by D_Iᵀ, then each off-diagonal tile
+// takes the block's contribution, two warps per tile (sixteen columns each,
+// the lane halves on sixteen rows each, added by one shuffle).  Every block
+// inverse is valid afterwards.
+__device__ void stream_backward(const double* Lt, double* dc, int* dvalid, const double* invd, double* v, int n,
+                                double* ring, DiagTile* D) {
   if (n <= 0) return;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  stream_pieces(L, ring, BackwardPieces{((n - 1) / kSB) * kSB, 0, n}, [&](const Piece& pc, const double* S) {
-    if (pc.diag) {
-      if (warp == 0) {
-        double x = lane < pc.bw ? v[pc.r0 + lane] : 0.0;
-        for (int c = pc.bw - 1; c >= 0; --c) {
-          if (lane == c) x *= invd[pc.r0 + c];
-          const double xc = __shfl_sync(0xffffffffu, x, c);
-          if (lane < c) x -= S[c * kPieceLd + lane] * xc;
+  const int dv = *dvalid;
+  const int I1 = (n - 1) / kSB;
+  stream_steps(Lt, dc, dv, false, ring, BackwardSteps{I1, -1}, [&](const Step& st, const double* S) {
+    const int r0 = kSB * st.I, bw = min(kSB, n - r0);
+    if (st.diag) {
+      const bool cached = st.I < dv;
+      if (!cached) {
+        if (warp == 0) invert_tile(S, invd + r0, D);
+        __syncthreads();
+        store_inverse(D, dc, st.I);
+      }
+      if (warp == 0) {   // x = D_Iᵀ v_I, lane c one entry
+        double a[4] = {0.0, 0.0, 0.0, 0.0};
+        if (cached) {
+#pragma unroll
+          for (int r = 0; r < kSB; ++r)
+            if (r < bw) a[r & 3] = fma(S[r * kSB + lane], v[r0 + r], a[r & 3]);
+        } else {
+#pragma unroll
+          for (int r = 0; r < kSB; ++r)
+            if (r < bw) a[r & 3] = fma(D[r][lane], v[r0 + r], a[r & 3]);
         }
-        if (lane < pc.bw) v[pc.r0 + lane] = x;
+        __syncwarp();
+        if (lane < bw) v[r0 + lane] = (a[0] + a[1]) + (a[2] + a[3]);
       }
       return;
     }
-    const int j = 8 * warp + (lane & 7), q = lane >> 3;
-    double s = 0.0;
-    if (j < pc.cw) {
+    const int j = warp >> 1;
+    if (j < st.nt) {
+      const int c = 16 * (warp & 1) + (lane & 15), rh = 16 * (lane >> 4);
+      const double* T = S + j * kTileElems;
+      double a[4] = {0.0, 0.0, 0.0, 0.0};
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const int r = 8 * q + i;
-        if (r < pc.bw) s = fma(S[r * kPieceLd + j], v[pc.r0 + r], s);
+      for (int i = 0; i < 16; ++i) {
+        const int r = rh + i;
+        if (r < bw) a[i & 3] = fma(T[r * kSB + c], v[r0 + r], a[i & 3]);
       }
+      double s = (a[0] + a[1]) + (a[2] + a[3]);
+      s += __shfl_xor_sync(0xffffffffu, s, 16);
+      if (lane < 16) v[kSB * (st.J0 + j) + c] -= s;
     }
-    s += __shfl_xor_sync(0xffffffffu, s, 8);
-    s += __shfl_xor_sync(0xffffffffu, s, 16);
-    if (q == 0 && j < pc.cw) v[pc.c0 + j] -= s;
   });
+  if (threadIdx.x == 0) *dvalid = max(dv, I1 + 1);
+  __syncthreads();
 }
 
 // Us[e·ldu + q] = G[add_e, P_q] for e < R, q < np (all loads of a thread
@@ -927,8 +1009,13 @@ __device__ void factor_remove(double* L, double* invd, double* xv, double* rot, 
         if (k < jw) {
           const double lkk = __shfl_sync(0xffffffffu, v[k], k);
           const double xk = __shfl_sync(0xffffffffu, xr, k);
-          const double r = hypot(lkk, xk);
-          const double c = r / lkk, sn = xk / lkk, ic = lkk / r;
+          // r = sqrt(lkk² + xk²) through one reciprocal square root and one
+          // reciprocal (entries of a Cholesky factor of a Gram matrix of
+          // features in [0, 1]: no overflow); c = r/lkk, sn = xk/lkk, ic = lkk/r
+          const double rr = fma(lkk, lkk, xk * xk);
+          const double irr = rsqrt(rr), il = 1.0 / lkk;
+          const double r = rr * irr;
+          const double c = r * il, sn = xk * il, ic = lkk * irr;
           if (lane == k) v[k] = r;
           if (mine && lane > k) {
             v[k] = (v[k] + sn * xr) * ic;
@@ -990,6 +1077,109 @@ __device__ void factor_remove(double* L, double* invd, double* xv, double* rot, 
   __syncthreads();
 }
 
+// factor_remove for a tiled factor (same steps; elements addressed by tile).
+// The move runs over the new factor's tiles from row block q/32 on, in
+// storage order: every moved element's source lies after its destination,
+// and the sources of later chunks after every destination of earlier ones,
+// so each chunk is read before it is written.
+__device__ void factor_remove_tiled(double* L, double* invd, double* xv, double* rot, int q, int np) {
+  const int tid = threadIdx.x, nthr = blockDim.x, lane = tid & 31, warp = tid >> 5;
+  const int m = np - 1 - q;
+  const int o = q + 1;
+  for (int a = tid; a < m; a += nthr) xv[a] = L[tl(o + a, q)];
+  __syncthreads();
+  for (int J = 0; J < m; J += kRotBlock) {
+    const int jw = min(kRotBlock, m - J);
+    if (warp == 0) {
+      const bool mine = lane < jw;
+      const int rr = o + J + (mine ? lane : 0);
+      double v[kRotBlock];
+#pragma unroll
+      for (int c = 0; c < kRotBlock; ++c) v[c] = (mine && c <= lane) ? L[tl(rr, o + J + c)] : 0.0;
+      double xr = mine ? xv[J + lane] : 0.0;
+#pragma unroll
+      for (int k = 0; k < kRotBlock; ++k) {
+        if (k < jw) {
+          const double lkk = __shfl_sync(0xffffffffu, v[k], k);
+          const double xk = __shfl_sync(0xffffffffu, xr, k);
+          // r = sqrt(lkk² + xk²) through one reciprocal square root and one
+          // reciprocal (entries of a Cholesky factor of a Gram matrix of
+          // features in [0, 1]: no overflow); c = r/lkk, sn = xk/lkk, ic = lkk/r
+          const double rr = fma(lkk, lkk, xk * xk);
+          const double irr = rsqrt(rr), il = 1.0 / lkk;
+          const double r = rr * irr;
+          const double c = r * il, sn = xk * il, ic = lkk * irr;
+          if (lane == k) v[k] = r;
+          if (mine && lane > k) {
+            v[k] = (v[k] + sn * xr) * ic;
+            xr = c * xr - sn * v[k];
+          }
+          if (lane == 0) { rot[3 * k] = c; rot[3 * k + 1] = sn; rot[3 * k + 2] = ic; }
+        }
+      }
+      if (mine) {
+#pragma unroll
+        for (int c = 0; c < kRotBlock; ++c)
+          if (c <= lane) L[tl(rr, o + J + c)] = v[c];
+      }
+    }
+    __syncthreads();
+    for (int a = J + jw + tid; a < m; a += nthr) {
+      const int rr = o + a;
+      double v[kRotBlock];
+#pragma unroll
+      for (int c = 0; c < kRotBlock; ++c) v[c] = c < jw ? L[tl(rr, o + J + c)] : 0.0;
+      double xa = xv[a];
+#pragma unroll
+      for (int k = 0; k < kRotBlock; ++k) {
+        if (k < jw) {
+          v[k] = (v[k] + rot[3 * k + 1] * xa) * rot[3 * k + 2];
+          xa = rot[3 * k] * xa - rot[3 * k + 1] * v[k];
+        }
+      }
+#pragma unroll
+      for (int c = 0; c < kRotBlock; ++c)
+        if (c < jw) L[tl(rr, o + J + c)] = v[c];
+      xv[a] = xa;
+    }
+    __syncthreads();
+  }
+  // new (r, c) = old (r + 1, c + [c >= q]) for q <= r < np − 1, c <= r: the
+  // new factor's tiles from row block q/32 on, two per chunk, in storage order
+  const int nbn = (np - 1 + kSB - 1) / kSB;
+  int I = q >> 5, J = 0;
+  while (I < nbn) {
+    int ti[2], tj[2];
+    ti[0] = I;
+    tj[0] = J;
+    if (++J > I) { ++I; J = 0; }
+    const bool two = I < nbn;
+    ti[1] = I;
+    tj[1] = J;
+    if (two && ++J > I) { ++I; J = 0; }
+    double v[2][kTileElems / kNnlsThreads];
+    bool live[2][kTileElems / kNnlsThreads];
+#pragma unroll
+    for (int k = 0; k < 2; ++k)
+#pragma unroll
+      for (int u = 0; u < kTileElems / kNnlsThreads; ++u) {
+        const int l = tid + u * kNnlsThreads;
+        const int r = kSB * ti[k] + (l >> 5), c = kSB * tj[k] + (l & 31);
+        live[k][u] = (k == 0 || two) && r >= q && r < np - 1 && c <= r;
+        v[k][u] = live[k][u] ? L[tl(r + 1, c + (c >= q))] : 0.0;
+      }
+    __syncthreads();
+#pragma unroll
+    for (int k = 0; k < 2; ++k)
+#pragma unroll
+      for (int u = 0; u < kTileElems / kNnlsThreads; ++u)
+        if (live[k][u]) L[tile_at(ti[k], tj[k]) + tid + u * kNnlsThreads] = v[k][u];
+    __syncthreads();
+  }
+  for (int r = q + tid; r < np - 1; r += nthr) invd[r] = 1.0 / L[tl(r, r)];
+  __syncthreads();
+}
+
 // l_in_smem_max: heads with t at or below it keep the factor in shared
 // memory.  ucap > 0: the others stream their solves (ring and up to ucap new
 // rows of t doubles in shared memory after the vectors); 0: they read the
@@ -1027,14 +1217,19 @@ __global__ void __launch_bounds__(kNnlsThreads) k_nnls(Problem p, Work w, int pa
   double* Lg = w.L + gbase;
   double* L = l_smem ? reinterpret_cast<double*>(smem + nnls_vec_bytes(t)) : Lg;
   const bool streamed = !l_smem && ucap > 0;
-  double* ring = reinterpret_cast<double*>(smem + nnls_vec_bytes(t));   // streamed heads only
-  double* Us = ring + kRing * kStageDoubles;                              // ucap rows of t
+  // streamed heads: the tiled factor (16-byte aligned inside the head's t×t
+  // region), its cached block inverses, the copy ring and ucap new rows of t
+  double* Lt = w.L + ((gbase + 1) & ~(int64_t)1);
+  double* dc = dinv_cache(w, h);
+  double* ring = reinterpret_cast<double*>(smem + nnls_vec_bytes(t));
+  double* Us = ring + kSlots * kSlotDoubles;
   // the factor kept in shared memory arrives by one bulk copy (16-byte
   // aligned at both ends; rounding the size up reads at most one double past
   // the factor, still inside the head's t×t region and the shared buffer)
   const uint32_t lbytes = l_smem ? (uint32_t)((tri(np_old, 0) * 8 + 15) & ~(int64_t)15) : 0u;
   // ctl: 0 np, 1 nadd, 2 single mode, 4 argmin, 5 nneg, 7 ncand, 9 removed count, 10 valid y rows,
-  //      11 first factor row that differs from the stored factor
+  //      11 first factor row that differs from the stored factor, 12 leading row blocks whose
+  //      cached inverse is valid (streamed heads)
   const int maxit = p.nnls_max_iter > 0 ? p.nnls_max_iter : 3 * t + 50;
   const double mnorm = sqrt(w.mm[h]);
   auto diag = [&](int l) { return G[(int64_t)l * t + l]; };
@@ -1055,7 +1250,7 @@ __global__ void __launch_bounds__(kNnlsThreads) k_nnls(Problem p, Work w, int pa
   for (int q = tid; q < np_old; q += blockDim.x) P[q] = w.plist[base + q];
   const int ylen0 = min(w.ylen[h], np_old);
   for (int q = tid; q < ylen0; q += blockDim.x) yv[q] = w.ycache[base + q];
-  if (tid == 0) { ctl[0] = np_old; ctl[2] = 0; ctl[10] = ylen0; ctl[11] = np_old; }
+  if (tid == 0) { ctl[0] = np_old; ctl[2] = 0; ctl[10] = ylen0; ctl[11] = np_old; ctl[12] = w.dvalid[h]; }
   __syncthreads();   // the barrier is initialised before anyone waits on it
   const bool landed = lbytes == 0 || mbar_wait_bounded(lbar, 0, p.wait_cycles);
   if (__syncthreads_or(!landed)) {
@@ -1067,7 +1262,7 @@ __global__ void __launch_bounds__(kNnlsThreads) k_nnls(Problem p, Work w, int pa
   }
   for (int q = tid; q < np_old; q += blockDim.x) {
     inP[P[q]] = 1;
-    invd[q] = 1.0 / L[tri(q, q)];
+    invd[q] = 1.0 / (streamed ? Lt[tl(q, q)] : L[tri(q, q)]);
   }
   __syncthreads();
 
@@ -1159,10 +1354,10 @@ __global__ void __launch_bounds__(kNnlsThreads) k_nnls(Problem p, Work w, int pa
     }
   };
 
-  // Streamed heads: the same block append with the forward solves of the new
-  // rows streamed (kStreamRhs vectors per read of the factor), and, for at
-  // most ucap new rows, the rows, their Schur block and its Cholesky in
-  // shared memory until the block is accepted.
+  // Streamed heads: the same block append on the tiled factor, with the
+  // forward solves of the new rows streamed (kStreamRhs vectors per read of
+  // the factor) and, for at most ucap new rows, the rows, their Schur block
+  // and its Cholesky in shared memory until the block is accepted.
   auto append_streamed = [&]() {
     for (;;) {
       const int np = ctl[0], k = ctl[1];
@@ -1172,17 +1367,18 @@ __global__ void __launch_bounds__(kNnlsThreads) k_nnls(Problem p, Work w, int pa
       for (int e0 = 0; e0 < k; e0 += chunk) {
         const int rows = min(chunk, k - e0);
         gather_new_rows(Us, t, G, t, add + e0, rows, P, np);
+        __syncthreads();
         for (int c0 = 0; c0 < rows; c0 += kStreamRhs) {
           const int R = min(kStreamRhs, rows - c0);
           if (R == 1)
-            stream_forward<1>(Lg, invd, Us + c0 * t, t, 1, 0, np, ring);
+            stream_forward<1>(Lt, dc, &ctl[12], invd, Us + c0 * t, t, 1, 0, np, ring, D);
           else
-            stream_forward<kStreamRhs>(Lg, invd, Us + c0 * t, t, R, 0, np, ring);
+            stream_forward<kStreamRhs>(Lt, dc, &ctl[12], invd, Us + c0 * t, t, R, 0, np, ring, D);
         }
         if (!one) {
           for (int i = tid; i < rows * np; i += blockDim.x) {
             const int e = i / np, q = i - e * np;
-            Lg[tri(np + e0 + e, q)] = Us[e * t + q];
+            Lt[tl(np + e0 + e, q)] = Us[e * t + q];
           }
           __syncthreads();
         }
@@ -1194,14 +1390,16 @@ __global__ void __launch_bounds__(kNnlsThreads) k_nnls(Problem p, Work w, int pa
         int e = 0;
         while ((e + 1) * (e + 2) / 2 <= pr) ++e;
         const int f = pr - e * (e + 1) / 2;
-        const double* re = one ? Us + e * t : Lg + tri(np + e, 0);
-        const double* rf = one ? Us + f * t : Lg + tri(np + f, 0);
         double a4[4] = {0.0, 0.0, 0.0, 0.0};
         for (int q0 = lane; q0 < np; q0 += 128) {
 #pragma unroll
           for (int s = 0; s < 4; ++s) {
             const int q = q0 + 32 * s;
-            if (q < np) a4[s] = fma(re[q], rf[q], a4[s]);
+            if (q < np) {
+              const double xe = one ? Us[e * t + q] : Lt[tl(np + e, q)];
+              const double xf = one ? Us[f * t + q] : Lt[tl(np + f, q)];
+              a4[s] = fma(xe, xf, a4[s]);
+            }
           }
         }
         const double acc = warp_sum((a4[0] + a4[1]) + (a4[2] + a4[3]));
@@ -1210,7 +1408,7 @@ __global__ void __launch_bounds__(kNnlsThreads) k_nnls(Problem p, Work w, int pa
           if (small)
             D[e][f] = sv;
           else
-            Lg[tri(np + e, np + f)] = sv;
+            Lt[tl(np + e, np + f)] = sv;
         }
       }
       __syncthreads();
@@ -1241,19 +1439,19 @@ __global__ void __launch_bounds__(kNnlsThreads) k_nnls(Problem p, Work w, int pa
           }
         } else if (lane == 0) {
           for (int f = 0; f < k; ++f) {
-            const double piv = Lg[tri(np + f, np + f)];
+            const double piv = Lt[tl(np + f, np + f)];
             if (!(piv > 1e-13 * diag(add[f]))) {
               blocked[add[f]] = 1;
               failed = 1;
               break;
             }
             const double lff = sqrt(piv), il = 1.0 / lff;
-            Lg[tri(np + f, np + f)] = lff;
+            Lt[tl(np + f, np + f)] = lff;
             invd[np + f] = il;
-            for (int e = f + 1; e < k; ++e) Lg[tri(np + e, np + f)] *= il;
+            for (int e = f + 1; e < k; ++e) Lt[tl(np + e, np + f)] *= il;
             for (int e = f + 1; e < k; ++e) {
-              const double lef = Lg[tri(np + e, np + f)];
-              for (int q = f + 1; q <= e; ++q) Lg[tri(np + e, np + q)] -= lef * Lg[tri(np + q, np + f)];
+              const double lef = Lt[tl(np + e, np + f)];
+              for (int q = f + 1; q <= e; ++q) Lt[tl(np + e, np + q)] -= lef * Lt[tl(np + q, np + f)];
             }
           }
         }
@@ -1271,6 +1469,7 @@ __global__ void __launch_bounds__(kNnlsThreads) k_nnls(Problem p, Work w, int pa
             }
             ctl[0] = np + k;
             ctl[1] = 0;
+            ctl[12] = min(ctl[12], np / kSB);   // the block holding row np changed
           }
         }
       }
@@ -1280,11 +1479,11 @@ __global__ void __launch_bounds__(kNnlsThreads) k_nnls(Problem p, Work w, int pa
         if (one)
           for (int i = tid; i < k * np; i += blockDim.x) {
             const int e = i / np, q = i - e * np;
-            Lg[tri(np + e, q)] = Us[e * t + q];
+            Lt[tl(np + e, q)] = Us[e * t + q];
           }
         for (int i = tid; i < k * k; i += blockDim.x) {
           const int e = i / k, f = i - e * k;
-          if (f <= e) Lg[tri(np + e, np + f)] = D[e][f];
+          if (f <= e) Lt[tl(np + e, np + f)] = D[e][f];
         }
         for (int e = tid; e < k; e += blockDim.x) invd[np + e] = 1.0 / D[e][e];
       }
@@ -1369,12 +1568,13 @@ __global__ void __launch_bounds__(kNnlsThreads) k_nnls(Problem p, Work w, int pa
     bool abort = false;
     for (;;) {
       if (++iter > maxit) { abort = true; break; }
-      const int npc = ctl[0], y0 = ctl[10];
+      // streamed heads restart the extension at a row-block boundary
+      const int npc = ctl[0], y0 = streamed ? ctl[10] / kSB * kSB : ctl[10];
       // z = y on the cached rows; the forward solve extends it over the rest
       for (int q = tid; q < npc; q += blockDim.x) z[q] = q < y0 ? yv[q] : b[P[q]];
       __syncthreads();
       if (streamed) {
-        stream_forward<1>(Lg, invd, z, 0, 1, y0, npc, ring);
+        stream_forward<1>(Lt, dc, &ctl[12], invd, z, 0, 1, y0 / kSB, npc, ring, D);
       } else {
         double* U[kMaxRhs] = {z, z, z, z, z, z, z, z};
         block_forward(L, invd, U, 1, y0, npc, D);
@@ -1382,7 +1582,7 @@ __global__ void __launch_bounds__(kNnlsThreads) k_nnls(Problem p, Work w, int pa
       for (int q = y0 + tid; q < npc; q += blockDim.x) yv[q] = z[q];
       if (tid == 0) ctl[10] = npc;
       if (streamed)
-        stream_backward(Lg, invd, z, npc, ring);
+        stream_backward(Lt, dc, &ctl[12], invd, z, npc, ring, D);
       else
         block_backward(L, invd, z, npc, D);
       double best = INFINITY;
@@ -1471,10 +1671,16 @@ __global__ void __launch_bounds__(kNnlsThreads) k_nnls(Problem p, Work w, int pa
       __syncthreads();
       // delete the leavers from the factor, last position first
       const int nrm = ctl[9];
-      for (int i = nrm - 1, npr = ctl[0] + nrm; i >= 0; --i, --npr) factor_remove(L, invd, g, red, cand[i], npr);
+      for (int i = nrm - 1, npr = ctl[0] + nrm; i >= 0; --i, --npr) {
+        if (streamed)
+          factor_remove_tiled(Lt, invd, g, red, cand[i], npr);
+        else
+          factor_remove(L, invd, g, red, cand[i], npr);
+      }
       if (tid == 0 && nrm > 0) {
         ctl[10] = min(ctl[10], cand[0]);
         ctl[11] = min(ctl[11], cand[0]);
+        ctl[12] = min(ctl[12], cand[0] / kSB);
       }
       __syncthreads();
     }
@@ -1496,6 +1702,7 @@ __global__ void __launch_bounds__(kNnlsThreads) k_nnls(Problem p, Work w, int pa
   if (tid == 0) {
     w.np[h] = npf;
     w.ylen[h] = yl;
+    w.dvalid[h] = ctl[12];
     if (!converged) record_status(w.status + h, AM_WARN_NOT_CONVERGED);
   }
 }
@@ -1610,6 +1817,10 @@ cudaError_t launch_omp_init(const Problem& p, const Work& w, cudaStream_t s) {
 int nnls_stream_rows(int max_t) {
   const size_t fixed = nnls_vec_bytes(max_t) + kRingBytes, row = (size_t)max_t * sizeof(double);
   if (fixed + row > kSmemCap) return 0;
+  // the tiled factor must fit a streamed head's t×t region (t > the shared-memory cap)
+  int lcap = 0;
+  nnls_smem_bytes(max_t, &lcap);
+  if (tiled_doubles(lcap + 1) > (int64_t)(lcap + 1) * (lcap + 1)) return 0;
   const size_t r = (kSmemCap - fixed) / row;
   return r < (size_t)kAppendRows ? (int)r : kAppendRows;
 }

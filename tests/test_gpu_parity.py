@@ -238,6 +238,19 @@ def test_large_budget_global_factor():
 
 
 @needs_cuda
+def test_tiled_factor_refits_converge_within_a_few_iterations():
+    """Heads whose NNLS factor lives in the workspace as 32×32 tiles with
+    cached diagonal-block inverses (t above what shared memory holds), with the
+    refit's inner iterations capped at 12 per pass: warm-started refits take
+    one or two solves each, so every head must end converged (status 0) and
+    match the oracle.  A wrong streamed solve or a stale cached inverse shows
+    up here as NOT_CONVERGED after a bounded run."""
+    heads = [W.structured_head(396 + h, n=1536, T=1400) for h in range(2)]
+    out, _ = check_all(heads, [330, 270], 4, 2, label="tiled factor", nnls_max_iter=12)
+    assert all(s == 0 for s in out["status"]), out["status"]
+
+
+@needs_cuda
 def test_kv_chunked_long_sequence():
     """KV-based chunking: one long sequence cut into contiguous chunks that are
     compacted independently (sinks only in the first chunk); the full chunks
