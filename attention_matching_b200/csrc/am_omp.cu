@@ -1817,10 +1817,12 @@ cudaError_t launch_omp_init(const Problem& p, const Work& w, cudaStream_t s) {
 int nnls_stream_rows(int max_t) {
   const size_t fixed = nnls_vec_bytes(max_t) + kRingBytes, row = (size_t)max_t * sizeof(double);
   if (fixed + row > kSmemCap) return 0;
-  // the tiled factor must fit a streamed head's t×t region (t > the shared-memory cap)
+  // the tiled factor must fit every streamed head's t×t region (t above the
+  // shared-memory cap; it does for every t >= 102)
   int lcap = 0;
   nnls_smem_bytes(max_t, &lcap);
-  if (tiled_doubles(lcap + 1) > (int64_t)(lcap + 1) * (lcap + 1)) return 0;
+  for (int t = lcap + 1; t <= max_t; ++t)
+    if (tiled_doubles(t) > (int64_t)t * t) return 0;
   const size_t r = (kSmemCap - fixed) / row;
   return r < (size_t)kAppendRows ? (int)r : kAppendRows;
 }
