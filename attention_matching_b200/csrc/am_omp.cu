@@ -391,14 +391,20 @@ __global__ void __launch_bounds__(kGramWarps * 32, 2) k_gram_tile(Problem p, Wor
   for (int sl = blockIdx.y; sl < nslices; sl += gridDim.y) {
     const int c0 = sl * kGramSlice4;
     const int cw = min(kGramSlice4, n4 - c0);
-    // every load of the slice first: the new picks' columns, then this warp's row
+    // the new picks' columns go straight to shared memory (asynchronous 16-byte
+    // copies, zeros past the picks and the slice), in flight with this warp's row
     constexpr int kStage = (NB * kGramSlice4 + kGramWarps * 32 - 1) / (kGramWarps * 32);
-    float4 sv[kStage];
 #pragma unroll
     for (int u = 0; u < kStage; ++u) {
       const int e = threadIdx.x + u * kGramWarps * 32, b = e / kGramSlice4, i = e % kGramSlice4;
-      sv[u] = e < NB * kGramSlice4 && b < nb && i < cw ? newrow[b][c0 + i] : make_float4(0.f, 0.f, 0.f, 0.f);
+      if (e < NB * kGramSlice4) {
+        if (b < nb && i < cw)
+          cp_async16(&stage[b][i], &newrow[b][c0 + i]);
+        else
+          stage[b][i] = make_float4(0.f, 0.f, 0.f, 0.f);
+      }
     }
+    cp_async_commit();
     float4 xf[kGramPos];
     double2 xm[kGramPos][2];
     if (is_m) {
@@ -415,11 +421,7 @@ __global__ void __launch_bounds__(kGramWarps * 32, 2) k_gram_tile(Problem p, Wor
         xf[k] = live && i < cw ? row[c0 + i] : make_float4(0.f, 0.f, 0.f, 0.f);
       }
     }
-#pragma unroll
-    for (int u = 0; u < kStage; ++u) {
-      const int e = threadIdx.x + u * kGramWarps * 32;
-      if (e < NB * kGramSlice4) stage[e / kGramSlice4][e % kGramSlice4] = sv[u];
-    }
+    cp_async_wait<0>();
     __syncthreads();
     if (is_m) {
 #pragma unroll
