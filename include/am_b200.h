@@ -346,7 +346,7 @@ typedef enum am_stage {
   AM_STAGE_DESIGN = 10,  /* A = rownorm(Φ_S diag w)                  */
   AM_STAGE_NORMAL = 11,  /* AᵀA, AᵀY                                 */
   AM_STAGE_SOLVE = 12,   /* ridge Cholesky, C_v                      */
-  AM_STAGE_NORMS = 13,   /* bounded mode: ‖Φ_{:,j}‖, keys by norm    */
+  AM_STAGE_NORMS = 13,   /* bounded mode: column and group norms   */
   AM_STAGE_ROWS = 14,    /* bounded mode: exact c_j of listed keys,
                             threshold and picks                      */
   AM_STAGE_ATTEND = 15,  /* am_attend_packed                         */
