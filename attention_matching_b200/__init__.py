@@ -47,7 +47,8 @@ class AmWorkspaceView(ctypes.Structure):
     _fields_ = [("phiT", ctypes.c_size_t), ("mass", ctypes.c_size_t), ("target", ctypes.c_size_t),
                 ("shift", ctypes.c_size_t), ("ldn", ctypes.c_int32), ("reserved", ctypes.c_int32),
                 ("weights", ctypes.c_size_t), ("resid", ctypes.c_size_t),
-                ("rows_evaluated", ctypes.c_size_t), ("column_norms", ctypes.c_size_t)]
+                ("rows_evaluated", ctypes.c_size_t), ("column_norms", ctypes.c_size_t),
+                ("nnls_refits", ctypes.c_size_t), ("nnls_solves", ctypes.c_size_t)]
 
 
 class AmOpts(ctypes.Structure):
@@ -191,8 +192,29 @@ def features(out: Dict, n: int, T: int, d: int, budgets: Sequence[int], topk: in
         "resid": view(v.resid, H * v.ldn, torch.float32).view(H, v.ldn),
         "rows_evaluated": view(v.rows_evaluated, H, torch.int64),
         "column_norms": view(v.column_norms, H * T, torch.float64).view(H, T),
+        "nnls_refits": view(v.nnls_refits, H, torch.int32),
+        "nnls_solves": view(v.nnls_solves, H, torch.int32),
         "ldn": v.ldn,
     }
+
+
+def call_stats(out: Dict, n: int, T: int, d: int, budgets: Sequence[int], topk: int = 1,
+               refit_every: int = 1, dtype: int = BF16, corr_mode: int = CORR_AUTO,
+               select_mode: int = SELECT_OMP) -> Dict:
+    """Per-head statistics of a finished call, valid whether or not it ran in
+    one wave: keys whose correlation was evaluated (int64 [H]), NNLS refits and
+    their inner solves (int32 [H] each); views into the workspace's prefix."""
+    import torch
+    H = len(budgets)
+    opts = make_opts(dtype, topk, refit_every, corr_mode=corr_mode, select_mode=select_mode)
+    v = AmWorkspaceView()
+    rc = lib().am_workspace_view(n, T, d, H, _i32_array(budgets), ctypes.byref(opts), ctypes.byref(v))
+    if rc:
+        raise AmError(rc, "am_workspace_view")
+    ws = out["workspace"]
+    return {"rows_evaluated": ws[v.rows_evaluated:v.rows_evaluated + 8 * H].view(torch.int64),
+            "nnls_refits": ws[v.nnls_refits:v.nnls_refits + 4 * H].view(torch.int32),
+            "nnls_solves": ws[v.nnls_solves:v.nnls_solves + 4 * H].view(torch.int32)}
 
 
 def _ptr(t) -> Optional[int]:

@@ -37,7 +37,7 @@ struct Layout {
   size_t picks, pick_corr, plist, sorted_slot;
   size_t bvec, w, w_eff, ycache;
   size_t G, L, AtA, A, Apl, Ypl, AtY, nrm_part;
-  size_t cnorm, cnpart, rnorm, clist, clj, ccount, inv_m, gb, ghist, gtau, gcnt, cdone, cnblk, ctheta, rows_eval, gpart, gcount,
+  size_t cnorm, cnpart, rnorm, clist, clj, ccount, inv_m, gb, ghist, gtau, gcnt, cdone, cnblk, ctheta, gpart, gcount,
       rcount,
       dinv, vinv, ndinv, dvalid;
   size_t total;
@@ -74,10 +74,17 @@ bool tc_normal(const am_opts_t* o, int d) { return o->in_dtype == AM_BF16 && (d 
 // t, Th, order, group order [H] int32 (a multiple of 8).
 size_t table_bytes(int H) { return (size_t)(H + 1) * 8 * 3 + (size_t)H * 4 * 4; }
 
-// The workspace prefix for a call of H heads: header, H status words, and a
+// The workspace prefix for a call of H heads: header, H status words, a
 // tables region that holds every wave's tables (Σ over waves of
-// table_bytes(H_w) <= 64·H bytes for any split into waves).
-size_t prefix_bytes(int H) { return align_up(kWsHeaderBytes + (size_t)H * 4) + align_up((size_t)H * 64 + 256); }
+// table_bytes(H_w) <= 64·H bytes for any split into waves), and per-head call
+// statistics that outlive the waves: keys evaluated (int64 [H]), then NNLS
+// refits and their inner solves (int32 [H] each).
+// (each statistic's array starts 16-byte aligned)
+size_t round16(size_t x) { return (x + 15) & ~(size_t)15; }
+size_t stats_offset(int H) { return align_up(kWsHeaderBytes + (size_t)H * 4) + align_up((size_t)H * 64 + 256); }
+size_t refits_offset(int H) { return stats_offset(H) + round16((size_t)H * 8); }
+size_t solves_offset(int H) { return refits_offset(H) + round16((size_t)H * 4); }
+size_t prefix_bytes(int H) { return align_up(solves_offset(H) + (size_t)H * 4); }
 
 // One wave's region, from byte `o0` (the end of the prefix) on.
 Layout plan(int n, int T, int d, int H, int64_t sum_t, int64_t sum_t2, bool corr_bf16, size_t o0, bool tc_normal) {
@@ -131,7 +138,6 @@ Layout plan(int n, int T, int d, int H, int64_t sum_t, int64_t sum_t2, bool corr
   L.cdone = take((size_t)H * 4);
   L.cnblk = take((size_t)H * T * kRedBlocks * 4);
   L.ctheta = take((size_t)H * 8);
-  L.rows_eval = take((size_t)H * 8);
   L.gpart = take((size_t)kGramMaxSlices * ((size_t)sum_t + H) * kGramMaxNew * 8);
   L.gcount = take(((size_t)sum_t + H) * 4);
   L.rcount = take((size_t)H * 4);
@@ -307,7 +313,6 @@ Work bind(const Layout& L, char* base, bool corr_bf16) {
   w.cdone = reinterpret_cast<int32_t*>(base + L.cdone);
   w.cnblk = reinterpret_cast<float*>(base + L.cnblk);
   w.ctheta = reinterpret_cast<double*>(base + L.ctheta);
-  w.rows_eval = reinterpret_cast<unsigned long long*>(base + L.rows_eval);
   w.gpart = reinterpret_cast<double*>(base + L.gpart);
   w.gcount = reinterpret_cast<int32_t*>(base + L.gcount);
   w.rcount = reinterpret_cast<int32_t*>(base + L.rcount);
@@ -471,8 +476,10 @@ am_status_t am_workspace_view(int32_t n, int32_t T, int32_t d, int32_t num_heads
   view->reserved = 0;
   view->weights = L.w;
   view->resid = L.r;
-  view->rows_evaluated = L.rows_eval;
+  view->rows_evaluated = stats_offset(num_heads);
   view->column_norms = L.cnorm;
+  view->nnls_refits = refits_offset(num_heads);
+  view->nnls_solves = solves_offset(num_heads);
   return AM_OK;
 }
 
@@ -530,7 +537,6 @@ am_status_t run_wave(const Problem& p, Work w, const Tables& tb, int G, int32_t*
   }
   AM_TRY(launch_omp_init(p, w, s));
   if (p.corr_bounded) AM_TRY(launch_column_norms(p, w, s));
-  AM_TRY(cudaMemsetAsync(w.rows_eval, 0, (size_t)H * 8, s));
   AM_TRY(cudaMemsetAsync(w.gcount, 0, ((size_t)tb.sum_t + H) * 4, s));
   AM_TRY(cudaMemsetAsync(w.rcount, 0, (size_t)H * 4, s));
   AM_TRY(cudaMemsetAsync(w.ghist, 0, (size_t)H * 1024 * 4, s));
@@ -626,18 +632,22 @@ am_status_t compact_heads_impl(const void* Q, const void* K, const void* V, int3
     const Layout L = plan(n, T, d, Hw, wt[k].sum_t, wt[k].sum_t2, bf16, pre, tcn);
     ww[k] = bind(L, base, bf16);
     ww[k].status = reinterpret_cast<int32_t*>(base + kWsHeaderBytes) + h0;
+    ww[k].rows_eval = reinterpret_cast<unsigned long long*>(base + stats_offset(H)) + h0;
+    ww[k].nnls_refits = reinterpret_cast<int32_t*>(base + refits_offset(H)) + h0;
+    ww[k].nnls_solves = reinterpret_cast<int32_t*>(base + solves_offset(H)) + h0;
     ww[k].nrm_ata = wt[k].sum_t2;
     ww[k].nrm_stride = wt[k].sum_t2 + wt[k].sum_t * d;
     ww[k].sum_t = wt[k].sum_t;
     pack_tables(wt[k], Hw, &host_tables, &ww[k], base + tables_at + host_tables.size(), &wgorder[k]);
   }
-  if (host_tables.size() > pre - tables_at) return AM_ERR_WORKSPACE;   // cannot happen: 64 bytes per head
+  if (host_tables.size() > stats_offset(H) - tables_at) return AM_ERR_WORKSPACE;   // cannot happen: 64 bytes per head
 
   WsHeader hdr{kWsMagic, H};
   // Pageable sources: both copies are staged before cudaMemcpyAsync returns.
   AM_TRY(cudaMemcpyAsync(base, &hdr, sizeof(hdr), cudaMemcpyHostToDevice, s));
   AM_TRY(cudaMemcpyAsync(base + tables_at, host_tables.data(), host_tables.size(), cudaMemcpyHostToDevice, s));
   AM_TRY(cudaMemsetAsync(base + kWsHeaderBytes, 0, (size_t)H * 4, s));
+  AM_TRY(cudaMemsetAsync(base + stats_offset(H), 0, solves_offset(H) + (size_t)H * 4 - stats_offset(H), s));
 
   for (size_t k = 0; k < waves.size(); ++k) {
     const int h0 = waves[k].first, h1 = waves[k].second, Hw = h1 - h0;

@@ -93,6 +93,8 @@ struct Work {
                         // (group g: queries i with (i / 128) mod resid_blocks == g)
   double* ctheta;       // [H] this pass's threshold θ, the kk-th largest value the probe found
   unsigned long long* rows_eval;   // [H] keys evaluated, summed over the passes
+  int32_t* nnls_refits;            // [H] NNLS refits of the call
+  int32_t* nnls_solves;            // [H] inner solves of those refits
   double* gpart;        // [kGramMaxSlices·(Σt + H)·kR] Gram partial sums per query slice
   int32_t* gcount;      // [Σt + H] Gram blocks finished this pass, per head and row group
   int32_t* rcount;      // [H] bounded-correlation row blocks finished this launch

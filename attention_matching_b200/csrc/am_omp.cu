@@ -1705,6 +1705,8 @@ __global__ void __launch_bounds__(kNnlsThreads) k_nnls(Problem p, Work w, int pa
     w.np[h] = npf;
     w.ylen[h] = yl;
     w.dvalid[h] = ctl[12];
+    w.nnls_refits[h] += 1;
+    w.nnls_solves[h] += min(iter, maxit);
     if (!converged) record_status(w.status + h, AM_WARN_NOT_CONVERGED);
   }
 }

@@ -571,11 +571,13 @@ def run_ours(args, rank, world, local_rank):
     ms = max_over_ranks(ms, dist if world > 1 else None, dev)
     _, worst = am.get_status(ws, H)
     one_wave = ws_bytes >= full_ws
-    rows_eval = None
-    if one_wave and corr_kind == "bounded":
-        rows_eval = int(am.features({"workspace": ws}, n, T, d, wl.budgets, wl.topk, wl.refit_every,
-                                    am.BF16 if Q.dtype == torch.bfloat16 else am.FP32,
-                                    corr_mode, select_mode)["rows_evaluated"].sum().item())
+    # per-head statistics of the last call (kept in the workspace prefix, so
+    # valid after a call of several waves too)
+    cst = am.call_stats({"workspace": ws}, n, T, d, wl.budgets, wl.topk, wl.refit_every,
+                        am.BF16 if Q.dtype == torch.bfloat16 else am.FP32, corr_mode, select_mode)
+    rows_eval = int(cst["rows_evaluated"].sum().item()) if corr_kind == "bounded" else None
+    refits = int(cst["nnls_refits"].sum().item())
+    solves = int(cst["nnls_solves"].sum().item())
 
     # end to end through the public API with pinned host buffers
     e2e = None
@@ -610,11 +612,7 @@ def run_ours(args, rank, world, local_rank):
 
     ldn = (n + 31) // 32 * 32
     peaks = load_peaks()
-    if rows_eval is None and corr_kind == "bounded":
-        rows_eval = 0   # not readable after a multi-wave call (the views cover one wave)
     models = stage_models(wl, n, key_counts, d, ldn, corr_kind, rows_eval or 0, tc_ok)
-    if corr_kind == "bounded" and not one_wave:
-        models.pop("rows", None)
     rf = roofline(stages, prof_steps, models, peaks, clk, committed_traffic(wl.name))
     total_heads = H * world if my_heads is None else len(budgets_all)
     value = total_heads / (ms * 1e-3)
@@ -636,6 +634,9 @@ def run_ours(args, rank, world, local_rank):
         cfg["key_counts"] = f"{len(key_counts)} heads, {sorted(set(key_counts))}"
     if rows_eval:
         cfg["correlation_rows_evaluated_per_step"] = rows_eval
+    if refits:
+        cfg["nnls_refits_per_step"] = refits
+        cfg["nnls_inner_solves_per_step"] = solves
     if my_heads is not None:
         cfg["sharding"] = f"LPT over {world} ranks of one workload's {len(budgets_all)} heads, cost t*ceil(t/(k*R))"
     if args.workload == "qwen3_4b_layer":

@@ -217,6 +217,9 @@ am_status_t am_compact_heads(const void* Q_ref, const void* K, const void* V,
  *                             out_offsets[h] in PICK order (zero where w_l = 0)
  *   resid   fp32 [H][ldn]     r = m − Φ_S w after the last refit
  *   rows_evaluated            see the field below
+ * The last three fields (rows_evaluated, nnls_refits, nnls_solves) are per-head
+ * call statistics kept in the workspace's prefix: valid after any completed
+ * call, whether or not it ran in one wave.
  * Same argument rules as am_workspace_size. */
 typedef struct am_workspace_view {
   size_t phiT, mass, target, shift;
@@ -229,6 +232,9 @@ typedef struct am_workspace_view {
                               bound within a relative 2e-6 of the exact norm
                               (AM_SELECT_HIGHEST: each key's total-attention
                               score Σ_i Φ_ij / m_i instead) */
+  size_t nnls_refits;      /* int32 [H]: NNLS refits of the call (one per pass) */
+  size_t nnls_solves;      /* int32 [H]: inner least-squares solves of those
+                              refits (each at most nnls_max_iter per refit) */
 } am_workspace_view_t;
 
 am_status_t am_workspace_view(int32_t n, int32_t T, int32_t d, int32_t num_heads,

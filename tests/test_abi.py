@@ -134,8 +134,9 @@ def test_attend_packed_argument_errors():
     (700, 900, 128, [70, 45], 1), (33, 1, 16, [1], 0),
 ])
 def test_workspace_view_regions_fit_align_and_do_not_overlap(n, T, d, budgets, select):
-    """The feature regions am_workspace_view reports lie inside the size
-    am_workspace_size asks for, start 16-byte aligned and are disjoint."""
+    """The feature regions and call statistics am_workspace_view reports lie
+    inside the size am_workspace_size asks for, start 16-byte aligned and are
+    disjoint."""
     dt = am.BF16 if d in (64, 128) else am.FP32
     o = am.make_opts(dt, 4, 2, select_mode=select)
     size = am.workspace_size(n, T, d, budgets, o)
@@ -147,7 +148,7 @@ def test_workspace_view_regions_fit_align_and_do_not_overlap(n, T, d, budgets, s
     assert ldn % 32 == 0 and ldn >= n
     regions = [(v.phiT, H * T * ldn * 4), (v.mass, H * ldn * 8), (v.target, H * n * d * 4), (v.shift, H * 4),
                (v.weights, S * 8), (v.resid, H * ldn * 4), (v.rows_evaluated, H * 8),
-               (v.column_norms, H * T * 8)]
+               (v.column_norms, H * T * 8), (v.nnls_refits, H * 4), (v.nnls_solves, H * 4)]
     for off, sz in regions:
         assert off % 16 == 0 and off + sz <= size, (off, sz, size)
     spans = sorted(regions)

@@ -248,6 +248,11 @@ def test_tiled_factor_refits_converge_within_a_few_iterations():
     heads = [W.structured_head(396 + h, n=1536, T=1400) for h in range(2)]
     out, _ = check_all(heads, [330, 270], 4, 2, label="tiled factor", nnls_max_iter=12)
     assert all(s == 0 for s in out["status"]), out["status"]
+    import attention_matching_b200 as am
+    st = am.call_stats(out, 1536, 1400, 128, [330, 270], 4, 2)
+    refits, solves = st["nnls_refits"].tolist(), st["nnls_solves"].tolist()
+    assert refits == [42, 34]                                 # one refit per pass of 8 picks
+    assert all(0 < s <= 12 * r for r, s in zip(refits, solves)), (refits, solves)   # the iteration cap
 
 
 @needs_cuda
@@ -308,6 +313,10 @@ def test_waves_give_the_one_wave_result():
     rng = np.random.default_rng(581)
     kb = [np.float32(rng.normal(0.0, 0.3, h.T)) for h in heads]
     one = run_gpu_varlen(heads, budgets, 4, 2, key_bias=kb)
+    stats_one = {k: v.clone() for k, v in am.call_stats(one, 600, 777, 128, budgets, 4, 2).items()}
+    passes = [(t + 7) // 8 for t in budgets]
+    assert stats_one["nnls_refits"].tolist() == passes
+    assert all(0 < r for r in stats_one["rows_evaluated"].tolist())
     offs = W.key_offsets_of(heads)
     opts = am.make_opts(am.BF16, 4, 2)
     arr = (ctypes.c_int64 * len(offs))(*offs)
@@ -321,6 +330,10 @@ def test_waves_give_the_one_wave_result():
         for k in ("indices", "C_k", "beta", "pick_order", "shift", "residual"):
             assert torch.equal(got[k], one[k]), (wave, k)
         torch.testing.assert_close(got["C_v"], one["C_v"], rtol=1e-5, atol=1e-6)
+        # the call statistics live in the prefix: every wave's heads, as in one wave
+        st = am.call_stats(got, 600, 777, 128, budgets, 4, 2)
+        for k in ("rows_evaluated", "nnls_refits", "nnls_solves"):
+            assert torch.equal(st[k], stats_one[k]), (wave, k)
 
 
 @needs_cuda
