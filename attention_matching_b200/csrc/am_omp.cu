@@ -493,15 +493,18 @@ __global__ void __launch_bounds__(kGramWarps * 32, 2) k_gram_tile(Problem p, Wor
 // ---------------------------------------------------------------- NNLS ----
 // Lawson-Hanson active set on the normal equations G w = b in fp64, with
 // the Cholesky factor of G restricted to the passive set kept across refits.
-// Entering variables are appended as a block: their forward solves against
-// the current factor run on separate warps, then a small Cholesky of their
-// Schur complement finishes the new rows.  If an entering block holds a
-// variable that will not grow, the refit continues one variable at a time.
-// A variable that leaves the passive set is deleted from the factor by a
-// rank-one update of the rows below it (no refactorisation), and the forward
-// solve y = L⁻¹ b_P is kept (also across refits) for every factor row above
-// the first one that changed, so each solve only extends it.
-// Triangular solves multiply by stored reciprocal diagonals.
+// Entering variables are appended as a block: their rows are forward-solved
+// against the current factor as several right-hand sides at once, then a
+// small Cholesky of their Schur complement finishes the new rows.  If an
+// entering block holds a variable that will not grow, the refit continues one
+// variable at a time.  A variable that leaves the passive set is deleted from
+// the factor by a rank-one update of the rows below it (no refactorisation),
+// and the forward solve y = L⁻¹ b_P is kept (also across refits) for every
+// factor row above the first one that changed, so each solve only extends it.
+// The factor is packed by rows (in shared memory while the kernel runs, for
+// small budgets), or kept in the workspace as 32×32 tiles with cached
+// inverses of its diagonal tiles (larger budgets; see the tiled solves
+// below).  Triangular solves multiply by stored reciprocal diagonals.
 constexpr int kSB = 32;        // rows per block of the blocked triangular solves
 constexpr int kMaxRhs = 8;     // vectors one blocked forward solve carries
 constexpr size_t kDiagTileBytes = kSB * (kSB + 1) * sizeof(double);
