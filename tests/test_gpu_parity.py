@@ -456,8 +456,9 @@ def test_attend_packed_fp32_d64():
 
 @needs_cuda
 def test_bounded_correlation_long_key_axis():
-    """T = 20000 keys: the bounded correlation pass sorts the column norms in
-    workspace memory instead of shared memory (more than 16384 keys)."""
+    """T = 20000 keys, more than the 16384 the highest-attention sort holds:
+    the bounded correlation pass (bounds, their histogram, the interleaved row
+    scans and the selection over the evaluated keys) on a long key axis."""
     heads = [W.structured_head(480 + h, n=256, T=20000, d=64) for h in range(2)]
     check_all(heads, [40, 24], 4, 2, label="T=20000")
 
