@@ -217,9 +217,9 @@ am_status_t am_compact_heads(const void* Q_ref, const void* K, const void* V,
  *                             out_offsets[h] in PICK order (zero where w_l = 0)
  *   resid   fp32 [H][ldn]     r = m − Φ_S w after the last refit
  *   rows_evaluated            see the field below
- * The last three fields (rows_evaluated, nnls_refits, nnls_solves) are per-head
- * call statistics kept in the workspace's prefix: valid after any completed
- * call, whether or not it ran in one wave.
+ * rows_evaluated, nnls_refits and nnls_solves are per-head call statistics
+ * kept in the workspace's prefix: valid after any completed call, whether or
+ * not it ran in one wave.
  * Same argument rules as am_workspace_size. */
 typedef struct am_workspace_view {
   size_t phiT, mass, target, shift;
